@@ -1,0 +1,509 @@
+#!/usr/bin/env python
+"""Throughput of the HiLS attention forward pass on B200, one JSON line on stdout.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hils|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...        (one process per GPU)
+
+A step is one hils_forward call (score -> top-K -> chunk/window attention -> fusion) over one
+batch of the prefill workload (default: small_mha_bf16, B=4 x 16 heads x 8192 tokens, d=64, S=64,
+K=8, W=512), inputs resident in HBM.  Steps are timed with CUDA events recorded by the library
+between its kernels, so each kernel's duration comes from the same timed steps; L2 is flushed
+(256 MiB write) between steps, outside the timed intervals.  With N GPUs every rank runs its own
+independent batch (weak scaling, no data-path collective); the step time is the max over ranks.
+
+Also reported (single GPU): `e2e` (the same call from pinned host buffers, copies included),
+`cpu_baseline` (the fp64 CPU oracle on a bounded sample), `decode` (long_decode: 32 single-token
+queries over a 512K-token cache, timed as a CUDA graph replay, microseconds per step) and
+`prefill_gqa7b` (the 7B-like GQA prefill at N=131072), each with its dominant kernel's roofline.
+`--impl reference` times the fp64 CPU oracle as the reference arm.
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "HiLS fwd prefill tokens/s & decode µs/step at 1 B200; % of HBM/TC roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in PEAKS_FALLBACK}, "measured"
+    except Exception:
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+# --------------------------------------------------------------------------- work model
+def eligible(pos, S, W):
+    first = pos - W + 1
+    return 0 if first <= 0 else first // S
+
+
+def work_model(dims, S, K, W, q_pos0, es):
+    """Algorithmic FLOPs / bytes of one forward (es = bytes per element of the inputs)."""
+    B, Hq, Hkv, Nq, Nkv, d = (dims[k] for k in ("B", "Hq", "Hkv", "N_q", "N_kv", "d"))
+    pos = np.arange(q_pos0, q_pos0 + Nq, dtype=np.int64)
+    n = np.where(pos - W + 1 > 0, (pos - W + 1) // S, 0)
+    k_sel = np.minimum(n, K)
+    L = pos - S * n + 1
+    C = Nkv // S
+    sum_n = float(n.sum())
+    tokens = float((k_sel * S + L).sum())
+    m = {}
+    m["score_flops"] = 2.0 * d * Hq * B * sum_n
+    m["attn_flops"] = 4.0 * d * B * Hq * tokens
+    # compulsory bytes of each phase (every input byte read once, every output written once)
+    sel_rows, head_rows = B * Hkv * Nq, B * Hq * Nq
+    if Nq <= 16:   # decode: each query reads its own landmark rows and its selected K/V
+        m["select_bytes"] = B * Hkv * float((n * (d * es + 4)).sum()) + head_rows * d * es
+        m["attn_bytes"] = B * Hkv * float((k_sel * S + L).sum()) * 2 * d * es + head_rows * d * es
+    else:
+        m["select_bytes"] = (head_rows * d * es + B * Hkv * C * (d * es + 4) +
+                             sel_rows * K * 4 + head_rows * K * 4)
+        m["attn_bytes"] = (head_rows * d * es * 2 + B * Hkv * Nkv * d * es * 2 +
+                           sel_rows * K * 4 + head_rows * K * 4 + head_rows * 4)
+    m["tokens"] = B * Nq
+    return m
+
+
+def phase_work(name, wm):
+    """(bound, algorithmic work, unit) of a kernel, for its roofline."""
+    if name.startswith("select_split"):
+        return "hbm", wm["select_bytes"], "GB/s"
+    if name.startswith("select"):
+        return "tensor", wm["score_flops"], "TFLOP/s"
+    if name == "attn_units":
+        return "hbm", wm["attn_bytes"], "GB/s"
+    if name.startswith("attn"):
+        return "tensor", wm["attn_flops"], "TFLOP/s"
+    return "hbm", None, "GB/s"
+
+
+def roofline(name, ms, wm, peaks, sustained=False):
+    bound, work, unit = phase_work(name, wm)
+    if work is None or ms <= 0:
+        return None
+    if bound == "hbm":
+        achieved = work / (ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+    else:
+        achieved = work / (ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    return {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak, "traffic": traffic_for(name), "work_per_launch": work}
+
+
+def traffic_for(kernel):
+    """dram read+write bytes per launch from the committed ncu summary, if it was taken on the
+    current source of that kernel; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel)
+    except Exception:
+        return None
+    if not rec:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return rec["bytes_per_launch"] if sha == rec.get("source_sha") else None
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            self.path = "/tmp/hils_clocks_%d_%d.csv" % (os.getpid(), self.gpu)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return None
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for _, _, r in rows for k in range(4) if r[k] == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": rows[0][1],
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- timing
+def make_events(n):
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for e in evs:
+        e.record()          # materialise the CUDA event handles
+    torch.cuda.synchronize()
+    return evs
+
+
+class Runner:
+    """Preallocated buffers for repeated hils_forward calls on one workload."""
+
+    def __init__(self, wl):
+        from hierarchical_chunk_sparse_scoring_b200 import binding as hb
+        self.hb = hb
+        self.wl = wl
+        self.p = hb.params_for(wl.q, wl.K, **wl.kwargs())
+        self.phases = hb.phases(self.p)
+        B, Hq, Nq, d = wl.q.shape
+        self.out = torch.empty_like(wl.q)
+        self.lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=wl.q.device)
+        self.idx = torch.empty((B, wl.K.shape[1], Nq, wl.K_top), dtype=torch.int32,
+                               device=wl.q.device)
+        self.ws = hb.workspace(self.p, wl.q.device)
+
+    def __call__(self, events=None, inputs=None):
+        wl = self.wl
+        q, qc, K, V, klm, blm = inputs or (wl.q, wl.q_cal, wl.K, wl.V, wl.k_lm, wl.b_lm)
+        self.hb.forward_raw(self.p, q, qc, K, V, klm, blm, self.out, self.lse, self.idx, self.ws,
+                            events=events)
+
+
+def timed_steps(run, steps, flush, barrier=lambda: None):
+    n_ph = len(run.phases)
+    evs = [make_events(n_ph + 1) for _ in range(steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for k in range(steps):
+        flush()
+        run(events=evs[k])
+    torch.cuda.synchronize()
+    barrier()
+    step_ms = [evs[k][0].elapsed_time(evs[k][-1]) for k in range(steps)]
+    phase_ms = {name: statistics.mean(evs[k][j].elapsed_time(evs[k][j + 1]) for k in range(steps))
+                for j, name in enumerate(run.phases)}
+    return step_ms, phase_ms
+
+
+def make_flush(device):
+    buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+
+    def flush():
+        buf.fill_(1.0)
+    return flush
+
+
+# --------------------------------------------------------------------------- CPU oracle
+def oracle_sample_rate(wl, seconds, rng_seed=0, max_rows=None):
+    """Times the fp64 oracle on randomly chosen (b, g, query) rows of `wl` (all G heads of each
+    row), sized to run about `seconds`.  Returns (tokens/s, rows, threads, wall seconds)."""
+    import oracle
+    Hq, d = wl.q.shape[1], wl.q.shape[3]
+    Hkv, Nkv = wl.K.shape[1], wl.K.shape[2]
+    G = Hq // Hkv
+    B, Nq = wl.q.shape[0], wl.q.shape[2]
+    rng = np.random.default_rng(rng_seed)
+    cache = {}
+
+    def f64(t):
+        return t.detach().to("cpu", torch.float64).numpy()
+
+    def build(n_rows):
+        qs = []
+        for _ in range(n_rows):
+            b, g, i = int(rng.integers(B)), int(rng.integers(Hkv)), int(rng.integers(Nq))
+            if (b, g) not in cache:
+                cache[(b, g)] = (f64(wl.k_lm[b, g]), f64(wl.b_lm[b, g]), f64(wl.K[b, g]),
+                                 f64(wl.V[b, g]))
+            klm, blm, kr, vr = cache[(b, g)]
+            qs.append(oracle.Query(wl.q_pos0 + i, f64(wl.q[b, g * G:(g + 1) * G, i]),
+                                   f64(wl.q_cal[b, g * G:(g + 1) * G, i]), klm, blm, kr, vr))
+        return qs
+
+    threads = oracle.default_threads()
+    kw = dict(d=d, G=G, S=wl.S, K_top=wl.K_top, W=wl.W, threads=threads)
+    rows = max(threads, 8)
+    while True:
+        qs = build(rows)
+        t0 = time.perf_counter()
+        oracle.run_queries(qs, **kw)
+        dt = time.perf_counter() - t0
+        if dt >= seconds * 0.5 or (max_rows and rows >= max_rows):
+            break
+        rows = int(min(rows * max(2.0, seconds / max(dt, 1e-3)), max_rows or 1 << 30))
+    tokens = rows * G / Hq
+    return tokens / dt, rows, threads, dt
+
+
+# --------------------------------------------------------------------------- arms
+def primary_workload(args, device, rank):
+    from hierarchical_chunk_sparse_scoring_b200 import workloads as W
+    seed = W.SPECS[args.workload]["seed"] + 1000 * rank
+    return W.make(args.workload, device, seed=seed)
+
+
+def config_of(wl, n_gpus):
+    d = wl.dims
+    return {"workload": wl.name, "B": d["B"], "Hq": d["Hq"], "Hkv": d["Hkv"], "N": d["N_kv"],
+            "d": d["d"], "S": wl.S, "K_top": wl.K_top, "W": wl.W,
+            "global_batch": d["B"] * n_gpus, "seq_len": d["N_kv"],
+            "parallelism": "dp%d (independent batches per GPU)" % n_gpus,
+            "l2": "flushed between steps (256 MiB write), outside the timed intervals"}
+
+
+def measure_e2e(run, steps, warmup):
+    """The same call from pinned host buffers: H2D of every input, the forward, D2H of out."""
+    wl = run.wl
+    host = [t.cpu().pin_memory() for t in (wl.q, wl.q_cal, wl.K, wl.V, wl.k_lm, wl.b_lm)]
+    dev = [torch.empty_like(t) for t in (wl.q, wl.q_cal, wl.K, wl.V, wl.k_lm, wl.b_lm)]
+    out_host = torch.empty(run.out.shape, dtype=run.out.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host)
+    d2h = out_host.numel() * out_host.element_size()
+
+    def step():
+        for d_, h_ in zip(dev, host):
+            d_.copy_(h_, non_blocking=True)
+        run(inputs=dev)
+        out_host.copy_(run.out, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
+        a, b = make_events(2)
+        a.record()
+        step()
+        b.record()
+        torch.cuda.synchronize()
+        ms.append(a.elapsed_time(b))
+    t = statistics.mean(ms)
+    return {"value": wl.q.shape[0] * wl.q.shape[2] / (t * 1e-3), "unit": "tokens/s",
+            "ms_per_step": t, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def extra_prefill(name, steps, peaks, **overrides):
+    from hierarchical_chunk_sparse_scoring_b200 import workloads as W
+    wl = W.make(name, "cuda", **overrides)
+    run = Runner(wl)
+    flush = make_flush(wl.q.device)
+    run()
+    torch.cuda.synchronize()
+    step_ms, phase_ms = timed_steps(run, steps, flush)
+    es = wl.q.element_size()
+    wm = work_model(wl.dims, wl.S, wl.K_top, wl.W, wl.q_pos0, es)
+    t = statistics.mean(step_ms)
+    res = {"workload": name, "ms_per_step": t, "tokens_per_s": wm["tokens"] / (t * 1e-3),
+           "phases_ms": phase_ms,
+           "rooflines": [roofline(k, v, wm, peaks) for k, v in phase_ms.items()],
+           "score_tflop": wm["score_flops"] / 1e12, "attn_tflop": wm["attn_flops"] / 1e12}
+    del run, wl
+    torch.cuda.empty_cache()
+    return res
+
+
+def extra_decode(steps, peaks, **overrides):
+    from hierarchical_chunk_sparse_scoring_b200 import workloads as W
+    wl = W.make("long_decode", "cuda", **overrides)
+    run = Runner(wl)
+    flush = make_flush(wl.q.device)
+    run()
+    torch.cuda.synchronize()
+    step_ms, phase_ms = timed_steps(run, steps, flush)
+    # the step as one CUDA graph replay (the pages time decode with CUDA graphs)
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        run()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        run()
+    g.replay()
+    torch.cuda.synchronize()
+    gms = []
+    for _ in range(steps):
+        flush()
+        a, b = make_events(2)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        gms.append(a.elapsed_time(b))
+    es = wl.q.element_size()
+    wm = work_model(wl.dims, wl.S, wl.K_top, wl.W, wl.q_pos0, es)
+    total_bytes = wm["select_bytes"] + wm["attn_bytes"]
+    t_us = statistics.median(gms) * 1e3
+    res = {"workload": "long_decode", "us_per_step": t_us,
+           "us_per_step_eager": statistics.mean(step_ms) * 1e3, "phases_ms": phase_ms,
+           "step_bytes": total_bytes,
+           "step_roofline": {"bound": "hbm", "achieved": total_bytes / (t_us * 1e-6) / 1e9,
+                             "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": total_bytes / (t_us * 1e-6) / 1e9 / peaks["hbm_gbs"]},
+           "rooflines": [roofline(k, v, wm, peaks) for k, v in phase_ms.items()]}
+    del g, run, wl
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_hils(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the HiLS path has no CPU fallback)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=device)
+    barrier = (lambda: dist.barrier()) if dist else (lambda: None)
+    peaks, peaks_src = load_peaks()
+
+    wl = primary_workload(args, device, rank)
+    run = Runner(wl)
+    flush = make_flush(device)
+    for _ in range(args.warmup):
+        flush()
+        run()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        step_ms, phase_ms = timed_steps(run, args.steps, flush, barrier)
+    total_ms = sum(step_ms)
+    if dist:
+        t = torch.tensor([total_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    tokens_per_rank = wl.q.shape[0] * wl.q.shape[2]
+    value = tokens_per_rank * world / (ms_per_step * 1e-3)
+    es = wl.q.element_size()
+    wm = work_model(wl.dims, wl.S, wl.K_top, wl.W, wl.q_pos0, es)
+    dom = max(phase_ms, key=phase_ms.get)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if wl.q.dtype == torch.bfloat16 else "f32",
+        "data": "synthetic (seeded generator, hierarchical_chunk_sparse_scoring_b200/workloads.py)",
+        "config": config_of(wl, world),
+        "roofline": roofline(dom, phase_ms[dom], wm, peaks),
+        "peaks_source": peaks_src,
+        "phases_ms": phase_ms,
+        "gpu_launches": len(run.phases) * args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_extras:
+        line["e2e"] = measure_e2e(run, max(3, args.steps // 2), 1)
+        del run
+        torch.cuda.empty_cache()
+        line["prefill_gqa7b"] = extra_prefill("gqa7b_prefill", 3, peaks)
+        line["decode"] = extra_decode(max(5, args.steps), peaks)
+        rate, rows, threads, dt = oracle_sample_rate(wl, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": threads,
+                                "kind": "oracle",
+                                "sample": "%d random (b, kv-group, query) rows of %s, all heads "
+                                          "of each group, %.1f s wall" % (rows, wl.name, dt)}
+    if dist:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_reference(args):
+    """The reference arm: the fp64 CPU oracle, as it stands, on the host cores."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    from hierarchical_chunk_sparse_scoring_b200 import workloads as W
+    wl = W.make(args.workload, "cpu")
+    per_step = max(1.0, args.ref_step_seconds)
+    rates, rows_total, threads = [], 0, 1
+    for k in range(args.warmup + args.steps):
+        rate, rows, threads, dt = oracle_sample_rate(wl, per_step, rng_seed=k)
+        if k >= args.warmup:
+            rates.append(rate)
+            rows_total += rows
+    value = statistics.mean(rates)
+    n_tokens = wl.q.shape[0] * wl.q.shape[2]
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": n_tokens / value * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded generator, hierarchical_chunk_sparse_scoring_b200/workloads.py)",
+            "config": config_of(wl, 1),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
+                             "kind": "oracle",
+                             "sample": "%d random (b, kv-group, query) rows over %d steps, "
+                                       "extrapolated to the full batch" % (rows_total, args.steps)},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["hils", "reference"], default="hils")
+    ap.add_argument("--workload", default="small_mha_bf16")
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=6.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "hils":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_hils(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,317 @@
+// Host side of the C ABI declared in include/hils.h: argument checks, workspace layout and the
+// choice of kernels.  Every step of the computation runs in the kernels; nothing here touches
+// tensor data.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+#include "hils.h"
+#include "kernels.h"
+
+#ifndef HILS_GIT_DESCRIBE
+#define HILS_GIT_DESCRIBE "unknown"
+#endif
+
+namespace hils {
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kStatusBytes = 256;
+constexpr int kChunksPerSplit = 512;
+constexpr int64_t kDecodeMaxQueries = 16;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Plan {
+  Dims D;
+  bool bf16 = false;
+  bool decode = false;
+  int cps = 0, n_split = 0, n_pieces = 0;
+  size_t off_idx = 0, off_ssel = 0, off_pv = 0, off_pc = 0, off_po = 0, off_pl = 0;
+  size_t total = 0;
+};
+
+hils_status check_params(const hils_params* p) {
+  if (!p) return HILS_ERR_INVALID_ARG;
+  if (p->B < 0 || p->N_q < 0 || p->Hq < 1 || p->Hkv < 1 || p->N_kv < 1 || p->d < 1 ||
+      p->q_pos0 < 0 || p->S < 1 || p->K_top < 0 || p->W < 1)
+    return HILS_ERR_INVALID_ARG;
+  if (p->Hq % p->Hkv != 0) return HILS_ERR_INVALID_ARG;
+  if (p->q_pos0 + p->N_q > p->N_kv) return HILS_ERR_INVALID_ARG;
+  if (p->dtype != HILS_F32 && p->dtype != HILS_BF16) return HILS_ERR_INVALID_ARG;
+  if (std::isnan(p->scale) || std::isinf(p->scale)) return HILS_ERR_INVALID_ARG;
+  if (p->d > kMaxD || p->d % 4 != 0) return HILS_ERR_UNSUPPORTED;
+  if (p->K_top > kMaxK) return HILS_ERR_UNSUPPORTED;
+  if (p->Hq / p->Hkv > 16) return HILS_ERR_UNSUPPORTED;
+  if (p->S > 4096) return HILS_ERR_UNSUPPORTED;
+  if (p->N_kv / p->S > (int64_t)INT32_MAX - 1) return HILS_ERR_UNSUPPORTED;
+  return HILS_OK;
+}
+
+Plan make_plan(const hils_params* p) {
+  Plan P;
+  Dims& D = P.D;
+  D.B = p->B; D.Hq = p->Hq; D.Hkv = p->Hkv; D.N_q = p->N_q; D.N_kv = p->N_kv; D.d = p->d;
+  D.q_pos0 = p->q_pos0;
+  D.S = p->S; D.K = p->K_top; D.W = p->W;
+  D.G = (int32_t)(p->Hq / p->Hkv);
+  D.C = p->N_kv / p->S;
+  D.scale = p->scale > 0.f ? p->scale : (float)(1.0 / std::sqrt((double)p->d));
+  P.bf16 = p->dtype == HILS_BF16;
+  P.decode = p->N_q <= kDecodeMaxQueries && (p->d == 64 || p->d == 128);
+
+  const size_t sel_rows = (size_t)(p->B * p->Hkv * p->N_q);
+  const size_t head_rows = (size_t)(p->B * p->Hq * p->N_q);
+  size_t off = kStatusBytes;
+  P.off_idx = off;   off = align_up(off + sel_rows * (size_t)D.K * sizeof(int32_t));
+  P.off_ssel = off;  off = align_up(off + head_rows * (size_t)D.K * sizeof(float));
+  if (P.decode) {
+    int64_t n_max = 0, win_max = 1;
+    for (int64_t i = 0; i < p->N_q; ++i) {
+      const int64_t pos = p->q_pos0 + i;
+      const int64_t n = n_eligible(pos, D.S, D.W);
+      n_max = n > n_max ? n : n_max;
+      const int64_t win = pos - (int64_t)D.S * n + 1;
+      win_max = win > win_max ? win : win_max;
+    }
+    P.cps = kChunksPerSplit;
+    P.n_split = (int)((n_max + P.cps - 1) / P.cps);
+    if (P.n_split < 1) P.n_split = 1;
+    P.n_pieces = (int)((win_max + D.S - 1) / D.S);
+    const int NU = D.K + P.n_pieces;
+    P.off_pv = off; off = align_up(off + sel_rows * P.n_split * (size_t)D.K * sizeof(float));
+    P.off_pc = off; off = align_up(off + sel_rows * P.n_split * (size_t)D.K * sizeof(int32_t));
+    P.off_po = off; off = align_up(off + head_rows * NU * (size_t)D.d * sizeof(float));
+    P.off_pl = off; off = align_up(off + head_rows * NU * sizeof(float));
+  }
+  P.total = off;
+  return P;
+}
+
+hils_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HILS_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return HILS_ERR_CUDA;
+  if (major != 10 || minor != 0) return HILS_ERR_UNSUPPORTED;
+  return HILS_OK;
+}
+
+bool ok_ptr(const void* ptr, bool needed) { return !needed || (ptr && aligned16(ptr)); }
+
+}  // namespace
+}  // namespace hils
+
+using namespace hils;
+
+extern "C" size_t hils_workspace_size(const hils_params* p) {
+  if (check_params(p) != HILS_OK) return 0;
+  return make_plan(p).total;
+}
+
+namespace hils {
+namespace {
+
+// Records the caller's timing events between kernel launches (no-op without events).
+struct PhaseMarks {
+  void* const* ev;
+  int n;
+  int k;
+  cudaStream_t st;
+  void mark() {
+    if (ev && k < n && ev[k]) cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev[k]), st);
+    ++k;
+  }
+};
+
+int phase_names(const Plan& P, const char** names, int max_names) {
+  static const char* kDecode[] = {"select_split", "select_merge", "attn_units", "fuse_units"};
+  static const char* kPrefill[] = {"select_rows", "attn_rows"};
+  const char** src = P.decode ? kDecode : kPrefill;
+  const int n = P.decode ? 4 : 2;
+  for (int i = 0; i < n && i < max_names; ++i) names[i] = src[i];
+  return n;
+}
+
+hils_status forward_impl(const hils_params* p, const void* q, const void* q_cal, const void* K,
+                         const void* V, const void* k_lm, const float* b_lm, void* out,
+                         float* lse_out, int32_t* topk_idx_out, void* workspace,
+                         size_t workspace_bytes, hils_stream_t stream, void* const* events,
+                         int n_events) {
+  hils_status s = check_params(p);
+  if (s != HILS_OK) return s;
+  const Plan P = make_plan(p);
+  const bool any = p->B > 0 && p->N_q > 0;
+  const bool any_lm = any && P.D.C > 0;
+  if (!ok_ptr(q, any) || !ok_ptr(q_cal, any) || !ok_ptr(K, any) || !ok_ptr(V, any) ||
+      !ok_ptr(k_lm, any_lm) || !ok_ptr(b_lm, any_lm) || !ok_ptr(out, any) ||
+      (lse_out && !aligned16(lse_out)) || (topk_idx_out && !aligned16(topk_idx_out)))
+    return HILS_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < P.total) return HILS_ERR_WORKSPACE;
+  if (!any) return HILS_OK;
+  if ((s = check_device()) != HILS_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  PhaseMarks pm{events, n_events, 0, st};
+  char* ws = static_cast<char*>(workspace);
+  int32_t* idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t*>(ws + P.off_idx);
+  float* s_sel = reinterpret_cast<float*>(ws + P.off_ssel);
+  cudaError_t e;
+  pm.mark();
+  if (P.decode) {
+    float* pv = reinterpret_cast<float*>(ws + P.off_pv);
+    int32_t* pc = reinterpret_cast<int32_t*>(ws + P.off_pc);
+    float* po = reinterpret_cast<float*>(ws + P.off_po);
+    float* pl = reinterpret_cast<float*>(ws + P.off_pl);
+    e = launch_select_split(P.D, P.bf16, P.cps, P.n_split, q_cal, k_lm, b_lm, pv, pc, st);
+    pm.mark();
+    if (e == cudaSuccess)
+      e = launch_select_merge(P.D, P.bf16, P.n_split, pv, pc, q_cal, k_lm, b_lm, idx, s_sel, st);
+    pm.mark();
+    if (e == cudaSuccess) e = launch_attn_units(P.D, P.bf16, P.n_pieces, q, K, V, idx, po, pl, st);
+    pm.mark();
+    if (e == cudaSuccess) e = launch_fuse_units(P.D, P.bf16, P.n_pieces, s_sel, po, pl, out, lse_out, st);
+    pm.mark();
+  } else {
+    e = launch_select_rows(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
+    pm.mark();
+    if (e == cudaSuccess)
+      e = launch_attn_rows(P.D, P.bf16, q, K, V, idx, s_sel, out, lse_out, nullptr, nullptr, st);
+    pm.mark();
+  }
+  return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace hils
+
+extern "C" hils_status hils_forward(const hils_params* p, const void* q, const void* q_cal,
+                                    const void* K, const void* V, const void* k_lm,
+                                    const float* b_lm, void* out, float* lse_out,
+                                    int32_t* topk_idx_out, void* workspace,
+                                    size_t workspace_bytes, hils_stream_t stream) {
+  return forward_impl(p, q, q_cal, K, V, k_lm, b_lm, out, lse_out, topk_idx_out, workspace,
+                      workspace_bytes, stream, nullptr, 0);
+}
+
+extern "C" hils_status hils_forward_timed(const hils_params* p, const void* q, const void* q_cal,
+                                          const void* K, const void* V, const void* k_lm,
+                                          const float* b_lm, void* out, float* lse_out,
+                                          int32_t* topk_idx_out, void* workspace,
+                                          size_t workspace_bytes, hils_stream_t stream,
+                                          void* const* events, int n_events) {
+  return forward_impl(p, q, q_cal, K, V, k_lm, b_lm, out, lse_out, topk_idx_out, workspace,
+                      workspace_bytes, stream, events, n_events);
+}
+
+extern "C" int hils_forward_phases(const hils_params* p, const char** names, int max_names) {
+  if (check_params(p) != HILS_OK) return -1;
+  return phase_names(make_plan(p), names, names ? max_names : 0);
+}
+
+extern "C" hils_status hils_select(const hils_params* p, const void* q_cal, const void* k_lm,
+                                   const float* b_lm, int32_t* idx, float* s_sel,
+                                   void* workspace, size_t workspace_bytes,
+                                   hils_stream_t stream) {
+  hils_status s = check_params(p);
+  if (s != HILS_OK) return s;
+  const Plan P = make_plan(p);
+  const bool any = p->B > 0 && p->N_q > 0;
+  const bool any_lm = any && P.D.C > 0;
+  if (!ok_ptr(q_cal, any) || !ok_ptr(k_lm, any_lm) || !ok_ptr(b_lm, any_lm) ||
+      !ok_ptr(idx, any && p->K_top > 0) || (s_sel && !aligned16(s_sel)))
+    return HILS_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < P.total) return HILS_ERR_WORKSPACE;
+  if (!any) return HILS_OK;
+  if ((s = check_device()) != HILS_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  cudaError_t e;
+  if (P.decode) {
+    float* pv = reinterpret_cast<float*>(ws + P.off_pv);
+    int32_t* pc = reinterpret_cast<int32_t*>(ws + P.off_pc);
+    e = launch_select_split(P.D, P.bf16, P.cps, P.n_split, q_cal, k_lm, b_lm, pv, pc, st);
+    if (e == cudaSuccess)
+      e = launch_select_merge(P.D, P.bf16, P.n_split, pv, pc, q_cal, k_lm, b_lm, idx, s_sel, st);
+  } else
+    e = launch_select_rows(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
+  return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA;
+}
+
+extern "C" hils_status hils_chunk_attn(const hils_params* p, const void* q, const void* K,
+                                       const void* V, const int32_t* idx, float* unit_o,
+                                       float* unit_lse, hils_stream_t stream) {
+  hils_status s = check_params(p);
+  if (s != HILS_OK) return s;
+  const Plan P = make_plan(p);
+  const bool any = p->B > 0 && p->N_q > 0;
+  if (!ok_ptr(q, any) || !ok_ptr(K, any) || !ok_ptr(V, any) ||
+      !ok_ptr(idx, any && p->K_top > 0) || !ok_ptr(unit_o, any) || !ok_ptr(unit_lse, any))
+    return HILS_ERR_INVALID_ARG;
+  if (!any) return HILS_OK;
+  if ((s = check_device()) != HILS_OK) return s;
+  cudaError_t e = launch_attn_rows(P.D, P.bf16, q, K, V, idx, nullptr, nullptr, nullptr, unit_o,
+                                   unit_lse, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA;
+}
+
+extern "C" hils_status hils_fuse(const hils_params* p, const float* s_sel, const float* unit_o,
+                                 const float* unit_lse, void* out, float* lse_out,
+                                 hils_stream_t stream) {
+  hils_status s = check_params(p);
+  if (s != HILS_OK) return s;
+  const Plan P = make_plan(p);
+  const bool any = p->B > 0 && p->N_q > 0;
+  if (!ok_ptr(s_sel, any && p->K_top > 0) || !ok_ptr(unit_o, any) || !ok_ptr(unit_lse, any) ||
+      !ok_ptr(out, any) || (lse_out && !aligned16(lse_out)))
+    return HILS_ERR_INVALID_ARG;
+  if (!any) return HILS_OK;
+  if ((s = check_device()) != HILS_OK) return s;
+  cudaError_t e = launch_fuse_units(P.D, P.bf16, 1, s_sel, unit_o, unit_lse, out, lse_out,
+                                    reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA;
+}
+
+extern "C" hils_status hils_workspace_init(void* workspace, size_t workspace_bytes,
+                                           hils_stream_t stream) {
+  if (!workspace || !aligned16(workspace) || workspace_bytes < kStatusBytes)
+    return HILS_ERR_WORKSPACE;
+  return cudaMemsetAsync(workspace, 0, kStatusBytes, reinterpret_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? HILS_OK
+             : HILS_ERR_CUDA;
+}
+
+extern "C" hils_status hils_device_status(void* workspace, hils_stream_t stream,
+                                          int32_t* status) {
+  if (!workspace || !status) return HILS_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemsetAsync(workspace, 0, sizeof(word), st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return HILS_ERR_CUDA;
+  *status = word;
+  return HILS_OK;
+}
+
+extern "C" const char* hils_status_string(hils_status s) {
+  switch (s) {
+    case HILS_OK: return "ok";
+    case HILS_ERR_INVALID_ARG: return "invalid argument";
+    case HILS_ERR_UNSUPPORTED: return "unsupported configuration";
+    case HILS_ERR_WORKSPACE: return "workspace missing or too small";
+    case HILS_ERR_CUDA: return "CUDA error";
+    case HILS_ERR_DEVICE_CHECK: return "device-side check failed";
+    case HILS_ERR_TIMEOUT: return "bounded on-chip wait timed out";
+  }
+  return "unknown status";
+}
+
+extern "C" const char* hils_version(void) { return "hils-b200 " HILS_GIT_DESCRIBE " sm_100a"; }

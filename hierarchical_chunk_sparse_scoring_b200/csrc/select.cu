@@ -1,0 +1,432 @@
+// Steps 1-2 on CUDA cores: landmark scores, group max, top-K with ties to the lower chunk.
+//
+// Surrogate chunk score s_{h,c} = q_cal[h] . k_lm[c] * scale + b_lm[c] ([Reader] "The
+// HiLS-Attention Mechanism" surrogate step and the Q-Cal worked example in "Implementation and
+// Training Recipes"); the group keeps a chunk by the max over its heads ([Reader] GQA
+// paragraph); the K best distant chunks are kept ([Reader] "Limitations of Naive Sparse
+// Attention").  [Reader] = paperglide.net reader of "Hierarchical Sparse Attention Done Right".
+//
+// Two layouts of the same computation:
+//   select_rows_kernel   one warp per (b, g, query): lanes stride over chunks; used where there
+//                        are many queries (prefill) and for any d.
+//   select_split_kernel  many CTAs per (b, g, query) over disjoint chunk ranges, each writing
+//                        its own top-K; select_merge_kernel merges them.  Used for decode,
+//                        where one query's landmark stream (n x d) must be spread over the GPU.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace hils {
+
+// s_sel for the winners held by lanes 0..K-1 (lane r: chunk c_r); per-head dot on CUDA cores.
+template <typename T, int GM>
+__device__ __forceinline__ void write_selection(const Dims& D, int64_t b, int64_t g, int64_t i,
+                                                const float* qs /* [G][d] smem or null */,
+                                                const T* qc, const T* kb, const float* bb,
+                                                int lane, int c, int32_t* idx, float* s_sel) {
+  const int K = D.K, G = D.G, d = (int)D.d;
+  const int64_t sel_row = ((b * D.Hkv + g) * D.N_q + i) * K;
+  if (lane < K) {
+    const bool valid = c != INT_MAX;
+    idx[sel_row + lane] = valid ? c : -1;
+    if (s_sel) {
+      float acc[GM];
+#pragma unroll
+      for (int h = 0; h < GM; ++h) acc[h] = 0.f;
+      if (valid) {
+        const T* kr = kb + (int64_t)c * d;
+        for (int k = 0; k < d; k += 4) {
+          float kv[4];
+          Elem<T>::load4(kr + k, kv);
+#pragma unroll
+          for (int h = 0; h < GM; ++h) {
+            if (h < G) {
+              float qv[4];
+              if (qs) {
+                float4 t = *reinterpret_cast<const float4*>(qs + h * d + k);
+                qv[0] = t.x; qv[1] = t.y; qv[2] = t.z; qv[3] = t.w;
+              } else {
+                Elem<T>::load4(qc + (((b * D.Hq) + g * G + h) * D.N_q + i) * D.d + k, qv);
+              }
+              acc[h] = fmaf(qv[0], kv[0], acc[h]);
+              acc[h] = fmaf(qv[1], kv[1], acc[h]);
+              acc[h] = fmaf(qv[2], kv[2], acc[h]);
+              acc[h] = fmaf(qv[3], kv[3], acc[h]);
+            }
+          }
+        }
+      }
+      const float bc = valid ? bb[c] : 0.f;
+#pragma unroll
+      for (int h = 0; h < GM; ++h) {
+        if (h < G) {
+          const int64_t hrow = ((b * D.Hq) + g * G + h) * D.N_q + i;
+          s_sel[hrow * K + lane] = valid ? fmaf(acc[h], D.scale, bc) : -INFINITY;
+        }
+      }
+    }
+  }
+}
+
+template <typename T, int GM, int KM>
+__global__ void __launch_bounds__(256) select_rows_kernel(Dims D, const T* __restrict__ qc,
+                                                          const T* __restrict__ klm,
+                                                          const float* __restrict__ blm,
+                                                          int32_t* __restrict__ idx,
+                                                          float* __restrict__ s_sel) {
+  extern __shared__ __align__(16) float smem[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t rows = D.B * D.Hkv * D.N_q;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
+  if (row >= rows) return;
+  const int64_t i = row % D.N_q, bg = row / D.N_q, g = bg % D.Hkv, b = bg / D.Hkv;
+  const int d = (int)D.d, G = D.G;
+  float* qs = smem + (size_t)warp * G * d;
+  for (int e = lane; e < G * d; e += 32) {
+    const int h = e / d, k = e - h * d;
+    qs[e] = Elem<T>::to_f(qc[(((b * D.Hq) + g * G + h) * D.N_q + i) * D.d + k]);
+  }
+  __syncwarp();
+  const int64_t n = n_eligible(D.q_pos0 + i, D.S, D.W);
+  const T* kb = klm + bg * D.C * D.d;
+  const float* bb = blm + bg * D.C;
+  TopList<KM> L;
+  L.clear();
+  for (int64_t c = lane; c < n; c += 32) {
+    const T* kr = kb + c * d;
+    float acc[GM];
+#pragma unroll
+    for (int h = 0; h < GM; ++h) acc[h] = 0.f;
+    for (int k = 0; k < d; k += 4) {
+      float kv[4];
+      Elem<T>::load4(kr + k, kv);
+#pragma unroll
+      for (int h = 0; h < GM; ++h) {
+        if (h < G) {
+          float4 qv = *reinterpret_cast<const float4*>(qs + h * d + k);
+          acc[h] = fmaf(qv.x, kv[0], acc[h]);
+          acc[h] = fmaf(qv.y, kv[1], acc[h]);
+          acc[h] = fmaf(qv.z, kv[2], acc[h]);
+          acc[h] = fmaf(qv.w, kv[3], acc[h]);
+        }
+      }
+    }
+    const float bc = bb[c];
+    float sig = -INFINITY;
+#pragma unroll
+    for (int h = 0; h < GM; ++h)
+      if (h < G) sig = fmaxf(sig, fmaf(acc[h], D.scale, bc));
+    L.insert(sig, (int)c, D.K);
+  }
+  float wv;
+  int wc;
+  warp_merge_topk<KM>(L, D.K, lane, wv, wc);
+  write_selection<T, GM>(D, b, g, i, qs, qc, kb, bb, lane, wc, idx, s_sel);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Decode layout.  Lanes are grouped L per landmark row; lane l of a group owns the row's
+// 16-byte vectors l, l+L, l+2L, ... so one warp instruction reads 32/L whole rows contiguously.
+template <typename T, int D_, int GM>
+struct SplitShape {
+  static constexpr int DPL = GM <= 4 ? 16 : (GM == 8 ? 8 : 4);   // dims per lane
+  static constexpr int L = D_ / DPL;                              // lanes per row
+  static constexpr int VEC = (16 / (int)sizeof(T)) < DPL ? (16 / (int)sizeof(T)) : DPL;
+  static constexpr int NV = DPL / VEC;                            // vector loads per row
+  static constexpr int RPW = 32 / L;                              // rows per warp step
+  static_assert(L >= 1 && L <= 32 && (32 % L) == 0, "lane grouping");
+};
+
+template <typename T, int VEC>
+__device__ __forceinline__ void load_vec(const T* p, float (&v)[VEC]);
+
+template <>
+__device__ __forceinline__ void load_vec<__nv_bfloat16, 8>(const __nv_bfloat16* p, float (&v)[8]) {
+  uint4 t = __ldg(reinterpret_cast<const uint4*>(p));
+  v[0] = bf16_lo(t.x); v[1] = bf16_hi(t.x); v[2] = bf16_lo(t.y); v[3] = bf16_hi(t.y);
+  v[4] = bf16_lo(t.z); v[5] = bf16_hi(t.z); v[6] = bf16_lo(t.w); v[7] = bf16_hi(t.w);
+}
+template <>
+__device__ __forceinline__ void load_vec<__nv_bfloat16, 4>(const __nv_bfloat16* p, float (&v)[4]) {
+  Elem<__nv_bfloat16>::load4(p, v);
+}
+template <>
+__device__ __forceinline__ void load_vec<float, 4>(const float* p, float (&v)[4]) {
+  Elem<float>::load4(p, v);
+}
+
+constexpr int kSplitThreads = 256;
+constexpr int kSplitWarps = kSplitThreads / 32;
+
+template <typename T, int D_, int GM, int KM>
+__global__ void __launch_bounds__(kSplitThreads) select_split_kernel(
+    Dims D, int cps, int n_split, const T* __restrict__ qc, const T* __restrict__ klm,
+    const float* __restrict__ blm, float* __restrict__ part_v, int32_t* __restrict__ part_c) {
+  using SS = SplitShape<T, D_, GM>;
+  extern __shared__ __align__(16) float sig_buf[];   // [cps] scores, then [warps][K] lists
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int split = blockIdx.x;
+  const int64_t row = blockIdx.y;
+  const int64_t i = row % D.N_q, bg = row / D.N_q, g = bg % D.Hkv, b = bg / D.Hkv;
+  const int G = D.G, K = D.K;
+  const int64_t n = n_eligible(D.q_pos0 + i, D.S, D.W);
+  const int64_t c0 = (int64_t)split * cps;
+  const int64_t c1 = c0 + cps < n ? c0 + cps : n;
+  const int cnt = c1 > c0 ? (int)(c1 - c0) : 0;
+
+  // this lane's slice of every head's calibrated query, in registers
+  const int grp = lane / SS::L, gl = lane % SS::L;
+  float qreg[GM][SS::DPL];
+#pragma unroll
+  for (int h = 0; h < GM; ++h) {
+#pragma unroll
+    for (int v = 0; v < SS::NV; ++v) {
+      float t[SS::VEC];
+      if (h < G) {
+        load_vec<T, SS::VEC>(qc + (((b * D.Hq) + g * G + h) * D.N_q + i) * D_ +
+                                 (v * SS::L + gl) * SS::VEC, t);
+      } else {
+#pragma unroll
+        for (int e = 0; e < SS::VEC; ++e) t[e] = 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < SS::VEC; ++e) qreg[h][v * SS::VEC + e] = t[e];
+    }
+  }
+
+  const T* kb = klm + bg * D.C * D_;
+  const float* bb = blm + bg * D.C;
+  constexpr int U = 2;   // warp steps in flight per iteration
+  for (int base = warp * SS::RPW; base < cnt; base += kSplitWarps * SS::RPW * U) {
+    float kv[U][SS::DPL];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int r = base + u * kSplitWarps * SS::RPW + grp;
+      if (r < cnt) {
+        const T* kr = kb + (c0 + r) * D_;
+#pragma unroll
+        for (int v = 0; v < SS::NV; ++v) {
+          float t[SS::VEC];
+          load_vec<T, SS::VEC>(kr + (v * SS::L + gl) * SS::VEC, t);
+#pragma unroll
+          for (int e = 0; e < SS::VEC; ++e) kv[u][v * SS::VEC + e] = t[e];
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < SS::DPL; ++e) kv[u][e] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int r = base + u * kSplitWarps * SS::RPW + grp;
+      float acc[GM];
+#pragma unroll
+      for (int h = 0; h < GM; ++h) {
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < SS::DPL; ++e) a = fmaf(qreg[h][e], kv[u][e], a);
+        acc[h] = a;
+      }
+#pragma unroll
+      for (int o = SS::L / 2; o > 0; o >>= 1) {
+#pragma unroll
+        for (int h = 0; h < GM; ++h) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
+      }
+      if (gl == 0 && r < cnt) {
+        const float bc = bb[c0 + r];
+        float sig = -INFINITY;
+#pragma unroll
+        for (int h = 0; h < GM; ++h)
+          if (h < G) sig = fmaxf(sig, fmaf(acc[h], D.scale, bc));
+        sig_buf[r] = sig;
+      }
+    }
+  }
+  __syncthreads();
+
+  // top-K of this split: per-lane lists, warp merge, then one warp merges the warps' lists
+  TopList<KM> Ls;
+  Ls.clear();
+  for (int r = threadIdx.x; r < cnt; r += kSplitThreads) Ls.insert(sig_buf[r], (int)(c0 + r), K);
+  float wv;
+  int wc;
+  warp_merge_topk<KM>(Ls, K, lane, wv, wc);
+  __syncthreads();   // sig_buf is reused below
+  float* lv = sig_buf;                                           // [warps][K]
+  int* lc = reinterpret_cast<int*>(sig_buf + kSplitWarps * kMaxK);
+  if (lane < K) { lv[warp * K + lane] = wv; lc[warp * K + lane] = wc; }
+  __syncthreads();
+  if (warp == 0) {
+    int ptr = 0;
+    float* outv = part_v + (row * n_split + split) * K;
+    int32_t* outc = part_c + (row * n_split + split) * K;
+    for (int r = 0; r < K; ++r) {
+      float v = -INFINITY;
+      int c = INT_MAX;
+      if (lane < kSplitWarps && ptr < K) { v = lv[lane * K + ptr]; c = lc[lane * K + ptr]; }
+      float bv = v;
+      int bc = c;
+      warp_best(bv, bc);
+      if (lane < kSplitWarps && c == bc && bc != INT_MAX) ++ptr;
+      if (lane == 0) { outv[r] = bv; outc[r] = bc; }
+    }
+  }
+}
+
+template <typename T, int GM, int KM>
+__global__ void __launch_bounds__(128) select_merge_kernel(Dims D, int n_split,
+                                                           const float* __restrict__ part_v,
+                                                           const int32_t* __restrict__ part_c,
+                                                           const T* __restrict__ qc,
+                                                           const T* __restrict__ klm,
+                                                           const float* __restrict__ blm,
+                                                           int32_t* __restrict__ idx,
+                                                           float* __restrict__ s_sel) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t rows = D.B * D.Hkv * D.N_q;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
+  if (row >= rows) return;
+  const int64_t i = row % D.N_q, bg = row / D.N_q, g = bg % D.Hkv, b = bg / D.Hkv;
+  const int K = D.K;
+  TopList<KM> L;
+  L.clear();
+  const int total = n_split * K;
+  for (int e = lane; e < total; e += 32)
+    L.insert(part_v[row * total + e], part_c[row * total + e], K);
+  float wv;
+  int wc;
+  warp_merge_topk<KM>(L, K, lane, wv, wc);
+  write_selection<T, GM>(D, b, g, i, nullptr, qc, klm + bg * D.C * D.d, blm + bg * D.C, lane,
+                         wc, idx, s_sel);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Host-side launchers.
+
+template <typename T, int GM, int KM>
+static cudaError_t launch_rows_t(const Dims& D, const void* qc, const void* klm, const float* blm,
+                                 int32_t* idx, float* s_sel, cudaStream_t st) {
+  const int per_warp = D.G * (int)D.d * (int)sizeof(float);
+  int warps = 49152 / per_warp;
+  if (warps > 8) warps = 8;
+  if (warps < 1) warps = 1;
+  const int64_t rows = D.B * D.Hkv * D.N_q;
+  const int64_t blocks = (rows + warps - 1) / warps;
+  select_rows_kernel<T, GM, KM><<<(unsigned)blocks, warps * 32, (size_t)warps * per_warp, st>>>(
+      D, (const T*)qc, (const T*)klm, blm, idx, s_sel);
+  return cudaGetLastError();
+}
+
+template <typename T, int GM>
+static cudaError_t launch_rows_k(const Dims& D, const void* qc, const void* klm, const float* blm,
+                                 int32_t* idx, float* s_sel, cudaStream_t st) {
+  if (D.K <= 8) return launch_rows_t<T, GM, 8>(D, qc, klm, blm, idx, s_sel, st);
+  if (D.K <= 16) return launch_rows_t<T, GM, 16>(D, qc, klm, blm, idx, s_sel, st);
+  return launch_rows_t<T, GM, 32>(D, qc, klm, blm, idx, s_sel, st);
+}
+
+template <typename T>
+static cudaError_t launch_rows_g(const Dims& D, const void* qc, const void* klm, const float* blm,
+                                 int32_t* idx, float* s_sel, cudaStream_t st) {
+  if (D.G <= 1) return launch_rows_k<T, 1>(D, qc, klm, blm, idx, s_sel, st);
+  if (D.G <= 2) return launch_rows_k<T, 2>(D, qc, klm, blm, idx, s_sel, st);
+  if (D.G <= 4) return launch_rows_k<T, 4>(D, qc, klm, blm, idx, s_sel, st);
+  if (D.G <= 8) return launch_rows_k<T, 8>(D, qc, klm, blm, idx, s_sel, st);
+  return launch_rows_k<T, 16>(D, qc, klm, blm, idx, s_sel, st);
+}
+
+cudaError_t launch_select_rows(const Dims& D, bool bf16, const void* qc, const void* klm,
+                               const float* blm, int32_t* idx, float* s_sel, cudaStream_t st) {
+  if (D.B * D.Hkv * D.N_q == 0) return cudaSuccess;
+  return bf16 ? launch_rows_g<__nv_bfloat16>(D, qc, klm, blm, idx, s_sel, st)
+              : launch_rows_g<float>(D, qc, klm, blm, idx, s_sel, st);
+}
+
+size_t split_smem_bytes(int cps) {
+  size_t a = (size_t)cps * sizeof(float);
+  size_t b = (size_t)kSplitWarps * kMaxK * (sizeof(float) + sizeof(int));
+  return a > b ? a : b;
+}
+
+template <typename T, int D_, int GM, int KM>
+static cudaError_t launch_split_t(const Dims& D, int cps, int n_split, const void* qc,
+                                  const void* klm, const float* blm, float* pv, int32_t* pc,
+                                  cudaStream_t st) {
+  const int64_t rows = D.B * D.Hkv * D.N_q;
+  const size_t smem = split_smem_bytes(cps);
+  auto kern = select_split_kernel<T, D_, GM, KM>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid((unsigned)n_split, (unsigned)rows);
+  kern<<<grid, kSplitThreads, smem, st>>>(D, cps, n_split, (const T*)qc, (const T*)klm, blm, pv,
+                                          pc);
+  return cudaGetLastError();
+}
+
+template <typename T, int GM, int KM>
+static cudaError_t launch_merge_t(const Dims& D, int n_split, const float* pv, const int32_t* pc,
+                                  const void* qc, const void* klm, const float* blm, int32_t* idx,
+                                  float* s_sel, cudaStream_t st) {
+  const int64_t rows = D.B * D.Hkv * D.N_q;
+  select_merge_kernel<T, GM, KM><<<(unsigned)((rows + 3) / 4), 128, 0, st>>>(
+      D, n_split, pv, pc, (const T*)qc, (const T*)klm, blm, idx, s_sel);
+  return cudaGetLastError();
+}
+
+// Dispatch on (dtype, d, group size, list length) for a callable templated on them.
+template <template <typename, int, int, int> class F, typename... A>
+static cudaError_t dispatch_tdgk(bool bf16, int64_t d, int G, int K, A... a) {
+#define HILS_K(T, D_, GM)                                         \
+  if (K <= 8) return F<T, D_, GM, 8>::run(a...);                  \
+  if (K <= 16) return F<T, D_, GM, 16>::run(a...);                \
+  return F<T, D_, GM, 32>::run(a...);
+#define HILS_G(T, D_)                                             \
+  if (G <= 4) { HILS_K(T, D_, 4) }                                \
+  if (G <= 8) { HILS_K(T, D_, 8) }                                \
+  HILS_K(T, D_, 16)
+  if (bf16) {
+    if (d == 128) { HILS_G(__nv_bfloat16, 128) }
+    HILS_G(__nv_bfloat16, 64)
+  }
+  if (d == 128) { HILS_G(float, 128) }
+  HILS_G(float, 64)
+#undef HILS_G
+#undef HILS_K
+}
+
+template <typename T, int D_, int GM, int KM>
+struct SplitRun {
+  static cudaError_t run(const Dims* D, int cps, int n_split, const void* qc, const void* klm,
+                         const float* blm, float* pv, int32_t* pc, cudaStream_t st) {
+    return launch_split_t<T, D_, GM, KM>(*D, cps, n_split, qc, klm, blm, pv, pc, st);
+  }
+};
+
+template <typename T, int D_, int GM, int KM>
+struct MergeRun {
+  static cudaError_t run(const Dims* D, int n_split, const float* pv, const int32_t* pc,
+                         const void* qc, const void* klm, const float* blm, int32_t* idx,
+                         float* s_sel, cudaStream_t st) {
+    return launch_merge_t<T, GM, KM>(*D, n_split, pv, pc, qc, klm, blm, idx, s_sel, st);
+  }
+};
+
+cudaError_t launch_select_split(const Dims& D, bool bf16, int cps, int n_split, const void* qc,
+                                const void* klm, const float* blm, float* part_v,
+                                int32_t* part_c, cudaStream_t st) {
+  if (D.B * D.Hkv * D.N_q == 0) return cudaSuccess;
+  return dispatch_tdgk<SplitRun>(bf16, D.d, D.G, D.K, &D, cps, n_split, qc, klm, blm, part_v,
+                                 part_c, st);
+}
+
+cudaError_t launch_select_merge(const Dims& D, bool bf16, int n_split, const float* part_v,
+                                const int32_t* part_c, const void* qc, const void* klm,
+                                const float* blm, int32_t* idx, float* s_sel, cudaStream_t st) {
+  if (D.B * D.Hkv * D.N_q == 0) return cudaSuccess;
+  return dispatch_tdgk<MergeRun>(bf16, D.d, D.G, D.K, &D, n_split, part_v, part_c, qc, klm, blm,
+                                 idx, s_sel, st);
+}
+
+}  // namespace hils

@@ -1,0 +1,154 @@
+/*
+ * hils.h -- C ABI of the B200 (sm_100a) HiLS attention forward pass.
+ *
+ * HiLS = Hierarchical Landmark Sparse attention, from the paper "Hierarchical Sparse Attention
+ * Done Right: Toward Infinite Context Modeling" (arXiv 2607.02980).  Citations name the page
+ * and its section or figure:
+ *   [Reader]   paperglide.net simplified reader of the paper
+ *   [Abstract] engineersofai.com paper breakdown, "Abstract"
+ *   [Essay]    nestfrontier.com, "Long context just stopped being a memory problem"
+ *
+ * Notation.  B batch; Hq query heads; Hkv KV heads; G = Hq/Hkv; query head h reads KV head
+ * floor(h/G) ([Reader] "Implementation and Training Recipes", GQA paragraph: heads sharing a KV
+ * head).  d head dim; S chunk size; C = floor(N_kv/S) completed chunks, each with one landmark
+ * key k_lm[c] and bias b_lm[c]; K = K_top; W local window.  Query i sits at position
+ * p = q_pos0 + i.  Eligible distant chunks: n = floor(max(0, p-W+1)/S), chunks 0..n-1; the
+ * local window is tokens [S*n, p] (covers every token <= p exactly once with the chunks).
+ *
+ * Layouts (row-major, contiguous, base pointers 16-byte aligned, all device memory):
+ *   q, q_cal, out       [B, Hq,  N_q,  d]   dtype
+ *   K, V                [B, Hkv, N_kv, d]   dtype
+ *   k_lm                [B, Hkv, C,    d]   dtype
+ *   b_lm                [B, Hkv, C]         fp32
+ *   idx                 [B, Hkv, N_q, K]    int32, ordered (sigma desc, c asc), -1 padded
+ *   s_sel               [B, Hq,  N_q, K]    fp32 per-head score of each selected chunk
+ *                                           (-inf where idx is -1)
+ *   unit_o              [B, Hq,  N_q, K+1, d] fp32; slot k < K = chunk idx[k], slot K = window
+ *   unit_lse, lse       [B, Hq,  N_q, K+1] / [B, Hq, N_q] fp32
+ *
+ * Ownership and errors.  The caller owns every buffer, including the workspace; the library
+ * allocates no device memory and keeps no state between calls.  Arguments are checked on the
+ * host before anything is launched: a bad argument returns an error with nothing written.
+ * Otherwise the call is asynchronous on `stream` and returns HILS_ERR_CUDA if a launch fails.
+ * Kernels that wait on on-chip barriers give up after a bounded number of polls and record
+ * HILS_ERR_TIMEOUT in the workspace's status word (read it with hils_device_status after the
+ * stream is synchronised).  No exception crosses this interface.
+ *
+ * Supported: sm_100a device; dtype fp32 (CUDA-core FFMA, no TF32) or bf16 (fp32 accumulate);
+ * 4 <= d <= 128 with d % 4 == 0; 1 <= S <= 4096; 0 <= K <= 32; W >= 1; 1 <= G <= 16;
+ * q_pos0 + N_q <= N_kv; B or N_q may be 0 (nothing is launched).  Anything else returns HILS_ERR_UNSUPPORTED or
+ * HILS_ERR_INVALID_ARG; there is no fallback path.
+ */
+#ifndef HILS_H
+#define HILS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* hils_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  HILS_OK = 0,
+  HILS_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, inconsistent sizes */
+  HILS_ERR_UNSUPPORTED = 2,  /* valid but outside the supported set above */
+  HILS_ERR_WORKSPACE = 3,    /* workspace missing or smaller than hils_workspace_size() */
+  HILS_ERR_CUDA = 4,         /* a CUDA call or kernel launch failed */
+  HILS_ERR_DEVICE_CHECK = 5, /* a kernel's own bounds check fired (status word) */
+  HILS_ERR_TIMEOUT = 6       /* a bounded on-chip wait gave up (status word) */
+} hils_status;
+
+typedef enum { HILS_F32 = 0, HILS_BF16 = 1 } hils_dtype;
+
+typedef struct {
+  int64_t B, Hq, Hkv;
+  int64_t N_q, N_kv, d;
+  int64_t q_pos0;   /* position of query 0: prefill 0 (N_q == N_kv); decode N_kv - 1 (N_q == 1) */
+  int32_t S, K_top, W;
+  int32_t dtype;    /* hils_dtype of q, q_cal, K, V, k_lm and out */
+  float scale;      /* logit scale for chunk and token scores; <= 0 means 1/sqrt(d) */
+} hils_params;
+
+/* Bytes of scratch the calls below need for these parameters (>= 256). */
+size_t hils_workspace_size(const hils_params* p);
+
+/*
+ * The whole forward pass, steps 1-4 ([Essay] "The routing problem hiding inside sparse
+ * attention": score the chunk summaries, keep the top K distant chunks, token attention inside
+ * them and the local window, hierarchical softmax; [Reader] Fig. 3 caption):
+ *   out[b,h,i]  = sum_u w_u o_u, w = softmax_u(score_u), score = s_{h,c} for each selected chunk
+ *                 and the window's exact log-sum-exp for the window ([Abstract]: per-chunk
+ *                 outputs fused according to chunk retrieval scores);
+ *   lse_out     = logsumexp_u score_u (nullable);
+ *   topk_idx_out = the selection (nullable).
+ * q scores tokens, q_cal scores chunks ([Reader] "Implementation and Training Recipes", Q-Cal).
+ */
+hils_status hils_forward(const hils_params* p, const void* q, const void* q_cal, const void* K,
+                         const void* V, const void* k_lm, const float* b_lm, void* out,
+                         float* lse_out, int32_t* topk_idx_out, void* workspace,
+                         size_t workspace_bytes, hils_stream_t stream);
+
+/*
+ * hils_forward with phase timing: `events` holds n_events cudaEvent_t handles created by the
+ * caller; events[0] is recorded on `stream` before the first kernel and events[k] right after
+ * the k-th kernel (k >= 1), as far as n_events reaches.  Everything else is hils_forward.
+ */
+hils_status hils_forward_timed(const hils_params* p, const void* q, const void* q_cal,
+                               const void* K, const void* V, const void* k_lm, const float* b_lm,
+                               void* out, float* lse_out, int32_t* topk_idx_out, void* workspace,
+                               size_t workspace_bytes, hils_stream_t stream, void* const* events,
+                               int n_events);
+
+/* Number of kernels hils_forward launches for these parameters (-1 if they are invalid); the
+ * first max_names of their names are stored in names (static strings; names may be NULL). */
+int hils_forward_phases(const hils_params* p, const char** names, int max_names);
+
+/*
+ * Steps 1-2: s_{h,i,c} = q_cal[b,h,i] . k_lm[b,g,c] * scale + b_lm[b,g,c] for every eligible c
+ * ([Reader] "The HiLS-Attention Mechanism", surrogate score; Q-Cal worked example), group score
+ * sigma = max over the G heads of KV head g ([Reader] GQA paragraph), and the K largest sigma
+ * with ties to the lower chunk index ([Reader] "Limitations of Naive Sparse Attention": top-K
+ * distant chunks).  Writes idx and, if non-NULL, s_sel (the per-head scores of those chunks).
+ */
+hils_status hils_select(const hils_params* p, const void* q_cal, const void* k_lm,
+                        const float* b_lm, int32_t* idx, float* s_sel, void* workspace,
+                        size_t workspace_bytes, hils_stream_t stream);
+
+/*
+ * Step 3: exact softmax attention of q[b,h,i] inside each selected chunk (idx as produced by
+ * hils_select; -1 entries, and ids that are not eligible chunks of that query, give
+ * unit_o = 0, unit_lse = -inf) and inside the local window
+ * ([Reader] Fig. 3 caption: intra-chunk softmax; [Abstract]: each query attends independently
+ * with each retrieved chunk).  Writes unit_o and unit_lse (layouts above).
+ */
+hils_status hils_chunk_attn(const hils_params* p, const void* q, const void* K, const void* V,
+                            const int32_t* idx, float* unit_o, float* unit_lse,
+                            hils_stream_t stream);
+
+/*
+ * Step 4: w_u = softmax over {s_sel[k] : idx[k] >= 0} and the window's unit_lse[K];
+ * out = sum_u w_u unit_o[u]; lse_out = logsumexp (nullable).  ([Reader] Fig. 3 caption:
+ * inter-chunk softmax; [Abstract]: fusion by chunk retrieval scores.)
+ */
+hils_status hils_fuse(const hils_params* p, const float* s_sel, const float* unit_o,
+                      const float* unit_lse, void* out, float* lse_out, hils_stream_t stream);
+
+/* Zeroes the workspace's status word; call once on a newly allocated workspace. */
+hils_status hils_workspace_init(void* workspace, size_t workspace_bytes, hils_stream_t stream);
+
+/* Copies the workspace's status word to *status (HILS_OK or the first failure a kernel
+ * recorded) and clears it.  Synchronous on `stream`. */
+hils_status hils_device_status(void* workspace, hils_stream_t stream, int32_t* status);
+
+const char* hils_status_string(hils_status s);
+
+/* Library build identification: "hils-b200 <git-describe> sm_100a". */
+const char* hils_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -139,9 +139,11 @@ class Query:
         self.idx_in = None if idx_in is None else np.ascontiguousarray(idx_in, np.int32)
 
 
-def run_queries(queries, *, d, G, S, K_top, W, scale=0.0, units=False, threads=0):
+def run_queries(queries, *, d, G, S, K_top, W, scale=0.0, units=False, threads=0,
+                select_only=False):
     """Runs independent (query, KV head) problems; returns one result dict per query with
-    idx [K], sigma [K], gap, s_sel [G,K], out [G,d], lse [G] (+ unit_o, unit_lse)."""
+    idx [K], sigma [K], gap, s_sel [G,K], out [G,d], lse [G] (+ unit_o, unit_lse).
+    select_only: steps 1-2 only (out / lse are not computed and no K/V rows are read)."""
     n = len(queries)
     jobs = (Job * max(n, 1))()
     results = []
@@ -162,8 +164,11 @@ def run_queries(queries, *, d, G, S, K_top, W, scale=0.0, units=False, threads=0
         jb.idx_in = _ptr(qu.idx_in)
         jb.idx_out, jb.sigma_out, jb.gap_out = _ptr(r["idx"]), _ptr(r["sigma"]), _ptr(r["gap"])
         jb.s_sel_out, jb.s_sel_hs = _ptr(r["s_sel"]), K_top
-        jb.out, jb.out_hs = _ptr(r["out"]), d
-        jb.lse_out, jb.lse_hs = _ptr(r["lse"]), 1
+        if select_only:
+            r.pop("out")
+            r.pop("lse")
+        jb.out, jb.out_hs = _ptr(r.get("out")), d
+        jb.lse_out, jb.lse_hs = _ptr(r.get("lse")), 1
         jb.unit_o_out, jb.unit_o_hs = _ptr(r.get("unit_o")), (K_top + 1) * d
         jb.unit_lse_out, jb.unit_lse_hs = _ptr(r.get("unit_lse")), K_top + 1
         results.append(r)

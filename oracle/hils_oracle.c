@@ -159,17 +159,29 @@ static int run_job(const hils_oracle_cfg* cfg, hils_oracle_job* jb) {
     for (int r = 0; r < Kt; ++r) jb->sigma_out[r] = r < k_sel ? sel_sigma[r] : -INFINITY;
   if (jb->gap_out) *jb->gap_out = gap;
 
-  /* Steps 3 and 4 for each head of the group. */
+  /* Steps 3 and 4 for each head of the group (skipped when none of their outputs is wanted,
+   * so a selection-only job needs no K/V rows). */
+  const int want_attend = jb->out || jb->lse_out || jb->unit_o_out || jb->unit_lse_out;
   for (int h = 0; h < G; ++h) {
     const double* qh = jb->q + h * jb->q_hs;
     const double* qch = jb->qc + h * jb->qc_hs;
+    /* this head's own surrogate score of each selected chunk (R4) */
+    for (int64_t r = 0; r < k_sel; ++r) {
+      int64_t c = sel[r];
+      score[r] = dot(qch, jb->klm + c * (int64_t)d, d) * scale + jb->blm[c];
+    }
+    if (!want_attend) {
+      if (jb->s_sel_out)
+        for (int r = 0; r < Kt; ++r)
+          jb->s_sel_out[h * jb->s_sel_hs + r] = r < k_sel ? score[r] : -INFINITY;
+      continue;
+    }
     /* step 3: one unit per selected chunk, then the local window as unit Kt */
     for (int64_t r = 0; r < k_sel; ++r) {
       int64_t c = sel[r];
       rc = attend_unit(qh, &jb->K, &jb->V, c * S, c * S + S, d, scale, x_buf, &unit_lse[r],
                        unit_o + r * d);
       if (rc) goto done;
-      score[r] = dot(qch, jb->klm + c * (int64_t)d, d) * scale + jb->blm[c];
     }
     for (int64_t r = k_sel; r < Kt; ++r) {
       unit_lse[r] = -INFINITY;
