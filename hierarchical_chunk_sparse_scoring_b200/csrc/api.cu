@@ -63,7 +63,9 @@ Plan make_plan(const hils_params* p) {
   D.C = p->N_kv / p->S;
   D.scale = p->scale > 0.f ? p->scale : (float)(1.0 / std::sqrt((double)p->d));
   P.bf16 = p->dtype == HILS_BF16;
-  P.decode = p->N_q <= kDecodeMaxQueries && (p->d == 64 || p->d == 128);
+  // decode kernels put (b, g, query) rows on grid.y (<= 65535)
+  P.decode = p->N_q <= kDecodeMaxQueries && (p->d == 64 || p->d == 128) &&
+             p->B * p->Hkv * p->N_q <= 65535;
 
   const size_t sel_rows = (size_t)(p->B * p->Hkv * p->N_q);
   const size_t head_rows = (size_t)(p->B * p->Hq * p->N_q);
