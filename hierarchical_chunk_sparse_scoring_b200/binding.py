@@ -99,7 +99,7 @@ def workspace_size(p):
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    return None if t is None or t.numel() == 0 else ctypes.c_void_p(t.data_ptr())
 
 
 def _stream(stream):
@@ -135,7 +135,8 @@ def workspace(p, device, stream=None):
     from the same stream."""
     need = workspace_size(p)
     if need == 0:
-        raise HilsError(1, "hils_workspace_size")
+        # invalid or unsupported parameters: the library call reports which, before any launch
+        return torch.empty(0, dtype=torch.uint8, device=device)
     st = stream if stream is not None else torch.cuda.current_stream(device)
     key = (torch.device(device).index, st.cuda_stream)
     buf = _ws_cache.get(key)

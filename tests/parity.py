@@ -31,6 +31,8 @@ def check_selection(gidx, oidx, gap, sig_gpu, sig_ora, n):
     the oracle's sorted sigmas; n [R] eligible counts.  Returns (exact_rows, tie_rows)."""
     R, K = gidx.shape
     exact = ties = 0
+    if K == 0:
+        return R, 0
     for r in range(R):
         k = min(K, int(n[r]))
         g = gidx[r]
@@ -82,9 +84,10 @@ def full_check(wl, out, lse, idx, threads=0):
     forced = oracle.forward(*arrs, idx_in=gidx, **kw)
     B, Hkv, Nq, K = gidx.shape
     n = np.array([eligible(wl.q_pos0 + i, wl.S, wl.W) for i in range(Nq)])
-    exact, ties = check_selection(gidx.reshape(-1, K), own["idx"].reshape(-1, K),
-                                  own["gap"].reshape(-1), forced["sigma"].reshape(-1, K),
-                                  own["sigma"].reshape(-1, K), np.tile(n, B * Hkv))
+    R = B * Hkv * Nq
+    exact, ties = check_selection(gidx.reshape(R, K), own["idx"].reshape(R, K),
+                                  own["gap"].reshape(R), forced["sigma"].reshape(R, K),
+                                  own["sigma"].reshape(R, K), np.tile(n, B * Hkv))
     errs = compare_outputs(f64(out), forced["out"], f64(lse), forced["lse"], wl.q.dtype)
     errs.update(exact_rows=exact, tie_rows=ties)
     return errs
