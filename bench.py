@@ -84,10 +84,10 @@ def work_model(dims, S, K, W, q_pos0, es):
 
 def phase_work(name, wm):
     """(bound, algorithmic work, unit) of a kernel, for its roofline."""
-    if name.startswith("select_split"):
-        return "hbm", wm["select_bytes"], "GB/s"
-    if name.startswith("select"):
+    if name in ("score_topk_tc", "select_rows"):
         return "tensor", wm["score_flops"], "TFLOP/s"
+    if name == "select_split":
+        return "hbm", wm["select_bytes"], "GB/s"
     if name == "attn_units":
         return "hbm", wm["attn_bytes"], "GB/s"
     if name.startswith("attn"):

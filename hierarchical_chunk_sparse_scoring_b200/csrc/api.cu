@@ -31,6 +31,7 @@ struct Plan {
   Dims D;
   bool bf16 = false;
   bool decode = false;
+  bool tc_select = false;
   int cps = 0, n_split = 0, n_pieces = 0;
   size_t off_idx = 0, off_ssel = 0, off_pv = 0, off_pc = 0, off_po = 0, off_pl = 0;
   size_t total = 0;
@@ -66,6 +67,7 @@ Plan make_plan(const hils_params* p) {
   // decode kernels put (b, g, query) rows on grid.y (<= 65535)
   P.decode = p->N_q <= kDecodeMaxQueries && (p->d == 64 || p->d == 128) &&
              p->B * p->Hkv * p->N_q <= 65535;
+  P.tc_select = !P.decode && score_tc_supported(D, P.bf16);
 
   const size_t sel_rows = (size_t)(p->B * p->Hkv * p->N_q);
   const size_t head_rows = (size_t)(p->B * p->Hq * p->N_q);
@@ -136,8 +138,9 @@ struct PhaseMarks {
 int phase_names(const Plan& P, const char** names, int max_names) {
   static const char* kDecode[] = {"select_split", "select_merge", "attn_units", "fuse_units"};
   static const char* kPrefill[] = {"select_rows", "attn_rows"};
-  const char** src = P.decode ? kDecode : kPrefill;
-  const int n = P.decode ? 4 : 2;
+  static const char* kPrefillTc[] = {"score_topk_tc", "select_scores", "attn_rows"};
+  const char** src = P.decode ? kDecode : (P.tc_select ? kPrefillTc : kPrefill);
+  const int n = P.decode ? 4 : (P.tc_select ? 3 : 2);
   for (int i = 0; i < n && i < max_names; ++i) names[i] = src[i];
   return n;
 }
@@ -181,7 +184,13 @@ hils_status forward_impl(const hils_params* p, const void* q, const void* q_cal,
     if (e == cudaSuccess) e = launch_fuse_units(P.D, P.bf16, P.n_pieces, s_sel, po, pl, out, lse_out, st);
     pm.mark();
   } else {
-    e = launch_select_rows(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
+    if (P.tc_select) {
+      e = launch_score_topk_tc(P.D, q_cal, k_lm, b_lm, idx, reinterpret_cast<int32_t*>(ws), st);
+      pm.mark();
+      if (e == cudaSuccess) e = launch_select_scores(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
+    } else {
+      e = launch_select_rows(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
+    }
     pm.mark();
     if (e == cudaSuccess)
       e = launch_attn_rows(P.D, P.bf16, q, K, V, idx, s_sel, out, lse_out, nullptr, nullptr, st);
@@ -241,8 +250,13 @@ extern "C" hils_status hils_select(const hils_params* p, const void* q_cal, cons
     e = launch_select_split(P.D, P.bf16, P.cps, P.n_split, q_cal, k_lm, b_lm, pv, pc, st);
     if (e == cudaSuccess)
       e = launch_select_merge(P.D, P.bf16, P.n_split, pv, pc, q_cal, k_lm, b_lm, idx, s_sel, st);
-  } else
+  } else if (P.tc_select) {
+    e = launch_score_topk_tc(P.D, q_cal, k_lm, b_lm, idx, reinterpret_cast<int32_t*>(ws), st);
+    if (e == cudaSuccess && s_sel)
+      e = launch_select_scores(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
+  } else {
     e = launch_select_rows(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
+  }
   return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA;
 }
 

@@ -12,6 +12,15 @@ struct Dims;
 cudaError_t launch_select_rows(const Dims& D, bool bf16, const void* qc, const void* klm,
                                const float* blm, int32_t* idx, float* s_sel, cudaStream_t st);
 
+cudaError_t launch_select_scores(const Dims& D, bool bf16, const void* qc, const void* klm,
+                                 const float* blm, const int32_t* idx, float* s_sel,
+                                 cudaStream_t st);
+
+bool score_tc_supported(const Dims& D, bool bf16);
+cudaError_t launch_score_topk_tc(const Dims& D, const void* qc, const void* klm,
+                                 const float* blm, int32_t* idx, int32_t* status,
+                                 cudaStream_t st);
+
 size_t split_smem_bytes(int cps);
 cudaError_t launch_select_split(const Dims& D, bool bf16, int cps, int n_split, const void* qc,
                                 const void* klm, const float* blm, float* part_v,

@@ -123,6 +123,79 @@ __global__ void __launch_bounds__(256) select_rows_kernel(Dims D, const T* __res
   write_selection<T, GM>(D, b, g, i, qs, qc, kb, bb, lane, wc, idx, s_sel);
 }
 
+// Per-head scores of already selected chunks (used after the tensor-core selection, which
+// keeps only the group score): one warp per (b, g, query), lane r handles idx[r].
+template <typename T, int GM>
+__global__ void __launch_bounds__(128) select_scores_kernel(Dims D, const T* __restrict__ qc,
+                                                            const T* __restrict__ klm,
+                                                            const float* __restrict__ blm,
+                                                            const int32_t* __restrict__ idx,
+                                                            float* __restrict__ s_sel) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t rows = D.B * D.Hkv * D.N_q;
+  const int64_t row = (int64_t)blockIdx.x * 4 + warp;
+  if (row >= rows) return;
+  const int64_t i = row % D.N_q, bg = row / D.N_q, g = bg % D.Hkv, b = bg / D.Hkv;
+  const int K = D.K, G = D.G, d = (int)D.d;
+  if (lane >= K) return;
+  const int c = idx[row * K + lane];
+  const bool valid = c >= 0 && c < D.C;
+  float acc[GM];
+#pragma unroll
+  for (int h = 0; h < GM; ++h) acc[h] = 0.f;
+  if (valid) {
+    const T* kr = klm + (bg * D.C + c) * d;
+    for (int k = 0; k < d; k += 4) {
+      float kv[4];
+      Elem<T>::load4(kr + k, kv);
+#pragma unroll
+      for (int h = 0; h < GM; ++h) {
+        if (h < G) {
+          float qv[4];
+          Elem<T>::load4(qc + (((b * D.Hq) + g * G + h) * D.N_q + i) * D.d + k, qv);
+          acc[h] = fmaf(qv[0], kv[0], acc[h]);
+          acc[h] = fmaf(qv[1], kv[1], acc[h]);
+          acc[h] = fmaf(qv[2], kv[2], acc[h]);
+          acc[h] = fmaf(qv[3], kv[3], acc[h]);
+        }
+      }
+    }
+  }
+  const float bc = valid ? blm[bg * D.C + c] : 0.f;
+#pragma unroll
+  for (int h = 0; h < GM; ++h) {
+    if (h < G) {
+      const int64_t hrow = ((b * D.Hq) + g * G + h) * D.N_q + i;
+      s_sel[hrow * K + lane] = valid ? fmaf(acc[h], D.scale, bc) : -INFINITY;
+    }
+  }
+}
+
+template <typename T>
+static cudaError_t launch_scores_g(const Dims& D, const void* qc, const void* klm,
+                                   const float* blm, const int32_t* idx, float* s_sel,
+                                   cudaStream_t st) {
+  const int64_t rows = D.B * D.Hkv * D.N_q;
+  const unsigned blocks = (unsigned)((rows + 3) / 4);
+#define HILS_SC(GM) select_scores_kernel<T, GM><<<blocks, 128, 0, st>>>(D, (const T*)qc, \
+                        (const T*)klm, blm, idx, s_sel)
+  if (D.G <= 1) HILS_SC(1);
+  else if (D.G <= 2) HILS_SC(2);
+  else if (D.G <= 4) HILS_SC(4);
+  else if (D.G <= 8) HILS_SC(8);
+  else HILS_SC(16);
+#undef HILS_SC
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_scores(const Dims& D, bool bf16, const void* qc, const void* klm,
+                                 const float* blm, const int32_t* idx, float* s_sel,
+                                 cudaStream_t st) {
+  if (D.B * D.Hkv * D.N_q == 0 || D.K == 0) return cudaSuccess;
+  return bf16 ? launch_scores_g<__nv_bfloat16>(D, qc, klm, blm, idx, s_sel, st)
+              : launch_scores_g<float>(D, qc, klm, blm, idx, s_sel, st);
+}
+
 // ---------------------------------------------------------------------------------------------
 // Decode layout.  Lanes are grouped L per landmark row; lane l of a group owns the row's
 // 16-byte vectors l, l+L, l+2L, ... so one warp instruction reads 32/L whole rows contiguously.
