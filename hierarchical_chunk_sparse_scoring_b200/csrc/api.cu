@@ -32,6 +32,7 @@ struct Plan {
   bool bf16 = false;
   bool decode = false;
   bool tc_select = false;
+  bool tc_attn = false;
   int cps = 0, n_split = 0, n_pieces = 0;
   size_t off_idx = 0, off_ssel = 0, off_pv = 0, off_pc = 0, off_po = 0, off_pl = 0;
   size_t total = 0;
@@ -68,6 +69,7 @@ Plan make_plan(const hils_params* p) {
   P.decode = p->N_q <= kDecodeMaxQueries && (p->d == 64 || p->d == 128) &&
              p->B * p->Hkv * p->N_q <= 65535;
   P.tc_select = !P.decode && score_tc_supported(D, P.bf16);
+  P.tc_attn = !P.decode && attn_tc_supported(D, P.bf16);
 
   const size_t sel_rows = (size_t)(p->B * p->Hkv * p->N_q);
   const size_t head_rows = (size_t)(p->B * p->Hq * p->N_q);
@@ -137,11 +139,16 @@ struct PhaseMarks {
 
 int phase_names(const Plan& P, const char** names, int max_names) {
   static const char* kDecode[] = {"select_split", "select_merge", "attn_units", "fuse_units"};
-  static const char* kPrefill[] = {"select_rows", "attn_rows"};
-  static const char* kPrefillTc[] = {"score_topk_tc", "select_scores", "attn_rows"};
-  const char** src = P.decode ? kDecode : (P.tc_select ? kPrefillTc : kPrefill);
-  const int n = P.decode ? 4 : (P.tc_select ? 3 : 2);
-  for (int i = 0; i < n && i < max_names; ++i) names[i] = src[i];
+  const char* pre[3];
+  int n = 0;
+  if (P.decode) {
+    for (int i = 0; i < 4 && i < max_names; ++i) names[i] = kDecode[i];
+    return 4;
+  }
+  if (P.tc_select) { pre[n++] = "score_topk_tc"; pre[n++] = "select_scores"; }
+  else pre[n++] = "select_rows";
+  pre[n++] = P.tc_attn ? "attn_tc" : "attn_rows";
+  for (int i = 0; i < n && i < max_names; ++i) names[i] = pre[i];
   return n;
 }
 
@@ -193,7 +200,10 @@ hils_status forward_impl(const hils_params* p, const void* q, const void* q_cal,
     }
     pm.mark();
     if (e == cudaSuccess)
-      e = launch_attn_rows(P.D, P.bf16, q, K, V, idx, s_sel, out, lse_out, nullptr, nullptr, st);
+      e = P.tc_attn ? launch_attn_tc(P.D, q, K, V, idx, s_sel, out, lse_out,
+                                     reinterpret_cast<int32_t*>(ws), st)
+                    : launch_attn_rows(P.D, P.bf16, q, K, V, idx, s_sel, out, lse_out, nullptr,
+                                       nullptr, st);
     pm.mark();
   }
   return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA;

@@ -1,0 +1,530 @@
+// Steps 3-4 for prefill on the tcgen05 tensor cores (bf16 inputs, fp32 accumulation, S = 64).
+//
+// [Reader] "Implementation and Training Recipes", Figure 4: pack M adjacent queries and the G
+// heads of their KV group into one tile of M*G rows and attend the union of the rows' chunks,
+// so one (M*G, d) x (d, S) product serves every row that uses the chunk.  Here M*G = 128 rows
+// (the tcgen05 tile height).  The union is taken over the queries' selected chunks plus the
+// chunks their local windows cover; for each (row, tile) the row either
+//   * selected this chunk: intra-chunk softmax with the chunk's own log-sum-exp, weighted by the
+//     row's surrogate score s_{h,c} ([Reader] Fig. 3 caption: inter-chunk softmax gives a
+//     chunk's mass, the intra-chunk softmax spreads it; [Abstract]: each query attends each
+//     retrieved chunk independently and the outputs are fused by the retrieval scores);
+//   * has the tile inside its causal local window: plain online softmax over those tokens
+//     (the window is one fusion unit scored by its exact log-sum-exp);
+//   * or does not use it: weight 0 (each row attends only its own chunks, so packing never
+//     changes a row's result).
+// Every weight is measured against one running reference m per row that starts at the row's
+// largest selected-chunk score, so chunk units never rescale the accumulator; window tiles
+// raise it only when a logit exceeds it by more than 8 (the O row in TMEM is then rescaled).
+//
+// CTA = (b, g, 128/G queries); 6 warps: warp 0 TMA (Q once, then K and V tiles of the union),
+// warp 1 TMEM owner and MMA issuer (S = Q K^T into a double-buffered TMEM tile, O += P V into a
+// TMEM accumulator), warps 2-5 one row per thread (classification, softmax, P to shared memory
+// in the 128-byte-swizzled K-major layout the P V product reads).
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace hils {
+using namespace sm100;
+
+namespace {
+
+constexpr int kAtThreads = 192;
+constexpr int kAtRows = 128;
+constexpr int kTile = 64;                    // tokens per tile (= chunk size S)
+constexpr uint32_t kAtPollLimit = 1u << 24;
+constexpr float kRescaleMargin = 8.0f;       // natural-log units
+constexpr int kAtSmemLimit = 227 * 1024;
+
+template <int DD, int G>
+struct AtShape {
+  static constexpr int TQ = kAtRows / G;                 // queries per CTA
+  static constexpr int KB = DD / 64;
+  static constexpr int Q_BOX = kAtRows * 128;            // [128 rows x 64] per 64-col box
+  static constexpr int Q_BYTES = KB * Q_BOX;
+  static constexpr int KV_BOX = kTile * 128;             // [64 tokens x 64]
+  static constexpr int KV_BYTES = KB * KV_BOX;           // one K (or V) tile
+  static constexpr int P_BYTES = kAtRows * 128;          // [128 rows x 64 tokens] bf16
+  static constexpr int STAGES = DD == 128 ? 3 : 4;
+  static constexpr int FIXED = Q_BYTES + STAGES * 2 * KV_BYTES + 2 * P_BYTES + 1024 /*bars*/ +
+                               1024 /*align*/ + 1024 /*scan*/;
+  static constexpr uint32_t TMEM_COLS = 256;            // S[2] (2 x 64) + O (DD)
+  static constexpr uint32_t O_COL = 128;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&t);
+}
+
+// Block-wide exclusive scan of one int per thread (blockDim.x <= 1024); returns the total.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) scratch[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < nw ? scratch[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < nw) scratch[32 + lane] = w;   // inclusive warp prefix
+  }
+  __syncthreads();
+  total = scratch[32 + nw - 1];
+  const int before = warp > 0 ? scratch[32 + warp - 1] : 0;
+  return before + x - v;
+}
+
+}  // namespace
+
+template <int DD, int G, int KM>
+__global__ void __launch_bounds__(kAtThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, Dims D,
+                   const int32_t* __restrict__ idx, const float* __restrict__ s_sel,
+                   __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out,
+                   int list_cap, int bitmap_words, int32_t* __restrict__ status) {
+  using SH = AtShape<DD, G>;
+  constexpr int TQ = SH::TQ;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + SH::Q_BYTES;
+  uint8_t* sV = sK + SH::STAGES * SH::KV_BYTES;
+  uint8_t* sP = sV + SH::STAGES * SH::KV_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * SH::P_BYTES);
+  uint64_t* kv_full = bars;                       // [STAGES]
+  uint64_t* kv_empty = bars + SH::STAGES;         // [STAGES]
+  uint64_t* q_full = bars + 2 * SH::STAGES;
+  uint64_t* s_full = q_full + 1;                  // [2]
+  uint64_t* s_empty = s_full + 2;                 // [2]
+  uint64_t* p_full = s_empty + 2;                 // [2]
+  uint64_t* p_empty = p_full + 2;                 // [2]
+  uint64_t* o_done = p_empty + 2;
+  uint64_t* o_final = o_done + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(o_final + 1);
+  int* scan = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + 1024);   // [64]
+  int* n_tiles_sh = scan + 64;
+  int* tiles = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + 2048);  // [list_cap]
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(tiles + list_cap);             // [words]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t bg = blockIdx.y;
+  const int64_t g = bg % D.Hkv, b = bg / D.Hkv;
+  const int64_t i0 = (int64_t)blockIdx.x * TQ;
+  const int64_t i_last = (i0 + TQ - 1 < D.N_q - 1) ? i0 + TQ - 1 : D.N_q - 1;
+  const int64_t p_first = D.q_pos0 + i0;
+  const int64_t p_max = D.q_pos0 + i_last;
+  const int64_t n_first = n_eligible(p_first, D.S, D.W);
+  const int64_t last_chunk = p_max / kTile;
+  const int K = D.K;
+
+  // ---------------------------------------------------------------- barriers, TMEM, tile list
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SH::STAGES; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
+    mbar_init(q_full, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&s_full[x], 1);
+      mbar_init(&s_empty[x], 4);
+      mbar_init(&p_full[x], 4);
+      mbar_init(&p_empty[x], 1);
+    }
+    mbar_init(o_done, 1);
+    mbar_init(o_final, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_holder, SH::TMEM_COLS);
+  const int nbw = (int)(last_chunk / 32) + 1;
+  for (int w = threadIdx.x; w < nbw; w += kAtThreads) bitmap[w] = 0u;
+  __syncthreads();
+  // selected chunks of every valid query of the tile, and the chunks of the local windows
+  for (int e = threadIdx.x; e < TQ * K; e += kAtThreads) {
+    const int qi = e / K, k = e - qi * K;
+    const int64_t i = i0 + qi;
+    if (i < D.N_q) {
+      const int c = idx[(bg * D.N_q + i) * K + k];
+      if (c >= 0 && c < D.C) atomicOr(&bitmap[c >> 5], 1u << (c & 31));
+    }
+  }
+  for (int64_t c = n_first + threadIdx.x; c <= last_chunk; c += kAtThreads)
+    atomicOr(&bitmap[c >> 5], 1u << (c & 31));
+  __syncthreads();
+  {
+    const int per = (nbw + kAtThreads - 1) / kAtThreads;
+    const int w0 = threadIdx.x * per;
+    const int w1 = w0 + per < nbw ? w0 + per : nbw;
+    int cnt = 0;
+    for (int w = w0; w < w1; ++w) cnt += __popc(bitmap[w]);
+    int total;
+    int pos = block_exclusive_scan(cnt, scan, total);
+    for (int w = w0; w < w1; ++w) {
+      uint32_t bits = bitmap[w];
+      while (bits) {
+        const int bit = __ffs(bits) - 1;
+        bits &= bits - 1;
+        if (pos < list_cap) tiles[pos] = w * 32 + bit;
+        ++pos;
+      }
+    }
+    if (threadIdx.x == 0) {
+      if (total > list_cap) record_status(status, kStatusDeviceCheck);
+      *n_tiles_sh = total < list_cap ? total : list_cap;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int n_tiles = *n_tiles_sh;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmQ);
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      mbar_expect_tx(q_full, SH::Q_BYTES);
+      for (int h = 0; h < G; ++h)
+        for (int kb = 0; kb < SH::KB; ++kb)
+          tma_load_2d(sQ + kb * SH::Q_BOX + h * TQ * 128, &tmQ, kb * 64,
+                      (int32_t)((b * D.Hq + g * G + h) * D.N_q + i0), q_full);
+      int last_s = -1;
+      uint32_t last_par = 0;
+      for (int t = 0; t < n_tiles; ++t) {
+        const int s = t % SH::STAGES;
+        const uint32_t u = (uint32_t)(t / SH::STAGES);
+        if (!mbar_wait(&kv_empty[s], (u & 1u) ^ 1u, kAtPollLimit)) {
+          record_status(status, kStatusTimeout);
+          break;
+        }
+        mbar_expect_tx(&kv_full[s], 2 * SH::KV_BYTES);
+        const int32_t y = (int32_t)(bg * D.N_kv + (int64_t)tiles[t] * kTile);
+        for (int kb = 0; kb < SH::KB; ++kb) {
+          tma_load_2d(sK + s * SH::KV_BYTES + kb * SH::KV_BOX, &tmK, kb * 64, y, &kv_full[s]);
+          tma_load_2d(sV + s * SH::KV_BYTES + kb * SH::KV_BOX, &tmV, kb * 64, y, &kv_full[s]);
+        }
+        last_s = s;
+        last_par = u & 1u;
+      }
+      if (last_s >= 0) mbar_wait(&kv_full[last_s], last_par, kAtPollLimit);
+      mbar_wait(q_full, 0, kAtPollLimit);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_QK = idesc_bf16_f32(kAtRows, kTile);
+      constexpr uint32_t IDESC_PV = idesc_bf16_f32(kAtRows, DD) | (1u << 16);   // V is MN-major
+      bool ok = mbar_wait(q_full, 0, kAtPollLimit);
+      tc_fence_after();
+      auto issue_qk = [&](int t) -> bool {
+        const int s = t % SH::STAGES, x = t & 1;
+        const uint32_t u = (uint32_t)(t / SH::STAGES), v = (uint32_t)(t >> 1);
+        if (!mbar_wait(&kv_full[s], u & 1u, kAtPollLimit)) return false;
+        if (!mbar_wait(&s_empty[x], (v & 1u) ^ 1u, kAtPollLimit)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < DD / 16; ++ks) {
+          const int kb = ks >> 2, kin = ks & 3;
+          const uint64_t ad = desc_kmajor_sw128(smem_u32(sQ + kb * SH::Q_BOX) + kin * 32);
+          const uint64_t bd =
+              desc_kmajor_sw128(smem_u32(sK + s * SH::KV_BYTES + kb * SH::KV_BOX) + kin * 32);
+          mma_bf16_ss(tmem + (uint32_t)(x * kTile), ad, bd, IDESC_QK, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(&s_full[x]);
+        return true;
+      };
+      if (ok && n_tiles > 0) ok = issue_qk(0);
+      if (ok && n_tiles > 1) ok = issue_qk(1);
+      for (int t = 0; ok && t < n_tiles; ++t) {
+        const int s = t % SH::STAGES, x = t & 1;
+        const uint32_t v = (uint32_t)(t >> 1);
+        if (!mbar_wait(&p_full[x], v & 1u, kAtPollLimit)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < kTile / 16; ++ks) {
+          const uint64_t ad = desc_kmajor_sw128(smem_u32(sP + x * SH::P_BYTES) + ks * 32);
+          const uint64_t bd = desc_mnmajor_sw128(
+              smem_u32(sV + s * SH::KV_BYTES) + ks * 16 * 128, SH::KV_BOX);
+          mma_bf16_ss(tmem + SH::O_COL, ad, bd, IDESC_PV, (t > 0 || ks > 0) ? 1u : 0u);
+        }
+        mma_commit(&kv_empty[s]);
+        mma_commit(&p_empty[x]);
+        mma_commit(o_done);
+        if (t == n_tiles - 1) mma_commit(o_final);
+        if (t + 2 < n_tiles) ok = issue_qk(t + 2);
+      }
+      if (!ok) record_status(status, kStatusTimeout);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax rows
+    const int qd = warp & 3;
+    const int r = qd * 32 + lane;
+    const int h = r / TQ, qi = r - h * TQ;
+    const int64_t i = i0 + qi;
+    const bool valid = i < D.N_q;
+    const int64_t pos = D.q_pos0 + (valid ? i : i_last);
+    const int64_t n_i = n_eligible(pos, D.S, D.W);
+    const int64_t hrow = (b * D.Hq + g * G + h) * D.N_q + i;
+    int sc[KM];
+    float su[KM];
+    float m_run = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < KM; ++k) {
+      sc[k] = -1;
+      su[k] = -INFINITY;
+      if (valid && k < K) {
+        sc[k] = idx[(bg * D.N_q + i) * K + k];
+        su[k] = sc[k] >= 0 ? s_sel[hrow * K + k] : -INFINITY;
+        m_run = fmaxf(m_run, su[k]);
+      }
+    }
+    float l = 0.f;
+    const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
+    uint8_t* prow_base = sP + (r >> 3) * 1024 + (r & 7) * 128;
+    bool ok = true;
+    for (int t = 0; t < n_tiles; ++t) {
+      const int x = t & 1;
+      const uint32_t v = (uint32_t)(t >> 1);
+      if (!mbar_wait_warp(&s_full[x], v & 1u, kAtPollLimit)) { ok = false; break; }
+      tc_fence_after();
+      float p[kTile];
+#pragma unroll
+      for (int j = 0; j < kTile / 16; ++j) {
+        float tmp[16];
+        tmem_ld16(lane_base + (uint32_t)(x * kTile + 16 * j), tmp);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) p[16 * j + e] = tmp[e];
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[x]);
+
+      const int c = tiles[t];
+      float u = -INFINITY;
+      bool is_sel = false;
+#pragma unroll
+      for (int k = 0; k < KM; ++k)
+        if (sc[k] == c) { is_sel = true; u = su[k]; }
+      const int64_t t0 = (int64_t)c * kTile;
+      const bool is_win = valid && !is_sel && c >= n_i && t0 <= pos;
+      bool rescale = false;
+      float factor = 1.f;
+      if (is_sel && u != -INFINITY) {
+        // intra-chunk softmax of this chunk, weighted by exp(u - m_run) (u <= m_run)
+        float mx = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < kTile; ++j) { p[j] *= D.scale; mx = fmaxf(mx, p[j]); }
+        float sum = 0.f;
+#pragma unroll
+        for (int j = 0; j < kTile; ++j) { p[j] = __expf(p[j] - mx); sum += p[j]; }
+        const float w = __expf(u - m_run);
+        const float f = w / sum;
+#pragma unroll
+        for (int j = 0; j < kTile; ++j) p[j] *= f;
+        l += w;
+      } else if (is_win) {
+        float mt = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < kTile; ++j) {
+          p[j] = (t0 + j <= pos) ? p[j] * D.scale : -INFINITY;
+          mt = fmaxf(mt, p[j]);
+        }
+        if (mt > m_run + kRescaleMargin) {
+          if (l > 0.f) {
+            factor = __expf(m_run - mt);
+            l *= factor;
+            rescale = true;
+          }
+          m_run = mt;
+        }
+        float sum = 0.f;
+#pragma unroll
+        for (int j = 0; j < kTile; ++j) {
+          p[j] = p[j] == -INFINITY ? 0.f : __expf(p[j] - m_run);
+          sum += p[j];
+        }
+        l += sum;
+      } else {
+#pragma unroll
+        for (int j = 0; j < kTile; ++j) p[j] = 0.f;
+      }
+      // the P buffer is free once the P V product of tile t-2 has completed
+      if (!mbar_wait_warp(&p_empty[x], (v & 1u) ^ 1u, kAtPollLimit)) { ok = false; break; }
+      if (__any_sync(0xffffffffu, rescale)) {
+        // O row *= factor, after the P V product of tile t-1 has landed
+        if (!mbar_wait_warp(o_done, (uint32_t)((t - 1) & 1), kAtPollLimit)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int j = 0; j < DD / 16; ++j) {
+          float o[16];
+          tmem_ld16(lane_base + SH::O_COL + 16 * j, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] *= factor;
+          tmem_st16(lane_base + SH::O_COL + 16 * j, o);
+        }
+        tmem_wait_st();
+      }
+      uint8_t* prow = prow_base + x * SH::P_BYTES;
+#pragma unroll
+      for (int k8 = 0; k8 < kTile / 8; ++k8) {
+        uint4 w4;
+        w4.x = pack_bf16(p[8 * k8 + 0], p[8 * k8 + 1]);
+        w4.y = pack_bf16(p[8 * k8 + 2], p[8 * k8 + 3]);
+        w4.z = pack_bf16(p[8 * k8 + 4], p[8 * k8 + 5]);
+        w4.w = pack_bf16(p[8 * k8 + 6], p[8 * k8 + 7]);
+        *reinterpret_cast<uint4*>(prow + ((k8 ^ (r & 7)) << 4)) = w4;
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[x]);
+    }
+    // ---------------------------------------------------------------- output rows
+    const bool fin = __all_sync(0xffffffffu, ok) && n_tiles > 0 &&
+                     mbar_wait_warp(o_final, 0, kAtPollLimit);
+    if (fin) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* orow = out + hrow * DD;
+#pragma unroll
+      for (int j = 0; j < DD / 16; ++j) {
+        float o[16];
+        tmem_ld16(lane_base + SH::O_COL + 16 * j, o);
+        tmem_wait_ld();
+        if (valid) {
+          uint4 a, c4;
+          a.x = pack_bf16(o[0] * inv, o[1] * inv);
+          a.y = pack_bf16(o[2] * inv, o[3] * inv);
+          a.z = pack_bf16(o[4] * inv, o[5] * inv);
+          a.w = pack_bf16(o[6] * inv, o[7] * inv);
+          c4.x = pack_bf16(o[8] * inv, o[9] * inv);
+          c4.y = pack_bf16(o[10] * inv, o[11] * inv);
+          c4.z = pack_bf16(o[12] * inv, o[13] * inv);
+          c4.w = pack_bf16(o[14] * inv, o[15] * inv);
+          *reinterpret_cast<uint4*>(orow + 16 * j) = a;
+          *reinterpret_cast<uint4*>(orow + 16 * j + 8) = c4;
+        }
+      }
+      if (valid && lse_out) lse_out[hrow] = m_run + __logf(l);
+    } else if (!ok || n_tiles > 0) {
+      record_status(status, kStatusTimeout);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, SH::TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------------------------
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_at() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+bool make_map_at(CUtensorMap* map, const void* base, uint64_t rows, uint64_t d, uint32_t box_rows) {
+  auto enc = get_encode_at();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {d, rows};
+  cuuint64_t strides[1] = {d * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int list_capacity(const Dims& D, int TQ) {
+  // union of TQ queries' selections plus the chunks their windows cover
+  return TQ * D.K + (int)((D.W + kTile + TQ) / kTile) + 4;
+}
+
+template <int DD, int G, int KM>
+cudaError_t launch_at_t(const Dims& D, const void* q, const void* K, const void* V,
+                        const int32_t* idx, const float* s_sel, void* out, float* lse,
+                        int32_t* status, cudaStream_t st) {
+  using SH = AtShape<DD, G>;
+  CUtensorMap tmQ, tmK, tmV;
+  if (!make_map_at(&tmQ, q, (uint64_t)(D.B * D.Hq * D.N_q), DD, SH::TQ) ||
+      !make_map_at(&tmK, K, (uint64_t)(D.B * D.Hkv * D.N_kv), DD, kTile) ||
+      !make_map_at(&tmV, V, (uint64_t)(D.B * D.Hkv * D.N_kv), DD, kTile))
+    return cudaErrorInvalidValue;
+  const int cap = list_capacity(D, SH::TQ);
+  const int words = (int)((D.N_kv / kTile) / 32) + 2;
+  const int smem = SH::FIXED + 1024 + cap * 4 + words * 4;
+  if (smem > kAtSmemLimit) return cudaErrorInvalidConfiguration;
+  auto kern = attn_tc_kernel<DD, G, KM>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((D.N_q + SH::TQ - 1) / SH::TQ), (unsigned)(D.B * D.Hkv));
+  kern<<<grid, kAtThreads, smem, st>>>(tmQ, tmK, tmV, D, idx, s_sel, (__nv_bfloat16*)out, lse,
+                                       cap, words, status);
+  return cudaGetLastError();
+}
+
+template <int DD, int G>
+cudaError_t launch_at_k(const Dims& D, const void* q, const void* K, const void* V,
+                        const int32_t* idx, const float* s_sel, void* out, float* lse,
+                        int32_t* status, cudaStream_t st) {
+  if (D.K <= 16) return launch_at_t<DD, G, 16>(D, q, K, V, idx, s_sel, out, lse, status, st);
+  return launch_at_t<DD, G, 32>(D, q, K, V, idx, s_sel, out, lse, status, st);
+}
+
+}  // namespace
+
+bool attn_tc_supported(const Dims& D, bool bf16) {
+  if (!bf16 || D.S != kTile || D.K > kMaxK) return false;
+  if (D.d != 64 && D.d != 128) return false;
+  if (D.G != 1 && D.G != 2 && D.G != 4 && D.G != 8) return false;
+  if (D.B * D.Hkv > 65535) return false;
+  const int TQ = kAtRows / D.G;
+  const int64_t cap = (int64_t)TQ * D.K + (D.W + kTile + TQ) / kTile + 4;
+  const int64_t words = (D.N_kv / kTile) / 32 + 2;
+  const int fixed = D.d == 128 ? AtShape<128, 1>::FIXED : AtShape<64, 1>::FIXED;
+  return fixed + 1024 + (cap + words) * 4 <= kAtSmemLimit;
+}
+
+cudaError_t launch_attn_tc(const Dims& D, const void* q, const void* K, const void* V,
+                           const int32_t* idx, const float* s_sel, void* out, float* lse,
+                           int32_t* status, cudaStream_t st) {
+  if (D.B * D.Hq * D.N_q == 0) return cudaSuccess;
+#define HILS_AT(DD, GG) return launch_at_k<DD, GG>(D, q, K, V, idx, s_sel, out, lse, status, st)
+  if (D.d == 128) {
+    if (D.G == 1) HILS_AT(128, 1);
+    if (D.G == 2) HILS_AT(128, 2);
+    if (D.G == 4) HILS_AT(128, 4);
+    HILS_AT(128, 8);
+  }
+  if (D.G == 1) HILS_AT(64, 1);
+  if (D.G == 2) HILS_AT(64, 2);
+  if (D.G == 4) HILS_AT(64, 4);
+  HILS_AT(64, 8);
+#undef HILS_AT
+}
+
+}  // namespace hils

@@ -99,25 +99,17 @@ struct TopList {
     for (int k = 0; k < KM; ++k) { v[k] = -INFINITY; c[k] = INT_MAX; }
   }
 
-  // Inserts (x, ci) if it beats slot K-1; keeps the list ordered by `better`.
+  // Inserts (x, ci) if it beats slot K-1; keeps the list ordered by `better`.  The new entry
+  // walks down the list swapping with every slot it beats (static indexing only, so the list
+  // stays in registers); the displaced last entry falls off.
   __device__ __forceinline__ void insert(float x, int ci, int K) {
-    if (K <= 0) return;
-    float lv = -INFINITY;
-    int lc = INT_MAX;
 #pragma unroll
-    for (int k = 0; k < KM; ++k)
-      if (k == K - 1) { lv = v[k]; lc = c[k]; }
-    if (!better(x, ci, lv, lc)) return;
-#pragma unroll
-    for (int k = KM - 1; k > 0; --k) {
-      if (k < K) {
-        bool above = better(x, ci, v[k - 1], c[k - 1]);
-        bool here = better(x, ci, v[k], c[k]);
-        if (above) { v[k] = v[k - 1]; c[k] = c[k - 1]; }
-        else if (here) { v[k] = x; c[k] = ci; }
-      }
+    for (int k = 0; k < KM; ++k) {
+      const bool sw = (k < K) && better(x, ci, v[k], c[k]);
+      const float tv = v[k];
+      const int tc = c[k];
+      if (sw) { v[k] = x; c[k] = ci; x = tv; ci = tc; }
     }
-    if (better(x, ci, v[0], c[0])) { v[0] = x; c[0] = ci; }
   }
 
   __device__ __forceinline__ void pop_front() {

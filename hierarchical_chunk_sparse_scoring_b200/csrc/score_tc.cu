@@ -197,39 +197,49 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int t = 0; t < n_tiles; ++t) {
       const int a = t & 1;
       const uint32_t v = (uint32_t)(t >> 1);
-      if (!mbar_wait(&acc_full[a], v & 1u, kPollLimit)) { ok = false; break; }
+      if (!mbar_wait_warp(&acc_full[a], v & 1u, kPollLimit)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll 1
       for (int sb = 0; sb < SH::HALF / 16; ++sb) {
         const int col0 = ch * SH::HALF + sb * 16;
+        const int64_t c0 = (int64_t)t * NT + col0;
+        // landmark biases of these 16 chunks: one load per lane, then broadcast
+        const int64_t cb = c0 + (lane & 15);
+        const float bl = cb < n_max ? __ldg(bb + cb) : 0.f;
         float sig[16];
-        tmem_ld16(lane_base + (uint32_t)(a * G * NT + col0), sig);
+        constexpr int HG = G < 4 ? G : 4;     // heads whose TMEM loads are in flight together
 #pragma unroll
-        for (int h = 1; h < G; ++h) {
-          float tmp[16];
-          tmem_ld16(lane_base + (uint32_t)((a * G + h) * NT + col0), tmp);
+        for (int h0 = 0; h0 < G; h0 += HG) {
+          float tmp[HG][16];
+#pragma unroll
+          for (int hh = 0; hh < HG; ++hh)
+            tmem_ld16(lane_base + (uint32_t)((a * G + h0 + hh) * NT + col0), tmp[hh]);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) sig[j] = fmaxf(sig[j], tmp[j]);
+          for (int hh = 0; hh < HG; ++hh)
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              sig[j] = (h0 + hh == 0) ? tmp[hh][j] : fmaxf(sig[j], tmp[hh][j]);
         }
-        tmem_wait_ld();
-        const int64_t c0 = (int64_t)t * NT + col0;
         uint32_t pass = 0;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int64_t c = c0 + j;
-          float s = -INFINITY;
-          if (c < n_max) s = fmaf(sig[j], D.scale, __ldg(bb + c));
-          if (c < n_i && better(s, (int)c, thv, thc)) pass |= 1u << j;
-          st[j * 256] = s;
+          const float bj = __shfl_sync(0xffffffffu, bl, j);
+          sig[j] = fmaf(sig[j], D.scale, bj);
+          if (c < n_i && better(sig[j], (int)c, thv, thc)) pass |= 1u << j;
         }
-        if (pass) {
-          while (pass) {
-            const int j = __ffs(pass) - 1;
-            pass &= pass - 1;
-            L.insert(st[j * 256], (int)(c0 + j), K);
+        if (__any_sync(0xffffffffu, pass != 0)) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) st[j * 256] = sig[j];
+          if (pass) {
+            while (pass) {
+              const int j = __ffs(pass) - 1;
+              pass &= pass - 1;
+              L.insert(st[j * 256], (int)(c0 + j), K);
+            }
+            kth<KM>(L, K, thv, thc);
           }
-          kth<KM>(L, K, thv, thc);
         }
       }
       tc_fence_before();

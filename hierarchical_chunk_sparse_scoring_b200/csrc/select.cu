@@ -124,19 +124,28 @@ __global__ void __launch_bounds__(256) select_rows_kernel(Dims D, const T* __res
 }
 
 // Per-head scores of already selected chunks (used after the tensor-core selection, which
-// keeps only the group score): one warp per (b, g, query), lane r handles idx[r].
+// keeps only the group score): one warp per (b, g, query); the group's calibrated queries are
+// staged in shared memory and lane r handles idx[r].
 template <typename T, int GM>
 __global__ void __launch_bounds__(128) select_scores_kernel(Dims D, const T* __restrict__ qc,
                                                             const T* __restrict__ klm,
                                                             const float* __restrict__ blm,
                                                             const int32_t* __restrict__ idx,
                                                             float* __restrict__ s_sel) {
+  __shared__ __align__(16) float qs[4][GM * kMaxD];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t rows = D.B * D.Hkv * D.N_q;
   const int64_t row = (int64_t)blockIdx.x * 4 + warp;
   if (row >= rows) return;
   const int64_t i = row % D.N_q, bg = row / D.N_q, g = bg % D.Hkv, b = bg / D.Hkv;
   const int K = D.K, G = D.G, d = (int)D.d;
+  for (int e = lane * 4; e < G * d; e += 128) {
+    const int h = e / d, k = e - h * d;
+    float v[4];
+    Elem<T>::load4(qc + (((b * D.Hq) + g * G + h) * D.N_q + i) * D.d + k, v);
+    Elem<float>::store4(&qs[warp][e], v);
+  }
+  __syncwarp();
   if (lane >= K) return;
   const int c = idx[row * K + lane];
   const bool valid = c >= 0 && c < D.C;
@@ -151,12 +160,11 @@ __global__ void __launch_bounds__(128) select_scores_kernel(Dims D, const T* __r
 #pragma unroll
       for (int h = 0; h < GM; ++h) {
         if (h < G) {
-          float qv[4];
-          Elem<T>::load4(qc + (((b * D.Hq) + g * G + h) * D.N_q + i) * D.d + k, qv);
-          acc[h] = fmaf(qv[0], kv[0], acc[h]);
-          acc[h] = fmaf(qv[1], kv[1], acc[h]);
-          acc[h] = fmaf(qv[2], kv[2], acc[h]);
-          acc[h] = fmaf(qv[3], kv[3], acc[h]);
+          const float4 qv = *reinterpret_cast<const float4*>(&qs[warp][h * d + k]);
+          acc[h] = fmaf(qv.x, kv[0], acc[h]);
+          acc[h] = fmaf(qv.y, kv[1], acc[h]);
+          acc[h] = fmaf(qv.z, kv[2], acc[h]);
+          acc[h] = fmaf(qv.w, kv[3], acc[h]);
         }
       }
     }
