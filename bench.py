@@ -282,7 +282,7 @@ def oracle_sample_rate(wl, seconds, rng_seed=0, max_rows=None):
 def primary_workload(args, device, rank):
     from hierarchical_chunk_sparse_scoring_b200 import workloads as W
     seed = W.SPECS[args.workload]["seed"] + 1000 * rank
-    return W.make(args.workload, device, seed=seed)
+    return W.make(args.workload, device, seed=seed, N=args.N, B=args.B)
 
 
 def config_of(wl, n_gpus):
@@ -461,7 +461,7 @@ def run_reference(args):
     if int(os.environ.get("RANK", "0")) != 0:
         return
     from hierarchical_chunk_sparse_scoring_b200 import workloads as W
-    wl = W.make(args.workload, "cpu")
+    wl = W.make(args.workload, "cpu", N=args.N, B=args.B)
     per_step = max(1.0, args.ref_step_seconds)
     rates, rows_total, threads = [], 0, 1
     for k in range(args.warmup + args.steps):
@@ -493,6 +493,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["hils", "reference"], default="hils")
     ap.add_argument("--workload", default="small_mha_bf16")
+    ap.add_argument("--N", type=int, default=None, help="override the workload's sequence length")
+    ap.add_argument("--B", type=int, default=None, help="override the workload's batch")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=6.0)
