@@ -43,6 +43,8 @@ SIGNATURES = {
                                           ctypes.c_size_t, _V, ctypes.POINTER(_V), ctypes.c_int]),
     "hils_forward_phases": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_char_p), ctypes.c_int]),
     "hils_select": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V, ctypes.c_size_t, _V]),
+    "hils_select_noalloc": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V]),
+    "hils_select_noalloc_max_bytes": (ctypes.c_size_t, []),
     "hils_chunk_attn": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V, _V]),
     "hils_fuse": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V]),
     "hils_workspace_init": (ctypes.c_int, [_V, ctypes.c_size_t, _V]),

@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "hils.h"
@@ -341,3 +342,82 @@ extern "C" const char* hils_status_string(hils_status s) {
 }
 
 extern "C" const char* hils_version(void) { return "hils-b200 " HILS_GIT_DESCRIBE " sm_100a"; }
+
+// ---------------------------------------------------------------------------------------------
+// Steps 1-2 with the library's own scratch memory, for callers that cannot hand the library a
+// workspace buffer.  The scratch (the status word and the decode path's per-split candidate
+// lists) lives in one file-scope device array of fixed size; every device that loads the
+// library holds its own copy until the process exits.
+namespace hils {
+namespace {
+
+constexpr size_t kStaticScratchBytes = 8u << 20;   // 8 MiB per device
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of this device's scratch array.  In host code `g_static_scratch` names a host
+// stand-in, not device memory, so the address is looked up once per device (with that device
+// current) and cached.
+hils_status static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HILS_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return HILS_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return HILS_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return HILS_OK;
+}
+
+}  // namespace
+}  // namespace hils
+
+extern "C" size_t hils_select_noalloc_max_bytes(void) { return hils::kStaticScratchBytes; }
+
+extern "C" hils_status hils_select_noalloc(const hils_params* p, const void* q_cal,
+                                           const void* k_lm, const float* b_lm, int32_t* idx,
+                                           float* s_sel, hils_stream_t stream) {
+  hils_status s = check_params(p);
+  if (s != HILS_OK) return s;
+  const Plan P = make_plan(p);
+  const bool any = p->B > 0 && p->N_q > 0;
+  const bool any_lm = any && P.D.C > 0;
+  if (!ok_ptr(q_cal, any) || !ok_ptr(k_lm, any_lm) || !ok_ptr(b_lm, any_lm) ||
+      !ok_ptr(idx, any && p->K_top > 0) || (s_sel && !aligned16(s_sel)))
+    return HILS_ERR_INVALID_ARG;
+  // scratch layout: [status word | decode split lists (values) | decode split lists (ids)]
+  const size_t sel_rows = (size_t)(p->B * p->Hkv * p->N_q);
+  const size_t list_bytes =
+      P.decode ? align_up(sel_rows * (size_t)P.n_split * (size_t)P.D.K * sizeof(float)) : 0;
+  const size_t need = kStatusBytes + 2 * list_bytes;
+  if (need > kStaticScratchBytes) return HILS_ERR_WORKSPACE;
+  if (!any) return HILS_OK;
+  if ((s = check_device()) != HILS_OK) return s;
+  void* scratch = nullptr;
+  if ((s = static_scratch(&scratch)) != HILS_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(scratch);
+  // the status word is shared by every call: start it at zero
+  if (cudaMemsetAsync(ws, 0, kStatusBytes, st) != cudaSuccess) return HILS_ERR_CUDA;
+  cudaError_t e;
+  if (P.decode) {
+    float* pv = reinterpret_cast<float*>(ws + kStatusBytes);
+    int32_t* pc = reinterpret_cast<int32_t*>(ws + kStatusBytes + list_bytes);
+    e = launch_select_split(P.D, P.bf16, P.cps, P.n_split, q_cal, k_lm, b_lm, pv, pc, st);
+    if (e == cudaSuccess)
+      e = launch_select_merge(P.D, P.bf16, P.n_split, pv, pc, q_cal, k_lm, b_lm, idx, s_sel, st);
+  } else if (P.tc_select) {
+    e = launch_score_topk_tc(P.D, q_cal, k_lm, b_lm, idx, reinterpret_cast<int32_t*>(ws), st);
+    if (e == cudaSuccess && s_sel)
+      e = launch_select_scores(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
+  } else {
+    e = launch_select_rows(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
+  }
+  return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA;
+}

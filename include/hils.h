@@ -136,6 +136,30 @@ hils_status hils_chunk_attn(const hils_params* p, const void* q, const void* K, 
 hils_status hils_fuse(const hils_params* p, const float* s_sel, const float* unit_o,
                       const float* unit_lse, void* out, float* lse_out, hils_stream_t stream);
 
+/*
+ * hils_select without a caller-provided workspace.  The paper has no counterpart: this entry
+ * point exists for callers that cannot allocate device memory or pass a scratch buffer, e.g. a
+ * plugin host that hands a kernel only its input and output tensors, or a serving loop whose
+ * device memory is planned up front so that cudaMalloc (which may synchronise the device) is
+ * not allowed on the request path.  It computes exactly what hils_select computes.
+ *
+ * Scratch: a fixed array of hils_select_noalloc_max_bytes() bytes (8 MiB) inside the library,
+ * one per device, held by every device that loads the library until the process exits.  The
+ * first call on a device looks up that device's copy (cudaGetSymbolAddress, with the device
+ * current); make that first call before any stream capture.  Calls whose scratch would exceed
+ * the maximum (decode shapes with B*Hkv*N_q * ceil(n/512) * K * 8 bytes beyond ~8 MiB) return
+ * HILS_ERR_WORKSPACE before launching anything.  Every call on a device shares the same
+ * scratch, so calls that overlap on the GPU (different streams, or concurrent host threads)
+ * race and give undefined results: order them on one stream.  The library's status word is
+ * cleared at the start of every call.  Allocates nothing.
+ */
+hils_status hils_select_noalloc(const hils_params* p, const void* q_cal, const void* k_lm,
+                                const float* b_lm, int32_t* idx, float* s_sel,
+                                hils_stream_t stream);
+
+/* Size in bytes of the fixed scratch array hils_select_noalloc uses. */
+size_t hils_select_noalloc_max_bytes(void);
+
 /* Zeroes the workspace's status word; call once on a newly allocated workspace. */
 hils_status hils_workspace_init(void* workspace, size_t workspace_bytes, hils_stream_t stream);
 
