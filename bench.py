@@ -86,7 +86,7 @@ def phase_work(name, wm):
     """(bound, algorithmic work, unit) of a kernel, for its roofline."""
     if name in ("score_topk_tc", "select_rows"):
         return "tensor", wm["score_flops"], "TFLOP/s"
-    if name == "select_split":
+    if name in ("select_split", "select_stream"):
         return "hbm", wm["select_bytes"], "GB/s"
     if name == "attn_units":
         return "hbm", wm["attn_bytes"], "GB/s"

@@ -23,6 +23,7 @@ constexpr size_t kAlign = 256;
 constexpr size_t kStatusBytes = 256;
 constexpr int kChunksPerSplit = 512;
 constexpr int64_t kDecodeMaxQueries = 16;
+constexpr int kStreamRows = 128;   // landmark rows per streaming CTA (one bulk copy)
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -36,6 +37,8 @@ struct Plan {
   bool tc_attn = false;
   int cps = 0, n_split = 0, n_pieces = 0;
   size_t off_idx = 0, off_ssel = 0, off_pv = 0, off_pc = 0, off_po = 0, off_pl = 0;
+  size_t off_sig = 0;
+  int64_t n_stride = 0;
   size_t total = 0;
 };
 
@@ -95,9 +98,17 @@ Plan make_plan(const hils_params* p) {
     P.off_pc = off; off = align_up(off + sel_rows * P.n_split * (size_t)D.K * sizeof(int32_t));
     P.off_po = off; off = align_up(off + head_rows * NU * (size_t)D.d * sizeof(float));
     P.off_pl = off; off = align_up(off + head_rows * NU * sizeof(float));
+    P.n_stride = (n_max + 3) / 4 * 4;
+    P.off_sig = off; off = align_up(off + sel_rows * (size_t)P.n_stride * sizeof(float));
   }
   P.total = off;
   return P;
+}
+
+int n_stream_split(const Plan& P) {
+  const int64_t n_max = P.n_stride;
+  const int64_t s = (n_max + kStreamRows - 1) / kStreamRows;
+  return (int)(s < 1 ? 1 : s);
 }
 
 hils_status check_device() {
@@ -139,7 +150,7 @@ struct PhaseMarks {
 };
 
 int phase_names(const Plan& P, const char** names, int max_names) {
-  static const char* kDecode[] = {"select_split", "select_merge", "attn_units", "fuse_units"};
+  static const char* kDecode[] = {"select_stream", "select_topk", "attn_units", "fuse_units"};
   const char* pre[3];
   int n = 0;
   if (P.decode) {
@@ -182,12 +193,17 @@ hils_status forward_impl(const hils_params* p, const void* q, const void* q_cal,
     int32_t* pc = reinterpret_cast<int32_t*>(ws + P.off_pc);
     float* po = reinterpret_cast<float*>(ws + P.off_po);
     float* pl = reinterpret_cast<float*>(ws + P.off_pl);
-    e = launch_select_split(P.D, P.bf16, P.cps, P.n_split, q_cal, k_lm, b_lm, pv, pc, st);
+    float* sig = reinterpret_cast<float*>(ws + P.off_sig);
+    (void)pv;
+    (void)pc;
+    e = launch_select_stream(P.D, P.bf16, kStreamRows, n_stream_split(P), P.n_stride, q_cal, k_lm,
+                             b_lm, sig, reinterpret_cast<int32_t*>(ws), st);
     pm.mark();
     if (e == cudaSuccess)
-      e = launch_select_merge(P.D, P.bf16, P.n_split, pv, pc, q_cal, k_lm, b_lm, idx, s_sel, st);
+      e = launch_select_topk(P.D, P.bf16, P.n_stride, sig, q_cal, k_lm, b_lm, idx, s_sel, st);
     pm.mark();
-    if (e == cudaSuccess) e = launch_attn_units(P.D, P.bf16, P.n_pieces, q, K, V, idx, po, pl, st);
+    if (e == cudaSuccess) e = launch_attn_units(P.D, P.bf16, P.n_pieces, q, K, V, idx, po, pl,
+                                                  reinterpret_cast<int32_t*>(ws), st);
     pm.mark();
     if (e == cudaSuccess) e = launch_fuse_units(P.D, P.bf16, P.n_pieces, s_sel, po, pl, out, lse_out, st);
     pm.mark();
@@ -256,11 +272,11 @@ extern "C" hils_status hils_select(const hils_params* p, const void* q_cal, cons
   char* ws = static_cast<char*>(workspace);
   cudaError_t e;
   if (P.decode) {
-    float* pv = reinterpret_cast<float*>(ws + P.off_pv);
-    int32_t* pc = reinterpret_cast<int32_t*>(ws + P.off_pc);
-    e = launch_select_split(P.D, P.bf16, P.cps, P.n_split, q_cal, k_lm, b_lm, pv, pc, st);
+    float* sig = reinterpret_cast<float*>(ws + P.off_sig);
+    e = launch_select_stream(P.D, P.bf16, kStreamRows, n_stream_split(P), P.n_stride, q_cal, k_lm,
+                             b_lm, sig, reinterpret_cast<int32_t*>(ws), st);
     if (e == cudaSuccess)
-      e = launch_select_merge(P.D, P.bf16, P.n_split, pv, pc, q_cal, k_lm, b_lm, idx, s_sel, st);
+      e = launch_select_topk(P.D, P.bf16, P.n_stride, sig, q_cal, k_lm, b_lm, idx, s_sel, st);
   } else if (P.tc_select) {
     e = launch_score_topk_tc(P.D, q_cal, k_lm, b_lm, idx, reinterpret_cast<int32_t*>(ws), st);
     if (e == cudaSuccess && s_sel)

@@ -15,6 +15,7 @@
 //   fuse_units_kernel  one warp per (b, h, query): combines chunk units and window pieces.
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace hils {
 
@@ -134,29 +135,47 @@ __global__ void __launch_bounds__(128) attn_rows_kernel(Dims D, const T* __restr
 }
 
 // ---------------------------------------------------------------------------------------------
+// Decode units.  One CTA per (b, g, query, unit) serves all G heads of the group, so each K/V row
+// of the unit is read from memory once.  Per tile of up to 64 tokens the K and V rows (contiguous
+// in memory) arrive by two bulk copies into shared memory; then L lanes share a token row, lane
+// l holding d/L of its dimensions (the grouping of the decode selection): pass 1 computes the
+// G x 64 logits, the tile's softmax statistics update the running (m, l) per head, pass 2
+// accumulates p * V into per-lane partial outputs, reduced across lane groups and warps at the
+// end.
 constexpr int kUnitThreads = 128;
-constexpr int kUnitTile = 32;   // tokens per smem tile
+constexpr int kUnitWarps = kUnitThreads / 32;
+constexpr int kUnitTile = 64;   // tokens per tile
 
-template <typename T>
+// Lane grouping of the unit kernel: 8 dims per lane (4 for 16 heads), so that both the group's
+// query slice and its output accumulators stay in registers.
+template <typename T, int D_, int GM>
+struct UnitShape {
+  static constexpr int DPL = GM <= 8 ? 8 : 4;
+  static constexpr int L = D_ / DPL;
+  static constexpr int VEC = (16 / (int)sizeof(T)) < DPL ? (16 / (int)sizeof(T)) : DPL;
+  static constexpr int NV = DPL / VEC;
+  static constexpr int RPW = 32 / L;
+  static_assert(L >= 1 && L <= 32 && (32 % L) == 0, "lane grouping");
+};
+
+template <typename T, int D_, int GM>
 __global__ void __launch_bounds__(kUnitThreads) attn_units_kernel(
     Dims D, int n_pieces, const T* __restrict__ q, const T* __restrict__ Kc,
     const T* __restrict__ Vc, const int32_t* __restrict__ idx, float* __restrict__ part_o,
-    float* __restrict__ part_lse) {
-  extern __shared__ __align__(16) float sm[];
-  const int d = (int)D.d, G = D.G, K = D.K;
-  const int dp = d + 4;                                  // padded row (floats)
-  float* qf = sm;                                        // [G][d]
-  float* Ks = qf + G * d;                                // [tile][dp]
-  float* Vs = Ks + kUnitTile * dp;                       // [tile][dp]
-  float* xs = Vs + kUnitTile * dp;                       // [G][tile]
-  float* mst = xs + G * kUnitTile;                       // [G] running max
-  float* lst = mst + G;                                  // [G] running sum
-  float* cst = lst + G;                                  // [G] rescale of this tile
-
+    float* __restrict__ part_lse, int32_t* __restrict__ status) {
+  using SS = UnitShape<T, D_, GM>;
+  extern __shared__ __align__(128) uint8_t sm_units[];
+  T* Ks = reinterpret_cast<T*>(sm_units);                       // [64][D_]
+  T* Vs = Ks + kUnitTile * D_;                                   // [64][D_]
+  float* red = reinterpret_cast<float*>(Vs + kUnitTile * D_);    // [warps][GM*D_/4]
+  __shared__ float xs[GM][kUnitTile];
+  __shared__ float mst[GM], lst[GM], cst[GM];
+  __shared__ uint64_t full;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int unit = blockIdx.x;
   const int64_t row = blockIdx.y;                        // (b, g, i)
   const int64_t i = row % D.N_q, bg = row / D.N_q, g = bg % D.Hkv, b = bg / D.Hkv;
+  const int G = D.G, K = D.K;
   const int NU = K + n_pieces;
   const int64_t pos = D.q_pos0 + i;
   const int64_t n = n_eligible(pos, D.S, D.W);
@@ -170,99 +189,176 @@ __global__ void __launch_bounds__(kUnitThreads) attn_units_kernel(
     t1 = t0 + D.S < pos + 1 ? t0 + D.S : pos + 1;
     if (t1 < t0) t1 = t0;
   }
-  const int64_t hrow0 = (b * D.Hq + g * G) * D.N_q + i;   // head g*G, stride N_q per head
-
-  for (int e = tid; e < G * d; e += kUnitThreads) {
-    const int hh = e / d, k = e - hh * d;
-    qf[e] = Elem<T>::to_f(q[(hrow0 + (int64_t)hh * D.N_q) * d + k]);
+  const int64_t hrow0 = (b * D.Hq + g * G) * D.N_q + i;   // head g*G; stride N_q per head
+  if (tid == 0) {
+    sm100::mbar_init(&full, 1);
+    sm100::fence_barrier_init();
   }
-  if (tid < G) { mst[tid] = -INFINITY; lst[tid] = 0.f; }
-  const T* Kb = Kc + bg * D.N_kv * d;
-  const T* Vb = Vc + bg * D.N_kv * d;
-
-  // this thread's (head, dim) outputs: pairs tid, tid + 128, ...
-  constexpr int kMaxPairs = 16 * kMaxD / kUnitThreads;
-  float acc[kMaxPairs];
+  if (tid < GM) { mst[tid] = -INFINITY; lst[tid] = 0.f; cst[tid] = 1.f; }
+  __syncthreads();
+  const int grp = lane / SS::L, gl = lane % SS::L;
+  float qreg[GM][SS::DPL];
 #pragma unroll
-  for (int r = 0; r < kMaxPairs; ++r) acc[r] = 0.f;
-  const int n_pairs = G * d;
+  for (int h = 0; h < GM; ++h) {
+#pragma unroll
+    for (int v = 0; v < SS::NV; ++v) {
+      float t[SS::VEC];
+      if (h < G) {
+        load_vec<T, SS::VEC>(q + (hrow0 + (int64_t)h * D.N_q) * D_ + (v * SS::L + gl) * SS::VEC, t);
+      } else {
+#pragma unroll
+        for (int e = 0; e < SS::VEC; ++e) t[e] = 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < SS::VEC; ++e) qreg[h][v * SS::VEC + e] = t[e];
+    }
+  }
+  const T* Kb = Kc + bg * D.N_kv * D_;
+  const T* Vb = Vc + bg * D.N_kv * D_;
+  constexpr int TPW = kUnitTile / kUnitWarps;            // tokens per warp per tile (16)
+  constexpr int STEPS = TPW / SS::RPW;
+  float oacc[GM][SS::DPL];
+#pragma unroll
+  for (int h = 0; h < GM; ++h)
+#pragma unroll
+    for (int e = 0; e < SS::DPL; ++e) oacc[h][e] = 0.f;
 
+  uint32_t phase = 0;
+  bool ok = true;
   for (int64_t j0 = t0; j0 < t1; j0 += kUnitTile) {
     const int cnt = (int)(t1 - j0 < kUnitTile ? t1 - j0 : kUnitTile);
-    __syncthreads();   // previous tile fully consumed; qf / stats initialised
-    for (int e = tid * 4; e < kUnitTile * d; e += kUnitThreads * 4) {
-      const int t = e / d, k = e - t * d;
-      float kv[4] = {0.f, 0.f, 0.f, 0.f}, vv[4] = {0.f, 0.f, 0.f, 0.f};
-      if (t < cnt) {
-        Elem<T>::load4(Kb + (j0 + t) * d + k, kv);
-        Elem<T>::load4(Vb + (j0 + t) * d + k, vv);
-      }
-      Elem<float>::store4(Ks + t * dp + k, kv);
-      Elem<float>::store4(Vs + t * dp + k, vv);
+    if (tid == 0) {
+      const uint32_t bytes = (uint32_t)cnt * D_ * sizeof(T);
+      sm100::mbar_expect_tx(&full, 2 * bytes);
+      sm100::bulk_load(Ks, Kb + j0 * D_, bytes, &full);
+      sm100::bulk_load(Vs, Vb + j0 * D_, bytes, &full);
     }
-    __syncthreads();
-    for (int pr = tid; pr < G * kUnitTile; pr += kUnitThreads) {
-      const int hh = pr / kUnitTile, t = pr - hh * kUnitTile;
-      float x = -INFINITY;
-      if (t < cnt) {
-        const float* kr = Ks + t * dp;
-        const float* qr = qf + hh * d;
-        float a = 0.f;
-        for (int k = 0; k < d; k += 4) {
-          const float4 kv = *reinterpret_cast<const float4*>(kr + k);
-          const float4 qv = *reinterpret_cast<const float4*>(qr + k);
-          a = fmaf(qv.x, kv.x, a);
-          a = fmaf(qv.y, kv.y, a);
-          a = fmaf(qv.z, kv.z, a);
-          a = fmaf(qv.w, kv.w, a);
+    const bool landed = sm100::mbar_wait(&full, phase, 1u << 24);
+    phase ^= 1u;
+    if (!__syncthreads_and(landed)) { ok = false; break; }
+    // pass 1: logits of this warp's tokens
+#pragma unroll
+    for (int st = 0; st < STEPS; ++st) {
+      const int tk = warp * TPW + st * SS::RPW + grp;
+      float kv[SS::DPL];
+      if (tk < cnt) {
+#pragma unroll
+        for (int v = 0; v < SS::NV; ++v) {
+          float t[SS::VEC];
+          load_vec_shared<T, SS::VEC>(Ks + tk * D_ + (v * SS::L + gl) * SS::VEC, t);
+#pragma unroll
+          for (int e = 0; e < SS::VEC; ++e) kv[v * SS::VEC + e] = t[e];
         }
-        x = a * D.scale;
+      } else {
+#pragma unroll
+        for (int e = 0; e < SS::DPL; ++e) kv[e] = 0.f;
       }
-      xs[pr] = x;
+      float acc[GM];
+#pragma unroll
+      for (int h = 0; h < GM; ++h) {
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < SS::DPL; ++e) a = fmaf(qreg[h][e], kv[e], a);
+        acc[h] = a;
+      }
+#pragma unroll
+      for (int o = SS::L / 2; o > 0; o >>= 1)
+#pragma unroll
+        for (int h = 0; h < GM; ++h) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
+      if (gl == 0) {
+#pragma unroll
+        for (int h = 0; h < GM; ++h) xs[h][tk] = tk < cnt ? acc[h] * D.scale : -INFINITY;
+      }
     }
     __syncthreads();
-    // online softmax statistics, one warp per head (kUnitTile == 32)
-    for (int hh = warp; hh < G; hh += kUnitThreads / 32) {
-      const float x = xs[hh * kUnitTile + lane];
-      const float m_old = mst[hh];
-      const float mn = fmaxf(m_old, warp_max(x));
-      const float p = (x == -INFINITY) ? 0.f : expf(x - mn);
-      const float s = warp_sum(p);
-      xs[hh * kUnitTile + lane] = p;
+    // softmax statistics of the tile, one warp per head
+    for (int h = warp; h < G; h += kUnitWarps) {
+      const float x0 = xs[h][lane], x1 = xs[h][lane + 32];
+      const float m_old = mst[h];
+      const float mn = fmaxf(m_old, warp_max(fmaxf(x0, x1)));
+      const float p0 = x0 == -INFINITY ? 0.f : __expf(x0 - mn);
+      const float p1 = x1 == -INFINITY ? 0.f : __expf(x1 - mn);
+      const float sum = warp_sum(p0 + p1);
+      xs[h][lane] = p0;
+      xs[h][lane + 32] = p1;
       if (lane == 0) {
-        const float corr = (m_old == -INFINITY) ? 0.f : expf(m_old - mn);
-        cst[hh] = corr;
-        lst[hh] = lst[hh] * corr + s;
-        mst[hh] = mn;
+        const float corr = m_old == -INFINITY ? 0.f : __expf(m_old - mn);
+        cst[h] = corr;
+        lst[h] = lst[h] * corr + sum;
+        mst[h] = mn;
       }
     }
     __syncthreads();
+    // pass 2: p * V for this warp's tokens
 #pragma unroll
-    for (int r = 0; r < kMaxPairs; ++r) {
-      const int pr = tid + r * kUnitThreads;
-      if (pr < n_pairs) {
-        const int hh = pr / d, k = pr - hh * d;
-        float a = acc[r] * cst[hh];
-        const float* pp = xs + hh * kUnitTile;
-        for (int t = 0; t < cnt; ++t) a = fmaf(pp[t], Vs[t * dp + k], a);
-        acc[r] = a;
+    for (int h = 0; h < GM; ++h) {
+      const float cr = h < G ? cst[h] : 1.f;
+#pragma unroll
+      for (int e = 0; e < SS::DPL; ++e) oacc[h][e] *= cr;
+    }
+#pragma unroll
+    for (int st = 0; st < STEPS; ++st) {
+      const int tk = warp * TPW + st * SS::RPW + grp;
+      if (tk < cnt) {
+        float vv[SS::DPL];
+#pragma unroll
+        for (int v = 0; v < SS::NV; ++v) {
+          float t[SS::VEC];
+          load_vec_shared<T, SS::VEC>(Vs + tk * D_ + (v * SS::L + gl) * SS::VEC, t);
+#pragma unroll
+          for (int e = 0; e < SS::VEC; ++e) vv[v * SS::VEC + e] = t[e];
+        }
+#pragma unroll
+        for (int h = 0; h < GM; ++h) {
+          const float pv = h < G ? xs[h][tk] : 0.f;
+#pragma unroll
+          for (int e = 0; e < SS::DPL; ++e) oacc[h][e] = fmaf(pv, vv[e], oacc[h][e]);
+        }
       }
     }
+    __syncthreads();   // Ks / Vs / xs / cst are rewritten by the next tile
   }
-  __syncthreads();
+  if (!ok && tid == 0) record_status(status, kStatusTimeout);
+  // reduce partial outputs: across the lane groups of a warp, then across warps
 #pragma unroll
-  for (int r = 0; r < kMaxPairs; ++r) {
-    const int pr = tid + r * kUnitThreads;
-    if (pr < n_pairs) {
-      const int hh = pr / d, k = pr - hh * d;
-      const float l = lst[hh];
-      const float v = l > 0.f ? acc[r] / l : 0.f;
-      part_o[((hrow0 + (int64_t)hh * D.N_q) * NU + unit) * d + k] = v;
+  for (int o = SS::L; o < 32; o <<= 1)
+#pragma unroll
+    for (int h = 0; h < GM; ++h)
+#pragma unroll
+      for (int e = 0; e < SS::DPL; ++e) oacc[h][e] += __shfl_xor_sync(0xffffffffu, oacc[h][e], o);
+  constexpr int QUARTER = GM * D_ / 4;
+#pragma unroll
+  for (int qq = 0; qq < 4; ++qq) {
+    if (grp == 0) {
+#pragma unroll
+      for (int h = 0; h < GM; ++h)
+#pragma unroll
+        for (int v = 0; v < SS::NV; ++v)
+#pragma unroll
+          for (int e = 0; e < SS::VEC; ++e) {
+            const int flat = h * D_ + (v * SS::L + gl) * SS::VEC + e;
+            if (flat / QUARTER == qq)
+              red[warp * QUARTER + flat - qq * QUARTER] = oacc[h][v * SS::VEC + e];
+          }
     }
+    __syncthreads();
+    for (int f = tid; f < QUARTER; f += kUnitThreads) {
+      const int flat = qq * QUARTER + f;
+      const int h = flat / D_, k = flat - h * D_;
+      if (h < G) {
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kUnitWarps; ++w) sum += red[w * QUARTER + f];
+        const float l = lst[h];
+        part_o[((hrow0 + (int64_t)h * D.N_q) * NU + unit) * D_ + k] = l > 0.f ? sum / l : 0.f;
+      }
+    }
+    __syncthreads();
   }
   if (tid < G) {
     const float l = lst[tid];
-    part_lse[(hrow0 + (int64_t)tid * D.N_q) * NU + unit] = l > 0.f ? mst[tid] + logf(l) : -INFINITY;
+    part_lse[(hrow0 + (int64_t)tid * D.N_q) * NU + unit] =
+        l > 0.f ? mst[tid] + logf(l) : -INFINITY;
   }
 }
 
@@ -327,32 +423,44 @@ cudaError_t launch_attn_rows(const Dims& D, bool bf16, const void* q, const void
   return cudaGetLastError();
 }
 
-size_t units_smem_bytes(const Dims& D) {
-  const size_t dp = (size_t)D.d + 4;
-  return sizeof(float) * ((size_t)D.G * D.d + 2 * kUnitTile * dp + (size_t)D.G * kUnitTile +
-                          3 * (size_t)D.G);
+size_t units_smem_bytes(const Dims& D) { (void)D; return 0; }
+
+template <typename T, int D_>
+static cudaError_t launch_units_d(const Dims& D, int n_pieces, const void* q, const void* K,
+                                  const void* V, const int32_t* idx, float* part_o,
+                                  float* part_lse, int32_t* status, cudaStream_t st) {
+  dim3 grid((unsigned)(D.K + n_pieces), (unsigned)(D.B * D.Hkv * D.N_q));
+#define HILS_UNITS(GM)                                                                        \
+  do {                                                                                        \
+    const size_t smem = 2 * kUnitTile * D_ * sizeof(T) +                                     \
+                        (size_t)kUnitWarps * GM * D_ / 4 * sizeof(float);                    \
+    cudaError_t e = cudaFuncSetAttribute(attn_units_kernel<T, D_, GM>,                        \
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,         \
+                                         (int)smem);                                          \
+    if (e != cudaSuccess) return e;                                                           \
+    e = cudaFuncSetAttribute(attn_units_kernel<T, D_, GM>,                                    \
+                             cudaFuncAttributePreferredSharedMemoryCarveout,                  \
+                             cudaSharedmemCarveoutMaxShared);                                 \
+    if (e != cudaSuccess) return e;                                                           \
+    attn_units_kernel<T, D_, GM><<<grid, kUnitThreads, smem, st>>>(                           \
+        D, n_pieces, (const T*)q, (const T*)K, (const T*)V, idx, part_o, part_lse, status);   \
+  } while (0)
+  if (D.G <= 4) HILS_UNITS(4);
+  else if (D.G <= 8) HILS_UNITS(8);
+  else HILS_UNITS(16);
+#undef HILS_UNITS
+  return cudaGetLastError();
 }
 
 cudaError_t launch_attn_units(const Dims& D, bool bf16, int n_pieces, const void* q,
                               const void* K, const void* V, const int32_t* idx, float* part_o,
-                              float* part_lse, cudaStream_t st) {
-  const int64_t rows = D.B * D.Hkv * D.N_q;
-  if (rows == 0) return cudaSuccess;
-  const size_t smem = units_smem_bytes(D);
-  dim3 grid((unsigned)(D.K + n_pieces), (unsigned)rows);
-  if (bf16) {
-    auto k = attn_units_kernel<__nv_bfloat16>;
-    if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<grid, kUnitThreads, smem, st>>>(D, n_pieces, (const __nv_bfloat16*)q,
-                                        (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, idx,
-                                        part_o, part_lse);
-  } else {
-    auto k = attn_units_kernel<float>;
-    if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<grid, kUnitThreads, smem, st>>>(D, n_pieces, (const float*)q, (const float*)K,
-                                        (const float*)V, idx, part_o, part_lse);
-  }
-  return cudaGetLastError();
+                              float* part_lse, int32_t* status, cudaStream_t st) {
+  if (D.B * D.Hkv * D.N_q == 0) return cudaSuccess;
+  if (D.d == 128)
+    return bf16 ? launch_units_d<__nv_bfloat16, 128>(D, n_pieces, q, K, V, idx, part_o, part_lse, status, st)
+                : launch_units_d<float, 128>(D, n_pieces, q, K, V, idx, part_o, part_lse, status, st);
+  return bf16 ? launch_units_d<__nv_bfloat16, 64>(D, n_pieces, q, K, V, idx, part_o, part_lse, status, st)
+              : launch_units_d<float, 64>(D, n_pieces, q, K, V, idx, part_o, part_lse, status, st);
 }
 
 cudaError_t launch_fuse_units(const Dims& D, bool bf16, int n_pieces, const float* s_sel,

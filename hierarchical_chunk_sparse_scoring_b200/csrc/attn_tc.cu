@@ -55,6 +55,15 @@ struct AtShape {
   static constexpr uint32_t O_COL = 128;
 };
 
+constexpr float kLog2e = 1.4426950408889634f;
+
+// 2^x with the SFU's approximate base-2 exponential (ex2.approx; 2^-inf = 0).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&t);
@@ -322,41 +331,58 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       const bool is_win = valid && !is_sel && c >= n_i && t0 <= pos;
       bool rescale = false;
       float factor = 1.f;
+      // base-2 exponentials throughout: x * scale * log2(e) is the logit in log2 units
+      const float sc2 = D.scale * kLog2e;
       if (is_sel && u != -INFINITY) {
         // intra-chunk softmax of this chunk, weighted by exp(u - m_run) (u <= m_run)
-        float mx = -INFINITY;
+        float pm[8];
 #pragma unroll
-        for (int j = 0; j < kTile; ++j) { p[j] *= D.scale; mx = fmaxf(mx, p[j]); }
-        float sum = 0.f;
+        for (int q8 = 0; q8 < 8; ++q8) pm[q8] = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < kTile; ++j) { p[j] = __expf(p[j] - mx); sum += p[j]; }
-        const float w = __expf(u - m_run);
+        for (int j = 0; j < kTile; ++j) pm[j & 7] = fmaxf(pm[j & 7], p[j]);
+        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        const float off = -mx * sc2;
+        float ps[8];
+#pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8) ps[q8] = 0.f;
+#pragma unroll
+        for (int j = 0; j < kTile; ++j) { p[j] = fast_exp2(fmaf(p[j], sc2, off)); ps[j & 7] += p[j]; }
+        const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        const float w = fast_exp2((u - m_run) * kLog2e);
         const float f = w / sum;
 #pragma unroll
         for (int j = 0; j < kTile; ++j) p[j] *= f;
         l += w;
       } else if (is_win) {
-        float mt = -INFINITY;
+        float pm[8];
+#pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8) pm[q8] = -INFINITY;
 #pragma unroll
         for (int j = 0; j < kTile; ++j) {
           p[j] = (t0 + j <= pos) ? p[j] * D.scale : -INFINITY;
-          mt = fmaxf(mt, p[j]);
+          pm[j & 7] = fmaxf(pm[j & 7], p[j]);
         }
+        const float mt = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
         if (mt > m_run + kRescaleMargin) {
           if (l > 0.f) {
-            factor = __expf(m_run - mt);
+            factor = fast_exp2((m_run - mt) * kLog2e);
             l *= factor;
             rescale = true;
           }
           m_run = mt;
         }
-        float sum = 0.f;
+        const float off = -m_run * kLog2e;
+        float ps[8];
+#pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8) ps[q8] = 0.f;
 #pragma unroll
         for (int j = 0; j < kTile; ++j) {
-          p[j] = p[j] == -INFINITY ? 0.f : __expf(p[j] - m_run);
-          sum += p[j];
+          p[j] = p[j] == -INFINITY ? 0.f : fast_exp2(fmaf(p[j], kLog2e, off));
+          ps[j & 7] += p[j];
         }
-        l += sum;
+        l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       } else {
 #pragma unroll
         for (int j = 0; j < kTile; ++j) p[j] = 0.f;
@@ -419,7 +445,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           *reinterpret_cast<uint4*>(orow + 16 * j + 8) = c4;
         }
       }
-      if (valid && lse_out) lse_out[hrow] = m_run + __logf(l);
+      if (valid && lse_out) lse_out[hrow] = m_run + logf(l);
     } else if (!ok || n_tiles > 0) {
       record_status(status, kStatusTimeout);
     }

@@ -146,6 +146,59 @@ __device__ __forceinline__ void warp_merge_topk(TopList<KM>& L, int K, int lane,
   }
 }
 
+// Decode layout.  Lanes are grouped L per landmark row; lane l of a group owns the row's
+// 16-byte vectors l, l+L, l+2L, ... so one warp instruction reads 32/L whole rows contiguously.
+template <typename T, int D_, int GM>
+struct SplitShape {
+  static constexpr int DPL = GM <= 4 ? 16 : (GM == 8 ? 8 : 4);   // dims per lane
+  static constexpr int L = D_ / DPL;                              // lanes per row
+  static constexpr int VEC = (16 / (int)sizeof(T)) < DPL ? (16 / (int)sizeof(T)) : DPL;
+  static constexpr int NV = DPL / VEC;                            // vector loads per row
+  static constexpr int RPW = 32 / L;                              // rows per warp step
+  static_assert(L >= 1 && L <= 32 && (32 % L) == 0, "lane grouping");
+};
+
+template <typename T, int VEC>
+__device__ __forceinline__ void load_vec(const T* p, float (&v)[VEC]);
+
+template <>
+__device__ __forceinline__ void load_vec<__nv_bfloat16, 8>(const __nv_bfloat16* p, float (&v)[8]) {
+  uint4 t = __ldg(reinterpret_cast<const uint4*>(p));
+  v[0] = bf16_lo(t.x); v[1] = bf16_hi(t.x); v[2] = bf16_lo(t.y); v[3] = bf16_hi(t.y);
+  v[4] = bf16_lo(t.z); v[5] = bf16_hi(t.z); v[6] = bf16_lo(t.w); v[7] = bf16_hi(t.w);
+}
+template <>
+__device__ __forceinline__ void load_vec<__nv_bfloat16, 4>(const __nv_bfloat16* p, float (&v)[4]) {
+  Elem<__nv_bfloat16>::load4(p, v);
+}
+template <>
+__device__ __forceinline__ void load_vec<float, 4>(const float* p, float (&v)[4]) {
+  Elem<float>::load4(p, v);
+}
+
+// Same vectors from shared memory (no read-only cache path).
+template <typename T, int VEC>
+__device__ __forceinline__ void load_vec_shared(const T* p, float (&v)[VEC]);
+
+template <>
+__device__ __forceinline__ void load_vec_shared<__nv_bfloat16, 8>(const __nv_bfloat16* p,
+                                                                  float (&v)[8]) {
+  const uint4 t = *reinterpret_cast<const uint4*>(p);
+  v[0] = bf16_lo(t.x); v[1] = bf16_hi(t.x); v[2] = bf16_lo(t.y); v[3] = bf16_hi(t.y);
+  v[4] = bf16_lo(t.z); v[5] = bf16_hi(t.z); v[6] = bf16_lo(t.w); v[7] = bf16_hi(t.w);
+}
+template <>
+__device__ __forceinline__ void load_vec_shared<__nv_bfloat16, 4>(const __nv_bfloat16* p,
+                                                                  float (&v)[4]) {
+  const uint2 t = *reinterpret_cast<const uint2*>(p);
+  v[0] = bf16_lo(t.x); v[1] = bf16_hi(t.x); v[2] = bf16_lo(t.y); v[3] = bf16_hi(t.y);
+}
+template <>
+__device__ __forceinline__ void load_vec_shared<float, 4>(const float* p, float (&v)[4]) {
+  const float4 t = *reinterpret_cast<const float4*>(p);
+  v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+}
+
 __device__ __forceinline__ void record_status(int32_t* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }

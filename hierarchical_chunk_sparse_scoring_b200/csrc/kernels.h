@@ -30,6 +30,13 @@ size_t split_smem_bytes(int cps);
 cudaError_t launch_select_split(const Dims& D, bool bf16, int cps, int n_split, const void* qc,
                                 const void* klm, const float* blm, float* part_v,
                                 int32_t* part_c, cudaStream_t st);
+cudaError_t launch_select_stream(const Dims& D, bool bf16, int cps, int n_split,
+                                 int64_t n_stride, const void* qc, const void* klm,
+                                 const float* blm, float* sigma, int32_t* status,
+                                 cudaStream_t st);
+cudaError_t launch_select_topk(const Dims& D, bool bf16, int64_t n_stride, const float* sigma,
+                               const void* qc, const void* klm, const float* blm, int32_t* idx,
+                               float* s_sel, cudaStream_t st);
 cudaError_t launch_select_merge(const Dims& D, bool bf16, int n_split, const float* part_v,
                                 const int32_t* part_c, const void* qc, const void* klm,
                                 const float* blm, int32_t* idx, float* s_sel, cudaStream_t st);
@@ -41,7 +48,7 @@ cudaError_t launch_attn_rows(const Dims& D, bool bf16, const void* q, const void
 size_t units_smem_bytes(const Dims& D);
 cudaError_t launch_attn_units(const Dims& D, bool bf16, int n_pieces, const void* q,
                               const void* K, const void* V, const int32_t* idx, float* part_o,
-                              float* part_lse, cudaStream_t st);
+                              float* part_lse, int32_t* status, cudaStream_t st);
 
 cudaError_t launch_fuse_units(const Dims& D, bool bf16, int n_pieces, const float* s_sel,
                               const float* part_o, const float* part_lse, void* out, float* lse,

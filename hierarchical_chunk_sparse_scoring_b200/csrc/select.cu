@@ -14,6 +14,7 @@
 //                        where one query's landmark stream (n x d) must be spread over the GPU.
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace hils {
 
@@ -204,37 +205,6 @@ cudaError_t launch_select_scores(const Dims& D, bool bf16, const void* qc, const
               : launch_scores_g<float>(D, qc, klm, blm, idx, s_sel, st);
 }
 
-// ---------------------------------------------------------------------------------------------
-// Decode layout.  Lanes are grouped L per landmark row; lane l of a group owns the row's
-// 16-byte vectors l, l+L, l+2L, ... so one warp instruction reads 32/L whole rows contiguously.
-template <typename T, int D_, int GM>
-struct SplitShape {
-  static constexpr int DPL = GM <= 4 ? 16 : (GM == 8 ? 8 : 4);   // dims per lane
-  static constexpr int L = D_ / DPL;                              // lanes per row
-  static constexpr int VEC = (16 / (int)sizeof(T)) < DPL ? (16 / (int)sizeof(T)) : DPL;
-  static constexpr int NV = DPL / VEC;                            // vector loads per row
-  static constexpr int RPW = 32 / L;                              // rows per warp step
-  static_assert(L >= 1 && L <= 32 && (32 % L) == 0, "lane grouping");
-};
-
-template <typename T, int VEC>
-__device__ __forceinline__ void load_vec(const T* p, float (&v)[VEC]);
-
-template <>
-__device__ __forceinline__ void load_vec<__nv_bfloat16, 8>(const __nv_bfloat16* p, float (&v)[8]) {
-  uint4 t = __ldg(reinterpret_cast<const uint4*>(p));
-  v[0] = bf16_lo(t.x); v[1] = bf16_hi(t.x); v[2] = bf16_lo(t.y); v[3] = bf16_hi(t.y);
-  v[4] = bf16_lo(t.z); v[5] = bf16_hi(t.z); v[6] = bf16_lo(t.w); v[7] = bf16_hi(t.w);
-}
-template <>
-__device__ __forceinline__ void load_vec<__nv_bfloat16, 4>(const __nv_bfloat16* p, float (&v)[4]) {
-  Elem<__nv_bfloat16>::load4(p, v);
-}
-template <>
-__device__ __forceinline__ void load_vec<float, 4>(const float* p, float (&v)[4]) {
-  Elem<float>::load4(p, v);
-}
-
 constexpr int kSplitThreads = 256;
 constexpr int kSplitWarps = kSplitThreads / 32;
 
@@ -381,6 +351,151 @@ __global__ void __launch_bounds__(128) select_merge_kernel(Dims D, int n_split,
 }
 
 // ---------------------------------------------------------------------------------------------
+// Decode, streaming form.  select_stream_kernel reads every eligible landmark row of a query
+// exactly once (coalesced 16-byte loads, several rows in flight per lane group) and writes the
+// group score sigma_c = max_h s_{h,c} to a scratch row; select_topk_kernel then selects the K
+// best of each row and computes the per-head scores of the winners.  The scratch write is
+// 4 bytes per landmark row read (d * 2 bytes), under 2% extra traffic for d = 128.
+constexpr int kStreamThreads = 128;
+constexpr int kStreamWarps = kStreamThreads / 32;
+
+template <typename T, int D_, int GM>
+__global__ void __launch_bounds__(kStreamThreads) select_stream_kernel(
+    Dims D, int cps, int64_t n_stride, const T* __restrict__ qc, const T* __restrict__ klm,
+    const float* __restrict__ blm, float* __restrict__ sigma, int32_t* __restrict__ status) {
+  using SS = SplitShape<T, D_, GM>;
+  extern __shared__ __align__(128) uint8_t sm_stream[];
+  T* rows_sm = reinterpret_cast<T*>(sm_stream);   // [cps][D_]
+  __shared__ uint64_t full;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int split = blockIdx.x;
+  const int64_t row = blockIdx.y;
+  const int64_t i = row % D.N_q, bg = row / D.N_q, g = bg % D.Hkv, b = bg / D.Hkv;
+  const int G = D.G;
+  const int64_t n = n_eligible(D.q_pos0 + i, D.S, D.W);
+  const int64_t c0 = (int64_t)split * cps;
+  const int64_t c1 = c0 + cps < n ? c0 + cps : n;
+  const int cnt = c1 > c0 ? (int)(c1 - c0) : 0;
+  if (cnt == 0) return;
+  // one bulk copy of this CTA's contiguous landmark rows
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&full, 1);
+    sm100::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t bytes = (uint32_t)cnt * D_ * sizeof(T);
+    sm100::mbar_expect_tx(&full, bytes);
+    sm100::bulk_load(rows_sm, klm + (bg * D.C + c0) * D_, bytes, &full);
+  }
+  // this lane's slice of every head's calibrated query stays in registers
+  const int grp = lane / SS::L, gl = lane % SS::L;
+  float qreg[GM][SS::DPL];
+#pragma unroll
+  for (int h = 0; h < GM; ++h) {
+#pragma unroll
+    for (int v = 0; v < SS::NV; ++v) {
+      float t[SS::VEC];
+      if (h < G) {
+        load_vec<T, SS::VEC>(qc + (((b * D.Hq) + g * G + h) * D.N_q + i) * D_ +
+                                 (v * SS::L + gl) * SS::VEC, t);
+      } else {
+#pragma unroll
+        for (int e = 0; e < SS::VEC; ++e) t[e] = 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < SS::VEC; ++e) qreg[h][v * SS::VEC + e] = t[e];
+    }
+  }
+  const bool landed = sm100::mbar_wait(&full, 0, 1u << 24);
+  if (!landed) record_status(status, kStatusTimeout);
+  if (!__syncthreads_and(landed)) return;
+  const float* bb = blm + bg * D.C + c0;
+  float* out = sigma + row * n_stride + c0;
+  constexpr int STEP = kStreamWarps * SS::RPW;
+  for (int base = warp * SS::RPW; base < cnt; base += STEP) {
+    const int r = base + grp;
+    float kv[SS::DPL];
+    if (r < cnt) {
+      const T* kr = rows_sm + (size_t)r * D_;
+#pragma unroll
+      for (int v = 0; v < SS::NV; ++v) {
+        float t[SS::VEC];
+        load_vec_shared<T, SS::VEC>(kr + (v * SS::L + gl) * SS::VEC, t);
+#pragma unroll
+        for (int e = 0; e < SS::VEC; ++e) kv[v * SS::VEC + e] = t[e];
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < SS::DPL; ++e) kv[e] = 0.f;
+    }
+    float acc[GM];
+#pragma unroll
+    for (int h = 0; h < GM; ++h) {
+      float a = 0.f;
+#pragma unroll
+      for (int e = 0; e < SS::DPL; ++e) a = fmaf(qreg[h][e], kv[e], a);
+      acc[h] = a;
+    }
+#pragma unroll
+    for (int o = SS::L / 2; o > 0; o >>= 1)
+#pragma unroll
+      for (int h = 0; h < GM; ++h) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
+    if (gl == 0 && r < cnt) {
+      const float bc = __ldg(bb + r);
+      float sig = -INFINITY;
+#pragma unroll
+      for (int h = 0; h < GM; ++h)
+        if (h < G) sig = fmaxf(sig, fmaf(acc[h], D.scale, bc));
+      out[r] = sig;
+    }
+  }
+}
+
+// One CTA per (b, g, query): top-K of the row's n group scores, then per-head scores of the
+// winners.  Lists per thread, merged per warp, then across warps.
+template <typename T, int GM, int KM>
+__global__ void __launch_bounds__(256) select_topk_kernel(Dims D, int64_t n_stride,
+                                                          const float* __restrict__ sigma,
+                                                          const T* __restrict__ qc,
+                                                          const T* __restrict__ klm,
+                                                          const float* __restrict__ blm,
+                                                          int32_t* __restrict__ idx,
+                                                          float* __restrict__ s_sel) {
+  __shared__ float lv[8 * kMaxK];
+  __shared__ int lc[8 * kMaxK];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t row = blockIdx.x;
+  const int64_t i = row % D.N_q, bg = row / D.N_q, g = bg % D.Hkv, b = bg / D.Hkv;
+  const int K = D.K;
+  const int64_t n = n_eligible(D.q_pos0 + i, D.S, D.W);
+  const float* sr = sigma + row * n_stride;
+  TopList<KM> L;
+  L.clear();
+  for (int64_t c = threadIdx.x; c < n; c += 256) L.insert(sr[c], (int)c, K);
+  float wv;
+  int wc;
+  warp_merge_topk<KM>(L, K, lane, wv, wc);
+  if (lane < K) { lv[warp * K + lane] = wv; lc[warp * K + lane] = wc; }
+  __syncthreads();
+  if (warp != 0) return;
+  int ptr = 0;
+  int mine = INT_MAX;
+  for (int r = 0; r < K; ++r) {
+    float v = -INFINITY;
+    int c = INT_MAX;
+    if (lane < 8 && ptr < K) { v = lv[lane * K + ptr]; c = lc[lane * K + ptr]; }
+    float bv = v;
+    int bc = c;
+    warp_best(bv, bc);
+    if (lane < 8 && c == bc && bc != INT_MAX) ++ptr;
+    if (lane == r) mine = bc;
+  }
+  write_selection<T, GM>(D, b, g, i, nullptr, qc, klm + bg * D.C * D.d, blm + bg * D.C, lane,
+                         mine, idx, s_sel);
+}
+
+// ---------------------------------------------------------------------------------------------
 // Host-side launchers.
 
 template <typename T, int GM, int KM>
@@ -508,6 +623,57 @@ cudaError_t launch_select_merge(const Dims& D, bool bf16, int n_split, const flo
   if (D.B * D.Hkv * D.N_q == 0) return cudaSuccess;
   return dispatch_tdgk<MergeRun>(bf16, D.d, D.G, D.K, &D, n_split, part_v, part_c, qc, klm, blm,
                                  idx, s_sel, st);
+}
+
+template <typename T, int D_, int GM, int KM>
+struct StreamOnly {
+  static cudaError_t run(const Dims* D, int cps, int n_split, int64_t n_stride, const void* qc,
+                         const void* klm, const float* blm, float* sigma, int32_t* status,
+                         cudaStream_t st) {
+    const int64_t rows = D->B * D->Hkv * D->N_q;
+    dim3 grid((unsigned)n_split, (unsigned)rows);
+    const size_t smem = (size_t)cps * D_ * sizeof(T);
+    cudaError_t e = cudaFuncSetAttribute(select_stream_kernel<T, D_, GM>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    // many small CTAs per SM keep many bulk copies in flight: ask for the largest carveout
+    e = cudaFuncSetAttribute(select_stream_kernel<T, D_, GM>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    select_stream_kernel<T, D_, GM><<<grid, kStreamThreads, smem, st>>>(
+        *D, cps, n_stride, (const T*)qc, (const T*)klm, blm, sigma, status);
+    return cudaGetLastError();
+  }
+};
+
+template <typename T, int D_, int GM, int KM>
+struct TopkOnly {
+  static cudaError_t run(const Dims* D, int64_t n_stride, const float* sigma, const void* qc,
+                         const void* klm, const float* blm, int32_t* idx, float* s_sel,
+                         cudaStream_t st) {
+    const int64_t rows = D->B * D->Hkv * D->N_q;
+    select_topk_kernel<T, GM, KM><<<(unsigned)rows, 256, 0, st>>>(
+        *D, n_stride, sigma, (const T*)qc, (const T*)klm, blm, idx, s_sel);
+    return cudaGetLastError();
+  }
+};
+
+cudaError_t launch_select_stream(const Dims& D, bool bf16, int cps, int n_split,
+                                 int64_t n_stride, const void* qc, const void* klm,
+                                 const float* blm, float* sigma, int32_t* status,
+                                 cudaStream_t st) {
+  if (D.B * D.Hkv * D.N_q == 0) return cudaSuccess;
+  return dispatch_tdgk<StreamOnly>(bf16, D.d, D.G, D.K, &D, cps, n_split, n_stride, qc, klm,
+                                   blm, sigma, status, st);
+}
+
+cudaError_t launch_select_topk(const Dims& D, bool bf16, int64_t n_stride, const float* sigma,
+                               const void* qc, const void* klm, const float* blm, int32_t* idx,
+                               float* s_sel, cudaStream_t st) {
+  if (D.B * D.Hkv * D.N_q == 0) return cudaSuccess;
+  return dispatch_tdgk<TopkOnly>(bf16, D.d, D.G, D.K, &D, n_stride, sigma, qc, klm, blm, idx,
+                                 s_sel, st);
 }
 
 }  // namespace hils

@@ -198,3 +198,20 @@ __device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t smem_addr,
 
 }  // namespace sm100
 }  // namespace hils
+
+namespace hils {
+namespace sm100 {
+
+// Contiguous global -> shared copy by the bulk-copy engine (TMA, 1-D); completes `bytes` of
+// transaction count on `bar`.  Addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gmem_src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+}  // namespace sm100
+}  // namespace hils
