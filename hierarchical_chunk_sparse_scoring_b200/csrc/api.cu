@@ -23,7 +23,7 @@ constexpr size_t kAlign = 256;
 constexpr size_t kStatusBytes = 256;
 constexpr int kChunksPerSplit = 512;
 constexpr int64_t kDecodeMaxQueries = 16;
-constexpr int kStreamRows = 128;   // landmark rows per streaming CTA (one bulk copy)
+constexpr int kStreamRows = 1024;  // landmark rows per streaming CTA (a ring of bulk copies)
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -105,6 +105,14 @@ Plan make_plan(const hils_params* p) {
   return P;
 }
 
+// segments per row for the decode top-K (<= n_split, so the split lists fit the workspace)
+int n_topk_segments(const Plan& P) {
+  int64_t s = (P.n_stride + 1023) / 1024;
+  if (s > 16) s = 16;
+  if (s > P.n_split) s = P.n_split;
+  return (int)(s < 1 ? 1 : s);
+}
+
 int n_stream_split(const Plan& P) {
   const int64_t n_max = P.n_stride;
   const int64_t s = (n_max + kStreamRows - 1) / kStreamRows;
@@ -150,12 +158,13 @@ struct PhaseMarks {
 };
 
 int phase_names(const Plan& P, const char** names, int max_names) {
-  static const char* kDecode[] = {"select_stream", "select_topk", "attn_units", "fuse_units"};
+  static const char* kDecode[] = {"select_stream", "select_topk", "select_merge", "attn_units",
+                                  "fuse_units"};
   const char* pre[3];
   int n = 0;
   if (P.decode) {
-    for (int i = 0; i < 4 && i < max_names; ++i) names[i] = kDecode[i];
-    return 4;
+    for (int i = 0; i < 5 && i < max_names; ++i) names[i] = kDecode[i];
+    return 5;
   }
   if (P.tc_select) { pre[n++] = "score_topk_tc"; pre[n++] = "select_scores"; }
   else pre[n++] = "select_rows";
@@ -194,13 +203,14 @@ hils_status forward_impl(const hils_params* p, const void* q, const void* q_cal,
     float* po = reinterpret_cast<float*>(ws + P.off_po);
     float* pl = reinterpret_cast<float*>(ws + P.off_pl);
     float* sig = reinterpret_cast<float*>(ws + P.off_sig);
-    (void)pv;
-    (void)pc;
     e = launch_select_stream(P.D, P.bf16, kStreamRows, n_stream_split(P), P.n_stride, q_cal, k_lm,
                              b_lm, sig, reinterpret_cast<int32_t*>(ws), st);
     pm.mark();
+    const int n_seg = n_topk_segments(P);
+    if (e == cudaSuccess) e = launch_select_topk(P.D, n_seg, P.n_stride, sig, pv, pc, st);
+    pm.mark();
     if (e == cudaSuccess)
-      e = launch_select_topk(P.D, P.bf16, P.n_stride, sig, q_cal, k_lm, b_lm, idx, s_sel, st);
+      e = launch_select_merge(P.D, P.bf16, n_seg, pv, pc, q_cal, k_lm, b_lm, idx, s_sel, st);
     pm.mark();
     if (e == cudaSuccess) e = launch_attn_units(P.D, P.bf16, P.n_pieces, q, K, V, idx, po, pl,
                                                   reinterpret_cast<int32_t*>(ws), st);
@@ -275,8 +285,12 @@ extern "C" hils_status hils_select(const hils_params* p, const void* q_cal, cons
     float* sig = reinterpret_cast<float*>(ws + P.off_sig);
     e = launch_select_stream(P.D, P.bf16, kStreamRows, n_stream_split(P), P.n_stride, q_cal, k_lm,
                              b_lm, sig, reinterpret_cast<int32_t*>(ws), st);
+    float* pv = reinterpret_cast<float*>(ws + P.off_pv);
+    int32_t* pc = reinterpret_cast<int32_t*>(ws + P.off_pc);
+    const int n_seg = n_topk_segments(P);
+    if (e == cudaSuccess) e = launch_select_topk(P.D, n_seg, P.n_stride, sig, pv, pc, st);
     if (e == cudaSuccess)
-      e = launch_select_topk(P.D, P.bf16, P.n_stride, sig, q_cal, k_lm, b_lm, idx, s_sel, st);
+      e = launch_select_merge(P.D, P.bf16, n_seg, pv, pc, q_cal, k_lm, b_lm, idx, s_sel, st);
   } else if (P.tc_select) {
     e = launch_score_topk_tc(P.D, q_cal, k_lm, b_lm, idx, reinterpret_cast<int32_t*>(ws), st);
     if (e == cudaSuccess && s_sel)

@@ -363,7 +363,9 @@ __global__ void __launch_bounds__(kUnitThreads) attn_units_kernel(
 }
 
 // Fusion of K chunk units (scores s_sel) and n_pieces window pieces (scores = their lse, whose
-// log-sum-exp is the window's lse).  Units with score -inf get weight 0.
+// log-sum-exp is the window's lse).  Units with score -inf get weight 0.  One warp per
+// (b, h, query): lane u first holds unit u's weight, then the lanes sweep d with the weights
+// broadcast, loading eight units' vectors before accumulating them.
 template <typename T>
 __global__ void __launch_bounds__(128) fuse_units_kernel(Dims D, int n_pieces,
                                                          const float* __restrict__ s_sel,
@@ -385,22 +387,41 @@ __global__ void __launch_bounds__(128) fuse_units_kernel(Dims D, int n_pieces,
   float Z = 0.f;
   for (int u = lane; u < NU; u += 32) {
     const float s = score_of(u);
-    Z += (s == -INFINITY) ? 0.f : expf(s - M);
+    Z += (s == -INFINITY) ? 0.f : __expf(s - M);
   }
   Z = warp_sum(Z);
   const float invZ = 1.f / Z;
-  for (int k0 = lane * 4; k0 < d; k0 += 128) {
+  const float* pr = part_o + row * NU * d;
+  // every lane runs every iteration (the loop body shuffles); lanes past d only skip memory
+  for (int kb = 0; kb < d; kb += 128) {
+    const int k0 = kb + lane * 4;
+    const bool act = k0 < d;
     float o[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int u = 0; u < NU; ++u) {
-      const float s = score_of(u);
-      if (s == -INFINITY) continue;
-      const float w = expf(s - M) * invZ;
-      float v[4];
-      Elem<float>::load4(part_o + (row * NU + u) * d + k0, v);
+    for (int ub = 0; ub < NU; ub += 32) {
+      const int um = ub + lane;
+      const float su = um < NU ? score_of(um) : -INFINITY;
+      const float wl = su == -INFINITY ? 0.f : __expf(su - M) * invZ;   // lane's unit weight
+      const int cnt = NU - ub < 32 ? NU - ub : 32;
+      for (int u8 = 0; u8 < cnt; u8 += 8) {
+        float v[8][4];
+        float w[8];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) o[e] = fmaf(w, v[e], o[e]);
+        for (int e = 0; e < 8; ++e) {
+          w[e] = __shfl_sync(0xffffffffu, wl, (u8 + e) & 31);
+          if (u8 + e < cnt && act) {
+            Elem<float>::load4(pr + (int64_t)(ub + u8 + e) * d + k0, v[e]);
+          } else {
+            w[e] = 0.f;
+            v[e][0] = v[e][1] = v[e][2] = v[e][3] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+#pragma unroll
+          for (int x = 0; x < 4; ++x) o[x] = fmaf(w[e], v[e][x], o[x]);
+      }
     }
-    Elem<T>::store4(out + row * d + k0, o);
+    if (act) Elem<T>::store4(out + row * d + k0, o);
   }
   if (lse_out && lane == 0) lse_out[row] = M + logf(Z);
 }

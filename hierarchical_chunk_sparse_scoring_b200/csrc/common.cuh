@@ -99,16 +99,21 @@ struct TopList {
     for (int k = 0; k < KM; ++k) { v[k] = -INFINITY; c[k] = INT_MAX; }
   }
 
-  // Inserts (x, ci) if it beats slot K-1; keeps the list ordered by `better`.  The new entry
-  // walks down the list swapping with every slot it beats (static indexing only, so the list
-  // stays in registers); the displaced last entry falls off.
+  // Inserts (x, ci) if it beats slot K-1; keeps the list ordered by `better`.  Because the list
+  // is sorted, "x beats slot k" holds exactly for the slots from x's position on, so every slot's
+  // new content follows from the old list in parallel (no dependent chain through the slots):
+  // slot k takes x if x beats it but not slot k-1, slot k-1's old entry if x beats both.
   __device__ __forceinline__ void insert(float x, int ci, int K) {
+    bool m[KM];
 #pragma unroll
-    for (int k = 0; k < KM; ++k) {
-      const bool sw = (k < K) && better(x, ci, v[k], c[k]);
-      const float tv = v[k];
-      const int tc = c[k];
-      if (sw) { v[k] = x; c[k] = ci; x = tv; ci = tc; }
+    for (int k = 0; k < KM; ++k) m[k] = (k < K) && better(x, ci, v[k], c[k]);
+#pragma unroll
+    for (int k = KM - 1; k >= 0; --k) {
+      if (m[k]) {
+        const bool shift = k > 0 && m[k - 1];
+        v[k] = shift ? v[k - 1] : x;
+        c[k] = shift ? c[k - 1] : ci;
+      }
     }
   }
 
@@ -118,6 +123,42 @@ struct TopList {
     v[KM - 1] = -INFINITY;
     c[KM - 1] = INT_MAX;
   }
+};
+
+// Sorted list of the K best candidates kept in the LAST K of KM register slots; the first KM-K
+// slots hold unbeatable sentinels (+inf), so the K-th best is always slot KM-1 and no access
+// depends on the runtime K (dynamic indexing would move the list to local memory).
+template <int KM>
+struct TailList {
+  float v[KM];
+  int c[KM];
+
+  __device__ __forceinline__ void clear(int K) {
+#pragma unroll
+    for (int k = 0; k < KM; ++k) {
+      const bool sentinel = k < KM - K;
+      v[k] = sentinel ? INFINITY : -INFINITY;
+      c[k] = sentinel ? -1 : INT_MAX;
+    }
+  }
+
+  // Parallel insertion as in TopList::insert (sentinels are never beaten).
+  __device__ __forceinline__ void insert(float x, int ci) {
+    bool m[KM];
+#pragma unroll
+    for (int k = 0; k < KM; ++k) m[k] = better(x, ci, v[k], c[k]);
+#pragma unroll
+    for (int k = KM - 1; k >= 0; --k) {
+      if (m[k]) {
+        const bool shift = k > 0 && m[k - 1];
+        v[k] = shift ? v[k - 1] : x;
+        c[k] = shift ? c[k - 1] : ci;
+      }
+    }
+  }
+
+  __device__ __forceinline__ float kth_v() const { return v[KM - 1]; }
+  __device__ __forceinline__ int kth_c() const { return c[KM - 1]; }
 };
 
 // Warp-wide arg-best of one (value, index) per lane under `better`; every lane gets it.

@@ -44,7 +44,8 @@ struct TcShape {
   static constexpr int B_STAGE = KB * B_BOX;
   static constexpr int STASH_BYTES = (16 * 256 * 4) > (kRows * KM * 8) ? (16 * 256 * 4)
                                                                        : (kRows * KM * 8);
-  static constexpr int FIXED = A_BYTES + STASH_BYTES + 1024 /*barriers*/ + 1024 /*align*/;
+  static constexpr int FIXED = A_BYTES + STASH_BYTES + 1024 /*barriers*/ + 1024 /*align*/ +
+                               2048 /*shared thresholds*/;
   static constexpr int STAGES_FIT = (kSmemLimit - FIXED) / B_STAGE;
   static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
   // more than half of the SM's shared memory, so a second CTA can never be co-resident and
@@ -57,15 +58,6 @@ struct TcShape {
   static_assert(STAGES >= 2, "shared memory too small for this shape");
   static_assert(HALF % 16 == 0, "sub-blocks of 16 columns");
 };
-
-template <int KM>
-__device__ __forceinline__ void kth(const TopList<KM>& L, int K, float& v, int& c) {
-  v = -INFINITY;
-  c = INT_MAX;
-#pragma unroll
-  for (int k = 0; k < KM; ++k)
-    if (k == K - 1) { v = L.v[k]; c = L.c[k]; }
-}
 
 }  // namespace
 
@@ -91,6 +83,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* acc_full = a_full + 1;      // [2]
   uint64_t* acc_empty = acc_full + 2;   // [2]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  // each epilogue thread's current K-th best (value, chunk), read by the thread serving the
+  // same query in the other column half: [2 halves][128 rows]
+  float* th_v = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 1024);
+  int* th_c = reinterpret_cast<int*>(th_v + 2 * kRows);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t qt = (int64_t)gridDim.x - 1 - blockIdx.x;   // longest query tiles first
@@ -188,10 +184,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int64_t n_i = valid ? n_eligible(D.q_pos0 + i, D.S, D.W) : 0;
     const float* bb = blm + bg * D.C;
     float* st = stash + e * 32 + lane;      // stash[j * 256 + thread]
-    TopList<KM> L;
-    L.clear();
+    TailList<KM> L;
+    L.clear(K);
     float thv = -INFINITY;
     int thc = INT_MAX;
+    th_v[ch * kRows + r] = -INFINITY;
+    th_c[ch * kRows + r] = INT_MAX;
+    float* my_tv = th_v + ch * kRows + r;
+    int* my_tc = th_c + ch * kRows + r;
+    const float* pa_tv = th_v + (1 - ch) * kRows + r;
+    const int* pa_tc = th_c + (1 - ch) * kRows + r;
+    asm volatile("bar.sync 1, 256;" ::: "memory");   // thresholds initialised
     const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
     bool ok = true;
     for (int t = 0; t < n_tiles; ++t) {
@@ -221,13 +224,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int j = 0; j < 16; ++j)
               sig[j] = (h0 + hh == 0) ? tmp[hh][j] : fmaxf(sig[j], tmp[hh][j]);
         }
+        // a candidate must beat both this list's K-th best and the other half's (either list
+        // already holds K candidates at least that good)
+        const float pv = *reinterpret_cast<const volatile float*>(pa_tv);
+        const int pc = *reinterpret_cast<const volatile int*>(pa_tc);
         uint32_t pass = 0;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int64_t c = c0 + j;
           const float bj = __shfl_sync(0xffffffffu, bl, j);
           sig[j] = fmaf(sig[j], D.scale, bj);
-          if (c < n_i && better(sig[j], (int)c, thv, thc)) pass |= 1u << j;
+          if (c < n_i && better(sig[j], (int)c, thv, thc) && better(sig[j], (int)c, pv, pc))
+            pass |= 1u << j;
         }
         if (__any_sync(0xffffffffu, pass != 0)) {
 #pragma unroll
@@ -236,9 +244,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             while (pass) {
               const int j = __ffs(pass) - 1;
               pass &= pass - 1;
-              L.insert(st[j * 256], (int)(c0 + j), K);
+              L.insert(st[j * 256], (int)(c0 + j));
             }
-            kth<KM>(L, K, thv, thc);
+            thv = L.kth_v();
+            thc = L.kth_c();
+            *reinterpret_cast<volatile float*>(my_tv) = thv;
+            *reinterpret_cast<volatile int*>(my_tc) = thc;
           }
         }
       }
@@ -257,14 +268,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     asm volatile("bar.sync 1, 256;" ::: "memory");
     if (ch == 0 && valid) {
-      for (int k = 0; k < K; ++k) {
+      // the partner's live entries are its last K slots
+      for (int k = KM - K; k < KM; ++k) {
         const int c = xc[r * KM + k];
-        if (c != INT_MAX) L.insert(xv[r * KM + k], c, K);
+        if (c != INT_MAX) L.insert(xv[r * KM + k], c);
       }
-      int32_t* out = idx + (bg * D.N_q + i) * K;
+      int32_t* out = idx + (bg * D.N_q + i) * K - (KM - K);
 #pragma unroll
       for (int k = 0; k < KM; ++k)
-        if (k < K) out[k] = (L.c[k] == INT_MAX) ? -1 : L.c[k];
+        if (k >= KM - K) out[k] = (L.c[k] == INT_MAX) ? -1 : L.c[k];
     }
   }
   tc_fence_before();

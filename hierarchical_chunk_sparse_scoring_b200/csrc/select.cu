@@ -356,8 +356,10 @@ __global__ void __launch_bounds__(128) select_merge_kernel(Dims D, int n_split,
 // group score sigma_c = max_h s_{h,c} to a scratch row; select_topk_kernel then selects the K
 // best of each row and computes the per-head scores of the winners.  The scratch write is
 // 4 bytes per landmark row read (d * 2 bytes), under 2% extra traffic for d = 128.
-constexpr int kStreamThreads = 128;
-constexpr int kStreamWarps = kStreamThreads / 32;
+constexpr int kStreamWarps = 4;                          // consumer warps
+constexpr int kStreamThreads = (kStreamWarps + 1) * 32;  // + one producer warp
+constexpr int kStreamStages = 4;
+constexpr int kStreamStageRows = 64;
 
 template <typename T, int D_, int GM>
 __global__ void __launch_bounds__(kStreamThreads) select_stream_kernel(
@@ -365,8 +367,8 @@ __global__ void __launch_bounds__(kStreamThreads) select_stream_kernel(
     const float* __restrict__ blm, float* __restrict__ sigma, int32_t* __restrict__ status) {
   using SS = SplitShape<T, D_, GM>;
   extern __shared__ __align__(128) uint8_t sm_stream[];
-  T* rows_sm = reinterpret_cast<T*>(sm_stream);   // [cps][D_]
-  __shared__ uint64_t full;
+  T* ring = reinterpret_cast<T*>(sm_stream);   // [kStreamStages][kStreamStageRows][D_]
+  __shared__ uint64_t full[kStreamStages], empty[kStreamStages];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int split = blockIdx.x;
   const int64_t row = blockIdx.y;
@@ -377,18 +379,37 @@ __global__ void __launch_bounds__(kStreamThreads) select_stream_kernel(
   const int64_t c1 = c0 + cps < n ? c0 + cps : n;
   const int cnt = c1 > c0 ? (int)(c1 - c0) : 0;
   if (cnt == 0) return;
-  // one bulk copy of this CTA's contiguous landmark rows
+  const int n_stages = (cnt + kStreamStageRows - 1) / kStreamStageRows;
   if (threadIdx.x == 0) {
-    sm100::mbar_init(&full, 1);
+    for (int s = 0; s < kStreamStages; ++s) {
+      sm100::mbar_init(&full[s], 1);
+      sm100::mbar_init(&empty[s], kStreamWarps);
+    }
     sm100::fence_barrier_init();
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    const uint32_t bytes = (uint32_t)cnt * D_ * sizeof(T);
-    sm100::mbar_expect_tx(&full, bytes);
-    sm100::bulk_load(rows_sm, klm + (bg * D.C + c0) * D_, bytes, &full);
+  const T* src = klm + (bg * D.C + c0) * D_;
+  if (warp == kStreamWarps) {
+    // producer warp: keeps up to kStreamStages bulk copies of landmark rows in flight
+    if (lane == 0) {
+      for (int t = 0; t < n_stages; ++t) {
+        const int s = t % kStreamStages;
+        const uint32_t u = (uint32_t)(t / kStreamStages);
+        if (!sm100::mbar_wait(&empty[s], (u & 1u) ^ 1u, 1u << 24)) {
+          record_status(status, kStatusTimeout);
+          break;
+        }
+        const int r0 = t * kStreamStageRows;
+        const int rows_here = cnt - r0 < kStreamStageRows ? cnt - r0 : kStreamStageRows;
+        const uint32_t bytes = (uint32_t)rows_here * D_ * sizeof(T);
+        sm100::mbar_expect_tx(&full[s], bytes);
+        sm100::bulk_load(ring + (size_t)s * kStreamStageRows * D_, src + (int64_t)r0 * D_, bytes,
+                         &full[s]);
+      }
+    }
+    return;
   }
-  // this lane's slice of every head's calibrated query stays in registers
+  // consumer warps: this lane's slice of every head's calibrated query stays in registers
   const int grp = lane / SS::L, gl = lane % SS::L;
   float qreg[GM][SS::DPL];
 #pragma unroll
@@ -407,72 +428,95 @@ __global__ void __launch_bounds__(kStreamThreads) select_stream_kernel(
       for (int e = 0; e < SS::VEC; ++e) qreg[h][v * SS::VEC + e] = t[e];
     }
   }
-  const bool landed = sm100::mbar_wait(&full, 0, 1u << 24);
-  if (!landed) record_status(status, kStatusTimeout);
-  if (!__syncthreads_and(landed)) return;
   const float* bb = blm + bg * D.C + c0;
   float* out = sigma + row * n_stride + c0;
   constexpr int STEP = kStreamWarps * SS::RPW;
-  for (int base = warp * SS::RPW; base < cnt; base += STEP) {
-    const int r = base + grp;
-    float kv[SS::DPL];
-    if (r < cnt) {
-      const T* kr = rows_sm + (size_t)r * D_;
+  constexpr int PER_STAGE = (kStreamStageRows + STEP - 1) / STEP;   // row-steps per warp
+  for (int t = 0; t < n_stages; ++t) {
+    const int s = t % kStreamStages;
+    const uint32_t u = (uint32_t)(t / kStreamStages);
+    const int r0 = t * kStreamStageRows;
+    const int rows_here = cnt - r0 < kStreamStageRows ? cnt - r0 : kStreamStageRows;
+    // landmark biases of this warp's rows, requested before waiting for the rows themselves
+    float bias[PER_STAGE];
 #pragma unroll
-      for (int v = 0; v < SS::NV; ++v) {
-        float t[SS::VEC];
-        load_vec_shared<T, SS::VEC>(kr + (v * SS::L + gl) * SS::VEC, t);
+    for (int k = 0; k < PER_STAGE; ++k) {
+      const int r = warp * SS::RPW + k * STEP + grp;
+      bias[k] = r < rows_here ? __ldg(bb + r0 + r) : 0.f;
+    }
+    if (!sm100::mbar_wait(&full[s], u & 1u, 1u << 24)) {
+      record_status(status, kStatusTimeout);
+      break;
+    }
+    const T* stage = ring + (size_t)s * kStreamStageRows * D_;
 #pragma unroll
-        for (int e = 0; e < SS::VEC; ++e) kv[v * SS::VEC + e] = t[e];
+    for (int k = 0; k < PER_STAGE; ++k) {
+      const int base = warp * SS::RPW + k * STEP;
+      if (base >= rows_here) break;
+      const int r = base + grp;
+      float kv[SS::DPL];
+      if (r < rows_here) {
+        const T* kr = stage + (size_t)r * D_;
+#pragma unroll
+        for (int v = 0; v < SS::NV; ++v) {
+          float tv[SS::VEC];
+          load_vec_shared<T, SS::VEC>(kr + (v * SS::L + gl) * SS::VEC, tv);
+#pragma unroll
+          for (int e = 0; e < SS::VEC; ++e) kv[v * SS::VEC + e] = tv[e];
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < SS::DPL; ++e) kv[e] = 0.f;
       }
-    } else {
+      float acc[GM];
 #pragma unroll
-      for (int e = 0; e < SS::DPL; ++e) kv[e] = 0.f;
+      for (int h = 0; h < GM; ++h) {
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < SS::DPL; ++e) a = fmaf(qreg[h][e], kv[e], a);
+        acc[h] = a;
+      }
+#pragma unroll
+      for (int o = SS::L / 2; o > 0; o >>= 1)
+#pragma unroll
+        for (int h = 0; h < GM; ++h) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
+      if (gl == 0 && r < rows_here) {
+        const float bc = bias[k];
+        float sig = -INFINITY;
+#pragma unroll
+        for (int h = 0; h < GM; ++h)
+          if (h < G) sig = fmaxf(sig, fmaf(acc[h], D.scale, bc));
+        out[r0 + r] = sig;
+      }
     }
-    float acc[GM];
-#pragma unroll
-    for (int h = 0; h < GM; ++h) {
-      float a = 0.f;
-#pragma unroll
-      for (int e = 0; e < SS::DPL; ++e) a = fmaf(qreg[h][e], kv[e], a);
-      acc[h] = a;
-    }
-#pragma unroll
-    for (int o = SS::L / 2; o > 0; o >>= 1)
-#pragma unroll
-      for (int h = 0; h < GM; ++h) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
-    if (gl == 0 && r < cnt) {
-      const float bc = __ldg(bb + r);
-      float sig = -INFINITY;
-#pragma unroll
-      for (int h = 0; h < GM; ++h)
-        if (h < G) sig = fmaxf(sig, fmaf(acc[h], D.scale, bc));
-      out[r] = sig;
-    }
+    __syncwarp();
+    if (lane == 0) sm100::mbar_arrive(&empty[s]);
   }
 }
 
-// One CTA per (b, g, query): top-K of the row's n group scores, then per-head scores of the
-// winners.  Lists per thread, merged per warp, then across warps.
-template <typename T, int GM, int KM>
-__global__ void __launch_bounds__(256) select_topk_kernel(Dims D, int64_t n_stride,
+// Top-K of one segment of a row's group scores (blockIdx.x = segment, blockIdx.y = (b, g,
+// query)): per-thread lists, merged per warp, then across warps; the segment's K best go to
+// part_v / part_c [rows][segments][K] for select_merge_kernel.
+template <int KM>
+__global__ void __launch_bounds__(256) select_topk_kernel(Dims D, int64_t n_stride, int n_seg,
                                                           const float* __restrict__ sigma,
-                                                          const T* __restrict__ qc,
-                                                          const T* __restrict__ klm,
-                                                          const float* __restrict__ blm,
-                                                          int32_t* __restrict__ idx,
-                                                          float* __restrict__ s_sel) {
+                                                          float* __restrict__ part_v,
+                                                          int32_t* __restrict__ part_c) {
   __shared__ float lv[8 * kMaxK];
   __shared__ int lc[8 * kMaxK];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t row = blockIdx.x;
-  const int64_t i = row % D.N_q, bg = row / D.N_q, g = bg % D.Hkv, b = bg / D.Hkv;
+  const int seg = blockIdx.x;
+  const int64_t row = blockIdx.y;
+  const int64_t i = row % D.N_q;
   const int K = D.K;
   const int64_t n = n_eligible(D.q_pos0 + i, D.S, D.W);
+  const int64_t per = (n + n_seg - 1) / n_seg;
+  const int64_t c0 = (int64_t)seg * per;
+  const int64_t c1 = c0 + per < n ? c0 + per : n;
   const float* sr = sigma + row * n_stride;
   TopList<KM> L;
   L.clear();
-  for (int64_t c = threadIdx.x; c < n; c += 256) L.insert(sr[c], (int)c, K);
+  for (int64_t c = c0 + threadIdx.x; c < c1; c += 256) L.insert(sr[c], (int)c, K);
   float wv;
   int wc;
   warp_merge_topk<KM>(L, K, lane, wv, wc);
@@ -480,7 +524,8 @@ __global__ void __launch_bounds__(256) select_topk_kernel(Dims D, int64_t n_stri
   __syncthreads();
   if (warp != 0) return;
   int ptr = 0;
-  int mine = INT_MAX;
+  float* outv = part_v + (row * n_seg + seg) * K;
+  int32_t* outc = part_c + (row * n_seg + seg) * K;
   for (int r = 0; r < K; ++r) {
     float v = -INFINITY;
     int c = INT_MAX;
@@ -489,10 +534,8 @@ __global__ void __launch_bounds__(256) select_topk_kernel(Dims D, int64_t n_stri
     int bc = c;
     warp_best(bv, bc);
     if (lane < 8 && c == bc && bc != INT_MAX) ++ptr;
-    if (lane == r) mine = bc;
+    if (lane == 0) { outv[r] = bv; outc[r] = bc; }
   }
-  write_selection<T, GM>(D, b, g, i, nullptr, qc, klm + bg * D.C * D.d, blm + bg * D.C, lane,
-                         mine, idx, s_sel);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -632,7 +675,7 @@ struct StreamOnly {
                          cudaStream_t st) {
     const int64_t rows = D->B * D->Hkv * D->N_q;
     dim3 grid((unsigned)n_split, (unsigned)rows);
-    const size_t smem = (size_t)cps * D_ * sizeof(T);
+    const size_t smem = (size_t)kStreamStages * kStreamStageRows * D_ * sizeof(T);
     cudaError_t e = cudaFuncSetAttribute(select_stream_kernel<T, D_, GM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -647,18 +690,6 @@ struct StreamOnly {
   }
 };
 
-template <typename T, int D_, int GM, int KM>
-struct TopkOnly {
-  static cudaError_t run(const Dims* D, int64_t n_stride, const float* sigma, const void* qc,
-                         const void* klm, const float* blm, int32_t* idx, float* s_sel,
-                         cudaStream_t st) {
-    const int64_t rows = D->B * D->Hkv * D->N_q;
-    select_topk_kernel<T, GM, KM><<<(unsigned)rows, 256, 0, st>>>(
-        *D, n_stride, sigma, (const T*)qc, (const T*)klm, blm, idx, s_sel);
-    return cudaGetLastError();
-  }
-};
-
 cudaError_t launch_select_stream(const Dims& D, bool bf16, int cps, int n_split,
                                  int64_t n_stride, const void* qc, const void* klm,
                                  const float* blm, float* sigma, int32_t* status,
@@ -668,12 +699,18 @@ cudaError_t launch_select_stream(const Dims& D, bool bf16, int cps, int n_split,
                                    blm, sigma, status, st);
 }
 
-cudaError_t launch_select_topk(const Dims& D, bool bf16, int64_t n_stride, const float* sigma,
-                               const void* qc, const void* klm, const float* blm, int32_t* idx,
-                               float* s_sel, cudaStream_t st) {
-  if (D.B * D.Hkv * D.N_q == 0) return cudaSuccess;
-  return dispatch_tdgk<TopkOnly>(bf16, D.d, D.G, D.K, &D, n_stride, sigma, qc, klm, blm, idx,
-                                 s_sel, st);
+cudaError_t launch_select_topk(const Dims& D, int n_seg, int64_t n_stride, const float* sigma,
+                               float* part_v, int32_t* part_c, cudaStream_t st) {
+  const int64_t rows = D.B * D.Hkv * D.N_q;
+  if (rows == 0) return cudaSuccess;
+  dim3 grid((unsigned)n_seg, (unsigned)rows);
+  if (D.K <= 8)
+    select_topk_kernel<8><<<grid, 256, 0, st>>>(D, n_stride, n_seg, sigma, part_v, part_c);
+  else if (D.K <= 16)
+    select_topk_kernel<16><<<grid, 256, 0, st>>>(D, n_stride, n_seg, sigma, part_v, part_c);
+  else
+    select_topk_kernel<32><<<grid, 256, 0, st>>>(D, n_stride, n_seg, sigma, part_v, part_c);
+  return cudaGetLastError();
 }
 
 }  // namespace hils
