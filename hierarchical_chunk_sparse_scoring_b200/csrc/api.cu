@@ -158,13 +158,12 @@ struct PhaseMarks {
 };
 
 int phase_names(const Plan& P, const char** names, int max_names) {
-  static const char* kDecode[] = {"select_stream", "select_topk", "select_merge", "attn_units",
-                                  "fuse_units"};
+  static const char* kDecode[] = {"select_stream", "select_topk", "attn_units", "fuse_units"};
   const char* pre[3];
   int n = 0;
   if (P.decode) {
-    for (int i = 0; i < 5 && i < max_names; ++i) names[i] = kDecode[i];
-    return 5;
+    for (int i = 0; i < 4 && i < max_names; ++i) names[i] = kDecode[i];
+    return 4;
   }
   if (P.tc_select) { pre[n++] = "score_topk_tc"; pre[n++] = "select_scores"; }
   else pre[n++] = "select_rows";
@@ -206,11 +205,10 @@ hils_status forward_impl(const hils_params* p, const void* q, const void* q_cal,
     e = launch_select_stream(P.D, P.bf16, kStreamRows, n_stream_split(P), P.n_stride, q_cal, k_lm,
                              b_lm, sig, reinterpret_cast<int32_t*>(ws), st);
     pm.mark();
-    const int n_seg = n_topk_segments(P);
-    if (e == cudaSuccess) e = launch_select_topk(P.D, n_seg, P.n_stride, sig, pv, pc, st);
-    pm.mark();
+    (void)pv;
+    (void)pc;
     if (e == cudaSuccess)
-      e = launch_select_merge(P.D, P.bf16, n_seg, pv, pc, q_cal, k_lm, b_lm, idx, s_sel, st);
+      e = launch_select_topk_row(P.D, P.bf16, P.n_stride, sig, q_cal, k_lm, b_lm, idx, s_sel, st);
     pm.mark();
     if (e == cudaSuccess) e = launch_attn_units(P.D, P.bf16, P.n_pieces, q, K, V, idx, po, pl,
                                                   reinterpret_cast<int32_t*>(ws), st);
@@ -285,12 +283,8 @@ extern "C" hils_status hils_select(const hils_params* p, const void* q_cal, cons
     float* sig = reinterpret_cast<float*>(ws + P.off_sig);
     e = launch_select_stream(P.D, P.bf16, kStreamRows, n_stream_split(P), P.n_stride, q_cal, k_lm,
                              b_lm, sig, reinterpret_cast<int32_t*>(ws), st);
-    float* pv = reinterpret_cast<float*>(ws + P.off_pv);
-    int32_t* pc = reinterpret_cast<int32_t*>(ws + P.off_pc);
-    const int n_seg = n_topk_segments(P);
-    if (e == cudaSuccess) e = launch_select_topk(P.D, n_seg, P.n_stride, sig, pv, pc, st);
     if (e == cudaSuccess)
-      e = launch_select_merge(P.D, P.bf16, n_seg, pv, pc, q_cal, k_lm, b_lm, idx, s_sel, st);
+      e = launch_select_topk_row(P.D, P.bf16, P.n_stride, sig, q_cal, k_lm, b_lm, idx, s_sel, st);
   } else if (P.tc_select) {
     e = launch_score_topk_tc(P.D, q_cal, k_lm, b_lm, idx, reinterpret_cast<int32_t*>(ws), st);
     if (e == cudaSuccess && s_sel)

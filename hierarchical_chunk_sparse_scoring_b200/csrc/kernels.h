@@ -36,6 +36,9 @@ cudaError_t launch_select_stream(const Dims& D, bool bf16, int cps, int n_split,
                                  cudaStream_t st);
 cudaError_t launch_select_topk(const Dims& D, int n_seg, int64_t n_stride, const float* sigma,
                                float* part_v, int32_t* part_c, cudaStream_t st);
+cudaError_t launch_select_topk_row(const Dims& D, bool bf16, int64_t n_stride,
+                                   const float* sigma, const void* qc, const void* klm,
+                                   const float* blm, int32_t* idx, float* s_sel, cudaStream_t st);
 cudaError_t launch_select_merge(const Dims& D, bool bf16, int n_split, const float* part_v,
                                 const int32_t* part_c, const void* qc, const void* klm,
                                 const float* blm, int32_t* idx, float* s_sel, cudaStream_t st);

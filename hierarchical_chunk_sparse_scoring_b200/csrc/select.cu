@@ -180,6 +180,109 @@ __global__ void __launch_bounds__(128) select_scores_kernel(Dims D, const T* __r
   }
 }
 
+// bf16 variant: one warp per (b, g, query); LPC lanes share a selected chunk, each holding
+// D_/LPC of its landmark dimensions in registers (16-byte loads, all issued before use); the
+// group's calibrated queries are staged in shared memory as fp32.
+template <int D_, int GM, int LPC>
+__global__ void __launch_bounds__(128) select_scores_bf16_kernel(
+    Dims D, const __nv_bfloat16* __restrict__ qc, const __nv_bfloat16* __restrict__ klm,
+    const float* __restrict__ blm, const int32_t* __restrict__ idx, float* __restrict__ s_sel) {
+  constexpr int DPL = D_ / LPC;          // dims per lane
+  constexpr int NV = DPL / 8;            // 16-byte vectors per lane
+  __shared__ __align__(16) float qs[4][GM * D_];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t rows = D.B * D.Hkv * D.N_q;
+  const int64_t row = (int64_t)blockIdx.x * 4 + warp;
+  if (row >= rows) return;
+  const int64_t i = row % D.N_q, bg = row / D.N_q, g = bg % D.Hkv, b = bg / D.Hkv;
+  const int K = D.K, G = D.G;
+  const int slot = lane / LPC, part = lane % LPC;
+  // independent loads first (the selection and this row's calibrated queries), then the
+  // selected landmark rows and biases, which depend on the selection
+  const int c = slot < K ? idx[row * K + slot] : -1;
+  constexpr int QV = (GM * D_ + 255) / 256;   // 16-byte query vectors per lane
+  float qv[QV][8];
+#pragma unroll
+  for (int x = 0; x < QV; ++x) {
+    const int e = x * 256 + lane * 8;
+    if (e < G * D_) {
+      const int h = e / D_, k = e - h * D_;
+      load_vec<__nv_bfloat16, 8>(qc + (((b * D.Hq) + g * G + h) * D.N_q + i) * D_ + k, qv[x]);
+    }
+  }
+  const bool valid = c >= 0 && c < D.C;
+  float kv[DPL];
+  if (valid) {
+    const __nv_bfloat16* kr = klm + (bg * D.C + c) * D_ + part * DPL;
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      float t[8];
+      load_vec<__nv_bfloat16, 8>(kr + v * 8, t);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) kv[v * 8 + e] = t[e];
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) kv[e] = 0.f;
+  }
+  const float bc = valid ? __ldg(blm + bg * D.C + c) : 0.f;
+#pragma unroll
+  for (int x = 0; x < QV; ++x) {
+    const int e = x * 256 + lane * 8;
+    if (e < G * D_) {
+      *reinterpret_cast<float4*>(&qs[warp][e]) = make_float4(qv[x][0], qv[x][1], qv[x][2], qv[x][3]);
+      *reinterpret_cast<float4*>(&qs[warp][e + 4]) = make_float4(qv[x][4], qv[x][5], qv[x][6], qv[x][7]);
+    }
+  }
+  __syncwarp();
+#pragma unroll
+  for (int h = 0; h < GM; ++h) {
+    if (h >= G) break;
+    float a = 0.f;
+#pragma unroll
+    for (int e4 = 0; e4 < DPL; e4 += 4) {
+      const float4 q4 = *reinterpret_cast<const float4*>(&qs[warp][h * D_ + part * DPL + e4]);
+      a = fmaf(q4.x, kv[e4 + 0], a);
+      a = fmaf(q4.y, kv[e4 + 1], a);
+      a = fmaf(q4.z, kv[e4 + 2], a);
+      a = fmaf(q4.w, kv[e4 + 3], a);
+    }
+#pragma unroll
+    for (int o = LPC / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    if (part == 0 && slot < K) {
+      const int64_t hrow = ((b * D.Hq) + g * G + h) * D.N_q + i;
+      s_sel[hrow * K + slot] = valid ? fmaf(a, D.scale, bc) : -INFINITY;
+    }
+  }
+}
+
+template <int D_, int GM>
+static cudaError_t launch_scores_bf16_g(const Dims& D, const void* qc, const void* klm,
+                                        const float* blm, const int32_t* idx, float* s_sel,
+                                        cudaStream_t st) {
+  const int64_t rows = D.B * D.Hkv * D.N_q;
+  const unsigned blocks = (unsigned)((rows + 3) / 4);
+  const auto* q = (const __nv_bfloat16*)qc;
+  const auto* k = (const __nv_bfloat16*)klm;
+  if (D.K <= 8)
+    select_scores_bf16_kernel<D_, GM, 4><<<blocks, 128, 0, st>>>(D, q, k, blm, idx, s_sel);
+  else if (D.K <= 16)
+    select_scores_bf16_kernel<D_, GM, 2><<<blocks, 128, 0, st>>>(D, q, k, blm, idx, s_sel);
+  else
+    select_scores_bf16_kernel<D_, GM, 1><<<blocks, 128, 0, st>>>(D, q, k, blm, idx, s_sel);
+  return cudaGetLastError();
+}
+
+template <int D_>
+static cudaError_t launch_scores_bf16_d(const Dims& D, const void* qc, const void* klm,
+                                        const float* blm, const int32_t* idx, float* s_sel,
+                                        cudaStream_t st) {
+  if (D.G <= 1) return launch_scores_bf16_g<D_, 1>(D, qc, klm, blm, idx, s_sel, st);
+  if (D.G <= 2) return launch_scores_bf16_g<D_, 2>(D, qc, klm, blm, idx, s_sel, st);
+  if (D.G <= 4) return launch_scores_bf16_g<D_, 4>(D, qc, klm, blm, idx, s_sel, st);
+  return launch_scores_bf16_g<D_, 8>(D, qc, klm, blm, idx, s_sel, st);
+}
+
 template <typename T>
 static cudaError_t launch_scores_g(const Dims& D, const void* qc, const void* klm,
                                    const float* blm, const int32_t* idx, float* s_sel,
@@ -201,6 +304,9 @@ cudaError_t launch_select_scores(const Dims& D, bool bf16, const void* qc, const
                                  const float* blm, const int32_t* idx, float* s_sel,
                                  cudaStream_t st) {
   if (D.B * D.Hkv * D.N_q == 0 || D.K == 0) return cudaSuccess;
+  if (bf16 && D.G <= 8 && (D.d == 64 || D.d == 128))
+    return D.d == 128 ? launch_scores_bf16_d<128>(D, qc, klm, blm, idx, s_sel, st)
+                      : launch_scores_bf16_d<64>(D, qc, klm, blm, idx, s_sel, st);
   return bf16 ? launch_scores_g<__nv_bfloat16>(D, qc, klm, blm, idx, s_sel, st)
               : launch_scores_g<float>(D, qc, klm, blm, idx, s_sel, st);
 }
@@ -538,6 +644,113 @@ __global__ void __launch_bounds__(256) select_topk_kernel(Dims D, int64_t n_stri
   }
 }
 
+// Decode top-K of one query row's group scores, one 1024-thread CTA per (b, g, query).
+//   1. every warp takes the best (value, chunk) of its candidates: 32 warp maxima;
+//   2. warp 0 sorts them (bitonic network over shuffles); the K-th of them, theta, is a lower
+//      bound of the row's K-th best (those K maxima are K distinct candidates >= theta);
+//   3. every candidate >= theta is appended to a shared list (typically a few dozen);
+//   4. one warp takes the exact top-K of that list (register lists, warp merge) and writes idx
+//      and the per-head scores.  If more than kSurvivorCap candidates tie at or above theta,
+//      step 4 runs over all candidates instead (slower, same result).
+constexpr int kTopkThreads = 1024;
+constexpr int kSurvivorCap = 2048;
+
+// ascending-by-`better` position: true if (v, c) should come before (ov, oc)
+__device__ __forceinline__ void cmpx(float& v, int& c, int partner_lane_xor, bool keep_better) {
+  const float ov = __shfl_xor_sync(0xffffffffu, v, partner_lane_xor);
+  const int oc = __shfl_xor_sync(0xffffffffu, c, partner_lane_xor);
+  const bool other_better = better(ov, oc, v, c);
+  if (keep_better == other_better) { v = ov; c = oc; }
+}
+
+template <typename T, int GM, int KM>
+__global__ void __launch_bounds__(kTopkThreads) select_topk_row_kernel(
+    Dims D, int64_t n_stride, const float* __restrict__ sigma, const T* __restrict__ qc,
+    const T* __restrict__ klm, const float* __restrict__ blm, int32_t* __restrict__ idx,
+    float* __restrict__ s_sel) {
+  __shared__ float wv_sh[32];
+  __shared__ int wc_sh[32];
+  __shared__ float th_v;
+  __shared__ int th_c;
+  __shared__ int n_surv;
+  __shared__ float sv[kSurvivorCap];
+  __shared__ int scn[kSurvivorCap];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t row = blockIdx.x;
+  const int64_t i = row % D.N_q, bg = row / D.N_q, g = bg % D.Hkv, b = bg / D.Hkv;
+  const int K = D.K;
+  const int64_t n = n_eligible(D.q_pos0 + i, D.S, D.W);
+  const float* sr = sigma + row * n_stride;
+  // 1. warp maxima
+  float mv = -INFINITY;
+  int mc = INT_MAX;
+  for (int64_t c = tid; c < n; c += kTopkThreads) {
+    const float v = sr[c];
+    if (better(v, (int)c, mv, mc)) { mv = v; mc = (int)c; }
+  }
+  warp_best(mv, mc);
+  if (lane == 0) { wv_sh[warp] = mv; wc_sh[warp] = mc; }
+  if (tid == 0) n_surv = 0;
+  __syncthreads();
+  // 2. theta = K-th best warp maximum (bitonic sort of 32 pairs, best first)
+  if (warp == 0) {
+    float v = wv_sh[lane];
+    int c = wc_sh[lane];
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        const bool up = ((lane & size) == 0);          // this 'size' block sorts best-first
+        const bool lower = ((lane & stride) == 0);     // lower index of the compared pair
+        cmpx(v, c, stride, up == lower);
+      }
+    }
+    const int kk = K < 32 ? K : 32;
+    const float tv = __shfl_sync(0xffffffffu, v, kk - 1);
+    const int tcc = __shfl_sync(0xffffffffu, c, kk - 1);
+    if (lane == 0) { th_v = tv; th_c = tcc; }
+  }
+  __syncthreads();
+  // 3. survivors: candidates not worse than theta
+  const float tv = th_v;
+  const int tcc = th_c;
+  for (int64_t c = tid; c < n; c += kTopkThreads) {
+    const float v = sr[c];
+    if (!better(tv, tcc, v, (int)c)) {
+      const int slot = atomicAdd(&n_surv, 1);
+      if (slot < kSurvivorCap) { sv[slot] = v; scn[slot] = (int)c; }
+    }
+  }
+  __syncthreads();
+  const int ns = n_surv;
+  if (warp != 0) return;
+  // 4. exact top-K of the survivors (or of every candidate if too many tied at theta)
+  TopList<KM> L;
+  L.clear();
+  if (ns <= kSurvivorCap) {
+    for (int e = lane; e < ns; e += 32) L.insert(sv[e], scn[e], K);
+  } else {
+    for (int64_t c = lane; c < n; c += 32) L.insert(sr[c], (int)c, K);
+  }
+  float wv;
+  int wc;
+  warp_merge_topk<KM>(L, K, lane, wv, wc);
+  write_selection<T, GM>(D, b, g, i, nullptr, qc, klm + bg * D.C * D.d, blm + bg * D.C, lane,
+                         wc, idx, s_sel);
+}
+
+template <typename T, int D_, int GM, int KM>
+struct TopkRowRun {
+  static cudaError_t run(const Dims* D, int64_t n_stride, const float* sigma, const void* qc,
+                         const void* klm, const float* blm, int32_t* idx, float* s_sel,
+                         cudaStream_t st) {
+    const int64_t rows = D->B * D->Hkv * D->N_q;
+    select_topk_row_kernel<T, GM, KM><<<(unsigned)rows, kTopkThreads, 0, st>>>(
+        *D, n_stride, sigma, (const T*)qc, (const T*)klm, blm, idx, s_sel);
+    return cudaGetLastError();
+  }
+};
+
 // ---------------------------------------------------------------------------------------------
 // Host-side launchers.
 
@@ -711,6 +924,14 @@ cudaError_t launch_select_topk(const Dims& D, int n_seg, int64_t n_stride, const
   else
     select_topk_kernel<32><<<grid, 256, 0, st>>>(D, n_stride, n_seg, sigma, part_v, part_c);
   return cudaGetLastError();
+}
+
+cudaError_t launch_select_topk_row(const Dims& D, bool bf16, int64_t n_stride,
+                                   const float* sigma, const void* qc, const void* klm,
+                                   const float* blm, int32_t* idx, float* s_sel, cudaStream_t st) {
+  if (D.B * D.Hkv * D.N_q == 0) return cudaSuccess;
+  return dispatch_tdgk<TopkRowRun>(bf16, D.d, D.G, D.K, &D, n_stride, sigma, qc, klm, blm, idx,
+                                   s_sel, st);
 }
 
 }  // namespace hils
