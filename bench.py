@@ -415,14 +415,11 @@ def run_hils(args):
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         step_ms, phase_ms = timed_steps(run, args.steps, flush, barrier)
-    total_ms = sum(step_ms)
-    if dist:
-        t = torch.tensor([total_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    from hierarchical_chunk_sparse_scoring_b200 import sharding
+    total_ms = sharding.max_over_ranks(sum(step_ms), device=device if dist else None)
     ms_per_step = total_ms / args.steps
     tokens_per_rank = wl.q.shape[0] * wl.q.shape[2]
-    value = tokens_per_rank * world / (ms_per_step * 1e-3)
+    value = sharding.aggregate_tokens_per_s(tokens_per_rank, ms_per_step, world)
     es = wl.q.element_size()
     wm = work_model(wl.dims, wl.S, wl.K_top, wl.W, wl.q_pos0, es)
     dom = max(phase_ms, key=phase_ms.get)
