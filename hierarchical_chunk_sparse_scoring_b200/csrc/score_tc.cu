@@ -45,7 +45,7 @@ struct TcShape {
   static constexpr int STASH_BYTES = (16 * 256 * 4) > (kRows * KM * 8) ? (16 * 256 * 4)
                                                                        : (kRows * KM * 8);
   static constexpr int FIXED = A_BYTES + STASH_BYTES + 1024 /*barriers*/ + 1024 /*align*/ +
-                               2048 /*shared thresholds*/;
+                               2048 /*shared thresholds*/ + 4 * NT * 4 /*bias tiles*/;
   static constexpr int STAGES_FIT = (kSmemLimit - FIXED) / B_STAGE;
   static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
   // more than half of the SM's shared memory, so a second CTA can never be co-resident and
@@ -79,7 +79,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                                SH::STASH_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + SH::STAGES;
-  uint64_t* a_full = bars + 2 * SH::STAGES;
+  uint64_t* bias_empty = bars + 2 * SH::STAGES;   // epilogue done with a stage's biases
+  uint64_t* a_full = bars + 3 * SH::STAGES;
   uint64_t* acc_full = a_full + 1;      // [2]
   uint64_t* acc_empty = acc_full + 2;   // [2]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
@@ -87,6 +88,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // same query in the other column half: [2 halves][128 rows]
   float* th_v = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 1024);
   int* th_c = reinterpret_cast<int*>(th_v + 2 * kRows);
+  // landmark biases of each stage's tile (bulk-copied with the landmark rows when aligned)
+  float* sbias = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 3072);
+  const bool bias_bulk = (D.C % 4) == 0 && (reinterpret_cast<uintptr_t>(blm) & 15) == 0;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t qt = (int64_t)gridDim.x - 1 - blockIdx.x;   // longest query tiles first
@@ -99,7 +103,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int K = D.K;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SH::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int s = 0; s < SH::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&bias_empty[s], 8);
+    }
     mbar_init(a_full, 1);
     for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], 8); }
     fence_barrier_init();
@@ -125,14 +133,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int t = 0; t < n_tiles; ++t) {
         const int s = t % SH::STAGES;
         const uint32_t u = (uint32_t)(t / SH::STAGES);
-        if (!mbar_wait(&empty[s], (u & 1u) ^ 1u, kPollLimit)) {
+        if (!mbar_wait(&empty[s], (u & 1u) ^ 1u, kPollLimit) ||
+            !mbar_wait(&bias_empty[s], (u & 1u) ^ 1u, kPollLimit)) {
           record_status(status, kStatusTimeout);
           break;
         }
-        mbar_expect_tx(&full[s], SH::B_STAGE);
+        const int64_t cb0 = (int64_t)t * NT;
+        const int brows = (int)(D.C - cb0 < NT ? D.C - cb0 : NT);
+        const uint32_t bias_bytes = bias_bulk ? (uint32_t)((brows + 3) / 4 * 16) : 0u;
+        mbar_expect_tx(&full[s], SH::B_STAGE + bias_bytes);
         for (int kb = 0; kb < SH::KB; ++kb)
           tma_load_2d(sB + s * SH::B_STAGE + kb * SH::B_BOX, &tmB, kb * 64,
-                      (int32_t)(bg * D.C + (int64_t)t * NT), &full[s]);
+                      (int32_t)(bg * D.C + cb0), &full[s]);
+        if (bias_bulk) bulk_load(sbias + s * NT, blm + bg * D.C + cb0, bias_bytes, &full[s]);
         last_s = s;
         last_par = u & 1u;
       }
@@ -187,28 +200,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     TailList<KM> L;
     L.clear(K);
     float thv = -INFINITY;
-    int thc = INT_MAX;
     th_v[ch * kRows + r] = -INFINITY;
-    th_c[ch * kRows + r] = INT_MAX;
     float* my_tv = th_v + ch * kRows + r;
-    int* my_tc = th_c + ch * kRows + r;
     const float* pa_tv = th_v + (1 - ch) * kRows + r;
-    const int* pa_tc = th_c + (1 - ch) * kRows + r;
     asm volatile("bar.sync 1, 256;" ::: "memory");   // thresholds initialised
     const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
     bool ok = true;
     for (int t = 0; t < n_tiles; ++t) {
       const int a = t & 1;
       const uint32_t v = (uint32_t)(t >> 1);
-      if (!mbar_wait_warp(&acc_full[a], v & 1u, kPollLimit)) { ok = false; break; }
+      const int bs = t % SH::STAGES;
+      const uint32_t bu = (uint32_t)(t / SH::STAGES);
+      // accumulators of tile t, and (for the biases) the stage's own completion
+      if (!mbar_wait_warp(&acc_full[a], v & 1u, kPollLimit) ||
+          !mbar_wait_warp(&full[bs], bu & 1u, kPollLimit)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll 1
       for (int sb = 0; sb < SH::HALF / 16; ++sb) {
         const int col0 = ch * SH::HALF + sb * 16;
         const int64_t c0 = (int64_t)t * NT + col0;
-        // landmark biases of these 16 chunks: one load per lane, then broadcast
-        const int64_t cb = c0 + (lane & 15);
-        const float bl = cb < n_max ? __ldg(bb + cb) : 0.f;
+        // landmark biases of these 16 chunks
+        float bl = 0.f;
+        if (!bias_bulk) {
+          const int64_t cb = c0 + (lane & 15);
+          bl = cb < n_max ? __ldg(bb + cb) : 0.f;
+        }
         float sig[16];
         constexpr int HG = G < 4 ? G : 4;     // heads whose TMEM loads are in flight together
 #pragma unroll
@@ -224,19 +240,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int j = 0; j < 16; ++j)
               sig[j] = (h0 + hh == 0) ? tmp[hh][j] : fmaxf(sig[j], tmp[hh][j]);
         }
-        // a candidate must beat both this list's K-th best and the other half's (either list
-        // already holds K candidates at least that good)
+        // a candidate must reach both this list's K-th best and the other half's (either list
+        // already holds K candidates at least that good); exact ties at the threshold are
+        // passed on and resolved by the insertion itself
         const float pv = *reinterpret_cast<const volatile float*>(pa_tv);
-        const int pc = *reinterpret_cast<const volatile int*>(pa_tc);
+        const float thr = fmaxf(thv, pv);
+        const int64_t left = n_i - c0;
+        const uint32_t vmask = left >= 16 ? 0xFFFFu : (left <= 0 ? 0u : (1u << left) - 1u);
+        const float* sbt = sbias + bs * NT + col0;
         uint32_t pass = 0;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const int64_t c = c0 + j;
-          const float bj = __shfl_sync(0xffffffffu, bl, j);
+          const float bj = bias_bulk ? sbt[j] : __shfl_sync(0xffffffffu, bl, j);
           sig[j] = fmaf(sig[j], D.scale, bj);
-          if (c < n_i && better(sig[j], (int)c, thv, thc) && better(sig[j], (int)c, pv, pc))
-            pass |= 1u << j;
+          pass |= (sig[j] >= thr ? 1u : 0u) << j;
         }
+        pass &= vmask;
         if (__any_sync(0xffffffffu, pass != 0)) {
 #pragma unroll
           for (int j = 0; j < 16; ++j) st[j * 256] = sig[j];
@@ -247,15 +266,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               L.insert(st[j * 256], (int)(c0 + j));
             }
             thv = L.kth_v();
-            thc = L.kth_c();
             *reinterpret_cast<volatile float*>(my_tv) = thv;
-            *reinterpret_cast<volatile int*>(my_tc) = thc;
           }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[a]);
+      if (lane == 0) {
+        mbar_arrive(&bias_empty[bs]);
+        mbar_arrive(&acc_empty[a]);
+      }
     }
     if (!ok) record_status(status, kStatusTimeout);
     // merge the two column halves' lists of each query
