@@ -165,8 +165,12 @@ int phase_names(const Plan& P, const char** names, int max_names) {
     for (int i = 0; i < 4 && i < max_names; ++i) names[i] = kDecode[i];
     return 4;
   }
-  if (P.tc_select) { pre[n++] = "score_topk_tc"; pre[n++] = "select_scores"; }
-  else pre[n++] = "select_rows";
+  if (P.tc_select) {
+    pre[n++] = "score_topk_tc";
+    if (!P.tc_attn) pre[n++] = "select_scores";
+  } else {
+    pre[n++] = "select_rows";
+  }
   pre[n++] = P.tc_attn ? "attn_tc" : "attn_rows";
   for (int i = 0; i < n && i < max_names; ++i) names[i] = pre[i];
   return n;
@@ -218,14 +222,17 @@ hils_status forward_impl(const hils_params* p, const void* q, const void* q_cal,
   } else {
     if (P.tc_select) {
       e = launch_score_topk_tc(P.D, q_cal, k_lm, b_lm, idx, reinterpret_cast<int32_t*>(ws), st);
-      pm.mark();
-      if (e == cudaSuccess) e = launch_select_scores(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
+      // the tensor-core attention computes the selected chunks' per-head scores itself
+      if (e == cudaSuccess && !P.tc_attn) {
+        pm.mark();
+        e = launch_select_scores(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
+      }
     } else {
       e = launch_select_rows(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
     }
     pm.mark();
     if (e == cudaSuccess)
-      e = P.tc_attn ? launch_attn_tc(P.D, q, K, V, idx, s_sel, out, lse_out,
+      e = P.tc_attn ? launch_attn_tc(P.D, q, q_cal, K, V, idx, k_lm, b_lm, out, lse_out,
                                      reinterpret_cast<int32_t*>(ws), st)
                     : launch_attn_rows(P.D, P.bf16, q, K, V, idx, s_sel, out, lse_out, nullptr,
                                        nullptr, st);

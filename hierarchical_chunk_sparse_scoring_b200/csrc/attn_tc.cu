@@ -49,10 +49,16 @@ struct AtShape {
   static constexpr int KV_BYTES = KB * KV_BOX;           // one K (or V) tile
   static constexpr int P_BYTES = kAtRows * 128;          // [128 rows x 64 tokens] bf16
   static constexpr int STAGES = DD == 128 ? 3 : 4;
-  static constexpr int FIXED = Q_BYTES + STAGES * 2 * KV_BYTES + 2 * P_BYTES + 1024 /*bars*/ +
-                               1024 /*align*/ + 1024 /*scan*/;
-  static constexpr uint32_t TMEM_COLS = 256;            // S[2] (2 x 64) + O (DD)
+  static constexpr int KLM_ROWS = 64;                    // landmark rows staged in smem
+  static constexpr int KLM_BYTES = KB * KLM_ROWS * 128;  // same swizzled layout as a K tile
+  static constexpr int FIXED = 2 * Q_BYTES /*q and q_cal*/ + STAGES * 2 * KV_BYTES +
+                               2 * P_BYTES + 1024 /*bars*/ + 1024 /*align*/ + 1024 /*scan*/;
+  static_assert(KLM_BYTES <= 2 * P_BYTES, "landmark rows overlay the P buffers");
+  static constexpr uint32_t TMEM_COLS = 512;            // S[2] (2 x 64) + O (DD) + landmark S
   static constexpr uint32_t O_COL = 128;
+  static constexpr uint32_t LM_COL = 256;
+  // 512 TMEM columns are the whole SM's: the shared memory footprint keeps a second CTA away
+  static_assert(FIXED > 232448 / 2, "one CTA per SM");
 };
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -99,9 +105,10 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int& to
 
 template <int DD, int G, int KM>
 __global__ void __launch_bounds__(kAtThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, Dims D,
-                   const int32_t* __restrict__ idx, const float* __restrict__ s_sel,
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQc,
+                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                   Dims D, const int32_t* __restrict__ idx, const __nv_bfloat16* __restrict__ klm,
+                   const float* __restrict__ blm,
                    __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out,
                    int list_cap, int bitmap_words, int32_t* __restrict__ status) {
   using SH = AtShape<DD, G>;
@@ -110,9 +117,13 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem;
-  uint8_t* sK = sQ + SH::Q_BYTES;
+  uint8_t* sQc = sQ + SH::Q_BYTES;   // calibrated queries (surrogate scores of the selection)
+  uint8_t* sK = sQc + SH::Q_BYTES;
   uint8_t* sV = sK + SH::STAGES * SH::KV_BYTES;
   uint8_t* sP = sV + SH::STAGES * SH::KV_BYTES;
+  // landmark rows of the first 64 tiles (K-tile layout); dead once their product has completed,
+  // before any P row is written
+  uint8_t* sKlm = sP;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * SH::P_BYTES);
   uint64_t* kv_full = bars;                       // [STAGES]
   uint64_t* kv_empty = bars + SH::STAGES;         // [STAGES]
@@ -123,7 +134,8 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   uint64_t* p_empty = p_full + 2;                 // [2]
   uint64_t* o_done = p_empty + 2;
   uint64_t* o_final = o_done + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(o_final + 1);
+  uint64_t* lm_done = o_final + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(lm_done + 1);
   int* scan = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + 1024);   // [64]
   int* n_tiles_sh = scan + 64;
   int* tiles = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + 2048);  // [list_cap]
@@ -152,6 +164,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     }
     mbar_init(o_done, 1);
     mbar_init(o_final, 1);
+    mbar_init(lm_done, 1);
     fence_barrier_init();
   }
   if (warp == 1) tmem_alloc(tmem_holder, SH::TMEM_COLS);
@@ -204,11 +217,14 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
-      mbar_expect_tx(q_full, SH::Q_BYTES);
+      prefetch_tensormap(&tmQc);
+      mbar_expect_tx(q_full, 2 * SH::Q_BYTES);
       for (int h = 0; h < G; ++h)
-        for (int kb = 0; kb < SH::KB; ++kb)
-          tma_load_2d(sQ + kb * SH::Q_BOX + h * TQ * 128, &tmQ, kb * 64,
-                      (int32_t)((b * D.Hq + g * G + h) * D.N_q + i0), q_full);
+        for (int kb = 0; kb < SH::KB; ++kb) {
+          const int32_t y = (int32_t)((b * D.Hq + g * G + h) * D.N_q + i0);
+          tma_load_2d(sQ + kb * SH::Q_BOX + h * TQ * 128, &tmQ, kb * 64, y, q_full);
+          tma_load_2d(sQc + kb * SH::Q_BOX + h * TQ * 128, &tmQc, kb * 64, y, q_full);
+        }
       int last_s = -1;
       uint32_t last_par = 0;
       for (int t = 0; t < n_tiles; ++t) {
@@ -292,13 +308,117 @@ __global__ void __launch_bounds__(kAtThreads, 1)
 #pragma unroll
     for (int k = 0; k < KM; ++k) {
       sc[k] = -1;
-      su[k] = -INFINITY;
-      if (valid && k < K) {
-        sc[k] = idx[(bg * D.N_q + i) * K + k];
-        su[k] = sc[k] >= 0 ? s_sel[hrow * K + k] : -INFINITY;
+      if (valid && k < K) sc[k] = idx[(bg * D.N_q + i) * K + k];
+    }
+    // This head's surrogate score of each selected chunk, q_cal . k_lm[c] * scale + b_lm[c].
+    // The landmark rows of the first 64 tiles of the (sorted) tile list are staged in shared
+    // memory in the K-tile layout and one (128 x d) x (d x 64) product on the tensor core scores
+    // every row of the tile against them; a chunk beyond those 64 is scored by a plain dot.
+    const int nk = n_tiles < SH::KLM_ROWS ? n_tiles : SH::KLM_ROWS;
+    int slot[KM];
+    float bsel[KM];
+#pragma unroll
+    for (int k = 0; k < KM; ++k) {
+      int lo = 0, hi = nk;   // first tile >= c in [0, nk)
+      const int c = sc[k];
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (tiles[mid] < c) lo = mid + 1; else hi = mid;
+      }
+      slot[k] = (c >= 0 && lo < nk && tiles[lo] == c) ? lo : -1;
+      bsel[k] = (c >= 0 && c < D.C) ? __ldg(blm + bg * D.C + c) : 0.f;
+    }
+    {
+      constexpr int UPR = DD / 8;   // 16-byte units per landmark row
+      const int tid = threadIdx.x - 64;
+      uint4 u[SH::KLM_ROWS * UPR / 128];
+#pragma unroll
+      for (int e = 0; e < SH::KLM_ROWS * UPR / 128; ++e) {
+        const int f = tid + e * 128, t = f / UPR, j = f - t * UPR;
+        const int c = t < nk ? tiles[t] : D.C;
+        u[e] = c < D.C ? __ldg(reinterpret_cast<const uint4*>(klm + (bg * D.C + c) * DD) + j)
+                       : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int e = 0; e < SH::KLM_ROWS * UPR / 128; ++e) {
+        const int f = tid + e * 128, t = f / UPR, j = f - t * UPR;
+        const int kb = j >> 3, jj = j & 7;
+        *reinterpret_cast<uint4*>(sKlm + kb * SH::KV_BOX + (t >> 3) * 1024 + (t & 7) * 128 +
+                                  ((jj ^ (t & 7)) << 4)) = u[e];
+      }
+      fence_async_smem();
+      asm volatile("bar.sync 1, 128;" ::: "memory");   // the four softmax warps
+    }
+    const bool q_ok = mbar_wait_warp(q_full, 0, kAtPollLimit);
+    if (warp == 2 && lane == 0 && q_ok) {
+      tc_fence_after();
+      constexpr uint32_t IDESC_LM = idesc_bf16_f32(kAtRows, SH::KLM_ROWS);
+#pragma unroll
+      for (int ks = 0; ks < DD / 16; ++ks) {
+        const int kb = ks >> 2, kin = ks & 3;
+        const uint64_t ad = desc_kmajor_sw128(smem_u32(sQc + kb * SH::Q_BOX) + kin * 32);
+        const uint64_t bd = desc_kmajor_sw128(smem_u32(sKlm + kb * SH::KV_BOX) + kin * 32);
+        mma_bf16_ss(tmem + SH::LM_COL, ad, bd, IDESC_LM, ks > 0 ? 1u : 0u);
+      }
+      mma_commit(lm_done);
+    }
+    const bool lm_ok = q_ok && mbar_wait_warp(lm_done, 0, kAtPollLimit);
+    {
+      // the row's 64 landmark scores, parked in this thread's own P rows of both buffers (the
+      // staged landmark rows there are dead: their product completed), 16-byte slots rotated
+      uint8_t* park = sP + r * 128;
+      if (lm_ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int part = 0; part < 4; ++part) {
+          float vv[16];
+          tmem_ld16(tmem + ((uint32_t)(qd * 32) << 16) + SH::LM_COL + part * 16, vv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int col4 = part * 4 + q4;   // 4-column group 0..15
+            *reinterpret_cast<float4*>(park + (col4 >> 3) * SH::P_BYTES +
+                                       (((col4 & 7) + r) & 7) * 16) =
+                make_float4(vv[q4 * 4], vv[q4 * 4 + 1], vv[q4 * 4 + 2], vv[q4 * 4 + 3]);
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < KM; ++k) {
+        su[k] = -INFINITY;
+        const int c = sc[k];
+        if (!lm_ok || c < 0 || c >= D.C) continue;
+        float a;
+        if (slot[k] >= 0) {
+          const int col4 = slot[k] >> 2;
+          a = *reinterpret_cast<const float*>(park + (col4 >> 3) * SH::P_BYTES +
+                                              (((col4 & 7) + r) & 7) * 16 + (slot[k] & 3) * 4);
+        } else {
+          const __nv_bfloat16* kr = klm + (bg * D.C + c) * DD;
+          a = 0.f;
+#pragma unroll
+          for (int kb = 0; kb < SH::KB; ++kb) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const uint4 qv = *reinterpret_cast<const uint4*>(
+                  sQc + kb * SH::Q_BOX + (r >> 3) * 1024 + (r & 7) * 128 + ((j ^ (r & 7)) << 4));
+              const uint4 kv = __ldg(reinterpret_cast<const uint4*>(kr + kb * 64 + j * 8));
+              a = fmaf(bf16_lo(qv.x), bf16_lo(kv.x), a);
+              a = fmaf(bf16_hi(qv.x), bf16_hi(kv.x), a);
+              a = fmaf(bf16_lo(qv.y), bf16_lo(kv.y), a);
+              a = fmaf(bf16_hi(qv.y), bf16_hi(kv.y), a);
+              a = fmaf(bf16_lo(qv.z), bf16_lo(kv.z), a);
+              a = fmaf(bf16_hi(qv.z), bf16_hi(kv.z), a);
+              a = fmaf(bf16_lo(qv.w), bf16_lo(kv.w), a);
+              a = fmaf(bf16_hi(qv.w), bf16_hi(kv.w), a);
+            }
+          }
+        }
+        su[k] = fmaf(a, D.scale, bsel[k]);
         m_run = fmaxf(m_run, su[k]);
       }
     }
+    if (!lm_ok) record_status(status, kStatusTimeout);
     float l = 0.f;
     const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
     uint8_t* prow_base = sP + (r >> 3) * 1024 + (r & 7) * 128;
@@ -491,12 +611,13 @@ int list_capacity(const Dims& D, int TQ) {
 }
 
 template <int DD, int G, int KM>
-cudaError_t launch_at_t(const Dims& D, const void* q, const void* K, const void* V,
-                        const int32_t* idx, const float* s_sel, void* out, float* lse,
-                        int32_t* status, cudaStream_t st) {
+cudaError_t launch_at_t(const Dims& D, const void* q, const void* qc, const void* K,
+                        const void* V, const int32_t* idx, const void* klm, const float* blm,
+                        void* out, float* lse, int32_t* status, cudaStream_t st) {
   using SH = AtShape<DD, G>;
-  CUtensorMap tmQ, tmK, tmV;
+  CUtensorMap tmQ, tmQc, tmK, tmV;
   if (!make_map_at(&tmQ, q, (uint64_t)(D.B * D.Hq * D.N_q), DD, SH::TQ) ||
+      !make_map_at(&tmQc, qc, (uint64_t)(D.B * D.Hq * D.N_q), DD, SH::TQ) ||
       !make_map_at(&tmK, K, (uint64_t)(D.B * D.Hkv * D.N_kv), DD, kTile) ||
       !make_map_at(&tmV, V, (uint64_t)(D.B * D.Hkv * D.N_kv), DD, kTile))
     return cudaErrorInvalidValue;
@@ -508,17 +629,19 @@ cudaError_t launch_at_t(const Dims& D, const void* q, const void* K, const void*
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((D.N_q + SH::TQ - 1) / SH::TQ), (unsigned)(D.B * D.Hkv));
-  kern<<<grid, kAtThreads, smem, st>>>(tmQ, tmK, tmV, D, idx, s_sel, (__nv_bfloat16*)out, lse,
+  kern<<<grid, kAtThreads, smem, st>>>(tmQ, tmQc, tmK, tmV, D, idx,
+                                       (const __nv_bfloat16*)klm, blm, (__nv_bfloat16*)out, lse,
                                        cap, words, status);
   return cudaGetLastError();
 }
 
 template <int DD, int G>
-cudaError_t launch_at_k(const Dims& D, const void* q, const void* K, const void* V,
-                        const int32_t* idx, const float* s_sel, void* out, float* lse,
-                        int32_t* status, cudaStream_t st) {
-  if (D.K <= 16) return launch_at_t<DD, G, 16>(D, q, K, V, idx, s_sel, out, lse, status, st);
-  return launch_at_t<DD, G, 32>(D, q, K, V, idx, s_sel, out, lse, status, st);
+cudaError_t launch_at_k(const Dims& D, const void* q, const void* qc, const void* K,
+                        const void* V, const int32_t* idx, const void* klm, const float* blm,
+                        void* out, float* lse, int32_t* status, cudaStream_t st) {
+  if (D.K <= 16)
+    return launch_at_t<DD, G, 16>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st);
+  return launch_at_t<DD, G, 32>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st);
 }
 
 }  // namespace
@@ -532,14 +655,16 @@ bool attn_tc_supported(const Dims& D, bool bf16) {
   const int64_t cap = (int64_t)TQ * D.K + (D.W + kTile + TQ) / kTile + 4;
   const int64_t words = (D.N_kv / kTile) / 32 + 2;
   const int fixed = D.d == 128 ? AtShape<128, 1>::FIXED : AtShape<64, 1>::FIXED;
+  if (D.C >= (int64_t)INT32_MAX) return false;
   return fixed + 1024 + (cap + words) * 4 <= kAtSmemLimit;
 }
 
-cudaError_t launch_attn_tc(const Dims& D, const void* q, const void* K, const void* V,
-                           const int32_t* idx, const float* s_sel, void* out, float* lse,
-                           int32_t* status, cudaStream_t st) {
+cudaError_t launch_attn_tc(const Dims& D, const void* q, const void* qc, const void* K,
+                           const void* V, const int32_t* idx, const void* klm, const float* blm,
+                           void* out, float* lse, int32_t* status, cudaStream_t st) {
   if (D.B * D.Hq * D.N_q == 0) return cudaSuccess;
-#define HILS_AT(DD, GG) return launch_at_k<DD, GG>(D, q, K, V, idx, s_sel, out, lse, status, st)
+#define HILS_AT(DD, GG) \
+  return launch_at_k<DD, GG>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st)
   if (D.d == 128) {
     if (D.G == 1) HILS_AT(128, 1);
     if (D.G == 2) HILS_AT(128, 2);

@@ -157,6 +157,25 @@ struct TailList {
     }
   }
 
+  // Insertion for a candidate from the thread's own chunk stream: every entry already in the
+  // list came earlier in that stream (lower chunk index), so an equal value never moves ahead of
+  // one and a strict value compare gives the same order as `better`.  -inf is clamped to the
+  // lowest finite value so it still fills an empty (-inf) slot.
+  __device__ __forceinline__ void insert_stream(float x, int ci) {
+    x = fmaxf(x, -FLT_MAX);
+    bool m[KM];
+#pragma unroll
+    for (int k = 0; k < KM; ++k) m[k] = x > v[k];
+#pragma unroll
+    for (int k = KM - 1; k >= 0; --k) {
+      if (m[k]) {
+        const bool shift = k > 0 && m[k - 1];
+        v[k] = shift ? v[k - 1] : x;
+        c[k] = shift ? c[k - 1] : ci;
+      }
+    }
+  }
+
   __device__ __forceinline__ float kth_v() const { return v[KM - 1]; }
   __device__ __forceinline__ int kth_c() const { return c[KM - 1]; }
 };

@@ -22,9 +22,9 @@ cudaError_t launch_score_topk_tc(const Dims& D, const void* qc, const void* klm,
                                  cudaStream_t st);
 
 bool attn_tc_supported(const Dims& D, bool bf16);
-cudaError_t launch_attn_tc(const Dims& D, const void* q, const void* K, const void* V,
-                           const int32_t* idx, const float* s_sel, void* out, float* lse,
-                           int32_t* status, cudaStream_t st);
+cudaError_t launch_attn_tc(const Dims& D, const void* q, const void* qc, const void* K,
+                           const void* V, const int32_t* idx, const void* klm, const float* blm,
+                           void* out, float* lse, int32_t* status, cudaStream_t st);
 
 size_t split_smem_bytes(int cps);
 cudaError_t launch_select_split(const Dims& D, bool bf16, int cps, int n_split, const void* qc,

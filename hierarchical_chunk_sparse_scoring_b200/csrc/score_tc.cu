@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             while (pass) {
               const int j = __ffs(pass) - 1;
               pass &= pass - 1;
-              L.insert(st[j * 256], (int)(c0 + j));
+              L.insert_stream(st[j * 256], (int)(c0 + j));
             }
             thv = L.kth_v();
             *reinterpret_cast<volatile float*>(my_tv) = thv;
