@@ -24,6 +24,7 @@ import json
 import math
 import os
 import statistics
+import threading
 import subprocess
 import sys
 import time
@@ -95,7 +96,7 @@ def phase_work(name, wm):
     return "hbm", None, "GB/s"
 
 
-def roofline(name, ms, wm, peaks, sustained=False):
+def roofline(name, ms, wm, peaks, workload, sustained=False):
     bound, work, unit = phase_work(name, wm)
     if work is None or ms <= 0:
         return None
@@ -106,78 +107,103 @@ def roofline(name, ms, wm, peaks, sustained=False):
         achieved = work / (ms * 1e-3) / 1e12
         peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
     return {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-            "frac": achieved / peak, "traffic": traffic_for(name), "work_per_launch": work}
+            "frac": achieved / peak, "traffic": traffic_for(name, workload), "work_per_launch": work}
 
 
-def traffic_for(kernel):
-    """dram read+write bytes per launch from the committed ncu summary, if it was taken on the
-    current source of that kernel; else None."""
+KERNEL_SOURCES = {
+    "score_topk_tc": ["score_tc.cu"], "attn_tc": ["attn_tc.cu"],
+    "select_stream": ["select.cu"], "select_topk": ["select.cu"], "select_rows": ["select.cu"],
+    "select_split": ["select.cu"], "attn_units": ["attn.cu"], "attn_rows": ["attn.cu"],
+    "fuse_units": ["attn.cu"],
+}
+SHARED_SOURCES = ["common.cuh", "sm100.cuh"]
+
+
+def source_sha(kernel):
+    """Hash of the CUDA sources a kernel is built from (its file and the shared headers)."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "hierarchical_chunk_sparse_scoring_b200", "csrc")
+    for f in KERNEL_SOURCES.get(kernel, []) + SHARED_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel, workload):
+    """DRAM read+write bytes per launch of `kernel` on `workload`, from the committed ncu
+    summaries (profiles/traffic.json), if they were taken on the kernel's current source;
+    else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            rec = json.load(f).get(kernel)
+            rec = json.load(f).get("%s@%s" % (kernel, workload))
+        if not rec or kernel not in KERNEL_SOURCES:
+            return None
+        return rec["bytes_per_launch"] if rec.get("source_sha") == source_sha(kernel) else None
     except Exception:
         return None
-    if not rec:
-        return None
-    src = os.path.join(ROOT, rec["source"])
-    try:
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    except OSError:
-        return None
-    return rec["bytes_per_launch"] if sha == rec.get("source_sha") else None
 
 
 # --------------------------------------------------------------------------- clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons of one GPU, polled through NVML from a thread while the
+    timed region runs (read-only queries; no setting is touched)."""
+    REASONS = (("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20),
+               ("hw_thermal_slowdown", 0x40), ("sw_power_cap", 0x4))
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+    def __init__(self, cuda_index):
+        self.cuda_index = cuda_index
+        self.rows = []
+        self.max_mhz = None
+        self.err = None
+        self._stop = threading.Event()
+        self._thread = None
+
+    def _handle(self, nv):
+        try:
+            pr = torch.cuda.get_device_properties(self.cuda_index)
+            bus = "%08x:%02x:%02x.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+            return nv.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.cuda_index)
+
+    def _poll(self, nv, h):
+        reasons_fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while True:
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                bits = reasons_fn(h)
+                self.rows.append((float(mhz), int(bits)))
+            except Exception as e:       # keep whatever was sampled
+                self.err = repr(e)
+                return
+            if self._stop.wait(0.001):
+                return
 
     def __enter__(self):
         try:
-            self.path = "/tmp/hils_clocks_%d_%d.csv" % (os.getpid(), self.gpu)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
-                stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self._thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+            self._thread.start()
+        except Exception as e:
+            self.err = repr(e)
         return self
 
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-            self.f.close()
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
 
     def summary(self):
-        if self.proc is None or not self.path:
+        if not self.rows:
             return None
-        rows = []
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
-            except ValueError:
-                continue
-        if not rows:
-            return None
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[k] for _, _, r in rows for k in range(4) if r[k] == "Active"})
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": rows[0][1],
-                "reasons": reasons, "samples": len(rows)}
+        reasons = sorted({name for _, bits in self.rows for name, m in self.REASONS if bits & m})
+        return {"sm_mhz": statistics.median(r[0] for r in self.rows), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.rows), "source": "nvml"}
 
 
 # --------------------------------------------------------------------------- timing
@@ -338,7 +364,7 @@ def extra_prefill(name, steps, peaks, **overrides):
     t = statistics.mean(step_ms)
     res = {"workload": name, "ms_per_step": t, "tokens_per_s": wm["tokens"] / (t * 1e-3),
            "phases_ms": phase_ms,
-           "rooflines": [roofline(k, v, wm, peaks) for k, v in phase_ms.items()],
+           "rooflines": [roofline(k, v, wm, peaks, name) for k, v in phase_ms.items()],
            "score_tflop": wm["score_flops"] / 1e12, "attn_tflop": wm["attn_flops"] / 1e12}
     del run, wl
     torch.cuda.empty_cache()
@@ -384,7 +410,7 @@ def extra_decode(steps, peaks, **overrides):
            "step_roofline": {"bound": "hbm", "achieved": total_bytes / (t_us * 1e-6) / 1e9,
                              "peak": peaks["hbm_gbs"], "unit": "GB/s",
                              "frac": total_bytes / (t_us * 1e-6) / 1e9 / peaks["hbm_gbs"]},
-           "rooflines": [roofline(k, v, wm, peaks) for k, v in phase_ms.items()]}
+           "rooflines": [roofline(k, v, wm, peaks, "long_decode") for k, v in phase_ms.items()]}
     del g, run, wl
     torch.cuda.empty_cache()
     return res
@@ -430,7 +456,7 @@ def run_hils(args):
         "dtype": "bf16" if wl.q.dtype == torch.bfloat16 else "f32",
         "data": "synthetic (seeded generator, hierarchical_chunk_sparse_scoring_b200/workloads.py)",
         "config": config_of(wl, world),
-        "roofline": roofline(dom, phase_ms[dom], wm, peaks),
+        "roofline": roofline(dom, phase_ms[dom], wm, peaks, wl.name),
         "peaks_source": peaks_src,
         "phases_ms": phase_ms,
         "gpu_launches": len(run.phases) * args.steps,

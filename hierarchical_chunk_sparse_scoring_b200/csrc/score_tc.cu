@@ -8,15 +8,15 @@
 // heads ([Reader] GQA paragraph) and a streaming top-K with ties to the lower chunk index
 // ([Reader] "Limitations of Naive Sparse Attention").  No score is written to memory.
 //
-// CTA = one (b, g) and 128 consecutive queries; 10 warps:
+// CTA = one (b, g) and 128 consecutive queries; 2 + 4*NCG warps:
 //   warp 0     TMA producer: the G calibrated-query tiles once, then the landmark tiles
 //              through a ring of shared-memory stages;
 //   warp 1     allocates 512 TMEM columns (two accumulator sets of G x NT columns) and issues
 //              tcgen05.mma from one thread;
-//   warps 2-9  epilogue: warp w reads TMEM lanes 32*(w%4).. (its 32 queries) and one half of
-//              each tile's columns, so every query has two partial top-K lists, merged at the
-//              end.  Candidates that beat a thread's current K-th best are inserted into its
-//              sorted register list.
+//   warps 2..  epilogue: warp w reads TMEM lanes 32*(w%4).. (its 32 queries) and one of NCG
+//              column groups of each tile, so every query has NCG partial top-K lists, merged
+//              pairwise at the end.  Candidates that reach the best of the NCG lists' current
+//              K-th values are inserted into the thread's sorted register list.
 // Every mbarrier wait gives up after a bounded number of polls and records HILS_ERR_TIMEOUT.
 #include <cudaTypedefs.h>
 
@@ -29,21 +29,30 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kTcThreads = 320;
 constexpr int kRows = 128;
+
+// max of three floats in one instruction (sm_100 three-input max)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 constexpr uint32_t kPollLimit = 1u << 24;
 constexpr int kSmemLimit = 227 * 1024;
 
-template <int DD, int G, int KM>
+template <int DD, int G, int KM, int NCG>
 struct TcShape {
+  static constexpr int THREADS = 64 + 128 * NCG;
+  static constexpr int EPI = 128 * NCG;                       // epilogue threads
   static constexpr int NT = 256 / G < 256 ? 256 / G : 256;   // chunks per tile
   static constexpr int KB = DD / 64;                          // 128-byte boxes along d
   static constexpr int A_BOX = kRows * 128;
   static constexpr int A_BYTES = G * KB * A_BOX;
   static constexpr int B_BOX = NT * 128;
   static constexpr int B_STAGE = KB * B_BOX;
-  static constexpr int STASH_BYTES = (16 * 256 * 4) > (kRows * KM * 8) ? (16 * 256 * 4)
-                                                                       : (kRows * KM * 8);
+  static constexpr int STASH_A = 16 * EPI * 4;                  // 16 scores per thread
+  static constexpr int STASH_B = (NCG / 2) * kRows * KM * 8;     // lists in one merge round
+  static constexpr int STASH_BYTES = STASH_A > STASH_B ? STASH_A : STASH_B;
   static constexpr int FIXED = A_BYTES + STASH_BYTES + 1024 /*barriers*/ + 1024 /*align*/ +
                                2048 /*shared thresholds*/ + 4 * NT * 4 /*bias tiles*/;
   static constexpr int STAGES_FIT = (kSmemLimit - FIXED) / B_STAGE;
@@ -52,22 +61,24 @@ struct TcShape {
   // compete for the 512 TMEM columns this CTA allocates
   static constexpr int SMEM_USED = FIXED + STAGES * B_STAGE;
   static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
-  static constexpr int HALF = NT / 2;                          // columns per epilogue warp
+  static constexpr int CG = NT / NCG;                          // columns per epilogue warp
+  static constexpr int HG = G < 4 ? G : 4;   // heads whose TMEM loads are in flight together
   static constexpr uint32_t TMEM_COLS = 2 * G * NT;
   static_assert(TMEM_COLS == 512, "two accumulator sets fill TMEM");
   static_assert(STAGES >= 2, "shared memory too small for this shape");
-  static_assert(HALF % 16 == 0, "sub-blocks of 16 columns");
+  static_assert(CG % 16 == 0, "sub-blocks of 16 columns");
+  static_assert(NCG == 2 || NCG == 4, "two or four column groups");
 };
 
 }  // namespace
 
-template <int DD, int G, int KM>
-__global__ void __launch_bounds__(kTcThreads, 1)
+template <int DD, int G, int KM, int NCG>
+__global__ void __launch_bounds__(64 + 128 * NCG, 1)
     score_topk_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB, Dims D,
                          const float* __restrict__ blm, int32_t* __restrict__ idx,
                          int32_t* __restrict__ status) {
-  using SH = TcShape<DD, G, KM>;
+  using SH = TcShape<DD, G, KM, NCG>;
   constexpr int NT = SH::NT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -84,10 +95,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* acc_full = a_full + 1;      // [2]
   uint64_t* acc_empty = acc_full + 2;   // [2]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
-  // each epilogue thread's current K-th best (value, chunk), read by the thread serving the
-  // same query in the other column half: [2 halves][128 rows]
+  // each epilogue thread's current K-th best value, read by the threads serving the same query
+  // in the other column groups: [NCG groups][128 rows]
   float* th_v = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 1024);
-  int* th_c = reinterpret_cast<int*>(th_v + 2 * kRows);
   // landmark biases of each stage's tile (bulk-copied with the landmark rows when aligned)
   float* sbias = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 3072);
   const bool bias_bulk = (D.C % 4) == 0 && (reinterpret_cast<uintptr_t>(blm) & 15) == 0;
@@ -106,10 +116,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int s = 0; s < SH::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&bias_empty[s], 8);
+      mbar_init(&bias_empty[s], 4 * NCG);
     }
     mbar_init(a_full, 1);
-    for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], 8); }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4 * NCG);
+    }
     fence_barrier_init();
   }
   if (warp == 1) tmem_alloc(tmem_holder, SH::TMEM_COLS);
@@ -188,22 +201,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int e = warp - 2;                 // 0..7
+    const int e = warp - 2;                 // 0 .. 4*NCG-1
     const int qd = warp & 3;                // TMEM lane quadrant this warp may access
-    const int ch = e >> 2;                  // which half of each tile's columns
+    const int ch = e >> 2;                  // which column group of each tile
     const int r = qd * 32 + lane;           // query row within the tile
     const int64_t i = i0 + r;
     const bool valid = i < D.N_q;
     const int64_t n_i = valid ? n_eligible(D.q_pos0 + i, D.S, D.W) : 0;
     const float* bb = blm + bg * D.C;
-    float* st = stash + e * 32 + lane;      // stash[j * 256 + thread]
+    float* st = stash + e * 32 + lane;      // stash[j * EPI + thread]
     TailList<KM> L;
     L.clear(K);
     float thv = -INFINITY;
     th_v[ch * kRows + r] = -INFINITY;
     float* my_tv = th_v + ch * kRows + r;
-    const float* pa_tv = th_v + (1 - ch) * kRows + r;
-    asm volatile("bar.sync 1, 256;" ::: "memory");   // thresholds initialised
+    asm volatile("bar.sync 1, %0;" ::"n"(SH::EPI) : "memory");   // thresholds initialised
     const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
     bool ok = true;
     for (int t = 0; t < n_tiles; ++t) {
@@ -216,8 +228,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           !mbar_wait_warp(&full[bs], bu & 1u, kPollLimit)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll 1
-      for (int sb = 0; sb < SH::HALF / 16; ++sb) {
-        const int col0 = ch * SH::HALF + sb * 16;
+      for (int sb = 0; sb < SH::CG / 16; ++sb) {
+        const int col0 = ch * SH::CG + sb * 16;
         const int64_t c0 = (int64_t)t * NT + col0;
         // landmark biases of these 16 chunks
         float bl = 0.f;
@@ -226,7 +238,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           bl = cb < n_max ? __ldg(bb + cb) : 0.f;
         }
         float sig[16];
-        constexpr int HG = G < 4 ? G : 4;     // heads whose TMEM loads are in flight together
+        constexpr int HG = SH::HG;
 #pragma unroll
         for (int h0 = 0; h0 < G; h0 += HG) {
           float tmp[HG][16];
@@ -235,35 +247,59 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tmem_ld16(lane_base + (uint32_t)((a * G + h0 + hh) * NT + col0), tmp[hh]);
           tmem_wait_ld();
 #pragma unroll
-          for (int hh = 0; hh < HG; ++hh)
+          for (int j = 0; j < 16; ++j) {
+            // group max over the heads, two new heads per three-input max
+            int hh = 0;
+            if (h0 == 0) { sig[j] = tmp[0][j]; hh = 1; }
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              sig[j] = (h0 + hh == 0) ? tmp[hh][j] : fmaxf(sig[j], tmp[hh][j]);
+            for (; hh + 1 < HG; hh += 2) sig[j] = fmax3(sig[j], tmp[hh][j], tmp[hh + 1][j]);
+            if (hh < HG) sig[j] = fmaxf(sig[j], tmp[hh][j]);
+          }
         }
-        // a candidate must reach both this list's K-th best and the other half's (either list
-        // already holds K candidates at least that good); exact ties at the threshold are
-        // passed on and resolved by the insertion itself
-        const float pv = *reinterpret_cast<const volatile float*>(pa_tv);
-        const float thr = fmaxf(thv, pv);
+        // a candidate must reach every group's current K-th best (each list already holds K
+        // candidates at least that good); exact ties at the threshold are passed on and
+        // resolved by the insertion itself
+        float thr = thv;
+#pragma unroll
+        for (int o = 1; o < NCG; ++o)
+          thr = fmaxf(thr, *reinterpret_cast<const volatile float*>(
+                               th_v + ((ch + o) & (NCG - 1)) * kRows + r));
         const int64_t left = n_i - c0;
         const uint32_t vmask = left >= 16 ? 0xFFFFu : (left <= 0 ? 0u : (1u << left) - 1u);
-        const float* sbt = sbias + bs * NT + col0;
-        uint32_t pass = 0;
+        const float4* sbt = reinterpret_cast<const float4*>(sbias + bs * NT + col0);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float bj = bias_bulk ? sbt[j] : __shfl_sync(0xffffffffu, bl, j);
-          sig[j] = fmaf(sig[j], D.scale, bj);
-          pass |= (sig[j] >= thr ? 1u : 0u) << j;
+        for (int j4 = 0; j4 < 4; ++j4) {
+          float4 b4;
+          if (bias_bulk) {
+            b4 = sbt[j4];
+          } else {
+            b4.x = __shfl_sync(0xffffffffu, bl, 4 * j4);
+            b4.y = __shfl_sync(0xffffffffu, bl, 4 * j4 + 1);
+            b4.z = __shfl_sync(0xffffffffu, bl, 4 * j4 + 2);
+            b4.w = __shfl_sync(0xffffffffu, bl, 4 * j4 + 3);
+          }
+          sig[4 * j4] = fmaf(sig[4 * j4], D.scale, b4.x);
+          sig[4 * j4 + 1] = fmaf(sig[4 * j4 + 1], D.scale, b4.y);
+          sig[4 * j4 + 2] = fmaf(sig[4 * j4 + 2], D.scale, b4.z);
+          sig[4 * j4 + 3] = fmaf(sig[4 * j4 + 3], D.scale, b4.w);
         }
-        pass &= vmask;
-        if (__any_sync(0xffffffffu, pass != 0)) {
+        // the sub-block's best score decides whether any candidate can pass
+        const float m01 = fmax3(sig[0], sig[1], sig[2]), m02 = fmax3(sig[3], sig[4], sig[5]);
+        const float m03 = fmax3(sig[6], sig[7], sig[8]), m04 = fmax3(sig[9], sig[10], sig[11]);
+        const float m05 = fmax3(sig[12], sig[13], sig[14]);
+        const float mx = fmaxf(fmax3(m01, m02, m03), fmax3(m04, m05, sig[15]));
+        if (__any_sync(0xffffffffu, mx >= thr && vmask != 0u)) {
+          uint32_t pass = 0;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) st[j * 256] = sig[j];
+          for (int j = 0; j < 16; ++j) pass |= (sig[j] >= thr ? 1u : 0u) << j;
+          pass &= vmask;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) st[j * SH::EPI] = sig[j];
           if (pass) {
             while (pass) {
               const int j = __ffs(pass) - 1;
               pass &= pass - 1;
-              L.insert_stream(st[j * 256], (int)(c0 + j));
+              L.insert_stream(st[j * SH::EPI], (int)(c0 + j));
             }
             thv = L.kth_v();
             *reinterpret_cast<volatile float*>(my_tv) = thv;
@@ -278,21 +314,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     }
     if (!ok) record_status(status, kStatusTimeout);
-    // merge the two column halves' lists of each query
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    float* xv = stash;                                           // [128][KM]
-    int* xc = reinterpret_cast<int*>(stash + kRows * KM);        // [128][KM]
-    if (ch == 1) {
+    // merge the column groups' lists of each query pairwise: in each round the upper half of
+    // the remaining groups hands its lists to the lower half
+    float* xv = stash;                                                   // [NCG/2][128][KM]
+    int* xc = reinterpret_cast<int*>(stash + (NCG / 2) * kRows * KM);   // [NCG/2][128][KM]
 #pragma unroll
-      for (int k = 0; k < KM; ++k) { xv[r * KM + k] = L.v[k]; xc[r * KM + k] = L.c[k]; }
-    }
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    if (ch == 0 && valid) {
-      // the partner's live entries are its last K slots
-      for (int k = KM - K; k < KM; ++k) {
-        const int c = xc[r * KM + k];
-        if (c != INT_MAX) L.insert(xv[r * KM + k], c);
+    for (int half = NCG / 2; half >= 1; half >>= 1) {
+      asm volatile("bar.sync 1, %0;" ::"n"(SH::EPI) : "memory");
+      if (ch >= half && ch < 2 * half) {
+        const int o = ((ch - half) * kRows + r) * KM;
+#pragma unroll
+        for (int k = 0; k < KM; ++k) { xv[o + k] = L.v[k]; xc[o + k] = L.c[k]; }
       }
+      asm volatile("bar.sync 1, %0;" ::"n"(SH::EPI) : "memory");
+      if (ch < half) {
+        // the partner's live entries are its last K slots
+        const int o = (ch * kRows + r) * KM;
+        for (int k = KM - K; k < KM; ++k) {
+          const int c = xc[o + k];
+          if (c != INT_MAX) L.insert(xv[o + k], c);
+        }
+      }
+    }
+    if (ch == 0 && valid) {
       int32_t* out = idx + (bg * D.N_q + i) * K - (KM - K);
 #pragma unroll
       for (int k = 0; k < KM; ++k)
@@ -336,28 +380,30 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t d, uin
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int DD, int G, int KM>
+template <int DD, int G, int KM, int NCG>
 cudaError_t launch_tc_t(const Dims& D, const void* qc, const void* klm, const float* blm,
                         int32_t* idx, int32_t* status, cudaStream_t st) {
-  using SH = TcShape<DD, G, KM>;
+  using SH = TcShape<DD, G, KM, NCG>;
   CUtensorMap tmA, tmB;
   if (!make_map(&tmA, qc, (uint64_t)(D.B * D.Hq * D.N_q), DD, kRows) ||
       !make_map(&tmB, klm, (uint64_t)(D.B * D.Hkv * (D.C > 0 ? D.C : 1)), DD, SH::NT))
     return cudaErrorInvalidValue;
-  auto kern = score_topk_tc_kernel<DD, G, KM>;
+  auto kern = score_topk_tc_kernel<DD, G, KM, NCG>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SH::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((D.N_q + kRows - 1) / kRows), (unsigned)(D.B * D.Hkv));
-  kern<<<grid, kTcThreads, SH::SMEM, st>>>(tmA, tmB, D, blm, idx, status);
+  kern<<<grid, SH::THREADS, SH::SMEM, st>>>(tmA, tmB, D, blm, idx, status);
   return cudaGetLastError();
 }
 
 template <int DD, int G>
 cudaError_t launch_tc_k(const Dims& D, const void* qc, const void* klm, const float* blm,
                         int32_t* idx, int32_t* status, cudaStream_t st) {
-  if (D.K <= 16) return launch_tc_t<DD, G, 16>(D, qc, klm, blm, idx, status, st);
-  return launch_tc_t<DD, G, 32>(D, qc, klm, blm, idx, status, st);
+  // Two column groups: with four, the 18 warps cap a thread at 96 registers and the slower
+  // epilogue (spills, fewer TMEM loads in flight) outweighs the extra latency hiding.
+  if (D.K <= 16) return launch_tc_t<DD, G, 16, 2>(D, qc, klm, blm, idx, status, st);
+  return launch_tc_t<DD, G, 32, 2>(D, qc, klm, blm, idx, status, st);
 }
 
 }  // namespace
