@@ -79,7 +79,10 @@ Plan make_plan(const hils_params* p) {
   const size_t head_rows = (size_t)(p->B * p->Hq * p->N_q);
   size_t off = kStatusBytes;
   P.off_idx = off;   off = align_up(off + sel_rows * (size_t)D.K * sizeof(int32_t));
-  P.off_ssel = off;  off = align_up(off + head_rows * (size_t)D.K * sizeof(float));
+  if (!P.tc_attn) {   // the tensor-core attention scores the selected chunks itself
+    P.off_ssel = off;
+    off = align_up(off + head_rows * (size_t)D.K * sizeof(float));
+  }
   if (P.decode) {
     int64_t n_max = 0, win_max = 1;
     for (int64_t i = 0; i < p->N_q; ++i) {
