@@ -87,7 +87,7 @@ def phase_work(name, wm):
     """(bound, algorithmic work, unit) of a kernel, for its roofline."""
     if name in ("score_topk_tc", "select_rows"):
         return "tensor", wm["score_flops"], "TFLOP/s"
-    if name in ("select_split", "select_stream"):
+    if name in ("select_split", "select_stream", "select_stream_tc"):
         return "hbm", wm["select_bytes"], "GB/s"
     if name == "attn_units":
         return "hbm", wm["attn_bytes"], "GB/s"
@@ -113,7 +113,8 @@ def roofline(name, ms, wm, peaks, workload, sustained=False):
 KERNEL_SOURCES = {
     "score_topk_tc": ["score_tc.cu"], "attn_tc": ["attn_tc.cu"],
     "select_stream": ["select.cu"], "select_topk": ["select.cu"], "select_rows": ["select.cu"],
-    "select_split": ["select.cu"], "attn_units": ["attn.cu"], "attn_rows": ["attn.cu"],
+    "select_split": ["select.cu"], "select_stream_tc": ["stream_tc.cu"],
+    "attn_units": ["attn.cu"], "attn_rows": ["attn.cu"],
     "fuse_units": ["attn.cu"],
 }
 SHARED_SOURCES = ["common.cuh", "sm100.cuh"]

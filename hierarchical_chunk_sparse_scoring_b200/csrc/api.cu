@@ -35,6 +35,7 @@ struct Plan {
   bool decode = false;
   bool tc_select = false;
   bool tc_attn = false;
+  bool tc_stream = false;
   int cps = 0, n_split = 0, n_pieces = 0;
   size_t off_idx = 0, off_ssel = 0, off_pv = 0, off_pc = 0, off_po = 0, off_pl = 0;
   size_t off_sig = 0;
@@ -74,6 +75,7 @@ Plan make_plan(const hils_params* p) {
              p->B * p->Hkv * p->N_q <= 65535;
   P.tc_select = !P.decode && score_tc_supported(D, P.bf16);
   P.tc_attn = !P.decode && attn_tc_supported(D, P.bf16);
+  P.tc_stream = P.decode && stream_tc_supported(D, P.bf16);
 
   const size_t sel_rows = (size_t)(p->B * p->Hkv * p->N_q);
   const size_t head_rows = (size_t)(p->B * p->Hq * p->N_q);
@@ -162,10 +164,11 @@ struct PhaseMarks {
 
 int phase_names(const Plan& P, const char** names, int max_names) {
   static const char* kDecode[] = {"select_stream", "select_topk", "attn_units", "fuse_units"};
+  static const char* kDecodeTc[] = {"select_stream_tc", "select_topk", "attn_units", "fuse_units"};
   const char* pre[3];
   int n = 0;
   if (P.decode) {
-    for (int i = 0; i < 4 && i < max_names; ++i) names[i] = kDecode[i];
+    for (int i = 0; i < 4 && i < max_names; ++i) names[i] = P.tc_stream ? kDecodeTc[i] : kDecode[i];
     return 4;
   }
   if (P.tc_select) {
@@ -209,8 +212,11 @@ hils_status forward_impl(const hils_params* p, const void* q, const void* q_cal,
     float* po = reinterpret_cast<float*>(ws + P.off_po);
     float* pl = reinterpret_cast<float*>(ws + P.off_pl);
     float* sig = reinterpret_cast<float*>(ws + P.off_sig);
-    e = launch_select_stream(P.D, P.bf16, kStreamRows, n_stream_split(P), P.n_stride, q_cal, k_lm,
-                             b_lm, sig, reinterpret_cast<int32_t*>(ws), st);
+    e = P.tc_stream ? launch_select_stream_tc(P.D, q_cal, k_lm, b_lm, sig, P.n_stride,
+                                              reinterpret_cast<int32_t*>(ws), st)
+                    : launch_select_stream(P.D, P.bf16, kStreamRows, n_stream_split(P), P.n_stride,
+                                           q_cal, k_lm, b_lm, sig, reinterpret_cast<int32_t*>(ws),
+                                           st);
     pm.mark();
     (void)pv;
     (void)pc;
@@ -291,8 +297,11 @@ extern "C" hils_status hils_select(const hils_params* p, const void* q_cal, cons
   cudaError_t e;
   if (P.decode) {
     float* sig = reinterpret_cast<float*>(ws + P.off_sig);
-    e = launch_select_stream(P.D, P.bf16, kStreamRows, n_stream_split(P), P.n_stride, q_cal, k_lm,
-                             b_lm, sig, reinterpret_cast<int32_t*>(ws), st);
+    e = P.tc_stream ? launch_select_stream_tc(P.D, q_cal, k_lm, b_lm, sig, P.n_stride,
+                                              reinterpret_cast<int32_t*>(ws), st)
+                    : launch_select_stream(P.D, P.bf16, kStreamRows, n_stream_split(P), P.n_stride,
+                                           q_cal, k_lm, b_lm, sig, reinterpret_cast<int32_t*>(ws),
+                                           st);
     if (e == cudaSuccess)
       e = launch_select_topk_row(P.D, P.bf16, P.n_stride, sig, q_cal, k_lm, b_lm, idx, s_sel, st);
   } else if (P.tc_select) {

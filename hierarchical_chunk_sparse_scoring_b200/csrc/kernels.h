@@ -34,6 +34,10 @@ cudaError_t launch_select_stream(const Dims& D, bool bf16, int cps, int n_split,
                                  int64_t n_stride, const void* qc, const void* klm,
                                  const float* blm, float* sigma, int32_t* status,
                                  cudaStream_t st);
+bool stream_tc_supported(const Dims& D, bool bf16);
+cudaError_t launch_select_stream_tc(const Dims& D, const void* qc, const void* klm,
+                                    const float* blm, float* sigma, int64_t n_stride,
+                                    int32_t* status, cudaStream_t st);
 cudaError_t launch_select_topk(const Dims& D, int n_seg, int64_t n_stride, const float* sigma,
                                float* part_v, int32_t* part_c, cudaStream_t st);
 cudaError_t launch_select_topk_row(const Dims& D, bool bf16, int64_t n_stride,

@@ -88,6 +88,12 @@ EDGE_CASES = {
     "decode_short": dict(B=2, Hq=4, Hkv=1, N=100, d=128, S=64, K=4, W_=64, q_pos0=99, N_q=1),
     "decode_k32_g8": dict(B=2, Hq=8, Hkv=1, N=40000, d=128, S=32, K=32, W_=128,
                           q_pos0=39999, N_q=1),
+    # decode streaming scorer on the tensor core (bf16): 16 heads per group, and streams whose
+    # CTAs cross rows with ragged eligible counts per query
+    "decode_g16_d64": dict(B=2, Hq=16, Hkv=1, N=20000, d=64, S=64, K=8, W_=256,
+                           q_pos0=19999, N_q=1),
+    "decode_multi_query_tiles": dict(B=3, Hq=4, Hkv=2, N=70020, d=128, S=64, K=16, W_=512,
+                                     q_pos0=70013, N_q=3),
     # tensor-core selection shapes (bf16): ragged query tiles, every group size, K=32, S=128
     "tc_g2_d128": dict(B=1, Hq=4, Hkv=2, N=3000, d=128, S=64, K=8, W_=128),
     "tc_g8_d64": dict(B=1, Hq=8, Hkv=1, N=2500, d=64, S=32, K=16, W_=64),
