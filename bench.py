@@ -89,7 +89,7 @@ def phase_work(name, wm):
         return "tensor", wm["score_flops"], "TFLOP/s"
     if name in ("select_split", "select_stream", "select_stream_tc"):
         return "hbm", wm["select_bytes"], "GB/s"
-    if name == "attn_units":
+    if name in ("attn_units", "attn_units_tc"):
         return "hbm", wm["attn_bytes"], "GB/s"
     if name.startswith("attn"):
         return "tensor", wm["attn_flops"], "TFLOP/s"
@@ -114,7 +114,7 @@ KERNEL_SOURCES = {
     "score_topk_tc": ["score_tc.cu"], "attn_tc": ["attn_tc.cu"],
     "select_stream": ["select.cu"], "select_topk": ["select.cu"], "select_rows": ["select.cu"],
     "select_split": ["select.cu"], "select_stream_tc": ["stream_tc.cu"],
-    "attn_units": ["attn.cu"], "attn_rows": ["attn.cu"],
+    "attn_units": ["attn.cu"], "attn_units_tc": ["units_tc.cu"], "attn_rows": ["attn.cu"],
     "fuse_units": ["attn.cu"],
 }
 SHARED_SOURCES = ["common.cuh", "sm100.cuh"]

@@ -36,6 +36,7 @@ struct Plan {
   bool tc_select = false;
   bool tc_attn = false;
   bool tc_stream = false;
+  bool tc_units = false;
   int cps = 0, n_split = 0, n_pieces = 0;
   size_t off_idx = 0, off_ssel = 0, off_pv = 0, off_pc = 0, off_po = 0, off_pl = 0;
   size_t off_sig = 0;
@@ -76,6 +77,7 @@ Plan make_plan(const hils_params* p) {
   P.tc_select = !P.decode && score_tc_supported(D, P.bf16);
   P.tc_attn = !P.decode && attn_tc_supported(D, P.bf16);
   P.tc_stream = P.decode && stream_tc_supported(D, P.bf16);
+  P.tc_units = P.decode && units_tc_supported(D, P.bf16);
 
   const size_t sel_rows = (size_t)(p->B * p->Hkv * p->N_q);
   const size_t head_rows = (size_t)(p->B * p->Hq * p->N_q);
@@ -163,12 +165,14 @@ struct PhaseMarks {
 };
 
 int phase_names(const Plan& P, const char** names, int max_names) {
-  static const char* kDecode[] = {"select_stream", "select_topk", "attn_units", "fuse_units"};
-  static const char* kDecodeTc[] = {"select_stream_tc", "select_topk", "attn_units", "fuse_units"};
-  const char* pre[3];
+  const char* pre[4];
   int n = 0;
   if (P.decode) {
-    for (int i = 0; i < 4 && i < max_names; ++i) names[i] = P.tc_stream ? kDecodeTc[i] : kDecode[i];
+    pre[0] = P.tc_stream ? "select_stream_tc" : "select_stream";
+    pre[1] = "select_topk";
+    pre[2] = P.tc_units ? "attn_units_tc" : "attn_units";
+    pre[3] = "fuse_units";
+    for (int i = 0; i < 4 && i < max_names; ++i) names[i] = pre[i];
     return 4;
   }
   if (P.tc_select) {
@@ -223,8 +227,11 @@ hils_status forward_impl(const hils_params* p, const void* q, const void* q_cal,
     if (e == cudaSuccess)
       e = launch_select_topk_row(P.D, P.bf16, P.n_stride, sig, q_cal, k_lm, b_lm, idx, s_sel, st);
     pm.mark();
-    if (e == cudaSuccess) e = launch_attn_units(P.D, P.bf16, P.n_pieces, q, K, V, idx, po, pl,
-                                                  reinterpret_cast<int32_t*>(ws), st);
+    if (e == cudaSuccess)
+      e = P.tc_units ? launch_attn_units_tc(P.D, P.n_pieces, q, K, V, idx, po, pl,
+                                            reinterpret_cast<int32_t*>(ws), st)
+                     : launch_attn_units(P.D, P.bf16, P.n_pieces, q, K, V, idx, po, pl,
+                                         reinterpret_cast<int32_t*>(ws), st);
     pm.mark();
     if (e == cudaSuccess) e = launch_fuse_units(P.D, P.bf16, P.n_pieces, s_sel, po, pl, out, lse_out, st);
     pm.mark();

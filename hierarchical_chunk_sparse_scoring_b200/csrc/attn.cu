@@ -381,6 +381,37 @@ __global__ void __launch_bounds__(128) fuse_units_kernel(Dims D, int n_pieces,
   auto score_of = [&](int u) -> float {
     return u < K ? s_sel[row * K + u] : part_lse[row * NU + u];
   };
+  const float* pr = part_o + row * NU * d;
+  if (NU <= 32 && d == 128) {
+    // one unit per lane: its score is read once; then every lane reads its 4 output columns of
+    // all units, 16 loads in flight per batch
+    const float su = lane < NU ? score_of(lane) : -INFINITY;
+    const float M = warp_max(su);
+    const float e = su == -INFINITY ? 0.f : __expf(su - M);
+    const float Z = warp_sum(e);
+    const float wl = e / Z;
+    float o[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int u0 = 0; u0 < NU; u0 += 16) {
+      float v[16][4];
+#pragma unroll
+      for (int e2 = 0; e2 < 16; ++e2) {
+        if (u0 + e2 < NU) {
+          Elem<float>::load4(pr + (int64_t)(u0 + e2) * 128 + lane * 4, v[e2]);
+        } else {
+          v[e2][0] = v[e2][1] = v[e2][2] = v[e2][3] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int e2 = 0; e2 < 16; ++e2) {
+        const float w = __shfl_sync(0xffffffffu, wl, (u0 + e2) & 31);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) o[x] = fmaf(w, v[e2][x], o[x]);
+      }
+    }
+    Elem<T>::store4(out + row * 128 + lane * 4, o);
+    if (lse_out && lane == 0) lse_out[row] = M + logf(Z);
+    return;
+  }
   float M = -INFINITY;
   for (int u = lane; u < NU; u += 32) M = fmaxf(M, score_of(u));
   M = warp_max(M);
@@ -391,7 +422,6 @@ __global__ void __launch_bounds__(128) fuse_units_kernel(Dims D, int n_pieces,
   }
   Z = warp_sum(Z);
   const float invZ = 1.f / Z;
-  const float* pr = part_o + row * NU * d;
   // every lane runs every iteration (the loop body shuffles); lanes past d only skip memory
   for (int kb = 0; kb < d; kb += 128) {
     const int k0 = kb + lane * 4;

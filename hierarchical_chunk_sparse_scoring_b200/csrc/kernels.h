@@ -38,6 +38,10 @@ bool stream_tc_supported(const Dims& D, bool bf16);
 cudaError_t launch_select_stream_tc(const Dims& D, const void* qc, const void* klm,
                                     const float* blm, float* sigma, int64_t n_stride,
                                     int32_t* status, cudaStream_t st);
+bool units_tc_supported(const Dims& D, bool bf16);
+cudaError_t launch_attn_units_tc(const Dims& D, int n_pieces, const void* q, const void* K,
+                                 const void* V, const int32_t* idx, float* part_o,
+                                 float* part_lse, int32_t* status, cudaStream_t st);
 cudaError_t launch_select_topk(const Dims& D, int n_seg, int64_t n_stride, const float* sigma,
                                float* part_v, int32_t* part_c, cudaStream_t st);
 cudaError_t launch_select_topk_row(const Dims& D, bool bf16, int64_t n_stride,

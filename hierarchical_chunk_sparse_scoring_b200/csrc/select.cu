@@ -12,6 +12,8 @@
 //   select_split_kernel  many CTAs per (b, g, query) over disjoint chunk ranges, each writing
 //                        its own top-K; select_merge_kernel merges them.  Used for decode,
 //                        where one query's landmark stream (n x d) must be spread over the GPU.
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -65,6 +67,57 @@ __device__ __forceinline__ void write_selection(const Dims& D, int64_t b, int64_
         }
       }
     }
+  }
+}
+
+// Same result for bf16 inputs with the winners' landmark rows read by wide loads that are all in
+// flight at once, and the group's calibrated queries staged once per warp in shared memory
+// (qsh: [GM][D_] bf16); lane r < K handles winner c_r.
+template <int D_, int GM>
+__device__ __forceinline__ void write_selection_wide(const Dims& D, int64_t b, int64_t g,
+                                                     int64_t i, __nv_bfloat16* qsh,
+                                                     const __nv_bfloat16* qc,
+                                                     const __nv_bfloat16* kb, const float* bb,
+                                                     int lane, int c, int32_t* idx,
+                                                     float* s_sel) {
+  constexpr int NV = D_ / 8;   // 16-byte vectors per row
+  const int K = D.K, G = D.G;
+  uint4* q4 = reinterpret_cast<uint4*>(qsh);
+  for (int e = lane; e < G * NV; e += 32) {
+    const int h = e / NV, j = e - h * NV;
+    const int64_t hrow = ((b * D.Hq) + g * G + h) * D.N_q + i;
+    q4[h * NV + j] = __ldg(reinterpret_cast<const uint4*>(qc + hrow * D_) + j);
+  }
+  __syncwarp();
+  const int64_t sel_row = ((b * D.Hkv + g) * D.N_q + i) * K;
+  if (lane >= K) return;
+  const bool valid = c != INT_MAX;
+  idx[sel_row + lane] = valid ? c : -1;
+  if (!s_sel) return;
+  uint4 kv[NV];
+#pragma unroll
+  for (int j = 0; j < NV; ++j)
+    kv[j] = valid ? __ldg(reinterpret_cast<const uint4*>(kb + (int64_t)c * D_) + j)
+                  : make_uint4(0u, 0u, 0u, 0u);
+  const float bc = valid ? __ldg(bb + c) : 0.f;
+#pragma unroll
+  for (int h = 0; h < GM; ++h) {
+    if (h >= G) break;
+    float a = 0.f;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const uint4 qv = q4[h * NV + j];
+      a = fmaf(bf16_lo(qv.x), bf16_lo(kv[j].x), a);
+      a = fmaf(bf16_hi(qv.x), bf16_hi(kv[j].x), a);
+      a = fmaf(bf16_lo(qv.y), bf16_lo(kv[j].y), a);
+      a = fmaf(bf16_hi(qv.y), bf16_hi(kv[j].y), a);
+      a = fmaf(bf16_lo(qv.z), bf16_lo(kv[j].z), a);
+      a = fmaf(bf16_hi(qv.z), bf16_hi(kv[j].z), a);
+      a = fmaf(bf16_lo(qv.w), bf16_lo(kv[j].w), a);
+      a = fmaf(bf16_hi(qv.w), bf16_hi(kv[j].w), a);
+    }
+    const int64_t hrow = ((b * D.Hq) + g * G + h) * D.N_q + i;
+    s_sel[hrow * K + lane] = valid ? fmaf(a, D.scale, bc) : -INFINITY;
   }
 }
 
@@ -644,16 +697,19 @@ __global__ void __launch_bounds__(256) select_topk_kernel(Dims D, int64_t n_stri
   }
 }
 
-// Decode top-K of one query row's group scores, one 1024-thread CTA per (b, g, query).
-//   1. every warp takes the best (value, chunk) of its candidates: 32 warp maxima;
-//   2. warp 0 sorts them (bitonic network over shuffles); the K-th of them, theta, is a lower
+// Decode top-K of one query row's group scores, one warp per (b, g, query), four rows per CTA.
+//   1. every lane takes the best (value, chunk) of its share of the row: 32 lane maxima;
+//   2. the warp sorts them (bitonic network over shuffles); the K-th of them, theta, is a lower
 //      bound of the row's K-th best (those K maxima are K distinct candidates >= theta);
-//   3. every candidate >= theta is appended to a shared list (typically a few dozen);
-//   4. one warp takes the exact top-K of that list (register lists, warp merge) and writes idx
+//   3. every candidate >= theta is appended to the warp's shared list (ballot compaction;
+//      typically a few dozen);
+//   4. the warp takes the exact top-K of that list (register lists, warp merge) and writes idx
 //      and the per-head scores.  If more than kSurvivorCap candidates tie at or above theta,
 //      step 4 runs over all candidates instead (slower, same result).
-constexpr int kTopkThreads = 1024;
-constexpr int kSurvivorCap = 2048;
+constexpr int kTopkRowsPerCta = 4;
+constexpr int kTopkThreads = 32 * kTopkRowsPerCta;
+constexpr int kSurvivorCap = 768;
+constexpr int kTopkBatch = 16;
 
 // ascending-by-`better` position: true if (v, c) should come before (ov, oc)
 __device__ __forceinline__ void cmpx(float& v, int& c, int partner_lane_xor, bool keep_better) {
@@ -663,39 +719,56 @@ __device__ __forceinline__ void cmpx(float& v, int& c, int partner_lane_xor, boo
   if (keep_better == other_better) { v = ov; c = oc; }
 }
 
-template <typename T, int GM, int KM>
+template <typename T, int D_, int GM, int KM>
 __global__ void __launch_bounds__(kTopkThreads) select_topk_row_kernel(
     Dims D, int64_t n_stride, const float* __restrict__ sigma, const T* __restrict__ qc,
     const T* __restrict__ klm, const float* __restrict__ blm, int32_t* __restrict__ idx,
     float* __restrict__ s_sel) {
-  __shared__ float wv_sh[32];
-  __shared__ int wc_sh[32];
-  __shared__ float th_v;
-  __shared__ int th_c;
-  __shared__ int n_surv;
-  __shared__ float sv[kSurvivorCap];
-  __shared__ int scn[kSurvivorCap];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t row = blockIdx.x;
+  __shared__ float sv_all[kTopkRowsPerCta][kSurvivorCap];
+  __shared__ int scn_all[kTopkRowsPerCta][kSurvivorCap];
+  __shared__ __align__(16) __nv_bfloat16 qsh_all[kTopkRowsPerCta][GM * D_];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t row = (int64_t)blockIdx.x * kTopkRowsPerCta + warp;
+  if (row >= D.B * D.Hkv * D.N_q) return;
+  float* sv = sv_all[warp];
+  int* scn = scn_all[warp];
   const int64_t i = row % D.N_q, bg = row / D.N_q, g = bg % D.Hkv, b = bg / D.Hkv;
   const int K = D.K;
   const int64_t n = n_eligible(D.q_pos0 + i, D.S, D.W);
-  const float* sr = sigma + row * n_stride;
-  // 1. warp maxima
+  const float* sr = sigma + row * n_stride;             // 16-byte aligned (n_stride % 4 == 0)
+  const int64_t n4 = n >> 2;
+  // 1. lane maxima (each lane's chunks come in increasing order: a strict compare keeps the
+  //    lower index on ties)
   float mv = -INFINITY;
   int mc = INT_MAX;
-  for (int64_t c = tid; c < n; c += kTopkThreads) {
-    const float v = sr[c];
+  // batches of kTopkBatch independent 16-byte loads per lane keep the row's reads in flight
+  for (int64_t q0 = 0; q0 < n4; q0 += 32 * kTopkBatch) {
+    float4 t[kTopkBatch];
+#pragma unroll
+    for (int u = 0; u < kTopkBatch; ++u) {
+      const int64_t q4 = q0 + u * 32 + lane;
+      t[u] = q4 < n4 ? __ldg(reinterpret_cast<const float4*>(sr) + q4)
+                     : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    }
+#pragma unroll
+    for (int u = 0; u < kTopkBatch; ++u) {
+      const int c = (int)((q0 + u * 32 + lane) * 4);
+      if (t[u].x > mv) { mv = t[u].x; mc = c; }
+      if (t[u].y > mv) { mv = t[u].y; mc = c + 1; }
+      if (t[u].z > mv) { mv = t[u].z; mc = c + 2; }
+      if (t[u].w > mv) { mv = t[u].w; mc = c + 3; }
+    }
+  }
+  for (int64_t c = n4 * 4 + lane; c < n; c += 32) {
+    const float v = __ldg(sr + c);
     if (better(v, (int)c, mv, mc)) { mv = v; mc = (int)c; }
   }
-  warp_best(mv, mc);
-  if (lane == 0) { wv_sh[warp] = mv; wc_sh[warp] = mc; }
-  if (tid == 0) n_surv = 0;
-  __syncthreads();
-  // 2. theta = K-th best warp maximum (bitonic sort of 32 pairs, best first)
-  if (warp == 0) {
-    float v = wv_sh[lane];
-    int c = wc_sh[lane];
+  // 2. theta = K-th best lane maximum (bitonic sort of 32 pairs, best first)
+  float tv;
+  int tcc;
+  {
+    float v = mv;
+    int c = mc;
 #pragma unroll
     for (int size = 2; size <= 32; size <<= 1) {
 #pragma unroll
@@ -706,37 +779,68 @@ __global__ void __launch_bounds__(kTopkThreads) select_topk_row_kernel(
       }
     }
     const int kk = K < 32 ? K : 32;
-    const float tv = __shfl_sync(0xffffffffu, v, kk - 1);
-    const int tcc = __shfl_sync(0xffffffffu, c, kk - 1);
-    if (lane == 0) { th_v = tv; th_c = tcc; }
+    tv = __shfl_sync(0xffffffffu, v, kk - 1);
+    tcc = __shfl_sync(0xffffffffu, c, kk - 1);
   }
-  __syncthreads();
-  // 3. survivors: candidates not worse than theta
-  const float tv = th_v;
-  const int tcc = th_c;
-  for (int64_t c = tid; c < n; c += kTopkThreads) {
-    const float v = sr[c];
-    if (!better(tv, tcc, v, (int)c)) {
-      const int slot = atomicAdd(&n_surv, 1);
-      if (slot < kSurvivorCap) { sv[slot] = v; scn[slot] = (int)c; }
+  // 3. survivors: candidates not worse than theta, compacted in ballot order
+  int ns = 0;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int64_t q0 = 0; q0 < n4; q0 += 32 * kTopkBatch) {
+    float4 t[kTopkBatch];
+#pragma unroll
+    for (int u = 0; u < kTopkBatch; ++u) {
+      const int64_t q4 = q0 + u * 32 + lane;
+      t[u] = q4 < n4 ? __ldg(reinterpret_cast<const float4*>(sr) + q4)
+                     : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    }
+#pragma unroll
+    for (int u = 0; u < kTopkBatch; ++u) {
+      const int64_t q4 = q0 + u * 32 + lane;
+      const bool in = q4 < n4;
+      const float vv[4] = {t[u].x, t[u].y, t[u].z, t[u].w};
+      // most of a row is below theta: skip the compaction when no lane keeps anything
+      bool any = false;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) any |= in && !better(tv, tcc, vv[j], (int)(q4 * 4) + j);
+      if (!__any_sync(0xffffffffu, any)) continue;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = (int)(q4 * 4) + j;
+        const bool keep = in && !better(tv, tcc, vv[j], c);
+        const unsigned m = __ballot_sync(0xffffffffu, keep);
+        const int pos = ns + __popc(m & lt);
+        if (keep && pos < kSurvivorCap) { sv[pos] = vv[j]; scn[pos] = c; }
+        ns += __popc(m);
+      }
     }
   }
-  __syncthreads();
-  const int ns = n_surv;
-  if (warp != 0) return;
+  for (int64_t c0 = n4 * 4; c0 < n; c0 += 32) {
+    const int64_t c = c0 + lane;
+    const float v = c < n ? __ldg(sr + c) : -INFINITY;
+    const bool keep = c < n && !better(tv, tcc, v, (int)c);
+    const unsigned m = __ballot_sync(0xffffffffu, keep);
+    const int pos = ns + __popc(m & lt);
+    if (keep && pos < kSurvivorCap) { sv[pos] = v; scn[pos] = (int)c; }
+    ns += __popc(m);
+  }
+  __syncwarp();
   // 4. exact top-K of the survivors (or of every candidate if too many tied at theta)
   TopList<KM> L;
   L.clear();
   if (ns <= kSurvivorCap) {
     for (int e = lane; e < ns; e += 32) L.insert(sv[e], scn[e], K);
   } else {
-    for (int64_t c = lane; c < n; c += 32) L.insert(sr[c], (int)c, K);
+    for (int64_t c = lane; c < n; c += 32) L.insert(__ldg(sr + c), (int)c, K);
   }
   float wv;
   int wc;
   warp_merge_topk<KM>(L, K, lane, wv, wc);
-  write_selection<T, GM>(D, b, g, i, nullptr, qc, klm + bg * D.C * D.d, blm + bg * D.C, lane,
-                         wc, idx, s_sel);
+  if constexpr (std::is_same<T, __nv_bfloat16>::value)
+    write_selection_wide<D_, GM>(D, b, g, i, qsh_all[warp], qc, klm + bg * D.C * D_,
+                                 blm + bg * D.C, lane, wc, idx, s_sel);
+  else
+    write_selection<T, GM>(D, b, g, i, nullptr, qc, klm + bg * D.C * D.d, blm + bg * D.C, lane,
+                           wc, idx, s_sel);
 }
 
 template <typename T, int D_, int GM, int KM>
@@ -745,7 +849,8 @@ struct TopkRowRun {
                          const void* klm, const float* blm, int32_t* idx, float* s_sel,
                          cudaStream_t st) {
     const int64_t rows = D->B * D->Hkv * D->N_q;
-    select_topk_row_kernel<T, GM, KM><<<(unsigned)rows, kTopkThreads, 0, st>>>(
+    const int64_t ctas = (rows + kTopkRowsPerCta - 1) / kTopkRowsPerCta;
+    select_topk_row_kernel<T, D_, GM, KM><<<(unsigned)ctas, kTopkThreads, 0, st>>>(
         *D, n_stride, sigma, (const T*)qc, (const T*)klm, blm, idx, s_sel);
     return cudaGetLastError();
   }
