@@ -697,19 +697,22 @@ __global__ void __launch_bounds__(256) select_topk_kernel(Dims D, int64_t n_stri
   }
 }
 
-// Decode top-K of one query row's group scores, one warp per (b, g, query), four rows per CTA.
-//   1. every lane takes the best (value, chunk) of its share of the row: 32 lane maxima;
-//   2. the warp sorts them (bitonic network over shuffles); the K-th of them, theta, is a lower
-//      bound of the row's K-th best (those K maxima are K distinct candidates >= theta);
-//   3. every candidate >= theta is appended to the warp's shared list (ballot compaction;
-//      typically a few dozen);
-//   4. the warp takes the exact top-K of that list (register lists, warp merge) and writes idx
-//      and the per-head scores.  If more than kSurvivorCap candidates tie at or above theta,
-//      step 4 runs over all candidates instead (slower, same result).
-constexpr int kTopkRowsPerCta = 4;
-constexpr int kTopkThreads = 32 * kTopkRowsPerCta;
-constexpr int kSurvivorCap = 768;
-constexpr int kTopkBatch = 16;
+// Decode top-K of one query row's group scores, one 128-thread CTA per (b, g, query); warp w
+// takes the w-th quarter of the row.
+//   1. every lane takes the best (value, chunk) of its share: 32 lane maxima per warp;
+//   2. each warp sorts its maxima (bitonic network over shuffles); the K-th of them is a lower
+//      bound of its quarter's K-th best, so the largest of the four, theta, is a lower bound of
+//      the row's K-th best;
+//   3. every candidate >= theta is appended to a shared list (ballot compaction; typically a
+//      few dozen);
+//   4. warp 0 takes the exact top-K of that list -- one bitonic sort when it holds at most 32,
+//      register lists and a warp merge otherwise -- and writes idx and the per-head scores.  If
+//      more than kSurvivorCap candidates tie at or above theta, step 4 runs over all candidates
+//      (slower, same result).
+constexpr int kTopkWarps = 4;
+constexpr int kTopkThreads = 32 * kTopkWarps;
+constexpr int kSurvivorCap = 1024;
+constexpr int kTopkBatch = 8;
 
 // ascending-by-`better` position: true if (v, c) should come before (ov, oc)
 __device__ __forceinline__ void cmpx(float& v, int& c, int partner_lane_xor, bool keep_better) {
@@ -719,35 +722,50 @@ __device__ __forceinline__ void cmpx(float& v, int& c, int partner_lane_xor, boo
   if (keep_better == other_better) { v = ov; c = oc; }
 }
 
+// Sorts one (value, chunk) per lane, best first (lane 0 = best).
+__device__ __forceinline__ void warp_sort_best_first(float& v, int& c, int lane) {
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const bool up = ((lane & size) == 0);          // this 'size' block sorts best-first
+      const bool lower = ((lane & stride) == 0);     // lower index of the compared pair
+      cmpx(v, c, stride, up == lower);
+    }
+  }
+}
+
 template <typename T, int D_, int GM, int KM>
 __global__ void __launch_bounds__(kTopkThreads) select_topk_row_kernel(
     Dims D, int64_t n_stride, const float* __restrict__ sigma, const T* __restrict__ qc,
     const T* __restrict__ klm, const float* __restrict__ blm, int32_t* __restrict__ idx,
     float* __restrict__ s_sel) {
-  __shared__ float sv_all[kTopkRowsPerCta][kSurvivorCap];
-  __shared__ int scn_all[kTopkRowsPerCta][kSurvivorCap];
-  __shared__ __align__(16) __nv_bfloat16 qsh_all[kTopkRowsPerCta][GM * D_];
+  __shared__ float sv[kSurvivorCap];
+  __shared__ int scn[kSurvivorCap];
+  __shared__ float th_v[kTopkWarps];
+  __shared__ int th_c[kTopkWarps];
+  __shared__ int n_surv;
+  __shared__ __align__(16) __nv_bfloat16 qsh[GM * D_];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t row = (int64_t)blockIdx.x * kTopkRowsPerCta + warp;
-  if (row >= D.B * D.Hkv * D.N_q) return;
-  float* sv = sv_all[warp];
-  int* scn = scn_all[warp];
+  const int64_t row = blockIdx.x;
   const int64_t i = row % D.N_q, bg = row / D.N_q, g = bg % D.Hkv, b = bg / D.Hkv;
   const int K = D.K;
   const int64_t n = n_eligible(D.q_pos0 + i, D.S, D.W);
   const float* sr = sigma + row * n_stride;             // 16-byte aligned (n_stride % 4 == 0)
   const int64_t n4 = n >> 2;
-  // 1. lane maxima (each lane's chunks come in increasing order: a strict compare keeps the
-  //    lower index on ties)
+  // this warp's quarter of the row's float4 vectors (the scalar tail goes to the last warp)
+  const int64_t w0 = n4 * warp / kTopkWarps, w1 = n4 * (warp + 1) / kTopkWarps;
+  if (threadIdx.x == 0) n_surv = 0;
+  // 1. lane maxima (a lane's chunks come in increasing order: a strict compare keeps the lower
+  //    index on ties)
   float mv = -INFINITY;
   int mc = INT_MAX;
-  // batches of kTopkBatch independent 16-byte loads per lane keep the row's reads in flight
-  for (int64_t q0 = 0; q0 < n4; q0 += 32 * kTopkBatch) {
+  for (int64_t q0 = w0; q0 < w1; q0 += 32 * kTopkBatch) {
     float4 t[kTopkBatch];
 #pragma unroll
     for (int u = 0; u < kTopkBatch; ++u) {
       const int64_t q4 = q0 + u * 32 + lane;
-      t[u] = q4 < n4 ? __ldg(reinterpret_cast<const float4*>(sr) + q4)
+      t[u] = q4 < w1 ? __ldg(reinterpret_cast<const float4*>(sr) + q4)
                      : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
     }
 #pragma unroll
@@ -759,85 +777,95 @@ __global__ void __launch_bounds__(kTopkThreads) select_topk_row_kernel(
       if (t[u].w > mv) { mv = t[u].w; mc = c + 3; }
     }
   }
-  for (int64_t c = n4 * 4 + lane; c < n; c += 32) {
-    const float v = __ldg(sr + c);
-    if (better(v, (int)c, mv, mc)) { mv = v; mc = (int)c; }
+  if (warp == kTopkWarps - 1) {
+    for (int64_t c = n4 * 4 + lane; c < n; c += 32) {
+      const float v = __ldg(sr + c);
+      if (better(v, (int)c, mv, mc)) { mv = v; mc = (int)c; }
+    }
   }
-  // 2. theta = K-th best lane maximum (bitonic sort of 32 pairs, best first)
-  float tv;
-  int tcc;
+  // 2. theta = the best of the warps' K-th lane maxima
   {
     float v = mv;
     int c = mc;
-#pragma unroll
-    for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll
-      for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        const bool up = ((lane & size) == 0);          // this 'size' block sorts best-first
-        const bool lower = ((lane & stride) == 0);     // lower index of the compared pair
-        cmpx(v, c, stride, up == lower);
-      }
-    }
+    warp_sort_best_first(v, c, lane);
     const int kk = K < 32 ? K : 32;
-    tv = __shfl_sync(0xffffffffu, v, kk - 1);
-    tcc = __shfl_sync(0xffffffffu, c, kk - 1);
+    const float tv = __shfl_sync(0xffffffffu, v, kk - 1);
+    const int tcc = __shfl_sync(0xffffffffu, c, kk - 1);
+    if (lane == 0) { th_v[warp] = tv; th_c[warp] = tcc; }
   }
-  // 3. survivors: candidates not worse than theta, compacted in ballot order
-  int ns = 0;
+  __syncthreads();
+  float tv = th_v[0];
+  int tcc = th_c[0];
+#pragma unroll
+  for (int w = 1; w < kTopkWarps; ++w)
+    if (better(th_v[w], th_c[w], tv, tcc)) { tv = th_v[w]; tcc = th_c[w]; }
+  // 3. survivors: candidates not worse than theta, compacted in ballot order per warp batch
   const unsigned lt = (1u << lane) - 1u;
-  for (int64_t q0 = 0; q0 < n4; q0 += 32 * kTopkBatch) {
+  auto append = [&](bool keep, float v, int c) {
+    const unsigned m = __ballot_sync(0xffffffffu, keep);
+    if (m == 0u) return;
+    int base = 0;
+    if (lane == 0) base = atomicAdd(&n_surv, __popc(m));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    const int pos = base + __popc(m & lt);
+    if (keep && pos < kSurvivorCap) { sv[pos] = v; scn[pos] = c; }
+  };
+  for (int64_t q0 = w0; q0 < w1; q0 += 32 * kTopkBatch) {
     float4 t[kTopkBatch];
 #pragma unroll
     for (int u = 0; u < kTopkBatch; ++u) {
       const int64_t q4 = q0 + u * 32 + lane;
-      t[u] = q4 < n4 ? __ldg(reinterpret_cast<const float4*>(sr) + q4)
+      t[u] = q4 < w1 ? __ldg(reinterpret_cast<const float4*>(sr) + q4)
                      : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
     }
 #pragma unroll
     for (int u = 0; u < kTopkBatch; ++u) {
       const int64_t q4 = q0 + u * 32 + lane;
-      const bool in = q4 < n4;
-      const float vv[4] = {t[u].x, t[u].y, t[u].z, t[u].w};
+      const bool in = q4 < w1;
+      const int c = (int)(q4 * 4);
+      const bool k0 = in && !better(tv, tcc, t[u].x, c);
+      const bool k1 = in && !better(tv, tcc, t[u].y, c + 1);
+      const bool k2 = in && !better(tv, tcc, t[u].z, c + 2);
+      const bool k3 = in && !better(tv, tcc, t[u].w, c + 3);
       // most of a row is below theta: skip the compaction when no lane keeps anything
-      bool any = false;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) any |= in && !better(tv, tcc, vv[j], (int)(q4 * 4) + j);
-      if (!__any_sync(0xffffffffu, any)) continue;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int c = (int)(q4 * 4) + j;
-        const bool keep = in && !better(tv, tcc, vv[j], c);
-        const unsigned m = __ballot_sync(0xffffffffu, keep);
-        const int pos = ns + __popc(m & lt);
-        if (keep && pos < kSurvivorCap) { sv[pos] = vv[j]; scn[pos] = c; }
-        ns += __popc(m);
-      }
+      if (!__any_sync(0xffffffffu, k0 || k1 || k2 || k3)) continue;
+      append(k0, t[u].x, c);
+      append(k1, t[u].y, c + 1);
+      append(k2, t[u].z, c + 2);
+      append(k3, t[u].w, c + 3);
     }
   }
-  for (int64_t c0 = n4 * 4; c0 < n; c0 += 32) {
-    const int64_t c = c0 + lane;
-    const float v = c < n ? __ldg(sr + c) : -INFINITY;
-    const bool keep = c < n && !better(tv, tcc, v, (int)c);
-    const unsigned m = __ballot_sync(0xffffffffu, keep);
-    const int pos = ns + __popc(m & lt);
-    if (keep && pos < kSurvivorCap) { sv[pos] = v; scn[pos] = (int)c; }
-    ns += __popc(m);
+  if (warp == kTopkWarps - 1) {
+    for (int64_t c0 = n4 * 4; c0 < n; c0 += 32) {
+      const int64_t c = c0 + lane;
+      const float v = c < n ? __ldg(sr + c) : -INFINITY;
+      append(c < n && !better(tv, tcc, v, (int)c), v, (int)c);
+    }
   }
-  __syncwarp();
+  __syncthreads();
+  if (warp != 0) return;
+  const int ns = n_surv;
   // 4. exact top-K of the survivors (or of every candidate if too many tied at theta)
-  TopList<KM> L;
-  L.clear();
-  if (ns <= kSurvivorCap) {
-    for (int e = lane; e < ns; e += 32) L.insert(sv[e], scn[e], K);
-  } else {
-    for (int64_t c = lane; c < n; c += 32) L.insert(__ldg(sr + c), (int)c, K);
-  }
   float wv;
   int wc;
-  warp_merge_topk<KM>(L, K, lane, wv, wc);
+  if (ns <= 32) {
+    wv = lane < ns ? sv[lane] : -INFINITY;
+    wc = lane < ns ? scn[lane] : INT_MAX;
+    warp_sort_best_first(wv, wc, lane);
+    if (lane >= K) { wv = -INFINITY; wc = INT_MAX; }
+  } else {
+    TopList<KM> L;
+    L.clear();
+    if (ns <= kSurvivorCap) {
+      for (int e = lane; e < ns; e += 32) L.insert(sv[e], scn[e], K);
+    } else {
+      for (int64_t c = lane; c < n; c += 32) L.insert(__ldg(sr + c), (int)c, K);
+    }
+    warp_merge_topk<KM>(L, K, lane, wv, wc);
+  }
   if constexpr (std::is_same<T, __nv_bfloat16>::value)
-    write_selection_wide<D_, GM>(D, b, g, i, qsh_all[warp], qc, klm + bg * D.C * D_,
-                                 blm + bg * D.C, lane, wc, idx, s_sel);
+    write_selection_wide<D_, GM>(D, b, g, i, qsh, qc, klm + bg * D.C * D_, blm + bg * D.C, lane,
+                                 wc, idx, s_sel);
   else
     write_selection<T, GM>(D, b, g, i, nullptr, qc, klm + bg * D.C * D.d, blm + bg * D.C, lane,
                            wc, idx, s_sel);
@@ -849,8 +877,7 @@ struct TopkRowRun {
                          const void* klm, const float* blm, int32_t* idx, float* s_sel,
                          cudaStream_t st) {
     const int64_t rows = D->B * D->Hkv * D->N_q;
-    const int64_t ctas = (rows + kTopkRowsPerCta - 1) / kTopkRowsPerCta;
-    select_topk_row_kernel<T, D_, GM, KM><<<(unsigned)ctas, kTopkThreads, 0, st>>>(
+    select_topk_row_kernel<T, D_, GM, KM><<<(unsigned)rows, kTopkThreads, 0, st>>>(
         *D, n_stride, sigma, (const T*)qc, (const T*)klm, blm, idx, s_sel);
     return cudaGetLastError();
   }

@@ -13,8 +13,9 @@
 //     per head and write P (bf16) as a K-major [16 heads x 128 tokens] operand;
 //   * O_u^T = V_u^T . P_u (M = d = 128, N = 16, K = 64 tokens; V read as an MN-major operand) for
 //     each of the two units; the epilogue (one d-row per thread) divides by the unit's sum.
-// Persistent CTAs, three per SM, each with one stage: the stage is released as soon as the two
-// P.V products have read it, so the next tile's copies overlap this tile's output phase.
+// Persistent CTAs, three per SM, each with one stage whose K and V halves are released
+// separately: the next tile's K (and queries) load once this tile's Q.K^T has read K, its V once
+// the P.V products have read V, so both copies overlap this tile's softmax and output phases.
 // Every mbarrier wait gives up after a bounded number of polls and records HILS_ERR_TIMEOUT.
 #include <cudaTypedefs.h>
 
@@ -89,12 +90,14 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
   uint8_t* sQ = sV + SH::KT;
   uint8_t* sP = sQ + SH::QT;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sP + SH::P_BYTES);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + 1;
-  uint64_t* s_full = bars + 2;
-  uint64_t* p_full = bars + 3;
-  uint64_t* o_full = bars + 4;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 5);
+  uint64_t* k_full = bars;        // K and Q of the tile landed
+  uint64_t* v_full = bars + 1;    // V landed
+  uint64_t* k_empty = bars + 2;   // Q.K^T has read K and Q
+  uint64_t* v_empty = bars + 3;   // P.V has read V
+  uint64_t* s_full = bars + 4;
+  uint64_t* p_full = bars + 5;
+  uint64_t* o_full = bars + 6;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 7);
   float* red_m = reinterpret_cast<float*>(bars + 8);   // [2 parities][4 warps][16 heads]
   float* red_l = red_m + 2 * 4 * kUtCols;              // [2][4][16]
 
@@ -105,8 +108,10 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
   const int n_local = (int)(t_end - t_begin);
 
   if (threadIdx.x == 0) {
-    mbar_init(full, 1);
-    mbar_init(empty, 1);
+    mbar_init(k_full, 1);
+    mbar_init(v_full, 1);
+    mbar_init(k_empty, 1);
+    mbar_init(v_empty, 1);
     mbar_init(s_full, 1);
     mbar_init(p_full, 4);
     mbar_init(o_full, 1);
@@ -124,37 +129,54 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
-      for (int u = 0; u < n_local; ++u) {
-        if (!mbar_wait(empty, ((uint32_t)u & 1u) ^ 1u, kUtPoll)) {
-          record_status(status, kStatusTimeout);
-          break;
-        }
+      // token spans of a tile's two units (the idx reads of the next tile are issued before
+      // the waits for the current stage, so their latency hides behind them)
+      auto spans = [&](int u, int32_t (&y)[2], int32_t& qi, int32_t& qh) {
         const int64_t t = t_begin + u;
         const int64_t row = t / tiles_per_row, pr = t - row * tiles_per_row;
         const int64_t i = row % D.N_q, bg = row / D.N_q;
         const int64_t g = bg % D.Hkv, b = bg / D.Hkv;
         const int64_t pos = D.q_pos0 + i, n = n_eligible(pos, D.S, D.W);
-        mbar_expect_tx(full, SH::STAGE);
         for (int half = 0; half < 2; ++half) {
           int64_t t0;
           int len;
           unit_span(D, idx, row, n, pos, n_units, (int)(2 * pr + half), t0, len);
-          // an empty unit still loads (chunk 0 of the row); the softmax masks all its tokens
-          const int32_t y = (int32_t)(bg * D.N_kv + t0);
-          for (int kb = 0; kb < SH::KB; ++kb) {
-            tma_load_2d(sK + kb * SH::BLK + half * SH::UNIT_BOX, &tmK, kb * 64, y, full);
-            tma_load_2d(sV + kb * SH::BLK + half * SH::UNIT_BOX, &tmV, kb * 64, y, full);
-          }
+          // an empty unit still loads (from token 0 of the row); the softmax masks it
+          y[half] = (int32_t)(bg * D.N_kv + t0);
         }
+        qi = (int32_t)i;
+        qh = (int32_t)(b * D.Hq + g * D.G);
+      };
+      int32_t y[2], qi, qh;
+      spans(0, y, qi, qh);
+      bool ok = true;
+      for (int u = 0; u < n_local; ++u) {
+        const uint32_t ph = (uint32_t)u & 1u;
+        if (!mbar_wait(k_empty, ph ^ 1u, kUtPoll)) { ok = false; break; }
+        mbar_expect_tx(k_full, 2 * SH::KB * SH::UNIT_BOX + SH::QT);
+        for (int half = 0; half < 2; ++half)
+          for (int kb = 0; kb < SH::KB; ++kb)
+            tma_load_2d(sK + kb * SH::BLK + half * SH::UNIT_BOX, &tmK, kb * 64, y[half], k_full);
         for (int kb = 0; kb < SH::KB; ++kb)
           asm volatile(
               "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
               " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(sQ + kb * SH::Q_BOX)),
-              "l"(reinterpret_cast<uint64_t>(&tmQ)), "r"(kb * 64), "r"((int32_t)i),
-              "r"((int32_t)(b * D.Hq + g * D.G)), "r"(smem_u32(full))
+              "l"(reinterpret_cast<uint64_t>(&tmQ)), "r"(kb * 64), "r"(qi), "r"(qh),
+              "r"(smem_u32(k_full))
               : "memory");
+        if (!mbar_wait(v_empty, ph ^ 1u, kUtPoll)) { ok = false; break; }
+        mbar_expect_tx(v_full, 2 * SH::KB * SH::UNIT_BOX);
+        for (int half = 0; half < 2; ++half)
+          for (int kb = 0; kb < SH::KB; ++kb)
+            tma_load_2d(sV + kb * SH::BLK + half * SH::UNIT_BOX, &tmV, kb * 64, y[half], v_full);
+        if (u + 1 < n_local) spans(u + 1, y, qi, qh);
       }
-      if (n_local > 0) mbar_wait(full, (uint32_t)(n_local - 1) & 1u, kUtPoll);
+      if (!ok) record_status(status, kStatusTimeout);
+      // this thread's copies have landed before it leaves (bounded)
+      if (ok) {
+        mbar_wait(k_full, (uint32_t)(n_local - 1) & 1u, kUtPoll);
+        mbar_wait(v_full, (uint32_t)(n_local - 1) & 1u, kUtPoll);
+      }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -164,7 +186,7 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
       bool ok = true;
       for (int u = 0; ok && u < n_local; ++u) {
         const uint32_t ph = (uint32_t)u & 1u;
-        if (!mbar_wait(full, ph, kUtPoll)) { ok = false; break; }
+        if (!mbar_wait(k_full, ph, kUtPoll)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < kUtD / 16; ++ks) {
@@ -174,7 +196,11 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
                       ks > 0 ? 1u : 0u);
         }
         mma_commit(s_full);
-        if (!mbar_wait(p_full, ph, kUtPoll)) { ok = false; break; }
+        mma_commit(k_empty);
+        if (!mbar_wait(p_full, ph, kUtPoll) || !mbar_wait(v_full, ph, kUtPoll)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -188,7 +214,7 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
           }
         }
         mma_commit(o_full);
-        mma_commit(empty);
+        mma_commit(v_empty);
       }
       if (!ok) record_status(status, kStatusTimeout);
     }
