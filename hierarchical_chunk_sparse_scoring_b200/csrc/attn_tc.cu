@@ -639,6 +639,8 @@ template <int DD, int G>
 cudaError_t launch_at_k(const Dims& D, const void* q, const void* qc, const void* K,
                         const void* V, const int32_t* idx, const void* klm, const float* blm,
                         void* out, float* lse, int32_t* status, cudaStream_t st) {
+  if (D.K <= 8)
+    return launch_at_t<DD, G, 8>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st);
   if (D.K <= 16)
     return launch_at_t<DD, G, 16>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st);
   return launch_at_t<DD, G, 32>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st);

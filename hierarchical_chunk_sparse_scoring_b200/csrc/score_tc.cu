@@ -402,6 +402,8 @@ cudaError_t launch_tc_k(const Dims& D, const void* qc, const void* klm, const fl
                         int32_t* idx, int32_t* status, cudaStream_t st) {
   // Two column groups: with four, the 18 warps cap a thread at 96 registers and the slower
   // epilogue (spills, fewer TMEM loads in flight) outweighs the extra latency hiding.
+  // the list length follows K: an insertion costs a compare and two selects per slot
+  if (D.K <= 8) return launch_tc_t<DD, G, 8, 2>(D, qc, klm, blm, idx, status, st);
   if (D.K <= 16) return launch_tc_t<DD, G, 16, 2>(D, qc, klm, blm, idx, status, st);
   return launch_tc_t<DD, G, 32, 2>(D, qc, klm, blm, idx, status, st);
 }
