@@ -48,17 +48,25 @@ struct AtShape {
   static constexpr int KV_BOX = kTile * 128;             // [64 tokens x 64]
   static constexpr int KV_BYTES = KB * KV_BOX;           // one K (or V) tile
   static constexpr int P_BYTES = kAtRows * 128;          // [128 rows x 64 tokens] bf16
-  static constexpr int STAGES = DD == 128 ? 3 : 4;
+  // K/V ring: STAGES_MAIN stage pairs of their own, plus one that reuses the calibrated-query
+  // tile once the selected chunks' scores have been taken from it (same size: Q_BYTES = 2 KV)
+  // d = 64: two CTAs per SM (each one's prologue and softmax latency hide behind the other's)
+  static constexpr int STAGES_MAIN = DD == 128 ? 3 : 2;
+  static constexpr int STAGES = STAGES_MAIN + 1;
+  static_assert(Q_BYTES == 2 * KV_BYTES, "the q_cal tile holds one K/V stage pair");
   static constexpr int KLM_ROWS = 64;                    // landmark rows staged in smem
   static constexpr int KLM_BYTES = KB * KLM_ROWS * 128;  // same swizzled layout as a K tile
-  static constexpr int FIXED = 2 * Q_BYTES /*q and q_cal*/ + STAGES * 2 * KV_BYTES +
+  static constexpr int FIXED = 2 * Q_BYTES /*q and q_cal*/ + STAGES_MAIN * 2 * KV_BYTES +
                                2 * P_BYTES + 1024 /*bars*/ + 1024 /*align*/ + 1024 /*scan*/;
   static_assert(KLM_BYTES <= 2 * P_BYTES, "landmark rows overlay the P buffers");
-  static constexpr uint32_t TMEM_COLS = 512;            // S[2] (2 x 64) + O (DD) + landmark S
+  // TMEM: S[2] (2 x 64 columns), O (DD), the landmark scores (64); a power of two
   static constexpr uint32_t O_COL = 128;
-  static constexpr uint32_t LM_COL = 256;
-  // 512 TMEM columns are the whole SM's: the shared memory footprint keeps a second CTA away
-  static_assert(FIXED > 232448 / 2, "one CTA per SM");
+  static constexpr uint32_t LM_COL = O_COL + DD;
+  static constexpr uint32_t TMEM_COLS = LM_COL + 64 <= 256 ? 256 : 512;
+  // co-resident CTAs never exceed the SM's 512 TMEM columns: d = 64 runs two CTAs per SM on 256
+  // columns each; d = 128 needs 512 and its shared memory footprint keeps a second CTA away
+  static_assert(DD == 64 ? (TMEM_COLS == 256 && FIXED < 232448 / 2 - 8192)
+                         : FIXED > 232448 / 2, "CTAs per SM");
 };
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -104,7 +112,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int& to
 }  // namespace
 
 template <int DD, int G, int KM>
-__global__ void __launch_bounds__(kAtThreads, 1)
+__global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQc,
                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    Dims D, const int32_t* __restrict__ idx, const __nv_bfloat16* __restrict__ klm,
@@ -119,8 +127,15 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   uint8_t* sQ = smem;
   uint8_t* sQc = sQ + SH::Q_BYTES;   // calibrated queries (surrogate scores of the selection)
   uint8_t* sK = sQc + SH::Q_BYTES;
-  uint8_t* sV = sK + SH::STAGES * SH::KV_BYTES;
-  uint8_t* sP = sV + SH::STAGES * SH::KV_BYTES;
+  uint8_t* sV = sK + SH::STAGES_MAIN * SH::KV_BYTES;
+  uint8_t* sP = sV + SH::STAGES_MAIN * SH::KV_BYTES;
+  // stage s of the K/V ring (the last one lives in the q_cal tile)
+  auto stage_k = [&](int s) -> uint8_t* {
+    return s < SH::STAGES_MAIN ? sK + s * SH::KV_BYTES : sQc;
+  };
+  auto stage_v = [&](int s) -> uint8_t* {
+    return s < SH::STAGES_MAIN ? sV + s * SH::KV_BYTES : sQc + SH::KV_BYTES;
+  };
   // landmark rows of the first 64 tiles (K-tile layout); dead once their product has completed,
   // before any P row is written
   uint8_t* sKlm = sP;
@@ -135,11 +150,13 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   uint64_t* o_done = p_empty + 2;
   uint64_t* o_final = o_done + 1;
   uint64_t* lm_done = o_final + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(lm_done + 1);
+  uint64_t* qc_free = lm_done + 1;   // every softmax warp is done reading the q_cal tile
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qc_free + 1);
   int* scan = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + 1024);   // [64]
   int* n_tiles_sh = scan + 64;
   int* tiles = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + 2048);  // [list_cap]
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(tiles + list_cap);             // [words]
+  int* wpre = reinterpret_cast<int*>(bitmap + bitmap_words);   // list position of each word
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t bg = blockIdx.y;
@@ -165,12 +182,25 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     mbar_init(o_done, 1);
     mbar_init(o_final, 1);
     mbar_init(lm_done, 1);
+    mbar_init(qc_free, 4);
     fence_barrier_init();
   }
   if (warp == 1) tmem_alloc(tmem_holder, SH::TMEM_COLS);
   const int nbw = (int)(last_chunk / 32) + 1;
   for (int w = threadIdx.x; w < nbw; w += kAtThreads) bitmap[w] = 0u;
   __syncthreads();
+  if (threadIdx.x == 0) {
+    // the query and calibrated-query tiles load while the tile list is built
+    prefetch_tensormap(&tmQ);
+    prefetch_tensormap(&tmQc);
+    mbar_expect_tx(q_full, 2 * SH::Q_BYTES);
+    for (int h = 0; h < G; ++h)
+      for (int kb = 0; kb < SH::KB; ++kb) {
+        const int32_t y = (int32_t)((b * D.Hq + g * G + h) * D.N_q + i0);
+        tma_load_2d(sQ + kb * SH::Q_BOX + h * TQ * 128, &tmQ, kb * 64, y, q_full);
+        tma_load_2d(sQc + kb * SH::Q_BOX + h * TQ * 128, &tmQc, kb * 64, y, q_full);
+      }
+  }
   // selected chunks of every valid query of the tile, and the chunks of the local windows
   for (int e = threadIdx.x; e < TQ * K; e += kAtThreads) {
     const int qi = e / K, k = e - qi * K;
@@ -193,6 +223,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     int pos = block_exclusive_scan(cnt, scan, total);
     for (int w = w0; w < w1; ++w) {
       uint32_t bits = bitmap[w];
+      wpre[w] = pos;
       while (bits) {
         const int bit = __ffs(bits) - 1;
         bits &= bits - 1;
@@ -214,31 +245,23 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
-      prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
-      prefetch_tensormap(&tmQc);
-      mbar_expect_tx(q_full, 2 * SH::Q_BYTES);
-      for (int h = 0; h < G; ++h)
-        for (int kb = 0; kb < SH::KB; ++kb) {
-          const int32_t y = (int32_t)((b * D.Hq + g * G + h) * D.N_q + i0);
-          tma_load_2d(sQ + kb * SH::Q_BOX + h * TQ * 128, &tmQ, kb * 64, y, q_full);
-          tma_load_2d(sQc + kb * SH::Q_BOX + h * TQ * 128, &tmQc, kb * 64, y, q_full);
-        }
       int last_s = -1;
       uint32_t last_par = 0;
       for (int t = 0; t < n_tiles; ++t) {
         const int s = t % SH::STAGES;
         const uint32_t u = (uint32_t)(t / SH::STAGES);
-        if (!mbar_wait(&kv_empty[s], (u & 1u) ^ 1u, kAtPollLimit)) {
+        if (!mbar_wait(&kv_empty[s], (u & 1u) ^ 1u, kAtPollLimit) ||
+            (t == SH::STAGES_MAIN && !mbar_wait(qc_free, 0, kAtPollLimit))) {
           record_status(status, kStatusTimeout);
           break;
         }
         mbar_expect_tx(&kv_full[s], 2 * SH::KV_BYTES);
         const int32_t y = (int32_t)(bg * D.N_kv + (int64_t)tiles[t] * kTile);
         for (int kb = 0; kb < SH::KB; ++kb) {
-          tma_load_2d(sK + s * SH::KV_BYTES + kb * SH::KV_BOX, &tmK, kb * 64, y, &kv_full[s]);
-          tma_load_2d(sV + s * SH::KV_BYTES + kb * SH::KV_BOX, &tmV, kb * 64, y, &kv_full[s]);
+          tma_load_2d(stage_k(s) + kb * SH::KV_BOX, &tmK, kb * 64, y, &kv_full[s]);
+          tma_load_2d(stage_v(s) + kb * SH::KV_BOX, &tmV, kb * 64, y, &kv_full[s]);
         }
         last_s = s;
         last_par = u & 1u;
@@ -264,7 +287,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
           const int kb = ks >> 2, kin = ks & 3;
           const uint64_t ad = desc_kmajor_sw128(smem_u32(sQ + kb * SH::Q_BOX) + kin * 32);
           const uint64_t bd =
-              desc_kmajor_sw128(smem_u32(sK + s * SH::KV_BYTES + kb * SH::KV_BOX) + kin * 32);
+              desc_kmajor_sw128(smem_u32(stage_k(s) + kb * SH::KV_BOX) + kin * 32);
           mma_bf16_ss(tmem + (uint32_t)(x * kTile), ad, bd, IDESC_QK, ks > 0 ? 1u : 0u);
         }
         mma_commit(&s_full[x]);
@@ -281,7 +304,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         for (int ks = 0; ks < kTile / 16; ++ks) {
           const uint64_t ad = desc_kmajor_sw128(smem_u32(sP + x * SH::P_BYTES) + ks * 32);
           const uint64_t bd = desc_mnmajor_sw128(
-              smem_u32(sV + s * SH::KV_BYTES) + ks * 16 * 128, SH::KV_BOX);
+              smem_u32(stage_v(s)) + ks * 16 * 128, SH::KV_BOX);
           mma_bf16_ss(tmem + SH::O_COL, ad, bd, IDESC_PV, (t > 0 || ks > 0) ? 1u : 0u);
         }
         mma_commit(&kv_empty[s]);
@@ -315,19 +338,6 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     // memory in the K-tile layout and one (128 x d) x (d x 64) product on the tensor core scores
     // every row of the tile against them; a chunk beyond those 64 is scored by a plain dot.
     const int nk = n_tiles < SH::KLM_ROWS ? n_tiles : SH::KLM_ROWS;
-    int slot[KM];
-    float bsel[KM];
-#pragma unroll
-    for (int k = 0; k < KM; ++k) {
-      int lo = 0, hi = nk;   // first tile >= c in [0, nk)
-      const int c = sc[k];
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (tiles[mid] < c) lo = mid + 1; else hi = mid;
-      }
-      slot[k] = (c >= 0 && lo < nk && tiles[lo] == c) ? lo : -1;
-      bsel[k] = (c >= 0 && c < D.C) ? __ldg(blm + bg * D.C + c) : 0.f;
-    }
     {
       constexpr int UPR = DD / 8;   // 16-byte units per landmark row
       const int tid = threadIdx.x - 64;
@@ -388,11 +398,15 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         su[k] = -INFINITY;
         const int c = sc[k];
         if (!lm_ok || c < 0 || c >= D.C) continue;
+        const float bias = __ldg(blm + bg * D.C + c);
+        // the chunk's position in the (sorted) tile list: the rank of its bit in the bitmap
+        const int rank = wpre[c >> 5] + __popc(bitmap[c >> 5] & ((1u << (c & 31)) - 1u));
+        const int slot = rank < nk ? rank : -1;
         float a;
-        if (slot[k] >= 0) {
-          const int col4 = slot[k] >> 2;
+        if (slot >= 0) {
+          const int col4 = slot >> 2;
           a = *reinterpret_cast<const float*>(park + (col4 >> 3) * SH::P_BYTES +
-                                              (((col4 & 7) + r) & 7) * 16 + (slot[k] & 3) * 4);
+                                              (((col4 & 7) + r) & 7) * 16 + (slot & 3) * 4);
         } else {
           const __nv_bfloat16* kr = klm + (bg * D.C + c) * DD;
           a = 0.f;
@@ -414,10 +428,13 @@ __global__ void __launch_bounds__(kAtThreads, 1)
             }
           }
         }
-        su[k] = fmaf(a, D.scale, bsel[k]);
+        su[k] = fmaf(a, D.scale, bias);
         m_run = fmaxf(m_run, su[k]);
       }
     }
+    // the q_cal tile is read for the last time above: it becomes a K/V stage
+    __syncwarp();
+    if (lane == 0) mbar_arrive(qc_free);
     if (!lm_ok) record_status(status, kStatusTimeout);
     float l = 0.f;
     const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
@@ -623,7 +640,7 @@ cudaError_t launch_at_t(const Dims& D, const void* q, const void* qc, const void
     return cudaErrorInvalidValue;
   const int cap = list_capacity(D, SH::TQ);
   const int words = (int)((D.N_kv / kTile) / 32) + 2;
-  const int smem = SH::FIXED + 1024 + cap * 4 + words * 4;
+  const int smem = SH::FIXED + 1024 + cap * 4 + 2 * words * 4;
   if (smem > kAtSmemLimit) return cudaErrorInvalidConfiguration;
   auto kern = attn_tc_kernel<DD, G, KM>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -658,7 +675,7 @@ bool attn_tc_supported(const Dims& D, bool bf16) {
   const int64_t words = (D.N_kv / kTile) / 32 + 2;
   const int fixed = D.d == 128 ? AtShape<128, 1>::FIXED : AtShape<64, 1>::FIXED;
   if (D.C >= (int64_t)INT32_MAX) return false;
-  return fixed + 1024 + (cap + words) * 4 <= kAtSmemLimit;
+  return fixed + 1024 + (cap + 2 * words) * 4 <= kAtSmemLimit;
 }
 
 cudaError_t launch_attn_tc(const Dims& D, const void* q, const void* qc, const void* K,

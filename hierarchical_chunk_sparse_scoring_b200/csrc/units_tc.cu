@@ -240,14 +240,18 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
       const bool tok_ok = (tk & 63) < (half ? lenb : lena);
       float* rm = red_m + ph * 4 * kUtCols;
       float* rl = red_l + ph * 4 * kUtCols;
-      // ---- logits of this thread's token for the 16 head columns
-      if (!mbar_wait_warp(s_full, ph, kUtPoll)) { ok = false; break; }
-      tc_fence_after();
+      // ---- logits of this thread's token for the 16 head columns.  A failed (timed-out) wait
+      // does not leave the loop: the four warps meet at named barriers on every tile, so after
+      // a failure a warp only skips its waits and TMEM accesses (ok is warp-uniform).
+      if (ok) ok = mbar_wait_warp(s_full, ph, kUtPoll);
       float x[kUtCols];
-      tmem_ld16(lane_base + kColS, x);
-      tmem_wait_ld();
+      if (ok) {
+        tc_fence_after();
+        tmem_ld16(lane_base + kColS, x);
+        tmem_wait_ld();
+      }
 #pragma unroll
-      for (int h = 0; h < kUtCols; ++h) x[h] = (tok_ok && h < G) ? x[h] * D.scale : -INFINITY;
+      for (int h = 0; h < kUtCols; ++h) x[h] = (ok && tok_ok && h < G) ? x[h] * D.scale : -INFINITY;
       // ---- unit max per head over the unit's two warps
 #pragma unroll
       for (int h = 0; h < kUtCols; ++h) {
@@ -280,10 +284,11 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (ok && lane == 0) mbar_arrive(p_full);
       asm volatile("bar.sync 1, 128;" ::: "memory");   // unit sums complete
       // ---- O of both units: this thread is d-row tk
-      if (!mbar_wait_warp(o_full, ph, kUtPoll)) { ok = false; break; }
+      if (ok) ok = mbar_wait_warp(o_full, ph, kUtPoll);
+      if (!ok) continue;
       tc_fence_after();
       float oa[kUtCols], ob[kUtCols];
       tmem_ld16(lane_base + kColOA, oa);
