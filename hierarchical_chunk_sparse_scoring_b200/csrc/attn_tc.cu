@@ -78,6 +78,34 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): two lanes of work per instruction.
+__device__ __forceinline__ void fma2(float& x0, float& x1, float b, float c) {   // x = x*b + c
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%0, %1};\n\tmov.b64 rb, {%2, %2};\n\tmov.b64 rd, {%3, %3};\n\t"
+      "fma.rn.f32x2 ra, ra, rb, rd;\n\tmov.b64 {%0, %1}, ra;\n\t}"
+      : "+f"(x0), "+f"(x1)
+      : "f"(b), "f"(c));
+}
+__device__ __forceinline__ void add2(float& s0, float& s1, float x0, float x1) {   // s += x
+  asm("{\n\t.reg .b64 ra, rb;\n\t"
+      "mov.b64 ra, {%0, %1};\n\tmov.b64 rb, {%2, %3};\n\t"
+      "add.rn.f32x2 ra, ra, rb;\n\tmov.b64 {%0, %1}, ra;\n\t}"
+      : "+f"(s0), "+f"(s1)
+      : "f"(x0), "f"(x1));
+}
+__device__ __forceinline__ void mul2(float& x0, float& x1, float b) {   // x *= b
+  asm("{\n\t.reg .b64 ra, rb;\n\t"
+      "mov.b64 ra, {%0, %1};\n\tmov.b64 rb, {%2, %2};\n\t"
+      "mul.rn.f32x2 ra, ra, rb;\n\tmov.b64 {%0, %1}, ra;\n\t}"
+      : "+f"(x0), "+f"(x1)
+      : "f"(b));
+}
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&t);
@@ -472,24 +500,34 @@ __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
       const float sc2 = D.scale * kLog2e;
       if (is_sel && u != -INFINITY) {
         // intra-chunk softmax of this chunk, weighted by exp(u - m_run) (u <= m_run)
+        // (three-input maxima, and fp32 pairs for the affine, sum and scale passes)
+        static_assert(kTile == 64, "eight groups of eight logits");
         float pm[8];
 #pragma unroll
-        for (int q8 = 0; q8 < 8; ++q8) pm[q8] = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < kTile; ++j) pm[j & 7] = fmaxf(pm[j & 7], p[j]);
-        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        for (int q8 = 0; q8 < 8; ++q8) {
+          pm[q8] = fmax3f(p[q8], p[q8 + 8], p[q8 + 16]);
+          pm[q8] = fmax3f(pm[q8], p[q8 + 24], p[q8 + 32]);
+          pm[q8] = fmax3f(pm[q8], p[q8 + 40], p[q8 + 48]);
+          pm[q8] = fmaxf(pm[q8], p[q8 + 56]);
+        }
+        const float mx = fmaxf(fmax3f(pm[0], pm[1], pm[2]),
+                               fmaxf(fmax3f(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7])));
         const float off = -mx * sc2;
         float ps[8];
 #pragma unroll
         for (int q8 = 0; q8 < 8; ++q8) ps[q8] = 0.f;
 #pragma unroll
-        for (int j = 0; j < kTile; ++j) { p[j] = fast_exp2(fmaf(p[j], sc2, off)); ps[j & 7] += p[j]; }
+        for (int j = 0; j < kTile; j += 2) {
+          fma2(p[j], p[j + 1], sc2, off);
+          p[j] = fast_exp2(p[j]);
+          p[j + 1] = fast_exp2(p[j + 1]);
+          add2(ps[j & 7], ps[(j & 7) + 1], p[j], p[j + 1]);
+        }
         const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
         const float w = fast_exp2((u - m_run) * kLog2e);
         const float f = w / sum;
 #pragma unroll
-        for (int j = 0; j < kTile; ++j) p[j] *= f;
+        for (int j = 0; j < kTile; j += 2) mul2(p[j], p[j + 1], f);
         l += w;
       } else if (is_win) {
         float pm[8];
@@ -510,14 +548,17 @@ __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
           }
           m_run = mt;
         }
-        const float off = -m_run * kLog2e;
+        // a masked logit (-inf) gives 2^-inf = 0, unless m_run is still -inf (no finite logit)
+        const float off = m_run == -INFINITY ? -INFINITY : -m_run * kLog2e;
         float ps[8];
 #pragma unroll
         for (int q8 = 0; q8 < 8; ++q8) ps[q8] = 0.f;
 #pragma unroll
-        for (int j = 0; j < kTile; ++j) {
-          p[j] = p[j] == -INFINITY ? 0.f : fast_exp2(fmaf(p[j], kLog2e, off));
-          ps[j & 7] += p[j];
+        for (int j = 0; j < kTile; j += 2) {
+          fma2(p[j], p[j + 1], kLog2e, off);
+          p[j] = fast_exp2(p[j]);
+          p[j + 1] = fast_exp2(p[j + 1]);
+          add2(ps[j & 7], ps[(j & 7) + 1], p[j], p[j + 1]);
         }
         l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       } else {
