@@ -106,6 +106,20 @@ __device__ __forceinline__ float fmax3f(float a, float b, float c) {
   return r;
 }
 
+// max of a row's 64 logits: eight independent three-input chains, then a short tree
+__device__ __forceinline__ float max64(const float (&p)[64]) {
+  float pm[8];
+#pragma unroll
+  for (int q8 = 0; q8 < 8; ++q8) {
+    pm[q8] = fmax3f(p[q8], p[q8 + 8], p[q8 + 16]);
+    pm[q8] = fmax3f(pm[q8], p[q8 + 24], p[q8 + 32]);
+    pm[q8] = fmax3f(pm[q8], p[q8 + 40], p[q8 + 48]);
+    pm[q8] = fmaxf(pm[q8], p[q8 + 56]);
+  }
+  return fmaxf(fmax3f(pm[0], pm[1], pm[2]), fmaxf(fmax3f(pm[3], pm[4], pm[5]),
+                                                 fmaxf(pm[6], pm[7])));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&t);
@@ -185,6 +199,10 @@ __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
   int* tiles = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + 2048);  // [list_cap]
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(tiles + list_cap);             // [words]
   int* wpre = reinterpret_cast<int*>(bitmap + bitmap_words);   // list position of each word
+  // per row, its selected chunks in tile-list order: (tile index, surrogate score) [128][KM]
+  constexpr bool kSelSmem = KM <= 16;
+  int* sel_t = wpre + bitmap_words;
+  float* sel_u = reinterpret_cast<float*>(sel_t + (kSelSmem ? kAtRows * KM : 0));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t bg = blockIdx.y;
@@ -460,11 +478,29 @@ __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
         m_run = fmaxf(m_run, su[k]);
       }
     }
+    int n_sel = 0;   // selected chunks of this row (kSelSmem: their tile indices are in sel_t)
+    if constexpr (kSelSmem) {
+      // order the row's selected chunks by chunk index, which is their order in the tile list
+#pragma unroll
+      for (int k = 0; k < KM; ++k) {
+        const int c = sc[k];
+        if (c < 0 || c >= D.C || su[k] == -INFINITY) continue;
+        int pos = 0;
+#pragma unroll
+        for (int k2 = 0; k2 < KM; ++k2)
+          pos += (sc[k2] >= 0 && sc[k2] < c && su[k2] != -INFINITY) ? 1 : 0;
+        sel_t[r * KM + pos] = wpre[c >> 5] + __popc(bitmap[c >> 5] & ((1u << (c & 31)) - 1u));
+        sel_u[r * KM + pos] = su[k];
+        ++n_sel;
+      }
+    }
     // the q_cal tile is read for the last time above: it becomes a K/V stage
     __syncwarp();
     if (lane == 0) mbar_arrive(qc_free);
     if (!lm_ok) record_status(status, kStatusTimeout);
     float l = 0.f;
+    int sel_next = 0;
+    int sel_tn = (kSelSmem && n_sel > 0) ? sel_t[r * KM] : -1;
     const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
     uint8_t* prow_base = sP + (r >> 3) * 1024 + (r & 7) * 128;
     bool ok = true;
@@ -489,9 +525,19 @@ __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
       const int c = tiles[t];
       float u = -INFINITY;
       bool is_sel = false;
+      if constexpr (kSelSmem) {
+        // the next selected chunk of this row, in list order
+        if (sel_next < n_sel && sel_tn == t) {
+          is_sel = true;
+          u = sel_u[r * KM + sel_next];
+          ++sel_next;
+          sel_tn = sel_next < n_sel ? sel_t[r * KM + sel_next] : -1;
+        }
+      } else {
 #pragma unroll
-      for (int k = 0; k < KM; ++k)
-        if (sc[k] == c) { is_sel = true; u = su[k]; }
+        for (int k = 0; k < KM; ++k)
+          if (sc[k] == c) { is_sel = true; u = su[k]; }
+      }
       const int64_t t0 = (int64_t)c * kTile;
       const bool is_win = valid && !is_sel && c >= n_i && t0 <= pos;
       bool rescale = false;
@@ -501,17 +547,7 @@ __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
       if (is_sel && u != -INFINITY) {
         // intra-chunk softmax of this chunk, weighted by exp(u - m_run) (u <= m_run)
         // (three-input maxima, and fp32 pairs for the affine, sum and scale passes)
-        static_assert(kTile == 64, "eight groups of eight logits");
-        float pm[8];
-#pragma unroll
-        for (int q8 = 0; q8 < 8; ++q8) {
-          pm[q8] = fmax3f(p[q8], p[q8 + 8], p[q8 + 16]);
-          pm[q8] = fmax3f(pm[q8], p[q8 + 24], p[q8 + 32]);
-          pm[q8] = fmax3f(pm[q8], p[q8 + 40], p[q8 + 48]);
-          pm[q8] = fmaxf(pm[q8], p[q8 + 56]);
-        }
-        const float mx = fmaxf(fmax3f(pm[0], pm[1], pm[2]),
-                               fmaxf(fmax3f(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        const float mx = max64(p);
         const float off = -mx * sc2;
         float ps[8];
 #pragma unroll
@@ -530,16 +566,13 @@ __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
         for (int j = 0; j < kTile; j += 2) mul2(p[j], p[j + 1], f);
         l += w;
       } else if (is_win) {
-        float pm[8];
+        // raw logits; only the tile holding the query's own position needs the causal mask
+        if (t0 + kTile - 1 > pos) {
 #pragma unroll
-        for (int q8 = 0; q8 < 8; ++q8) pm[q8] = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < kTile; ++j) {
-          p[j] = (t0 + j <= pos) ? p[j] * D.scale : -INFINITY;
-          pm[j & 7] = fmaxf(pm[j & 7], p[j]);
+          for (int j = 0; j < kTile; ++j)
+            if (t0 + j > pos) p[j] = -INFINITY;
         }
-        const float mt = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        const float mt = max64(p) * D.scale;   // scale > 0
         if (mt > m_run + kRescaleMargin) {
           if (l > 0.f) {
             factor = fast_exp2((m_run - mt) * kLog2e);
@@ -555,7 +588,7 @@ __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
         for (int q8 = 0; q8 < 8; ++q8) ps[q8] = 0.f;
 #pragma unroll
         for (int j = 0; j < kTile; j += 2) {
-          fma2(p[j], p[j + 1], kLog2e, off);
+          fma2(p[j], p[j + 1], sc2, off);
           p[j] = fast_exp2(p[j]);
           p[j + 1] = fast_exp2(p[j + 1]);
           add2(ps[j & 7], ps[(j & 7) + 1], p[j], p[j + 1]);
@@ -681,7 +714,7 @@ cudaError_t launch_at_t(const Dims& D, const void* q, const void* qc, const void
     return cudaErrorInvalidValue;
   const int cap = list_capacity(D, SH::TQ);
   const int words = (int)((D.N_kv / kTile) / 32) + 2;
-  const int smem = SH::FIXED + 1024 + cap * 4 + 2 * words * 4;
+  const int smem = SH::FIXED + 1024 + cap * 4 + 2 * words * 4 + (KM <= 16 ? kAtRows * KM * 8 : 0);
   if (smem > kAtSmemLimit) return cudaErrorInvalidConfiguration;
   auto kern = attn_tc_kernel<DD, G, KM>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -716,7 +749,9 @@ bool attn_tc_supported(const Dims& D, bool bf16) {
   const int64_t words = (D.N_kv / kTile) / 32 + 2;
   const int fixed = D.d == 128 ? AtShape<128, 1>::FIXED : AtShape<64, 1>::FIXED;
   if (D.C >= (int64_t)INT32_MAX) return false;
-  return fixed + 1024 + (cap + 2 * words) * 4 <= kAtSmemLimit;
+  const int km = D.K <= 8 ? 8 : (D.K <= 16 ? 16 : 32);
+  const int64_t sel_bytes = km <= 16 ? (int64_t)kAtRows * km * 8 : 0;
+  return fixed + 1024 + (cap + 2 * words) * 4 + sel_bytes <= kAtSmemLimit;
 }
 
 cudaError_t launch_attn_tc(const Dims& D, const void* q, const void* qc, const void* K,
