@@ -363,7 +363,9 @@ def extra_prefill(name, steps, peaks, **overrides):
     es = wl.q.element_size()
     wm = work_model(wl.dims, wl.S, wl.K_top, wl.W, wl.q_pos0, es)
     t = statistics.mean(step_ms)
+    G = wl.q.shape[1] // wl.K.shape[1]
     res = {"workload": name, "ms_per_step": t, "tokens_per_s": wm["tokens"] / (t * 1e-3),
+           "union_per_K_128_rows": union_stat(run.idx, 128 // G, wl.K.shape[2] // wl.S),
            "phases_ms": phase_ms,
            "rooflines": [roofline(k, v, wm, peaks, name) for k, v in phase_ms.items()],
            "score_tflop": wm["score_flops"] / 1e12, "attn_tflop": wm["attn_flops"] / 1e12}
@@ -417,6 +419,54 @@ def extra_decode(steps, peaks, **overrides):
     return res
 
 
+def union_stat(idx, tq, C):
+    """Mean number of distinct chunks selected by tq adjacent queries of a KV group, divided by
+    K (how much the packed attention shares chunk loads)."""
+    R, Nq, K = idx.shape[0] * idx.shape[1], idx.shape[2], idx.shape[3]
+    nt = Nq // tq
+    if nt == 0 or K == 0:
+        return None
+    x = idx.reshape(R, Nq, K)[:, :nt * tq].reshape(R * nt, tq * K).long()
+    valid = (x >= 0) & (x < C)
+    hit = torch.zeros((R * nt, C + 1), dtype=torch.bool, device=idx.device)
+    hit.scatter_(1, torch.where(valid, x, torch.full_like(x, C)), True)
+    sizes = hit[:, :C].sum(1).float()
+    return float(sizes.mean().item()) / K
+
+
+def extra_extreme(steps, peaks, N=262144):
+    """The extreme-length sweep's first point: prefill of the whole sequence and one decode
+    step of its last query, on the same inputs."""
+    from hierarchical_chunk_sparse_scoring_b200 import workloads as W
+    wl = W.make("extreme", "cuda", N=N)
+    res = {"workload": "extreme", "N": N}
+    for mode in ("prefill", "decode"):
+        if mode == "decode":
+            wl = W.Workload("extreme_decode", wl.q[:, :, -1:].contiguous(),
+                            wl.q_cal[:, :, -1:].contiguous(), wl.K, wl.V, wl.k_lm, wl.b_lm,
+                            wl.S, wl.K_top, wl.W, q_pos0=N - 1)
+        run = Runner(wl)
+        flush = make_flush(wl.q.device)
+        run()
+        torch.cuda.synchronize()
+        step_ms, phase_ms = timed_steps(run, steps, flush)
+        wm = work_model(wl.dims, wl.S, wl.K_top, wl.W, wl.q_pos0, wl.q.element_size())
+        t = statistics.mean(step_ms)
+        res[mode] = {"ms_per_step": t, "phases_ms": phase_ms,
+                     "rooflines": [roofline(k, v, wm, peaks, "extreme_%s" % mode)
+                                   for k, v in phase_ms.items()]}
+        if mode == "prefill":
+            res[mode]["tokens_per_s"] = wm["tokens"] / (t * 1e-3)
+            res[mode]["score_tflop"] = wm["score_flops"] / 1e12
+            res[mode]["attn_tflop"] = wm["attn_flops"] / 1e12
+        else:
+            res[mode]["us_per_step"] = t * 1e3
+        del run
+    del wl
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_hils(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -461,6 +511,8 @@ def run_hils(args):
         "peaks_source": peaks_src,
         "phases_ms": phase_ms,
         "gpu_launches": len(run.phases) * args.steps,
+        "union_per_K_128_rows": union_stat(run.idx, 128 // (wl.q.shape[1] // wl.K.shape[1]),
+                                           wl.K.shape[2] // wl.S),
         "clocks": clk.summary(),
     }
     if world == 1 and not args.no_extras:
@@ -469,6 +521,7 @@ def run_hils(args):
         torch.cuda.empty_cache()
         line["prefill_gqa7b"] = extra_prefill("gqa7b_prefill", 3, peaks)
         line["decode"] = extra_decode(max(5, args.steps), peaks)
+        line["extreme_256k"] = extra_extreme(2, peaks)
         rate, rows, threads, dt = oracle_sample_rate(wl, args.cpu_seconds)
         line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": threads,
                                 "kind": "oracle",

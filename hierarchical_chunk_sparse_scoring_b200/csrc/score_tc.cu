@@ -17,6 +17,12 @@
 //              column groups of each tile, so every query has NCG partial top-K lists, merged
 //              pairwise at the end.  Candidates that reach the best of the NCG lists' current
 //              K-th values are inserted into the thread's sorted register list.
+//
+// Head pairs (HP = 2, used for G = 8 at d = 128, where the G query tiles of 128 rows would not fit
+// in shared memory): the 128 MMA rows are 64 queries x 2 heads, interleaved (row 2q + e is query
+// q, head 2m + e of accumulator m), loaded by a 3-D TMA box; G/2 accumulators per tile.  Each
+// query's score is the max over its two lanes (one shuffle) and the two lanes split the columns,
+// so a query has four partial lists (two lanes x two column halves), merged at the end.
 // Every mbarrier wait gives up after a bounded number of polls and records HILS_ERR_TIMEOUT.
 #include <cudaTypedefs.h>
 
@@ -40,14 +46,16 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 constexpr uint32_t kPollLimit = 1u << 24;
 constexpr int kSmemLimit = 227 * 1024;
 
-template <int DD, int G, int KM, int NCG>
+template <int DD, int G, int KM, int NCG, int HP>
 struct TcShape {
   static constexpr int THREADS = 64 + 128 * NCG;
   static constexpr int EPI = 128 * NCG;                       // epilogue threads
-  static constexpr int NT = 256 / G < 256 ? 256 / G : 256;   // chunks per tile
+  static constexpr int MQ = kRows / HP;                       // queries per CTA
+  static constexpr int GV = G / HP;                           // accumulators per tile
+  static constexpr int NT = 256 / GV < 256 ? 256 / GV : 256;  // chunks per tile
   static constexpr int KB = DD / 64;                          // 128-byte boxes along d
   static constexpr int A_BOX = kRows * 128;
-  static constexpr int A_BYTES = G * KB * A_BOX;
+  static constexpr int A_BYTES = GV * KB * A_BOX;
   static constexpr int B_BOX = NT * 128;
   static constexpr int B_STAGE = KB * B_BOX;
   static constexpr int STASH_A = 16 * EPI * 4;                  // 16 scores per thread
@@ -62,24 +70,26 @@ struct TcShape {
   static constexpr int SMEM_USED = FIXED + STAGES * B_STAGE;
   static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
   static constexpr int CG = NT / NCG;                          // columns per epilogue warp
-  static constexpr int HG = G < 4 ? G : 4;   // heads whose TMEM loads are in flight together
-  static constexpr uint32_t TMEM_COLS = 2 * G * NT;
+  static constexpr int HG = GV < 4 ? GV : 4;   // accumulators whose TMEM loads are in flight
+  static constexpr uint32_t TMEM_COLS = 2 * GV * NT;
   static_assert(TMEM_COLS == 512, "two accumulator sets fill TMEM");
   static_assert(STAGES >= 2, "shared memory too small for this shape");
   static_assert(CG % 16 == 0, "sub-blocks of 16 columns");
   static_assert(NCG == 2 || NCG == 4, "two or four column groups");
+  static_assert(HP == 1 || (HP == 2 && G % 2 == 0), "head pairs");
 };
 
 }  // namespace
 
-template <int DD, int G, int KM, int NCG>
+template <int DD, int G, int KM, int NCG, int HP>
 __global__ void __launch_bounds__(64 + 128 * NCG, 1)
     score_topk_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB, Dims D,
                          const float* __restrict__ blm, int32_t* __restrict__ idx,
                          int32_t* __restrict__ status) {
-  using SH = TcShape<DD, G, KM, NCG>;
+  using SH = TcShape<DD, G, KM, NCG, HP>;
   constexpr int NT = SH::NT;
+  constexpr int GV = SH::GV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -106,8 +116,8 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
   const int64_t qt = (int64_t)gridDim.x - 1 - blockIdx.x;   // longest query tiles first
   const int64_t bg = blockIdx.y;
   const int64_t g = bg % D.Hkv, b = bg / D.Hkv;
-  const int64_t i0 = qt * kRows;
-  const int64_t i_last = (i0 + kRows - 1 < D.N_q - 1) ? i0 + kRows - 1 : D.N_q - 1;
+  const int64_t i0 = qt * SH::MQ;
+  const int64_t i_last = (i0 + SH::MQ - 1 < D.N_q - 1) ? i0 + SH::MQ - 1 : D.N_q - 1;
   const int64_t n_max = n_eligible(D.q_pos0 + i_last, D.S, D.W);
   const int n_tiles = (int)((n_max + NT - 1) / NT);
   const int K = D.K;
@@ -137,10 +147,23 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
       prefetch_tensormap(&tmA);
       prefetch_tensormap(&tmB);
       mbar_expect_tx(a_full, SH::A_BYTES);
-      for (int h = 0; h < G; ++h)
-        for (int kb = 0; kb < SH::KB; ++kb)
-          tma_load_2d(sA + (h * SH::KB + kb) * SH::A_BOX, &tmA, kb * 64,
-                      (int32_t)((b * D.Hq + g * G + h) * D.N_q + i0), a_full);
+      for (int h = 0; h < GV; ++h)
+        for (int kb = 0; kb < SH::KB; ++kb) {
+          if constexpr (HP == 1) {
+            tma_load_2d(sA + (h * SH::KB + kb) * SH::A_BOX, &tmA, kb * 64,
+                        (int32_t)((b * D.Hq + g * G + h) * D.N_q + i0), a_full);
+          } else {
+            // [64 queries][2 heads][64] from the (d, head, query) view of q_cal
+            asm volatile(
+                "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+                " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+                    smem_u32(sA + (h * SH::KB + kb) * SH::A_BOX)),
+                "l"(reinterpret_cast<uint64_t>(&tmA)), "r"(kb * 64),
+                "r"((int32_t)(b * D.Hq + g * G + 2 * h)), "r"((int32_t)i0),
+                "r"(smem_u32(a_full))
+                : "memory");
+          }
+        }
       int last_s = -1;
       uint32_t last_par = 0;
       for (int t = 0; t < n_tiles; ++t) {
@@ -182,8 +205,8 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const uint32_t d_tmem = tmem + (uint32_t)((a * G + h) * NT);
+        for (int h = 0; h < GV; ++h) {
+          const uint32_t d_tmem = tmem + (uint32_t)((a * GV + h) * NT);
 #pragma unroll
           for (int ks = 0; ks < DD / 16; ++ks) {
             const int kb = ks >> 2, kin = ks & 3;
@@ -204,8 +227,8 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
     const int e = warp - 2;                 // 0 .. 4*NCG-1
     const int qd = warp & 3;                // TMEM lane quadrant this warp may access
     const int ch = e >> 2;                  // which column group of each tile
-    const int r = qd * 32 + lane;           // query row within the tile
-    const int64_t i = i0 + r;
+    const int r = qd * 32 + lane;           // MMA row (TMEM lane) of this thread
+    const int64_t i = i0 + r / HP;          // its query
     const bool valid = i < D.N_q;
     const int64_t n_i = valid ? n_eligible(D.q_pos0 + i, D.S, D.W) : 0;
     const float* bb = blm + bg * D.C;
@@ -240,11 +263,11 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
         float sig[16];
         constexpr int HG = SH::HG;
 #pragma unroll
-        for (int h0 = 0; h0 < G; h0 += HG) {
+        for (int h0 = 0; h0 < GV; h0 += HG) {
           float tmp[HG][16];
 #pragma unroll
           for (int hh = 0; hh < HG; ++hh)
-            tmem_ld16(lane_base + (uint32_t)((a * G + h0 + hh) * NT + col0), tmp[hh]);
+            tmem_ld16(lane_base + (uint32_t)((a * GV + h0 + hh) * NT + col0), tmp[hh]);
           tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
@@ -256,6 +279,11 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
             if (hh < HG) sig[j] = fmaxf(sig[j], tmp[hh][j]);
           }
         }
+        if constexpr (HP == 2) {
+          // the other head of each pair sits in the neighbouring lane
+#pragma unroll
+          for (int j = 0; j < 16; ++j) sig[j] = fmaxf(sig[j], __shfl_xor_sync(0xffffffffu, sig[j], 1));
+        }
         // a candidate must reach every group's current K-th best (each list already holds K
         // candidates at least that good); exact ties at the threshold are passed on and
         // resolved by the insertion itself
@@ -264,8 +292,16 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
         for (int o = 1; o < NCG; ++o)
           thr = fmaxf(thr, *reinterpret_cast<const volatile float*>(
                                th_v + ((ch + o) & (NCG - 1)) * kRows + r));
+        if constexpr (HP == 2) {
+          // the partner lane's lists serve the same query
+#pragma unroll
+          for (int o = 0; o < NCG; ++o)
+            thr = fmaxf(thr, *reinterpret_cast<const volatile float*>(
+                                 th_v + ((ch + o) & (NCG - 1)) * kRows + (r ^ 1)));
+        }
         const int64_t left = n_i - c0;
-        const uint32_t vmask = left >= 16 ? 0xFFFFu : (left <= 0 ? 0u : (1u << left) - 1u);
+        uint32_t vmask = left >= 16 ? 0xFFFFu : (left <= 0 ? 0u : (1u << left) - 1u);
+        if constexpr (HP == 2) vmask &= (lane & 1) ? 0xFF00u : 0x00FFu;   // the pair splits columns
         const float4* sbt = reinterpret_cast<const float4*>(sbias + bs * NT + col0);
 #pragma unroll
         for (int j4 = 0; j4 < 4; ++j4) {
@@ -336,7 +372,23 @@ __global__ void __launch_bounds__(64 + 128 * NCG, 1)
         }
       }
     }
-    if (ch == 0 && valid) {
+    if constexpr (HP == 2) {
+      // then the odd lane of each pair hands its (merged) list to the even lane
+      asm volatile("bar.sync 1, %0;" ::"n"(SH::EPI) : "memory");
+      if (ch == 0 && (r & 1)) {
+#pragma unroll
+        for (int k = 0; k < KM; ++k) { xv[r * KM + k] = L.v[k]; xc[r * KM + k] = L.c[k]; }
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(SH::EPI) : "memory");
+      if (ch == 0 && !(r & 1)) {
+        const int o = (r + 1) * KM;
+        for (int k = KM - K; k < KM; ++k) {
+          const int c = xc[o + k];
+          if (c != INT_MAX) L.insert(xv[o + k], c);
+        }
+      }
+    }
+    if (ch == 0 && valid && (HP == 1 || !(r & 1))) {
       int32_t* out = idx + (bg * D.N_q + i) * K - (KM - K);
 #pragma unroll
       for (int k = 0; k < KM; ++k)
@@ -380,19 +432,34 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t d, uin
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int DD, int G, int KM, int NCG>
+template <int DD, int G, int KM, int NCG, int HP>
 cudaError_t launch_tc_t(const Dims& D, const void* qc, const void* klm, const float* blm,
                         int32_t* idx, int32_t* status, cudaStream_t st) {
-  using SH = TcShape<DD, G, KM, NCG>;
+  using SH = TcShape<DD, G, KM, NCG, HP>;
   CUtensorMap tmA, tmB;
-  if (!make_map(&tmA, qc, (uint64_t)(D.B * D.Hq * D.N_q), DD, kRows) ||
-      !make_map(&tmB, klm, (uint64_t)(D.B * D.Hkv * (D.C > 0 ? D.C : 1)), DD, SH::NT))
+  bool ok_a;
+  if constexpr (HP == 1) {
+    ok_a = make_map(&tmA, qc, (uint64_t)(D.B * D.Hq * D.N_q), DD, kRows);
+  } else {
+    // q_cal viewed as (d, head [stride N_q d], query [stride d]): a box of 64 queries x 2 heads
+    // lands as 128 rows ordered (query, head)
+    auto enc = get_encode();
+    cuuint64_t dims[3] = {(cuuint64_t)DD, (cuuint64_t)(D.B * D.Hq), (cuuint64_t)D.N_q};
+    cuuint64_t strides[2] = {(cuuint64_t)(D.N_q * DD * 2), (cuuint64_t)DD * 2};
+    cuuint32_t box[3] = {64, 2, (cuuint32_t)SH::MQ};
+    cuuint32_t estr[3] = {1, 1, 1};
+    ok_a = enc && enc(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(qc), dims,
+                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
+  if (!ok_a || !make_map(&tmB, klm, (uint64_t)(D.B * D.Hkv * (D.C > 0 ? D.C : 1)), DD, SH::NT))
     return cudaErrorInvalidValue;
-  auto kern = score_topk_tc_kernel<DD, G, KM, NCG>;
+  auto kern = score_topk_tc_kernel<DD, G, KM, NCG, HP>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SH::SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((D.N_q + kRows - 1) / kRows), (unsigned)(D.B * D.Hkv));
+  dim3 grid((unsigned)((D.N_q + SH::MQ - 1) / SH::MQ), (unsigned)(D.B * D.Hkv));
   kern<<<grid, SH::THREADS, SH::SMEM, st>>>(tmA, tmB, D, blm, idx, status);
   return cudaGetLastError();
 }
@@ -403,9 +470,11 @@ cudaError_t launch_tc_k(const Dims& D, const void* qc, const void* klm, const fl
   // Two column groups: with four, the 18 warps cap a thread at 96 registers and the slower
   // epilogue (spills, fewer TMEM loads in flight) outweighs the extra latency hiding.
   // the list length follows K: an insertion costs a compare and two selects per slot
-  if (D.K <= 8) return launch_tc_t<DD, G, 8, 2>(D, qc, klm, blm, idx, status, st);
-  if (D.K <= 16) return launch_tc_t<DD, G, 16, 2>(D, qc, klm, blm, idx, status, st);
-  return launch_tc_t<DD, G, 32, 2>(D, qc, klm, blm, idx, status, st);
+  // eight heads of 128 dimensions: head pairs (the eight query tiles would not fit)
+  constexpr int HP = (G == 8 && DD == 128) ? 2 : 1;
+  if (D.K <= 8) return launch_tc_t<DD, G, 8, 2, HP>(D, qc, klm, blm, idx, status, st);
+  if (D.K <= 16) return launch_tc_t<DD, G, 16, 2, HP>(D, qc, klm, blm, idx, status, st);
+  return launch_tc_t<DD, G, 32, 2, HP>(D, qc, klm, blm, idx, status, st);
 }
 
 }  // namespace
@@ -413,7 +482,7 @@ cudaError_t launch_tc_k(const Dims& D, const void* qc, const void* klm, const fl
 bool score_tc_supported(const Dims& D, bool bf16) {
   if (!bf16 || D.K < 1 || D.K > kMaxK || D.C < 1) return false;
   if (D.B * D.Hkv > 65535) return false;
-  if (D.d == 128) return D.G == 1 || D.G == 2 || D.G == 4;
+  if (D.d == 128) return D.G == 1 || D.G == 2 || D.G == 4 || D.G == 8;
   if (D.d == 64) return D.G == 1 || D.G == 2 || D.G == 4 || D.G == 8;
   return false;
 }
@@ -425,7 +494,8 @@ cudaError_t launch_score_topk_tc(const Dims& D, const void* qc, const void* klm,
   if (D.d == 128) {
     if (D.G == 1) return launch_tc_k<128, 1>(D, qc, klm, blm, idx, status, st);
     if (D.G == 2) return launch_tc_k<128, 2>(D, qc, klm, blm, idx, status, st);
-    return launch_tc_k<128, 4>(D, qc, klm, blm, idx, status, st);
+    if (D.G == 4) return launch_tc_k<128, 4>(D, qc, klm, blm, idx, status, st);
+    return launch_tc_k<128, 8>(D, qc, klm, blm, idx, status, st);
   }
   if (D.G == 1) return launch_tc_k<64, 1>(D, qc, klm, blm, idx, status, st);
   if (D.G == 2) return launch_tc_k<64, 2>(D, qc, klm, blm, idx, status, st);

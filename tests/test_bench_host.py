@@ -69,3 +69,11 @@ def test_clock_summary_decodes_reasons():
     assert c.summary()["reasons"] == ["hw_slowdown", "hw_thermal_slowdown"]
     c.rows = []
     assert c.summary() is None
+
+
+def test_union_stat_counts_distinct_chunks():
+    import torch
+    # one KV group, 4 queries, K = 2; tiles of 2 queries
+    idx = torch.tensor([[[[0, 1], [1, 2], [5, -1], [5, 6]]]], dtype=torch.int32)
+    # tile 0: {0, 1, 2} -> 3; tile 1: {5, 6} -> 2; mean 2.5 / K
+    assert bench.union_stat(idx, 2, C=8) == 2.5 / 2

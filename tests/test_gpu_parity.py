@@ -101,6 +101,10 @@ EDGE_CASES = {
     "tc_g4_k32": dict(B=1, Hq=8, Hkv=2, N=6000, d=128, S=64, K=32, W_=128),
     "tc_s128": dict(B=1, Hq=4, Hkv=1, N=9000, d=128, S=128, K=16, W_=256),
     "tc_many_tiles": dict(B=1, Hq=4, Hkv=4, N=20000, d=64, S=16, K=8, W_=64),
+    # eight heads of 128 dimensions (head-pair scoring), with S = 64 and the extreme shape S = 128
+    "tc_g8_d128": dict(B=1, Hq=8, Hkv=1, N=3000, d=128, S=64, K=16, W_=128),
+    "tc_g8_d128_s128": dict(B=1, Hq=8, Hkv=1, N=6000, d=128, S=128, K=16, W_=256),
+    "tc_g8_d128_k8_b2": dict(B=2, Hq=16, Hkv=2, N=2100, d=128, S=64, K=8, W_=64),
 }
 
 
