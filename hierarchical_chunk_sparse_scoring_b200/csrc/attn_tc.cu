@@ -1,4 +1,8 @@
-// Steps 3-4 for prefill on the tcgen05 tensor cores (bf16 inputs, fp32 accumulation, S = 64).
+// Steps 3-4 for prefill on the tcgen05 tensor cores (bf16 inputs, fp32 accumulation, S = 64 or
+// 128).  The unit of work is a tile of 64 tokens; with S = 128 a chunk is two adjacent tiles of
+// the list, and its intra-chunk softmax is taken over both at the first one (the second tile's
+// logits are already in the other S buffer of TMEM): the first tile's P and the second's share
+// one max and one normaliser.
 //
 // [Reader] "Implementation and Training Recipes", Figure 4: pack M adjacent queries and the G
 // heads of their KV group into one tile of M*G rows and attend the union of the rows' chunks,
@@ -153,7 +157,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int& to
 
 }  // namespace
 
-template <int DD, int G, int KM>
+template <int DD, int G, int KM, int RS>
 __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQc,
                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -212,7 +216,8 @@ __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
   const int64_t p_first = D.q_pos0 + i0;
   const int64_t p_max = D.q_pos0 + i_last;
   const int64_t n_first = n_eligible(p_first, D.S, D.W);
-  const int64_t last_chunk = p_max / kTile;
+  const int64_t last_chunk = p_max / kTile;   // last tile (64 tokens) any window reaches
+  constexpr int rs = RS;                       // tiles per chunk = 1 << rs
   const int K = D.K;
 
   // ---------------------------------------------------------------- barriers, TMEM, tile list
@@ -253,10 +258,15 @@ __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
     const int64_t i = i0 + qi;
     if (i < D.N_q) {
       const int c = idx[(bg * D.N_q + i) * K + k];
-      if (c >= 0 && c < D.C) atomicOr(&bitmap[c >> 5], 1u << (c & 31));
+      if (c >= 0 && c < D.C) {
+        for (int e2 = 0; e2 <= rs; ++e2) {
+          const int tl = (c << rs) + e2;
+          atomicOr(&bitmap[tl >> 5], 1u << (tl & 31));
+        }
+      }
     }
   }
-  for (int64_t c = n_first + threadIdx.x; c <= last_chunk; c += kAtThreads)
+  for (int64_t c = (n_first << rs) + threadIdx.x; c <= last_chunk; c += kAtThreads)
     atomicOr(&bitmap[c >> 5], 1u << (c & 31));
   __syncthreads();
   {
@@ -391,7 +401,7 @@ __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
 #pragma unroll
       for (int e = 0; e < SH::KLM_ROWS * UPR / 128; ++e) {
         const int f = tid + e * 128, t = f / UPR, j = f - t * UPR;
-        const int c = t < nk ? tiles[t] : D.C;
+        const int c = t < nk ? (tiles[t] >> rs) : D.C;   // the tile's chunk
         u[e] = c < D.C ? __ldg(reinterpret_cast<const uint4*>(klm + (bg * D.C + c) * DD) + j)
                        : make_uint4(0u, 0u, 0u, 0u);
       }
@@ -446,7 +456,8 @@ __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
         if (!lm_ok || c < 0 || c >= D.C) continue;
         const float bias = __ldg(blm + bg * D.C + c);
         // the chunk's position in the (sorted) tile list: the rank of its bit in the bitmap
-        const int rank = wpre[c >> 5] + __popc(bitmap[c >> 5] & ((1u << (c & 31)) - 1u));
+        const int tc = c << rs;   // the chunk's first tile
+        const int rank = wpre[tc >> 5] + __popc(bitmap[tc >> 5] & ((1u << (tc & 31)) - 1u));
         const int slot = rank < nk ? rank : -1;
         float a;
         if (slot >= 0) {
@@ -489,7 +500,8 @@ __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
 #pragma unroll
         for (int k2 = 0; k2 < KM; ++k2)
           pos += (sc[k2] >= 0 && sc[k2] < c && su[k2] != -INFINITY) ? 1 : 0;
-        sel_t[r * KM + pos] = wpre[c >> 5] + __popc(bitmap[c >> 5] & ((1u << (c & 31)) - 1u));
+        const int tc = c << rs;   // the chunk's first tile
+        sel_t[r * KM + pos] = wpre[tc >> 5] + __popc(bitmap[tc >> 5] & ((1u << (tc & 31)) - 1u));
         sel_u[r * KM + pos] = su[k];
         ++n_sel;
       }
@@ -499,6 +511,8 @@ __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
     if (lane == 0) mbar_arrive(qc_free);
     if (!lm_ok) record_status(status, kStatusTimeout);
     float l = 0.f;
+    bool sec_pending = false;   // S = 128: this row's next tile is the second half of its chunk
+    float sec_off = 0.f, sec_f = 0.f;
     int sel_next = 0;
     int sel_tn = (kSelSmem && n_sel > 0) ? sel_t[r * KM] : -1;
     const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
@@ -522,9 +536,11 @@ __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[x]);
 
-      const int c = tiles[t];
+      const int c = tiles[t];   // tile index (64 tokens)
       float u = -INFINITY;
       bool is_sel = false;
+      const bool is_second = sec_pending;
+      sec_pending = false;
       if constexpr (kSelSmem) {
         // the next selected chunk of this row, in list order
         if (sel_next < n_sel && sel_tn == t) {
@@ -536,18 +552,64 @@ __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
       } else {
 #pragma unroll
         for (int k = 0; k < KM; ++k)
-          if (sc[k] == c) { is_sel = true; u = su[k]; }
+          if (sc[k] >= 0 && (sc[k] << rs) == c) { is_sel = true; u = su[k]; }
       }
       const int64_t t0 = (int64_t)c * kTile;
-      const bool is_win = valid && !is_sel && c >= n_i && t0 <= pos;
+      const bool is_win = valid && !is_sel && !is_second && c >= (n_i << rs) && t0 <= pos;
+      // S = 128: the first tile of a selected chunk also reads the second tile's logits
+      const bool first2 = RS && is_sel && u != -INFINITY && t + 1 < n_tiles;
+      // (TMEM loads are warp-collective: every lane runs these passes, a lane without a first
+      // half of its own ignores the results)
+      const float sc2 = D.scale * kLog2e;
+      float mxc = 0.f;          // the chunk's max over both tiles (raw logits)
+      float sum2_raw = 0.f;     // the second tile's exponentials' sum against that max
+      const int x2 = x ^ 1;
+      const bool need2 = RS && __any_sync(0xffffffffu, first2);
+      if (need2) {
+        if (!mbar_wait_warp(&s_full[x2], (uint32_t)((t + 1) >> 1) & 1u, kAtPollLimit)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float mx2 = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < kTile / 16; ++j) {
+          float tmp[16];
+          tmem_ld16(lane_base + (uint32_t)(x2 * kTile + 16 * j), tmp);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) mx2 = fmaxf(mx2, tmp[e]);
+        }
+        mxc = fmaxf(max64(p), mx2);
+        const float offc = -mxc * sc2;
+#pragma unroll
+        for (int j = 0; j < kTile / 16; ++j) {
+          float tmp[16];
+          tmem_ld16(lane_base + (uint32_t)(x2 * kTile + 16 * j), tmp);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            fma2(tmp[e], tmp[e + 1], sc2, offc);
+            sum2_raw += fast_exp2(tmp[e]) + fast_exp2(tmp[e + 1]);
+          }
+        }
+      }
       bool rescale = false;
       float factor = 1.f;
       // base-2 exponentials throughout: x * scale * log2(e) is the logit in log2 units
-      const float sc2 = D.scale * kLog2e;
-      if (is_sel && u != -INFINITY) {
+      if (is_second) {
+        // second half of a selected chunk: the max and normaliser of its first half
+#pragma unroll
+        for (int j = 0; j < kTile; j += 2) {
+          fma2(p[j], p[j + 1], sc2, sec_off);
+          p[j] = fast_exp2(p[j]);
+          p[j + 1] = fast_exp2(p[j + 1]);
+          mul2(p[j], p[j + 1], sec_f);
+        }
+      } else if (is_sel && u != -INFINITY) {
         // intra-chunk softmax of this chunk, weighted by exp(u - m_run) (u <= m_run)
         // (three-input maxima, and fp32 pairs for the affine, sum and scale passes)
-        const float mx = max64(p);
+        const float mx = first2 ? mxc : max64(p);
         const float off = -mx * sc2;
         float ps[8];
 #pragma unroll
@@ -559,12 +621,14 @@ __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
           p[j + 1] = fast_exp2(p[j + 1]);
           add2(ps[j & 7], ps[(j & 7) + 1], p[j], p[j + 1]);
         }
-        const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])) +
+                          (first2 ? sum2_raw : 0.f);
         const float w = fast_exp2((u - m_run) * kLog2e);
         const float f = w / sum;
 #pragma unroll
         for (int j = 0; j < kTile; j += 2) mul2(p[j], p[j + 1], f);
         l += w;
+        if (first2) { sec_pending = true; sec_off = off; sec_f = f; }
       } else if (is_win) {
         // raw logits; only the tile holding the query's own position needs the causal mask
         if (t0 + kTile - 1 > pos) {
@@ -697,11 +761,11 @@ bool make_map_at(CUtensorMap* map, const void* base, uint64_t rows, uint64_t d, 
 }
 
 int list_capacity(const Dims& D, int TQ) {
-  // union of TQ queries' selections plus the chunks their windows cover
-  return TQ * D.K + (int)((D.W + kTile + TQ) / kTile) + 4;
+  // union of TQ queries' selections (S / 64 tiles each) plus the tiles their windows cover
+  return TQ * D.K * (D.S / kTile) + (int)((D.W + D.S + TQ) / kTile) + 4;
 }
 
-template <int DD, int G, int KM>
+template <int DD, int G, int KM, int RS>
 cudaError_t launch_at_t(const Dims& D, const void* q, const void* qc, const void* K,
                         const void* V, const int32_t* idx, const void* klm, const float* blm,
                         void* out, float* lse, int32_t* status, cudaStream_t st) {
@@ -716,7 +780,7 @@ cudaError_t launch_at_t(const Dims& D, const void* q, const void* qc, const void
   const int words = (int)((D.N_kv / kTile) / 32) + 2;
   const int smem = SH::FIXED + 1024 + cap * 4 + 2 * words * 4 + (KM <= 16 ? kAtRows * KM * 8 : 0);
   if (smem > kAtSmemLimit) return cudaErrorInvalidConfiguration;
-  auto kern = attn_tc_kernel<DD, G, KM>;
+  auto kern = attn_tc_kernel<DD, G, KM, RS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((D.N_q + SH::TQ - 1) / SH::TQ), (unsigned)(D.B * D.Hkv));
@@ -730,22 +794,33 @@ template <int DD, int G>
 cudaError_t launch_at_k(const Dims& D, const void* q, const void* qc, const void* K,
                         const void* V, const int32_t* idx, const void* klm, const float* blm,
                         void* out, float* lse, int32_t* status, cudaStream_t st) {
+  if constexpr (DD == 128) {
+    // chunks of 128 tokens (two tiles per chunk) are built for d = 128 only
+    if (D.S == 2 * kTile) {
+      if (D.K <= 8)
+        return launch_at_t<DD, G, 8, 1>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st);
+      if (D.K <= 16)
+        return launch_at_t<DD, G, 16, 1>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st);
+      return launch_at_t<DD, G, 32, 1>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st);
+    }
+  }
   if (D.K <= 8)
-    return launch_at_t<DD, G, 8>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st);
+    return launch_at_t<DD, G, 8, 0>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st);
   if (D.K <= 16)
-    return launch_at_t<DD, G, 16>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st);
-  return launch_at_t<DD, G, 32>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st);
+    return launch_at_t<DD, G, 16, 0>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st);
+  return launch_at_t<DD, G, 32, 0>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st);
 }
 
 }  // namespace
 
 bool attn_tc_supported(const Dims& D, bool bf16) {
-  if (!bf16 || D.S != kTile || D.K > kMaxK) return false;
+  if (!bf16 || D.K > kMaxK) return false;
+  if (D.S != kTile && !(D.S == 2 * kTile && D.d == 128)) return false;
   if (D.d != 64 && D.d != 128) return false;
   if (D.G != 1 && D.G != 2 && D.G != 4 && D.G != 8) return false;
   if (D.B * D.Hkv > 65535) return false;
   const int TQ = kAtRows / D.G;
-  const int64_t cap = (int64_t)TQ * D.K + (D.W + kTile + TQ) / kTile + 4;
+  const int64_t cap = (int64_t)TQ * D.K * (D.S / kTile) + (D.W + D.S + TQ) / kTile + 4;
   const int64_t words = (D.N_kv / kTile) / 32 + 2;
   const int fixed = D.d == 128 ? AtShape<128, 1>::FIXED : AtShape<64, 1>::FIXED;
   if (D.C >= (int64_t)INT32_MAX) return false;
