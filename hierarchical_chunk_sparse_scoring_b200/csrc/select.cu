@@ -100,7 +100,9 @@ __device__ __forceinline__ void write_selection_wide(const Dims& D, int64_t b, i
     kv[j] = valid ? __ldg(reinterpret_cast<const uint4*>(kb + (int64_t)c * D_) + j)
                   : make_uint4(0u, 0u, 0u, 0u);
   const float bc = valid ? __ldg(bb + c) : 0.f;
-#pragma unroll
+  // (loops kept rolled: this runs once per row, and straight-line code this long would be
+  // fetched from L2 instruction by instruction)
+#pragma unroll 1
   for (int h = 0; h < GM; ++h) {
     if (h >= G) break;
     float a = 0.f;
@@ -735,6 +737,20 @@ __device__ __forceinline__ void warp_sort_best_first(float& v, int& c, int lane)
   }
 }
 
+// Appends the lanes' kept candidates to the shared survivor list (ballot order).  Not inlined:
+// it runs only for the few batches that hold survivors, and inlining it at every call site would
+// multiply the kernel's code (fetched instruction by instruction on a cold start).
+__device__ __noinline__ void topk_append(bool keep, float v, int c, int lane, unsigned lt,
+                                         int* n_surv, float* sv, int* scn) {
+  const unsigned m = __ballot_sync(0xffffffffu, keep);
+  if (m == 0u) return;
+  int base = 0;
+  if (lane == 0) base = atomicAdd(n_surv, __popc(m));
+  base = __shfl_sync(0xffffffffu, base, 0);
+  const int pos = base + __popc(m & lt);
+  if (keep && pos < kSurvivorCap) { sv[pos] = v; scn[pos] = c; }
+}
+
 template <typename T, int D_, int GM, int KM>
 __global__ void __launch_bounds__(kTopkThreads) select_topk_row_kernel(
     Dims D, int64_t n_stride, const float* __restrict__ sigma, const T* __restrict__ qc,
@@ -801,15 +817,7 @@ __global__ void __launch_bounds__(kTopkThreads) select_topk_row_kernel(
     if (better(th_v[w], th_c[w], tv, tcc)) { tv = th_v[w]; tcc = th_c[w]; }
   // 3. survivors: candidates not worse than theta, compacted in ballot order per warp batch
   const unsigned lt = (1u << lane) - 1u;
-  auto append = [&](bool keep, float v, int c) {
-    const unsigned m = __ballot_sync(0xffffffffu, keep);
-    if (m == 0u) return;
-    int base = 0;
-    if (lane == 0) base = atomicAdd(&n_surv, __popc(m));
-    base = __shfl_sync(0xffffffffu, base, 0);
-    const int pos = base + __popc(m & lt);
-    if (keep && pos < kSurvivorCap) { sv[pos] = v; scn[pos] = c; }
-  };
+  auto append = [&](bool keep, float v, int c) { topk_append(keep, v, c, lane, lt, &n_surv, sv, scn); };
   for (int64_t q0 = w0; q0 < w1; q0 += 32 * kTopkBatch) {
     float4 t[kTopkBatch];
 #pragma unroll
