@@ -110,6 +110,31 @@ __device__ __forceinline__ float fmax3f(float a, float b, float c) {
   return r;
 }
 
+// q_cal row r (128-byte-swizzled tile) . k_lm row, for a selected chunk whose landmark row was
+// not staged.  Out of line: it is rare, and one inlined copy per list slot would bloat the
+// kernel.
+template <int KB, int Q_BOX>
+__device__ __noinline__ float lm_dot(const uint8_t* sQc, int r, const __nv_bfloat16* kr) {
+  float a = 0.f;
+  for (int kb = 0; kb < KB; ++kb) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint4 qv = *reinterpret_cast<const uint4*>(
+          sQc + kb * Q_BOX + (r >> 3) * 1024 + (r & 7) * 128 + ((j ^ (r & 7)) << 4));
+      const uint4 kv = __ldg(reinterpret_cast<const uint4*>(kr + kb * 64 + j * 8));
+      a = fmaf(bf16_lo(qv.x), bf16_lo(kv.x), a);
+      a = fmaf(bf16_hi(qv.x), bf16_hi(kv.x), a);
+      a = fmaf(bf16_lo(qv.y), bf16_lo(kv.y), a);
+      a = fmaf(bf16_hi(qv.y), bf16_hi(kv.y), a);
+      a = fmaf(bf16_lo(qv.z), bf16_lo(kv.z), a);
+      a = fmaf(bf16_hi(qv.z), bf16_hi(kv.z), a);
+      a = fmaf(bf16_lo(qv.w), bf16_lo(kv.w), a);
+      a = fmaf(bf16_hi(qv.w), bf16_hi(kv.w), a);
+    }
+  }
+  return a;
+}
+
 // max of a row's 64 logits: eight independent three-input chains, then a short tree
 __device__ __forceinline__ float max64(const float (&p)[64]) {
   float pm[8];
@@ -449,14 +474,21 @@ __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
           }
         }
       }
+      // the biases first, all loads in flight at once
+      float bsel[KM];
+#pragma unroll
+      for (int k = 0; k < KM; ++k) {
+        const int c = sc[k];
+        bsel[k] = (lm_ok && c >= 0 && c < D.C) ? __ldg(blm + bg * D.C + c) : 0.f;
+      }
 #pragma unroll
       for (int k = 0; k < KM; ++k) {
         su[k] = -INFINITY;
         const int c = sc[k];
         if (!lm_ok || c < 0 || c >= D.C) continue;
-        const float bias = __ldg(blm + bg * D.C + c);
-        // the chunk's position in the (sorted) tile list: the rank of its bit in the bitmap
-        const int tc = c << rs;   // the chunk's first tile
+        const float bias = bsel[k];
+        // the chunk's position in the (sorted) tile list: the rank of its first tile's bit
+        const int tc = c << rs;
         const int rank = wpre[tc >> 5] + __popc(bitmap[tc >> 5] & ((1u << (tc & 31)) - 1u));
         const int slot = rank < nk ? rank : -1;
         float a;
@@ -465,25 +497,7 @@ __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
           a = *reinterpret_cast<const float*>(park + (col4 >> 3) * SH::P_BYTES +
                                               (((col4 & 7) + r) & 7) * 16 + (slot & 3) * 4);
         } else {
-          const __nv_bfloat16* kr = klm + (bg * D.C + c) * DD;
-          a = 0.f;
-#pragma unroll
-          for (int kb = 0; kb < SH::KB; ++kb) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const uint4 qv = *reinterpret_cast<const uint4*>(
-                  sQc + kb * SH::Q_BOX + (r >> 3) * 1024 + (r & 7) * 128 + ((j ^ (r & 7)) << 4));
-              const uint4 kv = __ldg(reinterpret_cast<const uint4*>(kr + kb * 64 + j * 8));
-              a = fmaf(bf16_lo(qv.x), bf16_lo(kv.x), a);
-              a = fmaf(bf16_hi(qv.x), bf16_hi(kv.x), a);
-              a = fmaf(bf16_lo(qv.y), bf16_lo(kv.y), a);
-              a = fmaf(bf16_hi(qv.y), bf16_hi(kv.y), a);
-              a = fmaf(bf16_lo(qv.z), bf16_lo(kv.z), a);
-              a = fmaf(bf16_hi(qv.z), bf16_hi(kv.z), a);
-              a = fmaf(bf16_lo(qv.w), bf16_lo(kv.w), a);
-              a = fmaf(bf16_hi(qv.w), bf16_hi(kv.w), a);
-            }
-          }
+          a = lm_dot<SH::KB, SH::Q_BOX>(sQc, r, klm + (bg * D.C + c) * DD);
         }
         su[k] = fmaf(a, D.scale, bias);
         m_run = fmaxf(m_run, su[k]);
