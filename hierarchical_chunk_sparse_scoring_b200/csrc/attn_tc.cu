@@ -183,7 +183,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int& to
 }  // namespace
 
 template <int DD, int G, int KM, int RS>
-__global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
+__global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQc,
                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    Dims D, const int32_t* __restrict__ idx, const __nv_bfloat16* __restrict__ klm,
@@ -278,11 +278,19 @@ __global__ void __launch_bounds__(kAtThreads, DD == 64 ? 2 : 1)
       }
   }
   // selected chunks of every valid query of the tile, and the chunks of the local windows
-  for (int e = threadIdx.x; e < TQ * K; e += kAtThreads) {
-    const int qi = e / K, k = e - qi * K;
-    const int64_t i = i0 + qi;
-    if (i < D.N_q) {
-      const int c = idx[(bg * D.N_q + i) * K + k];
+  // (the index reads go out four at a time before their bits are set)
+  for (int e0 = threadIdx.x; e0 < TQ * K; e0 += 4 * kAtThreads) {
+    int cs[4];
+#pragma unroll
+    for (int u4 = 0; u4 < 4; ++u4) {
+      const int e = e0 + u4 * kAtThreads;
+      const int qi = e / K, k = e - qi * K;
+      const int64_t i = i0 + qi;
+      cs[u4] = (e < TQ * K && i < D.N_q) ? __ldg(idx + (bg * D.N_q + i) * K + k) : -1;
+    }
+#pragma unroll
+    for (int u4 = 0; u4 < 4; ++u4) {
+      const int c = cs[u4];
       if (c >= 0 && c < D.C) {
         for (int e2 = 0; e2 <= rs; ++e2) {
           const int tl = (c << rs) + e2;

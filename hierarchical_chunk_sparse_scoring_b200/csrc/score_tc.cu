@@ -46,13 +46,14 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 constexpr uint32_t kPollLimit = 1u << 24;
 constexpr int kSmemLimit = 227 * 1024;
 
-template <int DD, int G, int KM, int NCG, int HP>
+template <int DD, int G, int KM, int NCG, int HP, int CPS>
 struct TcShape {
   static constexpr int THREADS = 64 + 128 * NCG;
   static constexpr int EPI = 128 * NCG;                       // epilogue threads
   static constexpr int MQ = kRows / HP;                       // queries per CTA
   static constexpr int GV = G / HP;                           // accumulators per tile
-  static constexpr int NT = 256 / GV < 256 ? 256 / GV : 256;  // chunks per tile
+  // CPS CTAs per SM share its 512 TMEM columns: two accumulator sets of GV x NT each
+  static constexpr int NT = (256 / CPS) / GV < 256 ? (256 / CPS) / GV : 256;   // chunks per tile
   static constexpr int KB = DD / 64;                          // 128-byte boxes along d
   static constexpr int A_BOX = kRows * 128;
   static constexpr int A_BYTES = GV * KB * A_BOX;
@@ -63,16 +64,18 @@ struct TcShape {
   static constexpr int STASH_BYTES = STASH_A > STASH_B ? STASH_A : STASH_B;
   static constexpr int FIXED = A_BYTES + STASH_BYTES + 1024 /*barriers*/ + 1024 /*align*/ +
                                2048 /*shared thresholds*/ + 4 * NT * 4 /*bias tiles*/;
-  static constexpr int STAGES_FIT = (kSmemLimit - FIXED) / B_STAGE;
+  static constexpr int STAGES_FIT = ((CPS == 1 ? kSmemLimit : kSmemLimit / CPS - 1024) - FIXED) /
+                                    B_STAGE;
   static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
   // more than half of the SM's shared memory, so a second CTA can never be co-resident and
   // compete for the 512 TMEM columns this CTA allocates
   static constexpr int SMEM_USED = FIXED + STAGES * B_STAGE;
-  static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
+  static constexpr int SMEM =
+      CPS == 1 ? (SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024) : SMEM_USED;
   static constexpr int CG = NT / NCG;                          // columns per epilogue warp
   static constexpr int HG = GV < 4 ? GV : 4;   // accumulators whose TMEM loads are in flight
   static constexpr uint32_t TMEM_COLS = 2 * GV * NT;
-  static_assert(TMEM_COLS == 512, "two accumulator sets fill TMEM");
+  static_assert(TMEM_COLS * CPS == 512, "the accumulator sets fill TMEM");
   static_assert(STAGES >= 2, "shared memory too small for this shape");
   static_assert(CG % 16 == 0, "sub-blocks of 16 columns");
   static_assert(NCG == 2 || NCG == 4, "two or four column groups");
@@ -81,13 +84,13 @@ struct TcShape {
 
 }  // namespace
 
-template <int DD, int G, int KM, int NCG, int HP>
-__global__ void __launch_bounds__(64 + 128 * NCG, 1)
+template <int DD, int G, int KM, int NCG, int HP, int CPS>
+__global__ void __launch_bounds__(64 + 128 * NCG, CPS)
     score_topk_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB, Dims D,
                          const float* __restrict__ blm, int32_t* __restrict__ idx,
                          int32_t* __restrict__ status) {
-  using SH = TcShape<DD, G, KM, NCG, HP>;
+  using SH = TcShape<DD, G, KM, NCG, HP, CPS>;
   constexpr int NT = SH::NT;
   constexpr int GV = SH::GV;
   extern __shared__ uint8_t smem_raw[];
@@ -432,10 +435,10 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t d, uin
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int DD, int G, int KM, int NCG, int HP>
+template <int DD, int G, int KM, int NCG, int HP, int CPS>
 cudaError_t launch_tc_t(const Dims& D, const void* qc, const void* klm, const float* blm,
                         int32_t* idx, int32_t* status, cudaStream_t st) {
-  using SH = TcShape<DD, G, KM, NCG, HP>;
+  using SH = TcShape<DD, G, KM, NCG, HP, CPS>;
   CUtensorMap tmA, tmB;
   bool ok_a;
   if constexpr (HP == 1) {
@@ -455,7 +458,7 @@ cudaError_t launch_tc_t(const Dims& D, const void* qc, const void* klm, const fl
   }
   if (!ok_a || !make_map(&tmB, klm, (uint64_t)(D.B * D.Hkv * (D.C > 0 ? D.C : 1)), DD, SH::NT))
     return cudaErrorInvalidValue;
-  auto kern = score_topk_tc_kernel<DD, G, KM, NCG, HP>;
+  auto kern = score_topk_tc_kernel<DD, G, KM, NCG, HP, CPS>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SH::SMEM);
   if (e != cudaSuccess) return e;
@@ -472,9 +475,15 @@ cudaError_t launch_tc_k(const Dims& D, const void* qc, const void* klm, const fl
   // the list length follows K: an insertion costs a compare and two selects per slot
   // eight heads of 128 dimensions: head pairs (the eight query tiles would not fit)
   constexpr int HP = (G == 8 && DD == 128) ? 2 : 1;
-  if (D.K <= 8) return launch_tc_t<DD, G, 8, 2, HP>(D, qc, klm, blm, idx, status, st);
-  if (D.K <= 16) return launch_tc_t<DD, G, 16, 2, HP>(D, qc, klm, blm, idx, status, st);
-  return launch_tc_t<DD, G, 32, 2, HP>(D, qc, klm, blm, idx, status, st);
+  if (D.K <= 8) {
+    // small query tiles and short lists: two CTAs per SM (each one's epilogue latency hides
+    // behind the other's)
+    if constexpr (DD == 64 && G <= 2)
+      return launch_tc_t<DD, G, 8, 2, HP, 2>(D, qc, klm, blm, idx, status, st);
+    return launch_tc_t<DD, G, 8, 2, HP, 1>(D, qc, klm, blm, idx, status, st);
+  }
+  if (D.K <= 16) return launch_tc_t<DD, G, 16, 2, HP, 1>(D, qc, klm, blm, idx, status, st);
+  return launch_tc_t<DD, G, 32, 2, HP, 1>(D, qc, klm, blm, idx, status, st);
 }
 
 }  // namespace
