@@ -105,10 +105,11 @@ __device__ __forceinline__ void write_selection_wide(const Dims& D, int64_t b, i
 #pragma unroll 1
   for (int h = 0; h < GM; ++h) {
     if (h >= G) break;
-    float a = 0.f;
+    float a4[4] = {0.f, 0.f, 0.f, 0.f};   // four short dependency chains
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
       const uint4 qv = q4[h * NV + j];
+      float& a = a4[j & 3];
       a = fmaf(bf16_lo(qv.x), bf16_lo(kv[j].x), a);
       a = fmaf(bf16_hi(qv.x), bf16_hi(kv[j].x), a);
       a = fmaf(bf16_lo(qv.y), bf16_lo(kv[j].y), a);
@@ -118,6 +119,7 @@ __device__ __forceinline__ void write_selection_wide(const Dims& D, int64_t b, i
       a = fmaf(bf16_lo(qv.w), bf16_lo(kv[j].w), a);
       a = fmaf(bf16_hi(qv.w), bf16_hi(kv[j].w), a);
     }
+    const float a = (a4[0] + a4[1]) + (a4[2] + a4[3]);
     const int64_t hrow = ((b * D.Hq) + g * G + h) * D.N_q + i;
     s_sel[hrow * K + lane] = valid ? fmaf(a, D.scale, bc) : -INFINITY;
   }
@@ -737,20 +739,6 @@ __device__ __forceinline__ void warp_sort_best_first(float& v, int& c, int lane)
   }
 }
 
-// Appends the lanes' kept candidates to the shared survivor list (ballot order).  Not inlined:
-// it runs only for the few batches that hold survivors, and inlining it at every call site would
-// multiply the kernel's code (fetched instruction by instruction on a cold start).
-__device__ __noinline__ void topk_append(bool keep, float v, int c, int lane, unsigned lt,
-                                         int* n_surv, float* sv, int* scn) {
-  const unsigned m = __ballot_sync(0xffffffffu, keep);
-  if (m == 0u) return;
-  int base = 0;
-  if (lane == 0) base = atomicAdd(n_surv, __popc(m));
-  base = __shfl_sync(0xffffffffu, base, 0);
-  const int pos = base + __popc(m & lt);
-  if (keep && pos < kSurvivorCap) { sv[pos] = v; scn[pos] = c; }
-}
-
 template <typename T, int D_, int GM, int KM>
 __global__ void __launch_bounds__(kTopkThreads) select_topk_row_kernel(
     Dims D, int64_t n_stride, const float* __restrict__ sigma, const T* __restrict__ qc,
@@ -760,7 +748,7 @@ __global__ void __launch_bounds__(kTopkThreads) select_topk_row_kernel(
   __shared__ int scn[kSurvivorCap];
   __shared__ float th_v[kTopkWarps];
   __shared__ int th_c[kTopkWarps];
-  __shared__ int n_surv;
+  __shared__ int wcnt[kTopkWarps];   // survivors per warp
   __shared__ __align__(16) __nv_bfloat16 qsh[GM * D_];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t row = blockIdx.x;
@@ -771,7 +759,6 @@ __global__ void __launch_bounds__(kTopkThreads) select_topk_row_kernel(
   const int64_t n4 = n >> 2;
   // this warp's quarter of the row's float4 vectors (the scalar tail goes to the last warp)
   const int64_t w0 = n4 * warp / kTopkWarps, w1 = n4 * (warp + 1) / kTopkWarps;
-  if (threadIdx.x == 0) n_surv = 0;
   // 1. lane maxima (a lane's chunks come in increasing order: a strict compare keeps the lower
   //    index on ties)
   float mv = -INFINITY;
@@ -817,7 +804,17 @@ __global__ void __launch_bounds__(kTopkThreads) select_topk_row_kernel(
     if (better(th_v[w], th_c[w], tv, tcc)) { tv = th_v[w]; tcc = th_c[w]; }
   // 3. survivors: candidates not worse than theta, compacted in ballot order per warp batch
   const unsigned lt = (1u << lane) - 1u;
-  auto append = [&](bool keep, float v, int c) { topk_append(keep, v, c, lane, lt, &n_surv, sv, scn); };
+  // each warp appends to its own region of the list: a ballot and a prefix count, no atomics
+  constexpr int kCapW = kSurvivorCap / kTopkWarps;
+  float* svw = sv + warp * kCapW;
+  int* scw = scn + warp * kCapW;
+  int ns_w = 0;   // warp-uniform
+  auto append = [&](bool keep, float v, int c) {
+    const unsigned m = __ballot_sync(0xffffffffu, keep);
+    const int pos = ns_w + __popc(m & lt);
+    if (keep && pos < kCapW) { svw[pos] = v; scw[pos] = c; }
+    ns_w += __popc(m);
+  };
   for (int64_t q0 = w0; q0 < w1; q0 += 32 * kTopkBatch) {
     float4 t[kTopkBatch];
 #pragma unroll
@@ -850,22 +847,65 @@ __global__ void __launch_bounds__(kTopkThreads) select_topk_row_kernel(
       append(c < n && !better(tv, tcc, v, (int)c), v, (int)c);
     }
   }
+  if (lane == 0) wcnt[warp] = ns_w;
   __syncthreads();
   if (warp != 0) return;
-  const int ns = n_surv;
+  int cnt[kTopkWarps], ns = 0;
+  bool overflow = false;
+#pragma unroll
+  for (int w = 0; w < kTopkWarps; ++w) {
+    cnt[w] = wcnt[w];
+    overflow |= cnt[w] > kCapW;
+    ns += cnt[w];
+  }
+  // survivor e of the concatenated warp regions
+  auto survivor = [&](int e, float& v, int& c) {
+    v = -INFINITY;
+    c = INT_MAX;
+#pragma unroll
+    for (int w = 0; w < kTopkWarps; ++w) {
+      if (e >= 0 && e < cnt[w]) { v = sv[w * kCapW + e]; c = scn[w * kCapW + e]; }
+      e -= cnt[w];
+    }
+  };
   // 4. exact top-K of the survivors (or of every candidate if too many tied at theta)
   float wv;
   int wc;
-  if (ns <= 32) {
-    wv = lane < ns ? sv[lane] : -INFINITY;
-    wc = lane < ns ? scn[lane] : INT_MAX;
-    warp_sort_best_first(wv, wc, lane);
-    if (lane >= K) { wv = -INFINITY; wc = INT_MAX; }
+  if (!overflow && ns <= 64) {
+    // one bitonic sort of up to 64 survivors, two per lane (elements lane and lane + 32)
+    float va, vb;
+    int ca, cb;
+    survivor(lane, va, ca);
+    survivor(lane + 32, vb, cb);
+#pragma unroll
+    for (int size = 2; size <= 64; size <<= 1) {
+#pragma unroll
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        if (stride == 32) {
+          // elements lane and lane + 32, both in blocks sorted best first
+          if (better(vb, cb, va, ca)) {
+            const float tv2 = va; va = vb; vb = tv2;
+            const int tc2 = ca; ca = cb; cb = tc2;
+          }
+        } else {
+          const bool lower = (lane & stride) == 0;
+          cmpx(va, ca, stride, ((lane & size) == 0) == lower);
+          cmpx(vb, cb, stride, (((lane + 32) & size) == 0) == lower);
+        }
+      }
+    }
+    wv = lane < K ? va : -INFINITY;
+    wc = lane < K ? ca : INT_MAX;
   } else {
     TopList<KM> L;
     L.clear();
-    if (ns <= kSurvivorCap) {
-      for (int e = lane; e < ns; e += 32) L.insert(sv[e], scn[e], K);
+    if (!overflow) {
+      for (int e = lane; e < ns; e += 32) {
+        float v;
+        int c;
+        survivor(e, v, c);
+        L.insert(v, c, K);
+      }
     } else {
       for (int64_t c = lane; c < n; c += 32) L.insert(__ldg(sr + c), (int)c, K);
     }
