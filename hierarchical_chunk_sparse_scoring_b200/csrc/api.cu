@@ -112,14 +112,6 @@ Plan make_plan(const hils_params* p) {
   return P;
 }
 
-// segments per row for the decode top-K (<= n_split, so the split lists fit the workspace)
-int n_topk_segments(const Plan& P) {
-  int64_t s = (P.n_stride + 1023) / 1024;
-  if (s > 16) s = 16;
-  if (s > P.n_split) s = P.n_split;
-  return (int)(s < 1 ? 1 : s);
-}
-
 int n_stream_split(const Plan& P) {
   const int64_t n_max = P.n_stride;
   const int64_t s = (n_max + kStreamRows - 1) / kStreamRows;

@@ -474,7 +474,6 @@ cudaError_t launch_attn_rows(const Dims& D, bool bf16, const void* q, const void
   return cudaGetLastError();
 }
 
-size_t units_smem_bytes(const Dims& D) { (void)D; return 0; }
 
 template <typename T, int D_>
 static cudaError_t launch_units_d(const Dims& D, int n_pieces, const void* q, const void* K,

@@ -42,8 +42,6 @@ bool units_tc_supported(const Dims& D, bool bf16);
 cudaError_t launch_attn_units_tc(const Dims& D, int n_pieces, const void* q, const void* K,
                                  const void* V, const int32_t* idx, float* part_o,
                                  float* part_lse, int32_t* status, cudaStream_t st);
-cudaError_t launch_select_topk(const Dims& D, int n_seg, int64_t n_stride, const float* sigma,
-                               float* part_v, int32_t* part_c, cudaStream_t st);
 cudaError_t launch_select_topk_row(const Dims& D, bool bf16, int64_t n_stride,
                                    const float* sigma, const void* qc, const void* klm,
                                    const float* blm, int32_t* idx, float* s_sel, cudaStream_t st);
@@ -55,7 +53,6 @@ cudaError_t launch_attn_rows(const Dims& D, bool bf16, const void* q, const void
                              const void* V, const int32_t* idx, const float* s_sel, void* out,
                              float* lse, float* unit_o, float* unit_lse, cudaStream_t st);
 
-size_t units_smem_bytes(const Dims& D);
 cudaError_t launch_attn_units(const Dims& D, bool bf16, int n_pieces, const void* q,
                               const void* K, const void* V, const int32_t* idx, float* part_o,
                               float* part_lse, int32_t* status, cudaStream_t st);

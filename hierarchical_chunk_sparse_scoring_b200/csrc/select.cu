@@ -516,7 +516,7 @@ __global__ void __launch_bounds__(128) select_merge_kernel(Dims D, int n_split,
 // ---------------------------------------------------------------------------------------------
 // Decode, streaming form.  select_stream_kernel reads every eligible landmark row of a query
 // exactly once (coalesced 16-byte loads, several rows in flight per lane group) and writes the
-// group score sigma_c = max_h s_{h,c} to a scratch row; select_topk_kernel then selects the K
+// group score sigma_c = max_h s_{h,c} to a scratch row; select_topk_row_kernel then selects the K
 // best of each row and computes the per-head scores of the winners.  The scratch write is
 // 4 bytes per landmark row read (d * 2 bytes), under 2% extra traffic for d = 128.
 constexpr int kStreamWarps = 4;                          // consumer warps
@@ -654,50 +654,6 @@ __global__ void __launch_bounds__(kStreamThreads) select_stream_kernel(
     }
     __syncwarp();
     if (lane == 0) sm100::mbar_arrive(&empty[s]);
-  }
-}
-
-// Top-K of one segment of a row's group scores (blockIdx.x = segment, blockIdx.y = (b, g,
-// query)): per-thread lists, merged per warp, then across warps; the segment's K best go to
-// part_v / part_c [rows][segments][K] for select_merge_kernel.
-template <int KM>
-__global__ void __launch_bounds__(256) select_topk_kernel(Dims D, int64_t n_stride, int n_seg,
-                                                          const float* __restrict__ sigma,
-                                                          float* __restrict__ part_v,
-                                                          int32_t* __restrict__ part_c) {
-  __shared__ float lv[8 * kMaxK];
-  __shared__ int lc[8 * kMaxK];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int seg = blockIdx.x;
-  const int64_t row = blockIdx.y;
-  const int64_t i = row % D.N_q;
-  const int K = D.K;
-  const int64_t n = n_eligible(D.q_pos0 + i, D.S, D.W);
-  const int64_t per = (n + n_seg - 1) / n_seg;
-  const int64_t c0 = (int64_t)seg * per;
-  const int64_t c1 = c0 + per < n ? c0 + per : n;
-  const float* sr = sigma + row * n_stride;
-  TopList<KM> L;
-  L.clear();
-  for (int64_t c = c0 + threadIdx.x; c < c1; c += 256) L.insert(sr[c], (int)c, K);
-  float wv;
-  int wc;
-  warp_merge_topk<KM>(L, K, lane, wv, wc);
-  if (lane < K) { lv[warp * K + lane] = wv; lc[warp * K + lane] = wc; }
-  __syncthreads();
-  if (warp != 0) return;
-  int ptr = 0;
-  float* outv = part_v + (row * n_seg + seg) * K;
-  int32_t* outc = part_c + (row * n_seg + seg) * K;
-  for (int r = 0; r < K; ++r) {
-    float v = -INFINITY;
-    int c = INT_MAX;
-    if (lane < 8 && ptr < K) { v = lv[lane * K + ptr]; c = lc[lane * K + ptr]; }
-    float bv = v;
-    int bc = c;
-    warp_best(bv, bc);
-    if (lane < 8 && c == bc && bc != INT_MAX) ++ptr;
-    if (lane == 0) { outv[r] = bv; outc[r] = bc; }
   }
 }
 
@@ -1090,20 +1046,6 @@ cudaError_t launch_select_stream(const Dims& D, bool bf16, int cps, int n_split,
   if (D.B * D.Hkv * D.N_q == 0) return cudaSuccess;
   return dispatch_tdgk<StreamOnly>(bf16, D.d, D.G, D.K, &D, cps, n_split, n_stride, qc, klm,
                                    blm, sigma, status, st);
-}
-
-cudaError_t launch_select_topk(const Dims& D, int n_seg, int64_t n_stride, const float* sigma,
-                               float* part_v, int32_t* part_c, cudaStream_t st) {
-  const int64_t rows = D.B * D.Hkv * D.N_q;
-  if (rows == 0) return cudaSuccess;
-  dim3 grid((unsigned)n_seg, (unsigned)rows);
-  if (D.K <= 8)
-    select_topk_kernel<8><<<grid, 256, 0, st>>>(D, n_stride, n_seg, sigma, part_v, part_c);
-  else if (D.K <= 16)
-    select_topk_kernel<16><<<grid, 256, 0, st>>>(D, n_stride, n_seg, sigma, part_v, part_c);
-  else
-    select_topk_kernel<32><<<grid, 256, 0, st>>>(D, n_stride, n_seg, sigma, part_v, part_c);
-  return cudaGetLastError();
 }
 
 cudaError_t launch_select_topk_row(const Dims& D, bool bf16, int64_t n_stride,
