@@ -154,32 +154,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&t);
 }
 
-// Block-wide exclusive scan of one int per thread (blockDim.x <= 1024); returns the total.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int& total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) scratch[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    int w = lane < nw ? scratch[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    if (lane < nw) scratch[32 + lane] = w;   // inclusive warp prefix
-  }
-  __syncthreads();
-  total = scratch[32 + nw - 1];
-  const int before = warp > 0 ? scratch[32 + warp - 1] : 0;
-  return before + x - v;
-}
-
 }  // namespace
 
 template <int DD, int G, int KM, int RS>
@@ -223,8 +197,7 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
   uint64_t* lm_done = o_final + 1;
   uint64_t* qc_free = lm_done + 1;   // every softmax warp is done reading the q_cal tile
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qc_free + 1);
-  int* scan = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + 1024);   // [64]
-  int* n_tiles_sh = scan + 64;
+  int* n_tiles_sh = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + 1024);
   int* tiles = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + 2048);  // [list_cap]
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(tiles + list_cap);             // [words]
   int* wpre = reinterpret_cast<int*>(bitmap + bitmap_words);   // list position of each word
@@ -244,6 +217,18 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
   const int64_t last_chunk = p_max / kTile;   // last tile (64 tokens) any window reaches
   constexpr int rs = RS;                       // tiles per chunk = 1 << rs
   const int K = D.K;
+  // warps 2-5 own one row each: (head h, query qi) = row r
+  const bool is_row = warp >= 2;
+  const int qd = warp & 3;
+  const int r = qd * 32 + lane;
+  const int h = r / TQ, qi = r - h * TQ;
+  const int64_t i = i0 + qi;
+  const bool valid = i < D.N_q;
+  // the row's selected chunks go out first: they feed both the tile list and the row's scores
+  int sc[KM];
+#pragma unroll
+  for (int k = 0; k < KM; ++k)
+    sc[k] = (is_row && valid && k < K) ? __ldg(idx + (bg * D.N_q + i) * K + k) : -1;
 
   // ---------------------------------------------------------------- barriers, TMEM, tile list
   if (threadIdx.x == 0) {
@@ -270,28 +255,21 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
     prefetch_tensormap(&tmQ);
     prefetch_tensormap(&tmQc);
     mbar_expect_tx(q_full, 2 * SH::Q_BYTES);
-    for (int h = 0; h < G; ++h)
+    for (int hh = 0; hh < G; ++hh)
       for (int kb = 0; kb < SH::KB; ++kb) {
-        const int32_t y = (int32_t)((b * D.Hq + g * G + h) * D.N_q + i0);
-        tma_load_2d(sQ + kb * SH::Q_BOX + h * TQ * 128, &tmQ, kb * 64, y, q_full);
-        tma_load_2d(sQc + kb * SH::Q_BOX + h * TQ * 128, &tmQc, kb * 64, y, q_full);
+        const int32_t y = (int32_t)((b * D.Hq + g * G + hh) * D.N_q + i0);
+        tma_load_2d(sQ + kb * SH::Q_BOX + hh * TQ * 128, &tmQ, kb * 64, y, q_full);
+        tma_load_2d(sQc + kb * SH::Q_BOX + hh * TQ * 128, &tmQc, kb * 64, y, q_full);
       }
   }
-  // selected chunks of every valid query of the tile, and the chunks of the local windows
-  // (the index reads go out four at a time before their bits are set)
-  for (int e0 = threadIdx.x; e0 < TQ * K; e0 += 4 * kAtThreads) {
-    int cs[4];
+  // selected chunks of every valid query of the tile (the G rows of a query hold the same
+  // selection: row (h, qi) sets the bits of the entries k = h mod G), and the chunks of the
+  // local windows
+  if (is_row) {
 #pragma unroll
-    for (int u4 = 0; u4 < 4; ++u4) {
-      const int e = e0 + u4 * kAtThreads;
-      const int qi = e / K, k = e - qi * K;
-      const int64_t i = i0 + qi;
-      cs[u4] = (e < TQ * K && i < D.N_q) ? __ldg(idx + (bg * D.N_q + i) * K + k) : -1;
-    }
-#pragma unroll
-    for (int u4 = 0; u4 < 4; ++u4) {
-      const int c = cs[u4];
-      if (c >= 0 && c < D.C) {
+    for (int k = 0; k < KM; ++k) {
+      const int c = sc[k];
+      if (k % G == h && c >= 0 && c < D.C && ((int64_t)c << rs) <= last_chunk) {
         for (int e2 = 0; e2 <= rs; ++e2) {
           const int tl = (c << rs) + e2;
           atomicOr(&bitmap[tl >> 5], 1u << (tl & 31));
@@ -299,30 +277,43 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
       }
     }
   }
+  // the biases of the row's chunks load while the list is built
+  float bsel[KM];
+#pragma unroll
+  for (int k = 0; k < KM; ++k) {
+    const int c = sc[k];
+    bsel[k] = (c >= 0 && c < D.C) ? __ldg(blm + bg * D.C + c) : 0.f;
+  }
   for (int64_t c = (n_first << rs) + threadIdx.x; c <= last_chunk; c += kAtThreads)
     atomicOr(&bitmap[c >> 5], 1u << (c & 31));
   __syncthreads();
-  {
-    const int per = (nbw + kAtThreads - 1) / kAtThreads;
-    const int w0 = threadIdx.x * per;
-    const int w1 = w0 + per < nbw ? w0 + per : nbw;
-    int cnt = 0;
-    for (int w = w0; w < w1; ++w) cnt += __popc(bitmap[w]);
-    int total;
-    int pos = block_exclusive_scan(cnt, scan, total);
-    for (int w = w0; w < w1; ++w) {
-      uint32_t bits = bitmap[w];
-      wpre[w] = pos;
-      while (bits) {
-        const int bit = __ffs(bits) - 1;
-        bits &= bits - 1;
-        if (pos < list_cap) tiles[pos] = w * 32 + bit;
-        ++pos;
+  if (warp == 0) {
+    // list position of each bitmap word: one warp-wide scan per 32 words
+    int carry = 0;
+    for (int w0 = 0; w0 < nbw; w0 += 32) {
+      const int w = w0 + lane;
+      const int cnt = w < nbw ? __popc(bitmap[w]) : 0;
+      int x = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
       }
+      if (w < nbw) wpre[w] = carry + x - cnt;
+      carry += __shfl_sync(0xffffffffu, x, 31);
     }
-    if (threadIdx.x == 0) {
-      if (total > list_cap) record_status(status, kStatusDeviceCheck);
-      *n_tiles_sh = total < list_cap ? total : list_cap;
+    if (lane == 0) {
+      if (carry > list_cap) record_status(status, kStatusDeviceCheck);
+      *n_tiles_sh = carry < list_cap ? carry : list_cap;
+    }
+  }
+  __syncthreads();
+  // every thread places the set bits of its tiles: the list is the bitmap in ascending order
+  for (int tl = threadIdx.x; tl <= (int)last_chunk; tl += kAtThreads) {
+    const uint32_t wb = bitmap[tl >> 5];
+    if ((wb >> (tl & 31)) & 1u) {
+      const int pos = wpre[tl >> 5] + __popc(wb & ((1u << (tl & 31)) - 1u));
+      if (pos < list_cap) tiles[pos] = tl;
     }
   }
   tc_fence_before();
@@ -406,27 +397,18 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
     }
   } else {
     // ---------------------------------------------------------------- softmax rows
-    const int qd = warp & 3;
-    const int r = qd * 32 + lane;
-    const int h = r / TQ, qi = r - h * TQ;
-    const int64_t i = i0 + qi;
-    const bool valid = i < D.N_q;
     const int64_t pos = D.q_pos0 + (valid ? i : i_last);
     const int64_t n_i = n_eligible(pos, D.S, D.W);
     const int64_t hrow = (b * D.Hq + g * G + h) * D.N_q + i;
-    int sc[KM];
     float su[KM];
     float m_run = -INFINITY;
-#pragma unroll
-    for (int k = 0; k < KM; ++k) {
-      sc[k] = -1;
-      if (valid && k < K) sc[k] = idx[(bg * D.N_q + i) * K + k];
-    }
     // This head's surrogate score of each selected chunk, q_cal . k_lm[c] * scale + b_lm[c].
     // The landmark rows of the first 64 tiles of the (sorted) tile list are staged in shared
     // memory in the K-tile layout and one (128 x d) x (d x 64) product on the tensor core scores
     // every row of the tile against them; a chunk beyond those 64 is scored by a plain dot.
     const int nk = n_tiles < SH::KLM_ROWS ? n_tiles : SH::KLM_ROWS;
+    int rk[KM];   // list position of each selected chunk's first tile (INT_MAX: none)
+    int at[kSelSmem ? KM : 1];   // its place in the row's queue
     {
       constexpr int UPR = DD / 8;   // 16-byte units per landmark row
       const int tid = threadIdx.x - 64;
@@ -437,6 +419,27 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
         const int c = t < nk ? (tiles[t] >> rs) : D.C;   // the tile's chunk
         u[e] = c < D.C ? __ldg(reinterpret_cast<const uint4*>(klm + (bg * D.C + c) * DD) + j)
                        : make_uint4(0u, 0u, 0u, 0u);
+      }
+      // while those rows load: each selected chunk's position in the (sorted) tile list, the
+      // rank of its first tile's bit, and the chunk's place in the row's list-ordered queue
+      // (distinct chunks have distinct ranks)
+#pragma unroll
+      for (int k = 0; k < KM; ++k) {
+        const int c = sc[k];
+        rk[k] = INT_MAX;
+        if (c >= 0 && c < D.C && ((int64_t)c << rs) <= last_chunk) {
+          const int tc = c << rs;
+          rk[k] = wpre[tc >> 5] + __popc(bitmap[tc >> 5] & ((1u << (tc & 31)) - 1u));
+        }
+      }
+      if constexpr (kSelSmem) {
+#pragma unroll
+        for (int k = 0; k < KM; ++k) {
+          int a = 0;
+#pragma unroll
+          for (int k2 = 0; k2 < KM; ++k2) a += rk[k2] < rk[k] ? 1 : 0;
+          at[k] = a;
+        }
       }
 #pragma unroll
       for (int e = 0; e < SH::KLM_ROWS * UPR / 128; ++e) {
@@ -482,23 +485,13 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
           }
         }
       }
-      // the biases first, all loads in flight at once
-      float bsel[KM];
-#pragma unroll
-      for (int k = 0; k < KM; ++k) {
-        const int c = sc[k];
-        bsel[k] = (lm_ok && c >= 0 && c < D.C) ? __ldg(blm + bg * D.C + c) : 0.f;
-      }
 #pragma unroll
       for (int k = 0; k < KM; ++k) {
         su[k] = -INFINITY;
         const int c = sc[k];
-        if (!lm_ok || c < 0 || c >= D.C) continue;
+        if (!lm_ok || rk[k] == INT_MAX) continue;
         const float bias = bsel[k];
-        // the chunk's position in the (sorted) tile list: the rank of its first tile's bit
-        const int tc = c << rs;
-        const int rank = wpre[tc >> 5] + __popc(bitmap[tc >> 5] & ((1u << (tc & 31)) - 1u));
-        const int slot = rank < nk ? rank : -1;
+        const int slot = rk[k] < nk ? rk[k] : -1;
         float a;
         if (slot >= 0) {
           const int col4 = slot >> 2;
@@ -513,18 +506,12 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
     }
     int n_sel = 0;   // selected chunks of this row (kSelSmem: their tile indices are in sel_t)
     if constexpr (kSelSmem) {
-      // order the row's selected chunks by chunk index, which is their order in the tile list
+      // the row's selected chunks in list order (a chunk scored -inf carries weight 0)
 #pragma unroll
       for (int k = 0; k < KM; ++k) {
-        const int c = sc[k];
-        if (c < 0 || c >= D.C || su[k] == -INFINITY) continue;
-        int pos = 0;
-#pragma unroll
-        for (int k2 = 0; k2 < KM; ++k2)
-          pos += (sc[k2] >= 0 && sc[k2] < c && su[k2] != -INFINITY) ? 1 : 0;
-        const int tc = c << rs;   // the chunk's first tile
-        sel_t[r * KM + pos] = wpre[tc >> 5] + __popc(bitmap[tc >> 5] & ((1u << (tc & 31)) - 1u));
-        sel_u[r * KM + pos] = su[k];
+        if (rk[k] == INT_MAX) continue;
+        sel_t[r * KM + at[k]] = rk[k];
+        sel_u[r * KM + at[k]] = su[k];
         ++n_sel;
       }
     }
