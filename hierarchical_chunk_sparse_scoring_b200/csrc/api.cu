@@ -83,7 +83,10 @@ Plan make_plan(const hils_params* p) {
   const size_t head_rows = (size_t)(p->B * p->Hq * p->N_q);
   size_t off = kStatusBytes;
   P.off_idx = off;   off = align_up(off + sel_rows * (size_t)D.K * sizeof(int32_t));
-  if (!P.tc_attn) {   // the tensor-core attention scores the selected chunks itself
+  // per-head scores of the selected chunks: the tensor-core attention takes them from the
+  // scoring kernel when a KV group has one head (sel_rows = head_rows) and otherwise scores the
+  // selected chunks itself
+  if (!P.tc_attn || !P.tc_select || D.G == 1) {
     P.off_ssel = off;
     off = align_up(off + head_rows * (size_t)D.K * sizeof(float));
   }
@@ -229,8 +232,10 @@ hils_status forward_impl(const hils_params* p, const void* q, const void* q_cal,
     pm.mark();
   } else {
     if (P.tc_select) {
-      e = launch_score_topk_tc(P.D, q_cal, k_lm, b_lm, idx, reinterpret_cast<int32_t*>(ws), st);
-      // the tensor-core attention computes the selected chunks' per-head scores itself
+      e = launch_score_topk_tc(P.D, q_cal, k_lm, b_lm, idx,
+                               P.tc_attn && P.D.G == 1 ? s_sel : nullptr,
+                               reinterpret_cast<int32_t*>(ws), st);
+      // the tensor-core attention takes the scores from there, or scores per head itself
       if (e == cudaSuccess && !P.tc_attn) {
         pm.mark();
         e = launch_select_scores(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
@@ -240,7 +245,7 @@ hils_status forward_impl(const hils_params* p, const void* q, const void* q_cal,
     }
     pm.mark();
     if (e == cudaSuccess)
-      e = P.tc_attn ? launch_attn_tc(P.D, q, q_cal, K, V, idx, k_lm, b_lm, out, lse_out,
+      e = P.tc_attn ? launch_attn_tc(P.D, q, q_cal, K, V, idx, s_sel, k_lm, b_lm, out, lse_out,
                                      reinterpret_cast<int32_t*>(ws), st)
                     : launch_attn_rows(P.D, P.bf16, q, K, V, idx, s_sel, out, lse_out, nullptr,
                                        nullptr, st);
@@ -304,8 +309,10 @@ extern "C" hils_status hils_select(const hils_params* p, const void* q_cal, cons
     if (e == cudaSuccess)
       e = launch_select_topk_row(P.D, P.bf16, P.n_stride, sig, q_cal, k_lm, b_lm, idx, s_sel, st);
   } else if (P.tc_select) {
-    e = launch_score_topk_tc(P.D, q_cal, k_lm, b_lm, idx, reinterpret_cast<int32_t*>(ws), st);
-    if (e == cudaSuccess && s_sel)
+    // with one head per KV group the scores the selection ranked by are the per-head scores
+    e = launch_score_topk_tc(P.D, q_cal, k_lm, b_lm, idx, P.D.G == 1 ? s_sel : nullptr,
+                             reinterpret_cast<int32_t*>(ws), st);
+    if (e == cudaSuccess && s_sel && P.D.G != 1)
       e = launch_select_scores(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
   } else {
     e = launch_select_rows(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
@@ -455,8 +462,10 @@ extern "C" hils_status hils_select_noalloc(const hils_params* p, const void* q_c
     if (e == cudaSuccess)
       e = launch_select_merge(P.D, P.bf16, P.n_split, pv, pc, q_cal, k_lm, b_lm, idx, s_sel, st);
   } else if (P.tc_select) {
-    e = launch_score_topk_tc(P.D, q_cal, k_lm, b_lm, idx, reinterpret_cast<int32_t*>(ws), st);
-    if (e == cudaSuccess && s_sel)
+    // with one head per KV group the scores the selection ranked by are the per-head scores
+    e = launch_score_topk_tc(P.D, q_cal, k_lm, b_lm, idx, P.D.G == 1 ? s_sel : nullptr,
+                             reinterpret_cast<int32_t*>(ws), st);
+    if (e == cudaSuccess && s_sel && P.D.G != 1)
       e = launch_select_scores(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
   } else {
     e = launch_select_rows(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);

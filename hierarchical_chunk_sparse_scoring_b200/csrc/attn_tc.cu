@@ -160,8 +160,8 @@ template <int DD, int G, int KM, int RS>
 __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQc,
                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                   Dims D, const int32_t* __restrict__ idx, const __nv_bfloat16* __restrict__ klm,
-                   const float* __restrict__ blm,
+                   Dims D, const int32_t* __restrict__ idx, const float* __restrict__ s_sig,
+                   const __nv_bfloat16* __restrict__ klm, const float* __restrict__ blm,
                    __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out,
                    int list_cap, int bitmap_words, int32_t* __restrict__ status) {
   using SH = AtShape<DD, G>;
@@ -224,11 +224,19 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
   const int h = r / TQ, qi = r - h * TQ;
   const int64_t i = i0 + qi;
   const bool valid = i < D.N_q;
+  // With one head per KV group the row's surrogate score of a selected chunk is the score the
+  // selection ranked it by (s_sig); with several, each head's own score comes from a landmark
+  // product below.
+  constexpr bool kOwnScores = G > 1;
   // the row's selected chunks go out first: they feed both the tile list and the row's scores
   int sc[KM];
+  float su[KM];
 #pragma unroll
-  for (int k = 0; k < KM; ++k)
-    sc[k] = (is_row && valid && k < K) ? __ldg(idx + (bg * D.N_q + i) * K + k) : -1;
+  for (int k = 0; k < KM; ++k) {
+    const bool has = is_row && valid && k < K;
+    sc[k] = has ? __ldg(idx + (bg * D.N_q + i) * K + k) : -1;
+    if constexpr (!kOwnScores) su[k] = has ? __ldg(s_sig + (bg * D.N_q + i) * K + k) : -INFINITY;
+  }
 
   // ---------------------------------------------------------------- barriers, TMEM, tile list
   if (threadIdx.x == 0) {
@@ -254,12 +262,13 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
     // the query and calibrated-query tiles load while the tile list is built
     prefetch_tensormap(&tmQ);
     prefetch_tensormap(&tmQc);
-    mbar_expect_tx(q_full, 2 * SH::Q_BYTES);
+    mbar_expect_tx(q_full, (kOwnScores ? 2 : 1) * SH::Q_BYTES);
     for (int hh = 0; hh < G; ++hh)
       for (int kb = 0; kb < SH::KB; ++kb) {
         const int32_t y = (int32_t)((b * D.Hq + g * G + hh) * D.N_q + i0);
         tma_load_2d(sQ + kb * SH::Q_BOX + hh * TQ * 128, &tmQ, kb * 64, y, q_full);
-        tma_load_2d(sQc + kb * SH::Q_BOX + hh * TQ * 128, &tmQc, kb * 64, y, q_full);
+        if constexpr (kOwnScores)
+          tma_load_2d(sQc + kb * SH::Q_BOX + hh * TQ * 128, &tmQc, kb * 64, y, q_full);
       }
   }
   // selected chunks of every valid query of the tile (the G rows of a query hold the same
@@ -278,11 +287,13 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
     }
   }
   // the biases of the row's chunks load while the list is built
-  float bsel[KM];
+  float bsel[kOwnScores ? KM : 1];
+  if constexpr (kOwnScores) {
 #pragma unroll
-  for (int k = 0; k < KM; ++k) {
-    const int c = sc[k];
-    bsel[k] = (c >= 0 && c < D.C) ? __ldg(blm + bg * D.C + c) : 0.f;
+    for (int k = 0; k < KM; ++k) {
+      const int c = sc[k];
+      bsel[k] = (c >= 0 && c < D.C) ? __ldg(blm + bg * D.C + c) : 0.f;
+    }
   }
   for (int64_t c = (n_first << rs) + threadIdx.x; c <= last_chunk; c += kAtThreads)
     atomicOr(&bitmap[c >> 5], 1u << (c & 31));
@@ -400,29 +411,13 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
     const int64_t pos = D.q_pos0 + (valid ? i : i_last);
     const int64_t n_i = n_eligible(pos, D.S, D.W);
     const int64_t hrow = (b * D.Hq + g * G + h) * D.N_q + i;
-    float su[KM];
     float m_run = -INFINITY;
-    // This head's surrogate score of each selected chunk, q_cal . k_lm[c] * scale + b_lm[c].
-    // The landmark rows of the first 64 tiles of the (sorted) tile list are staged in shared
-    // memory in the K-tile layout and one (128 x d) x (d x 64) product on the tensor core scores
-    // every row of the tile against them; a chunk beyond those 64 is scored by a plain dot.
-    const int nk = n_tiles < SH::KLM_ROWS ? n_tiles : SH::KLM_ROWS;
     int rk[KM];   // list position of each selected chunk's first tile (INT_MAX: none)
     int at[kSelSmem ? KM : 1];   // its place in the row's queue
-    {
-      constexpr int UPR = DD / 8;   // 16-byte units per landmark row
-      const int tid = threadIdx.x - 64;
-      uint4 u[SH::KLM_ROWS * UPR / 128];
-#pragma unroll
-      for (int e = 0; e < SH::KLM_ROWS * UPR / 128; ++e) {
-        const int f = tid + e * 128, t = f / UPR, j = f - t * UPR;
-        const int c = t < nk ? (tiles[t] >> rs) : D.C;   // the tile's chunk
-        u[e] = c < D.C ? __ldg(reinterpret_cast<const uint4*>(klm + (bg * D.C + c) * DD) + j)
-                       : make_uint4(0u, 0u, 0u, 0u);
-      }
-      // while those rows load: each selected chunk's position in the (sorted) tile list, the
-      // rank of its first tile's bit, and the chunk's place in the row's list-ordered queue
-      // (distinct chunks have distinct ranks)
+    // each selected chunk's position in the (sorted) tile list, the rank of its first tile's
+    // bit, and the chunk's place in the row's list-ordered queue (distinct chunks have distinct
+    // ranks)
+    auto rank_chunks = [&]() {
 #pragma unroll
       for (int k = 0; k < KM; ++k) {
         const int c = sc[k];
@@ -441,31 +436,51 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
           at[k] = a;
         }
       }
+    };
+    bool lm_ok = true;
+    if constexpr (kOwnScores) {
+      // This head's surrogate score of each selected chunk, q_cal . k_lm[c] * scale + b_lm[c].
+      // The landmark rows of the first 64 tiles of the (sorted) tile list are staged in shared
+      // memory in the K-tile layout and one (128 x d) x (d x 64) product on the tensor core
+      // scores every row of the tile against them; a chunk beyond those 64 is scored by a
+      // plain dot.
+      const int nk = n_tiles < SH::KLM_ROWS ? n_tiles : SH::KLM_ROWS;
+      {
+        constexpr int UPR = DD / 8;   // 16-byte units per landmark row
+        const int tid = threadIdx.x - 64;
+        uint4 u[SH::KLM_ROWS * UPR / 128];
 #pragma unroll
-      for (int e = 0; e < SH::KLM_ROWS * UPR / 128; ++e) {
-        const int f = tid + e * 128, t = f / UPR, j = f - t * UPR;
-        const int kb = j >> 3, jj = j & 7;
-        *reinterpret_cast<uint4*>(sKlm + kb * SH::KV_BOX + (t >> 3) * 1024 + (t & 7) * 128 +
-                                  ((jj ^ (t & 7)) << 4)) = u[e];
-      }
-      fence_async_smem();
-      asm volatile("bar.sync 1, 128;" ::: "memory");   // the four softmax warps
-    }
-    const bool q_ok = mbar_wait_warp(q_full, 0, kAtPollLimit);
-    if (warp == 2 && lane == 0 && q_ok) {
-      tc_fence_after();
-      constexpr uint32_t IDESC_LM = idesc_bf16_f32(kAtRows, SH::KLM_ROWS);
+        for (int e = 0; e < SH::KLM_ROWS * UPR / 128; ++e) {
+          const int f = tid + e * 128, t = f / UPR, j = f - t * UPR;
+          const int c = t < nk ? (tiles[t] >> rs) : D.C;   // the tile's chunk
+          u[e] = c < D.C ? __ldg(reinterpret_cast<const uint4*>(klm + (bg * D.C + c) * DD) + j)
+                         : make_uint4(0u, 0u, 0u, 0u);
+        }
+        rank_chunks();   // while those rows load
 #pragma unroll
-      for (int ks = 0; ks < DD / 16; ++ks) {
-        const int kb = ks >> 2, kin = ks & 3;
-        const uint64_t ad = desc_kmajor_sw128(smem_u32(sQc + kb * SH::Q_BOX) + kin * 32);
-        const uint64_t bd = desc_kmajor_sw128(smem_u32(sKlm + kb * SH::KV_BOX) + kin * 32);
-        mma_bf16_ss(tmem + SH::LM_COL, ad, bd, IDESC_LM, ks > 0 ? 1u : 0u);
+        for (int e = 0; e < SH::KLM_ROWS * UPR / 128; ++e) {
+          const int f = tid + e * 128, t = f / UPR, j = f - t * UPR;
+          const int kb = j >> 3, jj = j & 7;
+          *reinterpret_cast<uint4*>(sKlm + kb * SH::KV_BOX + (t >> 3) * 1024 + (t & 7) * 128 +
+                                    ((jj ^ (t & 7)) << 4)) = u[e];
+        }
+        fence_async_smem();
+        asm volatile("bar.sync 1, 128;" ::: "memory");   // the four softmax warps
       }
-      mma_commit(lm_done);
-    }
-    const bool lm_ok = q_ok && mbar_wait_warp(lm_done, 0, kAtPollLimit);
-    {
+      const bool q_ok = mbar_wait_warp(q_full, 0, kAtPollLimit);
+      if (warp == 2 && lane == 0 && q_ok) {
+        tc_fence_after();
+        constexpr uint32_t IDESC_LM = idesc_bf16_f32(kAtRows, SH::KLM_ROWS);
+#pragma unroll
+        for (int ks = 0; ks < DD / 16; ++ks) {
+          const int kb = ks >> 2, kin = ks & 3;
+          const uint64_t ad = desc_kmajor_sw128(smem_u32(sQc + kb * SH::Q_BOX) + kin * 32);
+          const uint64_t bd = desc_kmajor_sw128(smem_u32(sKlm + kb * SH::KV_BOX) + kin * 32);
+          mma_bf16_ss(tmem + SH::LM_COL, ad, bd, IDESC_LM, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(lm_done);
+      }
+      lm_ok = q_ok && mbar_wait_warp(lm_done, 0, kAtPollLimit);
       // the row's 64 landmark scores, parked in this thread's own P rows of both buffers (the
       // staged landmark rows there are dead: their product completed), 16-byte slots rotated
       uint8_t* park = sP + r * 128;
@@ -501,6 +516,13 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
           a = lm_dot<SH::KB, SH::Q_BOX>(sQc, r, klm + (bg * D.C + c) * DD);
         }
         su[k] = fmaf(a, D.scale, bias);
+        m_run = fmaxf(m_run, su[k]);
+      }
+    } else {
+      rank_chunks();
+#pragma unroll
+      for (int k = 0; k < KM; ++k) {
+        if (rk[k] == INT_MAX) su[k] = -INFINITY;
         m_run = fmaxf(m_run, su[k]);
       }
     }
@@ -776,7 +798,8 @@ int list_capacity(const Dims& D, int TQ) {
 
 template <int DD, int G, int KM, int RS>
 cudaError_t launch_at_t(const Dims& D, const void* q, const void* qc, const void* K,
-                        const void* V, const int32_t* idx, const void* klm, const float* blm,
+                        const void* V, const int32_t* idx, const float* s_sig, const void* klm,
+                        const float* blm,
                         void* out, float* lse, int32_t* status, cudaStream_t st) {
   using SH = AtShape<DD, G>;
   CUtensorMap tmQ, tmQc, tmK, tmV;
@@ -793,7 +816,7 @@ cudaError_t launch_at_t(const Dims& D, const void* q, const void* qc, const void
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((D.N_q + SH::TQ - 1) / SH::TQ), (unsigned)(D.B * D.Hkv));
-  kern<<<grid, kAtThreads, smem, st>>>(tmQ, tmQc, tmK, tmV, D, idx,
+  kern<<<grid, kAtThreads, smem, st>>>(tmQ, tmQc, tmK, tmV, D, idx, s_sig,
                                        (const __nv_bfloat16*)klm, blm, (__nv_bfloat16*)out, lse,
                                        cap, words, status);
   return cudaGetLastError();
@@ -801,23 +824,25 @@ cudaError_t launch_at_t(const Dims& D, const void* q, const void* qc, const void
 
 template <int DD, int G>
 cudaError_t launch_at_k(const Dims& D, const void* q, const void* qc, const void* K,
-                        const void* V, const int32_t* idx, const void* klm, const float* blm,
+                        const void* V, const int32_t* idx, const float* s_sig, const void* klm,
+                        const float* blm,
                         void* out, float* lse, int32_t* status, cudaStream_t st) {
   if constexpr (DD == 128) {
     // chunks of 128 tokens (two tiles per chunk) are built for d = 128 only
     if (D.S == 2 * kTile) {
       if (D.K <= 8)
-        return launch_at_t<DD, G, 8, 1>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st);
+        return launch_at_t<DD, G, 8, 1>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status,
+                                        st);
       if (D.K <= 16)
-        return launch_at_t<DD, G, 16, 1>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st);
-      return launch_at_t<DD, G, 32, 1>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st);
+        return launch_at_t<DD, G, 16, 1>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status, st);
+      return launch_at_t<DD, G, 32, 1>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status, st);
     }
   }
   if (D.K <= 8)
-    return launch_at_t<DD, G, 8, 0>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st);
+    return launch_at_t<DD, G, 8, 0>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status, st);
   if (D.K <= 16)
-    return launch_at_t<DD, G, 16, 0>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st);
-  return launch_at_t<DD, G, 32, 0>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st);
+    return launch_at_t<DD, G, 16, 0>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status, st);
+  return launch_at_t<DD, G, 32, 0>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status, st);
 }
 
 }  // namespace
@@ -839,11 +864,12 @@ bool attn_tc_supported(const Dims& D, bool bf16) {
 }
 
 cudaError_t launch_attn_tc(const Dims& D, const void* q, const void* qc, const void* K,
-                           const void* V, const int32_t* idx, const void* klm, const float* blm,
+                           const void* V, const int32_t* idx, const float* s_sig, const void* klm,
+                        const float* blm,
                            void* out, float* lse, int32_t* status, cudaStream_t st) {
   if (D.B * D.Hq * D.N_q == 0) return cudaSuccess;
 #define HILS_AT(DD, GG) \
-  return launch_at_k<DD, GG>(D, q, qc, K, V, idx, klm, blm, out, lse, status, st)
+  return launch_at_k<DD, GG>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status, st)
   if (D.d == 128) {
     if (D.G == 1) HILS_AT(128, 1);
     if (D.G == 2) HILS_AT(128, 2);

@@ -17,14 +17,18 @@ cudaError_t launch_select_scores(const Dims& D, bool bf16, const void* qc, const
                                  cudaStream_t st);
 
 bool score_tc_supported(const Dims& D, bool bf16);
+// s_out (nullable): the winners' scores sigma, laid out like idx (-inf where idx is -1)
 cudaError_t launch_score_topk_tc(const Dims& D, const void* qc, const void* klm,
-                                 const float* blm, int32_t* idx, int32_t* status,
+                                 const float* blm, int32_t* idx, float* s_out, int32_t* status,
                                  cudaStream_t st);
 
 bool attn_tc_supported(const Dims& D, bool bf16);
+// s_sig: the scoring kernel's sigma of each selected chunk, required when D.G == 1 (it is then
+// the head's surrogate score); with G > 1 the kernel scores the selected chunks per head itself
 cudaError_t launch_attn_tc(const Dims& D, const void* q, const void* qc, const void* K,
-                           const void* V, const int32_t* idx, const void* klm, const float* blm,
-                           void* out, float* lse, int32_t* status, cudaStream_t st);
+                           const void* V, const int32_t* idx, const float* s_sig,
+                           const void* klm, const float* blm, void* out, float* lse,
+                           int32_t* status, cudaStream_t st);
 
 size_t split_smem_bytes(int cps);
 cudaError_t launch_select_split(const Dims& D, bool bf16, int cps, int n_split, const void* qc,

@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(64 + 128 * NCG, CPS)
     score_topk_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB, Dims D,
                          const float* __restrict__ blm, int32_t* __restrict__ idx,
-                         int32_t* __restrict__ status) {
+                         float* __restrict__ s_out, int32_t* __restrict__ status) {
   using SH = TcShape<DD, G, KM, NCG, HP, CPS>;
   constexpr int NT = SH::NT;
   constexpr int GV = SH::GV;
@@ -396,6 +396,14 @@ __global__ void __launch_bounds__(64 + 128 * NCG, CPS)
 #pragma unroll
       for (int k = 0; k < KM; ++k)
         if (k >= KM - K) out[k] = (L.c[k] == INT_MAX) ? -1 : L.c[k];
+      if (s_out) {
+        // the winners' scores sigma (with one head per group, that head's surrogate score)
+        float* so = s_out + (bg * D.N_q + i) * K - (KM - K);
+#pragma unroll
+        for (int k = 0; k < KM; ++k)
+          if (k >= KM - K)   // (a -inf score was kept as -FLT_MAX in the list)
+            so[k] = (L.c[k] == INT_MAX || L.v[k] <= -FLT_MAX) ? -INFINITY : L.v[k];
+      }
     }
   }
   tc_fence_before();
@@ -437,7 +445,7 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t d, uin
 
 template <int DD, int G, int KM, int NCG, int HP, int CPS>
 cudaError_t launch_tc_t(const Dims& D, const void* qc, const void* klm, const float* blm,
-                        int32_t* idx, int32_t* status, cudaStream_t st) {
+                        int32_t* idx, float* s_out, int32_t* status, cudaStream_t st) {
   using SH = TcShape<DD, G, KM, NCG, HP, CPS>;
   CUtensorMap tmA, tmB;
   bool ok_a;
@@ -463,13 +471,13 @@ cudaError_t launch_tc_t(const Dims& D, const void* qc, const void* klm, const fl
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SH::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((D.N_q + SH::MQ - 1) / SH::MQ), (unsigned)(D.B * D.Hkv));
-  kern<<<grid, SH::THREADS, SH::SMEM, st>>>(tmA, tmB, D, blm, idx, status);
+  kern<<<grid, SH::THREADS, SH::SMEM, st>>>(tmA, tmB, D, blm, idx, s_out, status);
   return cudaGetLastError();
 }
 
 template <int DD, int G>
 cudaError_t launch_tc_k(const Dims& D, const void* qc, const void* klm, const float* blm,
-                        int32_t* idx, int32_t* status, cudaStream_t st) {
+                        int32_t* idx, float* s_out, int32_t* status, cudaStream_t st) {
   // Two column groups: with four, the 18 warps cap a thread at 96 registers and the slower
   // epilogue (spills, fewer TMEM loads in flight) outweighs the extra latency hiding.
   // the list length follows K: an insertion costs a compare and two selects per slot
@@ -479,11 +487,11 @@ cudaError_t launch_tc_k(const Dims& D, const void* qc, const void* klm, const fl
     // small query tiles and short lists: two CTAs per SM (each one's epilogue latency hides
     // behind the other's)
     if constexpr (DD == 64 && G <= 2)
-      return launch_tc_t<DD, G, 8, 2, HP, 2>(D, qc, klm, blm, idx, status, st);
-    return launch_tc_t<DD, G, 8, 2, HP, 1>(D, qc, klm, blm, idx, status, st);
+      return launch_tc_t<DD, G, 8, 2, HP, 2>(D, qc, klm, blm, idx, s_out, status, st);
+    return launch_tc_t<DD, G, 8, 2, HP, 1>(D, qc, klm, blm, idx, s_out, status, st);
   }
-  if (D.K <= 16) return launch_tc_t<DD, G, 16, 2, HP, 1>(D, qc, klm, blm, idx, status, st);
-  return launch_tc_t<DD, G, 32, 2, HP, 1>(D, qc, klm, blm, idx, status, st);
+  if (D.K <= 16) return launch_tc_t<DD, G, 16, 2, HP, 1>(D, qc, klm, blm, idx, s_out, status, st);
+  return launch_tc_t<DD, G, 32, 2, HP, 1>(D, qc, klm, blm, idx, s_out, status, st);
 }
 
 }  // namespace
@@ -497,19 +505,19 @@ bool score_tc_supported(const Dims& D, bool bf16) {
 }
 
 cudaError_t launch_score_topk_tc(const Dims& D, const void* qc, const void* klm,
-                                 const float* blm, int32_t* idx, int32_t* status,
+                                 const float* blm, int32_t* idx, float* s_out, int32_t* status,
                                  cudaStream_t st) {
   if (D.B * D.Hkv * D.N_q == 0) return cudaSuccess;
   if (D.d == 128) {
-    if (D.G == 1) return launch_tc_k<128, 1>(D, qc, klm, blm, idx, status, st);
-    if (D.G == 2) return launch_tc_k<128, 2>(D, qc, klm, blm, idx, status, st);
-    if (D.G == 4) return launch_tc_k<128, 4>(D, qc, klm, blm, idx, status, st);
-    return launch_tc_k<128, 8>(D, qc, klm, blm, idx, status, st);
+    if (D.G == 1) return launch_tc_k<128, 1>(D, qc, klm, blm, idx, s_out, status, st);
+    if (D.G == 2) return launch_tc_k<128, 2>(D, qc, klm, blm, idx, s_out, status, st);
+    if (D.G == 4) return launch_tc_k<128, 4>(D, qc, klm, blm, idx, s_out, status, st);
+    return launch_tc_k<128, 8>(D, qc, klm, blm, idx, s_out, status, st);
   }
-  if (D.G == 1) return launch_tc_k<64, 1>(D, qc, klm, blm, idx, status, st);
-  if (D.G == 2) return launch_tc_k<64, 2>(D, qc, klm, blm, idx, status, st);
-  if (D.G == 4) return launch_tc_k<64, 4>(D, qc, klm, blm, idx, status, st);
-  return launch_tc_k<64, 8>(D, qc, klm, blm, idx, status, st);
+  if (D.G == 1) return launch_tc_k<64, 1>(D, qc, klm, blm, idx, s_out, status, st);
+  if (D.G == 2) return launch_tc_k<64, 2>(D, qc, klm, blm, idx, s_out, status, st);
+  if (D.G == 4) return launch_tc_k<64, 4>(D, qc, klm, blm, idx, s_out, status, st);
+  return launch_tc_k<64, 8>(D, qc, klm, blm, idx, s_out, status, st);
 }
 
 }  // namespace hils
