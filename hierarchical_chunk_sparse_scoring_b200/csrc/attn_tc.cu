@@ -23,8 +23,8 @@
 //
 // CTA = (b, g, 128/G queries); 6 warps: warp 0 TMA (Q once, then K and V tiles of the union),
 // warp 1 TMEM owner and MMA issuer (S = Q K^T into a double-buffered TMEM tile, O += P V into a
-// TMEM accumulator), warps 2-5 one row per thread (classification, softmax, P to shared memory
-// in the 128-byte-swizzled K-major layout the P V product reads).
+// TMEM accumulator, P read from TMEM as the A operand), warps 2-5 one row per thread
+// (classification, softmax, the row's P as bf16 into its own TMEM lane).
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -51,7 +51,9 @@ struct AtShape {
   static constexpr int Q_BYTES = KB * Q_BOX;
   static constexpr int KV_BOX = kTile * 128;             // [64 tokens x 64]
   static constexpr int KV_BYTES = KB * KV_BOX;           // one K (or V) tile
-  static constexpr int P_BYTES = kAtRows * 128;          // [128 rows x 64 tokens] bf16
+  // prologue scratch (two [128 x 128-byte] areas): the staged landmark rows, then each row's
+  // parked landmark scores
+  static constexpr int P_BYTES = kAtRows * 128;
   // K/V ring: STAGES_MAIN stage pairs of their own, plus one that reuses the calibrated-query
   // tile once the selected chunks' scores have been taken from it (same size: Q_BYTES = 2 KV)
   // d = 64: two CTAs per SM (each one's prologue and softmax latency hide behind the other's)
@@ -62,11 +64,15 @@ struct AtShape {
   static constexpr int KLM_BYTES = KB * KLM_ROWS * 128;  // same swizzled layout as a K tile
   static constexpr int FIXED = 2 * Q_BYTES /*q and q_cal*/ + STAGES_MAIN * 2 * KV_BYTES +
                                2 * P_BYTES + 1024 /*bars*/ + 1024 /*align*/ + 1024 /*scan*/;
-  static_assert(KLM_BYTES <= 2 * P_BYTES, "landmark rows overlay the P buffers");
-  // TMEM: S[2] (2 x 64 columns), O (DD), the landmark scores (64); a power of two
+  static_assert(KLM_BYTES <= 2 * P_BYTES, "landmark rows fit the prologue scratch");
+  // TMEM: S[2] (2 x 64 columns), O (DD), the landmark scores (64); a power of two.  Once the
+  // landmark scores are read, their columns hold P[2]: 64 bf16 per row, two per column, the A
+  // operand of the P V product.
   static constexpr uint32_t O_COL = 128;
   static constexpr uint32_t LM_COL = O_COL + DD;
+  static constexpr uint32_t P_COL = LM_COL;
   static constexpr uint32_t TMEM_COLS = LM_COL + 64 <= 256 ? 256 : 512;
+  static_assert(P_COL + 2 * (kTile / 2) <= TMEM_COLS, "P buffers in TMEM");
   // co-resident CTAs never exceed the SM's 512 TMEM columns: d = 64 runs two CTAs per SM on 256
   // columns each; d = 128 needs 512 and its shared memory footprint keeps a second CTA away
   static_assert(DD == 64 ? (TMEM_COLS == 256 && FIXED < 232448 / 2 - 8192)
@@ -181,8 +187,8 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
   auto stage_v = [&](int s) -> uint8_t* {
     return s < SH::STAGES_MAIN ? sV + s * SH::KV_BYTES : sQc + SH::KV_BYTES;
   };
-  // landmark rows of the first 64 tiles (K-tile layout); dead once their product has completed,
-  // before any P row is written
+  // landmark rows of the first 64 tiles (K-tile layout) in the prologue scratch; dead once their
+  // product has completed
   uint8_t* sKlm = sP;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * SH::P_BYTES);
   uint64_t* kv_full = bars;                       // [STAGES]
@@ -393,10 +399,11 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < kTile / 16; ++ks) {
-          const uint64_t ad = desc_kmajor_sw128(smem_u32(sP + x * SH::P_BYTES) + ks * 32);
+          // 16 tokens of P = 8 TMEM columns
+          const uint32_t at = tmem + SH::P_COL + (uint32_t)(x * (kTile / 2) + ks * 8);
           const uint64_t bd = desc_mnmajor_sw128(
               smem_u32(stage_v(s)) + ks * 16 * 128, SH::KV_BOX);
-          mma_bf16_ss(tmem + SH::O_COL, ad, bd, IDESC_PV, (t > 0 || ks > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + SH::O_COL, at, bd, IDESC_PV, (t > 0 || ks > 0) ? 1u : 0u);
         }
         mma_commit(&kv_empty[s]);
         mma_commit(&p_empty[x]);
@@ -481,8 +488,9 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
         mma_commit(lm_done);
       }
       lm_ok = q_ok && mbar_wait_warp(lm_done, 0, kAtPollLimit);
-      // the row's 64 landmark scores, parked in this thread's own P rows of both buffers (the
-      // staged landmark rows there are dead: their product completed), 16-byte slots rotated
+      // the row's 64 landmark scores, parked in this thread's own 128-byte rows of both scratch
+      // areas (the staged landmark rows there are dead: their product completed), 16-byte slots
+      // rotated
       uint8_t* park = sP + r * 128;
       if (lm_ok) {
         tc_fence_after();
@@ -547,7 +555,6 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
     int sel_next = 0;
     int sel_tn = (kSelSmem && n_sel > 0) ? sel_t[r * KM] : -1;
     const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
-    uint8_t* prow_base = sP + (r >> 3) * 1024 + (r & 7) * 128;
     bool ok = true;
     for (int t = 0; t < n_tiles; ++t) {
       const int x = t & 1;
@@ -710,17 +717,15 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
         }
         tmem_wait_st();
       }
-      uint8_t* prow = prow_base + x * SH::P_BYTES;
+      // the row's P into its TMEM lane: 64 bf16 in 32 columns
 #pragma unroll
-      for (int k8 = 0; k8 < kTile / 8; ++k8) {
-        uint4 w4;
-        w4.x = pack_bf16(p[8 * k8 + 0], p[8 * k8 + 1]);
-        w4.y = pack_bf16(p[8 * k8 + 2], p[8 * k8 + 3]);
-        w4.z = pack_bf16(p[8 * k8 + 4], p[8 * k8 + 5]);
-        w4.w = pack_bf16(p[8 * k8 + 6], p[8 * k8 + 7]);
-        *reinterpret_cast<uint4*>(prow + ((k8 ^ (r & 7)) << 4)) = w4;
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(p[32 * hf + 2 * e], p[32 * hf + 2 * e + 1]);
+        tmem_st16u(lane_base + SH::P_COL + (uint32_t)(x * (kTile / 2) + 16 * hf), pk);
       }
-      fence_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[x]);
