@@ -6,6 +6,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 from hierarchical_chunk_sparse_scoring_b200 import binding as hb
 from hierarchical_chunk_sparse_scoring_b200 import build as hbuild
@@ -65,6 +66,21 @@ def test_workspace_size(lib):
     assert dec > 256
     assert hb.workspace_size(_params(K_top=33)) == 0      # unsupported -> 0
     assert hb.workspace_size(_params(Hq=6, Hkv=4)) == 0   # Hq % Hkv != 0
+
+
+def test_prefill_workspace_layout(lib):
+    # status word, then idx [B, Hkv, N_q, K]; per-head scores [B, Hq, N_q, K] only where the
+    # tensor-core attention does not score the selected chunks itself: one head per KV group
+    # (it takes the scoring kernel's sigma of the winners) or no tensor-core path (fp32)
+    def rup(x):
+        return (x + 255) // 256 * 256
+    nq, k = 4096, 16
+    gqa = hb.workspace_size(_params(Hq=8, Hkv=2, N_q=nq, N_kv=nq, K_top=k))
+    assert gqa == 256 + rup(2 * nq * k * 4)
+    mha = hb.workspace_size(_params(Hq=8, Hkv=8, N_q=nq, N_kv=nq, K_top=k))
+    assert mha == 256 + rup(8 * nq * k * 4) + rup(8 * nq * k * 4)
+    f32 = hb.workspace_size(_params(Hq=8, Hkv=2, N_q=nq, N_kv=nq, K_top=k, dtype=torch.float32))
+    assert f32 == 256 + rup(2 * nq * k * 4) + rup(8 * nq * k * 4)
 
 
 BAD = [
