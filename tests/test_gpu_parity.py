@@ -98,6 +98,9 @@ EDGE_CASES = {
     "tc_g2_d128": dict(B=1, Hq=4, Hkv=2, N=3000, d=128, S=64, K=8, W_=128),
     "tc_g8_d64": dict(B=1, Hq=8, Hkv=1, N=2500, d=64, S=32, K=16, W_=64),
     "tc_g1_d128": dict(B=2, Hq=2, Hkv=2, N=5000, d=128, S=64, K=16, W_=256),
+    # one head per group with K > 16: the attention's per-row scan of the selection, scores
+    # taken from the selection kernel
+    "tc_g1_k24": dict(B=1, Hq=2, Hkv=2, N=5000, d=64, S=64, K=24, W_=128),
     "tc_g4_k32": dict(B=1, Hq=8, Hkv=2, N=6000, d=128, S=64, K=32, W_=128),
     "tc_s128": dict(B=1, Hq=4, Hkv=1, N=9000, d=128, S=128, K=16, W_=256),
     "tc_many_tiles": dict(B=1, Hq=4, Hkv=4, N=20000, d=64, S=16, K=8, W_=64),
@@ -140,6 +143,7 @@ def test_selection_is_deterministic():
 
 
 @pytest.mark.parametrize("name,kw", [("gqa7b_prefill", dict(N=4096)),
+                                     ("small_mha_bf16", dict(B=1, Hq=4, Hkv=4, N=2048)),
                                      ("long_decode", dict(B=3, N=40000)),
                                      ("tiny_fp32", {})])
 def test_select_step(name, kw):
