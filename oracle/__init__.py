@@ -61,6 +61,10 @@ def lib():
         l.hils_oracle_forward.restype = ctypes.c_int
         l.hils_oracle_forward.argtypes = [ctypes.POINTER(Problem)] + [ctypes.c_void_p] * 15 + [
             ctypes.c_int]
+        l.hils_oracle_landmarks.restype = ctypes.c_int
+        l.hils_oracle_landmarks.argtypes = [ctypes.c_int64] * 4 + [ctypes.c_int32,
+                                                                   ctypes.c_double] + [
+            ctypes.c_void_p] * 4
         l.hils_oracle_n_eligible.restype = ctypes.c_int64
         l.hils_oracle_n_eligible.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32]
         l.hils_oracle_default_threads.restype = ctypes.c_int
@@ -121,6 +125,22 @@ def forward(q, qc, K, V, klm, blm, *, S, K_top, W, q_pos0=0, scale=0.0, idx_in=N
     if rc != 0:
         raise RuntimeError("hils_oracle_forward failed with status %d" % rc)
     return r
+
+
+def landmarks(qlm, K, *, S, scale=0.0):
+    """Landmark construction (R15): qlm [B,Hkv,C,d] landmark queries, K [B,Hkv,N_kv,d] keys,
+    C = N_kv // S.  Returns (klm [B,Hkv,C,d], blm [B,Hkv,C])."""
+    qlm, K = _f64(qlm), _f64(K)
+    B, Hkv, Nkv, d = K.shape
+    C = Nkv // S if S > 0 else 0   # (S <= 0 is rejected by the C side)
+    assert qlm.shape == (B, Hkv, C, d), (qlm.shape, (B, Hkv, C, d))
+    klm = np.empty((B, Hkv, C, d))
+    blm = np.empty((B, Hkv, C))
+    rc = lib().hils_oracle_landmarks(B, Hkv, Nkv, d, S, float(scale), _ptr(qlm), _ptr(K),
+                                     _ptr(klm), _ptr(blm))
+    if rc != 0:
+        raise RuntimeError("hils_oracle_landmarks failed with status %d" % rc)
+    return klm, blm
 
 
 class Query:

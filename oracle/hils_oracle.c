@@ -337,3 +337,38 @@ int hils_oracle_forward(const hils_oracle_problem* pr, const double* q, const do
   free(jobs);
   return rc;
 }
+
+int hils_oracle_landmarks(int64_t B, int64_t Hkv, int64_t N_kv, int64_t d, int32_t S,
+                          double scale, const double* qlm, const double* K, double* klm,
+                          double* blm) {
+  if (B < 0 || Hkv <= 0 || N_kv < 0 || d <= 0 || S <= 0) return HILS_ORACLE_EINVAL;
+  const int64_t C = N_kv / S;
+  const double sc = scale > 0.0 ? scale : 1.0 / sqrt((double)d);
+  double* x = (double*)malloc((size_t)S * sizeof(double));
+  if (!x) return HILS_ORACLE_ENOMEM;
+  for (int64_t bg = 0; bg < B * Hkv; ++bg)
+    for (int64_t c = 0; c < C; ++c) {
+      const double* qv = qlm + (bg * C + c) * d;
+      const double* Kc = K + (bg * N_kv + c * S) * d;   /* the chunk's S keys */
+      double* kout = klm + (bg * C + c) * d;
+      /* the landmark query's logits and their softmax */
+      double m = -INFINITY;
+      for (int32_t j = 0; j < S; ++j) {
+        x[j] = sc * dot(qv, Kc + (int64_t)j * d, (int)d);
+        if (x[j] > m) m = x[j];
+      }
+      double z = 0.0;
+      for (int32_t j = 0; j < S; ++j) z += exp(x[j] - m);
+      /* summary key and entropy bias */
+      for (int64_t e = 0; e < d; ++e) kout[e] = 0.0;
+      double h = 0.0;
+      for (int32_t j = 0; j < S; ++j) {
+        const double pj = exp(x[j] - m) / z;
+        for (int64_t e = 0; e < d; ++e) kout[e] += pj * Kc[(int64_t)j * d + e];
+        if (pj > 0.0) h -= pj * log(pj);
+      }
+      blm[bg * C + c] = h;
+    }
+  free(x);
+  return HILS_ORACLE_OK;
+}

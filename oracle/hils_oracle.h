@@ -47,6 +47,17 @@
  *   R9  (packing) every query attends only its own selected chunks.
  *   R10 a bias of -inf is allowed (that chunk gets weight 0); NaN inputs are undefined.
  *   R11 decode: the query sits at p = N_kv - 1 and the cache already holds its token.
+ *   R15 landmark construction: one landmark query per completed chunk; its logits against the
+ *       chunk's keys use the same `scale` as step 1, so that the surrogate score at the
+ *       expansion point equals the chunk's log-mass exactly.
+ *
+ * Upstream of step 1, the producer of klm/blm (landmark construction):
+ *   p = softmax_j(scale * qlm_c . K_j) over the chunk's S keys; klm_c = sum_j p_j K_j;
+ *   blm_c = H(p) = -sum_j p_j log p_j ([Reader] "The HiLS-Attention Mechanism": the chunk
+ *   summary is the p-weighted sum of the chunk's keys and its bias the entropy of p; [Reader]
+ *   "Paper Primer": the surrogate is a first-order Taylor expansion of the full-attention chunk
+ *   mass, calibrated by an entropy term; [DevTo] "The Core Idea: Landmark Tokens and
+ *   Hierarchical Factorization").
  *
  * Every function here is pinned by CPU tests against values the pages print, closed forms
  * and brute force (no function is "parity unpinned").
@@ -127,6 +138,15 @@ int hils_oracle_forward(const hils_oracle_problem* pr, const double* q, const do
                         const int32_t* idx_in, int32_t* idx_out, double* sigma_out,
                         double* gap_out, double* s_sel_out, double* out, double* lse_out,
                         double* unit_o_out, double* unit_lse_out, int n_threads);
+
+/* Landmark construction (R15): for every (b, g) and completed chunk c < C = floor(N_kv / S),
+ *   x_j = scale * qlm[b,g,c] . K[b,g,c*S+j] (j < S), p = softmax(x),
+ *   klm[b,g,c] = sum_j p_j K[b,g,c*S+j],  blm[b,g,c] = -sum_{j: p_j > 0} p_j log p_j.
+ * qlm, klm [B,Hkv,C,d]; K [B,Hkv,N_kv,d]; blm [B,Hkv,C].  scale <= 0 means 1/sqrt(d).  The
+ * tokens of a partial last chunk get no landmark (R8). */
+int hils_oracle_landmarks(int64_t B, int64_t Hkv, int64_t N_kv, int64_t d, int32_t S,
+                          double scale, const double* qlm, const double* K, double* klm,
+                          double* blm);
 
 /* Rule R1: number of eligible distant chunks of the query at position pos. */
 int64_t hils_oracle_n_eligible(int64_t pos, int32_t S, int32_t W);

@@ -203,6 +203,112 @@ def test_exact_surrogates_select_like_block_sparse_attention():
     assert [int(c) for c in r["idx"][0, 0, 0]] == bsa
 
 
+# ---------------------------------------------------------------- landmark construction (R15)
+def _lse(x):
+    m = x.max()
+    return m + math.log(np.exp(x - m).sum())
+
+
+@pytest.mark.parametrize("scale", [0.0, 0.37])
+def test_landmark_surrogate_is_exact_at_its_expansion_point(scale):
+    """Gibbs identity: at the landmark query itself, scale * q'.k' + H(p) is the chunk's exact
+    log-mass log sum_j exp(scale * q'.K_j) (a wrong chunk offset, scale, weight or entropy sign
+    breaks it)."""
+    rng = np.random.default_rng(11)
+    B, Hkv, S, d = 2, 3, 16, 8
+    N = 5 * S + 7                                   # a partial last chunk gets no landmark
+    K = rng.standard_normal((B, Hkv, N, d))
+    C = N // S
+    qlm = rng.standard_normal((B, Hkv, C, d)) * 2
+    klm, blm = oracle.landmarks(qlm, K, S=S, scale=scale)
+    assert klm.shape == (B, Hkv, C, d) and blm.shape == (B, Hkv, C)
+    sc = scale if scale > 0 else 1 / math.sqrt(d)
+    for b, g, c in itertools.product(range(B), range(Hkv), range(C)):
+        ref = _lse(K[b, g, c * S:(c + 1) * S] @ qlm[b, g, c] * sc)
+        s_hat = sc * qlm[b, g, c] @ klm[b, g, c] + blm[b, g, c]
+        assert abs(s_hat - ref) < 1e-12 * max(1.0, abs(ref))
+
+
+def test_landmark_surrogate_is_a_tangent_of_the_chunk_log_mass():
+    """First-order Taylor expansion of the chunk log-mass at the landmark query ([Reader] "Paper
+    Primer"): moving the query by t leaves an error that shrinks as t^2, and the tangent plane
+    of the convex log-mass never lies above it."""
+    rng = np.random.default_rng(12)
+    d, S = 8, 32
+    K = rng.standard_normal((1, 1, S, d))
+    q0 = rng.standard_normal((1, 1, 1, d))
+    klm, blm = oracle.landmarks(q0, K, S=S)
+    sc = 1 / math.sqrt(d)
+    delta = rng.standard_normal(d)
+    errs = []
+    for t in (0.04, 0.02, 0.01):
+        q = q0[0, 0, 0] + t * delta
+        true = _lse(K[0, 0] @ q * sc)
+        s_hat = sc * q @ klm[0, 0, 0] + blm[0, 0, 0]
+        assert s_hat <= true + 1e-14
+        errs.append(true - s_hat)
+    assert 3.6 < errs[0] / errs[1] < 4.4 and 3.6 < errs[1] / errs[2] < 4.4
+
+
+def test_landmark_of_a_flat_chunk_is_the_mean_key_with_maximal_entropy():
+    """Uniform attention inside the chunk (a zero landmark query, or identical keys): the summary
+    is the mean-pooled key and the bias is log S, the largest entropy possible."""
+    rng = np.random.default_rng(13)
+    d, S, C = 4, 8, 3
+    K = rng.standard_normal((1, 2, C * S, d))
+    K[0, 1] = np.repeat(rng.standard_normal((C, 1, d)), S, axis=1).reshape(C * S, d)
+    qlm = np.zeros((1, 2, C, d))
+    qlm[0, 1] = rng.standard_normal((C, d)) * 5
+    klm, blm = oracle.landmarks(qlm, K, S=S)
+    np.testing.assert_allclose(blm, math.log(S), rtol=0, atol=1e-13)
+    for g in range(2):
+        np.testing.assert_allclose(klm[0, g], K[0, g].reshape(C, S, d).mean(axis=1),
+                                   rtol=0, atol=1e-13)
+    # any other chunk has a smaller entropy
+    qr = rng.standard_normal((1, 2, C, d)) * 3
+    _, b2 = oracle.landmarks(qr, rng.standard_normal((1, 2, C * S, d)), S=S)
+    assert (b2 > 0).all() and (b2 < math.log(S)).all()
+
+
+def test_landmark_of_a_concentrated_chunk_is_its_dominant_key():
+    """One key dominating the chunk's softmax: the summary is that key and the entropy bias
+    vanishes; a one-token chunk is exactly its key with bias 0."""
+    rng = np.random.default_rng(14)
+    d, S = 6, 16
+    K = rng.standard_normal((1, 1, S, d)) * 0.1
+    u = rng.standard_normal(d)
+    u /= np.linalg.norm(u)
+    K[0, 0, 5] = 40.0 * math.sqrt(d) * u     # logit about 40 above the rest
+    klm, blm = oracle.landmarks(u[None, None, None], K, S=S)
+    np.testing.assert_allclose(klm[0, 0, 0], K[0, 0, 5], rtol=0, atol=1e-12)
+    assert 0.0 <= blm[0, 0, 0] < 1e-14
+    K1 = rng.standard_normal((1, 1, 5, d))
+    k1, b1 = oracle.landmarks(rng.standard_normal((1, 1, 5, d)), K1, S=1)
+    np.testing.assert_array_equal(k1, K1)
+    np.testing.assert_array_equal(b1, np.zeros((1, 1, 5)))
+
+
+@pytest.mark.parametrize("S,W,N", [(4, 5, 37), (8, 8, 64)])
+def test_oracle_landmarks_give_full_attention(S, W, N):
+    """Landmarks built for the query itself (every chunk's landmark query = q) make every
+    surrogate exact, so with K covering all chunks HiLS is full causal attention."""
+    rng = np.random.default_rng(S + N)
+    d = 6
+    q = rng.standard_normal((1, 1, 1, d)) * 2
+    K = rng.standard_normal((1, 1, N, d))
+    V = rng.standard_normal((1, 1, N, d))
+    C = N // S
+    klm, blm = oracle.landmarks(np.broadcast_to(q, (1, 1, C, d)), K, S=S)
+    r = oracle.forward(q, q, K, V, klm, blm, S=S, K_top=C, W=W, q_pos0=N - 1)
+    ref = _sdpa(q, K, V, np.ones((1, N), dtype=bool), 1 / math.sqrt(d))
+    np.testing.assert_allclose(r["out"], ref, rtol=0, atol=1e-12)
+
+
+def test_landmarks_reject_bad_sizes():
+    with pytest.raises(RuntimeError):
+        oracle.landmarks(np.zeros((1, 1, 0, 4)), np.zeros((1, 1, 8, 4)), S=0)
+
+
 # ---------------------------------------------------------------- P4: K=0 is windowed attention
 def test_k0_is_sliding_window_attention():
     rng = np.random.default_rng(3)
