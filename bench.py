@@ -23,6 +23,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import threading
 import subprocess
@@ -120,13 +121,22 @@ KERNEL_SOURCES = {
 SHARED_SOURCES = ["common.cuh", "sm100.cuh"]
 
 
+def code_only(text):
+    """A CUDA source without its comments, whitespace runs collapsed: an edit of the comments
+    leaves it unchanged, any edit of the code changes it."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return re.sub(r"\s+", " ", text).strip()
+
+
 def source_sha(kernel):
-    """Hash of the CUDA sources a kernel is built from (its file and the shared headers)."""
+    """Hash of the code of the CUDA sources a kernel is built from (its file and the shared
+    headers), comments excluded."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "hierarchical_chunk_sparse_scoring_b200", "csrc")
     for f in KERNEL_SOURCES.get(kernel, []) + SHARED_SOURCES:
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            h.update(code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -176,7 +176,9 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem;
-  uint8_t* sQc = sQ + SH::Q_BYTES;   // calibrated queries (surrogate scores of the selection)
+  // calibrated queries (G > 1: the per-head scores of the selection; with G = 1 this tile is
+  // never loaded and serves only as a K/V stage)
+  uint8_t* sQc = sQ + SH::Q_BYTES;
   uint8_t* sK = sQc + SH::Q_BYTES;
   uint8_t* sV = sK + SH::STAGES_MAIN * SH::KV_BYTES;
   uint8_t* sP = sV + SH::STAGES_MAIN * SH::KV_BYTES;
@@ -545,7 +547,7 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
         ++n_sel;
       }
     }
-    // the q_cal tile is read for the last time above: it becomes a K/V stage
+    // the q_cal tile (if loaded) is read for the last time above: it becomes a K/V stage
     __syncwarp();
     if (lane == 0) mbar_arrive(qc_free);
     if (!lm_ok) record_status(status, kStatusTimeout);

@@ -47,14 +47,17 @@ def test_traffic_lookup_requires_current_source(tmp_path, monkeypatch):
     csrc = tmp_path / "hierarchical_chunk_sparse_scoring_b200" / "csrc"
     csrc.mkdir(parents=True)
     for f in ("attn_tc.cu", "common.cuh", "sm100.cuh"):
-        (csrc / f).write_text("// " + f)
+        (csrc / f).write_text("// " + f + "\nint x = 1;\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     sha = bench.source_sha("attn_tc")
     (prof / "traffic.json").write_text(json.dumps(
         {"attn_tc@small_mha_bf16": {"bytes_per_launch": 123.0, "source_sha": sha}}))
     assert bench.traffic_for("attn_tc", "small_mha_bf16") == 123.0
     assert bench.traffic_for("attn_tc", "gqa7b_prefill") is None
-    (csrc / "attn_tc.cu").write_text("// changed")
+    # comments and layout do not count; code does
+    (csrc / "attn_tc.cu").write_text("/* reworded\n comment */ int   x =\n 1; // note\n")
+    assert bench.traffic_for("attn_tc", "small_mha_bf16") == 123.0
+    (csrc / "attn_tc.cu").write_text("// attn_tc.cu\nint x = 2;\n")
     assert bench.traffic_for("attn_tc", "small_mha_bf16") is None
 
 
