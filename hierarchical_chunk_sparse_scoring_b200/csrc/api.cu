@@ -74,8 +74,13 @@ Plan make_plan(const hils_params* p) {
   // decode kernels put (b, g, query) rows on grid.y (<= 65535)
   P.decode = p->N_q <= kDecodeMaxQueries && (p->d == 64 || p->d == 128) &&
              p->B * p->Hkv * p->N_q <= 65535;
-  P.tc_select = !P.decode && score_tc_supported(D, P.bf16);
-  P.tc_attn = !P.decode && attn_tc_supported(D, P.bf16);
+  // the prefill tensor-core kernels address q/q_cal, K/V and landmark rows by 32-bit TMA
+  // coordinates; beyond that the CUDA-core kernels (64-bit offsets) run
+  const bool rows32 = D.B * D.Hq * D.N_q < (int64_t)INT32_MAX &&
+                      D.B * D.Hkv * D.N_kv < (int64_t)INT32_MAX &&
+                      D.B * D.Hkv * D.C < (int64_t)INT32_MAX;
+  P.tc_select = !P.decode && rows32 && score_tc_supported(D, P.bf16);
+  P.tc_attn = !P.decode && rows32 && attn_tc_supported(D, P.bf16);
   P.tc_stream = P.decode && stream_tc_supported(D, P.bf16);
   P.tc_units = P.decode && units_tc_supported(D, P.bf16);
 
