@@ -81,6 +81,11 @@ def test_prefill_workspace_layout(lib):
     assert mha == 256 + rup(8 * nq * k * 4) + rup(8 * nq * k * 4)
     f32 = hb.workspace_size(_params(Hq=8, Hkv=2, N_q=nq, N_kv=nq, K_top=k, dtype=torch.float32))
     assert f32 == 256 + rup(2 * nq * k * 4) + rup(8 * nq * k * 4)
+    # rows beyond 32-bit TMA coordinates (B * Hkv * N_kv >= 2^31): the CUDA-core kernels, which
+    # take the per-head scores from the workspace
+    big = 1 << 28
+    ws = hb.workspace_size(_params(Hq=32, Hkv=8, N_q=big, N_kv=big, K_top=k))
+    assert ws == 256 + rup(8 * big * k * 4) + rup(32 * big * k * 4)
 
 
 BAD = [
