@@ -806,8 +806,8 @@ int list_capacity(const Dims& D, int TQ) {
 template <int DD, int G, int KM, int RS>
 cudaError_t launch_at_t(const Dims& D, const void* q, const void* qc, const void* K,
                         const void* V, const int32_t* idx, const float* s_sig, const void* klm,
-                        const float* blm,
-                        void* out, float* lse, int32_t* status, cudaStream_t st) {
+                        const float* blm, void* out, float* lse, int32_t* status,
+                        cudaStream_t st) {
   using SH = AtShape<DD, G>;
   CUtensorMap tmQ, tmQc, tmK, tmV;
   if (!make_map_at(&tmQ, q, (uint64_t)(D.B * D.Hq * D.N_q), DD, SH::TQ) ||
@@ -832,8 +832,8 @@ cudaError_t launch_at_t(const Dims& D, const void* q, const void* qc, const void
 template <int DD, int G>
 cudaError_t launch_at_k(const Dims& D, const void* q, const void* qc, const void* K,
                         const void* V, const int32_t* idx, const float* s_sig, const void* klm,
-                        const float* blm,
-                        void* out, float* lse, int32_t* status, cudaStream_t st) {
+                        const float* blm, void* out, float* lse, int32_t* status,
+                        cudaStream_t st) {
   if constexpr (DD == 128) {
     // chunks of 128 tokens (two tiles per chunk) are built for d = 128 only
     if (D.S == 2 * kTile) {
@@ -871,9 +871,9 @@ bool attn_tc_supported(const Dims& D, bool bf16) {
 }
 
 cudaError_t launch_attn_tc(const Dims& D, const void* q, const void* qc, const void* K,
-                           const void* V, const int32_t* idx, const float* s_sig, const void* klm,
-                        const float* blm,
-                           void* out, float* lse, int32_t* status, cudaStream_t st) {
+                           const void* V, const int32_t* idx, const float* s_sig,
+                           const void* klm, const float* blm, void* out, float* lse,
+                           int32_t* status, cudaStream_t st) {
   if (D.B * D.Hq * D.N_q == 0) return cudaSuccess;
 #define HILS_AT(DD, GG) \
   return launch_at_k<DD, GG>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status, st)
