@@ -38,7 +38,7 @@ struct Plan {
   bool tc_stream = false;
   bool tc_units = false;
   int cps = 0, n_split = 0, n_pieces = 0;
-  size_t off_idx = 0, off_ssel = 0, off_pv = 0, off_pc = 0, off_po = 0, off_pl = 0;
+  size_t off_idx = 0, off_ssel = 0, off_po = 0, off_pl = 0;
   size_t off_sig = 0;
   int64_t n_stride = 0;
   size_t total = 0;
@@ -109,8 +109,6 @@ Plan make_plan(const hils_params* p) {
     if (P.n_split < 1) P.n_split = 1;
     P.n_pieces = (int)((win_max + D.S - 1) / D.S);
     const int NU = D.K + P.n_pieces;
-    P.off_pv = off; off = align_up(off + sel_rows * P.n_split * (size_t)D.K * sizeof(float));
-    P.off_pc = off; off = align_up(off + sel_rows * P.n_split * (size_t)D.K * sizeof(int32_t));
     P.off_po = off; off = align_up(off + head_rows * NU * (size_t)D.d * sizeof(float));
     P.off_pl = off; off = align_up(off + head_rows * NU * sizeof(float));
     P.n_stride = (n_max + 3) / 4 * 4;
@@ -211,8 +209,6 @@ hils_status forward_impl(const hils_params* p, const void* q, const void* q_cal,
   cudaError_t e;
   pm.mark();
   if (P.decode) {
-    float* pv = reinterpret_cast<float*>(ws + P.off_pv);
-    int32_t* pc = reinterpret_cast<int32_t*>(ws + P.off_pc);
     float* po = reinterpret_cast<float*>(ws + P.off_po);
     float* pl = reinterpret_cast<float*>(ws + P.off_pl);
     float* sig = reinterpret_cast<float*>(ws + P.off_sig);
@@ -222,8 +218,6 @@ hils_status forward_impl(const hils_params* p, const void* q, const void* q_cal,
                                            q_cal, k_lm, b_lm, sig, reinterpret_cast<int32_t*>(ws),
                                            st);
     pm.mark();
-    (void)pv;
-    (void)pc;
     if (e == cudaSuccess)
       e = launch_select_topk_row(P.D, P.bf16, P.n_stride, sig, q_cal, k_lm, b_lm, idx, s_sel, st);
     pm.mark();
