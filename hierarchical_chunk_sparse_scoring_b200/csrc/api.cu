@@ -227,7 +227,8 @@ hils_status forward_impl(const hils_params* p, const void* q, const void* q_cal,
                      : launch_attn_units(P.D, P.bf16, P.n_pieces, q, K, V, idx, po, pl,
                                          reinterpret_cast<int32_t*>(ws), st);
     pm.mark();
-    if (e == cudaSuccess) e = launch_fuse_units(P.D, P.bf16, P.n_pieces, s_sel, po, pl, out, lse_out, st);
+    if (e == cudaSuccess)
+      e = launch_fuse_units(P.D, P.bf16, P.n_pieces, s_sel, po, pl, out, lse_out, st);
     pm.mark();
   } else {
     if (P.tc_select) {

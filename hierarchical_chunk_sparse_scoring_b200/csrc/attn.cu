@@ -507,10 +507,14 @@ cudaError_t launch_attn_units(const Dims& D, bool bf16, int n_pieces, const void
                               float* part_lse, int32_t* status, cudaStream_t st) {
   if (D.B * D.Hkv * D.N_q == 0) return cudaSuccess;
   if (D.d == 128)
-    return bf16 ? launch_units_d<__nv_bfloat16, 128>(D, n_pieces, q, K, V, idx, part_o, part_lse, status, st)
-                : launch_units_d<float, 128>(D, n_pieces, q, K, V, idx, part_o, part_lse, status, st);
-  return bf16 ? launch_units_d<__nv_bfloat16, 64>(D, n_pieces, q, K, V, idx, part_o, part_lse, status, st)
-              : launch_units_d<float, 64>(D, n_pieces, q, K, V, idx, part_o, part_lse, status, st);
+    return bf16 ? launch_units_d<__nv_bfloat16, 128>(D, n_pieces, q, K, V, idx, part_o,
+                                                     part_lse, status, st)
+                : launch_units_d<float, 128>(D, n_pieces, q, K, V, idx, part_o, part_lse,
+                                             status, st);
+  return bf16 ? launch_units_d<__nv_bfloat16, 64>(D, n_pieces, q, K, V, idx, part_o, part_lse,
+                                                 status, st)
+              : launch_units_d<float, 64>(D, n_pieces, q, K, V, idx, part_o, part_lse, status,
+                                          st);
 }
 
 cudaError_t launch_fuse_units(const Dims& D, bool bf16, int n_pieces, const float* s_sel,

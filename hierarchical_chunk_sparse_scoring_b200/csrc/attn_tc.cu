@@ -164,7 +164,8 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 
 template <int DD, int G, int KM, int RS>
 __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQc,
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                   const __grid_constant__ CUtensorMap tmQc,
                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    Dims D, const int32_t* __restrict__ idx, const float* __restrict__ s_sig,
                    const __nv_bfloat16* __restrict__ klm, const float* __restrict__ blm,
@@ -661,7 +662,8 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
           p[j + 1] = fast_exp2(p[j + 1]);
           add2(ps[j & 7], ps[(j & 7) + 1], p[j], p[j + 1]);
         }
-        const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7])) +
+        const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) +
+                          ((ps[4] + ps[5]) + (ps[6] + ps[7])) +
                           (first2 ? sum2_raw : 0.f);
         const float w = fast_exp2((u - m_run) * kLog2e);
         const float f = w / sum;
@@ -841,7 +843,8 @@ cudaError_t launch_at_k(const Dims& D, const void* q, const void* qc, const void
         return launch_at_t<DD, G, 8, 1>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status,
                                         st);
       if (D.K <= 16)
-        return launch_at_t<DD, G, 16, 1>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status, st);
+        return launch_at_t<DD, G, 16, 1>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status,
+                                         st);
       return launch_at_t<DD, G, 32, 1>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status, st);
     }
   }

@@ -285,7 +285,8 @@ __global__ void __launch_bounds__(64 + 128 * NCG, CPS)
         if constexpr (HP == 2) {
           // the other head of each pair sits in the neighbouring lane
 #pragma unroll
-          for (int j = 0; j < 16; ++j) sig[j] = fmaxf(sig[j], __shfl_xor_sync(0xffffffffu, sig[j], 1));
+          for (int j = 0; j < 16; ++j)
+            sig[j] = fmaxf(sig[j], __shfl_xor_sync(0xffffffffu, sig[j], 1));
         }
         // a candidate must reach every group's current K-th best (each list already holds K
         // candidates at least that good); exact ties at the threshold are passed on and

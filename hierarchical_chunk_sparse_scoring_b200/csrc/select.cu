@@ -287,8 +287,10 @@ __global__ void __launch_bounds__(128) select_scores_bf16_kernel(
   for (int x = 0; x < QV; ++x) {
     const int e = x * 256 + lane * 8;
     if (e < G * D_) {
-      *reinterpret_cast<float4*>(&qs[warp][e]) = make_float4(qv[x][0], qv[x][1], qv[x][2], qv[x][3]);
-      *reinterpret_cast<float4*>(&qs[warp][e + 4]) = make_float4(qv[x][4], qv[x][5], qv[x][6], qv[x][7]);
+      *reinterpret_cast<float4*>(&qs[warp][e]) =
+          make_float4(qv[x][0], qv[x][1], qv[x][2], qv[x][3]);
+      *reinterpret_cast<float4*>(&qs[warp][e + 4]) =
+          make_float4(qv[x][4], qv[x][5], qv[x][6], qv[x][7]);
     }
   }
   __syncwarp();

@@ -12,8 +12,9 @@
 //
 // Persistent CTAs, three per SM: three producers with two stages each kept more copies in flight
 // than one CTA with a six-stage ring (measured 5.1 against 4.2 TB/s).  The tiles (row, 128-chunk
-// block) are split into contiguous ranges, one per CTA, so a CTA's stream crosses few rows.  Warp 0: TMA producer (a ring of
-// stages, each one landmark tile plus the row's query tile); warp 1: TMEM owner and MMA issuer;
+// block) are split into contiguous ranges, one per CTA, so a CTA's stream crosses few rows.
+// Warp 0: TMA producer (a ring of stages, each one landmark tile plus the row's query tile);
+// warp 1: TMEM owner and MMA issuer;
 // warps 2-5: epilogue (tcgen05.ld of 16 columns, group max, scale, bias, mask c < n).
 // Every mbarrier wait gives up after a bounded number of polls and records HILS_ERR_TIMEOUT.
 #include <cudaTypedefs.h>
