@@ -5,17 +5,21 @@
     torchrun --nproc-per-node N bench.py --gpus N ...        (one process per GPU)
 
 A step is one hils_forward call (score -> top-K -> chunk/window attention -> fusion) over one
-batch of the prefill workload (default: small_mha_bf16, B=4 x 16 heads x 8192 tokens, d=64, S=64,
-K=8, W=512), inputs resident in HBM.  Steps are timed with CUDA events recorded by the library
-between its kernels, so each kernel's duration comes from the same timed steps; L2 is flushed
-(256 MiB write) between steps, outside the timed intervals.  With N GPUs every rank runs its own
-independent batch (weak scaling, no data-path collective); the step time is the max over ranks.
+batch of the prefill workload, inputs resident in HBM.  The default workload is the largest
+single-GPU configuration: the extreme-length prefill at N = 4M tokens (B=1, 8 query heads / 1 KV
+head, d=128, S=128, K=16, W=2048; 140.6 TFLOP of landmark scoring).  Steps are timed with CUDA
+events recorded by the library between its kernels, so each kernel's duration comes from the
+same timed steps; L2 is flushed (256 MiB write) between steps, outside the timed intervals.
+With N GPUs every rank runs its own independent batch (weak scaling, no data-path collective);
+the step time is the max over ranks.
 
 Also reported (single GPU): `e2e` (the same call from pinned host buffers, copies included),
-`cpu_baseline` (the fp64 CPU oracle on a bounded sample), `decode` (long_decode: 32 single-token
-queries over a 512K-token cache, timed as a CUDA graph replay, microseconds per step) and
-`prefill_gqa7b` (the 7B-like GQA prefill at N=131072), each with its dominant kernel's roofline.
-`--impl reference` times the fp64 CPU oracle as the reference arm.
+`cpu_baseline` (the fp64 CPU oracle on a bounded sample of the same workload) with `parity`
+(the GPU's outputs on the oracle-timed rows), the 4M decode step, and the other workloads of the
+sweep: `prefill_small_mha` (B=4 x 16 heads x 8192 tokens), `prefill_gqa7b` (the 7B-like GQA
+prefill at N=131072), `decode` (32 single-token queries over a 512K-token cache, timed as a CUDA
+graph replay) and `extreme_256k` / `extreme_1m` (prefill and decode), each with per-kernel
+rooflines.  `--impl reference` times the fp64 CPU oracle as the reference arm.
 """
 import argparse
 import datetime
@@ -274,52 +278,99 @@ def make_flush(device):
 
 
 # --------------------------------------------------------------------------- CPU oracle
-def oracle_sample_rate(wl, seconds, rng_seed=0, max_rows=None):
+def oracle_sample(wl, seconds, rng_seed=0, max_rows=None, cache=None):
     """Times the fp64 oracle on randomly chosen (b, g, query) rows of `wl` (all G heads of each
-    row), sized to run about `seconds`.  Returns (tokens/s, rows, threads, wall seconds)."""
+    row), sized to run about `seconds`.  Returns a dict: tokens/s, rows, threads, wall seconds,
+    and the rows with the oracle's results (for the parity summary)."""
     import oracle
     Hq, d = wl.q.shape[1], wl.q.shape[3]
-    Hkv, Nkv = wl.K.shape[1], wl.K.shape[2]
+    Hkv = wl.K.shape[1]
     G = Hq // Hkv
     B, Nq = wl.q.shape[0], wl.q.shape[2]
     rng = np.random.default_rng(rng_seed)
-    cache = {}
+    cache = {} if cache is None else cache
 
     def f64(t):
-        return t.detach().to("cpu", torch.float64).numpy()
+        # converted on the tensor's own device, then copied to the host once
+        return t.detach().to(torch.float64).cpu().numpy()
 
     def build(n_rows):
-        qs = []
+        picks, qs = [], []
         for _ in range(n_rows):
             b, g, i = int(rng.integers(B)), int(rng.integers(Hkv)), int(rng.integers(Nq))
             if (b, g) not in cache:
                 cache[(b, g)] = (f64(wl.k_lm[b, g]), f64(wl.b_lm[b, g]), f64(wl.K[b, g]),
                                  f64(wl.V[b, g]))
             klm, blm, kr, vr = cache[(b, g)]
+            picks.append((b, g, i))
             qs.append(oracle.Query(wl.q_pos0 + i, f64(wl.q[b, g * G:(g + 1) * G, i]),
                                    f64(wl.q_cal[b, g * G:(g + 1) * G, i]), klm, blm, kr, vr))
-        return qs
+        return picks, qs
 
     threads = oracle.default_threads()
     kw = dict(d=d, G=G, S=wl.S, K_top=wl.K_top, W=wl.W, threads=threads)
     rows = max(threads, 8)
     while True:
-        qs = build(rows)
+        picks, qs = build(rows)
         t0 = time.perf_counter()
-        oracle.run_queries(qs, **kw)
+        res = oracle.run_queries(qs, **kw)
         dt = time.perf_counter() - t0
         if dt >= seconds * 0.5 or (max_rows and rows >= max_rows):
             break
         rows = int(min(rows * max(2.0, seconds / max(dt, 1e-3)), max_rows or 1 << 30))
     tokens = rows * G / Hq
-    return tokens / dt, rows, threads, dt
+    return {"rate": tokens / dt, "rows": rows, "threads": threads, "seconds": dt,
+            "picks": picks, "results": res}
+
+
+def oracle_sample_rate(wl, seconds, rng_seed=0, max_rows=None, cache=None):
+    r = oracle_sample(wl, seconds, rng_seed, max_rows, cache)
+    return r["rate"], r["rows"], r["threads"], r["seconds"]
+
+
+def parity_summary(run, sample, gap_tol=1e-3):
+    """The GPU run's outputs on the oracle-timed rows: how many rows select exactly the oracle's
+    chunks (rows whose rank-K gap exceeds gap_tol), how many are near ties, and the largest
+    output / log-sum-exp differences on the rows whose selection matches."""
+    wl = run.wl
+    G = wl.q.shape[1] // wl.K.shape[1]
+    K = wl.K_top
+    clear = match = ties = 0
+    out_err = lse_err = 0.0
+    for (b, g, i), r in zip(sample["picks"], sample["results"]):
+        gsel = run.idx[b, g, i].cpu().numpy()
+        osel = r["idx"]
+        same_set = set(int(c) for c in gsel if c >= 0) == set(int(c) for c in osel if c >= 0)
+        if r["gap"] > gap_tol:
+            clear += 1
+            match += int(same_set)
+        else:
+            ties += 1
+        if same_set:
+            o = run.out[b, g * G:(g + 1) * G, i].double().cpu().numpy()
+            l = run.lse[b, g * G:(g + 1) * G, i].double().cpu().numpy()
+            out_err = max(out_err, float(np.abs(o - r["out"]).max()))
+            lse_err = max(lse_err, float(np.abs(l - r["lse"]).max()))
+    return {"rows": len(sample["picks"]), "clear_gap_rows": clear,
+            "idx_match_rate": (match / clear) if clear else None, "near_tie_rows": ties,
+            "out_abs_max": out_err, "lse_abs_max": lse_err, "K": K,
+            "rule": "sets equal where the oracle's rank-K gap > 1e-3; errors on matching rows"}
 
 
 # --------------------------------------------------------------------------- arms
+HEADLINE = ("extreme", 1 << 22)   # the extreme-length prefill at N = 4M tokens
+
+
+def workload_N(args):
+    if args.N is None and args.workload == HEADLINE[0]:
+        return HEADLINE[1]
+    return args.N
+
+
 def primary_workload(args, device, rank):
     from hierarchical_chunk_sparse_scoring_b200 import workloads as W
     seed = W.SPECS[args.workload]["seed"] + 1000 * rank
-    return W.make(args.workload, device, seed=seed, N=args.N, B=args.B)
+    return W.make(args.workload, device, seed=seed, N=workload_N(args), B=args.B)
 
 
 def config_of(wl, n_gpus):
@@ -476,34 +527,37 @@ def union_stat(idx, tq, C):
     return float(sizes.mean().item()) / K
 
 
+def time_mode(wl, steps, peaks, label):
+    """Timed hils_forward steps of one workload (prefill or decode) with per-kernel rooflines."""
+    run = Runner(wl)
+    flush = make_flush(wl.q.device)
+    run()
+    torch.cuda.synchronize()
+    step_ms, phase_ms = timed_steps(run, steps, flush)
+    wm = work_model(wl.dims, wl.S, wl.K_top, wl.W, wl.q_pos0, wl.q.element_size())
+    t = statistics.mean(step_ms)
+    res = {"ms_per_step": t, "phases_ms": phase_ms,
+           "rooflines": [roofline(k, v, wm, peaks, label) for k, v in phase_ms.items()]}
+    if wl.q.shape[2] > 16:
+        res["tokens_per_s"] = wm["tokens"] / (t * 1e-3)
+        res["score_tflop"] = wm["score_flops"] / 1e12
+        res["attn_tflop"] = wm["attn_flops"] / 1e12
+    else:
+        res["us_per_step"] = t * 1e3
+        res["step_bytes"] = wm["select_bytes"] + wm["attn_bytes"]
+        res["step_hbm_frac"] = res["step_bytes"] / (t * 1e-3) / 1e9 / peaks["hbm_gbs"]
+    del run
+    return res
+
+
 def extra_extreme(steps, peaks, N=262144):
-    """The extreme-length sweep's first point: prefill of the whole sequence and one decode
+    """One point of the extreme-length sweep: prefill of the whole sequence and one decode
     step of its last query, on the same inputs."""
     from hierarchical_chunk_sparse_scoring_b200 import workloads as W
     wl = W.make("extreme", "cuda", N=N)
-    res = {"workload": "extreme", "N": N}
-    for mode in ("prefill", "decode"):
-        if mode == "decode":
-            wl = W.Workload("extreme_decode", wl.q[:, :, -1:].contiguous(),
-                            wl.q_cal[:, :, -1:].contiguous(), wl.K, wl.V, wl.k_lm, wl.b_lm,
-                            wl.S, wl.K_top, wl.W, q_pos0=N - 1)
-        run = Runner(wl)
-        flush = make_flush(wl.q.device)
-        run()
-        torch.cuda.synchronize()
-        step_ms, phase_ms = timed_steps(run, steps, flush)
-        wm = work_model(wl.dims, wl.S, wl.K_top, wl.W, wl.q_pos0, wl.q.element_size())
-        t = statistics.mean(step_ms)
-        res[mode] = {"ms_per_step": t, "phases_ms": phase_ms,
-                     "rooflines": [roofline(k, v, wm, peaks, "extreme_%s" % mode)
-                                   for k, v in phase_ms.items()]}
-        if mode == "prefill":
-            res[mode]["tokens_per_s"] = wm["tokens"] / (t * 1e-3)
-            res[mode]["score_tflop"] = wm["score_flops"] / 1e12
-            res[mode]["attn_tflop"] = wm["attn_flops"] / 1e12
-        else:
-            res[mode]["us_per_step"] = t * 1e3
-        del run
+    res = {"workload": "extreme", "N": N,
+           "prefill": time_mode(wl, steps, peaks, "extreme_prefill"),
+           "decode": time_mode(W.decode_view(wl), max(steps, 5), peaks, "extreme_decode")}
     del wl
     torch.cuda.empty_cache()
     return res
@@ -542,6 +596,7 @@ def run_hils(args):
     es = wl.q.element_size()
     wm = work_model(wl.dims, wl.S, wl.K_top, wl.W, wl.q_pos0, es)
     dom = max(phase_ms, key=phase_ms.get)
+    label = wl.name if workload_N(args) is None else "%s_N%d" % (wl.name, wl.dims["N_kv"])
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -549,26 +604,39 @@ def run_hils(args):
         "dtype": "bf16" if wl.q.dtype == torch.bfloat16 else "f32",
         "data": "synthetic (seeded generator, hierarchical_chunk_sparse_scoring_b200/workloads.py)",
         "config": config_of(wl, world),
-        "roofline": roofline(dom, phase_ms[dom], wm, peaks, wl.name),
+        "roofline": roofline(dom, phase_ms[dom], wm, peaks, label),
+        "rooflines": [roofline(k, v, wm, peaks, label) for k, v in phase_ms.items()],
         "peaks_source": peaks_src,
         "phases_ms": phase_ms,
+        "score_tflop": wm["score_flops"] / 1e12, "attn_tflop": wm["attn_flops"] / 1e12,
         "gpu_launches": len(run.phases) * args.steps,
         "union_per_K_128_rows": union_stat(run.idx, 128 // (wl.q.shape[1] // wl.K.shape[1]),
                                            wl.K.shape[2] // wl.S),
         "clocks": clk.summary(),
     }
     if world == 1 and not args.no_extras:
-        line["e2e"] = measure_e2e(run, max(3, args.steps // 2), 1)
-        del run
+        line["e2e"] = measure_e2e(run, max(3, args.steps // 4), 1)
         torch.cuda.empty_cache()
+        sample = oracle_sample(wl, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": sample["rate"], "unit": "tokens/s",
+                                "cores": sample["threads"], "kind": "oracle",
+                                "sample": "%d random (b, kv-group, query) rows of %s, all heads "
+                                          "of each group, %.1f s wall" % (
+                                              sample["rows"], label, sample["seconds"])}
+        line["parity"] = parity_summary(run, sample)
+        del sample, run
+        torch.cuda.empty_cache()
+        if wl.name == "extreme":
+            from hierarchical_chunk_sparse_scoring_b200 import workloads as W
+            line["extreme_%dk_decode" % (wl.dims["N_kv"] >> 10)] = time_mode(
+                W.decode_view(wl), max(5, args.steps), peaks, label + "_decode")
+        del wl
+        torch.cuda.empty_cache()
+        line["prefill_small_mha"] = extra_prefill("small_mha_bf16", 5, peaks)
         line["prefill_gqa7b"] = extra_prefill("gqa7b_prefill", 3, peaks)
         line["decode"] = extra_decode(max(5, args.steps), peaks)
-        line["extreme_256k"] = extra_extreme(2, peaks)
-        rate, rows, threads, dt = oracle_sample_rate(wl, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": threads,
-                                "kind": "oracle",
-                                "sample": "%d random (b, kv-group, query) rows of %s, all heads "
-                                          "of each group, %.1f s wall" % (rows, wl.name, dt)}
+        line["extreme_256k"] = extra_extreme(3, peaks, N=1 << 18)
+        line["extreme_1m"] = extra_extreme(2, peaks, N=1 << 20)
     if dist:
         dist.destroy_process_group()
     if rank == 0:
@@ -580,11 +648,16 @@ def run_reference(args):
     if int(os.environ.get("RANK", "0")) != 0:
         return
     from hierarchical_chunk_sparse_scoring_b200 import workloads as W
-    wl = W.make(args.workload, "cpu", N=args.N, B=args.B)
+    # the same seeded inputs as the GPU arm (drawn on the GPU when there is one: the generator
+    # streams differ between devices); the oracle itself runs on the host cores
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    wl = W.make(args.workload, dev, N=workload_N(args), B=args.B)
     per_step = max(1.0, args.ref_step_seconds)
     rates, rows_total, threads = [], 0, 1
+    cache = {}   # the (b, g) landmark and K/V arrays in fp64, converted once
     for k in range(args.warmup + args.steps):
-        rate, rows, threads, dt = oracle_sample_rate(wl, per_step, rng_seed=k)
+        rate, rows, threads, dt = oracle_sample_rate(wl, per_step if k >= args.warmup else 1.0,
+                                                     rng_seed=k, cache=cache)
         if k >= args.warmup:
             rates.append(rate)
             rows_total += rows
@@ -611,12 +684,12 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["hils", "reference"], default="hils")
-    ap.add_argument("--workload", default="small_mha_bf16")
+    ap.add_argument("--workload", default=HEADLINE[0])
     ap.add_argument("--N", type=int, default=None, help="override the workload's sequence length")
     ap.add_argument("--B", type=int, default=None, help="override the workload's batch")
     ap.add_argument("--no-extras", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--ref-step-seconds", type=float, default=6.0)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=4.0)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "hils":
         args.warmup = 3

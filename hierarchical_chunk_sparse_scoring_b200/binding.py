@@ -45,6 +45,8 @@ SIGNATURES = {
     "hils_select": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V, ctypes.c_size_t, _V]),
     "hils_select_noalloc": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V]),
     "hils_select_noalloc_max_bytes": (ctypes.c_size_t, []),
+    "hils_select_noalloc_status": (ctypes.c_int, [_V, ctypes.POINTER(ctypes.c_int32)]),
+    "hils_wait_check": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_int, _V, ctypes.c_size_t, _V]),
     "hils_chunk_attn": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V, _V]),
     "hils_fuse": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V]),
     "hils_workspace_init": (ctypes.c_int, [_V, ctypes.c_size_t, _V]),
@@ -228,6 +230,35 @@ def device_status(ws, stream=None):
     _check(lib().hils_device_status(_ptr(ws), _stream(stream), ctypes.byref(code)),
            "hils_device_status")
     return int(code.value)
+
+
+def select_noalloc(q_cal, k_lm, b_lm, *, N_kv, Hkv, S, K_top, W, q_pos0=0, scale=0.0,
+                   stream=None):
+    """hils_select_noalloc: steps 1-2 with the library's fixed scratch array (no workspace).
+    Returns (idx, s_sel)."""
+    B, Hq, N_q, d = q_cal.shape
+    p = make_params(B, Hq, Hkv, N_q, N_kv, d, S=S, K_top=K_top, W=W, q_pos0=q_pos0,
+                    dtype=q_cal.dtype, scale=scale)
+    idx = torch.empty((B, Hkv, N_q, K_top), dtype=torch.int32, device=q_cal.device)
+    s_sel = torch.empty((B, Hq, N_q, K_top), dtype=torch.float32, device=q_cal.device)
+    _check(lib().hils_select_noalloc(ctypes.byref(p), _ptr(q_cal), _ptr(k_lm), _ptr(b_lm),
+                                     _ptr(idx), _ptr(s_sel), _stream(stream)),
+           "hils_select_noalloc")
+    return idx, s_sel
+
+
+def select_noalloc_status(stream=None):
+    """Reads and clears this device's hils_select_noalloc status word."""
+    code = ctypes.c_int32(0)
+    _check(lib().hils_select_noalloc_status(_stream(stream), ctypes.byref(code)),
+           "hils_select_noalloc_status")
+    return int(code.value)
+
+
+def wait_check(polls, complete, ws, stream=None):
+    """hils_wait_check: one bounded mbarrier wait on the device (see include/hils.h)."""
+    _check(lib().hils_wait_check(int(polls), int(bool(complete)), _ptr(ws), ws.numel(),
+                                 _stream(stream)), "hils_wait_check")
 
 
 def version():

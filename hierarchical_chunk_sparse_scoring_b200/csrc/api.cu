@@ -377,6 +377,19 @@ extern "C" hils_status hils_device_status(void* workspace, hils_stream_t stream,
   return HILS_OK;
 }
 
+extern "C" hils_status hils_wait_check(uint32_t polls, int complete, void* workspace,
+                                       size_t workspace_bytes, hils_stream_t stream) {
+  if (!workspace || !aligned16(workspace) || workspace_bytes < kStatusBytes)
+    return HILS_ERR_WORKSPACE;
+  if (polls == 0) return HILS_ERR_INVALID_ARG;
+  hils_status s = check_device();
+  if (s != HILS_OK) return s;
+  return launch_wait_check(polls, complete, static_cast<int32_t*>(workspace),
+                           reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? HILS_OK
+             : HILS_ERR_CUDA;
+}
+
 extern "C" const char* hils_status_string(hils_status s) {
   switch (s) {
     case HILS_OK: return "ok";
@@ -409,8 +422,8 @@ void* g_scratch_addr[kMaxDevices] = {};
 
 // Device address of this device's scratch array.  In host code `g_static_scratch` names a host
 // stand-in, not device memory, so the address is looked up once per device (with that device
-// current) and cached.
-hils_status static_scratch(void** out) {
+// current) and cached; that first lookup also zeroes the array's status word on `st`.
+hils_status static_scratch(cudaStream_t st, void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return HILS_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return HILS_ERR_UNSUPPORTED;
@@ -418,6 +431,7 @@ hils_status static_scratch(void** out) {
   if (!g_scratch_addr[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return HILS_ERR_CUDA;
+    if (cudaMemsetAsync(p, 0, kStatusBytes, st) != cudaSuccess) return HILS_ERR_CUDA;
     g_scratch_addr[dev] = p;
   }
   *out = g_scratch_addr[dev];
@@ -448,12 +462,11 @@ extern "C" hils_status hils_select_noalloc(const hils_params* p, const void* q_c
   if (need > kStaticScratchBytes) return HILS_ERR_WORKSPACE;
   if (!any) return HILS_OK;
   if ((s = check_device()) != HILS_OK) return s;
-  void* scratch = nullptr;
-  if ((s = static_scratch(&scratch)) != HILS_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  void* scratch = nullptr;
+  if ((s = static_scratch(st, &scratch)) != HILS_OK) return s;
   char* ws = static_cast<char*>(scratch);
-  // the status word is shared by every call: start it at zero
-  if (cudaMemsetAsync(ws, 0, kStatusBytes, st) != cudaSuccess) return HILS_ERR_CUDA;
+  // the status word keeps the first failure since it was last read (hils_select_noalloc_status)
   cudaError_t e;
   if (P.decode) {
     float* pv = reinterpret_cast<float*>(ws + kStatusBytes);
@@ -471,4 +484,19 @@ extern "C" hils_status hils_select_noalloc(const hils_params* p, const void* q_c
     e = launch_select_rows(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
   }
   return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA;
+}
+
+extern "C" hils_status hils_select_noalloc_status(hils_stream_t stream, int32_t* status) {
+  if (!status) return HILS_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  void* scratch = nullptr;
+  hils_status s = static_scratch(st, &scratch);
+  if (s != HILS_OK) return s;
+  int32_t word = 0;
+  if (cudaMemcpyAsync(&word, scratch, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemsetAsync(scratch, 0, sizeof(word), st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return HILS_ERR_CUDA;
+  *status = word;
+  return HILS_OK;
 }

@@ -208,11 +208,14 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qc_free + 1);
   int* n_tiles_sh = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + 1024);
   int* tiles = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + 2048);  // [list_cap]
-  uint32_t* bitmap = reinterpret_cast<uint32_t*>(tiles + list_cap);             // [words]
-  int* wpre = reinterpret_cast<int*>(bitmap + bitmap_words);   // list position of each word
+  // the tile bitmap of the union and the list position of each of its words live in the
+  // prologue scratch (up to 2 x 16 KB): they are read for the last time by the rows' ranking,
+  // before the landmark rows are staged there
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(sP);                          // [words]
+  int* wpre = reinterpret_cast<int*>(sP + SH::P_BYTES);        // list position of each word
   // per row, its selected chunks in tile-list order: (tile index, surrogate score) [128][KM]
   constexpr bool kSelSmem = KM <= 16;
-  int* sel_t = wpre + bitmap_words;
+  int* sel_t = tiles + list_cap;
   float* sel_u = reinterpret_cast<float*>(sel_t + (kSelSmem ? kAtRows * KM : 0));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -467,6 +470,8 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
                          : make_uint4(0u, 0u, 0u, 0u);
         }
         rank_chunks();   // while those rows load
+        // every row has read the bitmap before the landmark rows overwrite it
+        asm volatile("bar.sync 1, 128;" ::: "memory");
 #pragma unroll
         for (int e = 0; e < SH::KLM_ROWS * UPR / 128; ++e) {
           const int f = tid + e * 128, t = f / UPR, j = f - t * UPR;
@@ -819,7 +824,8 @@ cudaError_t launch_at_t(const Dims& D, const void* q, const void* qc, const void
     return cudaErrorInvalidValue;
   const int cap = list_capacity(D, SH::TQ);
   const int words = (int)((D.N_kv / kTile) / 32) + 2;
-  const int smem = SH::FIXED + 1024 + cap * 4 + 2 * words * 4 + (KM <= 16 ? kAtRows * KM * 8 : 0);
+  if (words * 4 > SH::P_BYTES) return cudaErrorInvalidConfiguration;
+  const int smem = SH::FIXED + 1024 + cap * 4 + (KM <= 16 ? kAtRows * KM * 8 : 0);
   if (smem > kAtSmemLimit) return cudaErrorInvalidConfiguration;
   auto kern = attn_tc_kernel<DD, G, KM, RS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -865,12 +871,15 @@ bool attn_tc_supported(const Dims& D, bool bf16) {
   if (D.B * D.Hkv > 65535) return false;
   const int TQ = kAtRows / D.G;
   const int64_t cap = (int64_t)TQ * D.K * (D.S / kTile) + (D.W + D.S + TQ) / kTile + 4;
+  // the tile bitmap (one bit per 64-token tile of the sequence) fits one prologue scratch area
+  // of 16 KB: sequences of up to about 8.3 M tokens
   const int64_t words = (D.N_kv / kTile) / 32 + 2;
+  if (words * 4 > AtShape<64, 1>::P_BYTES) return false;
   const int fixed = D.d == 128 ? AtShape<128, 1>::FIXED : AtShape<64, 1>::FIXED;
   if (D.C >= (int64_t)INT32_MAX) return false;
   const int km = D.K <= 8 ? 8 : (D.K <= 16 ? 16 : 32);
   const int64_t sel_bytes = km <= 16 ? (int64_t)kAtRows * km * 8 : 0;
-  return fixed + 1024 + (cap + 2 * words) * 4 + sel_bytes <= kAtSmemLimit;
+  return fixed + 1024 + cap * 4 + sel_bytes <= kAtSmemLimit;
 }
 
 cudaError_t launch_attn_tc(const Dims& D, const void* q, const void* qc, const void* K,

@@ -145,13 +145,17 @@ hils_status hils_fuse(const hils_params* p, const float* s_sel, const float* uni
  *
  * Scratch: a fixed array of hils_select_noalloc_max_bytes() bytes (8 MiB) inside the library,
  * one per device, held by every device that loads the library until the process exits.  The
- * first call on a device looks up that device's copy (cudaGetSymbolAddress, with the device
- * current); make that first call before any stream capture.  Calls whose scratch would exceed
- * the maximum (decode shapes with B*Hkv*N_q * ceil(n/512) * K * 8 bytes beyond ~8 MiB) return
- * HILS_ERR_WORKSPACE before launching anything.  Every call on a device shares the same
- * scratch, so calls that overlap on the GPU (different streams, or concurrent host threads)
- * race and give undefined results: order them on one stream.  The library's status word is
- * cleared at the start of every call.  Allocates nothing.
+ * first call on a device (this one or hils_select_noalloc_status) looks up that device's copy
+ * (cudaGetSymbolAddress, with the device current), keeps the address for the life of the
+ * process and zeroes the array's status word on `stream`; make that first call before any
+ * stream capture.  The kept address does not survive cudaDeviceReset: resetting a device after
+ * the first call is not supported.  Calls whose scratch would exceed the maximum (decode shapes
+ * with B*Hkv*N_q * ceil(n/512) * K * 8 bytes beyond ~8 MiB) return HILS_ERR_WORKSPACE before
+ * launching anything.  Every call on a device shares the same scratch, so calls that overlap on
+ * the GPU (different streams, or concurrent host threads) race and give undefined results:
+ * order them on one stream.  Kernels record a failed bounded wait in the array's status word,
+ * which keeps the first failure until hils_select_noalloc_status reads and clears it.
+ * Allocates nothing.
  */
 hils_status hils_select_noalloc(const hils_params* p, const void* q_cal, const void* k_lm,
                                 const float* b_lm, int32_t* idx, float* s_sel,
@@ -160,12 +164,29 @@ hils_status hils_select_noalloc(const hils_params* p, const void* q_cal, const v
 /* Size in bytes of the fixed scratch array hils_select_noalloc uses. */
 size_t hils_select_noalloc_max_bytes(void);
 
+/* Copies this device's hils_select_noalloc status word to *status (HILS_OK, or the first
+ * failure a kernel recorded since the word was last read) and clears it.  Synchronous on
+ * `stream`; order it after the calls it reports on.  The paper has no counterpart. */
+hils_status hils_select_noalloc_status(hils_stream_t stream, int32_t* status);
+
 /* Zeroes the workspace's status word; call once on a newly allocated workspace. */
 hils_status hils_workspace_init(void* workspace, size_t workspace_bytes, hils_stream_t stream);
 
 /* Copies the workspace's status word to *status (HILS_OK or the first failure a kernel
  * recorded) and clears it.  Synchronous on `stream`. */
 hils_status hils_device_status(void* workspace, hils_stream_t stream, int32_t* status);
+
+/*
+ * Check of the bounded on-chip waits (the paper has no counterpart).  Every tensor-core kernel
+ * waits on mbarriers for its TMA copies and MMAs; each wait gives up after a bounded number of
+ * polls, records HILS_ERR_TIMEOUT in the workspace's status word and lets the kernel return, so
+ * a wait that can never finish cannot hang the GPU.  This launches one CTA that performs such a
+ * wait with a limit of `polls` polls: with `complete` nonzero the barrier phase is completed
+ * first (the wait succeeds, nothing is recorded); with `complete` zero nothing ever arrives and
+ * the wait must give up.  Read the outcome with hils_device_status.  Asynchronous on `stream`.
+ */
+hils_status hils_wait_check(uint32_t polls, int complete, void* workspace,
+                            size_t workspace_bytes, hils_stream_t stream);
 
 const char* hils_status_string(hils_status s);
 

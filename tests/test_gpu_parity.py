@@ -204,6 +204,24 @@ def test_device_status_clear_after_forward():
     assert hb.device_status(ws) == 0
 
 
+def test_bounded_wait_gives_up_and_reports():
+    # the bounded mbarrier wait of the tensor-core kernels: a phase that nothing completes makes
+    # the wait give up after its poll limit, record HILS_ERR_TIMEOUT and let the kernel return;
+    # a completed phase records nothing; the context stays usable either way
+    wl = W.make("gqa7b_prefill", "cuda", N=2048)
+    p = hb.params_for(wl.q, wl.K, **wl.kwargs())
+    ws = hb.workspace(p, wl.q.device)
+    assert hb.device_status(ws) == 0
+    hb.wait_check(1000, True, ws)
+    assert hb.device_status(ws) == 0
+    hb.wait_check(1000, False, ws)
+    assert hb.device_status(ws) == 6
+    assert hb.device_status(ws) == 0          # reading cleared it
+    out, lse, idx = _run(wl, ws=ws)           # and the next forward runs normally
+    parity.full_check(wl, out, lse, idx)
+    assert hb.device_status(ws) == 0
+
+
 def test_invalid_arguments_raise_before_launch():
     wl = W.make("gqa7b_prefill", "cuda", N=2048)
     with pytest.raises(hb.HilsError) as e:
@@ -215,21 +233,40 @@ def test_invalid_arguments_raise_before_launch():
 
 
 # ------------------------------------------------------------------- full workload sizes
-FULL = [("small_mha_bf16", 2048), ("gqa7b_prefill", 512), ("long_decode", 64),
-        ("extreme", 256)]
+FULL = [("small_mha_bf16", 2048, {}), ("gqa7b_prefill", 512, {}), ("long_decode", 64, {}),
+        ("extreme", 256, {}), ("extreme", 256, dict(N=1 << 20)), ("extreme", 256, dict(N=1 << 22))]
 
 
-@pytest.mark.parametrize("name,rows", FULL)
-def test_full_size_sampled(name, rows):
-    wl = W.make(name, "cuda")
+@pytest.mark.parametrize("name,rows,kw", FULL,
+                         ids=lambda x: x if isinstance(x, str) else (
+                             "N=%d" % x["N"] if isinstance(x, dict) and "N" in x else
+                             ("full" if isinstance(x, dict) else str(x))))
+def test_full_size_sampled(name, rows, kw):
+    wl = W.make(name, "cuda", **kw)
     out, lse, idx = _run(wl)
     sample = parity.sample_rows(wl, rows, seed=7)
     errs = parity.sampled_check(wl, out, lse, idx, sample)
     assert errs["rows"] >= rows
-    # properties that hold at any size, on every row
+    _every_row_properties(wl, out, lse, idx)
+    if name == "extreme":
+        # the decode step of the sequence's last query (the extreme sweep's decode point)
+        del out, lse, idx
+        _free()
+        dec = W.decode_view(wl)
+        out, lse, idx = _run(dec)
+        parity.sampled_check(dec, out, lse, idx, [(0, 0, 0)])
+        _every_row_properties(dec, out, lse, idx)
+    del wl, out, lse, idx
+    _free()
+
+
+def _every_row_properties(wl, out, lse, idx):
+    """Properties that hold at any size, on every row."""
     Kt = wl.K_top
-    n = torch.tensor([parity.eligible(wl.q_pos0 + i, wl.S, wl.W) for i in range(wl.q.shape[2])],
-                     device="cuda")
+    pos = torch.arange(wl.q.shape[2], device="cuda", dtype=torch.int64) + wl.q_pos0
+    first = pos - wl.W + 1
+    n = torch.where(first > 0, torch.div(first, wl.S, rounding_mode="floor"),
+                    torch.zeros_like(first))
     k = torch.clamp(n, max=Kt)
     valid = idx >= 0
     assert torch.equal(valid.sum(-1), k.expand_as(valid.sum(-1)).to(valid.sum(-1).dtype))
@@ -238,5 +275,3 @@ def test_full_size_sampled(name, rows):
     dup = (srt[..., 1:] == srt[..., :-1]) & (srt[..., 1:] >= 0)
     assert not bool(dup.any())
     assert bool(torch.isfinite(out.float()).all()) and bool(torch.isfinite(lse).all())
-    del wl, out, lse, idx
-    _free()
