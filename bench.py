@@ -90,7 +90,7 @@ def work_model(dims, S, K, W, q_pos0, es):
 
 def phase_work(name, wm):
     """(bound, algorithmic work, unit) of a kernel, for its roofline."""
-    if name in ("score_topk_tc", "select_rows"):
+    if name in ("score_topk_tc", "score_topk_t_tc", "select_rows"):
         return "tensor", wm["score_flops"], "TFLOP/s"
     if name in ("select_split", "select_stream", "select_stream_tc"):
         return "hbm", wm["select_bytes"], "GB/s"
@@ -116,7 +116,8 @@ def roofline(name, ms, wm, peaks, workload, sustained=False):
 
 
 KERNEL_SOURCES = {
-    "score_topk_tc": ["score_tc.cu"], "attn_tc": ["attn_tc.cu"],
+    "score_topk_tc": ["score_tc.cu"], "score_topk_t_tc": ["score_t_tc.cu"],
+    "attn_tc": ["attn_tc.cu"],
     "select_stream": ["select.cu"], "select_topk": ["select.cu"], "select_rows": ["select.cu"],
     "select_split": ["select.cu"], "select_stream_tc": ["stream_tc.cu"],
     "attn_units": ["attn.cu"], "attn_units_tc": ["units_tc.cu"], "attn_rows": ["attn.cu"],

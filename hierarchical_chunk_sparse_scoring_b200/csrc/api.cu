@@ -34,6 +34,7 @@ struct Plan {
   bool bf16 = false;
   bool decode = false;
   bool tc_select = false;
+  bool tc_select_t = false;   // the landmark-major scoring kernel (G = 2, 4, 8)
   bool tc_attn = false;
   bool tc_stream = false;
   bool tc_units = false;
@@ -80,6 +81,7 @@ Plan make_plan(const hils_params* p) {
                       D.B * D.Hkv * D.N_kv < (int64_t)INT32_MAX &&
                       D.B * D.Hkv * D.C < (int64_t)INT32_MAX;
   P.tc_select = !P.decode && rows32 && score_tc_supported(D, P.bf16);
+  P.tc_select_t = P.tc_select && score_t_tc_supported(D, P.bf16);
   P.tc_attn = !P.decode && rows32 && attn_tc_supported(D, P.bf16);
   P.tc_stream = P.decode && stream_tc_supported(D, P.bf16);
   P.tc_units = P.decode && units_tc_supported(D, P.bf16);
@@ -174,7 +176,7 @@ int phase_names(const Plan& P, const char** names, int max_names) {
     return 4;
   }
   if (P.tc_select) {
-    pre[n++] = "score_topk_tc";
+    pre[n++] = P.tc_select_t ? "score_topk_t_tc" : "score_topk_tc";
     if (!P.tc_attn) pre[n++] = "select_scores";
   } else {
     pre[n++] = "select_rows";
@@ -182,6 +184,16 @@ int phase_names(const Plan& P, const char** names, int max_names) {
   pre[n++] = P.tc_attn ? "attn_tc" : "attn_rows";
   for (int i = 0; i < n && i < max_names; ++i) names[i] = pre[i];
   return n;
+}
+
+// Steps 1-2 of a prefill plan on the tensor cores: the landmark-major kernel where it applies,
+// else the query-major one.
+cudaError_t launch_prefill_select_tc(const Plan& P, const void* q_cal, const void* k_lm,
+                                     const float* b_lm, int32_t* idx, float* s_out,
+                                     int32_t* status, cudaStream_t st) {
+  return P.tc_select_t
+             ? launch_score_topk_t_tc(P.D, q_cal, k_lm, b_lm, idx, s_out, status, st)
+             : launch_score_topk_tc(P.D, q_cal, k_lm, b_lm, idx, s_out, status, st);
 }
 
 hils_status forward_impl(const hils_params* p, const void* q, const void* q_cal, const void* K,
@@ -232,7 +244,7 @@ hils_status forward_impl(const hils_params* p, const void* q, const void* q_cal,
     pm.mark();
   } else {
     if (P.tc_select) {
-      e = launch_score_topk_tc(P.D, q_cal, k_lm, b_lm, idx,
+      e = launch_prefill_select_tc(P, q_cal, k_lm, b_lm, idx,
                                P.tc_attn && P.D.G == 1 ? s_sel : nullptr,
                                reinterpret_cast<int32_t*>(ws), st);
       // the tensor-core attention takes the scores from there, or scores per head itself
@@ -310,7 +322,7 @@ extern "C" hils_status hils_select(const hils_params* p, const void* q_cal, cons
       e = launch_select_topk_row(P.D, P.bf16, P.n_stride, sig, q_cal, k_lm, b_lm, idx, s_sel, st);
   } else if (P.tc_select) {
     // with one head per KV group the scores the selection ranked by are the per-head scores
-    e = launch_score_topk_tc(P.D, q_cal, k_lm, b_lm, idx, P.D.G == 1 ? s_sel : nullptr,
+    e = launch_prefill_select_tc(P, q_cal, k_lm, b_lm, idx, P.D.G == 1 ? s_sel : nullptr,
                              reinterpret_cast<int32_t*>(ws), st);
     if (e == cudaSuccess && s_sel && P.D.G != 1)
       e = launch_select_scores(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
@@ -476,7 +488,7 @@ extern "C" hils_status hils_select_noalloc(const hils_params* p, const void* q_c
       e = launch_select_merge(P.D, P.bf16, P.n_split, pv, pc, q_cal, k_lm, b_lm, idx, s_sel, st);
   } else if (P.tc_select) {
     // with one head per KV group the scores the selection ranked by are the per-head scores
-    e = launch_score_topk_tc(P.D, q_cal, k_lm, b_lm, idx, P.D.G == 1 ? s_sel : nullptr,
+    e = launch_prefill_select_tc(P, q_cal, k_lm, b_lm, idx, P.D.G == 1 ? s_sel : nullptr,
                              reinterpret_cast<int32_t*>(ws), st);
     if (e == cudaSuccess && s_sel && P.D.G != 1)
       e = launch_select_scores(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);

@@ -310,33 +310,44 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
   for (int64_t c = (n_first << rs) + threadIdx.x; c <= last_chunk; c += kAtThreads)
     atomicOr(&bitmap[c >> 5], 1u << (c & 31));
   __syncthreads();
-  if (warp == 0) {
-    // list position of each bitmap word: one warp-wide scan per 32 words
-    int carry = 0;
-    for (int w0 = 0; w0 < nbw; w0 += 32) {
-      const int w = w0 + lane;
-      const int cnt = w < nbw ? __popc(bitmap[w]) : 0;
-      int x = cnt;
+  {
+    // list position of each bitmap word and the list itself (ascending tile order): every
+    // thread owns a contiguous run of words, counts their bits, takes its offset from a
+    // block-wide scan of those counts and places its own tiles; the work per thread grows with
+    // the sequence only by one load per word of its run
+    int* warp_tot = n_tiles_sh + 4;   // [6] bits per warp
+    const int seg = (nbw + kAtThreads - 1) / kAtThreads;
+    const int w_lo = threadIdx.x * seg;
+    const int w_hi = w_lo + seg < nbw ? w_lo + seg : nbw;
+    int mine = 0;
+    for (int w = w_lo; w < w_hi; ++w) mine += __popc(bitmap[w]);
+    int x = mine;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[warp] = x;
+    __syncthreads();
+    int off = x - mine, total = 0;
+#pragma unroll
+    for (int w2 = 0; w2 < kAtThreads / 32; ++w2) {
+      const int t2 = warp_tot[w2];
+      off += w2 < warp ? t2 : 0;
+      total += t2;
+    }
+    if (threadIdx.x == 0) {
+      if (total > list_cap) record_status(status, kStatusDeviceCheck);
+      *n_tiles_sh = total < list_cap ? total : list_cap;
+    }
+    for (int w = w_lo; w < w_hi; ++w) {
+      wpre[w] = off;
+      uint32_t wb = bitmap[w];
+      while (wb) {
+        if (off < list_cap) tiles[off] = w * 32 + __ffs(wb) - 1;
+        ++off;
+        wb &= wb - 1u;
       }
-      if (w < nbw) wpre[w] = carry + x - cnt;
-      carry += __shfl_sync(0xffffffffu, x, 31);
-    }
-    if (lane == 0) {
-      if (carry > list_cap) record_status(status, kStatusDeviceCheck);
-      *n_tiles_sh = carry < list_cap ? carry : list_cap;
-    }
-  }
-  __syncthreads();
-  // every thread places the set bits of its tiles: the list is the bitmap in ascending order
-  for (int tl = threadIdx.x; tl <= (int)last_chunk; tl += kAtThreads) {
-    const uint32_t wb = bitmap[tl >> 5];
-    if ((wb >> (tl & 31)) & 1u) {
-      const int pos = wpre[tl >> 5] + __popc(wb & ((1u << (tl & 31)) - 1u));
-      if (pos < list_cap) tiles[pos] = tl;
     }
   }
   tc_fence_before();

@@ -22,6 +22,12 @@ cudaError_t launch_score_topk_tc(const Dims& D, const void* qc, const void* klm,
                                  const float* blm, int32_t* idx, float* s_out, int32_t* status,
                                  cudaStream_t st);
 
+// landmark-major variant (landmark rows as the MMA's M, all G heads of a block as its N)
+bool score_t_tc_supported(const Dims& D, bool bf16);
+cudaError_t launch_score_topk_t_tc(const Dims& D, const void* qc, const void* klm,
+                                   const float* blm, int32_t* idx, float* s_out,
+                                   int32_t* status, cudaStream_t st);
+
 bool attn_tc_supported(const Dims& D, bool bf16);
 // s_sig: the scoring kernel's sigma of each selected chunk, required when D.G == 1 (it is then
 // the head's surrogate score); with G > 1 the kernel scores the selected chunks per head itself
