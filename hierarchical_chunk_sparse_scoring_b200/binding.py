@@ -46,6 +46,7 @@ SIGNATURES = {
     "hils_select_noalloc": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V]),
     "hils_select_noalloc_max_bytes": (ctypes.c_size_t, []),
     "hils_select_noalloc_status": (ctypes.c_int, [_V, ctypes.POINTER(ctypes.c_int32)]),
+    "hils_landmarks": (ctypes.c_int, [_P, _V, _V, _V, _V, _V]),
     "hils_wait_check": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_int, _V, ctypes.c_size_t, _V]),
     "hils_chunk_attn": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V, _V]),
     "hils_fuse": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V]),
@@ -230,6 +231,25 @@ def device_status(ws, stream=None):
     _check(lib().hils_device_status(_ptr(ws), _stream(stream), ctypes.byref(code)),
            "hils_device_status")
     return int(code.value)
+
+
+def landmarks(q_lm, K, *, S, scale=0.0, k_lm=None, b_lm=None, stream=None):
+    """Landmark construction: q_lm [B,Hkv,C,d] landmark queries, K [B,Hkv,N_kv,d] keys with
+    C = N_kv // S.  Returns (k_lm [B,Hkv,C,d] in K's dtype, b_lm [B,Hkv,C] fp32)."""
+    B, Hkv, N_kv, d = K.shape
+    C = N_kv // S
+    _need(K, "K")
+    _need(q_lm, "q_lm", K.dtype, (B, Hkv, C, d))
+    if k_lm is None:
+        k_lm = torch.empty((B, Hkv, C, d), dtype=K.dtype, device=K.device)
+    if b_lm is None:
+        b_lm = torch.empty((B, Hkv, C), dtype=torch.float32, device=K.device)
+    _need(k_lm, "k_lm", K.dtype, (B, Hkv, C, d))
+    _need(b_lm, "b_lm", torch.float32, (B, Hkv, C))
+    p = make_params(B, Hkv, Hkv, 0, N_kv, d, S=S, K_top=0, W=1, dtype=K.dtype, scale=scale)
+    _check(lib().hils_landmarks(ctypes.byref(p), _ptr(q_lm), _ptr(K), _ptr(k_lm), _ptr(b_lm),
+                                _stream(stream)), "hils_landmarks")
+    return k_lm, b_lm
 
 
 def select_noalloc(q_cal, k_lm, b_lm, *, N_kv, Hkv, S, K_top, W, q_pos0=0, scale=0.0,

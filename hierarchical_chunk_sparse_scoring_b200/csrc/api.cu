@@ -366,6 +366,23 @@ extern "C" hils_status hils_fuse(const hils_params* p, const float* s_sel, const
   return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA;
 }
 
+extern "C" hils_status hils_landmarks(const hils_params* p, const void* q_lm, const void* K,
+                                      void* k_lm, float* b_lm, hils_stream_t stream) {
+  hils_status s = check_params(p);
+  if (s != HILS_OK) return s;
+  if (p->d != 16 && p->d != 32 && p->d != 64 && p->d != 128) return HILS_ERR_UNSUPPORTED;
+  const Plan P = make_plan(p);
+  const bool any = P.D.B > 0 && P.D.C > 0;
+  if (!ok_ptr(q_lm, any) || !ok_ptr(K, any) || !ok_ptr(k_lm, any) || !ok_ptr(b_lm, any))
+    return HILS_ERR_INVALID_ARG;
+  if (!any) return HILS_OK;
+  if ((s = check_device()) != HILS_OK) return s;
+  return launch_landmarks(P.D, P.bf16, q_lm, K, k_lm, b_lm,
+                          reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? HILS_OK
+             : HILS_ERR_CUDA;
+}
+
 extern "C" hils_status hils_workspace_init(void* workspace, size_t workspace_bytes,
                                            hils_stream_t stream) {
   if (!workspace || !aligned16(workspace) || workspace_bytes < kStatusBytes)

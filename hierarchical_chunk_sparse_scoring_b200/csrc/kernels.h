@@ -71,6 +71,10 @@ cudaError_t launch_fuse_units(const Dims& D, bool bf16, int n_pieces, const floa
                               const float* part_o, const float* part_lse, void* out, float* lse,
                               cudaStream_t st);
 
+// Landmark construction: k_lm = softmax(scale q_lm . K_chunk) K_chunk, b_lm = its entropy.
+cudaError_t launch_landmarks(const Dims& D, bool bf16, const void* qlm, const void* K,
+                             void* klm, float* blm, cudaStream_t st);
+
 // One CTA waits on an mbarrier phase for at most `polls` polls (completed first if `complete`);
 // a wait that gives up records HILS_ERR_TIMEOUT in *status.
 cudaError_t launch_wait_check(uint32_t polls, int complete, int32_t* status, cudaStream_t st);

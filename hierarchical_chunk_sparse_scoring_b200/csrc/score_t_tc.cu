@@ -48,19 +48,23 @@ template <int DD, int G, int KM>
 struct TtShape {
   static constexpr int MQ = kCols / G;             // queries per CTA
   static constexpr int QH = MQ / 2;                // queries of one epilogue half
-  static constexpr int QP = MQ < 64 ? MQ : 64;     // queries per full-column pass
+  static constexpr int QP = 32;                    // queries per full-column pass
   static constexpr int NPASS = MQ / QP;
-  static constexpr int TPQ = kTtEpi / QP;          // stripe threads per query (4 or 8)
+  static constexpr int TPQ = kTtEpi / QP;          // stripe threads per query (8)
   static constexpr int RM = (KM + TPQ - 1) / TPQ;  // stripe list slots
   static constexpr int SCR_LD = kLm + TPQ;         // scratch row stride: conflict-free stripes
-  static constexpr int CAP = 2 * KM;               // buffered candidates per query per tile
+  static constexpr int CAP = MQ >= 128 ? 32 : 64;  // buffered candidates per query per tile
+  // row strides of the lists and buffers: odd, so the threads of consecutive queries hit
+  // different banks
+  static constexpr int LS = KM + 1;
+  static constexpr int CS = CAP + 1;
   static constexpr int KB = DD / 64;
   static constexpr int B_BOX = kCols * 128;        // [256 (head, query) rows x 64 dims]
   static constexpr int B_BYTES = KB * B_BOX;
   static constexpr int A_BOX = kLm * 128;          // [128 landmark rows x 64 dims]
   static constexpr int A_STAGE = KB * A_BOX;
-  static constexpr int LIST_BYTES = MQ * KM * 8;
-  static constexpr int CAND_BYTES = MQ * CAP * 8;
+  static constexpr int LIST_BYTES = MQ * LS * 8;
+  static constexpr int CAND_BYTES = MQ * CS * 8;
   static constexpr int SCR_BYTES = QP * SCR_LD * 4;
   static constexpr int MISC_BYTES = MQ * 12 + 64;  // theta, counts, eligible counts, flags
   static constexpr int FIXED = B_BYTES + LIST_BYTES + CAND_BYTES + SCR_BYTES + MISC_BYTES +
@@ -89,17 +93,17 @@ __global__ void __launch_bounds__(kTtThreads, 1)
                       float* __restrict__ s_out, int32_t* __restrict__ status) {
   using SH = TtShape<DD, G, KM>;
   constexpr int MQ = SH::MQ, QH = SH::QH, QP = SH::QP, TPQ = SH::TPQ, CAP = SH::CAP;
-  constexpr int RM = SH::RM, LD = SH::SCR_LD;
+  constexpr int RM = SH::RM, LD = SH::SCR_LD, LS = SH::LS, CS = SH::CS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sB = smem;                                                      // q_cal block (N)
   uint8_t* sA = sB + SH::B_BYTES;                                          // landmark ring (M)
-  float* list_v = reinterpret_cast<float*>(sA + SH::STAGES * SH::A_STAGE);   // [MQ][KM]
-  int* list_c = reinterpret_cast<int*>(list_v + MQ * KM);                    // [MQ][KM]
-  float* cand_v = reinterpret_cast<float*>(list_c + MQ * KM);                // [MQ][CAP]
-  int* cand_c = reinterpret_cast<int*>(cand_v + MQ * CAP);                   // [MQ][CAP]
-  float* scr = reinterpret_cast<float*>(cand_c + MQ * CAP);                  // [QP][LD]
+  float* list_v = reinterpret_cast<float*>(sA + SH::STAGES * SH::A_STAGE);   // [MQ][LS]
+  int* list_c = reinterpret_cast<int*>(list_v + MQ * LS);                    // [MQ][LS]
+  float* cand_v = reinterpret_cast<float*>(list_c + MQ * LS);                // [MQ][CS]
+  int* cand_c = reinterpret_cast<int*>(cand_v + MQ * CS);                    // [MQ][CS]
+  float* scr = reinterpret_cast<float*>(cand_c + MQ * CS);                   // [QP][LD]
   float* theta = scr + QP * LD;                                              // [MQ]
   int* cnt = reinterpret_cast<int*>(theta + MQ);                             // [MQ]
   int* nq = cnt + MQ;                                                        // [MQ]
@@ -136,8 +140,8 @@ __global__ void __launch_bounds__(kTtThreads, 1)
     fence_barrier_init();
   }
   // lists start empty: K live slots (-inf, INT_MAX) at the end of KM, sentinels in front
-  for (int e = threadIdx.x; e < MQ * KM; e += kTtThreads) {
-    const bool sentinel = (e % KM) < KM - K;
+  for (int e = threadIdx.x; e < MQ * LS; e += kTtThreads) {
+    const bool sentinel = (e % LS) < KM - K;
     list_v[e] = sentinel ? INFINITY : -INFINITY;
     list_c[e] = sentinel ? -1 : INT_MAX;
   }
@@ -282,7 +286,7 @@ __global__ void __launch_bounds__(kTtThreads, 1)
       auto serial_merge = [&](int q, int p) {
         TailList<KM> L;
 #pragma unroll
-        for (int k = 0; k < KM; ++k) { L.v[k] = list_v[q * KM + k]; L.c[k] = list_c[q * KM + k]; }
+        for (int k = 0; k < KM; ++k) { L.v[k] = list_v[q * LS + k]; L.c[k] = list_c[q * LS + k]; }
         const int ne = (int)(nq[q] - cbase < kLm ? nq[q] - cbase : kLm);
         const float* row = scr + (q - p * QP) * LD;
         for (int k0 = 0; k0 < kLm; ++k0) {
@@ -293,7 +297,7 @@ __global__ void __launch_bounds__(kTtThreads, 1)
           if (better(x, cc, L.kth_v(), L.kth_c())) L.insert(x, cc);
         }
 #pragma unroll
-        for (int k = 0; k < KM; ++k) { list_v[q * KM + k] = L.v[k]; list_c[q * KM + k] = L.c[k]; }
+        for (int k = 0; k < KM; ++k) { list_v[q * LS + k] = L.v[k]; list_c[q * LS + k] = L.c[k]; }
         theta[q] = L.kth_c() == INT_MAX ? -INFINITY : L.kth_v();
         cnt[q] = 0;
       };
@@ -301,10 +305,10 @@ __global__ void __launch_bounds__(kTtThreads, 1)
       auto buffer_merge = [&](int q, int n) {
         TailList<KM> L;
 #pragma unroll
-        for (int k = 0; k < KM; ++k) { L.v[k] = list_v[q * KM + k]; L.c[k] = list_c[q * KM + k]; }
-        for (int j = 0; j < n; ++j) L.insert(cand_v[q * CAP + j], cand_c[q * CAP + j]);
+        for (int k = 0; k < KM; ++k) { L.v[k] = list_v[q * LS + k]; L.c[k] = list_c[q * LS + k]; }
+        for (int j = 0; j < n; ++j) L.insert(cand_v[q * CS + j], cand_c[q * CS + j]);
 #pragma unroll
-        for (int k = 0; k < KM; ++k) { list_v[q * KM + k] = L.v[k]; list_c[q * KM + k] = L.c[k]; }
+        for (int k = 0; k < KM; ++k) { list_v[q * LS + k] = L.v[k]; list_c[q * LS + k] = L.c[k]; }
         theta[q] = L.kth_c() == INT_MAX ? -INFINITY : L.kth_v();
         cnt[q] = 0;
       };
@@ -347,19 +351,32 @@ __global__ void __launch_bounds__(kTtThreads, 1)
             for (int k = j; k < ne; k += TPQ) {
               const float x = row[k];
               if (x >= th) {
-                cand_v[q * CAP + off] = x;
-                cand_c[q * CAP + off] = k;   // (chunk = k, the first tile)
+                cand_v[q * CS + off] = x;
+                cand_c[q * CS + off] = k;   // (chunk = k, the first tile)
                 ++off;
               }
             }
           }
-          if (j == 0) cnt[q] = total;
           asm volatile("bar.sync 1, %0;" ::"n"(kTtEpi) : "memory");
-          if (tid < QP) {
-            const int qm = p * QP + tid;
-            const int n = cnt[qm];
-            if (n > CAP) serial_merge(qm, p);
-            else if (n > 0) buffer_merge(qm, n);
+          if (total > CAP) {
+            // more candidates than the buffer holds: one thread merges the whole column
+            if (j == 0) serial_merge(q, p);
+          } else {
+            // the list is empty: each candidate's rank among the query's candidates is its
+            // place in the sorted list (ties to the lower chunk)
+            for (int i = j; i < total; i += TPQ) {
+              const float cv = cand_v[q * CS + i];
+              const int cc = cand_c[q * CS + i];
+              int rank = 0;
+              for (int i2 = 0; i2 < total; ++i2)
+                rank += better(cand_v[q * CS + i2], cand_c[q * CS + i2], cv, cc) ? 1 : 0;
+              if (rank < K) {
+                list_v[q * LS + KM - K + rank] = cv;
+                list_c[q * LS + KM - K + rank] = cc;
+                if (rank == K - 1) theta[q] = cv;
+              }
+            }
+            if (j == 0) cnt[q] = 0;
           }
           asm volatile("bar.sync 1, %0;" ::"n"(kTtEpi) : "memory");
         }
@@ -401,8 +418,8 @@ __global__ void __launch_bounds__(kTtThreads, 1)
               const int q = q0 + e;
               const int slot = atomicAdd(&cnt[q], 1);
               if (slot < CAP) {
-                cand_v[q * CAP + slot] = x;
-                cand_c[q * CAP + slot] = (int)c;
+                cand_v[q * CS + slot] = x;
+                cand_c[q * CS + slot] = (int)c;
               } else {
                 flags[t & 1] = 1;
               }
@@ -446,10 +463,10 @@ __global__ void __launch_bounds__(kTtThreads, 1)
       int32_t* out = idx + (bg * D.N_q + i) * K - (KM - K);
       float* so = s_out ? s_out + (bg * D.N_q + i) * K - (KM - K) : nullptr;
       for (int k = KM - K; k < KM; ++k) {
-        const int cc = list_c[q * KM + k];
+        const int cc = list_c[q * LS + k];
         out[k] = cc == INT_MAX ? -1 : cc;
         if (so) {
-          const float vv = list_v[q * KM + k];
+          const float vv = list_v[q * LS + k];
           so[k] = (cc == INT_MAX || vv <= -FLT_MAX) ? -INFINITY : vv;
         }
       }

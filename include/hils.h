@@ -137,6 +137,22 @@ hils_status hils_fuse(const hils_params* p, const float* s_sel, const float* uni
                       const float* unit_lse, void* out, float* lse_out, hils_stream_t stream);
 
 /*
+ * Landmark construction, upstream of step 1 (the producer of k_lm and b_lm): for every (b, g)
+ * and completed chunk c (tokens c*S .. c*S+S-1; a partial last chunk has none),
+ *   p = softmax_j(scale * q_lm[b,g,c] . K[b,g,c*S+j]),
+ *   k_lm[b,g,c] = sum_j p_j K[b,g,c*S+j],   b_lm[b,g,c] = -sum_j p_j ln p_j
+ * ([Reader] "The HiLS-Attention Mechanism": the chunk summary is the landmark query's
+ * attention-weighted sum of the chunk's keys and its bias the entropy of those weights; with the
+ * same scale as step 1 the surrogate score at q_lm equals the chunk's exact log-mass).
+ * q_lm: [B, Hkv, C, d] dtype, one landmark query per completed chunk and KV head; K as for
+ * hils_forward; k_lm: [B, Hkv, C, d] dtype and b_lm: [B, Hkv, C] fp32 are written.  Reads only
+ * B, Hkv, N_kv, d, S, dtype and scale of `p` (the other fields must still be valid); d must be
+ * 16, 32, 64 or 128.  Asynchronous on `stream`; allocates nothing and needs no workspace.
+ */
+hils_status hils_landmarks(const hils_params* p, const void* q_lm, const void* K, void* k_lm,
+                           float* b_lm, hils_stream_t stream);
+
+/*
  * hils_select without a caller-provided workspace.  The paper has no counterpart: this entry
  * point exists for callers that cannot allocate device memory or pass a scratch buffer, e.g. a
  * plugin host that hands a kernel only its input and output tensors, or a serving loop whose
