@@ -121,7 +121,7 @@ KERNEL_SOURCES = {
     "select_stream": ["select.cu"], "select_topk": ["select.cu"], "select_rows": ["select.cu"],
     "select_split": ["select.cu"], "select_stream_tc": ["stream_tc.cu"],
     "attn_units": ["attn.cu"], "attn_units_tc": ["units_tc.cu"], "attn_rows": ["attn.cu"],
-    "fuse_units": ["attn.cu"],
+    "fuse_units": ["attn.cu"], "landmarks": ["landmarks.cu"],
 }
 SHARED_SOURCES = ["common.cuh", "sm100.cuh"]
 
@@ -564,6 +564,39 @@ def extra_extreme(steps, peaks, N=262144):
     return res
 
 
+def extra_landmarks(peaks, B, Hkv, N, d, S, steps=5, seed=77):
+    """Landmark construction (hils_landmarks) over a whole cache: every key read once, one
+    summary row and bias written per chunk; HBM-bound."""
+    from hierarchical_chunk_sparse_scoring_b200 import binding as hb
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    C = N // S
+    K = (torch.randn((B, Hkv, N, d), generator=g, device="cuda") / math.sqrt(d)).to(torch.bfloat16)
+    q_lm = (torch.randn((B, Hkv, C, d), generator=g, device="cuda") /
+            math.sqrt(d)).to(torch.bfloat16)
+    k_lm = torch.empty((B, Hkv, C, d), dtype=torch.bfloat16, device="cuda")
+    b_lm = torch.empty((B, Hkv, C), dtype=torch.float32, device="cuda")
+    flush = make_flush(K.device)
+    hb.landmarks(q_lm, K, S=S, k_lm=k_lm, b_lm=b_lm)
+    ms = []
+    for _ in range(steps):
+        flush()
+        a, b_ = make_events(2)
+        a.record()
+        hb.landmarks(q_lm, K, S=S, k_lm=k_lm, b_lm=b_lm)
+        b_.record()
+        torch.cuda.synchronize()
+        ms.append(a.elapsed_time(b_))
+    t = statistics.mean(ms)
+    nbytes = B * Hkv * (N * d * 2 + C * d * 2 * 2 + C * 4)
+    gbs = nbytes / (t * 1e-3) / 1e9
+    del K, q_lm, k_lm, b_lm
+    torch.cuda.empty_cache()
+    return {"kernel": "landmarks", "shape": {"B": B, "Hkv": Hkv, "N": N, "d": d, "S": S},
+            "ms": t, "bytes": nbytes,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"]}}
+
+
 def run_hils(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -638,6 +671,8 @@ def run_hils(args):
         line["decode"] = extra_decode(max(5, args.steps), peaks)
         line["extreme_256k"] = extra_extreme(3, peaks, N=1 << 18)
         line["extreme_1m"] = extra_extreme(2, peaks, N=1 << 20)
+        line["landmarks"] = [extra_landmarks(peaks, 1, 1, 1 << 22, 128, 128),
+                             extra_landmarks(peaks, 1, 8, 131072, 128, 64)]
     if dist:
         dist.destroy_process_group()
     if rank == 0:

@@ -288,19 +288,26 @@ __global__ void __launch_bounds__(TtShape<DD, G, KM>::THREADS, 1)
         const float* row = dmp + q * LD;
         float* stage = dump + MQ * LD + q * LD;   // the row of dump 1 (rank buffer, list)
         const int R = (K + TPQ - 1) / TPQ;
+        // the stripe's values, loaded at once (independent loads in flight), kept for the passes
+        constexpr int NS = kLm / TPQ;
+        float xs[NS];
+#pragma unroll
+        for (int u = 0; u < NS; ++u) xs[u] = row[j + u * TPQ];
         TailList<RM> w;
         w.clear(R);
-        for (int k = j; k < ne; k += TPQ) {
-          const float x = row[k];
-          if (x > w.kth_v()) w.insert_stream(x, k);
-        }
+#pragma unroll
+        for (int u = 0; u < NS; ++u)
+          if (j + u * TPQ < ne && xs[u] > w.kth_v()) w.insert_stream(xs[u], u);
         // theta0: the smallest of the stripes' R-th values (TPQ * R >= K values reach it);
         // a stripe with fewer than R eligible values leaves -inf (every value is kept)
         float th = w.kth_c() == INT_MAX ? -INFINITY : w.kth_v();
 #pragma unroll
         for (int o = 1; o < TPQ; o <<= 1) th = fminf(th, __shfl_xor_sync(0xffffffffu, th, o));
-        int mine = 0;
-        for (int k = j; k < ne; k += TPQ) mine += row[k] >= th ? 1 : 0;
+        uint32_t keep = 0;   // bit u: value u of the stripe is a candidate
+#pragma unroll
+        for (int u = 0; u < NS; ++u)
+          keep |= (j + u * TPQ < ne && xs[u] >= th ? 1u : 0u) << u;
+        const int mine = __popc(keep);
         // offsets of the stripes' candidates: exclusive scan over the query's TPQ lanes
         int incl = mine;
 #pragma unroll
@@ -311,11 +318,11 @@ __global__ void __launch_bounds__(TtShape<DD, G, KM>::THREADS, 1)
         const int total = __shfl_sync(0xffffffffu, incl, TPQ - 1, TPQ);
         if (total <= CAP0) {
           int off = incl - mine;
-          for (int k = j; k < ne; k += TPQ) {
-            const float x = row[k];
-            if (x >= th) {
-              stage[off] = x;
-              stage[CAP0 + off] = __int_as_float(k);   // (chunk = k, the first tile)
+#pragma unroll
+          for (int u = 0; u < NS; ++u) {
+            if ((keep >> u) & 1u) {
+              stage[off] = xs[u];
+              stage[CAP0 + off] = __int_as_float(j + u * TPQ);   // (chunk, the first tile)
               ++off;
             }
           }
@@ -345,17 +352,44 @@ __global__ void __launch_bounds__(TtShape<DD, G, KM>::THREADS, 1)
           }
         } else {
           // each candidate's rank among the query's candidates is its place in the sorted
-          // list (ties to the lower chunk)
-          for (int i = j; i < total; i += TPQ) {
-            const float cv = stage[i];
-            const int cc = __float_as_int(stage[CAP0 + i]);
-            int rank = 0;
-            for (int i2 = 0; i2 < total; ++i2)
-              rank += better(stage[i2], __float_as_int(stage[CAP0 + i2]), cv, cc) ? 1 : 0;
-            if (rank < K) {
-              stage[LIST0 + KM - K + rank] = cv;
-              stage[LIST0 + KM + KM - K + rank] = __int_as_float(cc);
-              if (rank == K - 1) theta[q] = cv;
+          // list (ties to the lower chunk): this thread's candidates i = j, j + TPQ, ... are held
+          // in registers and every candidate of the query is read once
+          constexpr int NMC = (CAP0 + TPQ - 1) / TPQ;
+          float mv[NMC];
+          int mc[NMC], rk[NMC];
+#pragma unroll
+          for (int m = 0; m < NMC; ++m) {
+            const int i = j + m * TPQ;
+            mv[m] = i < total ? stage[i] : -INFINITY;
+            mc[m] = i < total ? __float_as_int(stage[CAP0 + i]) : INT_MAX;
+            rk[m] = 0;
+          }
+          int i2 = 0;
+          for (; i2 + 4 <= total; i2 += 4) {
+            float ov[4];
+            int oc[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              ov[e] = stage[i2 + e];
+              oc[e] = __float_as_int(stage[CAP0 + i2 + e]);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+#pragma unroll
+              for (int m = 0; m < NMC; ++m) rk[m] += better(ov[e], oc[e], mv[m], mc[m]) ? 1 : 0;
+          }
+          for (; i2 < total; ++i2) {
+            const float ov = stage[i2];
+            const int oc = __float_as_int(stage[CAP0 + i2]);
+#pragma unroll
+            for (int m = 0; m < NMC; ++m) rk[m] += better(ov, oc, mv[m], mc[m]) ? 1 : 0;
+          }
+#pragma unroll
+          for (int m = 0; m < NMC; ++m) {
+            if (j + m * TPQ < total && rk[m] < K) {
+              stage[LIST0 + KM - K + rk[m]] = mv[m];
+              stage[LIST0 + KM + KM - K + rk[m]] = __int_as_float(mc[m]);
+              if (rk[m] == K - 1) theta[q] = mv[m];
             }
           }
         }
