@@ -424,11 +424,14 @@ __global__ void __launch_bounds__(TtShape<DD, G, KM>::THREADS, 1)
               pass |= (sg[4 * e4 + 3] > th.w ? 1u : 0u) << (4 * e4 + 3);
             }
             pass &= emask;
+            // (once the thresholds have settled most groups have no survivor in the warp)
+            if (__any_sync(0xffffffffu, pass != 0u)) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              if ((pass >> e) & 1u) dmp[(q0 + e) * LD + r] = sg[e];
-              const uint32_t bits = __ballot_sync(0xffffffffu, (pass >> e) & 1u);
-              if (lane == 0 && bits) msk[(q0 + e) * 4 + qd] = bits;
+              for (int e = 0; e < 16; ++e) {
+                if ((pass >> e) & 1u) dmp[(q0 + e) * LD + r] = sg[e];
+                const uint32_t bits = __ballot_sync(0xffffffffu, (pass >> e) & 1u);
+                if (lane == 0 && bits) msk[(q0 + e) * 4 + qd] = bits;
+              }
             }
           }
         }
