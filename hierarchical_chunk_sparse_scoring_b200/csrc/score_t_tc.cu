@@ -573,7 +573,12 @@ bool score_t_tc_supported(const Dims& D, bool bf16) {
   if (!bf16 || D.K < 1 || D.K > kMaxK || D.C < 1) return false;
   if (D.B * D.Hkv > 65535) return false;
   if (D.d != 64 && D.d != 128) return false;
-  return D.G == 4 || D.G == 8;
+  // four heads: only for long sequences (at least 8192 chunks, 64 or more landmark tiles for the
+  // last query blocks).  Each block pays a start-up (its calibrated-query tile, the first
+  // tile's ranking) that the query-major kernel's blocks of 128 queries amortise better when
+  // blocks are short: on the 7B-like prefill (2048 chunks) that kernel measured 2.29 ms
+  // against 2.91 ms here.
+  return D.G == 8 || (D.G == 4 && D.C >= 8192);
 }
 
 cudaError_t launch_score_topk_t_tc(const Dims& D, const void* qc, const void* klm,

@@ -234,7 +234,9 @@ def test_invalid_arguments_raise_before_launch():
 
 # ------------------------------------------------------------------- full workload sizes
 FULL = [("small_mha_bf16", 2048, {}), ("gqa7b_prefill", 512, {}), ("long_decode", 64, {}),
-        ("extreme", 256, {}), ("extreme", 256, dict(N=1 << 20)), ("extreme", 256, dict(N=1 << 22))]
+        ("extreme", 256, {}), ("extreme", 256, dict(N=1 << 20)), ("extreme", 256, dict(N=1 << 22)),
+        # four heads per group over 8192 chunks: the landmark-major scoring kernel at G = 4
+        ("gqa7b_prefill", 256, dict(N=1 << 19))]
 
 
 @pytest.mark.parametrize("name,rows,kw", FULL,
