@@ -570,9 +570,7 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
     if (!lm_ok) record_status(status, kStatusTimeout);
     float l = 0.f;
     bool sec_pending = false;   // S = 128: this row's next tile is the second half of its chunk
-    // S = 128: the second half's weights, computed with the first half (its logits are read
-    // once) and kept until that tile comes up
-    float q2[RS ? kTile : 1];
+    float sec_off = 0.f, sec_f = 0.f;
     int sel_next = 0;
     int sel_tn = (kSelSmem && n_sel > 0) ? sel_t[r * KM] : -1;
     const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
@@ -594,19 +592,12 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[x]);
-      const bool is_second = sec_pending;
-      sec_pending = false;
-      if constexpr (RS) {
-        // the second half of a selected chunk: its weights are ready
-        if (is_second) {
-#pragma unroll
-          for (int j = 0; j < kTile; ++j) p[j] = q2[j];
-        }
-      }
 
       const int c = tiles[t];   // tile index (64 tokens)
       float u = -INFINITY;
       bool is_sel = false;
+      const bool is_second = sec_pending;
+      sec_pending = false;
       if constexpr (kSelSmem) {
         // the next selected chunk of this row, in list order
         if (sel_next < n_sel && sel_tn == t) {
@@ -629,36 +620,34 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
       const float sc2 = D.scale * kLog2e;
       float mxc = 0.f;          // the chunk's max over both tiles (raw logits)
       float sum2_raw = 0.f;     // the second tile's exponentials' sum against that max
-      if constexpr (RS) {
-        const int x2 = x ^ 1;
-        if (__any_sync(0xffffffffu, first2)) {
-          if (!mbar_wait_warp(&s_full[x2], (uint32_t)((t + 1) >> 1) & 1u, kAtPollLimit)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+      const int x2 = x ^ 1;
+      const bool need2 = RS && __any_sync(0xffffffffu, first2);
+      if (need2) {
+        if (!mbar_wait_warp(&s_full[x2], (uint32_t)((t + 1) >> 1) & 1u, kAtPollLimit)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float mx2 = -INFINITY;
 #pragma unroll
-          for (int j = 0; j < kTile / 16; ++j) {
-            float tmp[16];
-            tmem_ld16(lane_base + (uint32_t)(x2 * kTile + 16 * j), tmp);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) q2[16 * j + e] = tmp[e];
-          }
+        for (int j = 0; j < kTile / 16; ++j) {
+          float tmp[16];
+          tmem_ld16(lane_base + (uint32_t)(x2 * kTile + 16 * j), tmp);
           tmem_wait_ld();
-          if (first2) {
-            mxc = fmaxf(max64(p), max64(q2));
-            const float offc = -mxc * sc2;
-            float ps[8];
 #pragma unroll
-            for (int q8 = 0; q8 < 8; ++q8) ps[q8] = 0.f;
+          for (int e = 0; e < 16; ++e) mx2 = fmaxf(mx2, tmp[e]);
+        }
+        mxc = fmaxf(max64(p), mx2);
+        const float offc = -mxc * sc2;
 #pragma unroll
-            for (int j = 0; j < kTile; j += 2) {
-              fma2(q2[j], q2[j + 1], sc2, offc);
-              q2[j] = fast_exp2(q2[j]);
-              q2[j + 1] = fast_exp2(q2[j + 1]);
-              add2(ps[j & 7], ps[(j & 7) + 1], q2[j], q2[j + 1]);
-            }
-            sum2_raw = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        for (int j = 0; j < kTile / 16; ++j) {
+          float tmp[16];
+          tmem_ld16(lane_base + (uint32_t)(x2 * kTile + 16 * j), tmp);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            fma2(tmp[e], tmp[e + 1], sc2, offc);
+            sum2_raw += fast_exp2(tmp[e]) + fast_exp2(tmp[e + 1]);
           }
         }
       }
@@ -666,7 +655,14 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
       float factor = 1.f;
       // base-2 exponentials throughout: x * scale * log2(e) is the logit in log2 units
       if (is_second) {
-        // second half of a selected chunk: p holds its weights already
+        // second half of a selected chunk: the max and normaliser of its first half
+#pragma unroll
+        for (int j = 0; j < kTile; j += 2) {
+          fma2(p[j], p[j + 1], sc2, sec_off);
+          p[j] = fast_exp2(p[j]);
+          p[j + 1] = fast_exp2(p[j + 1]);
+          mul2(p[j], p[j + 1], sec_f);
+        }
       } else if (is_sel && u != -INFINITY) {
         // intra-chunk softmax of this chunk, weighted by exp(u - m_run) (u <= m_run)
         // (three-input maxima, and fp32 pairs for the affine, sum and scale passes)
@@ -690,13 +686,7 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
 #pragma unroll
         for (int j = 0; j < kTile; j += 2) mul2(p[j], p[j + 1], f);
         l += w;
-        if constexpr (RS) {
-          if (first2) {
-            sec_pending = true;
-#pragma unroll
-            for (int j = 0; j < kTile; j += 2) mul2(q2[j], q2[j + 1], f);
-          }
-        }
+        if (first2) { sec_pending = true; sec_off = off; sec_f = f; }
       } else if (is_win) {
         // raw logits; only the tile holding the query's own position needs the causal mask
         if (t0 + kTile - 1 > pos) {
