@@ -24,6 +24,10 @@ constexpr size_t kStatusBytes = 256;
 constexpr int kChunksPerSplit = 512;
 constexpr int64_t kDecodeMaxQueries = 16;
 constexpr int kStreamRows = 1024;  // landmark rows per streaming CTA (a ring of bulk copies)
+// decode with fewer (b, g, query) rows than this: steps 1-2 by the split kernels (each CTA scores
+// and ranks one range of chunks of a row, a merge kernel combines the ranges), so a row's top-K
+// is spread over many SMs instead of one CTA per row
+constexpr int64_t kSplitRows = 32;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -38,9 +42,10 @@ struct Plan {
   bool tc_attn = false;
   bool tc_stream = false;
   bool tc_units = false;
+  bool split_select = false;   // decode steps 1-2 by select_split + select_merge
   int cps = 0, n_split = 0, n_pieces = 0;
   size_t off_idx = 0, off_ssel = 0, off_po = 0, off_pl = 0;
-  size_t off_sig = 0;
+  size_t off_sig = 0, off_pv = 0, off_pc = 0;
   int64_t n_stride = 0;
   size_t total = 0;
 };
@@ -114,7 +119,14 @@ Plan make_plan(const hils_params* p) {
     P.off_po = off; off = align_up(off + head_rows * NU * (size_t)D.d * sizeof(float));
     P.off_pl = off; off = align_up(off + head_rows * NU * sizeof(float));
     P.n_stride = (n_max + 3) / 4 * 4;
-    P.off_sig = off; off = align_up(off + sel_rows * (size_t)P.n_stride * sizeof(float));
+    P.split_select = (int64_t)sel_rows < kSplitRows && P.n_split >= 4;
+    if (P.split_select) {
+      const size_t lst = sel_rows * (size_t)P.n_split * (size_t)D.K;
+      P.off_pv = off; off = align_up(off + lst * sizeof(float));
+      P.off_pc = off; off = align_up(off + lst * sizeof(int32_t));
+    } else {
+      P.off_sig = off; off = align_up(off + sel_rows * (size_t)P.n_stride * sizeof(float));
+    }
   }
   P.total = off;
   return P;
@@ -168,8 +180,8 @@ int phase_names(const Plan& P, const char** names, int max_names) {
   const char* pre[4];
   int n = 0;
   if (P.decode) {
-    pre[0] = P.tc_stream ? "select_stream_tc" : "select_stream";
-    pre[1] = "select_topk";
+    pre[0] = P.split_select ? "select_split" : (P.tc_stream ? "select_stream_tc" : "select_stream");
+    pre[1] = P.split_select ? "select_merge" : "select_topk";
     pre[2] = P.tc_units ? "attn_units_tc" : "attn_units";
     pre[3] = "fuse_units";
     for (int i = 0; i < 4 && i < max_names; ++i) names[i] = pre[i];
@@ -194,6 +206,34 @@ cudaError_t launch_prefill_select_tc(const Plan& P, const void* q_cal, const voi
   return P.tc_select_t
              ? launch_score_topk_t_tc(P.D, q_cal, k_lm, b_lm, idx, s_out, status, st)
              : launch_score_topk_tc(P.D, q_cal, k_lm, b_lm, idx, s_out, status, st);
+}
+
+// Steps 1-2 of a decode plan: the streaming scorer and one top-K CTA per row, or, with few rows,
+// the split kernels.  Marks the caller's phase events after each kernel.
+cudaError_t launch_decode_select(const Plan& P, const void* q_cal, const void* k_lm,
+                                 const float* b_lm, int32_t* idx, float* s_sel, char* ws,
+                                 cudaStream_t st, PhaseMarks& pm) {
+  cudaError_t e;
+  if (P.split_select) {
+    float* pv = reinterpret_cast<float*>(ws + P.off_pv);
+    int32_t* pc = reinterpret_cast<int32_t*>(ws + P.off_pc);
+    e = launch_select_split(P.D, P.bf16, P.cps, P.n_split, q_cal, k_lm, b_lm, pv, pc, st);
+    pm.mark();
+    if (e == cudaSuccess)
+      e = launch_select_merge(P.D, P.bf16, P.n_split, pv, pc, q_cal, k_lm, b_lm, idx, s_sel, st);
+    pm.mark();
+    return e;
+  }
+  float* sig = reinterpret_cast<float*>(ws + P.off_sig);
+  e = P.tc_stream ? launch_select_stream_tc(P.D, q_cal, k_lm, b_lm, sig, P.n_stride,
+                                            reinterpret_cast<int32_t*>(ws), st)
+                  : launch_select_stream(P.D, P.bf16, kStreamRows, n_stream_split(P), P.n_stride,
+                                         q_cal, k_lm, b_lm, sig, reinterpret_cast<int32_t*>(ws), st);
+  pm.mark();
+  if (e == cudaSuccess)
+    e = launch_select_topk_row(P.D, P.bf16, P.n_stride, sig, q_cal, k_lm, b_lm, idx, s_sel, st);
+  pm.mark();
+  return e;
 }
 
 hils_status forward_impl(const hils_params* p, const void* q, const void* q_cal, const void* K,
@@ -223,16 +263,7 @@ hils_status forward_impl(const hils_params* p, const void* q, const void* q_cal,
   if (P.decode) {
     float* po = reinterpret_cast<float*>(ws + P.off_po);
     float* pl = reinterpret_cast<float*>(ws + P.off_pl);
-    float* sig = reinterpret_cast<float*>(ws + P.off_sig);
-    e = P.tc_stream ? launch_select_stream_tc(P.D, q_cal, k_lm, b_lm, sig, P.n_stride,
-                                              reinterpret_cast<int32_t*>(ws), st)
-                    : launch_select_stream(P.D, P.bf16, kStreamRows, n_stream_split(P), P.n_stride,
-                                           q_cal, k_lm, b_lm, sig, reinterpret_cast<int32_t*>(ws),
-                                           st);
-    pm.mark();
-    if (e == cudaSuccess)
-      e = launch_select_topk_row(P.D, P.bf16, P.n_stride, sig, q_cal, k_lm, b_lm, idx, s_sel, st);
-    pm.mark();
+    e = launch_decode_select(P, q_cal, k_lm, b_lm, idx, s_sel, ws, st, pm);
     if (e == cudaSuccess)
       e = P.tc_units ? launch_attn_units_tc(P.D, P.n_pieces, q, K, V, idx, po, pl,
                                             reinterpret_cast<int32_t*>(ws), st)
@@ -312,14 +343,8 @@ extern "C" hils_status hils_select(const hils_params* p, const void* q_cal, cons
   char* ws = static_cast<char*>(workspace);
   cudaError_t e;
   if (P.decode) {
-    float* sig = reinterpret_cast<float*>(ws + P.off_sig);
-    e = P.tc_stream ? launch_select_stream_tc(P.D, q_cal, k_lm, b_lm, sig, P.n_stride,
-                                              reinterpret_cast<int32_t*>(ws), st)
-                    : launch_select_stream(P.D, P.bf16, kStreamRows, n_stream_split(P), P.n_stride,
-                                           q_cal, k_lm, b_lm, sig, reinterpret_cast<int32_t*>(ws),
-                                           st);
-    if (e == cudaSuccess)
-      e = launch_select_topk_row(P.D, P.bf16, P.n_stride, sig, q_cal, k_lm, b_lm, idx, s_sel, st);
+    PhaseMarks none{nullptr, 0, 0, st};
+    e = launch_decode_select(P, q_cal, k_lm, b_lm, idx, s_sel, ws, st, none);
   } else if (P.tc_select) {
     // with one head per KV group the scores the selection ranked by are the per-head scores
     e = launch_prefill_select_tc(P, q_cal, k_lm, b_lm, idx, P.D.G == 1 ? s_sel : nullptr,

@@ -39,9 +39,11 @@ CASES = {
     "tc_g2_d64_k32": (dict(B=1, Hq=4, Hkv=2, N=4000, d=64, S=32, K=32, W_=128),
                       torch.bfloat16, "score_topk_tc, 32-slot lists"),
     "tc_g4_d128": (dict(B=1, Hq=8, Hkv=2, N=20000, d=128, S=64, K=16, W_=128),
-                   torch.bfloat16, "score_topk_tc, four heads"),
+                   torch.bfloat16, "score_topk_tc, four heads over fewer than 8192 chunks"),
     "tc_g8_d128_s128": (dict(B=1, Hq=8, Hkv=1, N=40000, d=128, S=128, K=16, W_=256),
-                        torch.bfloat16, "score_topk_tc, eight heads of 128 dimensions"),
+                        torch.bfloat16, "score_topk_t_tc (landmark-major), eight heads"),
+    "tc_g8_d64_k32": (dict(B=1, Hq=8, Hkv=1, N=20000, d=64, S=32, K=32, W_=128),
+                      torch.bfloat16, "score_topk_t_tc, 32-slot lists, d = 64"),
     "rows_fp32": (dict(B=1, Hq=4, Hkv=2, N=3000, d=64, S=32, K=8, W_=96),
                   torch.float32, "select_rows"),
     "rows_g16": (dict(B=1, Hq=16, Hkv=1, N=2000, d=64, S=32, K=8, W_=64),
@@ -52,6 +54,9 @@ CASES = {
                             N_q=1), torch.bfloat16, "select_stream_tc, select_topk"),
     "decode_fp32": (dict(B=2, Hq=4, Hkv=2, N=50000, d=128, S=64, K=16, W_=512, q_pos0=49999,
                          N_q=1), torch.float32, "select_stream, select_topk"),
+    # one row over 4,680 chunks: the split kernels (few rows spread over many CTAs)
+    "decode_split_rows": (dict(B=1, Hq=8, Hkv=1, N=300000, d=128, S=64, K=16, W_=512,
+                               q_pos0=299999, N_q=1), torch.bfloat16, "select_split, select_merge"),
     "decode_multi_query": (dict(B=2, Hq=4, Hkv=2, N=9000, d=128, S=64, K=8, W_=256,
                                 q_pos0=8996, N_q=4), torch.bfloat16,
                            "select_stream_tc, select_topk"),
