@@ -513,6 +513,66 @@ def extra_decode(steps, peaks, **overrides):
     return res
 
 
+def extra_decode_step(steps, peaks):
+    """hils_decode_step on the long-decode cache (32 sequences, 512K tokens, 32/8 heads): append
+    the token, build the landmark of the chunk it completes, and the forward for its query, as one
+    CUDA graph replay; at a chunk boundary (pos = N - 1) and inside a chunk (pos = N - 2)."""
+    from hierarchical_chunk_sparse_scoring_b200 import binding as hb
+    from hierarchical_chunk_sparse_scoring_b200 import workloads as W
+    wl = W.make("long_decode", "cuda")
+    B, Hq, _, d = wl.q.shape
+    Hkv, N = wl.K.shape[1], wl.K.shape[2]
+    g = torch.Generator(device="cuda").manual_seed(99)
+    k_new = wl.K[:, :, -1].clone()
+    v_new = wl.V[:, :, -1].clone()
+    q_lm = (torch.randn((B, Hkv, d), generator=g, device="cuda") / math.sqrt(d)).to(wl.q.dtype)
+    flush = make_flush(wl.q.device)
+    res = {"workload": "long_decode", "B": B, "N": N}
+    for label, pos in (("chunk_boundary", N - 1), ("inside_chunk", N - 2)):
+        p = hb.make_params(B, Hq, Hkv, 1, N, d, S=wl.S, K_top=wl.K_top, W=wl.W, q_pos0=pos)
+        s = torch.cuda.Stream()
+        out = torch.empty_like(wl.q)
+        lse = torch.empty((B, Hq, 1), dtype=torch.float32, device="cuda")
+        idx = torch.empty((B, Hkv, 1, wl.K_top), dtype=torch.int32, device="cuda")
+        ws = hb.workspace(p, wl.q.device, stream=s)
+
+        def call():
+            hb.decode_step(wl.q, wl.q_cal, k_new, v_new, q_lm, wl.K, wl.V, wl.k_lm, wl.b_lm,
+                           pos=pos, S=wl.S, K_top=wl.K_top, W=wl.W, out=out, lse=lse, idx=idx,
+                           ws=ws, stream=s)
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            call()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=s):
+            call()
+        graph.replay()
+        torch.cuda.synchronize()
+        us = []
+        for _ in range(steps):
+            flush()
+            a, b_ = make_events(2)
+            a.record()
+            graph.replay()
+            b_.record()
+            torch.cuda.synchronize()
+            us.append(a.elapsed_time(b_) * 1e3)
+        del graph
+        wm = work_model(dict(B=B, Hq=Hq, Hkv=Hkv, N_q=1, N_kv=N, d=d), wl.S, wl.K_top, wl.W, pos,
+                        wl.q.element_size())
+        nbytes = wm["select_bytes"] + wm["attn_bytes"] + 2 * B * Hkv * d * 2 * 2
+        if pos == N - 1:
+            nbytes += B * Hkv * (wl.S * d * 2 + 2 * d * 2 + 4)
+        t = statistics.median(us)
+        res[label] = {"pos": pos, "us_per_step": t, "step_bytes": nbytes,
+                      "hbm_frac": nbytes / (t * 1e-6) / 1e9 / peaks["hbm_gbs"]}
+    del wl
+    torch.cuda.empty_cache()
+    return res
+
+
 def union_stat(idx, tq, C):
     """Mean number of distinct chunks selected by tq adjacent queries of a KV group, divided by
     K (how much the packed attention shares chunk loads)."""
@@ -669,6 +729,7 @@ def run_hils(args):
         line["prefill_small_mha"] = extra_prefill("small_mha_bf16", 5, peaks)
         line["prefill_gqa7b"] = extra_prefill("gqa7b_prefill", 3, peaks)
         line["decode"] = extra_decode(max(5, args.steps), peaks)
+        line["decode_step"] = extra_decode_step(max(5, args.steps), peaks)
         line["extreme_256k"] = extra_extreme(3, peaks, N=1 << 18)
         line["extreme_1m"] = extra_extreme(2, peaks, N=1 << 20)
         line["landmarks"] = [extra_landmarks(peaks, 1, 1, 1 << 22, 128, 128),

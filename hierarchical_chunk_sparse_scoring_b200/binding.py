@@ -47,6 +47,7 @@ SIGNATURES = {
     "hils_select_noalloc_max_bytes": (ctypes.c_size_t, []),
     "hils_select_noalloc_status": (ctypes.c_int, [_V, ctypes.POINTER(ctypes.c_int32)]),
     "hils_landmarks": (ctypes.c_int, [_P, _V, _V, _V, _V, _V]),
+    "hils_decode_step": (ctypes.c_int, [_P] + [_V] * 13 + [ctypes.c_size_t, _V]),
     "hils_wait_check": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_int, _V, ctypes.c_size_t, _V]),
     "hils_chunk_attn": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V, _V]),
     "hils_fuse": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V]),
@@ -250,6 +251,31 @@ def landmarks(q_lm, K, *, S, scale=0.0, k_lm=None, b_lm=None, stream=None):
     _check(lib().hils_landmarks(ctypes.byref(p), _ptr(q_lm), _ptr(K), _ptr(k_lm), _ptr(b_lm),
                                 _stream(stream)), "hils_landmarks")
     return k_lm, b_lm
+
+
+def decode_step(q, q_cal, k_new, v_new, q_lm_new, K, V, k_lm, b_lm, *, pos, S, K_top, W,
+                scale=0.0, out=None, lse=None, idx=None, ws=None, stream=None):
+    """One decode step over a cache of capacity K.shape[2]: appends (k_new, v_new) at `pos`,
+    builds the landmark of the chunk the token completes (q_lm_new, may be None otherwise) and
+    runs the forward for the query at `pos`.  Returns (out, lse, idx)."""
+    B, Hq, N_q, d = q.shape
+    _, Hkv, N_cap, _ = K.shape
+    p = make_params(B, Hq, Hkv, N_q, N_cap, d, S=S, K_top=K_top, W=W, q_pos0=pos,
+                    dtype=q.dtype, scale=scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, N_q), dtype=torch.float32, device=q.device)
+    if idx is None:
+        idx = torch.empty((B, Hkv, N_q, K_top), dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = workspace(p, q.device, stream)
+    _check(lib().hils_decode_step(ctypes.byref(p), _ptr(q), _ptr(q_cal), _ptr(k_new),
+                                  _ptr(v_new), _ptr(q_lm_new) if q_lm_new is not None else None,
+                                  _ptr(K), _ptr(V), _ptr(k_lm), _ptr(b_lm), _ptr(out), _ptr(lse),
+                                  _ptr(idx), _ptr(ws), ws.numel(), _stream(stream)),
+           "hils_decode_step")
+    return out, lse, idx
 
 
 def select_noalloc(q_cal, k_lm, b_lm, *, N_kv, Hkv, S, K_top, W, q_pos0=0, scale=0.0,

@@ -402,10 +402,47 @@ extern "C" hils_status hils_landmarks(const hils_params* p, const void* q_lm, co
     return HILS_ERR_INVALID_ARG;
   if (!any) return HILS_OK;
   if ((s = check_device()) != HILS_OK) return s;
-  return launch_landmarks(P.D, P.bf16, q_lm, K, k_lm, b_lm,
+  return launch_landmarks(P.D, P.bf16, 0, P.D.C, P.D.C, q_lm, K, k_lm, b_lm,
                           reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? HILS_OK
              : HILS_ERR_CUDA;
+}
+
+extern "C" hils_status hils_decode_step(const hils_params* p, const void* q, const void* q_cal,
+                                        const void* k_new, const void* v_new,
+                                        const void* q_lm_new, void* K, void* V, void* k_lm,
+                                        float* b_lm, void* out, float* lse_out,
+                                        int32_t* topk_idx_out, void* workspace,
+                                        size_t workspace_bytes, hils_stream_t stream) {
+  hils_status s = check_params(p);
+  if (s != HILS_OK) return s;
+  if (p->N_q != 1) return HILS_ERR_INVALID_ARG;
+  const Plan P = make_plan(p);
+  if (!P.decode || p->d % (p->dtype == HILS_BF16 ? 8 : 4) != 0) return HILS_ERR_UNSUPPORTED;
+  const int64_t pos = p->q_pos0;
+  // the new token completes chunk c_done when it is the chunk's last one
+  const bool completes = (pos + 1) % p->S == 0;
+  const bool any = p->B > 0;
+  if (!ok_ptr(k_new, any) || !ok_ptr(v_new, any) || !ok_ptr(K, any) || !ok_ptr(V, any) ||
+      !ok_ptr(q_lm_new, any && completes) || !ok_ptr(k_lm, any && completes) ||
+      !ok_ptr(b_lm, any && completes))
+    return HILS_ERR_INVALID_ARG;
+  if (!any) return HILS_OK;
+  // the forward's own checks come first, so a bad call writes nothing
+  if (!ok_ptr(q, true) || !ok_ptr(q_cal, true) || !ok_ptr(out, true) ||
+      (lse_out && !aligned16(lse_out)) || (topk_idx_out && !aligned16(topk_idx_out)) ||
+      (P.D.C > 0 && (!ok_ptr(k_lm, true) || !ok_ptr(b_lm, true))))
+    return HILS_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < P.total) return HILS_ERR_WORKSPACE;
+  if ((s = check_device()) != HILS_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (launch_append_kv(P.D, P.bf16, pos, k_new, v_new, K, V, st) != cudaSuccess)
+    return HILS_ERR_CUDA;
+  if (completes && launch_landmarks(P.D, P.bf16, pos / p->S, 1, 1, q_lm_new, K, k_lm, b_lm, st) !=
+                       cudaSuccess)
+    return HILS_ERR_CUDA;
+  return forward_impl(p, q, q_cal, K, V, k_lm, b_lm, out, lse_out, topk_idx_out, workspace,
+                      workspace_bytes, stream, nullptr, 0);
 }
 
 extern "C" hils_status hils_workspace_init(void* workspace, size_t workspace_bytes,

@@ -71,9 +71,14 @@ cudaError_t launch_fuse_units(const Dims& D, bool bf16, int n_pieces, const floa
                               const float* part_o, const float* part_lse, void* out, float* lse,
                               cudaStream_t st);
 
-// Landmark construction: k_lm = softmax(scale q_lm . K_chunk) K_chunk, b_lm = its entropy.
-cudaError_t launch_landmarks(const Dims& D, bool bf16, const void* qlm, const void* K,
-                             void* klm, float* blm, cudaStream_t st);
+// Landmark construction: k_lm = softmax(scale q_lm . K_chunk) K_chunk, b_lm = its entropy, for
+// chunks c0 .. c0+nc-1 of every (b, g); chunk c0 + cc's landmark query is row bg*qlm_rows + cc.
+cudaError_t launch_landmarks(const Dims& D, bool bf16, int64_t c0, int64_t nc,
+                             int64_t qlm_rows, const void* qlm, const void* K, void* klm,
+                             float* blm, cudaStream_t st);
+// K[b, g, pos] = k_new[b, g], V[b, g, pos] = v_new[b, g] (row stride of the cache: D.N_kv).
+cudaError_t launch_append_kv(const Dims& D, bool bf16, int64_t pos, const void* k_new,
+                             const void* v_new, void* K, void* V, cudaStream_t st);
 
 // One CTA waits on an mbarrier phase for at most `polls` polls (completed first if `complete`);
 // a wait that gives up records HILS_ERR_TIMEOUT in *status.

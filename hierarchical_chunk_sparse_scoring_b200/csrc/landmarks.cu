@@ -29,21 +29,26 @@ __device__ __forceinline__ void load4(const T* p, float (&v)[4]) {
   Elem<T>::load4(p, v);
 }
 
+// Chunks c0 .. c0+nc-1 of every (b, g); the landmark query of chunk c0 + cc of plane bg is row
+// bg * qlm_rows + cc of qlm.
 template <typename T, int DD>
 __global__ void __launch_bounds__(32 * kLmWarps)
-    landmarks_kernel(Dims D, const T* __restrict__ qlm, const T* __restrict__ K,
-                     T* __restrict__ klm, float* __restrict__ blm) {
+    landmarks_kernel(Dims D, int64_t c0, int64_t nc, int64_t qlm_rows,
+                     const T* __restrict__ qlm, const T* __restrict__ K, T* __restrict__ klm,
+                     float* __restrict__ blm) {
   constexpr int LPK = DD / 4;     // lanes per key row (4 elements each)
   constexpr int PAR = 32 / LPK;   // keys per warp step
   static_assert(DD >= 16 && DD <= 128 && (DD & (DD - 1)) == 0, "head dims 16, 32, 64, 128");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t chunk = (int64_t)blockIdx.x * kLmWarps + warp;   // over B * Hkv * C
-  if (chunk >= D.B * D.Hkv * D.C) return;   // (no block-wide barrier below)
-  const int64_t bg = chunk / D.C, c = chunk - bg * D.C;
+  const int64_t item = (int64_t)blockIdx.x * kLmWarps + warp;   // over B * Hkv * nc
+  if (item >= D.B * D.Hkv * nc) return;   // (no block-wide barrier below)
+  const int64_t bg = item / nc, cc = item - bg * nc;
+  const int64_t c = c0 + cc;
+  const int64_t chunk = bg * D.C + c;   // the landmark's row
   const int grp = lane / LPK, sl = lane % LPK;   // key group, 4-element slice of the row
   const int dim = sl * 4;
   float q[4];
-  load4(qlm + chunk * DD + dim, q);
+  load4(qlm + (bg * qlm_rows + cc) * DD + dim, q);
   // logits in base 2: y = x * log2(e)
   const float qs = D.scale * kLog2e;
 #pragma unroll
@@ -127,14 +132,16 @@ __global__ void __launch_bounds__(32 * kLmWarps)
 
 }  // namespace
 
-cudaError_t launch_landmarks(const Dims& D, bool bf16, const void* qlm, const void* K,
-                             void* klm, float* blm, cudaStream_t st) {
-  const int64_t n = D.B * D.Hkv * D.C;
+cudaError_t launch_landmarks(const Dims& D, bool bf16, int64_t c0, int64_t nc,
+                             int64_t qlm_rows, const void* qlm, const void* K, void* klm,
+                             float* blm, cudaStream_t st) {
+  const int64_t n = D.B * D.Hkv * nc;
   if (n == 0) return cudaSuccess;
   const dim3 grid((unsigned)((n + kLmWarps - 1) / kLmWarps));
 #define HILS_LM(TT, DDV)                                                                      \
   landmarks_kernel<TT, DDV><<<grid, 32 * kLmWarps, 0, st>>>(                                  \
-      D, static_cast<const TT*>(qlm), static_cast<const TT*>(K), static_cast<TT*>(klm), blm)
+      D, c0, nc, qlm_rows, static_cast<const TT*>(qlm), static_cast<const TT*>(K),            \
+      static_cast<TT*>(klm), blm)
   if (bf16) {
     if (D.d == 128) HILS_LM(__nv_bfloat16, 128);
     else if (D.d == 64) HILS_LM(__nv_bfloat16, 64);
@@ -149,6 +156,45 @@ cudaError_t launch_landmarks(const Dims& D, bool bf16, const void* qlm, const vo
     else return cudaErrorInvalidValue;
   }
 #undef HILS_LM
+  return cudaGetLastError();
+}
+
+}  // namespace hils
+
+namespace hils {
+namespace {
+
+// K[b, g, pos] = k_new[b, g] and V[b, g, pos] = v_new[b, g]: one 16-byte piece per thread.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    append_kv_kernel(Dims D, int64_t pos, const T* __restrict__ k_new,
+                     const T* __restrict__ v_new, T* __restrict__ K, T* __restrict__ V) {
+  constexpr int U = 16 / (int)sizeof(T);          // elements per 16-byte piece
+  const int64_t pieces = D.d / U;                 // per row
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= 2 * D.B * D.Hkv * pieces) return;
+  const int64_t kv = e / (D.B * D.Hkv * pieces), r = e - kv * D.B * D.Hkv * pieces;
+  const int64_t bg = r / pieces, u = r - bg * pieces;
+  const T* src = (kv == 0 ? k_new : v_new) + bg * D.d + u * U;
+  T* dst = (kv == 0 ? K : V) + (bg * D.N_kv + pos) * D.d + u * U;
+  *reinterpret_cast<uint4*>(dst) = __ldg(reinterpret_cast<const uint4*>(src));
+}
+
+}  // namespace
+
+cudaError_t launch_append_kv(const Dims& D, bool bf16, int64_t pos, const void* k_new,
+                             const void* v_new, void* K, void* V, cudaStream_t st) {
+  const int64_t n = 2 * D.B * D.Hkv * D.d / (bf16 ? 8 : 4);
+  if (n == 0) return cudaSuccess;
+  const unsigned grid = (unsigned)((n + 255) / 256);
+  if (bf16)
+    append_kv_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        D, pos, static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new),
+        static_cast<__nv_bfloat16*>(K), static_cast<__nv_bfloat16*>(V));
+  else
+    append_kv_kernel<float><<<grid, 256, 0, st>>>(D, pos, static_cast<const float*>(k_new),
+                                                  static_cast<const float*>(v_new),
+                                                  static_cast<float*>(K), static_cast<float*>(V));
   return cudaGetLastError();
 }
 

@@ -153,6 +153,30 @@ hils_status hils_landmarks(const hils_params* p, const void* q_lm, const void* K
                            float* b_lm, hils_stream_t stream);
 
 /*
+ * One decode step over a KV cache that grows by one token per call ([Reader] Fig. 6 caption:
+ * decode latency per token, timed with CUDA graphs; [Essay] "What the numbers actually say": the
+ * cache is paged by chunk, a chunk's landmark exists once the chunk is complete).  `p` describes
+ * the cache: N_kv is its capacity (rows per (b, g) plane of K, V; C = N_kv / S landmark rows per
+ * plane of k_lm, b_lm), q_pos0 = pos is the new token's position (pos < N_kv) and N_q = 1.  The
+ * call
+ *   1. appends the new token: K[b,g,pos] = k_new[b,g], V[b,g,pos] = v_new[b,g];
+ *   2. if the token completes chunk c = pos / S (that is, (pos + 1) % S == 0), builds that
+ *      chunk's landmark k_lm[b,g,c], b_lm[b,g,c] from its landmark query q_lm_new[b,g] as
+ *      hils_landmarks does (q_lm_new may be NULL otherwise);
+ *   3. runs hils_forward for the query at pos (q, q_cal [B, Hq, 1, d]; out, lse_out,
+ *      topk_idx_out as there).  Only tokens 0..pos and landmarks of chunks before the query's
+ *      window are read, so the cache beyond pos may hold anything.
+ * k_new, v_new, q_lm_new: [B, Hkv, d] in dtype.  Workspace: hils_workspace_size(p).  Supported:
+ * the decode shapes of hils_forward (d = 64 or 128).  Asynchronous on `stream`; the launches are
+ * fixed for given arguments, so a step can be captured in a CUDA graph and replayed.
+ */
+hils_status hils_decode_step(const hils_params* p, const void* q, const void* q_cal,
+                             const void* k_new, const void* v_new, const void* q_lm_new,
+                             void* K, void* V, void* k_lm, float* b_lm, void* out,
+                             float* lse_out, int32_t* topk_idx_out, void* workspace,
+                             size_t workspace_bytes, hils_stream_t stream);
+
+/*
  * hils_select without a caller-provided workspace.  The paper has no counterpart: this entry
  * point exists for callers that cannot allocate device memory or pass a scratch buffer, e.g. a
  * plugin host that hands a kernel only its input and output tensors, or a serving loop whose
