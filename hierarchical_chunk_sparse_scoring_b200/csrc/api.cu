@@ -24,10 +24,7 @@ constexpr size_t kStatusBytes = 256;
 constexpr int kChunksPerSplit = 512;
 constexpr int64_t kDecodeMaxQueries = 16;
 constexpr int kStreamRows = 1024;  // landmark rows per streaming CTA (a ring of bulk copies)
-// decode with fewer (b, g, query) rows than this: steps 1-2 by the split kernels (each CTA scores
-// and ranks one range of chunks of a row, a merge kernel combines the ranges), so a row's top-K
-// is spread over many SMs instead of one CTA per row
-constexpr int64_t kSplitRows = 32;
+
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -119,7 +116,9 @@ Plan make_plan(const hils_params* p) {
     P.off_po = off; off = align_up(off + head_rows * NU * (size_t)D.d * sizeof(float));
     P.off_pl = off; off = align_up(off + head_rows * NU * sizeof(float));
     P.n_stride = (n_max + 3) / 4 * 4;
-    P.split_select = (int64_t)sel_rows < kSplitRows && P.n_split >= 4;
+    // (measured slower than the streaming scorer and the per-row top-K on every shape tried:
+    // 119 against 64 us for one row of 32,752 chunks; kept for the allocation-free entry point)
+    P.split_select = false;
     if (P.split_select) {
       const size_t lst = sel_rows * (size_t)P.n_split * (size_t)D.K;
       P.off_pv = off; off = align_up(off + lst * sizeof(float));

@@ -54,9 +54,9 @@ CASES = {
                             N_q=1), torch.bfloat16, "select_stream_tc, select_topk"),
     "decode_fp32": (dict(B=2, Hq=4, Hkv=2, N=50000, d=128, S=64, K=16, W_=512, q_pos0=49999,
                          N_q=1), torch.float32, "select_stream, select_topk"),
-    # one row over 4,680 chunks: the split kernels (few rows spread over many CTAs)
-    "decode_split_rows": (dict(B=1, Hq=8, Hkv=1, N=300000, d=128, S=64, K=16, W_=512,
-                               q_pos0=299999, N_q=1), torch.bfloat16, "select_split, select_merge"),
+    # one row over 4,680 chunks (one top-K CTA for the whole row)
+    "decode_one_row": (dict(B=1, Hq=8, Hkv=1, N=300000, d=128, S=64, K=16, W_=512,
+                            q_pos0=299999, N_q=1), torch.bfloat16, "select_stream_tc, select_topk"),
     "decode_multi_query": (dict(B=2, Hq=4, Hkv=2, N=9000, d=128, S=64, K=8, W_=256,
                                 q_pos0=8996, N_q=4), torch.bfloat16,
                            "select_stream_tc, select_topk"),
