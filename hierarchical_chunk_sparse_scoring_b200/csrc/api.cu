@@ -39,10 +39,9 @@ struct Plan {
   bool tc_attn = false;
   bool tc_stream = false;
   bool tc_units = false;
-  bool split_select = false;   // decode steps 1-2 by select_split + select_merge
   int cps = 0, n_split = 0, n_pieces = 0;
   size_t off_idx = 0, off_ssel = 0, off_po = 0, off_pl = 0;
-  size_t off_sig = 0, off_pv = 0, off_pc = 0;
+  size_t off_sig = 0;
   int64_t n_stride = 0;
   size_t total = 0;
 };
@@ -116,16 +115,7 @@ Plan make_plan(const hils_params* p) {
     P.off_po = off; off = align_up(off + head_rows * NU * (size_t)D.d * sizeof(float));
     P.off_pl = off; off = align_up(off + head_rows * NU * sizeof(float));
     P.n_stride = (n_max + 3) / 4 * 4;
-    // (measured slower than the streaming scorer and the per-row top-K on every shape tried:
-    // 119 against 64 us for one row of 32,752 chunks; kept for the allocation-free entry point)
-    P.split_select = false;
-    if (P.split_select) {
-      const size_t lst = sel_rows * (size_t)P.n_split * (size_t)D.K;
-      P.off_pv = off; off = align_up(off + lst * sizeof(float));
-      P.off_pc = off; off = align_up(off + lst * sizeof(int32_t));
-    } else {
-      P.off_sig = off; off = align_up(off + sel_rows * (size_t)P.n_stride * sizeof(float));
-    }
+    P.off_sig = off; off = align_up(off + sel_rows * (size_t)P.n_stride * sizeof(float));
   }
   P.total = off;
   return P;
@@ -179,8 +169,8 @@ int phase_names(const Plan& P, const char** names, int max_names) {
   const char* pre[4];
   int n = 0;
   if (P.decode) {
-    pre[0] = P.split_select ? "select_split" : (P.tc_stream ? "select_stream_tc" : "select_stream");
-    pre[1] = P.split_select ? "select_merge" : "select_topk";
+    pre[0] = P.tc_stream ? "select_stream_tc" : "select_stream";
+    pre[1] = "select_topk";
     pre[2] = P.tc_units ? "attn_units_tc" : "attn_units";
     pre[3] = "fuse_units";
     for (int i = 0; i < 4 && i < max_names; ++i) names[i] = pre[i];
@@ -207,22 +197,12 @@ cudaError_t launch_prefill_select_tc(const Plan& P, const void* q_cal, const voi
              : launch_score_topk_tc(P.D, q_cal, k_lm, b_lm, idx, s_out, status, st);
 }
 
-// Steps 1-2 of a decode plan: the streaming scorer and one top-K CTA per row, or, with few rows,
-// the split kernels.  Marks the caller's phase events after each kernel.
+// Steps 1-2 of a decode plan: the streaming scorer (sigma rows in the workspace) and one top-K
+// CTA per row.  Marks the caller's phase events after each kernel.
 cudaError_t launch_decode_select(const Plan& P, const void* q_cal, const void* k_lm,
                                  const float* b_lm, int32_t* idx, float* s_sel, char* ws,
                                  cudaStream_t st, PhaseMarks& pm) {
   cudaError_t e;
-  if (P.split_select) {
-    float* pv = reinterpret_cast<float*>(ws + P.off_pv);
-    int32_t* pc = reinterpret_cast<int32_t*>(ws + P.off_pc);
-    e = launch_select_split(P.D, P.bf16, P.cps, P.n_split, q_cal, k_lm, b_lm, pv, pc, st);
-    pm.mark();
-    if (e == cudaSuccess)
-      e = launch_select_merge(P.D, P.bf16, P.n_split, pv, pc, q_cal, k_lm, b_lm, idx, s_sel, st);
-    pm.mark();
-    return e;
-  }
   float* sig = reinterpret_cast<float*>(ws + P.off_sig);
   e = P.tc_stream ? launch_select_stream_tc(P.D, q_cal, k_lm, b_lm, sig, P.n_stride,
                                             reinterpret_cast<int32_t*>(ws), st)
