@@ -36,6 +36,7 @@ struct Plan {
   bool decode = false;
   bool tc_select = false;
   bool tc_select_t = false;   // the landmark-major scoring kernel (G = 2, 4, 8)
+  bool attn_ext = false;      // the tensor-core attention reads per-head scores from s_sel
   bool tc_attn = false;
   bool tc_stream = false;
   bool tc_units = false;
@@ -84,6 +85,7 @@ Plan make_plan(const hils_params* p) {
   P.tc_select = !P.decode && rows32 && score_tc_supported(D, P.bf16);
   P.tc_select_t = P.tc_select && score_t_tc_supported(D, P.bf16);
   P.tc_attn = !P.decode && rows32 && attn_tc_supported(D, P.bf16);
+  P.attn_ext = P.tc_attn && attn_tc_external_scores(D);
   P.tc_stream = P.decode && stream_tc_supported(D, P.bf16);
   P.tc_units = P.decode && units_tc_supported(D, P.bf16);
 
@@ -94,7 +96,7 @@ Plan make_plan(const hils_params* p) {
   // per-head scores of the selected chunks: the tensor-core attention takes them from the
   // scoring kernel when a KV group has one head (sel_rows = head_rows) and otherwise scores the
   // selected chunks itself
-  if (!P.tc_attn || !P.tc_select || D.G == 1) {
+  if (!P.tc_attn || !P.tc_select || P.attn_ext) {
     P.off_ssel = off;
     off = align_up(off + head_rows * (size_t)D.K * sizeof(float));
   }
@@ -178,7 +180,7 @@ int phase_names(const Plan& P, const char** names, int max_names) {
   }
   if (P.tc_select) {
     pre[n++] = P.tc_select_t ? "score_topk_t_tc" : "score_topk_tc";
-    if (!P.tc_attn) pre[n++] = "select_scores";
+    if (!P.tc_attn || (P.attn_ext && P.D.G > 1)) pre[n++] = "select_scores";
   } else {
     pre[n++] = "select_rows";
   }
@@ -257,8 +259,9 @@ hils_status forward_impl(const hils_params* p, const void* q, const void* q_cal,
       e = launch_prefill_select_tc(P, q_cal, k_lm, b_lm, idx,
                                P.tc_attn && P.D.G == 1 ? s_sel : nullptr,
                                reinterpret_cast<int32_t*>(ws), st);
-      // the tensor-core attention takes the scores from there, or scores per head itself
-      if (e == cudaSuccess && !P.tc_attn) {
+      // the tensor-core attention takes the scores from there (one head per group), from the
+      // per-head scores of the winners (two attention CTAs per SM), or scores per head itself
+      if (e == cudaSuccess && (!P.tc_attn || (P.attn_ext && P.D.G > 1))) {
         pm.mark();
         e = launch_select_scores(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
       }

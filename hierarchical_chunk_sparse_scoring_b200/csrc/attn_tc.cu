@@ -27,6 +27,8 @@
 // (classification, softmax, the row's P as bf16 into its own TMEM lane).
 #include <cudaTypedefs.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -43,7 +45,12 @@ constexpr uint32_t kAtPollLimit = 1u << 24;
 constexpr float kRescaleMargin = 8.0f;       // natural-log units
 constexpr int kAtSmemLimit = 227 * 1024;
 
-template <int DD, int G>
+// TWO = 1: d = 128 with two CTAs per SM.  The per-head scores of the selected chunks come from
+// the selection step (no calibrated-query tile, no landmark product here), P is written into its
+// own S columns of TMEM (256 columns per CTA), the K/V ring has two stages and the tile bitmap is
+// built in the second of them; a CTA then needs under half of the SM's shared memory, so two
+// CTAs share each SM and one's softmax and prologue latencies hide behind the other's work.
+template <int DD, int G, int TWO = 0>
 struct AtShape {
   static constexpr int TQ = kAtRows / G;                 // queries per CTA
   static constexpr int KB = DD / 64;
@@ -57,26 +64,32 @@ struct AtShape {
   // K/V ring: STAGES_MAIN stage pairs of their own, plus one that reuses the calibrated-query
   // tile once the selected chunks' scores have been taken from it (same size: Q_BYTES = 2 KV)
   // d = 64: two CTAs per SM (each one's prologue and softmax latency hide behind the other's)
-  static constexpr int STAGES_MAIN = DD == 128 ? 3 : 2;
-  static constexpr int STAGES = STAGES_MAIN + 1;
+  static constexpr int STAGES_MAIN = TWO ? 2 : (DD == 128 ? 3 : 2);
+  static constexpr int STAGES = TWO ? STAGES_MAIN : STAGES_MAIN + 1;
   static_assert(Q_BYTES == 2 * KV_BYTES, "the q_cal tile holds one K/V stage pair");
   static constexpr int KLM_ROWS = 64;                    // landmark rows staged in smem
   static constexpr int KLM_BYTES = KB * KLM_ROWS * 128;  // same swizzled layout as a K tile
-  static constexpr int FIXED = 2 * Q_BYTES /*q and q_cal*/ + STAGES_MAIN * 2 * KV_BYTES +
-                               2 * P_BYTES + 1024 /*bars*/ + 1024 /*align*/ + 1024 /*scan*/;
+  static constexpr int FIXED =
+      TWO ? Q_BYTES + STAGES_MAIN * 2 * KV_BYTES + 256 /*bars*/ + 1024 /*align*/ + 64 /*scan*/
+          : 2 * Q_BYTES /*q and q_cal*/ + STAGES_MAIN * 2 * KV_BYTES + 2 * P_BYTES +
+                1024 /*bars*/ + 1024 /*align*/ + 1024 /*scan*/;
   static_assert(KLM_BYTES <= 2 * P_BYTES, "landmark rows fit the prologue scratch");
   // TMEM: S[2] (2 x 64 columns), O (DD), the landmark scores (64); a power of two.  Once the
   // landmark scores are read, their columns hold P[2]: 64 bf16 per row, two per column, the A
   // operand of the P V product.
   static constexpr uint32_t O_COL = 128;
   static constexpr uint32_t LM_COL = O_COL + DD;
-  static constexpr uint32_t P_COL = LM_COL;
-  static constexpr uint32_t TMEM_COLS = LM_COL + 64 <= 256 ? 256 : 512;
-  static_assert(P_COL + 2 * (kTile / 2) <= TMEM_COLS, "P buffers in TMEM");
-  // co-resident CTAs never exceed the SM's 512 TMEM columns: d = 64 runs two CTAs per SM on 256
-  // columns each; d = 128 needs 512 and its shared memory footprint keeps a second CTA away
-  static_assert(DD == 64 ? (TMEM_COLS == 256 && FIXED < 232448 / 2 - 8192)
-                         : FIXED > 232448 / 2, "CTAs per SM");
+  // P[x]: its own columns after the landmark scores, or (TWO) the first half of S[x]
+  static constexpr uint32_t P_COL = TWO ? 0 : LM_COL;
+  static constexpr uint32_t P_STRIDE = TWO ? kTile : kTile / 2;   // columns between P[0], P[1]
+  static constexpr uint32_t TMEM_COLS = TWO ? 256 : (LM_COL + 64 <= 256 ? 256 : 512);
+  static_assert(P_COL + P_STRIDE + kTile / 2 <= TMEM_COLS, "P buffers in TMEM");
+  static_assert(!TWO || O_COL + DD <= TMEM_COLS, "S and O in 256 columns");
+  // co-resident CTAs never exceed the SM's 512 TMEM columns: d = 64 and TWO run two CTAs per SM
+  // on 256 columns each; otherwise d = 128 needs 512 and its shared memory footprint keeps a
+  // second CTA away
+  static_assert(DD == 64 || TWO ? TMEM_COLS == 256 : FIXED > 232448 / 2, "CTAs per SM");
+  static_assert(DD == 64 ? FIXED < 232448 / 2 - 8192 : true, "d = 64: two CTAs per SM");
 };
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -162,8 +175,8 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 
 }  // namespace
 
-template <int DD, int G, int KM, int RS>
-__global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
+template <int DD, int G, int KM, int RS, int TWO>
+__global__ void __launch_bounds__(kAtThreads, ((DD == 64 && KM <= 16) || TWO) ? 2 : 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmQc,
                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -171,18 +184,19 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
                    const __nv_bfloat16* __restrict__ klm, const float* __restrict__ blm,
                    __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out,
                    int list_cap, int bitmap_words, int32_t* __restrict__ status) {
-  using SH = AtShape<DD, G>;
+  using SH = AtShape<DD, G, TWO>;
   constexpr int TQ = SH::TQ;
+  static_assert(!TWO || (DD == 128 && KM <= 16), "two CTAs per SM: d = 128, K <= 16");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem;
   // calibrated queries (G > 1: the per-head scores of the selection; with G = 1 this tile is
-  // never loaded and serves only as a K/V stage)
+  // never loaded and serves only as a K/V stage; absent with TWO)
   uint8_t* sQc = sQ + SH::Q_BYTES;
-  uint8_t* sK = sQc + SH::Q_BYTES;
+  uint8_t* sK = TWO ? sQc : sQc + SH::Q_BYTES;
   uint8_t* sV = sK + SH::STAGES_MAIN * SH::KV_BYTES;
-  uint8_t* sP = sV + SH::STAGES_MAIN * SH::KV_BYTES;
+  uint8_t* sP = sV + SH::STAGES_MAIN * SH::KV_BYTES;   // (TWO: only the barriers follow)
   // stage s of the K/V ring (the last one lives in the q_cal tile)
   auto stage_k = [&](int s) -> uint8_t* {
     return s < SH::STAGES_MAIN ? sK + s * SH::KV_BYTES : sQc;
@@ -193,7 +207,7 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
   // landmark rows of the first 64 tiles (K-tile layout) in the prologue scratch; dead once their
   // product has completed
   uint8_t* sKlm = sP;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * SH::P_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(TWO ? sP : sP + 2 * SH::P_BYTES);
   uint64_t* kv_full = bars;                       // [STAGES]
   uint64_t* kv_empty = bars + SH::STAGES;         // [STAGES]
   uint64_t* q_full = bars + 2 * SH::STAGES;
@@ -205,17 +219,21 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
   uint64_t* o_final = o_done + 1;
   uint64_t* lm_done = o_final + 1;
   uint64_t* qc_free = lm_done + 1;   // every softmax warp is done reading the q_cal tile
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qc_free + 1);
-  int* n_tiles_sh = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + 1024);
-  int* tiles = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + 2048);  // [list_cap]
+  uint64_t* bm_free = qc_free + 1;   // (TWO) every row has read the bitmap in K/V stage 1
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bm_free + 1);
+  int* n_tiles_sh = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + (TWO ? 256 : 1024));
+  int* tiles = TWO ? n_tiles_sh + 16
+                   : reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(bars) + 2048);  // [cap]
   // the tile bitmap of the union and the list position of each of its words live in the
-  // prologue scratch (up to 2 x 16 KB): they are read for the last time by the rows' ranking,
-  // before the landmark rows are staged there
-  uint32_t* bitmap = reinterpret_cast<uint32_t*>(sP);                          // [words]
-  int* wpre = reinterpret_cast<int*>(sP + SH::P_BYTES);        // list position of each word
+  // prologue scratch (up to 2 x 16 KB; TWO: K/V stage 1): they are read for the last time by the
+  // rows' ranking, before the landmark rows (or the stage's tiles) land there
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(TWO ? sK + SH::KV_BYTES : sP);   // [words]
+  int* wpre = reinterpret_cast<int*>(TWO ? sV + SH::KV_BYTES : sP + SH::P_BYTES);
   // per row, its selected chunks in tile-list order: (tile index, surrogate score) [128][KM]
+  // (TWO: tile indices as 16-bit integers)
   constexpr bool kSelSmem = KM <= 16;
-  int* sel_t = tiles + list_cap;
+  using SelT = typename std::conditional<TWO != 0, int16_t, int>::type;
+  SelT* sel_t = reinterpret_cast<SelT*>(tiles + list_cap);
   float* sel_u = reinterpret_cast<float*>(sel_t + (kSelSmem ? kAtRows * KM : 0));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -239,7 +257,7 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
   // With one head per KV group the row's surrogate score of a selected chunk is the score the
   // selection ranked it by (s_sig); with several, each head's own score comes from a landmark
   // product below.
-  constexpr bool kOwnScores = G > 1;
+  constexpr bool kOwnScores = G > 1 && !TWO;
   // the row's selected chunks go out first: they feed both the tile list and the row's scores
   int sc[KM];
   float su[KM];
@@ -247,7 +265,8 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
   for (int k = 0; k < KM; ++k) {
     const bool has = is_row && valid && k < K;
     sc[k] = has ? __ldg(idx + (bg * D.N_q + i) * K + k) : -1;
-    if constexpr (!kOwnScores) su[k] = has ? __ldg(s_sig + (bg * D.N_q + i) * K + k) : -INFINITY;
+    if constexpr (!kOwnScores)
+      su[k] = has ? __ldg(s_sig + (((b * D.Hq + g * G + h) * D.N_q + i) * K + k)) : -INFINITY;
   }
 
   // ---------------------------------------------------------------- barriers, TMEM, tile list
@@ -264,6 +283,7 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
     mbar_init(o_final, 1);
     mbar_init(lm_done, 1);
     mbar_init(qc_free, 4);
+    mbar_init(bm_free, 4);
     fence_barrier_init();
   }
   if (warp == 1) tmem_alloc(tmem_holder, SH::TMEM_COLS);
@@ -363,11 +383,14 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
       prefetch_tensormap(&tmV);
       int last_s = -1;
       uint32_t last_par = 0;
-      for (int t = 0; t < n_tiles; ++t) {
+      // (TWO: K/V stage 1 holds the bitmap until every row has ranked its chunks)
+      bool go = !TWO || mbar_wait(bm_free, 0, kAtPollLimit);
+      if (!go) record_status(status, kStatusTimeout);
+      for (int t = 0; go && t < n_tiles; ++t) {
         const int s = t % SH::STAGES;
         const uint32_t u = (uint32_t)(t / SH::STAGES);
         if (!mbar_wait(&kv_empty[s], (u & 1u) ^ 1u, kAtPollLimit) ||
-            (t == SH::STAGES_MAIN && !mbar_wait(qc_free, 0, kAtPollLimit))) {
+            (!TWO && t == SH::STAGES_MAIN && !mbar_wait(qc_free, 0, kAtPollLimit))) {
           record_status(status, kStatusTimeout);
           break;
         }
@@ -395,6 +418,9 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
         const uint32_t u = (uint32_t)(t / SH::STAGES), v = (uint32_t)(t >> 1);
         if (!mbar_wait(&kv_full[s], u & 1u, kAtPollLimit)) return false;
         if (!mbar_wait(&s_empty[x], (v & 1u) ^ 1u, kAtPollLimit)) return false;
+        // (TWO: P[x] lives in S[x]; the P V product of tile t-2 must have read it)
+        if (TWO && t >= 2 && !mbar_wait(&p_empty[x], (uint32_t)((t - 2) >> 1) & 1u, kAtPollLimit))
+          return false;
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < DD / 16; ++ks) {
@@ -417,7 +443,7 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
 #pragma unroll
         for (int ks = 0; ks < kTile / 16; ++ks) {
           // 16 tokens of P = 8 TMEM columns
-          const uint32_t at = tmem + SH::P_COL + (uint32_t)(x * (kTile / 2) + ks * 8);
+          const uint32_t at = tmem + SH::P_COL + (uint32_t)(x * SH::P_STRIDE + ks * 8);
           const uint64_t bd = desc_mnmajor_sw128(
               smem_u32(stage_v(s)) + ks * 16 * 128, SH::KV_BOX);
           mma_bf16_ts(tmem + SH::O_COL, at, bd, IDESC_PV, (t > 0 || ks > 0) ? 1u : 0u);
@@ -547,6 +573,11 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
       }
     } else {
       rank_chunks();
+      if constexpr (TWO) {
+        // the bitmap (in K/V stage 1) is read for the last time: the stage may fill
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bm_free);
+      }
 #pragma unroll
       for (int k = 0; k < KM; ++k) {
         if (rk[k] == INT_MAX) su[k] = -INFINITY;
@@ -559,7 +590,7 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
 #pragma unroll
       for (int k = 0; k < KM; ++k) {
         if (rk[k] == INT_MAX) continue;
-        sel_t[r * KM + at[k]] = rk[k];
+        sel_t[r * KM + at[k]] = (SelT)rk[k];
         sel_u[r * KM + at[k]] = su[k];
         ++n_sel;
       }
@@ -743,7 +774,7 @@ __global__ void __launch_bounds__(kAtThreads, (DD == 64 && KM <= 16) ? 2 : 1)
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(p[32 * hf + 2 * e], p[32 * hf + 2 * e + 1]);
-        tmem_st16u(lane_base + SH::P_COL + (uint32_t)(x * (kTile / 2) + 16 * hf), pk);
+        tmem_st16u(lane_base + SH::P_COL + (uint32_t)(x * SH::P_STRIDE + 16 * hf), pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -821,12 +852,22 @@ int list_capacity(const Dims& D, int TQ) {
   return TQ * D.K * (D.S / kTile) + (int)((D.W + D.S + TQ) / kTile) + 4;
 }
 
-template <int DD, int G, int KM, int RS>
+// shared memory of a CTA when two share an SM (each also reserves 1 KB of the SM's 228 KB)
+constexpr int kTwoCtaSmemLimit = (228 * 1024) / 2 - 1024;
+
+int64_t two_cta_smem(const Dims& D) {
+  const int TQ = kAtRows / D.G;
+  const int64_t cap = (int64_t)TQ * D.K * (D.S / kTile) + (D.W + D.S + TQ) / kTile + 4;
+  const int km = D.K <= 8 ? 8 : 16;
+  return AtShape<128, 1, 1>::FIXED + cap * 4 + (int64_t)kAtRows * km * 6;
+}
+
+template <int DD, int G, int KM, int RS, int TWO>
 cudaError_t launch_at_t(const Dims& D, const void* q, const void* qc, const void* K,
                         const void* V, const int32_t* idx, const float* s_sig, const void* klm,
                         const float* blm, void* out, float* lse, int32_t* status,
                         cudaStream_t st) {
-  using SH = AtShape<DD, G>;
+  using SH = AtShape<DD, G, TWO>;
   CUtensorMap tmQ, tmQc, tmK, tmV;
   if (!make_map_at(&tmQ, q, (uint64_t)(D.B * D.Hq * D.N_q), DD, SH::TQ) ||
       !make_map_at(&tmQc, qc, (uint64_t)(D.B * D.Hq * D.N_q), DD, SH::TQ) ||
@@ -835,10 +876,11 @@ cudaError_t launch_at_t(const Dims& D, const void* q, const void* qc, const void
     return cudaErrorInvalidValue;
   const int cap = list_capacity(D, SH::TQ);
   const int words = (int)((D.N_kv / kTile) / 32) + 2;
-  if (words * 4 > SH::P_BYTES) return cudaErrorInvalidConfiguration;
-  const int smem = SH::FIXED + 1024 + cap * 4 + (KM <= 16 ? kAtRows * KM * 8 : 0);
-  if (smem > kAtSmemLimit) return cudaErrorInvalidConfiguration;
-  auto kern = attn_tc_kernel<DD, G, KM, RS>;
+  if (words * 4 > (TWO ? SH::KV_BYTES : SH::P_BYTES)) return cudaErrorInvalidConfiguration;
+  const int smem = TWO ? SH::FIXED + cap * 4 + kAtRows * KM * 6
+                       : SH::FIXED + 1024 + cap * 4 + (KM <= 16 ? kAtRows * KM * 8 : 0);
+  if (smem > (TWO ? kTwoCtaSmemLimit : kAtSmemLimit)) return cudaErrorInvalidConfiguration;
+  auto kern = attn_tc_kernel<DD, G, KM, RS, TWO>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((D.N_q + SH::TQ - 1) / SH::TQ), (unsigned)(D.B * D.Hkv));
@@ -854,25 +896,49 @@ cudaError_t launch_at_k(const Dims& D, const void* q, const void* qc, const void
                         const float* blm, void* out, float* lse, int32_t* status,
                         cudaStream_t st) {
   if constexpr (DD == 128) {
+    if (attn_tc_two_cta(D)) {
+      if (D.S == 2 * kTile) {
+        if (D.K <= 8)
+          return launch_at_t<DD, G, 8, 1, 1>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse,
+                                             status, st);
+        return launch_at_t<DD, G, 16, 1, 1>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse,
+                                            status, st);
+      }
+      if (D.K <= 8)
+        return launch_at_t<DD, G, 8, 0, 1>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status,
+                                           st);
+      return launch_at_t<DD, G, 16, 0, 1>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status,
+                                          st);
+    }
     // chunks of 128 tokens (two tiles per chunk) are built for d = 128 only
     if (D.S == 2 * kTile) {
       if (D.K <= 8)
-        return launch_at_t<DD, G, 8, 1>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status,
+        return launch_at_t<DD, G, 8, 1, 0>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status,
                                         st);
       if (D.K <= 16)
-        return launch_at_t<DD, G, 16, 1>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status,
+        return launch_at_t<DD, G, 16, 1, 0>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status,
                                          st);
-      return launch_at_t<DD, G, 32, 1>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status, st);
+      return launch_at_t<DD, G, 32, 1, 0>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status, st);
     }
   }
   if (D.K <= 8)
-    return launch_at_t<DD, G, 8, 0>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status, st);
+    return launch_at_t<DD, G, 8, 0, 0>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status, st);
   if (D.K <= 16)
-    return launch_at_t<DD, G, 16, 0>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status, st);
-  return launch_at_t<DD, G, 32, 0>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status, st);
+    return launch_at_t<DD, G, 16, 0, 0>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status, st);
+  return launch_at_t<DD, G, 32, 0, 0>(D, q, qc, K, V, idx, s_sig, klm, blm, out, lse, status, st);
 }
 
 }  // namespace
+
+bool attn_tc_two_cta(const Dims& D) {
+  if (D.d != 128 || D.K > 16) return false;
+  if (D.S != kTile && D.S != 2 * kTile) return false;
+  if (D.G != 1 && D.G != 2 && D.G != 4 && D.G != 8) return false;
+  if ((D.N_kv / kTile) / 32 + 2 > AtShape<128, 1, 1>::KV_BYTES / 4) return false;
+  return two_cta_smem(D) <= kTwoCtaSmemLimit;
+}
+
+bool attn_tc_external_scores(const Dims& D) { return D.G == 1 || attn_tc_two_cta(D); }
 
 bool attn_tc_supported(const Dims& D, bool bf16) {
   if (!bf16 || D.K > kMaxK) return false;
@@ -890,7 +956,7 @@ bool attn_tc_supported(const Dims& D, bool bf16) {
   if (D.C >= (int64_t)INT32_MAX) return false;
   const int km = D.K <= 8 ? 8 : (D.K <= 16 ? 16 : 32);
   const int64_t sel_bytes = km <= 16 ? (int64_t)kAtRows * km * 8 : 0;
-  return fixed + 1024 + cap * 4 + sel_bytes <= kAtSmemLimit;
+  return attn_tc_two_cta(D) || fixed + 1024 + cap * 4 + sel_bytes <= kAtSmemLimit;
 }
 
 cudaError_t launch_attn_tc(const Dims& D, const void* q, const void* qc, const void* K,

@@ -29,8 +29,14 @@ cudaError_t launch_score_topk_t_tc(const Dims& D, const void* qc, const void* kl
                                    int32_t* status, cudaStream_t st);
 
 bool attn_tc_supported(const Dims& D, bool bf16);
-// s_sig: the scoring kernel's sigma of each selected chunk, required when D.G == 1 (it is then
-// the head's surrogate score); with G > 1 the kernel scores the selected chunks per head itself
+// d = 128 with K <= 16 where two attention CTAs fit one SM: the kernel then takes every head's
+// scores of the selected chunks from s_sig instead of scoring them itself
+bool attn_tc_two_cta(const Dims& D);
+// whether the attention kernel for D reads the per-head selected-chunk scores from s_sig
+bool attn_tc_external_scores(const Dims& D);
+// s_sig: per-head scores of the selected chunks [B, Hq, N_q, K], required when
+// attn_tc_external_scores(D) (with G == 1 the scoring kernel's sigma of the winners); otherwise
+// the kernel scores the selected chunks per head itself
 cudaError_t launch_attn_tc(const Dims& D, const void* q, const void* qc, const void* K,
                            const void* V, const int32_t* idx, const float* s_sig,
                            const void* klm, const float* blm, void* out, float* lse,
