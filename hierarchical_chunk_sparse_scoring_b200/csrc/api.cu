@@ -180,7 +180,7 @@ int phase_names(const Plan& P, const char** names, int max_names) {
   }
   if (P.tc_select) {
     pre[n++] = P.tc_select_t ? "score_topk_t_tc" : "score_topk_tc";
-    if (!P.tc_attn || (P.attn_ext && P.D.G > 1)) pre[n++] = "select_scores";
+    if (!P.tc_attn || (P.attn_ext && P.D.G > 1 && !P.tc_select_t)) pre[n++] = "select_scores";
   } else {
     pre[n++] = "select_rows";
   }
@@ -191,11 +191,15 @@ int phase_names(const Plan& P, const char** names, int max_names) {
 
 // Steps 1-2 of a prefill plan on the tensor cores: the landmark-major kernel where it applies,
 // else the query-major one.
+// s_head (nullable): every head's score of each selected chunk, written by the landmark-major
+// kernel itself; returns in *s_head_done whether it was.
 cudaError_t launch_prefill_select_tc(const Plan& P, const void* q_cal, const void* k_lm,
                                      const float* b_lm, int32_t* idx, float* s_out,
-                                     int32_t* status, cudaStream_t st) {
+                                     float* s_head, int32_t* status, cudaStream_t st,
+                                     bool* s_head_done) {
+  *s_head_done = P.tc_select_t && s_head;
   return P.tc_select_t
-             ? launch_score_topk_t_tc(P.D, q_cal, k_lm, b_lm, idx, s_out, status, st)
+             ? launch_score_topk_t_tc(P.D, q_cal, k_lm, b_lm, idx, s_out, s_head, status, st)
              : launch_score_topk_tc(P.D, q_cal, k_lm, b_lm, idx, s_out, status, st);
 }
 
@@ -256,12 +260,15 @@ hils_status forward_impl(const hils_params* p, const void* q, const void* q_cal,
     pm.mark();
   } else {
     if (P.tc_select) {
+      bool heads_done = false;
       e = launch_prefill_select_tc(P, q_cal, k_lm, b_lm, idx,
-                               P.tc_attn && P.D.G == 1 ? s_sel : nullptr,
-                               reinterpret_cast<int32_t*>(ws), st);
+                                   P.tc_attn && P.D.G == 1 ? s_sel : nullptr,
+                                   P.attn_ext && P.D.G > 1 ? s_sel : nullptr,
+                                   reinterpret_cast<int32_t*>(ws), st, &heads_done);
       // the tensor-core attention takes the scores from there (one head per group), from the
-      // per-head scores of the winners (two attention CTAs per SM), or scores per head itself
-      if (e == cudaSuccess && (!P.tc_attn || (P.attn_ext && P.D.G > 1))) {
+      // per-head scores of the winners (two attention CTAs per SM: the landmark-major scoring
+      // kernel writes them, else select_scores), or scores per head itself
+      if (e == cudaSuccess && !heads_done && (!P.tc_attn || (P.attn_ext && P.D.G > 1))) {
         pm.mark();
         e = launch_select_scores(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
       }
@@ -329,9 +336,11 @@ extern "C" hils_status hils_select(const hils_params* p, const void* q_cal, cons
     e = launch_decode_select(P, q_cal, k_lm, b_lm, idx, s_sel, ws, st, none);
   } else if (P.tc_select) {
     // with one head per KV group the scores the selection ranked by are the per-head scores
+    bool heads_done = false;
     e = launch_prefill_select_tc(P, q_cal, k_lm, b_lm, idx, P.D.G == 1 ? s_sel : nullptr,
-                             reinterpret_cast<int32_t*>(ws), st);
-    if (e == cudaSuccess && s_sel && P.D.G != 1)
+                                 P.D.G != 1 ? s_sel : nullptr, reinterpret_cast<int32_t*>(ws),
+                                 st, &heads_done);
+    if (e == cudaSuccess && s_sel && P.D.G != 1 && !heads_done)
       e = launch_select_scores(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
   } else {
     e = launch_select_rows(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
@@ -549,9 +558,11 @@ extern "C" hils_status hils_select_noalloc(const hils_params* p, const void* q_c
       e = launch_select_merge(P.D, P.bf16, P.n_split, pv, pc, q_cal, k_lm, b_lm, idx, s_sel, st);
   } else if (P.tc_select) {
     // with one head per KV group the scores the selection ranked by are the per-head scores
+    bool heads_done = false;
     e = launch_prefill_select_tc(P, q_cal, k_lm, b_lm, idx, P.D.G == 1 ? s_sel : nullptr,
-                             reinterpret_cast<int32_t*>(ws), st);
-    if (e == cudaSuccess && s_sel && P.D.G != 1)
+                                 P.D.G != 1 ? s_sel : nullptr, reinterpret_cast<int32_t*>(ws),
+                                 st, &heads_done);
+    if (e == cudaSuccess && s_sel && P.D.G != 1 && !heads_done)
       e = launch_select_scores(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);
   } else {
     e = launch_select_rows(P.D, P.bf16, q_cal, k_lm, b_lm, idx, s_sel, st);

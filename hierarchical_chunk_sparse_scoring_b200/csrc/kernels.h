@@ -22,11 +22,12 @@ cudaError_t launch_score_topk_tc(const Dims& D, const void* qc, const void* klm,
                                  const float* blm, int32_t* idx, float* s_out, int32_t* status,
                                  cudaStream_t st);
 
-// landmark-major variant (landmark rows as the MMA's M, all G heads of a block as its N)
+// landmark-major variant (landmark rows as the MMA's M, all G heads of a block as its N);
+// s_head (nullable): every head's score of each selected chunk, [B, Hq, N_q, K]
 bool score_t_tc_supported(const Dims& D, bool bf16);
 cudaError_t launch_score_topk_t_tc(const Dims& D, const void* qc, const void* klm,
                                    const float* blm, int32_t* idx, float* s_out,
-                                   int32_t* status, cudaStream_t st);
+                                   float* s_head, int32_t* status, cudaStream_t st);
 
 bool attn_tc_supported(const Dims& D, bool bf16);
 // d = 128 with K <= 16 where two attention CTAs fit one SM: the kernel then takes every head's

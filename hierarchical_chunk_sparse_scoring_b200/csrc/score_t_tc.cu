@@ -93,7 +93,8 @@ __global__ void __launch_bounds__(TtShape<DD, G, KM>::THREADS, 1)
     score_t_tc_kernel(const __grid_constant__ CUtensorMap tmQc,
                       const __grid_constant__ CUtensorMap tmKlm, Dims D,
                       const float* __restrict__ blm, int32_t* __restrict__ idx,
-                      float* __restrict__ s_out, int32_t* __restrict__ status) {
+                      float* __restrict__ s_out, float* __restrict__ s_head,
+                      const __nv_bfloat16* __restrict__ klm, int32_t* __restrict__ status) {
   using SH = TtShape<DD, G, KM>;
   constexpr int MQ = SH::MQ, QH = SH::QH, TPQ = SH::TPQ, RM = SH::RM, LD = SH::LD;
   constexpr int CAP0 = SH::CAP0, LIST0 = SH::LIST0;
@@ -491,7 +492,12 @@ __global__ void __launch_bounds__(TtShape<DD, G, KM>::THREADS, 1)
       }
     }
     if (!ok) record_status(status, kStatusTimeout);
-    // outputs: best first (sigma desc, c asc), -1 / -inf padded
+    // outputs: best first (sigma desc, c asc), -1 / -inf padded; the chunk ids also go to
+    // shared memory (the first dump, free now) for the per-head scores below
+    int* fin = reinterpret_cast<int*>(dump);   // [MQ][K]
+#pragma unroll
+    for (int k = 0; k < KM; ++k)
+      if (k >= KM - K) fin[q * K + k - (KM - K)] = L.c[k] == INT_MAX ? -1 : L.c[k];
     if (q < nqv) {
       const int64_t i = i0 + q;
       int32_t* out = idx + (bg * D.N_q + i) * K - (KM - K);
@@ -503,6 +509,50 @@ __global__ void __launch_bounds__(TtShape<DD, G, KM>::THREADS, 1)
           if (so) so[k] = (L.c[k] == INT_MAX || L.v[k] <= -FLT_MAX) ? -INFINITY : L.v[k];
         }
       }
+    }
+  }
+  if (s_head) {
+    // every head's surrogate score of each selected chunk, q_cal[h] . k_lm[c] * scale + b_lm[c],
+    // from the block's calibrated queries still in shared memory (the attention step reads them
+    // instead of scoring the chunks again): one thread per (query, slot)
+    __syncthreads();
+    const int* fin = reinterpret_cast<const int*>(dump);
+    const bool have_q = n_tiles > 0 && mbar_wait(b_full, 0, kTtPollLimit);
+    for (int pq = threadIdx.x; pq < nqv * K; pq += SH::THREADS) {
+      const int q = pq / K, k = pq - q * K;
+      const int c = have_q ? fin[q * K + k] : -1;
+      float acc[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) acc[h] = 0.f;
+      if (c >= 0) {
+        const uint4* kr = reinterpret_cast<const uint4*>(klm + (bg * D.C + c) * DD);
+#pragma unroll 4
+        for (int u = 0; u < DD / 8; ++u) {   // 16-byte units of the landmark row
+          const uint4 kv = __ldg(kr + u);
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const int row = h * MQ + q;   // the (head, query) row of the B operand
+            const uint4 qv = *reinterpret_cast<const uint4*>(
+                sB + (u >> 3) * SH::B_BOX + (row >> 3) * 1024 + (row & 7) * 128 +
+                (((u & 7) ^ (row & 7)) << 4));
+            float a = acc[h];
+            a = fmaf(bf16_lo(qv.x), bf16_lo(kv.x), a);
+            a = fmaf(bf16_hi(qv.x), bf16_hi(kv.x), a);
+            a = fmaf(bf16_lo(qv.y), bf16_lo(kv.y), a);
+            a = fmaf(bf16_hi(qv.y), bf16_hi(kv.y), a);
+            a = fmaf(bf16_lo(qv.z), bf16_lo(kv.z), a);
+            a = fmaf(bf16_hi(qv.z), bf16_hi(kv.z), a);
+            a = fmaf(bf16_lo(qv.w), bf16_lo(kv.w), a);
+            a = fmaf(bf16_hi(qv.w), bf16_hi(kv.w), a);
+            acc[h] = a;
+          }
+        }
+      }
+      const float bias = c >= 0 ? __ldg(blm + bg * D.C + c) : 0.f;
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+        s_head[((b * D.Hq + g * G + h) * D.N_q + i0 + q) * K + k] =
+            c >= 0 ? fmaf(acc[h], D.scale, bias) : -INFINITY;
     }
   }
   tc_fence_before();
@@ -545,7 +595,8 @@ bool make_map_t(CUtensorMap* map, const void* base, uint64_t rows, uint64_t d,
 
 template <int DD, int G, int KM>
 cudaError_t launch_t(const Dims& D, const void* qc, const void* klm, const float* blm,
-                     int32_t* idx, float* s_out, int32_t* status, cudaStream_t st) {
+                     int32_t* idx, float* s_out, float* s_head, int32_t* status,
+                     cudaStream_t st) {
   using SH = TtShape<DD, G, KM>;
   CUtensorMap tmQc, tmKlm;
   if (!make_map_t(&tmQc, qc, (uint64_t)(D.B * D.Hq * D.N_q), DD, SH::MQ) ||
@@ -556,15 +607,17 @@ cudaError_t launch_t(const Dims& D, const void* qc, const void* klm, const float
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SH::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((D.N_q + SH::MQ - 1) / SH::MQ), (unsigned)(D.B * D.Hkv));
-  kern<<<grid, SH::THREADS, SH::SMEM, st>>>(tmQc, tmKlm, D, blm, idx, s_out, status);
+  kern<<<grid, SH::THREADS, SH::SMEM, st>>>(tmQc, tmKlm, D, blm, idx, s_out, s_head,
+                                            (const __nv_bfloat16*)klm, status);
   return cudaGetLastError();
 }
 
 template <int DD, int G>
 cudaError_t launch_t_k(const Dims& D, const void* qc, const void* klm, const float* blm,
-                       int32_t* idx, float* s_out, int32_t* status, cudaStream_t st) {
-  if (D.K <= 16) return launch_t<DD, G, 16>(D, qc, klm, blm, idx, s_out, status, st);
-  return launch_t<DD, G, 32>(D, qc, klm, blm, idx, s_out, status, st);
+                       int32_t* idx, float* s_out, float* s_head, int32_t* status,
+                       cudaStream_t st) {
+  if (D.K <= 16) return launch_t<DD, G, 16>(D, qc, klm, blm, idx, s_out, s_head, status, st);
+  return launch_t<DD, G, 32>(D, qc, klm, blm, idx, s_out, s_head, status, st);
 }
 
 }  // namespace
@@ -583,14 +636,14 @@ bool score_t_tc_supported(const Dims& D, bool bf16) {
 
 cudaError_t launch_score_topk_t_tc(const Dims& D, const void* qc, const void* klm,
                                    const float* blm, int32_t* idx, float* s_out,
-                                   int32_t* status, cudaStream_t st) {
+                                   float* s_head, int32_t* status, cudaStream_t st) {
   if (D.B * D.Hkv * D.N_q == 0) return cudaSuccess;
   if (D.d == 128) {
-    if (D.G == 4) return launch_t_k<128, 4>(D, qc, klm, blm, idx, s_out, status, st);
-    return launch_t_k<128, 8>(D, qc, klm, blm, idx, s_out, status, st);
+    if (D.G == 4) return launch_t_k<128, 4>(D, qc, klm, blm, idx, s_out, s_head, status, st);
+    return launch_t_k<128, 8>(D, qc, klm, blm, idx, s_out, s_head, status, st);
   }
-  if (D.G == 4) return launch_t_k<64, 4>(D, qc, klm, blm, idx, s_out, status, st);
-  return launch_t_k<64, 8>(D, qc, klm, blm, idx, s_out, status, st);
+  if (D.G == 4) return launch_t_k<64, 4>(D, qc, klm, blm, idx, s_out, s_head, status, st);
+  return launch_t_k<64, 8>(D, qc, klm, blm, idx, s_out, s_head, status, st);
 }
 
 }  // namespace hils

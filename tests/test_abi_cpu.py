@@ -71,12 +71,19 @@ def test_workspace_size(lib):
 def test_prefill_workspace_layout(lib):
     # status word, then idx [B, Hkv, N_q, K]; per-head scores [B, Hq, N_q, K] only where the
     # tensor-core attention does not score the selected chunks itself: one head per KV group
-    # (it takes the scoring kernel's sigma of the winners) or no tensor-core path (fp32)
+    # (it takes the scoring kernel's sigma of the winners), the d = 128, K <= 16 attention that
+    # runs two CTAs per SM (it takes every head's scores from the selection step), or no
+    # tensor-core path (fp32)
     def rup(x):
         return (x + 255) // 256 * 256
     nq, k = 4096, 16
     gqa = hb.workspace_size(_params(Hq=8, Hkv=2, N_q=nq, N_kv=nq, K_top=k))
-    assert gqa == 256 + rup(2 * nq * k * 4)
+    assert gqa == 256 + rup(2 * nq * k * 4) + rup(8 * nq * k * 4)
+    # (K = 32 at d = 128: the attention CTA scores the selected chunks per head itself)
+    gqa32 = hb.workspace_size(_params(Hq=8, Hkv=2, N_q=nq, N_kv=nq, K_top=32))
+    assert gqa32 == 256 + rup(2 * nq * 32 * 4)
+    gqa64 = hb.workspace_size(_params(Hq=8, Hkv=2, N_q=nq, N_kv=nq, K_top=k, d=64))
+    assert gqa64 == 256 + rup(2 * nq * k * 4)
     mha = hb.workspace_size(_params(Hq=8, Hkv=8, N_q=nq, N_kv=nq, K_top=k))
     assert mha == 256 + rup(8 * nq * k * 4) + rup(8 * nq * k * 4)
     f32 = hb.workspace_size(_params(Hq=8, Hkv=2, N_q=nq, N_kv=nq, K_top=k, dtype=torch.float32))

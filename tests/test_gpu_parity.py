@@ -143,6 +143,8 @@ def test_selection_is_deterministic():
 
 
 @pytest.mark.parametrize("name,kw", [("gqa7b_prefill", dict(N=4096)),
+                                     # landmark-major scoring: per-head scores from its epilogue
+                                     ("extreme", dict(N=16384)),
                                      ("small_mha_bf16", dict(B=1, Hq=4, Hkv=4, N=2048)),
                                      ("long_decode", dict(B=3, N=40000)),
                                      ("tiny_fp32", {})])
