@@ -83,9 +83,15 @@ Plan make_plan(const hils_params* p) {
                       D.B * D.Hkv * D.N_kv < (int64_t)INT32_MAX &&
                       D.B * D.Hkv * D.C < (int64_t)INT32_MAX;
   P.tc_select = !P.decode && rows32 && score_tc_supported(D, P.bf16);
-  P.tc_select_t = P.tc_select && score_t_tc_supported(D, P.bf16);
   P.tc_attn = !P.decode && rows32 && attn_tc_supported(D, P.bf16);
   P.attn_ext = P.tc_attn && attn_tc_external_scores(D);
+  // the landmark-major scoring kernel: always for eight heads; for four, on long sequences
+  // (8192 chunks and more) or when its per-head scores of the winners feed the two-CTA
+  // attention.  Short four-head blocks alone favour the query-major kernel, whose blocks of 128
+  // queries amortise the per-block start-up better (7B-like prefill scoring: 2.29 ms against
+  // 2.91 ms), but that kernel leaves the per-head scores to a separate launch (2.5 ms there).
+  P.tc_select_t = P.tc_select && score_t_tc_supported(D, P.bf16) &&
+                  (D.G == 8 || D.C >= 8192 || (P.tc_attn && attn_tc_two_cta(D)));
   P.tc_stream = P.decode && stream_tc_supported(D, P.bf16);
   P.tc_units = P.decode && units_tc_supported(D, P.bf16);
 

@@ -81,12 +81,107 @@ struct TtShape {
   static_assert(32 % TPQ == 0 && MQ * TPQ == kTtCmp, "stripe threads");
   static_assert(TPQ * RM >= KM, "witnesses");
   static_assert(CAP0 >= KM, "rank buffer");
+  static_assert(MQ * KM * 4 <= A_STAGE, "final chunk ids in one ring stage");
 };
 
 // Parity of the wait for the u-th completion of a barrier phase sequence.
 __device__ __forceinline__ uint32_t par(int u) { return (uint32_t)u & 1u; }
 
 }  // namespace
+
+// m16n8k16 bf16 MMA with fp32 accumulation (the legacy warp-level form: the per-head scores of a
+// block's winners are a few hundred such products, a gather per query, not a streamed GEMM).
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Every head's surrogate score of each selected chunk, q_cal[h] . k_lm[c] * scale + b_lm[c]
+// (-inf for an empty slot), from the block's calibrated queries still in shared memory, so the
+// attention step need not score the chunks again.  A job is one query and 16 of its list slots:
+// one warp takes a 16 (slots) x 8 (heads) x d product on the tensor cores, A = the slots'
+// landmark rows gathered from global memory, B = the query's G head rows of the q_cal tile
+// (heads past G are zero).  A dot product does not depend on the order of its terms, so each
+// lane loads whole 16-byte pieces and the fragment's k positions are assigned to dims in the
+// order the pieces arrive: lane (r, c) = (lane / 4, lane % 4) holds dims 32m + 8c .. 32m + 8c + 7
+// of rows r and r + 8 of A and of column r of B, the first half of them for the MMA of k step 2m
+// and the second half for step 2m + 1, the same assignment on both operands.  The block waits
+// for this at its end, so the gathers of JB jobs per warp are issued together (one memory
+// latency per JB jobs rather than two per job).
+template <int DD, int G, int KM>
+__device__ __noinline__ void head_scores(const Dims& D, const int* __restrict__ fin,
+                                         const uint8_t* sB, bool have_q, int64_t b, int64_t g,
+                                         int64_t bg, int64_t i0, int nqv,
+                                         const __nv_bfloat16* __restrict__ klm,
+                                         const float* __restrict__ blm,
+                                         float* __restrict__ s_head) {
+  using SH = TtShape<DD, G, KM>;
+  constexpr int MQ = SH::MQ, NW = SH::THREADS / 32;
+  constexpr int MS = DD / 32;   // 32-dim segments of a row
+  constexpr int JB = 3;         // jobs of a warp in flight together
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = lane >> 2, c = lane & 3;
+  const int K = D.K;
+  const int n_t16 = (K + 15) / 16;
+  const int n_jobs = nqv * n_t16;
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  for (int base = warp; base < n_jobs; base += NW * JB) {
+    uint4 A0[JB][MS], A1[JB][MS];
+    int ca[JB], cb[JB];
+    float ba[JB], bb[JB];
+#pragma unroll
+    for (int jj = 0; jj < JB; ++jj) {
+      const int job = base + jj * NW;
+      const int q = job / n_t16, k0 = (job - q * n_t16) * 16;
+      const int ka = k0 + r, kb = ka + 8;
+      ca[jj] = job < n_jobs && ka < K ? fin[q * K + ka] : -1;
+      cb[jj] = job < n_jobs && kb < K ? fin[q * K + kb] : -1;
+      const uint4* ra = reinterpret_cast<const uint4*>(klm + (bg * D.C + max(ca[jj], 0)) * DD);
+      const uint4* rb = reinterpret_cast<const uint4*>(klm + (bg * D.C + max(cb[jj], 0)) * DD);
+#pragma unroll
+      for (int m = 0; m < MS; ++m) {
+        A0[jj][m] = have_q && ca[jj] >= 0 ? __ldg(ra + m * 4 + c) : z;
+        A1[jj][m] = have_q && cb[jj] >= 0 ? __ldg(rb + m * 4 + c) : z;
+      }
+      ba[jj] = ca[jj] >= 0 ? __ldg(blm + bg * D.C + ca[jj]) : 0.f;
+      bb[jj] = cb[jj] >= 0 ? __ldg(blm + bg * D.C + cb[jj]) : 0.f;
+    }
+#pragma unroll
+    for (int jj = 0; jj < JB; ++jj) {
+      const int job = base + jj * NW;
+      if (job >= n_jobs) break;   // (warp-uniform)
+      const int q = job / n_t16, k0 = (job - q * n_t16) * 16;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const int row = r * MQ + q;   // column r of B: head r's row of the q_cal tile
+#pragma unroll
+      for (int m = 0; m < MS; ++m) {
+        const int u = m * 4 + c;    // 16-byte piece of the row
+        const uint4 bq = have_q && r < G
+                             ? *reinterpret_cast<const uint4*>(
+                                   sB + (u >> 3) * SH::B_BOX + (row >> 3) * 1024 +
+                                   (row & 7) * 128 + (((u & 7) ^ (row & 7)) << 4))
+                             : z;
+        mma_16816(acc, A0[jj][m].x, A1[jj][m].x, A0[jj][m].y, A1[jj][m].y, bq.x, bq.y);
+        mma_16816(acc, A0[jj][m].z, A1[jj][m].z, A0[jj][m].w, A1[jj][m].w, bq.z, bq.w);
+      }
+      // acc: (slot ka, head 2c), (ka, 2c + 1), (kb, 2c), (kb, 2c + 1)
+      const int64_t i = i0 + q;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int h = 2 * c + (e & 1);
+        const int k = k0 + r + (e < 2 ? 0 : 8);
+        const int ch = e < 2 ? ca[jj] : cb[jj];
+        if (h < G && k < K)
+          s_head[((b * D.Hq + g * G + h) * D.N_q + i) * K + k] =
+              ch >= 0 ? fmaf(acc[e], D.scale, e < 2 ? ba[jj] : bb[jj]) : -INFINITY;
+      }
+    }
+  }
+}
 
 template <int DD, int G, int KM>
 __global__ void __launch_bounds__(TtShape<DD, G, KM>::THREADS, 1)
@@ -493,8 +588,10 @@ __global__ void __launch_bounds__(TtShape<DD, G, KM>::THREADS, 1)
     }
     if (!ok) record_status(status, kStatusTimeout);
     // outputs: best first (sigma desc, c asc), -1 / -inf padded; the chunk ids also go to
-    // shared memory (the first dump, free now) for the per-head scores below
-    int* fin = reinterpret_cast<int*>(dump);   // [MQ][K]
+    // shared memory for the per-head scores below, into the landmark ring: every tile's MMAs
+    // have completed once a merge warp is past the last tile (the dumps are not free yet: with
+    // two merge warps the other may still be reading one)
+    int* fin = reinterpret_cast<int*>(sA);   // [MQ][K]
 #pragma unroll
     for (int k = 0; k < KM; ++k)
       if (k >= KM - K) fin[q * K + k - (KM - K)] = L.c[k] == INT_MAX ? -1 : L.c[k];
@@ -512,48 +609,10 @@ __global__ void __launch_bounds__(TtShape<DD, G, KM>::THREADS, 1)
     }
   }
   if (s_head) {
-    // every head's surrogate score of each selected chunk, q_cal[h] . k_lm[c] * scale + b_lm[c],
-    // from the block's calibrated queries still in shared memory (the attention step reads them
-    // instead of scoring the chunks again): one thread per (query, slot)
-    __syncthreads();
-    const int* fin = reinterpret_cast<const int*>(dump);
+    __syncthreads();   // fin complete
     const bool have_q = n_tiles > 0 && mbar_wait(b_full, 0, kTtPollLimit);
-    for (int pq = threadIdx.x; pq < nqv * K; pq += SH::THREADS) {
-      const int q = pq / K, k = pq - q * K;
-      const int c = have_q ? fin[q * K + k] : -1;
-      float acc[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h) acc[h] = 0.f;
-      if (c >= 0) {
-        const uint4* kr = reinterpret_cast<const uint4*>(klm + (bg * D.C + c) * DD);
-#pragma unroll 4
-        for (int u = 0; u < DD / 8; ++u) {   // 16-byte units of the landmark row
-          const uint4 kv = __ldg(kr + u);
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const int row = h * MQ + q;   // the (head, query) row of the B operand
-            const uint4 qv = *reinterpret_cast<const uint4*>(
-                sB + (u >> 3) * SH::B_BOX + (row >> 3) * 1024 + (row & 7) * 128 +
-                (((u & 7) ^ (row & 7)) << 4));
-            float a = acc[h];
-            a = fmaf(bf16_lo(qv.x), bf16_lo(kv.x), a);
-            a = fmaf(bf16_hi(qv.x), bf16_hi(kv.x), a);
-            a = fmaf(bf16_lo(qv.y), bf16_lo(kv.y), a);
-            a = fmaf(bf16_hi(qv.y), bf16_hi(kv.y), a);
-            a = fmaf(bf16_lo(qv.z), bf16_lo(kv.z), a);
-            a = fmaf(bf16_hi(qv.z), bf16_hi(kv.z), a);
-            a = fmaf(bf16_lo(qv.w), bf16_lo(kv.w), a);
-            a = fmaf(bf16_hi(qv.w), bf16_hi(kv.w), a);
-            acc[h] = a;
-          }
-        }
-      }
-      const float bias = c >= 0 ? __ldg(blm + bg * D.C + c) : 0.f;
-#pragma unroll
-      for (int h = 0; h < G; ++h)
-        s_head[((b * D.Hq + g * G + h) * D.N_q + i0 + q) * K + k] =
-            c >= 0 ? fmaf(acc[h], D.scale, bias) : -INFINITY;
-    }
+    head_scores<DD, G, KM>(D, reinterpret_cast<const int*>(sA), sB, have_q, b, g, bg, i0, nqv,
+                           klm, blm, s_head);
   }
   tc_fence_before();
   __syncthreads();
@@ -626,12 +685,7 @@ bool score_t_tc_supported(const Dims& D, bool bf16) {
   if (!bf16 || D.K < 1 || D.K > kMaxK || D.C < 1) return false;
   if (D.B * D.Hkv > 65535) return false;
   if (D.d != 64 && D.d != 128) return false;
-  // four heads: only for long sequences (at least 8192 chunks, 64 or more landmark tiles for the
-  // last query blocks).  Each block pays a start-up (its calibrated-query tile, the first
-  // tile's ranking) that the query-major kernel's blocks of 128 queries amortise better when
-  // blocks are short: on the 7B-like prefill (2048 chunks) that kernel measured 2.29 ms
-  // against 2.91 ms here.
-  return D.G == 8 || (D.G == 4 && D.C >= 8192);
+  return D.G == 4 || D.G == 8;
 }
 
 cudaError_t launch_score_topk_t_tc(const Dims& D, const void* qc, const void* klm,

@@ -39,7 +39,10 @@ CASES = {
     "tc_g2_d64_k32": (dict(B=1, Hq=4, Hkv=2, N=4000, d=64, S=32, K=32, W_=128),
                       torch.bfloat16, "score_topk_tc, 32-slot lists"),
     "tc_g4_d128": (dict(B=1, Hq=8, Hkv=2, N=20000, d=128, S=64, K=16, W_=128),
-                   torch.bfloat16, "score_topk_tc, four heads over fewer than 8192 chunks"),
+                   torch.bfloat16, "score_topk_t_tc (two merge warps) with per-head scores "
+                   "for the two-CTA attention"),
+    "tc_g4_d64": (dict(B=1, Hq=8, Hkv=2, N=20000, d=64, S=64, K=16, W_=128),
+                  torch.bfloat16, "score_topk_tc, four heads over fewer than 8192 chunks"),
     "tc_g8_d128_s128": (dict(B=1, Hq=8, Hkv=1, N=40000, d=128, S=128, K=16, W_=256),
                         torch.bfloat16, "score_topk_t_tc (landmark-major), eight heads"),
     "tc_g8_d64_k32": (dict(B=1, Hq=8, Hkv=1, N=20000, d=64, S=32, K=32, W_=128),
