@@ -65,6 +65,9 @@ def lib():
         l.hils_oracle_landmarks.argtypes = [ctypes.c_int64] * 4 + [ctypes.c_int32,
                                                                    ctypes.c_double] + [
             ctypes.c_void_p] * 4
+        l.hils_oracle_backward.restype = ctypes.c_int
+        l.hils_oracle_backward.argtypes = [ctypes.POINTER(Problem)] + [ctypes.c_void_p] * 15 + [
+            ctypes.c_int]
         l.hils_oracle_n_eligible.restype = ctypes.c_int64
         l.hils_oracle_n_eligible.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32]
         l.hils_oracle_default_threads.restype = ctypes.c_int
@@ -141,6 +144,32 @@ def landmarks(qlm, K, *, S, scale=0.0):
     if rc != 0:
         raise RuntimeError("hils_oracle_landmarks failed with status %d" % rc)
     return klm, blm
+
+
+def backward(q, qc, K, V, klm, blm, idx, dO, dlse=None, *, S, K_top, W, q_pos0=0, scale=0.0,
+             threads=0):
+    """Gradients of sum(dO * out) + sum(dlse * lse) with the selection ``idx`` [B,Hkv,N_q,K_top]
+    held fixed.  Returns a dict with dq, dqc, dK, dV, dklm, dblm (fp64, shaped like q, qc, K, V,
+    klm, blm)."""
+    q, qc, K, V, klm, blm, dO = (_f64(x) for x in (q, qc, K, V, klm, blm, dO))
+    dlse = None if dlse is None else _f64(dlse)
+    B, Hq, Nq, d = q.shape
+    _, Hkv, Nkv, _ = K.shape
+    C = Nkv // S
+    assert klm.shape == (B, Hkv, C, d) and blm.shape == (B, Hkv, C) and dO.shape == q.shape
+    assert dlse is None or dlse.shape == (B, Hq, Nq)
+    idx = np.ascontiguousarray(np.asarray(idx, dtype=np.int32))
+    assert idx.shape == (B, Hkv, Nq, K_top)
+    pr = Problem(B, Hq, Hkv, Nq, Nkv, d, q_pos0, S, K_top, W, float(scale))
+    r = {"dq": np.empty_like(q), "dqc": np.empty_like(q), "dK": np.empty_like(K),
+         "dV": np.empty_like(K), "dklm": np.empty_like(klm), "dblm": np.empty_like(blm)}
+    rc = lib().hils_oracle_backward(
+        ctypes.byref(pr), _ptr(q), _ptr(qc), _ptr(K), _ptr(V), _ptr(klm), _ptr(blm), _ptr(idx),
+        _ptr(dO), _ptr(dlse), _ptr(r["dq"]), _ptr(r["dqc"]), _ptr(r["dK"]), _ptr(r["dV"]),
+        _ptr(r["dklm"]), _ptr(r["dblm"]), int(threads))
+    if rc != 0:
+        raise RuntimeError("hils_oracle_backward failed with status %d" % rc)
+    return r
 
 
 class Query:

@@ -59,6 +59,10 @@
  *   mass, calibrated by an entropy term; [DevTo] "The Core Idea: Landmark Tokens and
  *   Hierarchical Factorization").
  *
+ * Backward (hils_oracle_bwd.c): reverse-mode differentiation of steps 4, 1 and 3 above with
+ * the selection held fixed (R16: the top-K passes no gradient; the landmark keys and biases
+ * receive theirs through the fusion weights, [Reader] Fig. 3 caption).
+ *
  * Every function here is pinned by CPU tests against values the pages print, closed forms
  * and brute force (no function is "parity unpinned").
  */
@@ -147,6 +151,16 @@ int hils_oracle_forward(const hils_oracle_problem* pr, const double* q, const do
 int hils_oracle_landmarks(int64_t B, int64_t Hkv, int64_t N_kv, int64_t d, int32_t S,
                           double scale, const double* qlm, const double* K, double* klm,
                           double* blm);
+
+/* Backward pass (hils_oracle_bwd.c): the gradient of L = sum dO . out + sum dlse . lse with
+ * respect to q, qc, K, V, klm and blm, the selection idx [B,Hkv,N_q,K_top] (-1 padded, as
+ * idx_in) held fixed.  dO [B,Hq,N_q,d]; dlse [B,Hq,N_q] or NULL (zero); dq, dqc like q; dK, dV
+ * like K; dklm, dblm like klm, blm (all overwritten).  Threads over (b, g) pairs. */
+int hils_oracle_backward(const hils_oracle_problem* pr, const double* q, const double* qc,
+                         const double* K, const double* V, const double* klm, const double* blm,
+                         const int32_t* idx, const double* dO, const double* dlse, double* dq,
+                         double* dqc, double* dK, double* dV, double* dklm, double* dblm,
+                         int n_threads);
 
 /* Rule R1: number of eligible distant chunks of the query at position pos. */
 int64_t hils_oracle_n_eligible(int64_t pos, int32_t S, int32_t W);
