@@ -657,6 +657,58 @@ def extra_landmarks(peaks, B, Hkv, N, d, S, steps=5, seed=77):
                          "frac": gbs / peaks["hbm_gbs"]}}
 
 
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 fp32 lanes x 2 flops x 1.965 GHz (the
+# backward's products run there; no measured figure exists for this unit)
+FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def extra_backward(peaks, name="gqa7b_prefill", steps=3, **overrides):
+    """hils_backward on a prefill workload, the forward's own selection held fixed.  Algorithmic
+    FLOPs: 10 d per (row, attended token) (the logits and dout . V recomputed, then the dq, dK
+    and dV products) plus 4 d per (row, selected slot) (d q_cal and d k_lm)."""
+    from hierarchical_chunk_sparse_scoring_b200 import binding as hb
+    from hierarchical_chunk_sparse_scoring_b200 import workloads as W
+    wl = W.make(name, "cuda", **overrides)
+    kw = wl.kwargs()
+    _, _, idx = hb.forward(wl.q, wl.q_cal, wl.K, wl.V, wl.k_lm, wl.b_lm, **kw)
+    g = torch.Generator(device="cuda").manual_seed(5)
+    dout = torch.randn(wl.q.shape, generator=g, device="cuda").to(wl.q.dtype)
+    dlse = torch.randn(wl.q.shape[:3], generator=g, device="cuda")
+    p = hb.make_params(*[wl.dims[k] for k in ("B", "Hq", "Hkv", "N_q", "N_kv", "d")], S=wl.S,
+                       K_top=wl.K_top, W=wl.W, q_pos0=wl.q_pos0, dtype=wl.q.dtype)
+    ws = hb.backward_workspace(p, wl.q.device)
+    grads = hb.backward(wl.q, wl.q_cal, wl.K, wl.V, wl.k_lm, wl.b_lm, idx, dout, dlse, ws=ws,
+                        **kw)
+    flush = make_flush(wl.q.device)
+    ms = []
+    for _ in range(steps):
+        flush()
+        a, b_ = make_events(2)
+        a.record()
+        hb.backward(wl.q, wl.q_cal, wl.K, wl.V, wl.k_lm, wl.b_lm, idx, dout, dlse, ws=ws,
+                    out=grads, **kw)
+        b_.record()
+        torch.cuda.synchronize()
+        ms.append(a.elapsed_time(b_))
+    t = statistics.mean(ms)
+    wm = work_model(wl.dims, wl.S, wl.K_top, wl.W, wl.q_pos0, wl.q.element_size())
+    pos = np.arange(wl.q_pos0, wl.q_pos0 + wl.dims["N_q"], dtype=np.int64)
+    n = np.where(pos - wl.W + 1 > 0, (pos - wl.W + 1) // wl.S, 0)
+    slots = float(np.minimum(n, wl.K_top).sum()) * wl.dims["B"] * wl.dims["Hq"]
+    flops = 2.5 * wm["attn_flops"] + 4.0 * wl.dims["d"] * slots
+    tf = flops / (t * 1e-3) / 1e12
+    out = {"kernel": "bwd_rows + bwd_keys (+ index build)", "workload": name,
+           "shape": {k: wl.dims[k] for k in ("B", "Hq", "Hkv", "N_q", "N_kv", "d")},
+           "ms": t, "tflop": flops / 1e12, "tokens_per_s": wl.dims["B"] * wl.dims["N_q"] / (t * 1e-3),
+           "roofline": {"bound": "alu", "achieved": tf, "peak": FP32_FMA_TFLOPS,
+                        "unit": "TFLOP/s", "frac": tf / FP32_FMA_TFLOPS,
+                        "peak_note": "fp32 FMA of the CUDA cores, 148 SMs x 128 lanes x 2 x 1.965 GHz"},
+           "frac_of_bf16_tensor_peak": tf / peaks["bf16_tflops"]}
+    del wl, grads, ws, dout, dlse, idx
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_hils(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -734,6 +786,7 @@ def run_hils(args):
         line["extreme_1m"] = extra_extreme(2, peaks, N=1 << 20)
         line["landmarks"] = [extra_landmarks(peaks, 1, 1, 1 << 22, 128, 128),
                              extra_landmarks(peaks, 1, 8, 131072, 128, 64)]
+        line["backward_gqa7b"] = extra_backward(peaks, "gqa7b_prefill")
     if dist:
         dist.destroy_process_group()
     if rank == 0:

@@ -49,6 +49,8 @@ SIGNATURES = {
     "hils_landmarks": (ctypes.c_int, [_P, _V, _V, _V, _V, _V]),
     "hils_decode_step": (ctypes.c_int, [_P] + [_V] * 13 + [ctypes.c_size_t, _V]),
     "hils_wait_check": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_int, _V, ctypes.c_size_t, _V]),
+    "hils_backward_workspace_size": (ctypes.c_size_t, [_P]),
+    "hils_backward": (ctypes.c_int, [_P] + [_V] * 16 + [ctypes.c_size_t, _V]),
     "hils_chunk_attn": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V, _V]),
     "hils_fuse": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V]),
     "hils_workspace_init": (ctypes.c_int, [_V, ctypes.c_size_t, _V]),
@@ -276,6 +278,48 @@ def decode_step(q, q_cal, k_new, v_new, q_lm_new, K, V, k_lm, b_lm, *, pos, S, K
                                   _ptr(idx), _ptr(ws), ws.numel(), _stream(stream)),
            "hils_decode_step")
     return out, lse, idx
+
+
+def backward_workspace(p, device):
+    need = int(lib().hils_backward_workspace_size(ctypes.byref(p)))
+    if need == 0:
+        return None   # invalid or unsupported: hils_backward says which
+    return torch.empty(need, dtype=torch.uint8, device=device)
+
+
+def backward(q, q_cal, K, V, k_lm, b_lm, idx, dout, dlse=None, *, S, K_top, W, q_pos0=0,
+             scale=0.0, ws=None, out=None, stream=None):
+    """hils_backward: gradients of sum(dout * out) + sum(dlse * lse) with the selection `idx`
+    held fixed.  Returns a dict of fp32 tensors dq, dq_cal, dK, dV, dk_lm, db_lm."""
+    B, Hq, N_q, d = q.shape
+    _, Hkv, N_kv, _ = K.shape
+    C = N_kv // S
+    _need(q, "q")
+    _need(q_cal, "q_cal", q.dtype, q.shape)
+    _need(K, "K", q.dtype)
+    _need(V, "V", q.dtype, K.shape)
+    _need(k_lm, "k_lm", q.dtype, (B, Hkv, C, d))
+    _need(b_lm, "b_lm", torch.float32, (B, Hkv, C))
+    _need(idx, "idx", torch.int32, (B, Hkv, N_q, K_top))
+    _need(dout, "dout", q.dtype, q.shape)
+    if dlse is not None:
+        _need(dlse, "dlse", torch.float32, (B, Hq, N_q))
+    p = make_params(B, Hq, Hkv, N_q, N_kv, d, S=S, K_top=K_top, W=W, q_pos0=q_pos0,
+                    dtype=q.dtype, scale=scale)
+    if ws is None:
+        ws = backward_workspace(p, q.device)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = out if out is not None else {
+        "dq": torch.empty(q.shape, **f32), "dq_cal": torch.empty(q.shape, **f32),
+        "dK": torch.empty(K.shape, **f32), "dV": torch.empty(K.shape, **f32),
+        "dk_lm": torch.empty(k_lm.shape, **f32), "db_lm": torch.empty(b_lm.shape, **f32)}
+    _check(lib().hils_backward(ctypes.byref(p), _ptr(q), _ptr(q_cal), _ptr(K), _ptr(V),
+                               _ptr(k_lm), _ptr(b_lm), _ptr(idx), _ptr(dout), _ptr(dlse),
+                               _ptr(g["dq"]), _ptr(g["dq_cal"]), _ptr(g["dK"]), _ptr(g["dV"]),
+                               _ptr(g["dk_lm"]), _ptr(g["db_lm"]), _ptr(ws),
+                               0 if ws is None else ws.numel(), _stream(stream)),
+           "hils_backward")
+    return g
 
 
 def select_noalloc(q_cal, k_lm, b_lm, *, N_kv, Hkv, S, K_top, W, q_pos0=0, scale=0.0,

@@ -442,6 +442,46 @@ extern "C" hils_status hils_decode_step(const hils_params* p, const void* q, con
                       workspace_bytes, stream, nullptr, 0);
 }
 
+extern "C" size_t hils_backward_workspace_size(const hils_params* p) {
+  if (check_params(p) != HILS_OK) return 0;
+  const Plan P = make_plan(p);
+  if (!backward_supported(P.D)) return 0;
+  return backward_ws_layout(P.D, nullptr, nullptr);
+}
+
+extern "C" hils_status hils_backward(const hils_params* p, const void* q, const void* q_cal,
+                                     const void* K, const void* V, const void* k_lm,
+                                     const float* b_lm, const int32_t* topk_idx,
+                                     const void* dout, const float* dlse, float* dq,
+                                     float* dq_cal, float* dK, float* dV, float* dk_lm,
+                                     float* db_lm, void* workspace, size_t workspace_bytes,
+                                     hils_stream_t stream) {
+  hils_status s = check_params(p);
+  if (s != HILS_OK) return s;
+  const Plan P = make_plan(p);
+  if (!backward_supported(P.D)) return HILS_ERR_UNSUPPORTED;
+  const bool rows = p->B > 0 && p->N_q > 0;
+  const bool keys = p->B > 0;
+  const bool lm = keys && P.D.C > 0;
+  if (!ok_ptr(q, rows) || !ok_ptr(q_cal, rows) || !ok_ptr(dout, rows) || !ok_ptr(dq, rows) ||
+      !ok_ptr(dq_cal, rows) || !ok_ptr(topk_idx, rows && p->K_top > 0) || !ok_ptr(K, keys) ||
+      !ok_ptr(V, keys) || !ok_ptr(dK, keys) || !ok_ptr(dV, keys) || !ok_ptr(k_lm, lm) ||
+      !ok_ptr(b_lm, lm) || !ok_ptr(dk_lm, lm) || !ok_ptr(db_lm, lm) ||
+      (dlse && !aligned16(dlse)))
+    return HILS_ERR_INVALID_ARG;
+  const size_t need = backward_ws_layout(P.D, nullptr, nullptr);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < need) return HILS_ERR_WORKSPACE;
+  if (!keys) return HILS_OK;
+  if ((s = check_device()) != HILS_OK) return s;
+  BwdWs w;
+  backward_ws_layout(P.D, &w, static_cast<char*>(workspace));
+  BwdArgs a{q, q_cal, K, V, k_lm, b_lm, topk_idx, dout, dlse, dq, dq_cal, dK, dV, dk_lm, db_lm};
+  return launch_backward(P.D, P.bf16, a, w, reinterpret_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? HILS_OK
+             : HILS_ERR_CUDA;
+}
+
 extern "C" hils_status hils_workspace_init(void* workspace, size_t workspace_bytes,
                                            hils_stream_t stream) {
   if (!workspace || !aligned16(workspace) || workspace_bytes < kStatusBytes)

@@ -1,0 +1,860 @@
+// Backward pass: gradients of L = sum dO . O + sum dlse . LSE with respect to q, q_cal, K, V,
+// k_lm and b_lm, the forward's selection held fixed (the top-K is piecewise constant and passes
+// no gradient; the landmark keys and biases receive theirs through the fusion weights, [Reader]
+// Fig. 3 caption: the loss gradient flows back to the compressed key).
+//
+// Per row (query i, head h) with units u (its selected chunks, then the local window) and fused
+// weights w_u = exp(score_u - LSE), a token j of unit u has the fused weight a_j =
+// exp(x_j + lambda_u) with lambda_u = score_u - LSE - lse_u, and by the chain rule through
+// steps 4, 1 and 3 (the window's score is its own lse, so it adds its score gradient to its
+// tokens' logits):
+//   dV_j += a_j dO,  dx_j = a_j (dO . V_j - gamma_u),  dq += scale dx_j K_j,  dK_j += scale dx_j q
+//   gamma_c = delta_c = dO . o_c for a chunk, gamma_local = D - dlse with D = sum_u w_u delta_u,
+//   dscore_c = w_c (delta_c - D + dlse):  dq_cal += scale dscore_c k_lm_c,
+//   dk_lm_c += scale dscore_c q_cal,  db_lm_c += dscore_c.
+// delta_u needs a pass over the unit's tokens before any gradient can be formed, so:
+//   bwd_rows_kernel  (query-major; CTA = 64 rows of one KV group: 64/G queries x G heads over the
+//                    union of their chunks) pass 1: lse_u and delta_u by an online reduction of
+//                    the logits x = q K^T and dP = dO V^T; then the fusion terms per row, d q_cal,
+//                    and lambda, gamma, dscore to the workspace; pass 2: dq.
+//   inverse index    (count, scan, fill) chunk -> the (query, slot) entries that selected it.
+//   bwd_keys_kernel  (key-major; CTA = one tile of up to 64 keys of one chunk) over the rows whose
+//                    window covers the tile and the rows that selected its chunk: dK and dV held
+//                    in registers, then d k_lm and d b_lm from the selecting rows' dscore.
+// No gradient is accumulated with atomics.  The products are CUDA-core tiles: 4 x (T/16)
+// outputs per thread, operands staged in shared memory as fp32 (rows padded by 4 floats so the
+// 16-byte loads of consecutive rows fall in different banks).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace hils {
+namespace {
+
+constexpr int kBwdRows = 64;      // rows per batch
+constexpr int kBwdThreads = 256;
+constexpr int kBwdMaxK = 32;
+constexpr int kBwdMaxUnion = kBwdRows * kBwdMaxK;   // selected ids of one row tile
+constexpr float kB2 = 1.4426950408889634f;          // log2(e)
+constexpr float kLn2b = 0.6931471805599453f;
+
+template <int DD, int T>
+struct BwdShape {
+  static constexpr int LD = DD + 4;            // fp32 row stride of staged q / dO / K / V rows
+  static constexpr int LDA = T + 1;            // stride of the a / dx tiles
+  static constexpr int KPT = T / 16;           // keys per thread in the logit tiles
+  static constexpr int DG = DD / 64;           // float4 groups of dims per thread (dims td*4+64e)
+  static constexpr int ROWS_F = kBwdRows * LD;
+  static constexpr int KEYS_F = T * LD;
+  static constexpr int TILE_F = kBwdRows * LDA;
+  static_assert(DD == 64 || DD == 128, "head dims 64 and 128");
+  static_assert(T == 16 || T == 32 || T == 64, "key tiles of 16, 32 or 64");
+};
+
+template <typename TI>
+__device__ __forceinline__ void load_piece(const TI* src, float* dst);
+template <>
+__device__ __forceinline__ void load_piece<float>(const float* src, float* dst) {
+  *reinterpret_cast<float4*>(dst) = __ldg(reinterpret_cast<const float4*>(src));
+}
+template <>
+__device__ __forceinline__ void load_piece<__nv_bfloat16>(const __nv_bfloat16* src, float* dst) {
+  const uint4 t = __ldg(reinterpret_cast<const uint4*>(src));
+  *reinterpret_cast<float4*>(dst) = make_float4(bf16_lo(t.x), bf16_hi(t.x), bf16_lo(t.y),
+                                                bf16_hi(t.y));
+  *reinterpret_cast<float4*>(dst + 4) = make_float4(bf16_lo(t.z), bf16_hi(t.z), bf16_lo(t.w),
+                                                    bf16_hi(t.w));
+}
+
+// Rows r < n of dst (stride LD floats) from rowp[r] (nullptr: zeros), fp32.
+template <typename TI, int DD, int LD>
+__device__ __forceinline__ void stage_rows(float* dst, const TI* const* rowp, int n) {
+  constexpr int EPP = 16 / (int)sizeof(TI);   // elements per 16-byte piece
+  constexpr int PPR = DD / EPP;
+  for (int e = threadIdx.x; e < n * PPR; e += kBwdThreads) {
+    const int r = e / PPR, u = e - r * PPR;
+    const TI* src = rowp[r];
+    float* d = dst + r * LD + u * EPP;
+    if (src) {
+      load_piece<TI>(src + u * EPP, d);
+    } else {
+      *reinterpret_cast<float4*>(d) = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (EPP == 8) *reinterpret_cast<float4*>(d + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+}
+
+// Keys k0 .. k0 + T - 1 of one (b, g) plane (zeros past N_kv), fp32.
+template <typename TI, int DD, int LD, int T>
+__device__ __forceinline__ void stage_keys(float* dst, const TI* base, int64_t k0, int64_t nkv) {
+  constexpr int EPP = 16 / (int)sizeof(TI);
+  constexpr int PPR = DD / EPP;
+  for (int e = threadIdx.x; e < T * PPR; e += kBwdThreads) {
+    const int r = e / PPR, u = e - r * PPR;
+    float* d = dst + r * LD + u * EPP;
+    if (k0 + r < nkv) {
+      load_piece<TI>(base + (k0 + r) * DD + u * EPP, d);
+    } else {
+      *reinterpret_cast<float4*>(d) = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (EPP == 8) *reinterpret_cast<float4*>(d + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+}
+
+__device__ __forceinline__ float dot4(const float4 a, const float4 b, float acc) {
+  acc = fmaf(a.x, b.x, acc);
+  acc = fmaf(a.y, b.y, acc);
+  acc = fmaf(a.z, b.z, acc);
+  return fmaf(a.w, b.w, acc);
+}
+
+// X = Q K^T and P = dO V^T for rows tr*4 + i and keys tc + 16 e of the staged tiles.
+template <int DD, int T>
+__device__ __forceinline__ void logits_tile(const float* sQ, const float* sdO, const float* sK,
+                                            const float* sV, int tr, int tc,
+                                            float (&X)[4][T / 16], float (&P)[4][T / 16]) {
+  using SH = BwdShape<DD, T>;
+  constexpr int KPT = SH::KPT, LD = SH::LD;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int e = 0; e < KPT; ++e) X[i][e] = P[i][e] = 0.f;
+#pragma unroll 2
+  for (int k = 0; k < DD; k += 4) {
+    float4 kk[KPT], vv[KPT];
+#pragma unroll
+    for (int e = 0; e < KPT; ++e) {
+      kk[e] = *reinterpret_cast<const float4*>(sK + (tc + 16 * e) * LD + k);
+      vv[e] = *reinterpret_cast<const float4*>(sV + (tc + 16 * e) * LD + k);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 q = *reinterpret_cast<const float4*>(sQ + (tr * 4 + i) * LD + k);
+      const float4 o = *reinterpret_cast<const float4*>(sdO + (tr * 4 + i) * LD + k);
+#pragma unroll
+      for (int e = 0; e < KPT; ++e) {
+        X[i][e] = dot4(q, kk[e], X[i][e]);
+        P[i][e] = dot4(o, vv[e], P[i][e]);
+      }
+    }
+  }
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------------------------
+// Query-major kernel: CTA = (b, g, 64/G queries); row r = query r / G, head g G + r % G.
+template <typename TI, int DD, int T>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_rows_kernel(Dims D, const TI* __restrict__ q, const TI* __restrict__ qc,
+                    const TI* __restrict__ K, const TI* __restrict__ V,
+                    const TI* __restrict__ klm, const float* __restrict__ blm,
+                    const int32_t* __restrict__ idx, const TI* __restrict__ dO,
+                    const float* __restrict__ dlse, float* __restrict__ dq,
+                    float* __restrict__ dqc, float* __restrict__ lam_ws,
+                    float* __restrict__ gam_ws, float* __restrict__ ds_ws) {
+  using SH = BwdShape<DD, T>;
+  constexpr int LD = SH::LD, LDA = SH::LDA, KPT = SH::KPT, DG = SH::DG;
+  constexpr int SU = kBwdMaxK + 1;   // stats row stride (units)
+  extern __shared__ float4 smem_f4[];
+  float* sQ = reinterpret_cast<float*>(smem_f4);
+  float* sdO = sQ + SH::ROWS_F;
+  float* sK = sdO + SH::ROWS_F;
+  float* sV = sK + SH::KEYS_F;
+  float* sdX = sV + SH::KEYS_F;
+  float* sM = sdX + SH::TILE_F;              // [64][SU] running max (base 2), then lambda2
+  float* sL = sM + kBwdRows * SU;            // running sum, then gamma
+  float* sT = sL + kBwdRows * SU;            // running sum of p dP, then dscore
+  float* sS = sT + kBwdRows * SU;            // [64][32] chunk scores
+  int* sel = reinterpret_cast<int*>(sS + kBwdRows * kBwdMaxK);   // [QT][K]
+  int* sU = sel + kBwdMaxUnion;              // selected chunks below the window range, sorted
+  int64_t* sPos = reinterpret_cast<int64_t*>(sU + kBwdMaxUnion);   // [64]
+  float* sDl = reinterpret_cast<float*>(sPos + kBwdRows);          // [64] dlse
+  int* sUnit = reinterpret_cast<int*>(sDl + kBwdRows);             // [64]
+  const TI** rowp = reinterpret_cast<const TI**>(sUnit + kBwdRows + 2);   // [64]
+  int* sCount = reinterpret_cast<int*>(rowp + kBwdRows);                  // [1]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tr = tid >> 4, tc = tid & 15;
+  const int G = D.G, QT = kBwdRows / G, Kt = D.K;
+  const int64_t bg = blockIdx.y, b = bg / D.Hkv, g = bg - b * D.Hkv;
+  const int64_t i0 = (int64_t)blockIdx.x * QT;
+  const int nq = (int)(D.N_q - i0 < QT ? D.N_q - i0 : QT);
+  const float sc2 = D.scale * kB2;
+  const TI* Kb = K + bg * D.N_kv * DD;
+  const TI* Vb = V + bg * D.N_kv * DD;
+  auto grow_of = [&](int r) {   // global row of batch row r (valid rows only)
+    return (b * D.Hq + g * G + r % G) * D.N_q + i0 + r / G;
+  };
+
+  // ---- rows, selections, union of the selected chunks below the window range
+  if (tid < kBwdRows) {
+    const int qq = tid / G;
+    const bool valid = qq < nq;
+    sPos[tid] = valid ? D.q_pos0 + i0 + qq : INT64_MIN;
+    sDl[tid] = (valid && dlse) ? dlse[grow_of(tid)] : 0.f;
+    rowp[tid] = valid ? q + grow_of(tid) * DD : nullptr;
+  }
+  const int64_t c_lo = n_eligible(D.q_pos0 + i0, D.S, D.W);
+  const int64_t c_hi = (D.q_pos0 + i0 + nq - 1) / D.S;
+  int np = 1;
+  while (np < QT * Kt) np <<= 1;
+  for (int e = tid; e < np; e += kBwdThreads) {
+    int c = INT_MAX;
+    if (e < QT * Kt) {
+      const int qq = e / Kt;
+      int v = qq < nq ? idx[(bg * D.N_q + i0 + qq) * Kt + (e - qq * Kt)] : -1;
+      // an id outside the query's eligible chunks is an empty slot (no memory outside k_lm is
+      // read for it); a repeated id is attended once, in its first slot
+      if (v >= 0 && v >= n_eligible(D.q_pos0 + i0 + qq, D.S, D.W)) v = -1;
+      sel[e] = v;
+      if (v >= 0 && v < c_lo) c = v;
+    }
+    sU[e] = c;
+  }
+  __syncthreads();
+  stage_rows<TI, DD, LD>(sQ, rowp, kBwdRows);
+  __syncthreads();
+  if (tid < kBwdRows) rowp[tid] = sPos[tid] != INT64_MIN ? dO + grow_of(tid) * DD : nullptr;
+  __syncthreads();
+  // bitonic sort of the union candidates
+  for (int k2 = 2; k2 <= np; k2 <<= 1)
+    for (int j2 = k2 >> 1; j2 > 0; j2 >>= 1) {
+      for (int e = tid; e < np; e += kBwdThreads) {
+        const int f = e ^ j2;
+        if (f > e) {
+          const int a = sU[e], c = sU[f];
+          const bool up = (e & k2) == 0;
+          if ((a > c) == up) {
+            sU[e] = c;
+            sU[f] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  stage_rows<TI, DD, LD>(sdO, rowp, kBwdRows);
+  if (warp == 0) {   // compact the distinct ids to the front (sorted: a repeat follows its twin)
+    int n = 0, last = INT_MIN;
+    for (int e0 = 0; e0 < np; e0 += 32) {
+      const int e = e0 + lane;
+      const int v = e < np ? sU[e] : INT_MAX;
+      int prev = __shfl_up_sync(0xffffffffu, v, 1);
+      if (lane == 0) prev = last;
+      last = __shfl_sync(0xffffffffu, v, 31);
+      const bool keep = v != INT_MAX && v != prev;
+      const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+      __syncwarp();
+      if (keep) sU[n + __popc(bal & ((1u << lane) - 1u))] = v;
+      n += __popc(bal);
+      __syncwarp();
+    }
+    if (lane == 0) *sCount = n;
+  }
+  for (int e = tid; e < kBwdRows * SU; e += kBwdThreads) {
+    sM[e] = -INFINITY;
+    sL[e] = 0.f;
+    sT[e] = 0.f;
+  }
+  __syncthreads();
+  const int n_sel = *sCount;
+  const int SPT = D.S / T;   // key tiles per chunk
+  const int n_tiles = (n_sel + (int)(c_hi - c_lo + 1)) * SPT;
+
+  auto tile_k0 = [&](int t) -> int64_t {
+    const int ci = t / SPT;
+    const int64_t c = ci < n_sel ? (int64_t)sU[ci] : c_lo + (ci - n_sel);
+    return c * D.S + (int64_t)(t - ci * SPT) * T;
+  };
+  // unit of each row for the tile starting at k0 (-1: not attended)
+  auto set_units = [&](int64_t k0) {
+    if (tid < kBwdRows) {
+      const int64_t pos = sPos[tid];
+      int u = -1;
+      if (pos != INT64_MIN) {
+        const int64_t c = k0 / D.S;
+        if (c >= n_eligible(pos, D.S, D.W)) {
+          u = k0 <= pos ? Kt : -1;
+        } else {
+          const int* sr = sel + (tid / G) * Kt;
+          for (int k = Kt - 1; k >= 0; --k)
+            if (sr[k] == (int)c) u = k;
+        }
+      }
+      sUnit[tid] = u;
+    }
+  };
+
+  // ---- pass 1: per (row, unit) lse and delta = dO . o_u by online reduction
+  for (int t = 0; t < n_tiles; ++t) {
+    const int64_t k0 = tile_k0(t);
+    stage_keys<TI, DD, LD, T>(sK, Kb, k0, D.N_kv);
+    stage_keys<TI, DD, LD, T>(sV, Vb, k0, D.N_kv);
+    set_units(k0);
+    __syncthreads();
+    float X[4][KPT], P[4][KPT];
+    logits_tile<DD, T>(sQ, sdO, sK, sV, tr, tc, X, P);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = tr * 4 + i;
+      const int u = sUnit[r];
+      const int64_t pos = sPos[r];
+      float m = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < KPT; ++e) {
+        const int64_t j = k0 + tc + 16 * e;
+        const bool ok = u >= 0 && j <= pos && j < D.N_kv;
+        X[i][e] = ok ? X[i][e] * sc2 : -INFINITY;
+        m = fmaxf(m, X[i][e]);
+      }
+#pragma unroll
+      for (int o = 1; o < 16; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      float l = 0.f, tt = 0.f;
+#pragma unroll
+      for (int e = 0; e < KPT; ++e) {
+        const float w = X[i][e] == -INFINITY ? 0.f : exp2f(X[i][e] - m);
+        l += w;
+        tt = fmaf(w, P[i][e], tt);
+      }
+#pragma unroll
+      for (int o = 1; o < 16; o <<= 1) {
+        l += __shfl_xor_sync(0xffffffffu, l, o);
+        tt += __shfl_xor_sync(0xffffffffu, tt, o);
+      }
+      if (tc == 0 && u >= 0 && m != -INFINITY) {
+        float* pm = sM + r * SU + u;
+        float* pl = sL + r * SU + u;
+        float* pt = sT + r * SU + u;
+        const float M = *pm;
+        if (m > M) {
+          const float f = M == -INFINITY ? 0.f : exp2f(M - m);
+          *pl = *pl * f + l;
+          *pt = *pt * f + tt;
+          *pm = m;
+        } else {
+          const float f = exp2f(m - M);
+          *pl += l * f;
+          *pt += tt * f;
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  // ---- fusion terms per row
+  for (int r = warp; r < kBwdRows; r += kBwdThreads / 32) {   // chunk scores s = scale qc.klm + b
+    if (sPos[r] == INT64_MIN) continue;
+    constexpr int DL = DD / 32;
+    float qv[DL];
+    const TI* qr = qc + grow_of(r) * DD + lane * DL;
+#pragma unroll
+    for (int e = 0; e < DL; ++e) qv[e] = Elem<TI>::to_f(qr[e]);
+    for (int k = 0; k < Kt; ++k) {
+      const int c = sel[(r / G) * Kt + k];
+      if (c < 0) continue;
+      const TI* kr = klm + (bg * D.C + c) * DD + lane * DL;
+      float a = 0.f;
+#pragma unroll
+      for (int e = 0; e < DL; ++e) a = fmaf(qv[e], Elem<TI>::to_f(kr[e]), a);
+      a = warp_sum(a);
+      if (lane == 0) sS[r * kBwdMaxK + k] = fmaf(a, D.scale, blm[bg * D.C + c]);
+    }
+  }
+  __syncthreads();
+  if (tid < kBwdRows && sPos[tid] != INT64_MIN) {
+    const int r = tid;
+    const int* sr = sel + (r / G) * Kt;
+    float* M = sM + r * SU;
+    float* Ls = sL + r * SU;
+    float* Ts = sT + r * SU;
+    // lse_u (natural log) to M, delta_u to Ts, score_u to Ls; the window's score is its lse
+    float mx = -INFINITY;
+    for (int u = 0; u <= Kt; ++u) {
+      const bool present = u == Kt || (sr[u] >= 0 && Ls[u] > 0.f);
+      const float lse = present ? (M[u] + log2f(Ls[u])) * kLn2b : -INFINITY;
+      const float dlt = present ? Ts[u] / Ls[u] : 0.f;
+      const float score = u == Kt ? lse : (present ? sS[r * kBwdMaxK + u] : -INFINITY);
+      M[u] = lse;
+      Ts[u] = dlt;
+      Ls[u] = score;
+      mx = fmaxf(mx, score);
+    }
+    float z = 0.f;
+    for (int u = 0; u <= Kt; ++u) z += Ls[u] == -INFINITY ? 0.f : expf(Ls[u] - mx);
+    const float LSE = mx + logf(z);
+    float Dsum = 0.f;
+    for (int u = 0; u <= Kt; ++u)
+      if (Ls[u] != -INFINITY) Dsum = fmaf(expf(Ls[u] - LSE), Ts[u], Dsum);
+    const float dl = sDl[r];
+    const int64_t grow = grow_of(r);
+    for (int u = 0; u <= Kt; ++u) {
+      const float score = Ls[u];
+      const bool live = score != -INFINITY;
+      const float w = live ? expf(score - LSE) : 0.f;
+      const float lam2 = live ? (score - LSE - M[u]) * kB2 : -INFINITY;
+      const float gam = u == Kt ? Dsum - dl : Ts[u];
+      const float dsc = u == Kt ? 0.f : w * (Ts[u] - Dsum + dl);
+      M[u] = lam2;
+      Ls[u] = gam;
+      Ts[u] = dsc;
+      lam_ws[grow * (Kt + 1) + u] = lam2;
+      gam_ws[grow * (Kt + 1) + u] = gam;
+      if (u < Kt) ds_ws[grow * Kt + u] = dsc;
+    }
+  }
+  __syncthreads();
+  for (int r = warp; r < kBwdRows; r += kBwdThreads / 32) {   // d q_cal = scale sum ds k_lm
+    if (sPos[r] == INT64_MIN) continue;
+    constexpr int DL = DD / 32;
+    float acc[DL];
+#pragma unroll
+    for (int e = 0; e < DL; ++e) acc[e] = 0.f;
+    for (int k = 0; k < Kt; ++k) {
+      const int c = sel[(r / G) * Kt + k];
+      if (c < 0) continue;
+      const float dsc = sT[r * SU + k];
+      const TI* kr = klm + (bg * D.C + c) * DD + lane * DL;
+#pragma unroll
+      for (int e = 0; e < DL; ++e) acc[e] = fmaf(dsc, Elem<TI>::to_f(kr[e]), acc[e]);
+    }
+    float* out = dqc + grow_of(r) * DD + lane * DL;
+#pragma unroll
+    for (int e = 0; e < DL; ++e) out[e] = acc[e] * D.scale;
+  }
+
+  // ---- pass 2: dq = scale sum_j dx_j K_j
+  float acc[4][DG][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int e = 0; e < DG; ++e)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) acc[i][e][v] = 0.f;
+  for (int t = 0; t < n_tiles; ++t) {
+    const int64_t k0 = tile_k0(t);
+    __syncthreads();
+    stage_keys<TI, DD, LD, T>(sK, Kb, k0, D.N_kv);
+    stage_keys<TI, DD, LD, T>(sV, Vb, k0, D.N_kv);
+    set_units(k0);
+    __syncthreads();
+    float X[4][KPT], P[4][KPT];
+    logits_tile<DD, T>(sQ, sdO, sK, sV, tr, tc, X, P);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = tr * 4 + i;
+      const int u = sUnit[r];
+      const int64_t pos = sPos[r];
+      const float lam2 = u >= 0 ? sM[r * SU + u] : -INFINITY;
+      const float gam = u >= 0 ? sL[r * SU + u] : 0.f;
+#pragma unroll
+      for (int e = 0; e < KPT; ++e) {
+        const int64_t j = k0 + tc + 16 * e;
+        const bool ok = u >= 0 && j <= pos && j < D.N_kv && lam2 != -INFINITY;
+        const float a = ok ? exp2f(fmaf(X[i][e], sc2, lam2)) : 0.f;
+        sdX[r * LDA + tc + 16 * e] = a * (P[i][e] - gam);
+      }
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int j = 0; j < T; ++j) {
+      float w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w[i] = sdX[(tr * 4 + i) * LDA + j];
+#pragma unroll
+      for (int e = 0; e < DG; ++e) {
+        const float4 kv = *reinterpret_cast<const float4*>(sK + j * LD + tc * 4 + 64 * e);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[i][e][0] = fmaf(w[i], kv.x, acc[i][e][0]);
+          acc[i][e][1] = fmaf(w[i], kv.y, acc[i][e][1]);
+          acc[i][e][2] = fmaf(w[i], kv.z, acc[i][e][2]);
+          acc[i][e][3] = fmaf(w[i], kv.w, acc[i][e][3]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = tr * 4 + i;
+    if (sPos[r] == INT64_MIN) continue;
+    float* out = dq + grow_of(r) * DD;
+#pragma unroll
+    for (int e = 0; e < DG; ++e)
+      *reinterpret_cast<float4*>(out + tc * 4 + 64 * e) =
+          make_float4(acc[i][e][0] * D.scale, acc[i][e][1] * D.scale, acc[i][e][2] * D.scale,
+                      acc[i][e][3] * D.scale);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Key-major kernel: CTA = (b, g, keys k0 .. k0 + T - 1 of chunk c = k0 / S).  Its rows are the
+// window rows (queries whose local window [S n, p] reaches the tile: n <= c and p >= k0, all G
+// heads) and the selecting rows (the inverse index of chunk c, all G heads), in batches of 64.
+template <typename TI, int DD, int T>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_keys_kernel(Dims D, const TI* __restrict__ q, const TI* __restrict__ qc,
+                    const TI* __restrict__ K, const TI* __restrict__ V,
+                    const TI* __restrict__ dO, const float* __restrict__ lam_ws,
+                    const float* __restrict__ gam_ws, const float* __restrict__ ds_ws,
+                    const int32_t* __restrict__ inv_off, const int32_t* __restrict__ inv_list,
+                    float* __restrict__ dK, float* __restrict__ dV, float* __restrict__ dklm,
+                    float* __restrict__ dblm) {
+  using SH = BwdShape<DD, T>;
+  constexpr int LD = SH::LD, LDA = SH::LDA, KPT = SH::KPT, DG = SH::DG;
+  extern __shared__ float4 smem_f4[];
+  float* sQ = reinterpret_cast<float*>(smem_f4);
+  float* sdO = sQ + SH::ROWS_F;
+  float* sK = sdO + SH::ROWS_F;
+  float* sV = sK + SH::KEYS_F;
+  float* sA = sV + SH::KEYS_F;
+  float* sdX = sA + SH::TILE_F;
+  int64_t* sPos = reinterpret_cast<int64_t*>(sdX + SH::TILE_F);   // [64]
+  float* sLam = reinterpret_cast<float*>(sPos + kBwdRows);         // [64]
+  float* sGam = sLam + kBwdRows;                                   // [64]
+  const TI** rowq = reinterpret_cast<const TI**>(sGam + kBwdRows);   // [64]
+  const TI** rowo = rowq + kBwdRows;                                 // [64]
+
+  const int tid = threadIdx.x;
+  const int tr = tid >> 4, tc = tid & 15;
+  const int G = D.G, Kt = D.K;
+  const int64_t bg = blockIdx.y, b = bg / D.Hkv, g = bg - b * D.Hkv;
+  const int64_t k0 = (int64_t)blockIdx.x * T;
+  const int64_t c = k0 / D.S;
+  const float sc2 = D.scale * kB2;
+  // window rows: positions [max(k0, q_pos0), min((c + 1) S + W - 2, last query)]
+  const int64_t p_lo = k0 > D.q_pos0 ? k0 : D.q_pos0;
+  const int64_t p_last = D.q_pos0 + D.N_q - 1;
+  const int64_t p_cap = (c + 1) * D.S + D.W - 2;
+  const int64_t p_hi = p_cap < p_last ? p_cap : p_last;
+  const int64_t n_win = p_hi >= p_lo ? p_hi - p_lo + 1 : 0;
+  int64_t e_lo = 0, n_inv = 0;
+  if (c < D.C && Kt > 0) {
+    e_lo = inv_off[bg * (D.C + 1) + c];
+    n_inv = inv_off[bg * (D.C + 1) + c + 1] - e_lo;
+  }
+  const int32_t* ents = inv_list + bg * D.N_q * Kt + e_lo;
+  const int64_t total = (n_win + n_inv) * G;
+
+  stage_keys<TI, DD, LD, T>(sK, K + bg * D.N_kv * DD, k0, D.N_kv);
+  stage_keys<TI, DD, LD, T>(sV, V + bg * D.N_kv * DD, k0, D.N_kv);
+  float aK[KPT][DG][4], aV[KPT][DG][4];
+#pragma unroll
+  for (int i = 0; i < KPT; ++i)
+#pragma unroll
+    for (int e = 0; e < DG; ++e)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) aK[i][e][v] = aV[i][e][v] = 0.f;
+
+  for (int64_t f0 = 0; f0 < total; f0 += kBwdRows) {
+    __syncthreads();   // the previous batch's tiles are consumed
+    if (tid < kBwdRows) {
+      const int64_t f = f0 + tid;
+      if (f < total) {
+        int64_t qi;
+        int u, h;
+        if (f < n_win * G) {
+          qi = p_lo - D.q_pos0 + f / G;
+          h = (int)(f % G);
+          u = Kt;
+        } else {
+          const int64_t fe = f - n_win * G;
+          const int32_t ent = ents[fe / G];
+          qi = ent / Kt;
+          u = ent - (int)qi * Kt;
+          h = (int)(fe % G);
+        }
+        const int64_t grow = (b * D.Hq + g * G + h) * D.N_q + qi;
+        sPos[tid] = D.q_pos0 + qi;
+        sLam[tid] = lam_ws[grow * (Kt + 1) + u];
+        sGam[tid] = gam_ws[grow * (Kt + 1) + u];
+        rowq[tid] = q + grow * DD;
+        rowo[tid] = dO + grow * DD;
+      } else {
+        sPos[tid] = INT64_MIN;
+        sLam[tid] = -INFINITY;
+        sGam[tid] = 0.f;
+        rowq[tid] = nullptr;
+        rowo[tid] = nullptr;
+      }
+    }
+    __syncthreads();
+    stage_rows<TI, DD, LD>(sQ, rowq, kBwdRows);
+    stage_rows<TI, DD, LD>(sdO, rowo, kBwdRows);
+    __syncthreads();
+    float X[4][KPT], P[4][KPT];
+    logits_tile<DD, T>(sQ, sdO, sK, sV, tr, tc, X, P);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = tr * 4 + i;
+      const int64_t pos = sPos[r];
+      const float lam2 = sLam[r], gam = sGam[r];
+#pragma unroll
+      for (int e = 0; e < KPT; ++e) {
+        const int64_t j = k0 + tc + 16 * e;
+        const bool ok = pos != INT64_MIN && j <= pos && j < D.N_kv && lam2 != -INFINITY;
+        const float a = ok ? exp2f(fmaf(X[i][e], sc2, lam2)) : 0.f;
+        sA[r * LDA + tc + 16 * e] = a;
+        sdX[r * LDA + tc + 16 * e] = a * (P[i][e] - gam);
+      }
+    }
+    __syncthreads();
+#pragma unroll 2
+    for (int r = 0; r < kBwdRows; ++r) {
+      float xs[KPT], as[KPT];
+#pragma unroll
+      for (int i = 0; i < KPT; ++i) {
+        xs[i] = sdX[r * LDA + tr * KPT + i];
+        as[i] = sA[r * LDA + tr * KPT + i];
+      }
+#pragma unroll
+      for (int e = 0; e < DG; ++e) {
+        const float4 qv = *reinterpret_cast<const float4*>(sQ + r * LD + tc * 4 + 64 * e);
+        const float4 ov = *reinterpret_cast<const float4*>(sdO + r * LD + tc * 4 + 64 * e);
+#pragma unroll
+        for (int i = 0; i < KPT; ++i) {
+          aK[i][e][0] = fmaf(xs[i], qv.x, aK[i][e][0]);
+          aK[i][e][1] = fmaf(xs[i], qv.y, aK[i][e][1]);
+          aK[i][e][2] = fmaf(xs[i], qv.z, aK[i][e][2]);
+          aK[i][e][3] = fmaf(xs[i], qv.w, aK[i][e][3]);
+          aV[i][e][0] = fmaf(as[i], ov.x, aV[i][e][0]);
+          aV[i][e][1] = fmaf(as[i], ov.y, aV[i][e][1]);
+          aV[i][e][2] = fmaf(as[i], ov.z, aV[i][e][2]);
+          aV[i][e][3] = fmaf(as[i], ov.w, aV[i][e][3]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < KPT; ++i) {
+    const int64_t j = k0 + tr * KPT + i;
+    if (j >= D.N_kv) continue;
+#pragma unroll
+    for (int e = 0; e < DG; ++e) {
+      const int64_t o = (bg * D.N_kv + j) * DD + tc * 4 + 64 * e;
+      *reinterpret_cast<float4*>(dK + o) =
+          make_float4(aK[i][e][0] * D.scale, aK[i][e][1] * D.scale, aK[i][e][2] * D.scale,
+                      aK[i][e][3] * D.scale);
+      *reinterpret_cast<float4*>(dV + o) =
+          make_float4(aV[i][e][0], aV[i][e][1], aV[i][e][2], aV[i][e][3]);
+    }
+  }
+
+  // d k_lm and d b_lm of chunk c: scale sum dscore q_cal and sum dscore over its selecting rows
+  if (c < D.C && k0 == c * D.S) {
+    constexpr int PARTS = kBwdThreads / DD;
+    const int dim = tid % DD, part = tid / DD;
+    float acc = 0.f, dsum = 0.f;
+    for (int64_t f = part; f < n_inv * G; f += PARTS) {
+      const int32_t ent = ents[f / G];
+      const int64_t qi = ent / Kt;
+      const int u = ent - (int)qi * Kt;
+      const int64_t grow = (b * D.Hq + g * G + f % G) * D.N_q + qi;
+      const float dsc = ds_ws[grow * Kt + u];
+      acc = fmaf(dsc, Elem<TI>::to_f(qc[grow * DD + dim]), acc);
+      dsum += dsc;
+    }
+    __syncthreads();
+    float* red = sA;   // [PARTS][DD + 1]
+    red[part * (DD + 1) + dim] = acc;
+    if (dim == 0) red[part * (DD + 1) + DD] = dsum;
+    __syncthreads();
+    if (part == 0) {
+      float a = 0.f;
+      for (int p2 = 0; p2 < PARTS; ++p2) a += red[p2 * (DD + 1) + dim];
+      dklm[(bg * D.C + c) * DD + dim] = a * D.scale;
+      if (dim == 0) {
+        float t = 0.f;
+        for (int p2 = 0; p2 < PARTS; ++p2) t += red[p2 * (DD + 1) + DD];
+        dblm[bg * D.C + c] = t;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Inverse index: per (b, g) and chunk c the entries i * K + slot of the queries that selected c.
+__global__ void __launch_bounds__(256)
+    inv_count_kernel(Dims D, const int32_t* __restrict__ idx, int32_t* __restrict__ cnt) {
+  const int64_t per = D.N_q * D.K;
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= D.B * D.Hkv * per) return;
+  const int32_t c = idx[e];
+  if (c >= 0 && c < D.C) atomicAdd(&cnt[(e / per) * D.C + c], 1);
+}
+
+__global__ void __launch_bounds__(1024)
+    inv_scan_kernel(Dims D, const int32_t* __restrict__ cnt, int32_t* __restrict__ off) {
+  __shared__ int32_t wsum[32];
+  const int64_t bg = blockIdx.x;
+  const int64_t C = D.C;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t seg = (C + 1023) / 1024;
+  const int64_t lo = tid * seg < C ? tid * seg : C;
+  const int64_t hi = lo + seg < C ? lo + seg : C;
+  const int32_t* cb = cnt + bg * C;
+  int32_t s = 0;
+  for (int64_t x = lo; x < hi; ++x) s += cb[x];
+  // exclusive scan of the per-thread sums
+  int32_t inc = s;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) wsum[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t w = wsum[lane];
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    wsum[lane] = w;
+  }
+  __syncthreads();
+  int32_t run = inc - s + (warp > 0 ? wsum[warp - 1] : 0);
+  int32_t* ob = off + bg * (C + 1);
+  for (int64_t x = lo; x < hi; ++x) {
+    ob[x] = run;
+    run += cb[x];
+  }
+  if (tid == 1023) ob[C] = run;
+}
+
+__global__ void __launch_bounds__(256)
+    inv_fill_kernel(Dims D, const int32_t* __restrict__ idx, const int32_t* __restrict__ off,
+                    int32_t* __restrict__ cur, int32_t* __restrict__ list) {
+  const int64_t per = D.N_q * D.K;
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= D.B * D.Hkv * per) return;
+  const int32_t c = idx[e];
+  if (c < 0 || c >= D.C) return;
+  const int64_t bg = e / per;
+  const int32_t slot = atomicAdd(&cur[bg * D.C + c], 1);
+  list[bg * per + off[bg * (D.C + 1) + c] + slot] = (int32_t)(e - bg * per);
+}
+
+
+// ---------------------------------------------------------------------------------------------
+namespace {
+
+template <int DD, int T>
+constexpr size_t rows_smem() {
+  using SH = BwdShape<DD, T>;
+  return (size_t)(2 * SH::ROWS_F + 2 * SH::KEYS_F + SH::TILE_F + 3 * kBwdRows * (kBwdMaxK + 1) +
+                  kBwdRows * kBwdMaxK) * 4 +
+         (size_t)2 * kBwdMaxUnion * 4 + kBwdRows * 8 + kBwdRows * 4 + kBwdRows * 4 + 8 +
+         kBwdRows * 8 + 16;
+}
+
+template <int DD, int T>
+constexpr size_t keys_smem() {
+  using SH = BwdShape<DD, T>;
+  return (size_t)(2 * SH::ROWS_F + 2 * SH::KEYS_F + 2 * SH::TILE_F) * 4 + kBwdRows * 8 +
+         2 * kBwdRows * 4 + 2 * kBwdRows * 8;
+}
+
+template <typename TI, int DD, int T>
+cudaError_t launch_bwd_t(const Dims& D, const BwdArgs& a, const BwdWs& w, cudaStream_t st) {
+  constexpr size_t RS = rows_smem<DD, T>(), KS = keys_smem<DD, T>();
+  static_assert(RS <= 227 * 1024 && KS <= 227 * 1024, "shared memory");
+  auto kr = bwd_rows_kernel<TI, DD, T>;
+  auto kk = bwd_keys_kernel<TI, DD, T>;
+  cudaError_t e = cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RS);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KS);
+  if (e != cudaSuccess) return e;
+  const TI* q = static_cast<const TI*>(a.q);
+  const TI* qc = static_cast<const TI*>(a.q_cal);
+  const TI* K = static_cast<const TI*>(a.K);
+  const TI* V = static_cast<const TI*>(a.V);
+  const TI* klm = static_cast<const TI*>(a.k_lm);
+  const TI* dO = static_cast<const TI*>(a.dout);
+  const int QT = kBwdRows / D.G;
+  if (D.N_q > 0) {
+    const dim3 gr((unsigned)((D.N_q + QT - 1) / QT), (unsigned)(D.B * D.Hkv));
+    kr<<<gr, kBwdThreads, RS, st>>>(D, q, qc, K, V, klm, a.b_lm, a.idx, dO, a.dlse, a.dq, a.dq_cal,
+                                    w.lam, w.gam, w.ds);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  const dim3 gk((unsigned)((D.N_kv + T - 1) / T), (unsigned)(D.B * D.Hkv));
+  kk<<<gk, kBwdThreads, KS, st>>>(D, q, qc, K, V, dO, w.lam, w.gam, w.ds, w.inv_off, w.inv_list,
+                                  a.dK, a.dV, a.dk_lm, a.db_lm);
+  return cudaGetLastError();
+}
+
+template <typename TI>
+cudaError_t launch_bwd_d(const Dims& D, const BwdArgs& a, const BwdWs& w, cudaStream_t st) {
+  const int T = D.S < 64 ? D.S : 64;
+  if (D.d == 128) {
+    if (T == 64) return launch_bwd_t<TI, 128, 64>(D, a, w, st);
+    if (T == 32) return launch_bwd_t<TI, 128, 32>(D, a, w, st);
+    return launch_bwd_t<TI, 128, 16>(D, a, w, st);
+  }
+  if (T == 64) return launch_bwd_t<TI, 64, 64>(D, a, w, st);
+  if (T == 32) return launch_bwd_t<TI, 64, 32>(D, a, w, st);
+  return launch_bwd_t<TI, 64, 16>(D, a, w, st);
+}
+
+}  // namespace
+
+bool backward_supported(const Dims& D) {
+  if (D.d != 64 && D.d != 128) return false;
+  if (D.S != 16 && D.S != 32 && D.S != 64 && D.S != 128) return false;
+  if (D.G < 1 || D.G > kBwdRows || kBwdRows % D.G != 0) return false;
+  if (D.K < 0 || D.K > kBwdMaxK) return false;
+  if (D.B * D.Hkv > 65535) return false;
+  if (D.N_q * (int64_t)(D.K > 0 ? D.K : 1) >= (int64_t)INT32_MAX) return false;
+  if ((D.N_kv + 15) / 16 >= (int64_t)INT32_MAX) return false;
+  return true;
+}
+
+size_t backward_ws_layout(const Dims& D, BwdWs* w, char* base) {
+  const int64_t R = D.B * D.Hq * D.N_q;
+  const int64_t BG = D.B * D.Hkv;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 255) & ~size_t(255);
+    return base ? base + o : nullptr;
+  };
+  char* lam = take((size_t)R * (D.K + 1) * 4);
+  char* gam = take((size_t)R * (D.K + 1) * 4);
+  char* ds = take((size_t)R * (D.K > 0 ? D.K : 1) * 4);
+  char* cnt = take((size_t)BG * (D.C > 0 ? D.C : 1) * 4);
+  char* cur = take((size_t)BG * (D.C > 0 ? D.C : 1) * 4);
+  char* ioff = take((size_t)BG * (D.C + 1) * 4);
+  char* list = take((size_t)BG * D.N_q * (D.K > 0 ? D.K : 1) * 4);
+  if (w) {
+    w->lam = reinterpret_cast<float*>(lam);
+    w->gam = reinterpret_cast<float*>(gam);
+    w->ds = reinterpret_cast<float*>(ds);
+    w->inv_cnt = reinterpret_cast<int32_t*>(cnt);
+    w->inv_cur = reinterpret_cast<int32_t*>(cur);
+    w->inv_off = reinterpret_cast<int32_t*>(ioff);
+    w->inv_list = reinterpret_cast<int32_t*>(list);
+  }
+  return off;
+}
+
+cudaError_t launch_backward(const Dims& D, bool bf16, const BwdArgs& a, const BwdWs& w,
+                            cudaStream_t st) {
+  const int64_t BG = D.B * D.Hkv;
+  cudaError_t e = cudaSuccess;
+  if (D.K > 0 && D.C > 0 && D.N_q > 0) {
+    e = cudaMemsetAsync(w.inv_cnt, 0, (size_t)BG * D.C * 4, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(w.inv_cur, 0, (size_t)BG * D.C * 4, st);
+    if (e != cudaSuccess) return e;
+    const int64_t n = BG * D.N_q * D.K;
+    const unsigned grid = (unsigned)((n + 255) / 256);
+    inv_count_kernel<<<grid, 256, 0, st>>>(D, a.idx, w.inv_cnt);
+    inv_scan_kernel<<<(unsigned)BG, 1024, 0, st>>>(D, w.inv_cnt, w.inv_off);
+    inv_fill_kernel<<<grid, 256, 0, st>>>(D, a.idx, w.inv_off, w.inv_cur, w.inv_list);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  } else if (D.C > 0) {
+    // no selections: every chunk's list is empty
+    e = cudaMemsetAsync(w.inv_off, 0, (size_t)BG * (D.C + 1) * 4, st);
+    if (e != cudaSuccess) return e;
+  }
+  return bf16 ? launch_bwd_d<__nv_bfloat16>(D, a, w, st) : launch_bwd_d<float>(D, a, w, st);
+}
+
+}  // namespace hils

@@ -87,6 +87,26 @@ cudaError_t launch_landmarks(const Dims& D, bool bf16, int64_t c0, int64_t nc,
 cudaError_t launch_append_kv(const Dims& D, bool bf16, int64_t pos, const void* k_new,
                              const void* v_new, void* K, void* V, cudaStream_t st);
 
+// Backward pass (csrc/bwd.cu).  Inputs in the forward's dtype except b_lm / dlse (fp32); every
+// gradient fp32, overwritten.
+struct BwdArgs {
+  const void *q, *q_cal, *K, *V, *k_lm;
+  const float* b_lm;
+  const int32_t* idx;
+  const void* dout;
+  const float* dlse;   // nullable
+  float *dq, *dq_cal, *dK, *dV, *dk_lm, *db_lm;
+};
+struct BwdWs {
+  float *lam, *gam, *ds;              // per (row, unit): lambda * log2(e), gamma; dscore
+  int32_t *inv_cnt, *inv_cur, *inv_off, *inv_list;   // chunk -> selecting (query, slot)
+};
+bool backward_supported(const Dims& D);
+// Bytes of the backward's workspace; with base != nullptr also carves it into *w.
+size_t backward_ws_layout(const Dims& D, BwdWs* w, char* base);
+cudaError_t launch_backward(const Dims& D, bool bf16, const BwdArgs& a, const BwdWs& w,
+                            cudaStream_t st);
+
 // One CTA waits on an mbarrier phase for at most `polls` polls (completed first if `complete`);
 // a wait that gives up records HILS_ERR_TIMEOUT in *status.
 cudaError_t launch_wait_check(uint32_t polls, int complete, int32_t* status, cudaStream_t st);

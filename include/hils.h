@@ -177,6 +177,39 @@ hils_status hils_decode_step(const hils_params* p, const void* q, const void* q_
                              size_t workspace_bytes, hils_stream_t stream);
 
 /*
+ * Backward pass: the gradients of L = sum dout . out + sum dlse . lse (out, lse as hils_forward
+ * computes them) with respect to q, q_cal, K, V, k_lm and b_lm, with the selection topk_idx held
+ * fixed.  The top-K is piecewise constant in its inputs and passes no gradient; the landmark keys
+ * and biases receive theirs through the fusion weights ([Reader] Fig. 3 caption: the loss
+ * gradient flows back to the compressed key; "The HiLS-Attention Mechanism": the surrogate is
+ * differentiable where the exact chunk mass is not).  By the chain rule through steps 4, 1 and
+ * 3, per query-head row with units u (the selected chunks, then the window) and fused weights w:
+ *   d score_u = w_u (dout . o_u - dout . out + dlse);  a chunk's score passes it to q_cal, k_lm
+ *   and b_lm; the window's score is its own lse and passes it to the window's token logits;
+ *   dV_j += a_j dout, d x_j = a_j (dout . V_j - dout . o_u) (+ a_j d score_window for window
+ *   tokens), a_j = w_u exp(x_j - lse_u) the token's fused weight.
+ * Inputs as for hils_forward (p, q, q_cal, K, V, k_lm, b_lm, same dtype); topk_idx [B, Hkv, N_q,
+ * K_top] int32 the forward's selection (ids outside a query's eligible chunks count as empty
+ * slots and a repeated id is attended once; the forward never writes either); dout [B, Hq, N_q,
+ * d] in dtype; dlse [B, Hq, N_q] fp32 or NULL (zero).  Outputs, all fp32 and every element
+ * written: dq, dq_cal [B, Hq, N_q, d]; dK, dV [B, Hkv, N_kv, d]; dk_lm [B, Hkv, C, d]; db_lm
+ * [B, Hkv, C].  Workspace: hils_backward_workspace_size(p) bytes, 16-byte aligned (per-row
+ * fusion terms, 4 (2 K_top + 3) bytes per query-head, and a chunk -> selecting-query index,
+ * 4 K_top bytes per query and KV head).  Supported: d = 64 or 128, S in {16, 32, 64, 128},
+ * G = Hq / Hkv dividing 64, K_top <= 32; else HILS_ERR_UNSUPPORTED.  Every gradient is a sum
+ * formed in one thread's registers (no atomics), but the order in which the rows that selected a
+ * chunk reach the K, V, k_lm and b_lm gradients follows the index build and may differ between
+ * runs, so those four can differ between runs in the last bits.  Asynchronous on `stream`.
+ */
+size_t hils_backward_workspace_size(const hils_params* p);
+hils_status hils_backward(const hils_params* p, const void* q, const void* q_cal, const void* K,
+                          const void* V, const void* k_lm, const float* b_lm,
+                          const int32_t* topk_idx, const void* dout, const float* dlse,
+                          float* dq, float* dq_cal, float* dK, float* dV, float* dk_lm,
+                          float* db_lm, void* workspace, size_t workspace_bytes,
+                          hils_stream_t stream);
+
+/*
  * hils_select without a caller-provided workspace.  The paper has no counterpart: this entry
  * point exists for callers that cannot allocate device memory or pass a scratch buffer, e.g. a
  * plugin host that hands a kernel only its input and output tensors, or a serving loop whose
