@@ -68,6 +68,15 @@ def lib():
         l.hils_oracle_backward.restype = ctypes.c_int
         l.hils_oracle_backward.argtypes = [ctypes.POINTER(Problem)] + [ctypes.c_void_p] * 15 + [
             ctypes.c_int]
+        l.hils_oracle_hope_rotates.restype = ctypes.c_int
+        l.hils_oracle_hope_rotates.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_double,
+                                               ctypes.c_double]
+        l.hils_oracle_hope_rotate.restype = ctypes.c_int
+        l.hils_oracle_hope_rotate.argtypes = [ctypes.c_int64] * 5 + [ctypes.c_double] * 2 + [
+            ctypes.c_void_p] * 2
+        l.hils_oracle_qcal_hope.restype = ctypes.c_int
+        l.hils_oracle_qcal_hope.argtypes = [ctypes.c_int64] * 7 + [ctypes.c_double] * 2 + [
+            ctypes.c_void_p] * 6
         l.hils_oracle_n_eligible.restype = ctypes.c_int64
         l.hils_oracle_n_eligible.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32]
         l.hils_oracle_default_threads.restype = ctypes.c_int
@@ -170,6 +179,40 @@ def backward(q, qc, K, V, klm, blm, idx, dO, dlse=None, *, S, K_top, W, q_pos0=0
     if rc != 0:
         raise RuntimeError("hils_oracle_backward failed with status %d" % rc)
     return r
+
+
+def hope_rotates(m, d, base, train_len):
+    """HoPE (R17): whether dimension pair (m, m + d/2) rotates."""
+    return bool(lib().hils_oracle_hope_rotates(m, d, float(base), float(train_len)))
+
+
+def hope_rotate(x, *, base, train_len, pos0=0):
+    """HoPE (R17) of x [B, H, N, d], token n at position pos0 + n."""
+    x = _f64(x)
+    B, H, N, d = x.shape
+    out = np.empty_like(x)
+    rc = lib().hils_oracle_hope_rotate(B, H, N, d, pos0, float(base), float(train_len),
+                                       _ptr(x), _ptr(out))
+    if rc != 0:
+        raise RuntimeError("hils_oracle_hope_rotate failed with status %d" % rc)
+    return out
+
+
+def qcal_hope(q, hidden, W_down, W_up, *, base, train_len, pos0=0):
+    """Q-Cal and HoPE: q [B,Hq,N_q,d], hidden [B,N_q,d_model], W_down [Hq,r,d_model], W_up
+    [Hq,d,r].  Returns (HoPE(q), HoPE(q + W_up W_down hidden)) at positions pos0 + i."""
+    q, hidden, W_down, W_up = (_f64(x) for x in (q, hidden, W_down, W_up))
+    B, Hq, Nq, d = q.shape
+    dm = hidden.shape[2]
+    r = W_down.shape[1]
+    assert hidden.shape == (B, Nq, dm) and W_down.shape == (Hq, r, dm) and W_up.shape == (Hq, d, r)
+    q_out, qc_out = np.empty_like(q), np.empty_like(q)
+    rc = lib().hils_oracle_qcal_hope(B, Hq, Nq, d, dm, r, pos0, float(base), float(train_len),
+                                     _ptr(q), _ptr(hidden), _ptr(W_down), _ptr(W_up),
+                                     _ptr(q_out), _ptr(qc_out))
+    if rc != 0:
+        raise RuntimeError("hils_oracle_qcal_hope failed with status %d" % rc)
+    return q_out, qc_out
 
 
 class Query:

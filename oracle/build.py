@@ -9,7 +9,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 BUILD_DIR = os.path.join(HERE, "_build")
 LIB_PATH = os.path.join(BUILD_DIR, "libhils_oracle.so")
-SOURCES = [os.path.join(HERE, "hils_oracle.c"), os.path.join(HERE, "hils_oracle_bwd.c")]
+SOURCES = [os.path.join(HERE, "hils_oracle.c"), os.path.join(HERE, "hils_oracle_bwd.c"),
+           os.path.join(HERE, "hils_oracle_prologue.c")]
 HEADERS = [os.path.join(HERE, "hils_oracle.h")]
 
 

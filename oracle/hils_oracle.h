@@ -63,6 +63,9 @@
  * the selection held fixed (R16: the top-K passes no gradient; the landmark keys and biases
  * receive theirs through the fusion weights, [Reader] Fig. 3 caption).
  *
+ * Query prologue (hils_oracle_prologue.c): Q-Cal's low-rank correction of the query from the
+ * hidden state and HoPE's partial rotary encoding (R17), the producers of q_cal and q.
+ *
  * Every function here is pinned by CPU tests against values the pages print, closed forms
  * and brute force (no function is "parity unpinned").
  */
@@ -161,6 +164,20 @@ int hils_oracle_backward(const hils_oracle_problem* pr, const double* q, const d
                          const int32_t* idx, const double* dO, const double* dlse, double* dq,
                          double* dqc, double* dK, double* dV, double* dklm, double* dblm,
                          int n_threads);
+
+/* Query prologue (hils_oracle_prologue.c), reading R17.  HoPE: pair (m, m + d/2), m < d/2,
+ * turns by pos * base^(-2m/d) iff its period 2 pi base^(2m/d) <= train_len.
+ * hils_oracle_hope_rotate: x, out [B, H, N, d]; token n at position pos0 + n.
+ * hils_oracle_qcal_hope: q [B,Hq,N_q,d], hidden [B,N_q,d_model], W_down [Hq,r,d_model],
+ * W_up [Hq,d,r]; q_out = HoPE(q), qc_out = HoPE(q + W_up (W_down hidden)) at position
+ * pos0 + i. */
+int hils_oracle_hope_rotates(int64_t m, int64_t d, double base, double train_len);
+int hils_oracle_hope_rotate(int64_t B, int64_t H, int64_t N, int64_t d, int64_t pos0,
+                            double base, double train_len, const double* x, double* out);
+int hils_oracle_qcal_hope(int64_t B, int64_t Hq, int64_t N_q, int64_t d, int64_t d_model,
+                          int64_t r, int64_t pos0, double base, double train_len,
+                          const double* q, const double* hidden, const double* W_down,
+                          const double* W_up, double* q_out, double* qc_out);
 
 /* Rule R1: number of eligible distant chunks of the query at position pos. */
 int64_t hils_oracle_n_eligible(int64_t pos, int32_t S, int32_t W);
