@@ -709,6 +709,45 @@ def extra_backward(peaks, name="gqa7b_prefill", steps=3, **overrides):
     return out
 
 
+def extra_prologue(peaks, B=1, Hq=32, N=131072, d=128, d_model=4096, r=16, steps=5):
+    """hils_qcal_hope at the 7B-like prefill shape: the down-projection GEMM
+    ([B N, d_model] x [Hq r, d_model]^T, tcgen05) and the fused up-projection + HoPE pass
+    (q read, u read, q and q_cal written)."""
+    from hierarchical_chunk_sparse_scoring_b200 import binding as hb
+    g = torch.Generator(device="cuda").manual_seed(21)
+    bf = torch.bfloat16
+    q = (torch.randn((B, Hq, N, d), generator=g, device="cuda") / math.sqrt(d)).to(bf)
+    hidden = torch.randn((B, N, d_model), generator=g, device="cuda").to(bf)
+    W_down = (torch.randn((Hq, r, d_model), generator=g, device="cuda") /
+              math.sqrt(d_model)).to(bf)
+    W_up = (0.1 * torch.randn((Hq, d, r), generator=g, device="cuda")).to(bf)
+    q_out, q_cal = torch.empty_like(q), torch.empty_like(q)
+    kw = dict(rope_base=10000.0, train_len=32768.0, q_out=q_out, q_cal_out=q_cal)
+    hb.qcal_hope(q, hidden, W_down, W_up, **kw)
+    flush = make_flush(q.device)
+    ms = []
+    for _ in range(steps):
+        flush()
+        a, b_ = make_events(2)
+        a.record()
+        hb.qcal_hope(q, hidden, W_down, W_up, **kw)
+        b_.record()
+        torch.cuda.synchronize()
+        ms.append(a.elapsed_time(b_))
+    t = statistics.mean(ms)
+    gemm_flops = 2.0 * B * N * Hq * r * d_model
+    gemm_bytes = B * N * d_model * 2 + Hq * r * d_model * 2 + B * N * Hq * r * 4
+    pass_bytes = B * Hq * N * d * 2 * 3 + B * N * Hq * r * 4
+    # lower bound of the pair: the GEMM at the bf16 peak plus the pass at the HBM peak
+    floor_ms = (gemm_flops / (peaks["bf16_tflops"] * 1e12) +
+                (gemm_bytes + pass_bytes) / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    del q, hidden, W_down, W_up, q_out, q_cal
+    torch.cuda.empty_cache()
+    return {"kernel": "qdown (tcgen05) + qcal_hope", "shape": {"B": B, "Hq": Hq, "N": N, "d": d,
+            "d_model": d_model, "r": r}, "ms": t, "gemm_tflop": gemm_flops / 1e12,
+            "bytes": gemm_bytes + pass_bytes, "floor_ms": floor_ms, "frac_of_floor": floor_ms / t}
+
+
 def run_hils(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -787,6 +826,7 @@ def run_hils(args):
         line["landmarks"] = [extra_landmarks(peaks, 1, 1, 1 << 22, 128, 128),
                              extra_landmarks(peaks, 1, 8, 131072, 128, 64)]
         line["backward_gqa7b"] = extra_backward(peaks, "gqa7b_prefill")
+        line["prologue_gqa7b"] = extra_prologue(peaks)
     if dist:
         dist.destroy_process_group()
     if rank == 0:

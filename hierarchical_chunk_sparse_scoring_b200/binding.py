@@ -33,6 +33,12 @@ class Params(ctypes.Structure):
                 ("W", ctypes.c_int32), ("dtype", ctypes.c_int32), ("scale", ctypes.c_float)]
 
 
+class PrologueParams(ctypes.Structure):
+    """hils_prologue_params (include/hils.h)."""
+    _fields_ = [("d_model", ctypes.c_int64), ("r", ctypes.c_int32),
+                ("rope_base", ctypes.c_double), ("train_len", ctypes.c_double)]
+
+
 # every function the header declares, with its ctypes signature
 _P = ctypes.POINTER(Params)
 _V = ctypes.c_void_p
@@ -50,6 +56,12 @@ SIGNATURES = {
     "hils_decode_step": (ctypes.c_int, [_P] + [_V] * 13 + [ctypes.c_size_t, _V]),
     "hils_wait_check": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_int, _V, ctypes.c_size_t, _V]),
     "hils_backward_workspace_size": (ctypes.c_size_t, [_P]),
+    "hils_qcal_workspace_size": (ctypes.c_size_t, [_P, ctypes.POINTER(PrologueParams)]),
+    "hils_qcal_hope": (ctypes.c_int, [_P, ctypes.POINTER(PrologueParams)] + [_V] * 7 +
+                       [ctypes.c_size_t, _V]),
+    "hils_hope_rotate": (ctypes.c_int, [_P, ctypes.POINTER(PrologueParams), ctypes.c_int64,
+                                        ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, _V, _V,
+                                        _V]),
     "hils_backward": (ctypes.c_int, [_P] + [_V] * 16 + [ctypes.c_size_t, _V]),
     "hils_chunk_attn": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V, _V]),
     "hils_fuse": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V]),
@@ -278,6 +290,48 @@ def decode_step(q, q_cal, k_new, v_new, q_lm_new, K, V, k_lm, b_lm, *, pos, S, K
                                   _ptr(idx), _ptr(ws), ws.numel(), _stream(stream)),
            "hils_decode_step")
     return out, lse, idx
+
+
+def qcal_hope(q, hidden, W_down, W_up, *, rope_base, train_len, q_pos0=0, q_out=None,
+              q_cal_out=None, ws=None, stream=None):
+    """hils_qcal_hope: (HoPE(q), HoPE(q + W_up W_down hidden)) for query i at q_pos0 + i.
+    q [B,Hq,N_q,d] and W_up [Hq,d,r] in the model dtype; hidden [B,N_q,d_model] and W_down
+    [Hq,r,d_model] bf16 (W_down / W_up may be None for r = 0)."""
+    B, Hq, N_q, d = q.shape
+    _need(q, "q")
+    r = 0 if W_down is None else W_down.shape[1]
+    d_model = 0 if hidden is None else hidden.shape[2]
+    if r > 0:
+        _need(hidden, "hidden", torch.bfloat16, (B, N_q, d_model))
+        _need(W_down, "W_down", torch.bfloat16, (Hq, r, d_model))
+        _need(W_up, "W_up", q.dtype, (Hq, d, r))
+    p = make_params(B, Hq, Hq, N_q, max(N_q + q_pos0, 1), d, S=1, K_top=0, W=1, q_pos0=q_pos0,
+                    dtype=q.dtype)
+    c = PrologueParams(d_model, r, float(rope_base), float(train_len))
+    if q_out is None:
+        q_out = torch.empty_like(q)
+    if q_cal_out is None:
+        q_cal_out = torch.empty_like(q)
+    if ws is None:
+        need = int(lib().hils_qcal_workspace_size(ctypes.byref(p), ctypes.byref(c)))
+        ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=q.device)
+    _check(lib().hils_qcal_hope(ctypes.byref(p), ctypes.byref(c), _ptr(q), _ptr(hidden),
+                                _ptr(W_down), _ptr(W_up), _ptr(q_out), _ptr(q_cal_out), _ptr(ws),
+                                ws.numel(), _stream(stream)), "hils_qcal_hope")
+    return q_out, q_cal_out
+
+
+def hope_rotate(x, *, rope_base, train_len, pos0=0, out=None, stream=None):
+    """hils_hope_rotate: HoPE of x [B,H,N,d], token n at position pos0 + n."""
+    B, H, N, d = x.shape
+    _need(x, "x")
+    p = make_params(1, 1, 1, 1, 1, d, S=1, K_top=0, W=1, dtype=x.dtype)
+    c = PrologueParams(0, 0, float(rope_base), float(train_len))
+    if out is None:
+        out = torch.empty_like(x)
+    _check(lib().hils_hope_rotate(ctypes.byref(p), ctypes.byref(c), B, H, N, pos0, _ptr(x),
+                                  _ptr(out), _stream(stream)), "hils_hope_rotate")
+    return out
 
 
 def backward_workspace(p, device):

@@ -442,6 +442,79 @@ extern "C" hils_status hils_decode_step(const hils_params* p, const void* q, con
                       workspace_bytes, stream, nullptr, 0);
 }
 
+namespace hils {
+namespace {
+hils_status check_prologue(const hils_params* p, const hils_prologue_params* c) {
+  hils_status s = check_params(p);
+  if (s != HILS_OK) return s;
+  if (!c || !(c->rope_base > 1.0) || std::isnan(c->train_len) || c->r < 0 || c->d_model < 0)
+    return HILS_ERR_INVALID_ARG;
+  if (p->d != 64 && p->d != 128) return HILS_ERR_UNSUPPORTED;
+  if (c->r > 64) return HILS_ERR_UNSUPPORTED;
+  if (c->r > 0 && !qdown_supported(p->Hq * c->r, c->d_model)) return HILS_ERR_UNSUPPORTED;
+  if (p->B * p->N_q >= (int64_t)INT32_MAX || p->Hq > 65535 || p->B > 65535)
+    return HILS_ERR_UNSUPPORTED;
+  return HILS_OK;
+}
+}  // namespace
+}  // namespace hils
+
+extern "C" size_t hils_qcal_workspace_size(const hils_params* p, const hils_prologue_params* c) {
+  if (check_prologue(p, c) != HILS_OK) return 0;
+  return kStatusBytes + align_up((size_t)(p->B * p->N_q * p->Hq) * (size_t)c->r * 4);
+}
+
+extern "C" hils_status hils_qcal_hope(const hils_params* p, const hils_prologue_params* c,
+                                      const void* q, const void* hidden, const void* W_down,
+                                      const void* W_up, void* q_out, void* q_cal_out,
+                                      void* workspace, size_t workspace_bytes,
+                                      hils_stream_t stream) {
+  hils_status s = check_prologue(p, c);
+  if (s != HILS_OK) return s;
+  const bool any = p->B > 0 && p->N_q > 0;
+  const bool qcal = any && c->r > 0;
+  if (!ok_ptr(q, any) || !ok_ptr(q_out, any) || !ok_ptr(q_cal_out, any) ||
+      !ok_ptr(hidden, qcal) || !ok_ptr(W_down, qcal) || !ok_ptr(W_up, qcal))
+    return HILS_ERR_INVALID_ARG;
+  if (q_cal_out == q) return HILS_ERR_INVALID_ARG;
+  const size_t need = hils_qcal_workspace_size(p, c);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < need) return HILS_ERR_WORKSPACE;
+  if (!any) return HILS_OK;
+  if ((s = check_device()) != HILS_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  float* u = reinterpret_cast<float*>(ws + kStatusBytes);
+  cudaError_t e = cudaSuccess;
+  if (qcal)
+    e = launch_qdown(p->B * p->N_q, p->Hq * c->r, c->d_model, hidden, W_down, u,
+                     reinterpret_cast<int32_t*>(ws), st);
+  if (e == cudaSuccess)
+    e = launch_qcal_hope(p->B, p->Hq, p->N_q, p->d, p->q_pos0, c->r, c->rope_base,
+                         c->train_len, p->dtype == HILS_BF16, q, u, W_up, q_out, q_cal_out, st);
+  return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA;
+}
+
+extern "C" hils_status hils_hope_rotate(const hils_params* p, const hils_prologue_params* c,
+                                        int64_t B, int64_t H, int64_t N, int64_t pos0,
+                                        const void* x, void* x_out, hils_stream_t stream) {
+  hils_status s = check_params(p);
+  if (s != HILS_OK) return s;
+  if (!c || !(c->rope_base > 1.0) || std::isnan(c->train_len) || B < 0 || H < 0 || N < 0 ||
+      pos0 < 0)
+    return HILS_ERR_INVALID_ARG;
+  if (p->d != 64 && p->d != 128) return HILS_ERR_UNSUPPORTED;
+  if (B * H > 65535) return HILS_ERR_UNSUPPORTED;
+  const bool any = B > 0 && H > 0 && N > 0;
+  if (!ok_ptr(x, any) || !ok_ptr(x_out, any)) return HILS_ERR_INVALID_ARG;
+  if (!any) return HILS_OK;
+  if ((s = check_device()) != HILS_OK) return s;
+  return launch_hope_rotate(B * H, N, p->d, pos0, c->rope_base, c->train_len,
+                            p->dtype == HILS_BF16, x, x_out,
+                            reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? HILS_OK
+             : HILS_ERR_CUDA;
+}
+
 extern "C" size_t hils_backward_workspace_size(const hils_params* p) {
   if (check_params(p) != HILS_OK) return 0;
   const Plan P = make_plan(p);

@@ -107,6 +107,19 @@ size_t backward_ws_layout(const Dims& D, BwdWs* w, char* base);
 cudaError_t launch_backward(const Dims& D, bool bf16, const BwdArgs& a, const BwdWs& w,
                             cudaStream_t st);
 
+// Query prologue (csrc/prologue.cu).  u [M, N] fp32 = hidden [M, d_model] x W_down [N,
+// d_model]^T (bf16 operands, tcgen05); q_cal = R(q + W_up u), q = R(q) per head; R = HoPE.
+bool qdown_supported(int64_t N, int64_t d_model);
+cudaError_t launch_qdown(int64_t M, int64_t N, int64_t d_model, const void* hidden,
+                         const void* W_down, float* u, int32_t* status, cudaStream_t st);
+cudaError_t launch_qcal_hope(int64_t B, int64_t Hq, int64_t N_q, int64_t d, int64_t q_pos0,
+                             int r, double base, double train_len, bool bf16, const void* q,
+                             const float* u, const void* W_up, void* q_out, void* qc_out,
+                             cudaStream_t st);
+cudaError_t launch_hope_rotate(int64_t BH, int64_t N, int64_t d, int64_t pos0, double base,
+                               double train_len, bool bf16, const void* x, void* out,
+                               cudaStream_t st);
+
 // One CTA waits on an mbarrier phase for at most `polls` polls (completed first if `complete`);
 // a wait that gives up records HILS_ERR_TIMEOUT in *status.
 cudaError_t launch_wait_check(uint32_t polls, int complete, int32_t* status, cudaStream_t st);

@@ -1,0 +1,352 @@
+// Query prologue, upstream of steps 1 and 3: Q-Cal and HoPE.
+//
+// Q-Cal ([Reader] "Implementation and Training Recipes", Q-Cal worked example): per query head h
+// the calibrated query adds a low-rank correction computed from the token's hidden state,
+// q_cal = q + W_up[h] (W_down[h] hidden), W_down[h]: r x d_model, W_up[h]: d x r.
+// HoPE ([Reader] same section, HoPE vs RoPE; [Essay] "Hierarchical Positional Encoding"): the
+// dimension pairs (m, m + d/2) whose rotation period 2 pi base^(2m/d) fits the training length
+// turn by pos * base^(-2m/d); the others are left as they are (NoPE).  q and q_cal are turned at
+// the query's position, keys at their own (hope_rotate).
+//
+// Two kernels:
+//   qdown_kernel   u = hidden W_down^T for all heads at once: [B N_q, d_model] x [Hq r, d_model]^T,
+//                  a dense contraction on the tcgen05 tensor cores (bf16 operands by TMA with the
+//                  128-byte swizzle, fp32 accumulator in TMEM, 128 x BN tiles, a 4-stage ring).
+//   qcal_hope_kernel  per (b, h, 32 tokens): q_cal = R(q + W_up u), q = R(q); HBM-bound (q read,
+//                  both written, u read); W_up[h] staged transposed in shared memory; each lane
+//                  owns whole rotation pairs, the angle p theta_m reduced modulo 2 pi in fp64
+//                  (p up to 2^22 makes an fp32 product lose whole radians) before sincosf.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace hils {
+using namespace sm100;
+
+namespace {
+
+constexpr uint32_t kPrPollLimit = 1u << 24;
+constexpr int kQdBM = 128;        // token rows per tile (M)
+constexpr int kQdThreads = 192;   // TMA warp, MMA warp, 4 epilogue warps
+constexpr double kTwoPi = 6.283185307179586476925286766559;
+
+template <int BN>
+struct QdShape {
+  static constexpr int A_BYTES = kQdBM * 128;   // 128 rows x 64 bf16
+  static constexpr int B_BYTES = BN * 128;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int STAGES = 4;
+  static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
+  static constexpr uint32_t TMEM_COLS = BN;
+  static_assert(BN == 64 || BN == 128 || BN == 256, "N tiles of 64, 128 or 256");
+};
+
+template <int BN>
+__global__ void __launch_bounds__(kQdThreads, 1)
+    qdown_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW,
+                 int64_t M, int64_t N, int64_t Kdim, float* __restrict__ u,
+                 int32_t* __restrict__ status) {
+  using SH = QdShape<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SH::STAGES * SH::STAGE);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + SH::STAGES;
+  uint64_t* acc_full = bars + 2 * SH::STAGES;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t m0 = (int64_t)blockIdx.x * kQdBM, n0 = (int64_t)blockIdx.y * BN;
+  const int nk = (int)(Kdim / 64);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SH::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_holder, SH::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tensormap(&tmH);
+      prefetch_tensormap(&tmW);
+      int last_s = -1;
+      uint32_t last_par = 0;
+      for (int kt = 0; kt < nk; ++kt) {
+        const int s = kt % SH::STAGES;
+        const uint32_t v = (uint32_t)(kt / SH::STAGES);
+        if (!mbar_wait(&empty[s], (v & 1u) ^ 1u, kPrPollLimit)) {
+          record_status(status, kStatusTimeout);
+          break;
+        }
+        uint8_t* st = smem + s * SH::STAGE;
+        mbar_expect_tx(&full[s], SH::STAGE);
+        tma_load_2d(st, &tmH, kt * 64, (int32_t)m0, &full[s]);
+        tma_load_2d(st + SH::A_BYTES, &tmW, kt * 64, (int32_t)n0, &full[s]);
+        last_s = s;
+        last_par = v & 1u;
+      }
+      if (last_s >= 0) mbar_wait(&full[last_s], last_par, kPrPollLimit);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16_f32(kQdBM, BN);
+      bool ok = true;
+      for (int kt = 0; ok && kt < nk; ++kt) {
+        const int s = kt % SH::STAGES;
+        const uint32_t v = (uint32_t)(kt / SH::STAGES);
+        ok = mbar_wait(&full[s], v & 1u, kPrPollLimit);
+        if (!ok) break;
+        tc_fence_after();
+        const uint8_t* st = smem + s * SH::STAGE;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t ad = desc_kmajor_sw128(smem_u32(st) + ks * 32);
+          const uint64_t bd = desc_kmajor_sw128(smem_u32(st + SH::A_BYTES) + ks * 32);
+          mma_bf16_ss(tmem, ad, bd, IDESC, (kt | ks) > 0 ? 1u : 0u);
+        }
+        mma_commit(&empty[s]);
+      }
+      if (!ok) record_status(status, kStatusTimeout);
+      mma_commit(acc_full);   // (also after a timeout: the epilogue's wait then ends)
+    }
+  } else {
+    // epilogue: warp w reads TMEM lanes 32 (w % 4) ..: one token row per thread
+    const int qd = warp & 3;
+    const int64_t row = m0 + qd * 32 + lane;
+    const bool ok = mbar_wait_warp(acc_full, 0, kPrPollLimit);
+    if (!ok) record_status(status, kStatusTimeout);
+    tc_fence_after();
+    if (ok) {
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        float v[16];
+        tmem_ld16(tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)c0, v);
+        tmem_wait_ld();
+        if (row < M) {
+          float4* dst = reinterpret_cast<float4*>(u + row * N + n0 + c0);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, SH::TMEM_COLS);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// [rows, cols] bf16 row-major, boxes of [box_rows, 64] with the 128-byte swizzle.
+bool map_rows(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+              uint32_t box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN>
+cudaError_t launch_qdown_t(int64_t M, int64_t N, int64_t Kdim, const void* hidden,
+                           const void* W_down, float* u, int32_t* status, cudaStream_t st) {
+  using SH = QdShape<BN>;
+  CUtensorMap tmH, tmW;
+  if (!map_rows(&tmH, hidden, (uint64_t)M, (uint64_t)Kdim, kQdBM) ||
+      !map_rows(&tmW, W_down, (uint64_t)N, (uint64_t)Kdim, BN))
+    return cudaErrorInvalidValue;
+  auto kern = qdown_kernel<BN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SH::SMEM);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)((M + kQdBM - 1) / kQdBM), (unsigned)(N / BN));
+  kern<<<grid, kQdThreads, SH::SMEM, st>>>(tmH, tmW, M, N, Kdim, u, status);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------------------------
+constexpr int kQhTokens = 32;     // tokens per CTA
+constexpr int kQhThreads = 256;
+
+// Angle p theta_m reduced to [0, 2 pi) in fp64, then its sine and cosine.
+__device__ __forceinline__ void pair_turn(int64_t pos, double theta, float& c, float& s) {
+  double a = (double)pos * theta;
+  a -= kTwoPi * floor(a / kTwoPi);
+  sincosf((float)a, &s, &c);
+}
+
+// grid (token blocks, Hq, B); r = 0 leaves q_cal = R(q).
+template <typename T, int DD>
+__global__ void __launch_bounds__(kQhThreads)
+    qcal_hope_kernel(int64_t N_q, int64_t Hq, int64_t q_pos0, int r, double base,
+                     double train_len, const T* __restrict__ q, const float* __restrict__ u,
+                     const T* __restrict__ W_up, T* __restrict__ q_out, T* __restrict__ qc_out) {
+  constexpr int NP = DD / 64;   // rotation pairs per lane
+  __shared__ float sW[64 * DD];   // W_up[h] transposed: [r][DD]
+  __shared__ double sTheta[DD / 2];
+  __shared__ int sRot[DD / 2];
+  const int64_t h = blockIdx.y, b = blockIdx.z;
+  for (int e = threadIdx.x; e < r * DD; e += kQhThreads) {
+    const int dim = e / r, j = e - dim * r;   // reads W_up[h][dim][j] in order
+    sW[j * DD + dim] = Elem<T>::to_f(W_up[(h * DD + dim) * r + j]);
+  }
+  for (int m = threadIdx.x; m < DD / 2; m += kQhThreads) {
+    const double th = pow(base, -2.0 * (double)m / (double)DD);
+    sTheta[m] = th;
+    sRot[m] = kTwoPi / th <= train_len ? 1 : 0;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int t = warp; t < kQhTokens; t += kQhThreads / 32) {
+    const int64_t i = (int64_t)blockIdx.x * kQhTokens + t;
+    if (i >= N_q) break;
+    const int64_t row = (b * Hq + h) * N_q + i;
+    const int64_t pos = q_pos0 + i;
+    // u of this (token, head): r values, lanes j and j + 32
+    const float* ur = u + (b * N_q + i) * (Hq * r) + h * r;
+    const float u0 = lane < r ? ur[lane] : 0.f;
+    const float u1 = lane + 32 < r ? ur[lane + 32] : 0.f;
+#pragma unroll
+    for (int pp = 0; pp < NP; ++pp) {
+      const int m = lane + 32 * pp;
+      const int e0 = m, e1 = m + DD / 2;
+      float x0 = Elem<T>::to_f(q[row * DD + e0]);
+      float x1 = Elem<T>::to_f(q[row * DD + e1]);
+      float c0 = x0, c1 = x1;
+      for (int j = 0; j < r; ++j) {
+        const float uj = __shfl_sync(0xffffffffu, j < 32 ? u0 : u1, j & 31);
+        c0 = fmaf(sW[j * DD + e0], uj, c0);
+        c1 = fmaf(sW[j * DD + e1], uj, c1);
+      }
+      if (sRot[m]) {
+        float cs, sn;
+        pair_turn(pos, sTheta[m], cs, sn);
+        const float y0 = x0 * cs - x1 * sn, y1 = x0 * sn + x1 * cs;
+        const float z0 = c0 * cs - c1 * sn, z1 = c0 * sn + c1 * cs;
+        x0 = y0; x1 = y1; c0 = z0; c1 = z1;
+      }
+      q_out[row * DD + e0] = Elem<T>::from_f(x0);
+      q_out[row * DD + e1] = Elem<T>::from_f(x1);
+      qc_out[row * DD + e0] = Elem<T>::from_f(c0);
+      qc_out[row * DD + e1] = Elem<T>::from_f(c1);
+    }
+  }
+}
+
+// x [B H, N, d] -> R(x), token n at position pos0 + n; grid (token blocks, B H).
+template <typename T, int DD>
+__global__ void __launch_bounds__(kQhThreads)
+    hope_rotate_kernel(int64_t N, int64_t pos0, double base, double train_len,
+                       const T* __restrict__ x, T* __restrict__ out) {
+  constexpr int NP = DD / 64;
+  __shared__ double sTheta[DD / 2];
+  __shared__ int sRot[DD / 2];
+  for (int m = threadIdx.x; m < DD / 2; m += kQhThreads) {
+    const double th = pow(base, -2.0 * (double)m / (double)DD);
+    sTheta[m] = th;
+    sRot[m] = kTwoPi / th <= train_len ? 1 : 0;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t bh = blockIdx.y;
+  for (int t = warp; t < kQhTokens; t += kQhThreads / 32) {
+    const int64_t n = (int64_t)blockIdx.x * kQhTokens + t;
+    if (n >= N) break;
+    const int64_t row = bh * N + n;
+#pragma unroll
+    for (int pp = 0; pp < NP; ++pp) {
+      const int m = lane + 32 * pp;
+      float x0 = Elem<T>::to_f(x[row * DD + m]);
+      float x1 = Elem<T>::to_f(x[row * DD + m + DD / 2]);
+      if (sRot[m]) {
+        float cs, sn;
+        pair_turn(pos0 + n, sTheta[m], cs, sn);
+        const float y0 = x0 * cs - x1 * sn, y1 = x0 * sn + x1 * cs;
+        x0 = y0;
+        x1 = y1;
+      }
+      out[row * DD + m] = Elem<T>::from_f(x0);
+      out[row * DD + m + DD / 2] = Elem<T>::from_f(x1);
+    }
+  }
+}
+
+}  // namespace
+
+bool qdown_supported(int64_t N, int64_t d_model) {
+  return d_model >= 64 && d_model % 64 == 0 && N >= 64 && N % 64 == 0;
+}
+
+cudaError_t launch_qdown(int64_t M, int64_t N, int64_t d_model, const void* hidden,
+                         const void* W_down, float* u, int32_t* status, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  if (N % 256 == 0) return launch_qdown_t<256>(M, N, d_model, hidden, W_down, u, status, st);
+  if (N % 128 == 0) return launch_qdown_t<128>(M, N, d_model, hidden, W_down, u, status, st);
+  return launch_qdown_t<64>(M, N, d_model, hidden, W_down, u, status, st);
+}
+
+cudaError_t launch_qcal_hope(int64_t B, int64_t Hq, int64_t N_q, int64_t d, int64_t q_pos0,
+                             int r, double base, double train_len, bool bf16, const void* q,
+                             const float* u, const void* W_up, void* q_out, void* qc_out,
+                             cudaStream_t st) {
+  if (B == 0 || N_q == 0) return cudaSuccess;
+  const dim3 grid((unsigned)((N_q + kQhTokens - 1) / kQhTokens), (unsigned)Hq, (unsigned)B);
+#define HILS_QH(TT, DDV)                                                                      \
+  qcal_hope_kernel<TT, DDV><<<grid, kQhThreads, 0, st>>>(                                      \
+      N_q, Hq, q_pos0, r, base, train_len, static_cast<const TT*>(q), u,                       \
+      static_cast<const TT*>(W_up), static_cast<TT*>(q_out), static_cast<TT*>(qc_out))
+  if (bf16) {
+    if (d == 128) HILS_QH(__nv_bfloat16, 128);
+    else HILS_QH(__nv_bfloat16, 64);
+  } else {
+    if (d == 128) HILS_QH(float, 128);
+    else HILS_QH(float, 64);
+  }
+#undef HILS_QH
+  return cudaGetLastError();
+}
+
+cudaError_t launch_hope_rotate(int64_t BH, int64_t N, int64_t d, int64_t pos0, double base,
+                               double train_len, bool bf16, const void* x, void* out,
+                               cudaStream_t st) {
+  if (BH == 0 || N == 0) return cudaSuccess;
+  const dim3 grid((unsigned)((N + kQhTokens - 1) / kQhTokens), (unsigned)BH);
+#define HILS_HR(TT, DDV)                                                                      \
+  hope_rotate_kernel<TT, DDV><<<grid, kQhThreads, 0, st>>>(                                   \
+      N, pos0, base, train_len, static_cast<const TT*>(x), static_cast<TT*>(out))
+  if (bf16) {
+    if (d == 128) HILS_HR(__nv_bfloat16, 128);
+    else HILS_HR(__nv_bfloat16, 64);
+  } else {
+    if (d == 128) HILS_HR(float, 128);
+    else HILS_HR(float, 64);
+  }
+#undef HILS_HR
+  return cudaGetLastError();
+}
+
+}  // namespace hils

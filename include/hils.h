@@ -177,6 +177,51 @@ hils_status hils_decode_step(const hils_params* p, const void* q, const void* q_
                              size_t workspace_bytes, hils_stream_t stream);
 
 /*
+ * Query prologue: Q-Cal and HoPE, the producers of step 1's calibrated query and step 3's token
+ * query.  Q-Cal ([Reader] "Implementation and Training Recipes", Q-Cal worked example and the
+ * low-rank question): per query head h, dq = W_up[h] (W_down[h] hidden) with W_down[h] r x
+ * d_model and W_up[h] d x r, and q_cal = q + dq.  HoPE ([Reader] same section, HoPE vs RoPE;
+ * [Essay] "Hierarchical Positional Encoding"): the dimension pairs (m, m + d/2), m < d/2, whose
+ * rotation period 2 pi rope_base^(2m/d) is at most train_len turn by pos rope_base^(-2m/d)
+ * radians; the other pairs are left as they are (NoPE).  Queries are turned at their position,
+ * keys at theirs (hils_hope_rotate), so a query's products with the keys, and with the landmark
+ * keys built from them, see relative positions only along the turning pairs.
+ */
+typedef struct {
+  int64_t d_model;    /* width of the hidden state and of W_down's rows (a multiple of 64) */
+  int32_t r;          /* Q-Cal rank: 0 (no correction) or 1..64 with Hq * r a multiple of 64 */
+  double rope_base;   /* > 1 */
+  double train_len;   /* pairs with a longer period do not turn (<= 0: none turns) */
+} hils_prologue_params;
+
+/* Workspace of hils_qcal_hope: a 256-byte status word, then B N_q Hq r fp32 values of
+ * W_down hidden. */
+size_t hils_qcal_workspace_size(const hils_params* p, const hils_prologue_params* c);
+
+/*
+ * q_out = HoPE(q), q_cal_out = HoPE(q + W_up (W_down hidden)) for query i at position
+ * q_pos0 + i.  Reads B, Hq, N_q, d (64 or 128), q_pos0 and dtype of `p`.  q, q_out, q_cal_out
+ * [B, Hq, N_q, d] and W_up [Hq, d, r] in dtype; hidden [B, N_q, d_model] and W_down
+ * [Hq, r, d_model] bf16 (the down-projection, a dense GEMM, runs on the tcgen05 tensor cores with
+ * fp32 accumulation; unused when r = 0).  q_out may equal q (in place); q_cal_out must not
+ * overlap q.  Workspace: hils_qcal_workspace_size bytes, status word zeroed once
+ * (hils_workspace_init; read with hils_device_status).  Asynchronous on `stream`.
+ */
+hils_status hils_qcal_hope(const hils_params* p, const hils_prologue_params* c, const void* q,
+                           const void* hidden, const void* W_down, const void* W_up,
+                           void* q_out, void* q_cal_out, void* workspace,
+                           size_t workspace_bytes, hils_stream_t stream);
+
+/*
+ * x_out = HoPE(x) for x [B, H, N, d] (dtype of `p`, d = 64 or 128), token n at position
+ * pos0 + n: the keys' side of the encoding (turn K before hils_forward and before building
+ * landmarks).  Reads only d and dtype of `p` besides the arguments; x_out may equal x.
+ */
+hils_status hils_hope_rotate(const hils_params* p, const hils_prologue_params* c, int64_t B,
+                             int64_t H, int64_t N, int64_t pos0, const void* x, void* x_out,
+                             hils_stream_t stream);
+
+/*
  * Backward pass: the gradients of L = sum dout . out + sum dlse . lse (out, lse as hils_forward
  * computes them) with respect to q, q_cal, K, V, k_lm and b_lm, with the selection topk_idx held
  * fixed.  The top-K is piecewise constant in its inputs and passes no gradient; the landmark keys
