@@ -60,7 +60,7 @@
  *   Hierarchical Factorization").
  *
  * Backward (hils_oracle_bwd.c): reverse-mode differentiation of steps 4, 1 and 3 above with
- * the selection held fixed (R16: the top-K passes no gradient; the landmark keys and biases
+ * the selection held fixed (R18: the top-K passes no gradient; the landmark keys and biases
  * receive theirs through the fusion weights, [Reader] Fig. 3 caption).
  *
  * Query prologue (hils_oracle_prologue.c): Q-Cal's low-rank correction of the query from the
