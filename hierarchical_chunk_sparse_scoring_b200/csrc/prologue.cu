@@ -12,11 +12,15 @@
 //   qdown_kernel   u = hidden W_down^T for all heads at once: [B N_q, d_model] x [Hq r, d_model]^T,
 //                  a dense contraction on the tcgen05 tensor cores (bf16 operands by TMA with the
 //                  128-byte swizzle, fp32 accumulator in TMEM, 128 x BN tiles, a 4-stage ring).
-//   qcal_hope_kernel  per (b, h, 32 tokens): q_cal = R(q + W_up u), q = R(q); HBM-bound (q read,
-//                  both written, u read); W_up[h] staged transposed in shared memory; each lane
-//                  owns whole rotation pairs, the angle p theta_m reduced modulo 2 pi in fp64
-//                  (p up to 2^22 makes an fp32 product lose whole radians) before sincosf.
+//   qcal_hope_kernel  per (b, 32 tokens), every head in turn: q_cal = R(q + W_up u), q = R(q);
+//                  HBM-bound (q read, both written, u read); W_up[h] staged transposed in shared
+//                  memory; a warp per token, each lane d/32 consecutive dims (the pair partner in
+//                  lane ^ 16); the block's (token, pair) angles p theta_m reduced modulo 2 pi in
+//                  fp64 once (p up to 2^22 makes an fp32 product lose whole radians), then
+//                  sincosf, kept in shared memory for all heads.
 #include <cudaTypedefs.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -192,105 +196,160 @@ cudaError_t launch_qdown_t(int64_t M, int64_t N, int64_t Kdim, const void* hidde
 constexpr int kQhTokens = 32;     // tokens per CTA
 constexpr int kQhThreads = 256;
 
-// Angle p theta_m reduced to [0, 2 pi) in fp64, then its sine and cosine.
-__device__ __forceinline__ void pair_turn(int64_t pos, double theta, float& c, float& s) {
-  double a = (double)pos * theta;
-  a -= kTwoPi * floor(a / kTwoPi);
-  sincosf((float)a, &s, &c);
+// A lane's EPL = d/32 consecutive dims of a row: lanes 0-15 hold the first half (dims m of the
+// pairs), lanes 16-31 the second (dims m + d/2), so a pair's partner sits in lane ^ 16.
+template <typename T, int EPL>
+__device__ __forceinline__ void load_dims(const T* p, float (&v)[EPL]);
+template <>
+__device__ __forceinline__ void load_dims<__nv_bfloat16, 4>(const __nv_bfloat16* p, float (&v)[4]) {
+  const uint2 t = *reinterpret_cast<const uint2*>(p);
+  v[0] = bf16_lo(t.x); v[1] = bf16_hi(t.x); v[2] = bf16_lo(t.y); v[3] = bf16_hi(t.y);
+}
+template <>
+__device__ __forceinline__ void load_dims<__nv_bfloat16, 2>(const __nv_bfloat16* p, float (&v)[2]) {
+  const uint32_t t = *reinterpret_cast<const uint32_t*>(p);
+  v[0] = bf16_lo(t); v[1] = bf16_hi(t);
+}
+template <>
+__device__ __forceinline__ void load_dims<float, 4>(const float* p, float (&v)[4]) {
+  const float4 t = *reinterpret_cast<const float4*>(p);
+  v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+}
+template <>
+__device__ __forceinline__ void load_dims<float, 2>(const float* p, float (&v)[2]) {
+  const float2 t = *reinterpret_cast<const float2*>(p);
+  v[0] = t.x; v[1] = t.y;
+}
+template <typename T, int EPL>
+__device__ __forceinline__ void store_dims(T* p, const float (&v)[EPL]) {
+  if constexpr (std::is_same<T, float>::value) {
+    if constexpr (EPL == 4) *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    else *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+  } else {
+    uint32_t w[EPL / 2];
+#pragma unroll
+    for (int e = 0; e < EPL / 2; ++e) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+      w[e] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    if constexpr (EPL == 4) *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
+    else *reinterpret_cast<uint32_t*>(p) = w[0];
+  }
 }
 
-// grid (token blocks, Hq, B); r = 0 leaves q_cal = R(q).
+// Cosine and sine of every (token, pair) angle of a CTA's token block, fp64 reduction modulo
+// 2 pi (the angle p theta_m reaches 2^22 rad), once per CTA for all its heads; pairs that do not
+// turn get (1, 0).
+template <int DD>
+__device__ __forceinline__ void angle_table(float2* sCS, int64_t pos0, double base,
+                                            double train_len) {
+  for (int e = threadIdx.x; e < kQhTokens * (DD / 2); e += kQhThreads) {
+    const int t = e / (DD / 2), m = e - t * (DD / 2);
+    const double th = pow(base, -2.0 * (double)m / (double)DD);
+    float2 cs = make_float2(1.f, 0.f);
+    if (kTwoPi / th <= train_len) {
+      double a = (double)(pos0 + t) * th;
+      a -= kTwoPi * floor(a * (1.0 / kTwoPi));
+      sincosf((float)a, &cs.y, &cs.x);
+    }
+    sCS[e] = cs;
+  }
+}
+
+// Turns this lane's dims: pair m (first half) and m + d/2 (second half, the partner lane).
+template <int EPL>
+__device__ __forceinline__ void turn(float (&x)[EPL], float (&y)[EPL], int lane,
+                                     const float2* cs_row) {
+  const bool first = lane < 16;
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) {
+    const float2 cs = cs_row[(lane & 15) * EPL + e];
+    const float ox = __shfl_xor_sync(0xffffffffu, x[e], 16);
+    const float oy = __shfl_xor_sync(0xffffffffu, y[e], 16);
+    x[e] = first ? x[e] * cs.x - ox * cs.y : ox * cs.y + x[e] * cs.x;
+    y[e] = first ? y[e] * cs.x - oy * cs.y : oy * cs.y + y[e] * cs.x;
+  }
+}
+
+// grid (token blocks, B); every head of the block in turn.  r = 0 leaves q_cal = R(q).
 template <typename T, int DD>
 __global__ void __launch_bounds__(kQhThreads)
     qcal_hope_kernel(int64_t N_q, int64_t Hq, int64_t q_pos0, int r, double base,
                      double train_len, const T* __restrict__ q, const float* __restrict__ u,
                      const T* __restrict__ W_up, T* __restrict__ q_out, T* __restrict__ qc_out) {
-  constexpr int NP = DD / 64;   // rotation pairs per lane
-  __shared__ float sW[64 * DD];   // W_up[h] transposed: [r][DD]
-  __shared__ double sTheta[DD / 2];
-  __shared__ int sRot[DD / 2];
-  const int64_t h = blockIdx.y, b = blockIdx.z;
-  for (int e = threadIdx.x; e < r * DD; e += kQhThreads) {
-    const int dim = e / r, j = e - dim * r;   // reads W_up[h][dim][j] in order
-    sW[j * DD + dim] = Elem<T>::to_f(W_up[(h * DD + dim) * r + j]);
-  }
-  for (int m = threadIdx.x; m < DD / 2; m += kQhThreads) {
-    const double th = pow(base, -2.0 * (double)m / (double)DD);
-    sTheta[m] = th;
-    sRot[m] = kTwoPi / th <= train_len ? 1 : 0;
-  }
-  __syncthreads();
+  constexpr int EPL = DD / 32;
+  __shared__ __align__(16) float sW[64 * DD];   // W_up[h] transposed: [r][DD]
+  __shared__ float2 sCS[kQhTokens * (DD / 2)];
+  const int64_t b = blockIdx.y;
+  const int64_t i0 = (int64_t)blockIdx.x * kQhTokens;
+  angle_table<DD>(sCS, q_pos0 + i0, base, train_len);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int t = warp; t < kQhTokens; t += kQhThreads / 32) {
-    const int64_t i = (int64_t)blockIdx.x * kQhTokens + t;
-    if (i >= N_q) break;
-    const int64_t row = (b * Hq + h) * N_q + i;
-    const int64_t pos = q_pos0 + i;
-    // u of this (token, head): r values, lanes j and j + 32
-    const float* ur = u + (b * N_q + i) * (Hq * r) + h * r;
-    const float u0 = lane < r ? ur[lane] : 0.f;
-    const float u1 = lane + 32 < r ? ur[lane + 32] : 0.f;
+  const int dim0 = lane * EPL;
+  for (int64_t h = 0; h < Hq; ++h) {
+    __syncthreads();   // (the previous head's W_up is consumed)
+    for (int e = threadIdx.x; e < r * DD; e += kQhThreads) {
+      const int dim = e / r, j = e - dim * r;   // reads W_up[h][dim][j] in order
+      sW[j * DD + dim] = Elem<T>::to_f(W_up[(h * DD + dim) * r + j]);
+    }
+    __syncthreads();
+    for (int t = warp; t < kQhTokens; t += kQhThreads / 32) {
+      const int64_t i = i0 + t;
+      if (i >= N_q) break;
+      const int64_t row = (b * Hq + h) * N_q + i;
+      float x[EPL], c[EPL];
+      load_dims<T, EPL>(q + row * DD + dim0, x);
 #pragma unroll
-    for (int pp = 0; pp < NP; ++pp) {
-      const int m = lane + 32 * pp;
-      const int e0 = m, e1 = m + DD / 2;
-      float x0 = Elem<T>::to_f(q[row * DD + e0]);
-      float x1 = Elem<T>::to_f(q[row * DD + e1]);
-      float c0 = x0, c1 = x1;
-      for (int j = 0; j < r; ++j) {
-        const float uj = __shfl_sync(0xffffffffu, j < 32 ? u0 : u1, j & 31);
-        c0 = fmaf(sW[j * DD + e0], uj, c0);
-        c1 = fmaf(sW[j * DD + e1], uj, c1);
+      for (int e = 0; e < EPL; ++e) c[e] = x[e];
+      if (r > 0) {
+        // u of this (token, head): r values, lanes j and j + 32; dq = W_up u
+        const float* ur = u + (b * N_q + i) * (Hq * r) + h * r;
+        const float u0 = lane < r ? ur[lane] : 0.f;
+        const float u1 = lane + 32 < r ? ur[lane + 32] : 0.f;
+        for (int j = 0; j < r; ++j) {
+          const float uj = __shfl_sync(0xffffffffu, j < 32 ? u0 : u1, j & 31);
+          const float* wr = sW + j * DD + dim0;
+          if constexpr (EPL == 4) {
+            const float4 w = *reinterpret_cast<const float4*>(wr);
+            c[0] = fmaf(w.x, uj, c[0]);
+            c[1] = fmaf(w.y, uj, c[1]);
+            c[2] = fmaf(w.z, uj, c[2]);
+            c[3] = fmaf(w.w, uj, c[3]);
+          } else {
+            const float2 w = *reinterpret_cast<const float2*>(wr);
+            c[0] = fmaf(w.x, uj, c[0]);
+            c[1] = fmaf(w.y, uj, c[1]);
+          }
+        }
       }
-      if (sRot[m]) {
-        float cs, sn;
-        pair_turn(pos, sTheta[m], cs, sn);
-        const float y0 = x0 * cs - x1 * sn, y1 = x0 * sn + x1 * cs;
-        const float z0 = c0 * cs - c1 * sn, z1 = c0 * sn + c1 * cs;
-        x0 = y0; x1 = y1; c0 = z0; c1 = z1;
-      }
-      q_out[row * DD + e0] = Elem<T>::from_f(x0);
-      q_out[row * DD + e1] = Elem<T>::from_f(x1);
-      qc_out[row * DD + e0] = Elem<T>::from_f(c0);
-      qc_out[row * DD + e1] = Elem<T>::from_f(c1);
+      turn<EPL>(x, c, lane, sCS + t * (DD / 2));
+      store_dims<T, EPL>(q_out + row * DD + dim0, x);
+      store_dims<T, EPL>(qc_out + row * DD + dim0, c);
     }
   }
 }
 
-// x [B H, N, d] -> R(x), token n at position pos0 + n; grid (token blocks, B H).
+// x [B H, N, d] -> R(x), token n at position pos0 + n; grid (token blocks), every (b, h) in turn.
 template <typename T, int DD>
 __global__ void __launch_bounds__(kQhThreads)
-    hope_rotate_kernel(int64_t N, int64_t pos0, double base, double train_len,
+    hope_rotate_kernel(int64_t BH, int64_t N, int64_t pos0, double base, double train_len,
                        const T* __restrict__ x, T* __restrict__ out) {
-  constexpr int NP = DD / 64;
-  __shared__ double sTheta[DD / 2];
-  __shared__ int sRot[DD / 2];
-  for (int m = threadIdx.x; m < DD / 2; m += kQhThreads) {
-    const double th = pow(base, -2.0 * (double)m / (double)DD);
-    sTheta[m] = th;
-    sRot[m] = kTwoPi / th <= train_len ? 1 : 0;
-  }
+  constexpr int EPL = DD / 32;
+  __shared__ float2 sCS[kQhTokens * (DD / 2)];
+  const int64_t n0 = (int64_t)blockIdx.x * kQhTokens;
+  angle_table<DD>(sCS, pos0 + n0, base, train_len);
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t bh = blockIdx.y;
-  for (int t = warp; t < kQhTokens; t += kQhThreads / 32) {
-    const int64_t n = (int64_t)blockIdx.x * kQhTokens + t;
-    if (n >= N) break;
-    const int64_t row = bh * N + n;
+  for (int64_t bh = 0; bh < BH; ++bh) {
+    for (int t = warp; t < kQhTokens; t += kQhThreads / 32) {
+      const int64_t n = n0 + t;
+      if (n >= N) break;
+      const int64_t row = bh * N + n;
+      float v[EPL], w[EPL];
+      load_dims<T, EPL>(x + row * DD + lane * EPL, v);
 #pragma unroll
-    for (int pp = 0; pp < NP; ++pp) {
-      const int m = lane + 32 * pp;
-      float x0 = Elem<T>::to_f(x[row * DD + m]);
-      float x1 = Elem<T>::to_f(x[row * DD + m + DD / 2]);
-      if (sRot[m]) {
-        float cs, sn;
-        pair_turn(pos0 + n, sTheta[m], cs, sn);
-        const float y0 = x0 * cs - x1 * sn, y1 = x0 * sn + x1 * cs;
-        x0 = y0;
-        x1 = y1;
-      }
-      out[row * DD + m] = Elem<T>::from_f(x0);
-      out[row * DD + m + DD / 2] = Elem<T>::from_f(x1);
+      for (int e = 0; e < EPL; ++e) w[e] = 0.f;
+      turn<EPL>(v, w, lane, sCS + t * (DD / 2));
+      store_dims<T, EPL>(out + row * DD + lane * EPL, v);
     }
   }
 }
@@ -314,7 +373,7 @@ cudaError_t launch_qcal_hope(int64_t B, int64_t Hq, int64_t N_q, int64_t d, int6
                              const float* u, const void* W_up, void* q_out, void* qc_out,
                              cudaStream_t st) {
   if (B == 0 || N_q == 0) return cudaSuccess;
-  const dim3 grid((unsigned)((N_q + kQhTokens - 1) / kQhTokens), (unsigned)Hq, (unsigned)B);
+  const dim3 grid((unsigned)((N_q + kQhTokens - 1) / kQhTokens), (unsigned)B);
 #define HILS_QH(TT, DDV)                                                                      \
   qcal_hope_kernel<TT, DDV><<<grid, kQhThreads, 0, st>>>(                                      \
       N_q, Hq, q_pos0, r, base, train_len, static_cast<const TT*>(q), u,                       \
@@ -334,10 +393,10 @@ cudaError_t launch_hope_rotate(int64_t BH, int64_t N, int64_t d, int64_t pos0, d
                                double train_len, bool bf16, const void* x, void* out,
                                cudaStream_t st) {
   if (BH == 0 || N == 0) return cudaSuccess;
-  const dim3 grid((unsigned)((N + kQhTokens - 1) / kQhTokens), (unsigned)BH);
+  const dim3 grid((unsigned)((N + kQhTokens - 1) / kQhTokens));
 #define HILS_HR(TT, DDV)                                                                      \
   hope_rotate_kernel<TT, DDV><<<grid, kQhThreads, 0, st>>>(                                   \
-      N, pos0, base, train_len, static_cast<const TT*>(x), static_cast<TT*>(out))
+      BH, N, pos0, base, train_len, static_cast<const TT*>(x), static_cast<TT*>(out))
   if (bf16) {
     if (d == 128) HILS_HR(__nv_bfloat16, 128);
     else HILS_HR(__nv_bfloat16, 64);
