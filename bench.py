@@ -868,6 +868,26 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_only_extra(args):
+    """One extra measurement on its own (the commands the profiles/ summaries were taken with)."""
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the HiLS path has no CPU fallback)")
+    peaks, _ = load_peaks()
+    n = args.N
+    if args.only_extra == "backward":
+        out = extra_backward(peaks, args.workload if args.workload != HEADLINE[0] else
+                             "gqa7b_prefill", steps=args.steps, **({"N": n} if n else {}))
+    elif args.only_extra == "prologue":
+        out = extra_prologue(peaks, N=n or 131072, steps=args.steps)
+    elif args.only_extra == "decode":
+        out = extra_decode(max(3, args.steps), peaks)
+    elif args.only_extra == "decode_step":
+        out = extra_decode_step(max(3, args.steps), peaks)
+    else:
+        out = extra_landmarks(peaks, 1, 1, n or (1 << 22), 128, 128, steps=args.steps)
+    print(json.dumps(out), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -878,12 +898,17 @@ def main():
     ap.add_argument("--N", type=int, default=None, help="override the workload's sequence length")
     ap.add_argument("--B", type=int, default=None, help="override the workload's batch")
     ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--only-extra", choices=["backward", "prologue", "decode", "decode_step",
+                                             "landmarks"], default=None,
+                    help="run one extra measurement alone and print its JSON (for profiling)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "hils":
         args.warmup = 3
-    if args.impl == "reference":
+    if args.only_extra:
+        run_only_extra(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_hils(args)
