@@ -617,8 +617,8 @@ def extra_extreme(steps, peaks, N=262144):
     from hierarchical_chunk_sparse_scoring_b200 import workloads as W
     wl = W.make("extreme", "cuda", N=N)
     res = {"workload": "extreme", "N": N,
-           "prefill": time_mode(wl, steps, peaks, "extreme_prefill"),
-           "decode": time_mode(W.decode_view(wl), max(steps, 5), peaks, "extreme_decode")}
+           "prefill": time_mode(wl, steps, peaks, "extreme_N%d" % N),
+           "decode": time_mode(W.decode_view(wl), max(steps, 5), peaks, "extreme_N%d_decode" % N)}
     del wl
     torch.cuda.empty_cache()
     return res
