@@ -21,9 +21,12 @@
 //   bwd_keys_kernel  (key-major; CTA = one tile of up to 64 keys of one chunk) over the rows whose
 //                    window covers the tile and the rows that selected its chunk: dK and dV held
 //                    in registers, then d k_lm and d b_lm from the selecting rows' dscore.
-// No gradient is accumulated with atomics.  The products are CUDA-core tiles: 4 x (T/16)
-// outputs per thread, operands staged in shared memory as fp32 (rows padded by 4 floats so the
-// 16-byte loads of consecutive rows fall in different banks).
+// No gradient is accumulated with atomics.  fp32 inputs: the products are CUDA-core tiles, 4 x
+// (T/16) outputs per thread, operands staged in shared memory as fp32 (rows padded by 4 floats so
+// the 16-byte loads of consecutive rows fall in different banks).  bf16 inputs: warp-level
+// m16n8k16 tensor-core products (see the tensor-core tiles below).
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -56,15 +59,6 @@ template <>
 __device__ __forceinline__ void load_piece<float>(const float* src, float* dst) {
   *reinterpret_cast<float4*>(dst) = __ldg(reinterpret_cast<const float4*>(src));
 }
-template <>
-__device__ __forceinline__ void load_piece<__nv_bfloat16>(const __nv_bfloat16* src, float* dst) {
-  const uint4 t = __ldg(reinterpret_cast<const uint4*>(src));
-  *reinterpret_cast<float4*>(dst) = make_float4(bf16_lo(t.x), bf16_hi(t.x), bf16_lo(t.y),
-                                                bf16_hi(t.y));
-  *reinterpret_cast<float4*>(dst + 4) = make_float4(bf16_lo(t.z), bf16_hi(t.z), bf16_lo(t.w),
-                                                    bf16_hi(t.w));
-}
-
 // Rows r < n of dst (stride LD floats) from rowp[r] (nullptr: zeros), fp32.
 template <typename TI, int DD, int LD>
 __device__ __forceinline__ void stage_rows(float* dst, const TI* const* rowp, int n) {
@@ -139,11 +133,141 @@ __device__ __forceinline__ void logits_tile(const float* sQ, const float* sdO, c
   }
 }
 
+// ------------------------------------------------------------------ tensor-core (bf16) tiles
+// With bf16 inputs the products run as warp-level m16n8k16 bf16 MMAs with fp32 accumulation:
+// operands staged in shared memory as bf16 (rows padded by 8 elements, so the eight 16-byte rows
+// an ldmatrix reads fall in different banks), fragments loaded with ldmatrix (.trans where the
+// stored layout is the operand's transpose).  The logits and dO . V products take the bf16 inputs
+// exactly; the fused weights a and logit gradients dx enter the dq, dK and dV products rounded to
+// bf16, as the intermediate probabilities of a flash-attention backward do.
+constexpr int kPadB = 8;   // bf16 elements of row padding
+
+__device__ __forceinline__ uint32_t su32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void ldsm4(uint32_t a, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                      uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(a));
+}
+__device__ __forceinline__ void ldsm4t(uint32_t a, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                       uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(a));
+}
+__device__ __forceinline__ void ldsm2(uint32_t a, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];\n"
+               : "=r"(r0), "=r"(r1) : "r"(a));
+}
+__device__ __forceinline__ void ldsm2t(uint32_t a, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n"
+               : "=r"(r0), "=r"(r1) : "r"(a));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Rows r < n of a bf16 [n][DD + kPadB] tile from rowp[r] (nullptr: zeros).
+template <int DD>
+__device__ __forceinline__ void stage_rows_b(__nv_bfloat16* dst,
+                                             const __nv_bfloat16* const* rowp, int n) {
+  constexpr int PPR = DD / 8, LDB = DD + kPadB;
+  for (int e = threadIdx.x; e < n * PPR; e += kBwdThreads) {
+    const int r = e / PPR, u = e - r * PPR;
+    const __nv_bfloat16* src = rowp[r];
+    *reinterpret_cast<uint4*>(dst + r * LDB + u * 8) =
+        src ? __ldg(reinterpret_cast<const uint4*>(src + u * 8)) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// Keys k0 .. k0 + T - 1 of one (b, g) plane as bf16 [T][DD + kPadB] (zeros past N_kv).
+template <int DD, int T>
+__device__ __forceinline__ void stage_keys_b(__nv_bfloat16* dst, const __nv_bfloat16* base,
+                                             int64_t k0, int64_t nkv) {
+  constexpr int PPR = DD / 8, LDB = DD + kPadB;
+  for (int e = threadIdx.x; e < T * PPR; e += kBwdThreads) {
+    const int r = e / PPR, u = e - r * PPR;
+    *reinterpret_cast<uint4*>(dst + r * LDB + u * 8) =
+        k0 + r < nkv ? __ldg(reinterpret_cast<const uint4*>(base + (k0 + r) * DD + u * 8))
+                     : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// X = Q K^T and P = dO V^T for rows 16 rb .. 16 rb + 15 and keys kh T/2 .. (kh + 1) T/2 - 1:
+// NT = T/16 accumulator tiles of m16n8 each; element v of tile j is (row 16 rb + lane/4 + 8 (v/2),
+// key kh T/2 + 8 j + 2 (lane%4) + v%2).
+template <int DD, int T>
+__device__ __forceinline__ void logits_frag(const __nv_bfloat16* sQ, const __nv_bfloat16* sdO,
+                                            const __nv_bfloat16* sK, const __nv_bfloat16* sV,
+                                            int rb, int kh, float (&X)[T / 16][4],
+                                            float (&P)[T / 16][4]) {
+  constexpr int NT = T / 16, LDB = DD + kPadB;
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int j = 0; j < NT; ++j)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) X[j][v] = P[j][v] = 0.f;
+  const int arow = 16 * rb + (lane & 15), acol = (lane >> 4) * 8;
+  const int i8 = lane >> 3, r8 = lane & 7;
+#pragma unroll
+  for (int ks = 0; ks < DD / 16; ++ks) {
+    uint32_t aq[4], ao[4];
+    ldsm4(su32(sQ + arow * LDB + 16 * ks + acol), aq[0], aq[1], aq[2], aq[3]);
+    ldsm4(su32(sdO + arow * LDB + 16 * ks + acol), ao[0], ao[1], ao[2], ao[3]);
+    if constexpr (NT == 1) {
+      const int key = kh * (T / 2) + r8, dim = 16 * ks + (i8 & 1) * 8;
+      uint32_t k0, k1, v0, v1;
+      ldsm2(su32(sK + key * LDB + dim), k0, k1);
+      ldsm2(su32(sV + key * LDB + dim), v0, v1);
+      mma16816(X[0], aq, k0, k1);
+      mma16816(P[0], ao, v0, v1);
+    } else {
+#pragma unroll
+      for (int j = 0; j < NT; j += 2) {
+        const int key = kh * (T / 2) + 8 * j + r8 + (i8 >> 1) * 8, dim = 16 * ks + (i8 & 1) * 8;
+        uint32_t k0, k1, k2, k3, v0, v1, v2, v3;
+        ldsm4(su32(sK + key * LDB + dim), k0, k1, k2, k3);
+        ldsm4(su32(sV + key * LDB + dim), v0, v1, v2, v3);
+        mma16816(X[j], aq, k0, k1);
+        mma16816(X[j + 1], aq, k2, k3);
+        mma16816(P[j], ao, v0, v1);
+        mma16816(P[j + 1], ao, v2, v3);
+      }
+    }
+  }
+}
+
+// Bytes of a kernel's product operands at the start of its shared memory (the bookkeeping
+// follows): fp32 tiles for the CUDA cores, bf16 tiles for the tensor cores.
+template <int DD, int T, bool TC>
+constexpr int rows_prod_bytes() {
+  using SH = BwdShape<DD, T>;
+  return TC ? ((2 * kBwdRows + 2 * T) * (DD + kPadB) + kBwdRows * (T + kPadB)) * 2 +
+                  2 * kBwdRows * 3 * 4
+            : (2 * SH::ROWS_F + 2 * SH::KEYS_F + SH::TILE_F) * 4;
+}
+template <int DD, int T, bool TC>
+constexpr int keys_prod_bytes() {
+  using SH = BwdShape<DD, T>;
+  return TC ? ((2 * kBwdRows + 2 * T) * (DD + kPadB) + 2 * kBwdRows * (T + kPadB)) * 2
+            : (2 * SH::ROWS_F + 2 * SH::KEYS_F + 2 * SH::TILE_F) * 4;
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------------------------
 // Query-major kernel: CTA = (b, g, 64/G queries); row r = query r / G, head g G + r % G.
-template <typename TI, int DD, int T>
+// TC: the products on the tensor cores (bf16 inputs), else on the CUDA cores.
+template <typename TI, int DD, int T, bool TC>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_rows_kernel(Dims D, const TI* __restrict__ q, const TI* __restrict__ qc,
                     const TI* __restrict__ K, const TI* __restrict__ V,
@@ -155,13 +279,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   using SH = BwdShape<DD, T>;
   constexpr int LD = SH::LD, LDA = SH::LDA, KPT = SH::KPT, DG = SH::DG;
   constexpr int SU = kBwdMaxK + 1;   // stats row stride (units)
+  using BF = __nv_bfloat16;
+  constexpr int LDB = DD + kPadB, LDX = T + kPadB;
   extern __shared__ float4 smem_f4[];
-  float* sQ = reinterpret_cast<float*>(smem_f4);
+  uint8_t* smem = reinterpret_cast<uint8_t*>(smem_f4);
+  // the products' operands: fp32 tiles (CUDA cores) or bf16 tiles (tensor cores)
+  float* sQ = reinterpret_cast<float*>(smem);
   float* sdO = sQ + SH::ROWS_F;
   float* sK = sdO + SH::ROWS_F;
   float* sV = sK + SH::KEYS_F;
   float* sdX = sV + SH::KEYS_F;
-  float* sM = sdX + SH::TILE_F;              // [64][SU] running max (base 2), then lambda2
+  BF* bQ = reinterpret_cast<BF*>(smem);
+  BF* bdO = bQ + kBwdRows * LDB;
+  BF* bK = bdO + kBwdRows * LDB;
+  BF* bV = bK + T * LDB;
+  BF* bdX = bV + T * LDB;
+  float* sPart = reinterpret_cast<float*>(bdX + kBwdRows * LDX);   // [2 key halves][64][3]
+  float* sM = reinterpret_cast<float*>(smem + rows_prod_bytes<DD, T, TC>());   // [64][SU] running
+                                                                           // max (base 2), then lambda2
   float* sL = sM + kBwdRows * SU;            // running sum, then gamma
   float* sT = sL + kBwdRows * SU;            // running sum of p dP, then dscore
   float* sS = sT + kBwdRows * SU;            // [64][32] chunk scores
@@ -212,7 +347,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     sU[e] = c;
   }
   __syncthreads();
-  stage_rows<TI, DD, LD>(sQ, rowp, kBwdRows);
+  if constexpr (TC) stage_rows_b<DD>(bQ, reinterpret_cast<const BF* const*>(rowp), kBwdRows);
+  else stage_rows<TI, DD, LD>(sQ, rowp, kBwdRows);
   __syncthreads();
   if (tid < kBwdRows) rowp[tid] = sPos[tid] != INT64_MIN ? dO + grow_of(tid) * DD : nullptr;
   __syncthreads();
@@ -232,7 +368,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       __syncthreads();
     }
-  stage_rows<TI, DD, LD>(sdO, rowp, kBwdRows);
+  if constexpr (TC) stage_rows_b<DD>(bdO, reinterpret_cast<const BF* const*>(rowp), kBwdRows);
+  else stage_rows<TI, DD, LD>(sdO, rowp, kBwdRows);
   if (warp == 0) {   // compact the distinct ids to the front (sorted: a repeat follows its twin)
     int n = 0, last = INT_MIN;
     for (int e0 = 0; e0 < np; e0 += 32) {
@@ -284,57 +421,126 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   };
 
+  // merges a tile's (max, sum, sum p dP) of row r's unit u into the running state
+  auto merge_stats = [&](int r, int u, float m, float l, float tt) {
+    if (u < 0 || m == -INFINITY) return;
+    float* pm = sM + r * SU + u;
+    float* pl = sL + r * SU + u;
+    float* pt = sT + r * SU + u;
+    const float M = *pm;
+    if (m > M) {
+      const float f = M == -INFINITY ? 0.f : exp2f(M - m);
+      *pl = *pl * f + l;
+      *pt = *pt * f + tt;
+      *pm = m;
+    } else {
+      const float f = exp2f(m - M);
+      *pl += l * f;
+      *pt += tt * f;
+    }
+  };
+
   // ---- pass 1: per (row, unit) lse and delta = dO . o_u by online reduction
   for (int t = 0; t < n_tiles; ++t) {
     const int64_t k0 = tile_k0(t);
-    stage_keys<TI, DD, LD, T>(sK, Kb, k0, D.N_kv);
-    stage_keys<TI, DD, LD, T>(sV, Vb, k0, D.N_kv);
+    if constexpr (TC) {
+      stage_keys_b<DD, T>(bK, reinterpret_cast<const BF*>(Kb), k0, D.N_kv);
+      stage_keys_b<DD, T>(bV, reinterpret_cast<const BF*>(Vb), k0, D.N_kv);
+    } else {
+      stage_keys<TI, DD, LD, T>(sK, Kb, k0, D.N_kv);
+      stage_keys<TI, DD, LD, T>(sV, Vb, k0, D.N_kv);
+    }
     set_units(k0);
     __syncthreads();
-    float X[4][KPT], P[4][KPT];
-    logits_tile<DD, T>(sQ, sdO, sK, sV, tr, tc, X, P);
+    if constexpr (TC) {
+      // warp: rows 16 rb .., keys kh T/2 ..; a row's values sit in the 4 lanes of its quad
+      const int rb = warp & 3, kh = warp >> 2, g8 = lane >> 2, t4 = lane & 3;
+      float X[T / 16][4], P[T / 16][4];
+      logits_frag<DD, T>(bQ, bdO, bK, bV, rb, kh, X, P);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = tr * 4 + i;
-      const int u = sUnit[r];
-      const int64_t pos = sPos[r];
-      float m = -INFINITY;
+      for (int hr = 0; hr < 2; ++hr) {
+        const int r = 16 * rb + g8 + 8 * hr;
+        const int u = sUnit[r];
+        const int64_t pos = sPos[r];
+        float m = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < KPT; ++e) {
-        const int64_t j = k0 + tc + 16 * e;
-        const bool ok = u >= 0 && j <= pos && j < D.N_kv;
-        X[i][e] = ok ? X[i][e] * sc2 : -INFINITY;
-        m = fmaxf(m, X[i][e]);
-      }
+        for (int j = 0; j < T / 16; ++j)
 #pragma unroll
-      for (int o = 1; o < 16; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      float l = 0.f, tt = 0.f;
+          for (int v = 0; v < 2; ++v) {
+            const int64_t key = k0 + kh * (T / 2) + 8 * j + 2 * t4 + v;
+            const bool ok = u >= 0 && key <= pos && key < D.N_kv;
+            X[j][2 * hr + v] = ok ? X[j][2 * hr + v] * sc2 : -INFINITY;
+            m = fmaxf(m, X[j][2 * hr + v]);
+          }
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        float l = 0.f, tt = 0.f;
 #pragma unroll
-      for (int e = 0; e < KPT; ++e) {
-        const float w = X[i][e] == -INFINITY ? 0.f : exp2f(X[i][e] - m);
-        l += w;
-        tt = fmaf(w, P[i][e], tt);
-      }
+        for (int j = 0; j < T / 16; ++j)
 #pragma unroll
-      for (int o = 1; o < 16; o <<= 1) {
-        l += __shfl_xor_sync(0xffffffffu, l, o);
-        tt += __shfl_xor_sync(0xffffffffu, tt, o);
-      }
-      if (tc == 0 && u >= 0 && m != -INFINITY) {
-        float* pm = sM + r * SU + u;
-        float* pl = sL + r * SU + u;
-        float* pt = sT + r * SU + u;
-        const float M = *pm;
-        if (m > M) {
-          const float f = M == -INFINITY ? 0.f : exp2f(M - m);
-          *pl = *pl * f + l;
-          *pt = *pt * f + tt;
-          *pm = m;
-        } else {
-          const float f = exp2f(m - M);
-          *pl += l * f;
-          *pt += tt * f;
+          for (int v = 0; v < 2; ++v) {
+            const float x = X[j][2 * hr + v];
+            const float w = x == -INFINITY ? 0.f : exp2f(x - m);
+            l += w;
+            tt = fmaf(w, P[j][2 * hr + v], tt);
+          }
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1) {
+          l += __shfl_xor_sync(0xffffffffu, l, o);
+          tt += __shfl_xor_sync(0xffffffffu, tt, o);
         }
+        if (t4 == 0) {
+          float* pp = sPart + (kh * kBwdRows + r) * 3;
+          pp[0] = m;
+          pp[1] = l;
+          pp[2] = tt;
+        }
+      }
+      __syncthreads();
+      if (tid < kBwdRows) {   // the two key halves of row tid, then its unit's running state
+        const float* p0 = sPart + tid * 3;
+        const float* p1 = sPart + (kBwdRows + tid) * 3;
+        const float m = fmaxf(p0[0], p1[0]);
+        float l = 0.f, tt = 0.f;
+        if (m != -INFINITY) {
+          const float f0 = p0[0] == -INFINITY ? 0.f : exp2f(p0[0] - m);
+          const float f1 = p1[0] == -INFINITY ? 0.f : exp2f(p1[0] - m);
+          l = p0[1] * f0 + p1[1] * f1;
+          tt = p0[2] * f0 + p1[2] * f1;
+        }
+        merge_stats(tid, sUnit[tid], m, l, tt);
+      }
+    } else {
+      float X[4][KPT], P[4][KPT];
+      logits_tile<DD, T>(sQ, sdO, sK, sV, tr, tc, X, P);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = tr * 4 + i;
+        const int u = sUnit[r];
+        const int64_t pos = sPos[r];
+        float m = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < KPT; ++e) {
+          const int64_t j = k0 + tc + 16 * e;
+          const bool ok = u >= 0 && j <= pos && j < D.N_kv;
+          X[i][e] = ok ? X[i][e] * sc2 : -INFINITY;
+          m = fmaxf(m, X[i][e]);
+        }
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float l = 0.f, tt = 0.f;
+#pragma unroll
+        for (int e = 0; e < KPT; ++e) {
+          const float w = X[i][e] == -INFINITY ? 0.f : exp2f(X[i][e] - m);
+          l += w;
+          tt = fmaf(w, P[i][e], tt);
+        }
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) {
+          l += __shfl_xor_sync(0xffffffffu, l, o);
+          tt += __shfl_xor_sync(0xffffffffu, tt, o);
+        }
+        if (tc == 0) merge_stats(r, u, m, l, tt);
       }
     }
     __syncthreads();
@@ -422,66 +628,137 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 
   // ---- pass 2: dq = scale sum_j dx_j K_j
-  float acc[4][DG][4];
+  if constexpr (TC) {
+    // dx tile to shared memory as bf16, then dq += dx K on the tensor cores: warp = rows 16 rb ..
+    // and dims dh d/2 .. (NTD = d/16 accumulator tiles)
+    constexpr int NTD = DD / 16;
+    const int rb = warp & 3, kh = warp >> 2, g8 = lane >> 2, t4 = lane & 3;
+    const int dh = kh;
+    float acc[NTD][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+    for (int j = 0; j < NTD; ++j)
 #pragma unroll
-    for (int e = 0; e < DG; ++e)
+      for (int v = 0; v < 4; ++v) acc[j][v] = 0.f;
+    for (int t = 0; t < n_tiles; ++t) {
+      const int64_t k0 = tile_k0(t);
+      __syncthreads();
+      stage_keys_b<DD, T>(bK, reinterpret_cast<const BF*>(Kb), k0, D.N_kv);
+      stage_keys_b<DD, T>(bV, reinterpret_cast<const BF*>(Vb), k0, D.N_kv);
+      set_units(k0);
+      __syncthreads();
+      float X[T / 16][4], P[T / 16][4];
+      logits_frag<DD, T>(bQ, bdO, bK, bV, rb, kh, X, P);
 #pragma unroll
-      for (int v = 0; v < 4; ++v) acc[i][e][v] = 0.f;
-  for (int t = 0; t < n_tiles; ++t) {
-    const int64_t k0 = tile_k0(t);
-    __syncthreads();
-    stage_keys<TI, DD, LD, T>(sK, Kb, k0, D.N_kv);
-    stage_keys<TI, DD, LD, T>(sV, Vb, k0, D.N_kv);
-    set_units(k0);
-    __syncthreads();
-    float X[4][KPT], P[4][KPT];
-    logits_tile<DD, T>(sQ, sdO, sK, sV, tr, tc, X, P);
+      for (int hr = 0; hr < 2; ++hr) {
+        const int r = 16 * rb + g8 + 8 * hr;
+        const int u = sUnit[r];
+        const int64_t pos = sPos[r];
+        const float lam2 = u >= 0 ? sM[r * SU + u] : -INFINITY;
+        const float gam = u >= 0 ? sL[r * SU + u] : 0.f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = tr * 4 + i;
-      const int u = sUnit[r];
-      const int64_t pos = sPos[r];
-      const float lam2 = u >= 0 ? sM[r * SU + u] : -INFINITY;
-      const float gam = u >= 0 ? sL[r * SU + u] : 0.f;
+        for (int j = 0; j < T / 16; ++j) {
+          float dx[2];
 #pragma unroll
-      for (int e = 0; e < KPT; ++e) {
-        const int64_t j = k0 + tc + 16 * e;
-        const bool ok = u >= 0 && j <= pos && j < D.N_kv && lam2 != -INFINITY;
-        const float a = ok ? exp2f(fmaf(X[i][e], sc2, lam2)) : 0.f;
-        sdX[r * LDA + tc + 16 * e] = a * (P[i][e] - gam);
+          for (int v = 0; v < 2; ++v) {
+            const int64_t key = k0 + kh * (T / 2) + 8 * j + 2 * t4 + v;
+            const bool ok = u >= 0 && key <= pos && key < D.N_kv && lam2 != -INFINITY;
+            const float aw = ok ? exp2f(fmaf(X[j][2 * hr + v], sc2, lam2)) : 0.f;
+            dx[v] = aw * (P[j][2 * hr + v] - gam);
+          }
+          *reinterpret_cast<uint32_t*>(bdX + r * LDX + kh * (T / 2) + 8 * j + 2 * t4) =
+              pack_bf16(dx[0], dx[1]);
+        }
       }
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int j = 0; j < T; ++j) {
-      float w[4];
+      __syncthreads();
+      const int i8 = lane >> 3, r8 = lane & 7;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) w[i] = sdX[(tr * 4 + i) * LDA + j];
+      for (int ks = 0; ks < T / 16; ++ks) {
+        uint32_t af[4];
+        ldsm4(su32(bdX + (16 * rb + (lane & 15)) * LDX + 16 * ks + (lane >> 4) * 8), af[0], af[1],
+              af[2], af[3]);
 #pragma unroll
-      for (int e = 0; e < DG; ++e) {
-        const float4 kv = *reinterpret_cast<const float4*>(sK + j * LD + tc * 4 + 64 * e);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          acc[i][e][0] = fmaf(w[i], kv.x, acc[i][e][0]);
-          acc[i][e][1] = fmaf(w[i], kv.y, acc[i][e][1]);
-          acc[i][e][2] = fmaf(w[i], kv.z, acc[i][e][2]);
-          acc[i][e][3] = fmaf(w[i], kv.w, acc[i][e][3]);
+        for (int j = 0; j < NTD / 2; ++j) {   // two dim tiles per ldmatrix
+          const int key = 16 * ks + r8 + (i8 & 1) * 8;
+          const int dim = dh * (DD / 2) + 16 * j + (i8 >> 1) * 8;
+          uint32_t b0, b1, b2, b3;
+          ldsm4t(su32(bK + key * LDB + dim), b0, b1, b2, b3);
+          mma16816(acc[2 * j], af, b0, b1);
+          mma16816(acc[2 * j + 1], af, b2, b3);
         }
       }
     }
-  }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = tr * 4 + i;
-    if (sPos[r] == INT64_MIN) continue;
-    float* out = dq + grow_of(r) * DD;
+    for (int hr = 0; hr < 2; ++hr) {
+      const int r = 16 * rb + g8 + 8 * hr;
+      if (sPos[r] == INT64_MIN) continue;
+      float* out = dq + grow_of(r) * DD + dh * (DD / 2);
 #pragma unroll
-    for (int e = 0; e < DG; ++e)
-      *reinterpret_cast<float4*>(out + tc * 4 + 64 * e) =
-          make_float4(acc[i][e][0] * D.scale, acc[i][e][1] * D.scale, acc[i][e][2] * D.scale,
-                      acc[i][e][3] * D.scale);
+      for (int j = 0; j < NTD; ++j)
+        *reinterpret_cast<float2*>(out + 8 * j + 2 * t4) =
+            make_float2(acc[j][2 * hr] * D.scale, acc[j][2 * hr + 1] * D.scale);
+    }
+  } else {
+    float acc[4][DG][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int e = 0; e < DG; ++e)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[i][e][v] = 0.f;
+    for (int t = 0; t < n_tiles; ++t) {
+      const int64_t k0 = tile_k0(t);
+      __syncthreads();
+      stage_keys<TI, DD, LD, T>(sK, Kb, k0, D.N_kv);
+      stage_keys<TI, DD, LD, T>(sV, Vb, k0, D.N_kv);
+      set_units(k0);
+      __syncthreads();
+      float X[4][KPT], P[4][KPT];
+      logits_tile<DD, T>(sQ, sdO, sK, sV, tr, tc, X, P);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = tr * 4 + i;
+        const int u = sUnit[r];
+        const int64_t pos = sPos[r];
+        const float lam2 = u >= 0 ? sM[r * SU + u] : -INFINITY;
+        const float gam = u >= 0 ? sL[r * SU + u] : 0.f;
+#pragma unroll
+        for (int e = 0; e < KPT; ++e) {
+          const int64_t j = k0 + tc + 16 * e;
+          const bool ok = u >= 0 && j <= pos && j < D.N_kv && lam2 != -INFINITY;
+          const float aw = ok ? exp2f(fmaf(X[i][e], sc2, lam2)) : 0.f;
+          sdX[r * LDA + tc + 16 * e] = aw * (P[i][e] - gam);
+        }
+      }
+      __syncthreads();
+#pragma unroll 4
+      for (int j = 0; j < T; ++j) {
+        float w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] = sdX[(tr * 4 + i) * LDA + j];
+#pragma unroll
+        for (int e = 0; e < DG; ++e) {
+          const float4 kv = *reinterpret_cast<const float4*>(sK + j * LD + tc * 4 + 64 * e);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc[i][e][0] = fmaf(w[i], kv.x, acc[i][e][0]);
+            acc[i][e][1] = fmaf(w[i], kv.y, acc[i][e][1]);
+            acc[i][e][2] = fmaf(w[i], kv.z, acc[i][e][2]);
+            acc[i][e][3] = fmaf(w[i], kv.w, acc[i][e][3]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = tr * 4 + i;
+      if (sPos[r] == INT64_MIN) continue;
+      float* out = dq + grow_of(r) * DD;
+#pragma unroll
+      for (int e = 0; e < DG; ++e)
+        *reinterpret_cast<float4*>(out + tc * 4 + 64 * e) =
+            make_float4(acc[i][e][0] * D.scale, acc[i][e][1] * D.scale, acc[i][e][2] * D.scale,
+                        acc[i][e][3] * D.scale);
+    }
   }
 }
 
@@ -489,7 +766,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // Key-major kernel: CTA = (b, g, keys k0 .. k0 + T - 1 of chunk c = k0 / S).  Its rows are the
 // window rows (queries whose local window [S n, p] reaches the tile: n <= c and p >= k0, all G
 // heads) and the selecting rows (the inverse index of chunk c, all G heads), in batches of 64.
-template <typename TI, int DD, int T>
+// TC: the products on the tensor cores (bf16 inputs), else on the CUDA cores.
+template <typename TI, int DD, int T, bool TC>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_keys_kernel(Dims D, const TI* __restrict__ q, const TI* __restrict__ qc,
                     const TI* __restrict__ K, const TI* __restrict__ V,
@@ -499,21 +777,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     float* __restrict__ dK, float* __restrict__ dV, float* __restrict__ dklm,
                     float* __restrict__ dblm) {
   using SH = BwdShape<DD, T>;
+  using BF = __nv_bfloat16;
   constexpr int LD = SH::LD, LDA = SH::LDA, KPT = SH::KPT, DG = SH::DG;
+  constexpr int LDB = DD + kPadB, LDX = T + kPadB;
+  // tensor-core split of the [T keys x DD] outputs: KB key blocks of 16 x DGW dim groups
+  constexpr int KB = T / 16, DGW = (kBwdThreads / 32) / KB, DPG = DD / DGW, NTK = DPG / 8;
   extern __shared__ float4 smem_f4[];
-  float* sQ = reinterpret_cast<float*>(smem_f4);
+  uint8_t* smem = reinterpret_cast<uint8_t*>(smem_f4);
+  float* sQ = reinterpret_cast<float*>(smem);
   float* sdO = sQ + SH::ROWS_F;
   float* sK = sdO + SH::ROWS_F;
   float* sV = sK + SH::KEYS_F;
   float* sA = sV + SH::KEYS_F;
   float* sdX = sA + SH::TILE_F;
-  int64_t* sPos = reinterpret_cast<int64_t*>(sdX + SH::TILE_F);   // [64]
+  BF* bQ = reinterpret_cast<BF*>(smem);
+  BF* bdO = bQ + kBwdRows * LDB;
+  BF* bK = bdO + kBwdRows * LDB;
+  BF* bV = bK + T * LDB;
+  BF* bA = bV + T * LDB;
+  BF* bdX = bA + kBwdRows * LDX;
+  int64_t* sPos = reinterpret_cast<int64_t*>(smem + keys_prod_bytes<DD, T, TC>());   // [64]
   float* sLam = reinterpret_cast<float*>(sPos + kBwdRows);         // [64]
   float* sGam = sLam + kBwdRows;                                   // [64]
   const TI** rowq = reinterpret_cast<const TI**>(sGam + kBwdRows);   // [64]
   const TI** rowo = rowq + kBwdRows;                                 // [64]
 
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tr = tid >> 4, tc = tid & 15;
   const int G = D.G, Kt = D.K;
   const int64_t bg = blockIdx.y, b = bg / D.Hkv, g = bg - b * D.Hkv;
@@ -534,15 +823,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int32_t* ents = inv_list + bg * D.N_q * Kt + e_lo;
   const int64_t total = (n_win + n_inv) * G;
 
-  stage_keys<TI, DD, LD, T>(sK, K + bg * D.N_kv * DD, k0, D.N_kv);
-  stage_keys<TI, DD, LD, T>(sV, V + bg * D.N_kv * DD, k0, D.N_kv);
-  float aK[KPT][DG][4], aV[KPT][DG][4];
+  if constexpr (TC) {
+    stage_keys_b<DD, T>(bK, reinterpret_cast<const BF*>(K) + bg * D.N_kv * DD, k0, D.N_kv);
+    stage_keys_b<DD, T>(bV, reinterpret_cast<const BF*>(V) + bg * D.N_kv * DD, k0, D.N_kv);
+  } else {
+    stage_keys<TI, DD, LD, T>(sK, K + bg * D.N_kv * DD, k0, D.N_kv);
+    stage_keys<TI, DD, LD, T>(sV, V + bg * D.N_kv * DD, k0, D.N_kv);
+  }
+  float aK[KPT][DG][4], aV[KPT][DG][4];      // CUDA-core accumulators
+  float tK[NTK][4], tV[NTK][4];              // tensor-core accumulators
 #pragma unroll
   for (int i = 0; i < KPT; ++i)
 #pragma unroll
     for (int e = 0; e < DG; ++e)
 #pragma unroll
       for (int v = 0; v < 4; ++v) aK[i][e][v] = aV[i][e][v] = 0.f;
+#pragma unroll
+  for (int j = 0; j < NTK; ++j)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) tK[j][v] = tV[j][v] = 0.f;
 
   for (int64_t f0 = 0; f0 < total; f0 += kBwdRows) {
     __syncthreads();   // the previous batch's tiles are consumed
@@ -577,64 +876,141 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
     __syncthreads();
-    stage_rows<TI, DD, LD>(sQ, rowq, kBwdRows);
-    stage_rows<TI, DD, LD>(sdO, rowo, kBwdRows);
-    __syncthreads();
-    float X[4][KPT], P[4][KPT];
-    logits_tile<DD, T>(sQ, sdO, sK, sV, tr, tc, X, P);
+    if constexpr (TC) {
+      stage_rows_b<DD>(bQ, reinterpret_cast<const BF* const*>(rowq), kBwdRows);
+      stage_rows_b<DD>(bdO, reinterpret_cast<const BF* const*>(rowo), kBwdRows);
+      __syncthreads();
+      const int rb = warp & 3, kh = warp >> 2, g8 = lane >> 2, t4 = lane & 3;
+      float X[T / 16][4], P[T / 16][4];
+      logits_frag<DD, T>(bQ, bdO, bK, bV, rb, kh, X, P);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = tr * 4 + i;
-      const int64_t pos = sPos[r];
-      const float lam2 = sLam[r], gam = sGam[r];
+      for (int hr = 0; hr < 2; ++hr) {
+        const int r = 16 * rb + g8 + 8 * hr;
+        const int64_t pos = sPos[r];
+        const float lam2 = sLam[r], gam = sGam[r];
 #pragma unroll
-      for (int e = 0; e < KPT; ++e) {
-        const int64_t j = k0 + tc + 16 * e;
-        const bool ok = pos != INT64_MIN && j <= pos && j < D.N_kv && lam2 != -INFINITY;
-        const float a = ok ? exp2f(fmaf(X[i][e], sc2, lam2)) : 0.f;
-        sA[r * LDA + tc + 16 * e] = a;
-        sdX[r * LDA + tc + 16 * e] = a * (P[i][e] - gam);
+        for (int j = 0; j < T / 16; ++j) {
+          float aw[2], dx[2];
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+            const int64_t key = k0 + kh * (T / 2) + 8 * j + 2 * t4 + v;
+            const bool ok = pos != INT64_MIN && key <= pos && key < D.N_kv && lam2 != -INFINITY;
+            aw[v] = ok ? exp2f(fmaf(X[j][2 * hr + v], sc2, lam2)) : 0.f;
+            dx[v] = aw[v] * (P[j][2 * hr + v] - gam);
+          }
+          const int col = kh * (T / 2) + 8 * j + 2 * t4;
+          *reinterpret_cast<uint32_t*>(bA + r * LDX + col) = pack_bf16(aw[0], aw[1]);
+          *reinterpret_cast<uint32_t*>(bdX + r * LDX + col) = pack_bf16(dx[0], dx[1]);
+        }
       }
-    }
-    __syncthreads();
+      __syncthreads();
+      // dK += dx^T q, dV += a^T dO over the batch's 64 rows: warp = keys 16 kb .., dims dg DPG ..
+      const int kb = warp % KB, dg = warp / KB;
+      const int i8 = lane >> 3, r8 = lane & 7;
+#pragma unroll
+      for (int ks = 0; ks < kBwdRows / 16; ++ks) {
+        const int srow = 16 * ks + r8 + (i8 >> 1) * 8, skey = 16 * kb + (i8 & 1) * 8;
+        uint32_t ax[4], aa[4];
+        ldsm4t(su32(bdX + srow * LDX + skey), ax[0], ax[1], ax[2], ax[3]);
+        ldsm4t(su32(bA + srow * LDX + skey), aa[0], aa[1], aa[2], aa[3]);
+        if constexpr (NTK == 1) {
+          const int row = 16 * ks + r8 + (i8 & 1) * 8, dim = dg * DPG;
+          uint32_t q0, q1, o0, o1;
+          ldsm2t(su32(bQ + row * LDB + dim), q0, q1);
+          ldsm2t(su32(bdO + row * LDB + dim), o0, o1);
+          mma16816(tK[0], ax, q0, q1);
+          mma16816(tV[0], aa, o0, o1);
+        } else {
+#pragma unroll
+          for (int j = 0; j < NTK / 2; ++j) {
+            const int row = 16 * ks + r8 + (i8 & 1) * 8;
+            const int dim = dg * DPG + 16 * j + (i8 >> 1) * 8;
+            uint32_t q0, q1, q2, q3, o0, o1, o2, o3;
+            ldsm4t(su32(bQ + row * LDB + dim), q0, q1, q2, q3);
+            ldsm4t(su32(bdO + row * LDB + dim), o0, o1, o2, o3);
+            mma16816(tK[2 * j], ax, q0, q1);
+            mma16816(tK[2 * j + 1], ax, q2, q3);
+            mma16816(tV[2 * j], aa, o0, o1);
+            mma16816(tV[2 * j + 1], aa, o2, o3);
+          }
+        }
+      }
+    } else {
+      stage_rows<TI, DD, LD>(sQ, rowq, kBwdRows);
+      stage_rows<TI, DD, LD>(sdO, rowo, kBwdRows);
+      __syncthreads();
+      float X[4][KPT], P[4][KPT];
+      logits_tile<DD, T>(sQ, sdO, sK, sV, tr, tc, X, P);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = tr * 4 + i;
+        const int64_t pos = sPos[r];
+        const float lam2 = sLam[r], gam = sGam[r];
+#pragma unroll
+        for (int e = 0; e < KPT; ++e) {
+          const int64_t j = k0 + tc + 16 * e;
+          const bool ok = pos != INT64_MIN && j <= pos && j < D.N_kv && lam2 != -INFINITY;
+          const float aw = ok ? exp2f(fmaf(X[i][e], sc2, lam2)) : 0.f;
+          sA[r * LDA + tc + 16 * e] = aw;
+          sdX[r * LDA + tc + 16 * e] = aw * (P[i][e] - gam);
+        }
+      }
+      __syncthreads();
 #pragma unroll 2
-    for (int r = 0; r < kBwdRows; ++r) {
-      float xs[KPT], as[KPT];
-#pragma unroll
-      for (int i = 0; i < KPT; ++i) {
-        xs[i] = sdX[r * LDA + tr * KPT + i];
-        as[i] = sA[r * LDA + tr * KPT + i];
-      }
-#pragma unroll
-      for (int e = 0; e < DG; ++e) {
-        const float4 qv = *reinterpret_cast<const float4*>(sQ + r * LD + tc * 4 + 64 * e);
-        const float4 ov = *reinterpret_cast<const float4*>(sdO + r * LD + tc * 4 + 64 * e);
+      for (int r = 0; r < kBwdRows; ++r) {
+        float xs[KPT], as[KPT];
 #pragma unroll
         for (int i = 0; i < KPT; ++i) {
-          aK[i][e][0] = fmaf(xs[i], qv.x, aK[i][e][0]);
-          aK[i][e][1] = fmaf(xs[i], qv.y, aK[i][e][1]);
-          aK[i][e][2] = fmaf(xs[i], qv.z, aK[i][e][2]);
-          aK[i][e][3] = fmaf(xs[i], qv.w, aK[i][e][3]);
-          aV[i][e][0] = fmaf(as[i], ov.x, aV[i][e][0]);
-          aV[i][e][1] = fmaf(as[i], ov.y, aV[i][e][1]);
-          aV[i][e][2] = fmaf(as[i], ov.z, aV[i][e][2]);
-          aV[i][e][3] = fmaf(as[i], ov.w, aV[i][e][3]);
+          xs[i] = sdX[r * LDA + tr * KPT + i];
+          as[i] = sA[r * LDA + tr * KPT + i];
+        }
+#pragma unroll
+        for (int e = 0; e < DG; ++e) {
+          const float4 qv = *reinterpret_cast<const float4*>(sQ + r * LD + tc * 4 + 64 * e);
+          const float4 ov = *reinterpret_cast<const float4*>(sdO + r * LD + tc * 4 + 64 * e);
+#pragma unroll
+          for (int i = 0; i < KPT; ++i) {
+            aK[i][e][0] = fmaf(xs[i], qv.x, aK[i][e][0]);
+            aK[i][e][1] = fmaf(xs[i], qv.y, aK[i][e][1]);
+            aK[i][e][2] = fmaf(xs[i], qv.z, aK[i][e][2]);
+            aK[i][e][3] = fmaf(xs[i], qv.w, aK[i][e][3]);
+            aV[i][e][0] = fmaf(as[i], ov.x, aV[i][e][0]);
+            aV[i][e][1] = fmaf(as[i], ov.y, aV[i][e][1]);
+            aV[i][e][2] = fmaf(as[i], ov.z, aV[i][e][2]);
+            aV[i][e][3] = fmaf(as[i], ov.w, aV[i][e][3]);
+          }
         }
       }
     }
   }
+  if constexpr (TC) {
+    const int kb = warp % KB, dg = warp / KB, g8 = lane >> 2, t4 = lane & 3;
 #pragma unroll
-  for (int i = 0; i < KPT; ++i) {
-    const int64_t j = k0 + tr * KPT + i;
-    if (j >= D.N_kv) continue;
+    for (int hr = 0; hr < 2; ++hr) {
+      const int64_t j = k0 + 16 * kb + g8 + 8 * hr;
+      if (j >= D.N_kv) continue;
 #pragma unroll
-    for (int e = 0; e < DG; ++e) {
-      const int64_t o = (bg * D.N_kv + j) * DD + tc * 4 + 64 * e;
-      *reinterpret_cast<float4*>(dK + o) =
-          make_float4(aK[i][e][0] * D.scale, aK[i][e][1] * D.scale, aK[i][e][2] * D.scale,
-                      aK[i][e][3] * D.scale);
-      *reinterpret_cast<float4*>(dV + o) =
-          make_float4(aV[i][e][0], aV[i][e][1], aV[i][e][2], aV[i][e][3]);
+      for (int jt = 0; jt < NTK; ++jt) {
+        const int64_t o = (bg * D.N_kv + j) * DD + dg * DPG + 8 * jt + 2 * t4;
+        *reinterpret_cast<float2*>(dK + o) =
+            make_float2(tK[jt][2 * hr] * D.scale, tK[jt][2 * hr + 1] * D.scale);
+        *reinterpret_cast<float2*>(dV + o) = make_float2(tV[jt][2 * hr], tV[jt][2 * hr + 1]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < KPT; ++i) {
+      const int64_t j = k0 + tr * KPT + i;
+      if (j >= D.N_kv) continue;
+#pragma unroll
+      for (int e = 0; e < DG; ++e) {
+        const int64_t o = (bg * D.N_kv + j) * DD + tc * 4 + 64 * e;
+        *reinterpret_cast<float4*>(dK + o) =
+            make_float4(aK[i][e][0] * D.scale, aK[i][e][1] * D.scale, aK[i][e][2] * D.scale,
+                        aK[i][e][3] * D.scale);
+        *reinterpret_cast<float4*>(dV + o) =
+            make_float4(aV[i][e][0], aV[i][e][1], aV[i][e][2], aV[i][e][3]);
+      }
     }
   }
 
@@ -653,7 +1029,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       dsum += dsc;
     }
     __syncthreads();
-    float* red = sA;   // [PARTS][DD + 1]
+    float* red = reinterpret_cast<float*>(smem);   // [PARTS][DD + 1] (the products' area)
     red[part * (DD + 1) + dim] = acc;
     if (dim == 0) red[part * (DD + 1) + DD] = dsum;
     __syncthreads();
@@ -736,28 +1112,27 @@ __global__ void __launch_bounds__(256)
 // ---------------------------------------------------------------------------------------------
 namespace {
 
-template <int DD, int T>
+template <int DD, int T, bool TC>
 constexpr size_t rows_smem() {
-  using SH = BwdShape<DD, T>;
-  return (size_t)(2 * SH::ROWS_F + 2 * SH::KEYS_F + SH::TILE_F + 3 * kBwdRows * (kBwdMaxK + 1) +
-                  kBwdRows * kBwdMaxK) * 4 +
+  return (size_t)rows_prod_bytes<DD, T, TC>() +
+         (size_t)(3 * kBwdRows * (kBwdMaxK + 1) + kBwdRows * kBwdMaxK) * 4 +
          (size_t)2 * kBwdMaxUnion * 4 + kBwdRows * 8 + kBwdRows * 4 + kBwdRows * 4 + 8 +
          kBwdRows * 8 + 16;
 }
 
-template <int DD, int T>
+template <int DD, int T, bool TC>
 constexpr size_t keys_smem() {
-  using SH = BwdShape<DD, T>;
-  return (size_t)(2 * SH::ROWS_F + 2 * SH::KEYS_F + 2 * SH::TILE_F) * 4 + kBwdRows * 8 +
-         2 * kBwdRows * 4 + 2 * kBwdRows * 8;
+  return (size_t)keys_prod_bytes<DD, T, TC>() + kBwdRows * 8 + 2 * kBwdRows * 4 +
+         2 * kBwdRows * 8;
 }
 
 template <typename TI, int DD, int T>
 cudaError_t launch_bwd_t(const Dims& D, const BwdArgs& a, const BwdWs& w, cudaStream_t st) {
-  constexpr size_t RS = rows_smem<DD, T>(), KS = keys_smem<DD, T>();
+  constexpr bool TC = std::is_same<TI, __nv_bfloat16>::value;
+  constexpr size_t RS = rows_smem<DD, T, TC>(), KS = keys_smem<DD, T, TC>();
   static_assert(RS <= 227 * 1024 && KS <= 227 * 1024, "shared memory");
-  auto kr = bwd_rows_kernel<TI, DD, T>;
-  auto kk = bwd_keys_kernel<TI, DD, T>;
+  auto kr = bwd_rows_kernel<TI, DD, T, TC>;
+  auto kk = bwd_keys_kernel<TI, DD, T, TC>;
   cudaError_t e = cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RS);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KS);

@@ -4,12 +4,15 @@ Both sides differentiate sum(dout * out) + sum(dlse * lse) with the same selecti
 oracle's own forward makes (the top-K passes no gradient).  Every gradient element is compared:
 dq, dq_cal, dK, dV, dk_lm, db_lm.
 
-Tolerance.  The CUDA path stages every operand as fp32 and forms every product and sum in fp32
-(bf16 inputs are exact in fp32), so the only differences from the fp64 oracle are fp32
-rounding: of the logits (|x| eps), of the exponentials (a few ulp), and of sums of up to a few
-thousand terms per output.  Per gradient tensor and (b, kv-group) plane the largest absolute
-difference must stay within 3e-5 of that plane's largest reference magnitude (about 250 fp32
-ulps at that scale, room for sums of ~10^4 terms), for both input dtypes.
+Tolerance, per gradient tensor and (b, head or kv-group) plane, on the largest absolute
+difference relative to the plane's largest reference magnitude.
+* fp32 inputs: every product and sum is fp32, so the only differences from the fp64 oracle are
+  fp32 rounding (logits, exponentials, sums of up to ~10^4 terms): 3e-5 (about 250 fp32 ulps).
+* bf16 inputs: the logits and dout . V products take the inputs exactly, but the fused weights
+  a and the logit gradients dx enter the dq, dK and dV products rounded to bf16 (relative error
+  up to 2^-9 per term, independent between terms), so an output's error is a sum of n terms
+  each off by up to 2^-9 of itself: about 2^-9 / sqrt(3) * ||terms||_2, far below the plane's
+  maximum for the row counts here; 1e-2 of the plane's maximum bounds it with room.
 
 At the full 7B-like size (N = 131072) the oracle runs one query at a time: the sampled queries'
 dq and dq_cal rows (which depend on that query alone) are compared under the same rule, and two
@@ -47,7 +50,11 @@ def _arrays(wl):
     return [parity.f64(t) for t in (wl.q, wl.q_cal, wl.K, wl.V, wl.k_lm, wl.b_lm)]
 
 
-def _compare(got, want, name):
+def _tol(dtype):
+    return 3e-5 if dtype == torch.float32 else 1e-2
+
+
+def _compare(got, want, name, tol=TOL):
     got = got.detach().cpu().double().numpy()
     assert np.isfinite(got).all(), name
     assert got.shape == want.shape, (name, got.shape, want.shape)
@@ -62,7 +69,7 @@ def _compare(got, want, name):
             assert err == 0.0, (name, p, err)
             continue
         worst = max(worst, err / scale)
-        assert err <= TOL * scale, (name, p, err, scale)
+        assert err <= tol * scale, (name, p, err, scale)
     return worst
 
 
@@ -75,7 +82,8 @@ def _check_all(wl, dout, dlse):
     got = hb.backward(wl.q, wl.q_cal, wl.K, wl.V, wl.k_lm, wl.b_lm,
                       torch.from_numpy(idx).cuda(), dout, dlse, **kw)
     torch.cuda.synchronize()
-    return {name: _compare(got[name], ref[oname], name) for name, oname in GRADS}
+    return {name: _compare(got[name], ref[oname], name, _tol(wl.q.dtype))
+            for name, oname in GRADS}
 
 
 def _suffix(wl, n_q):
@@ -102,7 +110,7 @@ def test_backward_matches_oracle(name, kw, n_q):
     if n_q is not None:   # (the oracle's cost grows with W + K S per row)
         wl = _suffix(wl, n_q)
     dout, dlse = _upstream(wl, seed=len(name) + wl.q.shape[2])
-    _check_all(wl, dout, dlse)
+    print("worst |diff| / plane max:", name, kw, _check_all(wl, dout, dlse))
 
 
 def _random(B, Hq, Hkv, N, d, S, K, W_, dtype, seed, q_pos0=0, N_q=None):
@@ -136,7 +144,7 @@ def test_backward_edge_cases(case):
     kw = dict(EDGE[case])
     wl = _random(**kw, seed=len(case) * 7)
     dout, dlse = _upstream(wl, seed=3, with_dlse=case != "k0_window_only")
-    _check_all(wl, dout, dlse)
+    print("worst |diff| / plane max:", case, _check_all(wl, dout, dlse))
 
 
 def spread_selection(B, Hkv, N_q, K, S, W, q_pos0, seed):
@@ -192,5 +200,5 @@ def test_backward_full_size_sampled():
                                   Kf, Vf, klm, blm, idx[:, g:g + 1, sl].cpu().numpy(),
                                   parity.f64(dout[:, hs, sl]), parity.f64(dlse[:, hs, sl]),
                                   S=wl.S, K_top=wl.K_top, W=wl.W, q_pos0=i)
-            _compare(got["dq"][:, hs, sl], ref["dq"], "dq")
-            _compare(got["dq_cal"][:, hs, sl], ref["dqc"], "dq_cal")
+            _compare(got["dq"][:, hs, sl], ref["dq"], "dq", _tol(wl.q.dtype))
+            _compare(got["dq_cal"][:, hs, sl], ref["dqc"], "dq_cal", _tol(wl.q.dtype))
