@@ -36,7 +36,12 @@ namespace {
 constexpr int kBwdRows = 64;      // rows per batch
 constexpr int kBwdThreads = 256;
 constexpr int kBwdMaxK = 32;
-constexpr int kBwdMaxUnion = kBwdRows * kBwdMaxK;   // selected ids of one row tile
+
+__host__ __device__ constexpr int pow2_at_least(int n) {
+  int p = 1;
+  while (p < n) p <<= 1;
+  return p;
+}
 constexpr float kB2 = 1.4426950408889634f;          // log2(e)
 constexpr float kLn2b = 0.6931471805599453f;
 
@@ -176,6 +181,47 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// 16-byte asynchronous global -> shared copies (zero-filled when src_bytes is 0), in groups.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(su32(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// Rows r < n of a bf16 [n][DD + kPadB] tile from rowp[r] (nullptr: zeros), asynchronously (one
+// commit group per call).
+template <int DD>
+__device__ __forceinline__ void fetch_rows_b(__nv_bfloat16* dst, const __nv_bfloat16* const* rowp,
+                                             int n, const __nv_bfloat16* any) {
+  constexpr int PPR = DD / 8, LDB = DD + kPadB;
+  for (int e = threadIdx.x; e < n * PPR; e += kBwdThreads) {
+    const int r = e / PPR, u = e - r * PPR;
+    const __nv_bfloat16* src = rowp[r];
+    cp_async16(dst + r * LDB + u * 8, src ? src + u * 8 : any, src ? 16u : 0u);
+  }
+  cp_async_commit();
+}
+
+// Keys k0 .. k0 + T - 1 of one (b, g) plane, bf16 [T][DD + kPadB], asynchronously (zeros past
+// N_kv; no commit).
+template <int DD, int T>
+__device__ __forceinline__ void fetch_keys_b(__nv_bfloat16* dst, const __nv_bfloat16* base,
+                                             int64_t k0, int64_t nkv) {
+  constexpr int PPR = DD / 8, LDB = DD + kPadB;
+  for (int e = threadIdx.x; e < T * PPR; e += kBwdThreads) {
+    const int r = e / PPR, u = e - r * PPR;
+    const bool in = k0 + r < nkv;
+    cp_async16(dst + r * LDB + u * 8, in ? base + (k0 + r) * DD + u * 8 : base, in ? 16u : 0u);
+  }
+}
+
 // Rows r < n of a bf16 [n][DD + kPadB] tile from rowp[r] (nullptr: zeros).
 template <int DD>
 __device__ __forceinline__ void stage_rows_b(__nv_bfloat16* dst,
@@ -251,14 +297,14 @@ __device__ __forceinline__ void logits_frag(const __nv_bfloat16* sQ, const __nv_
 template <int DD, int T, bool TC>
 constexpr int rows_prod_bytes() {
   using SH = BwdShape<DD, T>;
-  return TC ? ((2 * kBwdRows + 2 * T) * (DD + kPadB) + kBwdRows * (T + kPadB)) * 2 +
+  return TC ? ((2 * kBwdRows + 4 * T) * (DD + kPadB) + kBwdRows * (T + kPadB)) * 2 +
                   2 * kBwdRows * 3 * 4
             : (2 * SH::ROWS_F + 2 * SH::KEYS_F + SH::TILE_F) * 4;
 }
 template <int DD, int T, bool TC>
 constexpr int keys_prod_bytes() {
   using SH = BwdShape<DD, T>;
-  return TC ? ((2 * kBwdRows + 2 * T) * (DD + kPadB) + 2 * kBwdRows * (T + kPadB)) * 2
+  return TC ? ((4 * kBwdRows + 2 * T) * (DD + kPadB) + 2 * kBwdRows * (T + kPadB)) * 2
             : (2 * SH::ROWS_F + 2 * SH::KEYS_F + 2 * SH::TILE_F) * 4;
 }
 
@@ -278,7 +324,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     float* __restrict__ gam_ws, float* __restrict__ ds_ws) {
   using SH = BwdShape<DD, T>;
   constexpr int LD = SH::LD, LDA = SH::LDA, KPT = SH::KPT, DG = SH::DG;
-  constexpr int SU = kBwdMaxK + 1;   // stats row stride (units)
+  const int SU = D.K + 1;   // stats row stride (units)
   using BF = __nv_bfloat16;
   constexpr int LDB = DD + kPadB, LDX = T + kPadB;
   extern __shared__ float4 smem_f4[];
@@ -291,18 +337,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   float* sdX = sV + SH::KEYS_F;
   BF* bQ = reinterpret_cast<BF*>(smem);
   BF* bdO = bQ + kBwdRows * LDB;
-  BF* bK = bdO + kBwdRows * LDB;
-  BF* bV = bK + T * LDB;
-  BF* bdX = bV + T * LDB;
+  BF* bK = bdO + kBwdRows * LDB;   // [2][T][LDB]: the next tile's keys load meanwhile
+  BF* bV = bK + 2 * T * LDB;       // [2][T][LDB]
+  BF* bdX = bV + 2 * T * LDB;
   float* sPart = reinterpret_cast<float*>(bdX + kBwdRows * LDX);   // [2 key halves][64][3]
   float* sM = reinterpret_cast<float*>(smem + rows_prod_bytes<DD, T, TC>());   // [64][SU] running
                                                                            // max (base 2), then lambda2
   float* sL = sM + kBwdRows * SU;            // running sum, then gamma
   float* sT = sL + kBwdRows * SU;            // running sum of p dP, then dscore
-  float* sS = sT + kBwdRows * SU;            // [64][32] chunk scores
-  int* sel = reinterpret_cast<int*>(sS + kBwdRows * kBwdMaxK);   // [QT][K]
-  int* sU = sel + kBwdMaxUnion;              // selected chunks below the window range, sorted
-  int64_t* sPos = reinterpret_cast<int64_t*>(sU + kBwdMaxUnion);   // [64]
+  float* sS = sT + kBwdRows * SU;            // [64][SU] chunk scores
+  // bookkeeping sized for this launch's K and G (see rows_smem)
+  const int n_ids = (kBwdRows / D.G) * D.K;
+  int* sel = reinterpret_cast<int*>(sS + kBwdRows * SU);   // [QT][K]
+  int* sU = sel + ((n_ids + 1) & ~1);        // selected chunks below the window range, sorted
+  int64_t* sPos = reinterpret_cast<int64_t*>(
+      sU + ((pow2_at_least(n_ids) + 1) & ~1));   // [64] (8-byte aligned: even int counts)
   float* sDl = reinterpret_cast<float*>(sPos + kBwdRows);          // [64] dlse
   int* sUnit = reinterpret_cast<int*>(sDl + kBwdRows);             // [64]
   const TI** rowp = reinterpret_cast<const TI**>(sUnit + kBwdRows + 2);   // [64]
@@ -331,8 +380,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
   const int64_t c_lo = n_eligible(D.q_pos0 + i0, D.S, D.W);
   const int64_t c_hi = (D.q_pos0 + i0 + nq - 1) / D.S;
-  int np = 1;
-  while (np < QT * Kt) np <<= 1;
+  const int np = pow2_at_least(QT * Kt);
   for (int e = tid; e < np; e += kBwdThreads) {
     int c = INT_MAX;
     if (e < QT * Kt) {
@@ -421,6 +469,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   };
 
+  // tensor cores: tile t's keys and values into buffer t & 1, one commit group
+  auto fetch_kv = [&](int t) {
+    const int64_t k0 = tile_k0(t);
+    fetch_keys_b<DD, T>(bK + (t & 1) * T * LDB, reinterpret_cast<const BF*>(Kb), k0, D.N_kv);
+    fetch_keys_b<DD, T>(bV + (t & 1) * T * LDB, reinterpret_cast<const BF*>(Vb), k0, D.N_kv);
+    cp_async_commit();
+  };
   // merges a tile's (max, sum, sum p dP) of row r's unit u into the running state
   auto merge_stats = [&](int r, int u, float m, float l, float tt) {
     if (u < 0 || m == -INFINITY) return;
@@ -441,11 +496,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   };
 
   // ---- pass 1: per (row, unit) lse and delta = dO . o_u by online reduction
+  if constexpr (TC) {
+    if (n_tiles > 0) fetch_kv(0);
+  }
   for (int t = 0; t < n_tiles; ++t) {
     const int64_t k0 = tile_k0(t);
     if constexpr (TC) {
-      stage_keys_b<DD, T>(bK, reinterpret_cast<const BF*>(Kb), k0, D.N_kv);
-      stage_keys_b<DD, T>(bV, reinterpret_cast<const BF*>(Vb), k0, D.N_kv);
+      if (t + 1 < n_tiles) fetch_kv(t + 1);
+      else cp_async_commit();
+      cp_async_wait<1>();   // tile t has landed (this thread's copies; the barrier below: all)
     } else {
       stage_keys<TI, DD, LD, T>(sK, Kb, k0, D.N_kv);
       stage_keys<TI, DD, LD, T>(sV, Vb, k0, D.N_kv);
@@ -456,7 +515,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // warp: rows 16 rb .., keys kh T/2 ..; a row's values sit in the 4 lanes of its quad
       const int rb = warp & 3, kh = warp >> 2, g8 = lane >> 2, t4 = lane & 3;
       float X[T / 16][4], P[T / 16][4];
-      logits_frag<DD, T>(bQ, bdO, bK, bV, rb, kh, X, P);
+      logits_frag<DD, T>(bQ, bdO, bK + (t & 1) * T * LDB, bV + (t & 1) * T * LDB, rb, kh, X, P);
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr) {
         const int r = 16 * rb + g8 + 8 * hr;
@@ -562,7 +621,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
       for (int e = 0; e < DL; ++e) a = fmaf(qv[e], Elem<TI>::to_f(kr[e]), a);
       a = warp_sum(a);
-      if (lane == 0) sS[r * kBwdMaxK + k] = fmaf(a, D.scale, blm[bg * D.C + c]);
+      if (lane == 0) sS[r * SU + k] = fmaf(a, D.scale, blm[bg * D.C + c]);
     }
   }
   __syncthreads();
@@ -578,7 +637,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool present = u == Kt || (sr[u] >= 0 && Ls[u] > 0.f);
       const float lse = present ? (M[u] + log2f(Ls[u])) * kLn2b : -INFINITY;
       const float dlt = present ? Ts[u] / Ls[u] : 0.f;
-      const float score = u == Kt ? lse : (present ? sS[r * kBwdMaxK + u] : -INFINITY);
+      const float score = u == Kt ? lse : (present ? sS[r * SU + u] : -INFINITY);
       M[u] = lse;
       Ts[u] = dlt;
       Ls[u] = score;
@@ -639,15 +698,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int j = 0; j < NTD; ++j)
 #pragma unroll
       for (int v = 0; v < 4; ++v) acc[j][v] = 0.f;
+    __syncthreads();   // (pass 1's tiles are consumed)
+    if (n_tiles > 0) fetch_kv(0);
     for (int t = 0; t < n_tiles; ++t) {
       const int64_t k0 = tile_k0(t);
-      __syncthreads();
-      stage_keys_b<DD, T>(bK, reinterpret_cast<const BF*>(Kb), k0, D.N_kv);
-      stage_keys_b<DD, T>(bV, reinterpret_cast<const BF*>(Vb), k0, D.N_kv);
+      __syncthreads();   // the previous tile is consumed: its buffer takes tile t + 1
+      if (t + 1 < n_tiles) fetch_kv(t + 1);
+      else cp_async_commit();
+      cp_async_wait<1>();
       set_units(k0);
       __syncthreads();
+      const BF* bKt = bK + (t & 1) * T * LDB;
       float X[T / 16][4], P[T / 16][4];
-      logits_frag<DD, T>(bQ, bdO, bK, bV, rb, kh, X, P);
+      logits_frag<DD, T>(bQ, bdO, bKt, bV + (t & 1) * T * LDB, rb, kh, X, P);
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr) {
         const int r = 16 * rb + g8 + 8 * hr;
@@ -681,7 +744,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const int key = 16 * ks + r8 + (i8 & 1) * 8;
           const int dim = dh * (DD / 2) + 16 * j + (i8 >> 1) * 8;
           uint32_t b0, b1, b2, b3;
-          ldsm4t(su32(bK + key * LDB + dim), b0, b1, b2, b3);
+          ldsm4t(su32(bKt + key * LDB + dim), b0, b1, b2, b3);
           mma16816(acc[2 * j], af, b0, b1);
           mma16816(acc[2 * j + 1], af, b2, b3);
         }
@@ -790,17 +853,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   float* sV = sK + SH::KEYS_F;
   float* sA = sV + SH::KEYS_F;
   float* sdX = sA + SH::TILE_F;
-  BF* bQ = reinterpret_cast<BF*>(smem);
-  BF* bdO = bQ + kBwdRows * LDB;
-  BF* bK = bdO + kBwdRows * LDB;
+  BF* bQ = reinterpret_cast<BF*>(smem);   // [2][64][LDB]: the next batch's rows load meanwhile
+  BF* bdO = bQ + 2 * kBwdRows * LDB;      // [2][64][LDB]
+  BF* bK = bdO + 2 * kBwdRows * LDB;
   BF* bV = bK + T * LDB;
   BF* bA = bV + T * LDB;
   BF* bdX = bA + kBwdRows * LDX;
-  int64_t* sPos = reinterpret_cast<int64_t*>(smem + keys_prod_bytes<DD, T, TC>());   // [64]
-  float* sLam = reinterpret_cast<float*>(sPos + kBwdRows);         // [64]
-  float* sGam = sLam + kBwdRows;                                   // [64]
-  const TI** rowq = reinterpret_cast<const TI**>(sGam + kBwdRows);   // [64]
-  const TI** rowo = rowq + kBwdRows;                                 // [64]
+  // row bookkeeping of a batch, [2] buffers (the CUDA-core path uses the first)
+  int64_t* sPos = reinterpret_cast<int64_t*>(smem + keys_prod_bytes<DD, T, TC>());   // [2][64]
+  float* sLam = reinterpret_cast<float*>(sPos + 2 * kBwdRows);     // [2][64]
+  float* sGam = sLam + 2 * kBwdRows;                               // [2][64]
+  const TI** rowq = reinterpret_cast<const TI**>(sGam + 2 * kBwdRows);   // [2][64]
+  const TI** rowo = rowq + 2 * kBwdRows;                                 // [2][64]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tr = tid >> 4, tc = tid & 15;
@@ -843,10 +907,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
     for (int v = 0; v < 4; ++v) tK[j][v] = tV[j][v] = 0.f;
 
-  for (int64_t f0 = 0; f0 < total; f0 += kBwdRows) {
-    __syncthreads();   // the previous batch's tiles are consumed
+  // the rows f0 .. f0 + 63 of the tile's row list into bookkeeping buffer `buf` (threads < 64)
+  auto prep = [&](int64_t f0, int buf) {
     if (tid < kBwdRows) {
       const int64_t f = f0 + tid;
+      const int o = buf * kBwdRows + tid;
       if (f < total) {
         int64_t qi;
         int u, h;
@@ -862,32 +927,60 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           h = (int)(fe % G);
         }
         const int64_t grow = (b * D.Hq + g * G + h) * D.N_q + qi;
-        sPos[tid] = D.q_pos0 + qi;
-        sLam[tid] = lam_ws[grow * (Kt + 1) + u];
-        sGam[tid] = gam_ws[grow * (Kt + 1) + u];
-        rowq[tid] = q + grow * DD;
-        rowo[tid] = dO + grow * DD;
+        sPos[o] = D.q_pos0 + qi;
+        sLam[o] = lam_ws[grow * (Kt + 1) + u];
+        sGam[o] = gam_ws[grow * (Kt + 1) + u];
+        rowq[o] = q + grow * DD;
+        rowo[o] = dO + grow * DD;
       } else {
-        sPos[tid] = INT64_MIN;
-        sLam[tid] = -INFINITY;
-        sGam[tid] = 0.f;
-        rowq[tid] = nullptr;
-        rowo[tid] = nullptr;
+        sPos[o] = INT64_MIN;
+        sLam[o] = -INFINITY;
+        sGam[o] = 0.f;
+        rowq[o] = nullptr;
+        rowo[o] = nullptr;
       }
     }
-    __syncthreads();
-    if constexpr (TC) {
-      stage_rows_b<DD>(bQ, reinterpret_cast<const BF* const*>(rowq), kBwdRows);
-      stage_rows_b<DD>(bdO, reinterpret_cast<const BF* const*>(rowo), kBwdRows);
+  };
+  if constexpr (TC) {
+    // batch i computes from buffer i & 1 while batch i + 1's rows load into the other
+    auto fetch = [&](int buf) {
+      fetch_rows_b<DD>(bQ + buf * kBwdRows * LDB,
+                       reinterpret_cast<const BF* const*>(rowq + buf * kBwdRows), kBwdRows,
+                       reinterpret_cast<const BF*>(q));
+      fetch_rows_b<DD>(bdO + buf * kBwdRows * LDB,
+                       reinterpret_cast<const BF* const*>(rowo + buf * kBwdRows), kBwdRows,
+                       reinterpret_cast<const BF*>(dO));
+    };
+    if (total > 0) {
+      prep(0, 0);
       __syncthreads();
+      fetch(0);
+    }
+    int bi = 0;
+    for (int64_t f0 = 0; f0 < total; f0 += kBwdRows, ++bi) {
+      const int buf = bi & 1;
+      if (f0 + kBwdRows < total) {
+        prep(f0 + kBwdRows, buf ^ 1);
+        __syncthreads();
+        fetch(buf ^ 1);
+        cp_async_wait<2>();   // this batch's two groups have landed
+      } else {
+        cp_async_wait<0>();
+      }
+      __syncthreads();
+      const BF* cQ = bQ + buf * kBwdRows * LDB;
+      const BF* cdO = bdO + buf * kBwdRows * LDB;
+      const int64_t* cPos = sPos + buf * kBwdRows;
+      const float* cLam = sLam + buf * kBwdRows;
+      const float* cGam = sGam + buf * kBwdRows;
       const int rb = warp & 3, kh = warp >> 2, g8 = lane >> 2, t4 = lane & 3;
       float X[T / 16][4], P[T / 16][4];
-      logits_frag<DD, T>(bQ, bdO, bK, bV, rb, kh, X, P);
+      logits_frag<DD, T>(cQ, cdO, bK, bV, rb, kh, X, P);
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr) {
         const int r = 16 * rb + g8 + 8 * hr;
-        const int64_t pos = sPos[r];
-        const float lam2 = sLam[r], gam = sGam[r];
+        const int64_t pos = cPos[r];
+        const float lam2 = cLam[r], gam = cGam[r];
 #pragma unroll
         for (int j = 0; j < T / 16; ++j) {
           float aw[2], dx[2];
@@ -916,8 +1009,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if constexpr (NTK == 1) {
           const int row = 16 * ks + r8 + (i8 & 1) * 8, dim = dg * DPG;
           uint32_t q0, q1, o0, o1;
-          ldsm2t(su32(bQ + row * LDB + dim), q0, q1);
-          ldsm2t(su32(bdO + row * LDB + dim), o0, o1);
+          ldsm2t(su32(cQ + row * LDB + dim), q0, q1);
+          ldsm2t(su32(cdO + row * LDB + dim), o0, o1);
           mma16816(tK[0], ax, q0, q1);
           mma16816(tV[0], aa, o0, o1);
         } else {
@@ -926,8 +1019,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int row = 16 * ks + r8 + (i8 & 1) * 8;
             const int dim = dg * DPG + 16 * j + (i8 >> 1) * 8;
             uint32_t q0, q1, q2, q3, o0, o1, o2, o3;
-            ldsm4t(su32(bQ + row * LDB + dim), q0, q1, q2, q3);
-            ldsm4t(su32(bdO + row * LDB + dim), o0, o1, o2, o3);
+            ldsm4t(su32(cQ + row * LDB + dim), q0, q1, q2, q3);
+            ldsm4t(su32(cdO + row * LDB + dim), o0, o1, o2, o3);
             mma16816(tK[2 * j], ax, q0, q1);
             mma16816(tK[2 * j + 1], ax, q2, q3);
             mma16816(tV[2 * j], aa, o0, o1);
@@ -935,7 +1028,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
         }
       }
-    } else {
+      __syncthreads();   // the batch's buffers are consumed (the next prep and fetch reuse them)
+    }
+  } else {
+  for (int64_t f0 = 0; f0 < total; f0 += kBwdRows) {
+    __syncthreads();   // the previous batch's tiles are consumed
+    prep(f0, 0);
+    __syncthreads();
+    {
       stage_rows<TI, DD, LD>(sQ, rowq, kBwdRows);
       stage_rows<TI, DD, LD>(sdO, rowo, kBwdRows);
       __syncthreads();
@@ -982,6 +1082,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
     }
+  }
   }
   if constexpr (TC) {
     const int kb = warp % KB, dg = warp / KB, g8 = lane >> 2, t4 = lane & 3;
@@ -1112,25 +1213,30 @@ __global__ void __launch_bounds__(256)
 // ---------------------------------------------------------------------------------------------
 namespace {
 
+// Shared memory of the query-major kernel for this launch: the product operands, then the
+// per-(row, unit) state, the chunk scores, the selections of the block's queries, the sorted
+// union and the row bookkeeping.
 template <int DD, int T, bool TC>
-constexpr size_t rows_smem() {
-  return (size_t)rows_prod_bytes<DD, T, TC>() +
-         (size_t)(3 * kBwdRows * (kBwdMaxK + 1) + kBwdRows * kBwdMaxK) * 4 +
-         (size_t)2 * kBwdMaxUnion * 4 + kBwdRows * 8 + kBwdRows * 4 + kBwdRows * 4 + 8 +
-         kBwdRows * 8 + 16;
+size_t rows_smem(const Dims& D) {
+  const int SU = D.K + 1, n_ids = (kBwdRows / D.G) * D.K;
+  return (size_t)rows_prod_bytes<DD, T, TC>() + (size_t)(4 * kBwdRows * SU) * 4 +
+         (size_t)(((n_ids + 1) & ~1) + ((pow2_at_least(n_ids) + 1) & ~1)) * 4 + kBwdRows * 8 +
+         kBwdRows * 4 + kBwdRows * 4 + 8 + kBwdRows * 8 + 16;
 }
 
 template <int DD, int T, bool TC>
 constexpr size_t keys_smem() {
-  return (size_t)keys_prod_bytes<DD, T, TC>() + kBwdRows * 8 + 2 * kBwdRows * 4 +
-         2 * kBwdRows * 8;
+  return (size_t)keys_prod_bytes<DD, T, TC>() + 2 * (kBwdRows * 8 + 2 * kBwdRows * 4 +
+                                                    2 * kBwdRows * 8);
 }
 
 template <typename TI, int DD, int T>
 cudaError_t launch_bwd_t(const Dims& D, const BwdArgs& a, const BwdWs& w, cudaStream_t st) {
   constexpr bool TC = std::is_same<TI, __nv_bfloat16>::value;
-  constexpr size_t RS = rows_smem<DD, T, TC>(), KS = keys_smem<DD, T, TC>();
-  static_assert(RS <= 227 * 1024 && KS <= 227 * 1024, "shared memory");
+  const size_t RS = rows_smem<DD, T, TC>(D);
+  constexpr size_t KS = keys_smem<DD, T, TC>();
+  static_assert(KS <= 227 * 1024, "shared memory");
+  if (RS > 227 * 1024) return cudaErrorInvalidValue;
   auto kr = bwd_rows_kernel<TI, DD, T, TC>;
   auto kk = bwd_keys_kernel<TI, DD, T, TC>;
   cudaError_t e = cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RS);
