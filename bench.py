@@ -697,13 +697,17 @@ def extra_backward(peaks, name="gqa7b_prefill", steps=3, **overrides):
     slots = float(np.minimum(n, wl.K_top).sum()) * wl.dims["B"] * wl.dims["Hq"]
     flops = 2.5 * wm["attn_flops"] + 4.0 * wl.dims["d"] * slots
     tf = flops / (t * 1e-3) / 1e12
+    if wl.q.dtype == torch.bfloat16:   # products on the tensor cores (m16n8k16 bf16 tiles)
+        rl = {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+              "frac": tf / peaks["bf16_tflops"]}
+    else:                              # fp32 products on the CUDA cores
+        rl = {"bound": "alu", "achieved": tf, "peak": FP32_FMA_TFLOPS, "unit": "TFLOP/s",
+              "frac": tf / FP32_FMA_TFLOPS,
+              "peak_note": "fp32 FMA of the CUDA cores, 148 SMs x 128 lanes x 2 x 1.965 GHz"}
     out = {"kernel": "bwd_rows + bwd_keys (+ index build)", "workload": name,
            "shape": {k: wl.dims[k] for k in ("B", "Hq", "Hkv", "N_q", "N_kv", "d")},
            "ms": t, "tflop": flops / 1e12, "tokens_per_s": wl.dims["B"] * wl.dims["N_q"] / (t * 1e-3),
-           "roofline": {"bound": "alu", "achieved": tf, "peak": FP32_FMA_TFLOPS,
-                        "unit": "TFLOP/s", "frac": tf / FP32_FMA_TFLOPS,
-                        "peak_note": "fp32 FMA of the CUDA cores, 148 SMs x 128 lanes x 2 x 1.965 GHz"},
-           "frac_of_bf16_tensor_peak": tf / peaks["bf16_tflops"]}
+           "roofline": rl}
     del wl, grads, ws, dout, dlse, idx
     torch.cuda.empty_cache()
     return out

@@ -608,20 +608,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // ---- fusion terms per row
   for (int r = warp; r < kBwdRows; r += kBwdThreads / 32) {   // chunk scores s = scale qc.klm + b
     if (sPos[r] == INT64_MIN) continue;
-    constexpr int DL = DD / 32;
+    constexpr int DL = DD / 32, U = 8;
     float qv[DL];
     const TI* qr = qc + grow_of(r) * DD + lane * DL;
 #pragma unroll
     for (int e = 0; e < DL; ++e) qv[e] = Elem<TI>::to_f(qr[e]);
-    for (int k = 0; k < Kt; ++k) {
-      const int c = sel[(r / G) * Kt + k];
-      if (c < 0) continue;
-      const TI* kr = klm + (bg * D.C + c) * DD + lane * DL;
-      float a = 0.f;
+    for (int k0 = 0; k0 < Kt; k0 += U) {   // eight landmark rows' loads in flight together
+      int cs[U];
+      float kv[U][DL], bias[U];
 #pragma unroll
-      for (int e = 0; e < DL; ++e) a = fmaf(qv[e], Elem<TI>::to_f(kr[e]), a);
-      a = warp_sum(a);
-      if (lane == 0) sS[r * SU + k] = fmaf(a, D.scale, blm[bg * D.C + c]);
+      for (int j = 0; j < U; ++j) {
+        cs[j] = k0 + j < Kt ? sel[(r / G) * Kt + k0 + j] : -1;
+        const TI* kr = klm + (bg * D.C + (cs[j] < 0 ? 0 : cs[j])) * DD + lane * DL;
+#pragma unroll
+        for (int e = 0; e < DL; ++e) kv[j][e] = cs[j] >= 0 ? Elem<TI>::to_f(kr[e]) : 0.f;
+        bias[j] = cs[j] >= 0 ? blm[bg * D.C + cs[j]] : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < U; ++j) {
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < DL; ++e) a = fmaf(qv[e], kv[j][e], a);
+        a = warp_sum(a);
+        if (lane == 0 && cs[j] >= 0) sS[r * SU + k0 + j] = fmaf(a, D.scale, bias[j]);
+      }
     }
   }
   __syncthreads();
@@ -669,17 +679,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   for (int r = warp; r < kBwdRows; r += kBwdThreads / 32) {   // d q_cal = scale sum ds k_lm
     if (sPos[r] == INT64_MIN) continue;
-    constexpr int DL = DD / 32;
+    constexpr int DL = DD / 32, U = 8;
     float acc[DL];
 #pragma unroll
     for (int e = 0; e < DL; ++e) acc[e] = 0.f;
-    for (int k = 0; k < Kt; ++k) {
-      const int c = sel[(r / G) * Kt + k];
-      if (c < 0) continue;
-      const float dsc = sT[r * SU + k];
-      const TI* kr = klm + (bg * D.C + c) * DD + lane * DL;
+    for (int k0 = 0; k0 < Kt; k0 += U) {   // eight landmark rows' loads in flight together
+      float kv[U][DL], dsv[U];
 #pragma unroll
-      for (int e = 0; e < DL; ++e) acc[e] = fmaf(dsc, Elem<TI>::to_f(kr[e]), acc[e]);
+      for (int j = 0; j < U; ++j) {
+        const int c = k0 + j < Kt ? sel[(r / G) * Kt + k0 + j] : -1;
+        dsv[j] = c >= 0 ? sT[r * SU + k0 + j] : 0.f;
+        const TI* kr = klm + (bg * D.C + (c < 0 ? 0 : c)) * DD + lane * DL;
+#pragma unroll
+        for (int e = 0; e < DL; ++e) kv[j][e] = c >= 0 ? Elem<TI>::to_f(kr[e]) : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < U; ++j)
+#pragma unroll
+        for (int e = 0; e < DL; ++e) acc[e] = fmaf(dsv[j], kv[j][e], acc[e]);
     }
     float* out = dqc + grow_of(r) * DD + lane * DL;
 #pragma unroll
@@ -859,12 +876,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   BF* bV = bK + T * LDB;
   BF* bA = bV + T * LDB;
   BF* bdX = bA + kBwdRows * LDX;
-  // row bookkeeping of a batch, [2] buffers (the CUDA-core path uses the first)
-  int64_t* sPos = reinterpret_cast<int64_t*>(smem + keys_prod_bytes<DD, T, TC>());   // [2][64]
-  float* sLam = reinterpret_cast<float*>(sPos + 2 * kBwdRows);     // [2][64]
-  float* sGam = sLam + 2 * kBwdRows;                               // [2][64]
-  const TI** rowq = reinterpret_cast<const TI**>(sGam + 2 * kBwdRows);   // [2][64]
-  const TI** rowo = rowq + 2 * kBwdRows;                                 // [2][64]
+  // row bookkeeping of a batch, [3] buffers (the CUDA-core path uses the first)
+  int64_t* sPos = reinterpret_cast<int64_t*>(smem + keys_prod_bytes<DD, T, TC>());   // [3][64]
+  float* sLam = reinterpret_cast<float*>(sPos + 3 * kBwdRows);     // [3][64]
+  float* sGam = sLam + 3 * kBwdRows;                               // [3][64]
+  const TI** rowq = reinterpret_cast<const TI**>(sGam + 3 * kBwdRows);   // [3][64]
+  const TI** rowo = rowq + 3 * kBwdRows;                                 // [3][64]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tr = tid >> 4, tc = tid & 15;
@@ -907,62 +924,75 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
     for (int v = 0; v < 4; ++v) tK[j][v] = tV[j][v] = 0.f;
 
-  // the rows f0 .. f0 + 63 of the tile's row list into bookkeeping buffer `buf` (threads < 64)
-  auto prep = [&](int64_t f0, int buf) {
-    if (tid < kBwdRows) {
-      const int64_t f = f0 + tid;
-      const int o = buf * kBwdRows + tid;
-      if (f < total) {
-        int64_t qi;
-        int u, h;
-        if (f < n_win * G) {
-          qi = p_lo - D.q_pos0 + f / G;
-          h = (int)(f % G);
-          u = Kt;
-        } else {
-          const int64_t fe = f - n_win * G;
-          const int32_t ent = ents[fe / G];
-          qi = ent / Kt;
-          u = ent - (int)qi * Kt;
-          h = (int)(fe % G);
-        }
-        const int64_t grow = (b * D.Hq + g * G + h) * D.N_q + qi;
-        sPos[o] = D.q_pos0 + qi;
-        sLam[o] = lam_ws[grow * (Kt + 1) + u];
-        sGam[o] = gam_ws[grow * (Kt + 1) + u];
-        rowq[o] = q + grow * DD;
-        rowo[o] = dO + grow * DD;
+  // the rows f0 .. f0 + 63 of the tile's row list: one row per thread < 64, loaded into registers
+  // (prep_load) and later stored into a bookkeeping buffer (prep_store)
+  struct RowMeta {
+    int64_t pos;   // INT64_MIN: no row
+    float lam, gam;
+    const TI* rq;
+    const TI* ro;
+  };
+  auto prep_load = [&](int64_t f0) -> RowMeta {
+    RowMeta m{INT64_MIN, -INFINITY, 0.f, nullptr, nullptr};
+    const int64_t f = f0 + tid;
+    if (tid < kBwdRows && f < total) {
+      int64_t qi;
+      int u, h;
+      if (f < n_win * G) {
+        qi = p_lo - D.q_pos0 + f / G;
+        h = (int)(f % G);
+        u = Kt;
       } else {
-        sPos[o] = INT64_MIN;
-        sLam[o] = -INFINITY;
-        sGam[o] = 0.f;
-        rowq[o] = nullptr;
-        rowo[o] = nullptr;
+        const int64_t fe = f - n_win * G;
+        const int32_t ent = ents[fe / G];
+        qi = ent / Kt;
+        u = ent - (int)qi * Kt;
+        h = (int)(fe % G);
       }
+      const int64_t grow = (b * D.Hq + g * G + h) * D.N_q + qi;
+      m.pos = D.q_pos0 + qi;
+      m.lam = lam_ws[grow * (Kt + 1) + u];
+      m.gam = gam_ws[grow * (Kt + 1) + u];
+      m.rq = q + grow * DD;
+      m.ro = dO + grow * DD;
+    }
+    return m;
+  };
+  auto prep_store = [&](const RowMeta& m, int buf) {
+    if (tid < kBwdRows) {
+      const int o = buf * kBwdRows + tid;
+      sPos[o] = m.pos;
+      sLam[o] = m.lam;
+      sGam[o] = m.gam;
+      rowq[o] = m.rq;
+      rowo[o] = m.ro;
     }
   };
+  auto prep = [&](int64_t f0, int buf) { prep_store(prep_load(f0), buf); };
   if constexpr (TC) {
-    // batch i computes from buffer i & 1 while batch i + 1's rows load into the other
-    auto fetch = [&](int buf) {
+    // batch i computes from row buffer i & 1 and bookkeeping buffer i % 3 while batch i + 1's
+    // rows load into the other row buffer and batch i + 2's bookkeeping loads into registers
+    // (stored after batch i's products, so its dependent loads overlap them)
+    auto fetch = [&](int buf, int mb) {
       fetch_rows_b<DD>(bQ + buf * kBwdRows * LDB,
-                       reinterpret_cast<const BF* const*>(rowq + buf * kBwdRows), kBwdRows,
+                       reinterpret_cast<const BF* const*>(rowq + mb * kBwdRows), kBwdRows,
                        reinterpret_cast<const BF*>(q));
       fetch_rows_b<DD>(bdO + buf * kBwdRows * LDB,
-                       reinterpret_cast<const BF* const*>(rowo + buf * kBwdRows), kBwdRows,
+                       reinterpret_cast<const BF* const*>(rowo + mb * kBwdRows), kBwdRows,
                        reinterpret_cast<const BF*>(dO));
     };
     if (total > 0) {
       prep(0, 0);
+      prep(kBwdRows, 1);
       __syncthreads();
-      fetch(0);
+      fetch(0, 0);
     }
     int bi = 0;
     for (int64_t f0 = 0; f0 < total; f0 += kBwdRows, ++bi) {
-      const int buf = bi & 1;
+      const int buf = bi & 1, mb = bi % 3;
+      const RowMeta ahead = prep_load(f0 + 2 * kBwdRows);
       if (f0 + kBwdRows < total) {
-        prep(f0 + kBwdRows, buf ^ 1);
-        __syncthreads();
-        fetch(buf ^ 1);
+        fetch(buf ^ 1, (bi + 1) % 3);
         cp_async_wait<2>();   // this batch's two groups have landed
       } else {
         cp_async_wait<0>();
@@ -970,9 +1000,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       __syncthreads();
       const BF* cQ = bQ + buf * kBwdRows * LDB;
       const BF* cdO = bdO + buf * kBwdRows * LDB;
-      const int64_t* cPos = sPos + buf * kBwdRows;
-      const float* cLam = sLam + buf * kBwdRows;
-      const float* cGam = sGam + buf * kBwdRows;
+      const int64_t* cPos = sPos + mb * kBwdRows;
+      const float* cLam = sLam + mb * kBwdRows;
+      const float* cGam = sGam + mb * kBwdRows;
       const int rb = warp & 3, kh = warp >> 2, g8 = lane >> 2, t4 = lane & 3;
       float X[T / 16][4], P[T / 16][4];
       logits_frag<DD, T>(cQ, cdO, bK, bV, rb, kh, X, P);
@@ -1028,6 +1058,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
         }
       }
+      prep_store(ahead, (bi + 2) % 3);
       __syncthreads();   // the batch's buffers are consumed (the next prep and fetch reuse them)
     }
   } else {
@@ -1115,34 +1146,59 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   }
 
-  // d k_lm and d b_lm of chunk c: scale sum dscore q_cal and sum dscore over its selecting rows
+  // d k_lm and d b_lm of chunk c: scale sum dscore q_cal and sum dscore over its selecting rows.
+  // A warp per row, lanes over dims; eight rows per warp have their loads in flight together
+  // (each row's loads depend on its index entry).
   if (c < D.C && k0 == c * D.S) {
-    constexpr int PARTS = kBwdThreads / DD;
-    const int dim = tid % DD, part = tid / DD;
-    float acc = 0.f, dsum = 0.f;
-    for (int64_t f = part; f < n_inv * G; f += PARTS) {
-      const int32_t ent = ents[f / G];
-      const int64_t qi = ent / Kt;
-      const int u = ent - (int)qi * Kt;
-      const int64_t grow = (b * D.Hq + g * G + f % G) * D.N_q + qi;
-      const float dsc = ds_ws[grow * Kt + u];
-      acc = fmaf(dsc, Elem<TI>::to_f(qc[grow * DD + dim]), acc);
-      dsum += dsc;
+    constexpr int EPL = DD / 32, NW = kBwdThreads / 32, U = 8;
+    float acc[EPL], dsum = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+    const int64_t nr = n_inv * G;
+    for (int64_t f0 = warp; f0 < nr; f0 += NW * U) {
+      int64_t grow[U];
+      int slot[U];
+#pragma unroll
+      for (int j = 0; j < U; ++j) {
+        const int64_t f = f0 + (int64_t)NW * j;
+        grow[j] = -1;
+        slot[j] = 0;
+        if (f < nr) {
+          const int32_t ent = ents[f / G];
+          const int64_t qi = ent / Kt;
+          slot[j] = ent - (int)qi * Kt;
+          grow[j] = (b * D.Hq + g * G + f % G) * D.N_q + qi;
+        }
+      }
+      float dsv[U], qv[U][EPL];
+#pragma unroll
+      for (int j = 0; j < U; ++j) {
+        dsv[j] = grow[j] >= 0 ? ds_ws[grow[j] * Kt + slot[j]] : 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e)
+          qv[j][e] = grow[j] >= 0 ? Elem<TI>::to_f(qc[grow[j] * DD + lane * EPL + e]) : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < U; ++j) {
+        dsum += dsv[j];
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[e] = fmaf(dsv[j], qv[j][e], acc[e]);
+      }
     }
     __syncthreads();
-    float* red = reinterpret_cast<float*>(smem);   // [PARTS][DD + 1] (the products' area)
-    red[part * (DD + 1) + dim] = acc;
-    if (dim == 0) red[part * (DD + 1) + DD] = dsum;
+    float* red = reinterpret_cast<float*>(smem);   // [NW][DD + 1] (the products' area)
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) red[warp * (DD + 1) + lane * EPL + e] = acc[e];
+    if (lane == 0) red[warp * (DD + 1) + DD] = dsum;
     __syncthreads();
-    if (part == 0) {
-      float a = 0.f;
-      for (int p2 = 0; p2 < PARTS; ++p2) a += red[p2 * (DD + 1) + dim];
-      dklm[(bg * D.C + c) * DD + dim] = a * D.scale;
-      if (dim == 0) {
-        float t = 0.f;
-        for (int p2 = 0; p2 < PARTS; ++p2) t += red[p2 * (DD + 1) + DD];
-        dblm[bg * D.C + c] = t;
-      }
+    if (tid < DD) {
+      float a2 = 0.f;
+      for (int w = 0; w < NW; ++w) a2 += red[w * (DD + 1) + tid];
+      dklm[(bg * D.C + c) * DD + tid] = a2 * D.scale;
+    } else if (tid == DD) {
+      float t = 0.f;
+      for (int w = 0; w < NW; ++w) t += red[w * (DD + 1) + DD];
+      dblm[bg * D.C + c] = t;
     }
   }
 }
@@ -1226,7 +1282,7 @@ size_t rows_smem(const Dims& D) {
 
 template <int DD, int T, bool TC>
 constexpr size_t keys_smem() {
-  return (size_t)keys_prod_bytes<DD, T, TC>() + 2 * (kBwdRows * 8 + 2 * kBwdRows * 4 +
+  return (size_t)keys_prod_bytes<DD, T, TC>() + 3 * (kBwdRows * 8 + 2 * kBwdRows * 4 +
                                                     2 * kBwdRows * 8);
 }
 
