@@ -247,11 +247,12 @@ __global__ void __launch_bounds__(kAtThreads, ((DD == 64 && KM <= 16) || TWO) ? 
   const int64_t last_chunk = p_max / kTile;   // last tile (64 tokens) any window reaches
   constexpr int rs = RS;                       // tiles per chunk = 1 << rs
   const int K = D.K;
-  // warps 2-5 own one row each: (head h, query qi) = row r
+  // warps 2-5 own one row each: row r = (query qi, head h), query-major, so a warp holds
+  // 32 / G whole queries and skips the softmax of every selected-chunk tile none of them chose
   const bool is_row = warp >= 2;
   const int qd = warp & 3;
   const int r = qd * 32 + lane;
-  const int h = r / TQ, qi = r - h * TQ;
+  const int qi = r / G, h = r - qi * G;
   const int64_t i = i0 + qi;
   const bool valid = i < D.N_q;
   // With one head per KV group the row's surrogate score of a selected chunk is the score the
@@ -295,13 +296,12 @@ __global__ void __launch_bounds__(kAtThreads, ((DD == 64 && KM <= 16) || TWO) ? 
     prefetch_tensormap(&tmQ);
     prefetch_tensormap(&tmQc);
     mbar_expect_tx(q_full, (kOwnScores ? 2 : 1) * SH::Q_BYTES);
-    for (int hh = 0; hh < G; ++hh)
-      for (int kb = 0; kb < SH::KB; ++kb) {
-        const int32_t y = (int32_t)((b * D.Hq + g * G + hh) * D.N_q + i0);
-        tma_load_2d(sQ + kb * SH::Q_BOX + hh * TQ * 128, &tmQ, kb * 64, y, q_full);
-        if constexpr (kOwnScores)
-          tma_load_2d(sQc + kb * SH::Q_BOX + hh * TQ * 128, &tmQc, kb * 64, y, q_full);
-      }
+    // one box of [TQ queries][G heads][64 dims] per 64 columns: rows land query-major
+    for (int kb = 0; kb < SH::KB; ++kb) {
+      const int32_t y = (int32_t)(b * D.Hq + g * G), z = (int32_t)i0;
+      tma_load_3d(sQ + kb * SH::Q_BOX, &tmQ, kb * 64, y, z, q_full);
+      if constexpr (kOwnScores) tma_load_3d(sQc + kb * SH::Q_BOX, &tmQc, kb * 64, y, z, q_full);
+    }
   }
   // selected chunks of every valid query of the tile (the G rows of a query hold the same
   // selection: row (h, qi) sets the bits of the entries k = h mod G), and the chunks of the
@@ -847,6 +847,22 @@ bool make_map_at(CUtensorMap* map, const void* base, uint64_t rows, uint64_t d, 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [B Hq, N_q, d] bf16 viewed as 3-D (dims, heads, queries), boxes of [TQ queries][G heads][64
+// dims] with the 128-byte swizzle: the G heads of a query are consecutive rows in shared memory.
+bool make_map_q3(CUtensorMap* map, const void* base, uint64_t heads, uint64_t n_q, uint64_t d,
+                 uint32_t G, uint32_t TQ) {
+  auto enc = get_encode_at();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {d, heads, n_q};
+  cuuint64_t strides[2] = {n_q * d * 2, d * 2};
+  cuuint32_t box[3] = {64, G, TQ};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int list_capacity(const Dims& D, int TQ) {
   // union of TQ queries' selections (S / 64 tiles each) plus the tiles their windows cover
   return TQ * D.K * (D.S / kTile) + (int)((D.W + D.S + TQ) / kTile) + 4;
@@ -869,8 +885,8 @@ cudaError_t launch_at_t(const Dims& D, const void* q, const void* qc, const void
                         cudaStream_t st) {
   using SH = AtShape<DD, G, TWO>;
   CUtensorMap tmQ, tmQc, tmK, tmV;
-  if (!make_map_at(&tmQ, q, (uint64_t)(D.B * D.Hq * D.N_q), DD, SH::TQ) ||
-      !make_map_at(&tmQc, qc, (uint64_t)(D.B * D.Hq * D.N_q), DD, SH::TQ) ||
+  if (!make_map_q3(&tmQ, q, (uint64_t)(D.B * D.Hq), (uint64_t)D.N_q, DD, G, SH::TQ) ||
+      !make_map_q3(&tmQc, qc, (uint64_t)(D.B * D.Hq), (uint64_t)D.N_q, DD, G, SH::TQ) ||
       !make_map_at(&tmK, K, (uint64_t)(D.B * D.Hkv * D.N_kv), DD, kTile) ||
       !make_map_at(&tmV, V, (uint64_t)(D.B * D.Hkv * D.N_kv), DD, kTile))
     return cudaErrorInvalidValue;
