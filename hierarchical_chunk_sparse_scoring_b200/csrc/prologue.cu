@@ -13,11 +13,11 @@
 //                  a dense contraction on the tcgen05 tensor cores (bf16 operands by TMA with the
 //                  128-byte swizzle, fp32 accumulator in TMEM, 128 x BN tiles, a 4-stage ring).
 //   qcal_hope_kernel  per (b, 32 tokens), every head in turn: q_cal = R(q + W_up u), q = R(q);
-//                  HBM-bound (q read, both written, u read); W_up[h] staged transposed in shared
-//                  memory; a warp per token, each lane d/32 consecutive dims (the pair partner in
-//                  lane ^ 16); the block's (token, pair) angles p theta_m reduced modulo 2 pi in
-//                  fp64 once (p up to 2^22 makes an fp32 product lose whole radians), then
-//                  sincosf, kept in shared memory for all heads.
+//                  HBM-bound (q read, both written, u read); W_up[h] read through L1; four
+//                  tokens per warp in flight together, each lane d/32 consecutive dims (the
+//                  pair partner in lane ^ 16); the block's (token, pair) angles p theta_m
+//                  reduced modulo 2 pi in fp64 once (p up to 2^22 makes an fp32 product lose
+//                  whole radians), then sincosf, kept in shared memory for all heads.
 #include <cudaTypedefs.h>
 
 #include <type_traits>
@@ -256,6 +256,22 @@ __device__ __forceinline__ void angle_table(float2* sCS, int64_t pos0, double ba
   }
 }
 
+// Eight consecutive elements (16 or 32 bytes, 16-byte aligned) as floats, through L1.
+template <typename T>
+__device__ __forceinline__ void load_piece8(const T* p, float (&v)[8]);
+template <>
+__device__ __forceinline__ void load_piece8<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 t = __ldg(reinterpret_cast<const uint4*>(p));
+  v[0] = bf16_lo(t.x); v[1] = bf16_hi(t.x); v[2] = bf16_lo(t.y); v[3] = bf16_hi(t.y);
+  v[4] = bf16_lo(t.z); v[5] = bf16_hi(t.z); v[6] = bf16_lo(t.w); v[7] = bf16_hi(t.w);
+}
+template <>
+__device__ __forceinline__ void load_piece8<float>(const float* p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
 // Turns this lane's dims: pair m (first half) and m + d/2 (second half, the partner lane).
 template <int EPL>
 __device__ __forceinline__ void turn(float (&x)[EPL], float (&y)[EPL], int lane,
@@ -271,59 +287,78 @@ __device__ __forceinline__ void turn(float (&x)[EPL], float (&y)[EPL], int lane,
   }
 }
 
-// grid (token blocks, B); every head of the block in turn.  r = 0 leaves q_cal = R(q).
+// grid (token blocks, B); every head of the block in turn.  r = 0 leaves q_cal = R(q).  Each
+// warp takes kQhTpw tokens together (their loads in flight at once); W_up[h]'s rows of the
+// lane's dims are read through L1 (every warp of every CTA reads the same d x r block), 8
+// columns at a time, and applied to all of the warp's tokens.
+constexpr int kQhTpw = kQhTokens / (kQhThreads / 32);
 template <typename T, int DD>
-__global__ void __launch_bounds__(kQhThreads)
+__global__ void __launch_bounds__(kQhThreads, 2)
     qcal_hope_kernel(int64_t N_q, int64_t Hq, int64_t q_pos0, int r, double base,
                      double train_len, const T* __restrict__ q, const float* __restrict__ u,
                      const T* __restrict__ W_up, T* __restrict__ q_out, T* __restrict__ qc_out) {
   constexpr int EPL = DD / 32;
-  __shared__ __align__(16) float sW[64 * DD];   // W_up[h] transposed: [r][DD]
   __shared__ float2 sCS[kQhTokens * (DD / 2)];
   const int64_t b = blockIdx.y;
   const int64_t i0 = (int64_t)blockIdx.x * kQhTokens;
   angle_table<DD>(sCS, q_pos0 + i0, base, train_len);
+  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int dim0 = lane * EPL;
+  const int t0 = warp * kQhTpw;
+  const bool vec_w = r % (sizeof(T) == 2 ? 8 : 4) == 0;
   for (int64_t h = 0; h < Hq; ++h) {
-    __syncthreads();   // (the previous head's W_up is consumed)
-    for (int e = threadIdx.x; e < r * DD; e += kQhThreads) {
-      const int dim = e / r, j = e - dim * r;   // reads W_up[h][dim][j] in order
-      sW[j * DD + dim] = Elem<T>::to_f(W_up[(h * DD + dim) * r + j]);
-    }
-    __syncthreads();
-    for (int t = warp; t < kQhTokens; t += kQhThreads / 32) {
-      const int64_t i = i0 + t;
-      if (i >= N_q) break;
-      const int64_t row = (b * Hq + h) * N_q + i;
-      float x[EPL], c[EPL];
-      load_dims<T, EPL>(q + row * DD + dim0, x);
+    float x[kQhTpw][EPL], c[kQhTpw][EPL], ua[kQhTpw], ub[kQhTpw];
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) c[e] = x[e];
-      if (r > 0) {
-        // u of this (token, head): r values, lanes j and j + 32; dq = W_up u
+    for (int tt = 0; tt < kQhTpw; ++tt) {
+      const int64_t i = i0 + t0 + tt;
+      if (i < N_q) {
+        load_dims<T, EPL>(q + ((b * Hq + h) * N_q + i) * DD + dim0, x[tt]);
         const float* ur = u + (b * N_q + i) * (Hq * r) + h * r;
-        const float u0 = lane < r ? ur[lane] : 0.f;
-        const float u1 = lane + 32 < r ? ur[lane + 32] : 0.f;
-        for (int j = 0; j < r; ++j) {
-          const float uj = __shfl_sync(0xffffffffu, j < 32 ? u0 : u1, j & 31);
-          const float* wr = sW + j * DD + dim0;
-          if constexpr (EPL == 4) {
-            const float4 w = *reinterpret_cast<const float4*>(wr);
-            c[0] = fmaf(w.x, uj, c[0]);
-            c[1] = fmaf(w.y, uj, c[1]);
-            c[2] = fmaf(w.z, uj, c[2]);
-            c[3] = fmaf(w.w, uj, c[3]);
-          } else {
-            const float2 w = *reinterpret_cast<const float2*>(wr);
-            c[0] = fmaf(w.x, uj, c[0]);
-            c[1] = fmaf(w.y, uj, c[1]);
-          }
+        ua[tt] = lane < r ? ur[lane] : 0.f;
+        ub[tt] = lane + 32 < r ? ur[lane + 32] : 0.f;
+      } else {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) x[tt][e] = 0.f;
+        ua[tt] = ub[tt] = 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) c[tt][e] = x[tt][e];
+    }
+    const T* wrow = W_up + (h * DD + dim0) * r;   // rows dim0 .. dim0 + EPL - 1, r each
+    for (int j0 = 0; j0 < r; j0 += 8) {
+      float w[EPL][8];
+      if (vec_w && j0 + 8 <= r) {   // 16-byte pieces of the rows (r a multiple of 8 / 4)
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) load_piece8<T>(wrow + e * r + j0, w[e]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e)
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj)
+            w[e][jj] = j0 + jj < r ? Elem<T>::to_f(__ldg(wrow + e * r + j0 + jj)) : 0.f;
+      }
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        const int j = j0 + jj;   // (warp-uniform)
+        if (j >= r) break;
+#pragma unroll
+        for (int tt = 0; tt < kQhTpw; ++tt) {
+          const float uj = __shfl_sync(0xffffffffu, j < 32 ? ua[tt] : ub[tt], j & 31);
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) c[tt][e] = fmaf(w[e][jj], uj, c[tt][e]);
         }
       }
-      turn<EPL>(x, c, lane, sCS + t * (DD / 2));
-      store_dims<T, EPL>(q_out + row * DD + dim0, x);
-      store_dims<T, EPL>(qc_out + row * DD + dim0, c);
+    }
+#pragma unroll
+    for (int tt = 0; tt < kQhTpw; ++tt) {
+      const int64_t i = i0 + t0 + tt;
+      turn<EPL>(x[tt], c[tt], lane, sCS + (t0 + tt) * (DD / 2));
+      if (i < N_q) {
+        const int64_t row = (b * Hq + h) * N_q + i;
+        store_dims<T, EPL>(q_out + row * DD + dim0, x[tt]);
+        store_dims<T, EPL>(qc_out + row * DD + dim0, c[tt]);
+      }
     }
   }
 }
