@@ -146,6 +146,10 @@ __device__ __forceinline__ void logits_tile(const float* sQ, const float* sdO, c
 // exactly; the fused weights a and logit gradients dx enter the dq, dK and dV products rounded to
 // bf16, as the intermediate probabilities of a flash-attention backward do.
 constexpr int kPadB = 8;   // bf16 elements of row padding
+// Staging buffers of the tensor-core kernels' streamed operands (K/V tiles, gathered row
+// batches): 1 keeps a CTA within half an SM's shared memory (two CTAs, 16 warps per SM, which
+// hides the MMA chains' latency), 2 prefetches the next tile within one CTA per SM instead.
+constexpr int kBwdBufs = 1;
 
 __device__ __forceinline__ uint32_t su32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -297,14 +301,14 @@ __device__ __forceinline__ void logits_frag(const __nv_bfloat16* sQ, const __nv_
 template <int DD, int T, bool TC>
 constexpr int rows_prod_bytes() {
   using SH = BwdShape<DD, T>;
-  return TC ? ((2 * kBwdRows + 4 * T) * (DD + kPadB) + kBwdRows * (T + kPadB)) * 2 +
+  return TC ? ((2 * kBwdRows + 2 * kBwdBufs * T) * (DD + kPadB) + kBwdRows * (T + kPadB)) * 2 +
                   2 * kBwdRows * 3 * 4
             : (2 * SH::ROWS_F + 2 * SH::KEYS_F + SH::TILE_F) * 4;
 }
 template <int DD, int T, bool TC>
 constexpr int keys_prod_bytes() {
   using SH = BwdShape<DD, T>;
-  return TC ? ((4 * kBwdRows + 2 * T) * (DD + kPadB) + 2 * kBwdRows * (T + kPadB)) * 2
+  return TC ? ((2 * kBwdBufs * kBwdRows + 2 * T) * (DD + kPadB) + 2 * kBwdRows * (T + kPadB)) * 2
             : (2 * SH::ROWS_F + 2 * SH::KEYS_F + 2 * SH::TILE_F) * 4;
 }
 
@@ -314,7 +318,7 @@ constexpr int keys_prod_bytes() {
 // Query-major kernel: CTA = (b, g, 64/G queries); row r = query r / G, head g G + r % G.
 // TC: the products on the tensor cores (bf16 inputs), else on the CUDA cores.
 template <typename TI, int DD, int T, bool TC>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, TC && kBwdBufs == 1 ? 2 : 1)
     bwd_rows_kernel(Dims D, const TI* __restrict__ q, const TI* __restrict__ qc,
                     const TI* __restrict__ K, const TI* __restrict__ V,
                     const TI* __restrict__ klm, const float* __restrict__ blm,
@@ -337,9 +341,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   float* sdX = sV + SH::KEYS_F;
   BF* bQ = reinterpret_cast<BF*>(smem);
   BF* bdO = bQ + kBwdRows * LDB;
-  BF* bK = bdO + kBwdRows * LDB;   // [2][T][LDB]: the next tile's keys load meanwhile
-  BF* bV = bK + 2 * T * LDB;       // [2][T][LDB]
-  BF* bdX = bV + 2 * T * LDB;
+  BF* bK = bdO + kBwdRows * LDB;   // [kBwdBufs][T][LDB]
+  BF* bV = bK + kBwdBufs * T * LDB;   // [kBwdBufs][T][LDB]
+  BF* bdX = bV + kBwdBufs * T * LDB;
   float* sPart = reinterpret_cast<float*>(bdX + kBwdRows * LDX);   // [2 key halves][64][3]
   float* sM = reinterpret_cast<float*>(smem + rows_prod_bytes<DD, T, TC>());   // [64][SU] running
                                                                            // max (base 2), then lambda2
@@ -469,12 +473,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   };
 
-  // tensor cores: tile t's keys and values into buffer t & 1, one commit group
+  // tensor cores: tile t's keys and values into buffer t % kBwdBufs, one commit group
   auto fetch_kv = [&](int t) {
     const int64_t k0 = tile_k0(t);
-    fetch_keys_b<DD, T>(bK + (t & 1) * T * LDB, reinterpret_cast<const BF*>(Kb), k0, D.N_kv);
-    fetch_keys_b<DD, T>(bV + (t & 1) * T * LDB, reinterpret_cast<const BF*>(Vb), k0, D.N_kv);
+    const int o = (t % kBwdBufs) * T * LDB;
+    fetch_keys_b<DD, T>(bK + o, reinterpret_cast<const BF*>(Kb), k0, D.N_kv);
+    fetch_keys_b<DD, T>(bV + o, reinterpret_cast<const BF*>(Vb), k0, D.N_kv);
     cp_async_commit();
+  };
+  // tile t in its buffer: the next tile prefetched (two buffers) or this one fetched now (one;
+  // the caller's barrier has retired the previous tile's readers)
+  auto land_kv = [&](int t) {
+    if constexpr (kBwdBufs == 2) {
+      if (t + 1 < n_tiles) fetch_kv(t + 1);
+      else cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      if (t > 0) fetch_kv(t);
+      cp_async_wait<0>();
+    }
   };
   // merges a tile's (max, sum, sum p dP) of row r's unit u into the running state
   auto merge_stats = [&](int r, int u, float m, float l, float tt) {
@@ -502,9 +519,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   for (int t = 0; t < n_tiles; ++t) {
     const int64_t k0 = tile_k0(t);
     if constexpr (TC) {
-      if (t + 1 < n_tiles) fetch_kv(t + 1);
-      else cp_async_commit();
-      cp_async_wait<1>();   // tile t has landed (this thread's copies; the barrier below: all)
+      land_kv(t);   // tile t has landed (this thread's copies; the barrier below: all)
     } else {
       stage_keys<TI, DD, LD, T>(sK, Kb, k0, D.N_kv);
       stage_keys<TI, DD, LD, T>(sV, Vb, k0, D.N_kv);
@@ -515,7 +530,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // warp: rows 16 rb .., keys kh T/2 ..; a row's values sit in the 4 lanes of its quad
       const int rb = warp & 3, kh = warp >> 2, g8 = lane >> 2, t4 = lane & 3;
       float X[T / 16][4], P[T / 16][4];
-      logits_frag<DD, T>(bQ, bdO, bK + (t & 1) * T * LDB, bV + (t & 1) * T * LDB, rb, kh, X, P);
+      logits_frag<DD, T>(bQ, bdO, bK + (t % kBwdBufs) * T * LDB, bV + (t % kBwdBufs) * T * LDB,
+                         rb, kh, X, P);
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr) {
         const int r = 16 * rb + g8 + 8 * hr;
@@ -719,15 +735,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (n_tiles > 0) fetch_kv(0);
     for (int t = 0; t < n_tiles; ++t) {
       const int64_t k0 = tile_k0(t);
-      __syncthreads();   // the previous tile is consumed: its buffer takes tile t + 1
-      if (t + 1 < n_tiles) fetch_kv(t + 1);
-      else cp_async_commit();
-      cp_async_wait<1>();
+      __syncthreads();   // the previous tile is consumed: its buffer takes the next one
+      land_kv(t);
       set_units(k0);
       __syncthreads();
-      const BF* bKt = bK + (t & 1) * T * LDB;
+      const BF* bKt = bK + (t % kBwdBufs) * T * LDB;
       float X[T / 16][4], P[T / 16][4];
-      logits_frag<DD, T>(bQ, bdO, bKt, bV + (t & 1) * T * LDB, rb, kh, X, P);
+      logits_frag<DD, T>(bQ, bdO, bKt, bV + (t % kBwdBufs) * T * LDB, rb, kh, X, P);
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr) {
         const int r = 16 * rb + g8 + 8 * hr;
@@ -848,7 +862,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // heads) and the selecting rows (the inverse index of chunk c, all G heads), in batches of 64.
 // TC: the products on the tensor cores (bf16 inputs), else on the CUDA cores.
 template <typename TI, int DD, int T, bool TC>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, TC && kBwdBufs == 1 ? 2 : 1)
     bwd_keys_kernel(Dims D, const TI* __restrict__ q, const TI* __restrict__ qc,
                     const TI* __restrict__ K, const TI* __restrict__ V,
                     const TI* __restrict__ dO, const float* __restrict__ lam_ws,
@@ -870,9 +884,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   float* sV = sK + SH::KEYS_F;
   float* sA = sV + SH::KEYS_F;
   float* sdX = sA + SH::TILE_F;
-  BF* bQ = reinterpret_cast<BF*>(smem);   // [2][64][LDB]: the next batch's rows load meanwhile
-  BF* bdO = bQ + 2 * kBwdRows * LDB;      // [2][64][LDB]
-  BF* bK = bdO + 2 * kBwdRows * LDB;
+  BF* bQ = reinterpret_cast<BF*>(smem);   // [kBwdBufs][64][LDB] gathered q rows
+  BF* bdO = bQ + kBwdBufs * kBwdRows * LDB;      // [kBwdBufs][64][LDB]
+  BF* bK = bdO + kBwdBufs * kBwdRows * LDB;
   BF* bV = bK + T * LDB;
   BF* bA = bV + T * LDB;
   BF* bdX = bA + kBwdRows * LDX;
@@ -970,9 +984,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   };
   auto prep = [&](int64_t f0, int buf) { prep_store(prep_load(f0), buf); };
   if constexpr (TC) {
-    // batch i computes from row buffer i & 1 and bookkeeping buffer i % 3 while batch i + 1's
-    // rows load into the other row buffer and batch i + 2's bookkeeping loads into registers
-    // (stored after batch i's products, so its dependent loads overlap them)
+    // batch i computes from row buffer i % kBwdBufs and bookkeeping buffer i % 3; with two row
+    // buffers batch i + 1's rows load into the other meanwhile; batch i + 2's bookkeeping loads
+    // into registers (stored after batch i's products, so its dependent loads overlap them)
     auto fetch = [&](int buf, int mb) {
       fetch_rows_b<DD>(bQ + buf * kBwdRows * LDB,
                        reinterpret_cast<const BF* const*>(rowq + mb * kBwdRows), kBwdRows,
@@ -989,12 +1003,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     int bi = 0;
     for (int64_t f0 = 0; f0 < total; f0 += kBwdRows, ++bi) {
-      const int buf = bi & 1, mb = bi % 3;
+      const int buf = bi % kBwdBufs, mb = bi % 3;
       const RowMeta ahead = prep_load(f0 + 2 * kBwdRows);
-      if (f0 + kBwdRows < total) {
-        fetch(buf ^ 1, (bi + 1) % 3);
-        cp_async_wait<2>();   // this batch's two groups have landed
+      if constexpr (kBwdBufs == 2) {
+        if (f0 + kBwdRows < total) {
+          fetch(buf ^ 1, (bi + 1) % 3);
+          cp_async_wait<2>();   // this batch's two groups have landed
+        } else {
+          cp_async_wait<0>();
+        }
       } else {
+        if (bi > 0) fetch(0, mb);   // (the previous batch's readers retired at its barrier)
         cp_async_wait<0>();
       }
       __syncthreads();
