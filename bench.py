@@ -9,7 +9,8 @@ batch of the prefill workload, inputs resident in HBM.  The default workload is 
 single-GPU configuration: the extreme-length prefill at N = 4M tokens (B=1, 8 query heads / 1 KV
 head, d=128, S=128, K=16, W=2048; 140.6 TFLOP of landmark scoring).  Steps are timed with CUDA
 events recorded by the library between its kernels, so each kernel's duration comes from the
-same timed steps; L2 is flushed (256 MiB write) between steps, outside the timed intervals.
+same timed steps; L2 is flushed between steps, outside the timed intervals (a 256 MiB write,
+then a 256 MiB read so that the write's dirty lines reach HBM before the next step starts).
 With N GPUs every rank runs its own independent batch (weak scaling, no data-path collective);
 the step time is the max over ranks.
 
@@ -271,10 +272,16 @@ def timed_steps(run, steps, flush, barrier=lambda: None):
 
 
 def make_flush(device):
+    """Evicts the previous step's data from L2: a write of a buffer larger than L2, then a read
+    of another one, whose clean lines displace the write's dirty ones (otherwise their write-back
+    to HBM would fall inside the next timed step)."""
     buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    src = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    acc = torch.empty((), dtype=torch.float32, device=device)
 
     def flush():
         buf.fill_(1.0)
+        torch.sum(src, dim=0, out=acc)
     return flush
 
 
@@ -380,7 +387,8 @@ def config_of(wl, n_gpus):
             "d": d["d"], "S": wl.S, "K_top": wl.K_top, "W": wl.W,
             "global_batch": d["B"] * n_gpus, "seq_len": d["N_kv"],
             "parallelism": "dp%d (independent batches per GPU)" % n_gpus,
-            "l2": "flushed between steps (256 MiB write), outside the timed intervals"}
+            "l2": "flushed between steps (256 MiB write, then 256 MiB read), outside the "
+                  "timed intervals"}
 
 
 def measure_e2e(run, steps, warmup):

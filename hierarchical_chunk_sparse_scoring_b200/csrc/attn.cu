@@ -158,6 +158,104 @@ struct UnitShape {
   static_assert(L >= 1 && L <= 32 && (32 % L) == 0, "lane grouping");
 };
 
+// Fusion of K chunk units (scores s_sel) and n_pieces window pieces (scores = their lse, whose
+// log-sum-exp is the window's lse).  Units with score -inf get weight 0.  One warp per
+// (b, h, query) row: the lanes first hold the units' weights, then sweep d with the weights
+// broadcast, loading several units' vectors before accumulating them.
+template <typename T>
+__device__ __forceinline__ void fuse_row(const Dims& D, int n_pieces, int64_t row, int lane,
+                                         const float* __restrict__ s_sel,
+                                         const float* __restrict__ part_o,
+                                         const float* __restrict__ part_lse, T* __restrict__ out,
+                                         float* __restrict__ lse_out) {
+  const int K = D.K, NU = K + n_pieces, d = (int)D.d;
+  // L2-coherent loads: inside the units kernel the partials come from other CTAs of the same
+  // launch, which the read-only path does not promise to see
+  auto score_of = [&](int u) -> float {
+    return u < K ? __ldcg(s_sel + row * K + u) : __ldcg(part_lse + row * NU + u);
+  };
+  auto load4cg = [](const float* p, float (&v)[4]) {
+    const float4 t = __ldcg(reinterpret_cast<const float4*>(p));
+    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+  };
+  const float* pr = part_o + row * NU * d;
+  if (NU <= 64 && d == 128) {
+    // lanes hold the weights of units lane and lane + 32 (scores read once); then every lane
+    // reads its 4 output columns of all units, 16 loads in flight per batch
+    const float s0 = lane < NU ? score_of(lane) : -INFINITY;
+    const float s1 = lane + 32 < NU ? score_of(lane + 32) : -INFINITY;
+    const float M = warp_max(fmaxf(s0, s1));
+    const float e0 = s0 == -INFINITY ? 0.f : __expf(s0 - M);
+    const float e1 = s1 == -INFINITY ? 0.f : __expf(s1 - M);
+    const float Z = warp_sum(e0 + e1);
+    const float w0 = e0 / Z, w1 = e1 / Z;
+    float o[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int u0 = 0; u0 < NU; u0 += 16) {
+      float v[16][4];
+#pragma unroll
+      for (int e2 = 0; e2 < 16; ++e2) {
+        if (u0 + e2 < NU) {
+          load4cg(pr + (int64_t)(u0 + e2) * 128 + lane * 4, v[e2]);
+        } else {
+          v[e2][0] = v[e2][1] = v[e2][2] = v[e2][3] = 0.f;
+        }
+      }
+      const float wsrc = u0 < 32 ? w0 : w1;   // a batch lies on one side of unit 32
+#pragma unroll
+      for (int e2 = 0; e2 < 16; ++e2) {
+        const float w = __shfl_sync(0xffffffffu, wsrc, (u0 + e2) & 31);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) o[x] = fmaf(w, v[e2][x], o[x]);
+      }
+    }
+    Elem<T>::store4(out + row * 128 + lane * 4, o);
+    if (lse_out && lane == 0) lse_out[row] = M + logf(Z);
+    return;
+  }
+  float M = -INFINITY;
+  for (int u = lane; u < NU; u += 32) M = fmaxf(M, score_of(u));
+  M = warp_max(M);
+  float Z = 0.f;
+  for (int u = lane; u < NU; u += 32) {
+    const float s = score_of(u);
+    Z += (s == -INFINITY) ? 0.f : __expf(s - M);
+  }
+  Z = warp_sum(Z);
+  const float invZ = 1.f / Z;
+  // every lane runs every iteration (the loop body shuffles); lanes past d only skip memory
+  for (int kb = 0; kb < d; kb += 128) {
+    const int k0 = kb + lane * 4;
+    const bool act = k0 < d;
+    float o[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int ub = 0; ub < NU; ub += 32) {
+      const int um = ub + lane;
+      const float su = um < NU ? score_of(um) : -INFINITY;
+      const float wl = su == -INFINITY ? 0.f : __expf(su - M) * invZ;   // lane's unit weight
+      const int cnt = NU - ub < 32 ? NU - ub : 32;
+      for (int u8 = 0; u8 < cnt; u8 += 8) {
+        float v[8][4];
+        float w[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          w[e] = __shfl_sync(0xffffffffu, wl, (u8 + e) & 31);
+          if (u8 + e < cnt && act) {
+            load4cg(pr + (int64_t)(ub + u8 + e) * d + k0, v[e]);
+          } else {
+            w[e] = 0.f;
+            v[e][0] = v[e][1] = v[e][2] = v[e][3] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+#pragma unroll
+          for (int x = 0; x < 4; ++x) o[x] = fmaf(w[e], v[e][x], o[x]);
+      }
+    }
+    if (act) Elem<T>::store4(out + row * d + k0, o);
+  }
+  if (lse_out && lane == 0) lse_out[row] = M + logf(Z);
+}
+
 template <typename T, int D_, int GM>
 __global__ void __launch_bounds__(kUnitThreads) attn_units_kernel(
     Dims D, int n_pieces, const T* __restrict__ q, const T* __restrict__ Kc,
@@ -362,10 +460,6 @@ __global__ void __launch_bounds__(kUnitThreads) attn_units_kernel(
   }
 }
 
-// Fusion of K chunk units (scores s_sel) and n_pieces window pieces (scores = their lse, whose
-// log-sum-exp is the window's lse).  Units with score -inf get weight 0.  One warp per
-// (b, h, query): lane u first holds unit u's weight, then the lanes sweep d with the weights
-// broadcast, loading eight units' vectors before accumulating them.
 template <typename T>
 __global__ void __launch_bounds__(128) fuse_units_kernel(Dims D, int n_pieces,
                                                          const float* __restrict__ s_sel,
@@ -377,83 +471,7 @@ __global__ void __launch_bounds__(128) fuse_units_kernel(Dims D, int n_pieces,
   const int64_t rows = D.B * D.Hq * D.N_q;
   const int64_t row = (int64_t)blockIdx.x * 4 + warp;
   if (row >= rows) return;
-  const int K = D.K, NU = K + n_pieces, d = (int)D.d;
-  auto score_of = [&](int u) -> float {
-    return u < K ? s_sel[row * K + u] : part_lse[row * NU + u];
-  };
-  const float* pr = part_o + row * NU * d;
-  if (NU <= 32 && d == 128) {
-    // one unit per lane: its score is read once; then every lane reads its 4 output columns of
-    // all units, 16 loads in flight per batch
-    const float su = lane < NU ? score_of(lane) : -INFINITY;
-    const float M = warp_max(su);
-    const float e = su == -INFINITY ? 0.f : __expf(su - M);
-    const float Z = warp_sum(e);
-    const float wl = e / Z;
-    float o[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int u0 = 0; u0 < NU; u0 += 16) {
-      float v[16][4];
-#pragma unroll
-      for (int e2 = 0; e2 < 16; ++e2) {
-        if (u0 + e2 < NU) {
-          Elem<float>::load4(pr + (int64_t)(u0 + e2) * 128 + lane * 4, v[e2]);
-        } else {
-          v[e2][0] = v[e2][1] = v[e2][2] = v[e2][3] = 0.f;
-        }
-      }
-#pragma unroll
-      for (int e2 = 0; e2 < 16; ++e2) {
-        const float w = __shfl_sync(0xffffffffu, wl, (u0 + e2) & 31);
-#pragma unroll
-        for (int x = 0; x < 4; ++x) o[x] = fmaf(w, v[e2][x], o[x]);
-      }
-    }
-    Elem<T>::store4(out + row * 128 + lane * 4, o);
-    if (lse_out && lane == 0) lse_out[row] = M + logf(Z);
-    return;
-  }
-  float M = -INFINITY;
-  for (int u = lane; u < NU; u += 32) M = fmaxf(M, score_of(u));
-  M = warp_max(M);
-  float Z = 0.f;
-  for (int u = lane; u < NU; u += 32) {
-    const float s = score_of(u);
-    Z += (s == -INFINITY) ? 0.f : __expf(s - M);
-  }
-  Z = warp_sum(Z);
-  const float invZ = 1.f / Z;
-  // every lane runs every iteration (the loop body shuffles); lanes past d only skip memory
-  for (int kb = 0; kb < d; kb += 128) {
-    const int k0 = kb + lane * 4;
-    const bool act = k0 < d;
-    float o[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int ub = 0; ub < NU; ub += 32) {
-      const int um = ub + lane;
-      const float su = um < NU ? score_of(um) : -INFINITY;
-      const float wl = su == -INFINITY ? 0.f : __expf(su - M) * invZ;   // lane's unit weight
-      const int cnt = NU - ub < 32 ? NU - ub : 32;
-      for (int u8 = 0; u8 < cnt; u8 += 8) {
-        float v[8][4];
-        float w[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          w[e] = __shfl_sync(0xffffffffu, wl, (u8 + e) & 31);
-          if (u8 + e < cnt && act) {
-            Elem<float>::load4(pr + (int64_t)(ub + u8 + e) * d + k0, v[e]);
-          } else {
-            w[e] = 0.f;
-            v[e][0] = v[e][1] = v[e][2] = v[e][3] = 0.f;
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-#pragma unroll
-          for (int x = 0; x < 4; ++x) o[x] = fmaf(w[e], v[e][x], o[x]);
-      }
-    }
-    if (act) Elem<T>::store4(out + row * d + k0, o);
-  }
-  if (lse_out && lane == 0) lse_out[row] = M + logf(Z);
+  fuse_row<T>(D, n_pieces, row, lane, s_sel, part_o, part_lse, out, lse_out);
 }
 
 // ---------------------------------------------------------------------------------------------

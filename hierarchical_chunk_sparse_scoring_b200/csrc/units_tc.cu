@@ -1,18 +1,21 @@
 // Step 3 for decode on the tcgen05 tensor cores: per-unit exact attention (o_u, lse_u) of the
-// G heads of a (b, g, query) row over each selected chunk and each window piece of S = 64 tokens.
+// G heads of a (b, g, query) row over each selected chunk and each window piece of S tokens
+// (S = 64 or 128).
 //
 // [Reader] Fig. 3 caption and [Abstract]: each retrieved chunk is attended on its own, with its
 // own softmax, and the per-chunk outputs are fused later by the retrieval scores; the local
 // window is one more unit (here cut into pieces of 64 tokens, recombined by their lse in the
 // fusion).  In decode the step streams the selected K/V chunks from HBM; the arithmetic is put on
 // the tensor core so the SMs only move data:
-//   * a tile is two units of one row: their K rows (2 x 64 tokens) form the 128-row A operand,
-//     the row's G query heads (N = 16 rows; rows past G are never read) the B operand:
-//     S = K_tile . Q^T (M = 128 tokens, N = 16, K = d);
-//   * the softmax warps (one token per thread) take each unit's max and sum over its 64 tokens
-//     per head and write P (bf16) as a K-major [16 heads x 128 tokens] operand;
-//   * O_u^T = V_u^T . P_u (M = d = 128, N = 16, K = 64 tokens; V read as an MN-major operand) for
-//     each of the two units; the epilogue (one d-row per thread) divides by the unit's sum.
+//   * a tile is 128 tokens of one row: two units when S = 64, one unit when S = 128 (its two
+//     64-token halves); their K rows form the 128-row A operand, the row's G query heads
+//     (N = 16 rows; rows past G are never read) the B operand: S = K_tile . Q^T (M = 128 tokens,
+//     N = 16, K = d);
+//   * the softmax warps (one token per thread) take each unit's max and sum over its tokens per
+//     head and write P (bf16) as a K-major [16 heads x 128 tokens] operand;
+//   * O_u^T = V_u^T . P_u (M = d = 128, N = 16, K = 64 tokens per half; V read as an MN-major
+//     operand): per half into its own accumulator when the halves are two units, both halves
+//     into one when they are one; the epilogue (one d-row per thread) divides by the unit's sum.
 // Persistent CTAs, three per SM, each with one stage whose K and V halves are released
 // separately: the next tile's K (and queries) load once this tile's Q.K^T has read K, its V once
 // the P.V products have read V, so both copies overlap this tile's softmax and output phases.
@@ -29,8 +32,8 @@ using namespace sm100;
 namespace {
 
 constexpr int kUtThreads = 192;
-constexpr int kUtTok = 64;          // tokens per unit (= S)
-constexpr int kUtRows = 128;        // tokens per tile: two units
+constexpr int kUtTok = 64;          // tokens per tile half (S = 64: one unit; S = 128: half of one)
+constexpr int kUtRows = 128;        // tokens per tile
 constexpr int kUtCols = 16;         // query heads per tile (MMA N)
 constexpr int kUtD = 128;           // head dim (MMA M of the P.V product)
 constexpr int kUtCtasPerSm = 3;
@@ -55,7 +58,7 @@ struct UtShape {
   static_assert(kUtCtasPerSm * kUtTmemCols <= 512, "TMEM columns");
 };
 
-// Unit x of a row: token range start and length (0: empty unit).
+// Unit x of a row: token range start and length (0: empty unit); units are S tokens long.
 __device__ __forceinline__ void unit_span(const Dims& D, const int32_t* __restrict__ idx,
                                           int64_t row, int64_t n, int64_t pos, int n_units, int x,
                                           int64_t& t0, int& len) {
@@ -63,12 +66,12 @@ __device__ __forceinline__ void unit_span(const Dims& D, const int32_t* __restri
   len = 0;
   if (x < D.K) {
     const int c = __ldg(idx + row * D.K + x);
-    if (c >= 0 && c < n) { t0 = (int64_t)c * kUtTok; len = kUtTok; }
+    if (c >= 0 && c < n) { t0 = (int64_t)c * D.S; len = D.S; }
   } else if (x < n_units) {
-    const int64_t s = (int64_t)D.S * n + (int64_t)(x - D.K) * kUtTok;
+    const int64_t s = (int64_t)D.S * n + (int64_t)(x - D.K) * D.S;
     const int64_t l = pos + 1 - s;
     t0 = s;
-    len = l <= 0 ? 0 : (l >= kUtTok ? kUtTok : (int)l);
+    len = l <= 0 ? 0 : (l >= D.S ? D.S : (int)l);
   }
 }
 
@@ -103,6 +106,7 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_units = D.K + n_pieces;
+  const bool wide = D.S == kUtRows;   // one unit per tile (S = 128), else two (S = 64)
   const int64_t t_begin = n_tiles_total * blockIdx.x / gridDim.x;
   const int64_t t_end = n_tiles_total * (blockIdx.x + 1) / gridDim.x;
   const int n_local = (int)(t_end - t_begin);
@@ -129,7 +133,7 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
-      // token spans of a tile's two units (the idx reads of the next tile are issued before
+      // token rows of a tile's two halves (the idx reads of the next tile are issued before
       // the waits for the current stage, so their latency hides behind them)
       auto spans = [&](int u, int32_t (&y)[2], int32_t& qi, int32_t& qh) {
         const int64_t t = t_begin + u;
@@ -137,12 +141,21 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
         const int64_t i = row % D.N_q, bg = row / D.N_q;
         const int64_t g = bg % D.Hkv, b = bg / D.Hkv;
         const int64_t pos = D.q_pos0 + i, n = n_eligible(pos, D.S, D.W);
-        for (int half = 0; half < 2; ++half) {
+        // an empty unit, or a unit's missing second half, still loads (from token 0 of the row,
+        // or past the unit's end); the softmax masks those tokens
+        if (wide) {
           int64_t t0;
           int len;
-          unit_span(D, idx, row, n, pos, n_units, (int)(2 * pr + half), t0, len);
-          // an empty unit still loads (from token 0 of the row); the softmax masks it
-          y[half] = (int32_t)(bg * D.N_kv + t0);
+          unit_span(D, idx, row, n, pos, n_units, (int)pr, t0, len);
+          y[0] = (int32_t)(bg * D.N_kv + t0);
+          y[1] = y[0] + kUtTok;
+        } else {
+          for (int half = 0; half < 2; ++half) {
+            int64_t t0;
+            int len;
+            unit_span(D, idx, row, n, pos, n_units, (int)(2 * pr + half), t0, len);
+            y[half] = (int32_t)(bg * D.N_kv + t0);
+          }
         }
         qi = (int32_t)i;
         qh = (int32_t)(b * D.Hq + g * D.G);
@@ -210,7 +223,12 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
             const uint64_t ad = desc_mnmajor_sw128(
                 smem_u32(sV + half * SH::UNIT_BOX + ks * 16 * 128), SH::BLK);
             const uint64_t bd = desc_kmajor_sw128(smem_u32(sP + half * SH::P_BLK) + ks * 32);
-            mma_bf16_ss(tmem + (half ? kColOB : kColOA), ad, bd, IDESC_O, ks > 0 ? 1u : 0u);
+            // two units: one accumulator each; one unit: both halves into the first.  (One MMA
+            // statement with the column and the accumulate flag as values: the same choice
+            // written as two MMA statements under a branch gave wrong S = 64 results.)
+            const uint32_t col = (wide || half == 0) ? kColOA : kColOB;
+            const uint32_t acc = (ks > 0 || (wide && half > 0)) ? 1u : 0u;
+            mma_bf16_ss(tmem + col, ad, bd, IDESC_O, acc);
           }
         }
         mma_commit(o_full);
@@ -235,9 +253,15 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
       const int64_t pos = D.q_pos0 + i, n = n_eligible(pos, D.S, D.W);
       int64_t t0a, t0b;
       int lena, lenb;
-      unit_span(D, idx, row, n, pos, n_units, (int)(2 * pr), t0a, lena);
-      unit_span(D, idx, row, n, pos, n_units, (int)(2 * pr + 1), t0b, lenb);
-      const bool tok_ok = (tk & 63) < (half ? lenb : lena);
+      bool tok_ok;
+      if (wide) {
+        unit_span(D, idx, row, n, pos, n_units, (int)pr, t0a, lena);
+        tok_ok = tk < lena;
+      } else {
+        unit_span(D, idx, row, n, pos, n_units, (int)(2 * pr), t0a, lena);
+        unit_span(D, idx, row, n, pos, n_units, (int)(2 * pr + 1), t0b, lenb);
+        tok_ok = (tk & 63) < (half ? lenb : lena);
+      }
       float* rm = red_m + ph * 4 * kUtCols;
       float* rl = red_l + ph * 4 * kUtCols;
       // ---- logits of this thread's token for the 16 head columns.  A failed (timed-out) wait
@@ -252,7 +276,7 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
       }
 #pragma unroll
       for (int h = 0; h < kUtCols; ++h) x[h] = (ok && tok_ok && h < G) ? x[h] * D.scale : -INFINITY;
-      // ---- unit max per head over the unit's two warps
+      // ---- unit max per head over the unit's warps (two, or all four when the tile is one unit)
 #pragma unroll
       for (int h = 0; h < kUtCols; ++h) {
         if (h >= G) break;
@@ -265,7 +289,8 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
       for (int h = 0; h < kUtCols; ++h) {
         p[h] = 0.f;
         if (h >= G) continue;
-        const float m = fmaxf(rm[qd * kUtCols + h], rm[(qd ^ 1) * kUtCols + h]);
+        float m = fmaxf(rm[qd * kUtCols + h], rm[(qd ^ 1) * kUtCols + h]);
+        if (wide) m = fmaxf(m, fmaxf(rm[(qd ^ 2) * kUtCols + h], rm[(qd ^ 3) * kUtCols + h]));
         p[h] = (x[h] == -INFINITY) ? 0.f : __expf(x[h] - m);
         const float ws = warp_sum(p[h]);
         if (lane == 0) rl[qd * kUtCols + h] = ws;
@@ -294,6 +319,22 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
       tmem_ld16(lane_base + kColOA, oa);
       tmem_ld16(lane_base + kColOB, ob);
       tmem_wait_ld();
+      if (wide) {
+#pragma unroll
+        for (int h = 0; h < kUtCols; ++h) {
+          if (h >= G) break;
+          const int64_t hrow = (b * D.Hq + g * G + h) * D.N_q + i;
+          const float l = (rl[0 * kUtCols + h] + rl[1 * kUtCols + h]) +
+                          (rl[2 * kUtCols + h] + rl[3 * kUtCols + h]);
+          part_o[(hrow * n_units + pr) * kUtD + tk] = l > 0.f ? oa[h] / l : 0.f;
+          if (tk == 0) {
+            const float m = fmaxf(fmaxf(rm[0 * kUtCols + h], rm[1 * kUtCols + h]),
+                                  fmaxf(rm[2 * kUtCols + h], rm[3 * kUtCols + h]));
+            part_lse[hrow * n_units + pr] = l > 0.f ? m + logf(l) : -INFINITY;
+          }
+        }
+        continue;
+      }
       const int ua = (int)(2 * pr), ub = ua + 1;
 #pragma unroll
       for (int h = 0; h < kUtCols; ++h) {
@@ -350,8 +391,10 @@ bool map_rows(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows
 }  // namespace
 
 bool units_tc_supported(const Dims& D, bool bf16) {
-  if (!bf16 || D.d != kUtD || D.S != kUtTok || D.G < 1 || D.G > kUtCols) return false;
-  if (D.B * D.Hkv * D.N_kv >= (int64_t)INT32_MAX) return false;
+  if (!bf16 || D.d != kUtD || (D.S != kUtTok && D.S != kUtRows) || D.G < 1 || D.G > kUtCols)
+    return false;
+  // token rows are int32 TMA coordinates, the second half of a unit up to 64 past its end
+  if (D.B * D.Hkv * D.N_kv + kUtRows >= (int64_t)INT32_MAX) return false;
   if (D.B * D.Hq >= (int64_t)INT32_MAX || D.N_q >= (int64_t)INT32_MAX) return false;
   return true;
 }
@@ -379,7 +422,7 @@ cudaError_t launch_attn_units_tc(const Dims& D, int n_pieces, const void* q, con
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  const int64_t tiles_per_row = (n_units + 1) / 2;
+  const int64_t tiles_per_row = D.S == kUtRows ? n_units : (n_units + 1) / 2;
   const int64_t total = rows * tiles_per_row;
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);

@@ -108,6 +108,17 @@ EDGE_CASES = {
     "tc_g8_d128": dict(B=1, Hq=8, Hkv=1, N=3000, d=128, S=64, K=16, W_=128),
     "tc_g8_d128_s128": dict(B=1, Hq=8, Hkv=1, N=6000, d=128, S=128, K=16, W_=256),
     "tc_g8_d128_k8_b2": dict(B=2, Hq=16, Hkv=2, N=2100, d=128, S=64, K=8, W_=64),
+    # decode units of S = 128 tokens on the tensor core (bf16): a ragged last window piece,
+    # more selected slots than eligible chunks (empty units), several queries with their own
+    # windows, and 16 heads per group
+    "decode_s128_window": dict(B=2, Hq=8, Hkv=1, N=9000, d=128, S=128, K=16, W_=300,
+                               q_pos0=8999, N_q=1),
+    "decode_s128_k_gt_n": dict(B=1, Hq=4, Hkv=1, N=700, d=128, S=128, K=16, W_=256,
+                               q_pos0=699, N_q=1),
+    "decode_s128_multi": dict(B=2, Hq=16, Hkv=2, N=5000, d=128, S=128, K=8, W_=129,
+                              q_pos0=4991, N_q=5),
+    "decode_s128_g16": dict(B=1, Hq=16, Hkv=1, N=12345, d=128, S=128, K=12, W_=2048,
+                            q_pos0=12344, N_q=1),
 }
 
 
