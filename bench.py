@@ -907,6 +907,13 @@ def run_only_extra(args):
         out = extra_decode(max(3, args.steps), peaks)
     elif args.only_extra == "decode_step":
         out = extra_decode_step(max(3, args.steps), peaks)
+    elif args.only_extra == "extreme_decode":
+        from hierarchical_chunk_sparse_scoring_b200 import workloads as W
+        N = n or 262144
+        wl = W.make("extreme", "cuda", N=N)
+        out = {"workload": "extreme", "N": N,
+               "decode": time_mode(W.decode_view(wl), max(5, args.steps), peaks,
+                                   "extreme_N%d_decode" % N)}
     else:
         out = extra_landmarks(peaks, 1, 1, n or (1 << 22), 128, 128, steps=args.steps)
     print(json.dumps(out), flush=True)
@@ -923,7 +930,7 @@ def main():
     ap.add_argument("--B", type=int, default=None, help="override the workload's batch")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--only-extra", choices=["backward", "prologue", "decode", "decode_step",
-                                             "landmarks"], default=None,
+                                             "extreme_decode", "landmarks"], default=None,
                     help="run one extra measurement alone and print its JSON (for profiling)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
