@@ -77,6 +77,8 @@ __device__ __forceinline__ void unit_span(const Dims& D, const int32_t* __restri
 
 }  // namespace
 
+// GM: a bound on the group's heads (4, 8 or 16), so the per-head loops unroll to G's size.
+template <int GM>
 __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
     attn_units_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
@@ -122,6 +124,10 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
     fence_barrier_init();
   }
   if (warp == 1) tmem_alloc(tmem_holder, kUtTmemCols);
+  // P rows of heads >= GM are never written in the loop: zero them once (they only feed output
+  // columns nobody reads, but stay finite)
+  for (int e = threadIdx.x; e < SH::P_BYTES / 16; e += kUtThreads)
+    reinterpret_cast<uint4*>(sP)[e] = make_uint4(0u, 0u, 0u, 0u);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -275,18 +281,18 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
         tmem_wait_ld();
       }
 #pragma unroll
-      for (int h = 0; h < kUtCols; ++h) x[h] = (ok && tok_ok && h < G) ? x[h] * D.scale : -INFINITY;
+      for (int h = 0; h < GM; ++h) x[h] = (ok && tok_ok && h < G) ? x[h] * D.scale : -INFINITY;
       // ---- unit max per head over the unit's warps (two, or all four when the tile is one unit)
 #pragma unroll
-      for (int h = 0; h < kUtCols; ++h) {
+      for (int h = 0; h < GM; ++h) {
         if (h >= G) break;
         const float wm = warp_max(x[h]);
         if (lane == 0) rm[qd * kUtCols + h] = wm;
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");
-      float p[kUtCols];
+      float p[GM];
 #pragma unroll
-      for (int h = 0; h < kUtCols; ++h) {
+      for (int h = 0; h < GM; ++h) {
         p[h] = 0.f;
         if (h >= G) continue;
         float m = fmaxf(rm[qd * kUtCols + h], rm[(qd ^ 1) * kUtCols + h]);
@@ -300,7 +306,7 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
         uint8_t* pb = sP + half * SH::P_BLK;
         const int tt = tk & 63;
 #pragma unroll
-        for (int h = 0; h < kUtCols; ++h) {
+        for (int h = 0; h < GM; ++h) {
           const int off = (h >> 3) * 1024 + (h & 7) * 128 + ((((tt >> 3) ^ (h & 7))) << 4) +
                           (tt & 7) * 2;
           *reinterpret_cast<__nv_bfloat16*>(pb + off) = __float2bfloat16_rn(p[h]);
@@ -321,7 +327,7 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
       tmem_wait_ld();
       if (wide) {
 #pragma unroll
-        for (int h = 0; h < kUtCols; ++h) {
+        for (int h = 0; h < GM; ++h) {
           if (h >= G) break;
           const int64_t hrow = (b * D.Hq + g * G + h) * D.N_q + i;
           const float l = (rl[0 * kUtCols + h] + rl[1 * kUtCols + h]) +
@@ -337,7 +343,7 @@ __global__ void __launch_bounds__(kUtThreads, kUtCtasPerSm)
       }
       const int ua = (int)(2 * pr), ub = ua + 1;
 #pragma unroll
-      for (int h = 0; h < kUtCols; ++h) {
+      for (int h = 0; h < GM; ++h) {
         if (h >= G) break;
         const int64_t hrow = (b * D.Hq + g * G + h) * D.N_q + i;
         const float la = rl[0 * kUtCols + h] + rl[1 * kUtCols + h];
@@ -430,10 +436,11 @@ cudaError_t launch_attn_units_tc(const Dims& D, int n_pieces, const void* q, con
   if (e != cudaSuccess) return e;
   const int64_t slots = (int64_t)kUtCtasPerSm * sms;
   const int64_t grid = total < slots ? total : slots;
-  e = cudaFuncSetAttribute(attn_units_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           UtShape::SMEM);
+  auto kern = D.G <= 4 ? attn_units_tc_kernel<4>
+                        : D.G <= 8 ? attn_units_tc_kernel<8> : attn_units_tc_kernel<16>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, UtShape::SMEM);
   if (e != cudaSuccess) return e;
-  attn_units_tc_kernel<<<(unsigned)grid, kUtThreads, UtShape::SMEM, st>>>(
+  kern<<<(unsigned)grid, kUtThreads, UtShape::SMEM, st>>>(
       tmQ, tmK, tmV, D, n_pieces, tiles_per_row, total, idx, part_o, part_lse, status);
   return cudaGetLastError();
 }
