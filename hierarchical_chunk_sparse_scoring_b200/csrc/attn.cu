@@ -180,8 +180,21 @@ __device__ __forceinline__ void fuse_row(const Dims& D, int n_pieces, int64_t ro
   };
   const float* pr = part_o + row * NU * d;
   if (NU <= 64 && d == 128) {
-    // lanes hold the weights of units lane and lane + 32 (scores read once); then every lane
-    // reads its 4 output columns of all units, 16 loads in flight per batch
+    // lanes hold the weights of units lane and lane + 32 (scores read once); every lane reads its
+    // 4 output columns of all units, 16 loads in flight per batch, the first batch issued before
+    // the score loads so that both are in flight together
+    float v[16][4];
+    auto load_batch = [&](int u0) {
+#pragma unroll
+      for (int e2 = 0; e2 < 16; ++e2) {
+        if (u0 + e2 < NU) {
+          load4cg(pr + (int64_t)(u0 + e2) * 128 + lane * 4, v[e2]);
+        } else {
+          v[e2][0] = v[e2][1] = v[e2][2] = v[e2][3] = 0.f;
+        }
+      }
+    };
+    load_batch(0);
     const float s0 = lane < NU ? score_of(lane) : -INFINITY;
     const float s1 = lane + 32 < NU ? score_of(lane + 32) : -INFINITY;
     const float M = warp_max(fmaxf(s0, s1));
@@ -191,15 +204,7 @@ __device__ __forceinline__ void fuse_row(const Dims& D, int n_pieces, int64_t ro
     const float w0 = e0 / Z, w1 = e1 / Z;
     float o[4] = {0.f, 0.f, 0.f, 0.f};
     for (int u0 = 0; u0 < NU; u0 += 16) {
-      float v[16][4];
-#pragma unroll
-      for (int e2 = 0; e2 < 16; ++e2) {
-        if (u0 + e2 < NU) {
-          load4cg(pr + (int64_t)(u0 + e2) * 128 + lane * 4, v[e2]);
-        } else {
-          v[e2][0] = v[e2][1] = v[e2][2] = v[e2][3] = 0.f;
-        }
-      }
+      if (u0 > 0) load_batch(u0);
       const float wsrc = u0 < 32 ? w0 : w1;   // a batch lies on one side of unit 32
 #pragma unroll
       for (int e2 = 0; e2 < 16; ++e2) {

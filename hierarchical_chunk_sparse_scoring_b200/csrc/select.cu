@@ -72,18 +72,19 @@ __device__ __forceinline__ void write_selection(const Dims& D, int64_t b, int64_
 
 // Same result for bf16 inputs with the winners' landmark rows read by wide loads that are all in
 // flight at once, and the group's calibrated queries staged once per warp in shared memory
-// (qsh: [GM][D_] bf16); lane r < K handles winner c_r.
+// (qsh: [GM][D_] bf16; already filled, and visible to this warp, when q_staged); lane r < K
+// handles winner c_r.
 template <int D_, int GM>
 __device__ __forceinline__ void write_selection_wide(const Dims& D, int64_t b, int64_t g,
                                                      int64_t i, __nv_bfloat16* qsh,
                                                      const __nv_bfloat16* qc,
                                                      const __nv_bfloat16* kb, const float* bb,
                                                      int lane, int c, int32_t* idx,
-                                                     float* s_sel) {
+                                                     float* s_sel, bool q_staged = false) {
   constexpr int NV = D_ / 8;   // 16-byte vectors per row
   const int K = D.K, G = D.G;
   uint4* q4 = reinterpret_cast<uint4*>(qsh);
-  for (int e = lane; e < G * NV; e += 32) {
+  for (int e = lane; !q_staged && e < G * NV; e += 32) {
     const int h = e / NV, j = e - h * NV;
     const int64_t hrow = ((b * D.Hq) + g * G + h) * D.N_q + i;
     q4[h * NV + j] = __ldg(reinterpret_cast<const uint4*>(qc + hrow * D_) + j);
@@ -712,6 +713,17 @@ __global__ void __launch_bounds__(kTopkThreads) select_topk_row_kernel(
   const int64_t row = blockIdx.x;
   const int64_t i = row % D.N_q, bg = row / D.N_q, g = bg % D.Hkv, b = bg / D.Hkv;
   const int K = D.K;
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    // the group's calibrated queries for the winners' per-head scores, staged now so that their
+    // loads overlap the selection (visible to warp 0 after the barrier below)
+    constexpr int NV = D_ / 8;
+    for (int e = threadIdx.x; e < D.G * NV; e += kTopkThreads) {
+      const int h = e / NV, j = e - h * NV;
+      const int64_t hrow = ((b * D.Hq) + g * D.G + h) * D.N_q + i;
+      reinterpret_cast<uint4*>(qsh)[h * NV + j] =
+          __ldg(reinterpret_cast<const uint4*>(qc + hrow * D_) + j);
+    }
+  }
   const int64_t n = n_eligible(D.q_pos0 + i, D.S, D.W);
   const float* sr = sigma + row * n_stride;             // 16-byte aligned (n_stride % 4 == 0)
   const int64_t n4 = n >> 2;
@@ -871,7 +883,7 @@ __global__ void __launch_bounds__(kTopkThreads) select_topk_row_kernel(
   }
   if constexpr (std::is_same<T, __nv_bfloat16>::value)
     write_selection_wide<D_, GM>(D, b, g, i, qsh, qc, klm + bg * D.C * D_, blm + bg * D.C, lane,
-                                 wc, idx, s_sel);
+                                 wc, idx, s_sel, /*q_staged=*/true);
   else
     write_selection<T, GM>(D, b, g, i, nullptr, qc, klm + bg * D.C * D.d, blm + bg * D.C, lane,
                            wc, idx, s_sel);
