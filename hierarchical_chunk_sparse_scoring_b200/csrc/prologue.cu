@@ -290,10 +290,12 @@ __device__ __forceinline__ void turn(float (&x)[EPL], float (&y)[EPL], int lane,
 // grid (token blocks, B); every head of the block in turn.  r = 0 leaves q_cal = R(q).  Each
 // warp takes kQhTpw tokens together (their loads in flight at once); W_up[h]'s rows of the
 // lane's dims are read through L1 (every warp of every CTA reads the same d x r block), 8
-// columns at a time, and applied to all of the warp's tokens.
+// columns at a time, and applied to all of the warp's tokens.  The pass is bound by instruction
+// issue, not memory: three CTAs per SM (80 registers, no spills) issue 10 % faster than two
+// (128 registers); four spill.
 constexpr int kQhTpw = kQhTokens / (kQhThreads / 32);
 template <typename T, int DD>
-__global__ void __launch_bounds__(kQhThreads, 2)
+__global__ void __launch_bounds__(kQhThreads, 3)
     qcal_hope_kernel(int64_t N_q, int64_t Hq, int64_t q_pos0, int r, double base,
                      double train_len, const T* __restrict__ q, const float* __restrict__ u,
                      const T* __restrict__ W_up, T* __restrict__ q_out, T* __restrict__ qc_out) {
