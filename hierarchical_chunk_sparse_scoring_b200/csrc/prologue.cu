@@ -196,8 +196,9 @@ cudaError_t launch_qdown_t(int64_t M, int64_t N, int64_t Kdim, const void* hidde
 constexpr int kQhTokens = 32;     // tokens per CTA
 constexpr int kQhThreads = 256;
 
-// A lane's EPL = d/32 consecutive dims of a row: lanes 0-15 hold the first half (dims m of the
-// pairs), lanes 16-31 the second (dims m + d/2), so a pair's partner sits in lane ^ 16.
+// EPL consecutive dims of a row as floats, and back.  (The rotation kernel's lanes hold d/32
+// consecutive dims each: lanes 0-15 the first half, dims m of the pairs, lanes 16-31 the second,
+// dims m + d/2, so a pair's partner sits in lane ^ 16.)
 template <typename T, int EPL>
 __device__ __forceinline__ void load_dims(const T* p, float (&v)[EPL]);
 template <>
@@ -287,26 +288,49 @@ __device__ __forceinline__ void turn(float (&x)[EPL], float (&y)[EPL], int lane,
   }
 }
 
+// HP consecutive elements (HP = 1 or 2) of a row as floats, and back.
+template <typename T, int HP>
+__device__ __forceinline__ void load_n(const T* p, float (&v)[HP]) {
+  if constexpr (HP == 2) {
+    load_dims<T, 2>(p, v);
+  } else {
+    v[0] = Elem<T>::to_f(p[0]);
+  }
+}
+template <typename T, int HP>
+__device__ __forceinline__ void store_n(T* p, const float (&v)[HP]) {
+  if constexpr (HP == 2) {
+    store_dims<T, 2>(p, v);
+  } else if constexpr (std::is_same<T, float>::value) {
+    p[0] = v[0];
+  } else {
+    p[0] = __float2bfloat16_rn(v[0]);
+  }
+}
+
 // grid (token blocks, B); every head of the block in turn.  r = 0 leaves q_cal = R(q).  Each
-// warp takes kQhTpw tokens together (their loads in flight at once); W_up[h]'s rows of the
-// lane's dims are read through L1 (every warp of every CTA reads the same d x r block), 8
-// columns at a time, and applied to all of the warp's tokens.  The pass is bound by instruction
-// issue, not memory: three CTAs per SM (80 registers, no spills) issue 10 % faster than two
-// (128 registers); four spill.
+// warp takes kQhTpw tokens together (their loads in flight at once).  A lane holds HP = d/64
+// whole rotation pairs, dims m0 .. m0 + HP - 1 and their partners m + d/2, so the rotation
+// needs no exchange between lanes; the rows of W_up[h] for the lane's dims are read through L1
+// (every warp of every CTA reads the same d x r block), 8 columns at a time, and applied to all
+// of the warp's tokens.  The pass is bound by instruction issue, not memory: three CTAs per SM
+// (no spills) issue faster than two; four spill.
 constexpr int kQhTpw = kQhTokens / (kQhThreads / 32);
 template <typename T, int DD>
 __global__ void __launch_bounds__(kQhThreads, 3)
     qcal_hope_kernel(int64_t N_q, int64_t Hq, int64_t q_pos0, int r, double base,
                      double train_len, const T* __restrict__ q, const float* __restrict__ u,
                      const T* __restrict__ W_up, T* __restrict__ q_out, T* __restrict__ qc_out) {
-  constexpr int EPL = DD / 32;
-  __shared__ float2 sCS[kQhTokens * (DD / 2)];
+  constexpr int EPL = DD / 32;   // dims per lane
+  constexpr int HP = EPL / 2;    // pairs per lane
+  constexpr int HALF = DD / 2;
+  __shared__ float2 sCS[kQhTokens * HALF];
   const int64_t b = blockIdx.y;
   const int64_t i0 = (int64_t)blockIdx.x * kQhTokens;
   angle_table<DD>(sCS, q_pos0 + i0, base, train_len);
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int dim0 = lane * EPL;
+  const int m0 = lane * HP;      // element e < HP: dim m0 + e; e >= HP: dim HALF + m0 + e - HP
   const int t0 = warp * kQhTpw;
   const bool vec_w = r % (sizeof(T) == 2 ? 8 : 4) == 0;
   for (int64_t h = 0; h < Hq; ++h) {
@@ -315,7 +339,12 @@ __global__ void __launch_bounds__(kQhThreads, 3)
     for (int tt = 0; tt < kQhTpw; ++tt) {
       const int64_t i = i0 + t0 + tt;
       if (i < N_q) {
-        load_dims<T, EPL>(q + ((b * Hq + h) * N_q + i) * DD + dim0, x[tt]);
+        const T* qr = q + ((b * Hq + h) * N_q + i) * DD;
+        float lo[HP], hi[HP];
+        load_n<T, HP>(qr + m0, lo);
+        load_n<T, HP>(qr + HALF + m0, hi);
+#pragma unroll
+        for (int k = 0; k < HP; ++k) { x[tt][k] = lo[k]; x[tt][HP + k] = hi[k]; }
         const float* ur = u + (b * N_q + i) * (Hq * r) + h * r;
         ua[tt] = lane < r ? ur[lane] : 0.f;
         ub[tt] = lane + 32 < r ? ur[lane + 32] : 0.f;
@@ -327,18 +356,21 @@ __global__ void __launch_bounds__(kQhThreads, 3)
 #pragma unroll
       for (int e = 0; e < EPL; ++e) c[tt][e] = x[tt][e];
     }
-    const T* wrow = W_up + (h * DD + dim0) * r;   // rows dim0 .. dim0 + EPL - 1, r each
+    // the rows of W_up[h] (d x r) of this lane's dims: element e's row at wrow(e)
+    const T* wlo = W_up + (h * DD + m0) * r;
+    const T* whi = wlo + HALF * r;
+    auto wrow = [&](int e) { return e < HP ? wlo + e * r : whi + (e - HP) * r; };
     for (int j0 = 0; j0 < r; j0 += 8) {
       float w[EPL][8];
       if (vec_w && j0 + 8 <= r) {   // 16-byte pieces of the rows (r a multiple of 8 / 4)
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) load_piece8<T>(wrow + e * r + j0, w[e]);
+        for (int e = 0; e < EPL; ++e) load_piece8<T>(wrow(e) + j0, w[e]);
       } else {
 #pragma unroll
         for (int e = 0; e < EPL; ++e)
 #pragma unroll
           for (int jj = 0; jj < 8; ++jj)
-            w[e][jj] = j0 + jj < r ? Elem<T>::to_f(__ldg(wrow + e * r + j0 + jj)) : 0.f;
+            w[e][jj] = j0 + jj < r ? Elem<T>::to_f(__ldg(wrow(e) + j0 + jj)) : 0.f;
       }
 #pragma unroll
       for (int jj = 0; jj < 8; ++jj) {
@@ -355,11 +387,28 @@ __global__ void __launch_bounds__(kQhThreads, 3)
 #pragma unroll
     for (int tt = 0; tt < kQhTpw; ++tt) {
       const int64_t i = i0 + t0 + tt;
-      turn<EPL>(x[tt], c[tt], lane, sCS + (t0 + tt) * (DD / 2));
+      const float2* cs_row = sCS + (t0 + tt) * HALF + m0;
+#pragma unroll
+      for (int k = 0; k < HP; ++k) {   // pair m0 + k: (m, m + d/2) turned by its angle
+        const float2 cs = cs_row[k];
+        const float xa = x[tt][k], xb = x[tt][HP + k];
+        x[tt][k] = xa * cs.x - xb * cs.y;
+        x[tt][HP + k] = xa * cs.y + xb * cs.x;
+        const float ca = c[tt][k], cb = c[tt][HP + k];
+        c[tt][k] = ca * cs.x - cb * cs.y;
+        c[tt][HP + k] = ca * cs.y + cb * cs.x;
+      }
       if (i < N_q) {
         const int64_t row = (b * Hq + h) * N_q + i;
-        store_dims<T, EPL>(q_out + row * DD + dim0, x[tt]);
-        store_dims<T, EPL>(qc_out + row * DD + dim0, c[tt]);
+        float lo[HP], hi[HP];
+#pragma unroll
+        for (int k = 0; k < HP; ++k) { lo[k] = x[tt][k]; hi[k] = x[tt][HP + k]; }
+        store_n<T, HP>(q_out + row * DD + m0, lo);
+        store_n<T, HP>(q_out + row * DD + HALF + m0, hi);
+#pragma unroll
+        for (int k = 0; k < HP; ++k) { lo[k] = c[tt][k]; hi[k] = c[tt][HP + k]; }
+        store_n<T, HP>(qc_out + row * DD + m0, lo);
+        store_n<T, HP>(qc_out + row * DD + HALF + m0, hi);
       }
     }
   }
