@@ -13,11 +13,12 @@
 //                  a dense contraction on the tcgen05 tensor cores (bf16 operands by TMA with the
 //                  128-byte swizzle, fp32 accumulator in TMEM, 128 x BN tiles, a 4-stage ring).
 //   qcal_hope_kernel  per (b, 32 tokens), every head in turn: q_cal = R(q + W_up u), q = R(q);
-//                  HBM-bound (q read, both written, u read); W_up[h] read through L1; four
-//                  tokens per warp in flight together, each lane d/32 consecutive dims (the
-//                  pair partner in lane ^ 16); the block's (token, pair) angles p theta_m
-//                  reduced modulo 2 pi in fp64 once (p up to 2^22 makes an fp32 product lose
-//                  whole radians), then sincosf, kept in shared memory for all heads.
+//                  q read, both written, u read; W_up[h] read through L1; four tokens per warp
+//                  in flight together, each lane d/64 whole rotation pairs (dims m and m + d/2,
+//                  so the rotation stays in the lane); the block's (token, pair) angles
+//                  p theta_m reduced modulo 2 pi in fp64 once (p up to 2^22 makes an fp32
+//                  product lose whole radians), then sincosf, kept in shared memory for all
+//                  heads.  hope_rotate_kernel turns keys the same way.
 #include <cudaTypedefs.h>
 
 #include <type_traits>
@@ -196,25 +197,13 @@ cudaError_t launch_qdown_t(int64_t M, int64_t N, int64_t Kdim, const void* hidde
 constexpr int kQhTokens = 32;     // tokens per CTA
 constexpr int kQhThreads = 256;
 
-// EPL consecutive dims of a row as floats, and back.  (The rotation kernel's lanes hold d/32
-// consecutive dims each: lanes 0-15 the first half, dims m of the pairs, lanes 16-31 the second,
-// dims m + d/2, so a pair's partner sits in lane ^ 16.)
+// Two consecutive dims of a row as floats, and back (EPL = 2).
 template <typename T, int EPL>
 __device__ __forceinline__ void load_dims(const T* p, float (&v)[EPL]);
-template <>
-__device__ __forceinline__ void load_dims<__nv_bfloat16, 4>(const __nv_bfloat16* p, float (&v)[4]) {
-  const uint2 t = *reinterpret_cast<const uint2*>(p);
-  v[0] = bf16_lo(t.x); v[1] = bf16_hi(t.x); v[2] = bf16_lo(t.y); v[3] = bf16_hi(t.y);
-}
 template <>
 __device__ __forceinline__ void load_dims<__nv_bfloat16, 2>(const __nv_bfloat16* p, float (&v)[2]) {
   const uint32_t t = *reinterpret_cast<const uint32_t*>(p);
   v[0] = bf16_lo(t); v[1] = bf16_hi(t);
-}
-template <>
-__device__ __forceinline__ void load_dims<float, 4>(const float* p, float (&v)[4]) {
-  const float4 t = *reinterpret_cast<const float4*>(p);
-  v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
 }
 template <>
 __device__ __forceinline__ void load_dims<float, 2>(const float* p, float (&v)[2]) {
@@ -223,18 +212,12 @@ __device__ __forceinline__ void load_dims<float, 2>(const float* p, float (&v)[2
 }
 template <typename T, int EPL>
 __device__ __forceinline__ void store_dims(T* p, const float (&v)[EPL]) {
+  static_assert(EPL == 2, "two dims");
   if constexpr (std::is_same<T, float>::value) {
-    if constexpr (EPL == 4) *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
-    else *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+    *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
   } else {
-    uint32_t w[EPL / 2];
-#pragma unroll
-    for (int e = 0; e < EPL / 2; ++e) {
-      const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-      w[e] = *reinterpret_cast<const uint32_t*>(&h);
-    }
-    if constexpr (EPL == 4) *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
-    else *reinterpret_cast<uint32_t*>(p) = w[0];
+    const __nv_bfloat162 h = __floats2bfloat162_rn(v[0], v[1]);
+    *reinterpret_cast<uint32_t*>(p) = *reinterpret_cast<const uint32_t*>(&h);
   }
 }
 
@@ -271,21 +254,6 @@ __device__ __forceinline__ void load_piece8<float>(const float* p, float (&v)[8]
   const float4 a = __ldg(reinterpret_cast<const float4*>(p));
   const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
   v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-
-// Turns this lane's dims: pair m (first half) and m + d/2 (second half, the partner lane).
-template <int EPL>
-__device__ __forceinline__ void turn(float (&x)[EPL], float (&y)[EPL], int lane,
-                                     const float2* cs_row) {
-  const bool first = lane < 16;
-#pragma unroll
-  for (int e = 0; e < EPL; ++e) {
-    const float2 cs = cs_row[(lane & 15) * EPL + e];
-    const float ox = __shfl_xor_sync(0xffffffffu, x[e], 16);
-    const float oy = __shfl_xor_sync(0xffffffffu, y[e], 16);
-    x[e] = first ? x[e] * cs.x - ox * cs.y : ox * cs.y + x[e] * cs.x;
-    y[e] = first ? y[e] * cs.x - oy * cs.y : oy * cs.y + y[e] * cs.x;
-  }
 }
 
 // HP consecutive elements (HP = 1 or 2) of a row as floats, and back.
@@ -419,23 +387,33 @@ template <typename T, int DD>
 __global__ void __launch_bounds__(kQhThreads)
     hope_rotate_kernel(int64_t BH, int64_t N, int64_t pos0, double base, double train_len,
                        const T* __restrict__ x, T* __restrict__ out) {
-  constexpr int EPL = DD / 32;
-  __shared__ float2 sCS[kQhTokens * (DD / 2)];
+  constexpr int HP = DD / 64;   // whole pairs per lane
+  constexpr int HALF = DD / 2;
+  __shared__ float2 sCS[kQhTokens * HALF];
   const int64_t n0 = (int64_t)blockIdx.x * kQhTokens;
   angle_table<DD>(sCS, pos0 + n0, base, train_len);
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = lane * HP;
   for (int64_t bh = 0; bh < BH; ++bh) {
     for (int t = warp; t < kQhTokens; t += kQhThreads / 32) {
       const int64_t n = n0 + t;
       if (n >= N) break;
       const int64_t row = bh * N + n;
-      float v[EPL], w[EPL];
-      load_dims<T, EPL>(x + row * DD + lane * EPL, v);
+      // this lane's pairs m0 .. m0 + HP - 1 with their partners m + d/2 (in place is safe: a
+      // lane writes back exactly the elements it read)
+      float lo[HP], hi[HP];
+      load_n<T, HP>(x + row * DD + m0, lo);
+      load_n<T, HP>(x + row * DD + HALF + m0, hi);
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) w[e] = 0.f;
-      turn<EPL>(v, w, lane, sCS + t * (DD / 2));
-      store_dims<T, EPL>(out + row * DD + lane * EPL, v);
+      for (int k = 0; k < HP; ++k) {
+        const float2 cs = sCS[t * HALF + m0 + k];
+        const float a = lo[k], bb = hi[k];
+        lo[k] = a * cs.x - bb * cs.y;
+        hi[k] = a * cs.y + bb * cs.x;
+      }
+      store_n<T, HP>(out + row * DD + m0, lo);
+      store_n<T, HP>(out + row * DD + HALF + m0, hi);
     }
   }
 }
