@@ -24,6 +24,10 @@ constexpr size_t kStatusBytes = 256;
 constexpr int kChunksPerSplit = 512;
 constexpr int64_t kDecodeMaxQueries = 16;
 constexpr int kStreamRows = 1024;  // landmark rows per streaming CTA (a ring of bulk copies)
+// decode rows from this many eligible chunks take the two-level top-K (group maxima): shorter
+// rows are read in one or two rounds per lane anyway, and there the group maxima's looser
+// threshold lets more candidates through than it saves (measured on 2K- and 8K-chunk rows)
+constexpr int64_t kTopkGroupMinChunks = 16384;
 
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -43,7 +47,8 @@ struct Plan {
   int cps = 0, n_split = 0, n_pieces = 0;
   size_t off_idx = 0, off_ssel = 0, off_po = 0, off_pl = 0;
   size_t off_sig = 0;
-  int64_t n_stride = 0;
+  size_t off_gmax = 0;        // decode on the tensor-core stream: maxima of 32 sigmas per row
+  int64_t n_stride = 0, g_stride = 0;
   size_t total = 0;
 };
 
@@ -124,6 +129,11 @@ Plan make_plan(const hils_params* p) {
     P.off_pl = off; off = align_up(off + head_rows * NU * sizeof(float));
     P.n_stride = (n_max + 3) / 4 * 4;
     P.off_sig = off; off = align_up(off + sel_rows * (size_t)P.n_stride * sizeof(float));
+    if (P.tc_stream && n_max >= kTopkGroupMinChunks) {   // four groups of 32 per 128-row tile
+      P.g_stride = (P.n_stride + 127) / 128 * 4;
+      P.off_gmax = off;
+      off = align_up(off + sel_rows * (size_t)P.g_stride * sizeof(float));
+    }
   }
   P.total = off;
   return P;
@@ -216,13 +226,15 @@ cudaError_t launch_decode_select(const Plan& P, const void* q_cal, const void* k
                                  cudaStream_t st, PhaseMarks& pm) {
   cudaError_t e;
   float* sig = reinterpret_cast<float*>(ws + P.off_sig);
+  float* gmax = P.g_stride > 0 ? reinterpret_cast<float*>(ws + P.off_gmax) : nullptr;
   e = P.tc_stream ? launch_select_stream_tc(P.D, q_cal, k_lm, b_lm, sig, P.n_stride,
-                                            reinterpret_cast<int32_t*>(ws), st)
+                                            reinterpret_cast<int32_t*>(ws), st, gmax, P.g_stride)
                   : launch_select_stream(P.D, P.bf16, kStreamRows, n_stream_split(P), P.n_stride,
                                          q_cal, k_lm, b_lm, sig, reinterpret_cast<int32_t*>(ws), st);
   pm.mark();
   if (e == cudaSuccess)
-    e = launch_select_topk_row(P.D, P.bf16, P.n_stride, sig, q_cal, k_lm, b_lm, idx, s_sel, st);
+    e = launch_select_topk_row(P.D, P.bf16, P.n_stride, sig, q_cal, k_lm, b_lm, idx, s_sel, st,
+                               gmax, P.g_stride);
   pm.mark();
   return e;
 }

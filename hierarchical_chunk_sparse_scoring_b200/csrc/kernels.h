@@ -52,16 +52,20 @@ cudaError_t launch_select_stream(const Dims& D, bool bf16, int cps, int n_split,
                                  const float* blm, float* sigma, int32_t* status,
                                  cudaStream_t st);
 bool stream_tc_supported(const Dims& D, bool bf16);
+// gmax (nullable): [rows][g_stride] maxima of 32 consecutive sigmas, g_stride >= 4 per
+// 128-landmark tile of the longest row.
 cudaError_t launch_select_stream_tc(const Dims& D, const void* qc, const void* klm,
                                     const float* blm, float* sigma, int64_t n_stride,
-                                    int32_t* status, cudaStream_t st);
+                                    int32_t* status, cudaStream_t st, float* gmax = nullptr,
+                                    int64_t g_stride = 0);
 bool units_tc_supported(const Dims& D, bool bf16);
 cudaError_t launch_attn_units_tc(const Dims& D, int n_pieces, const void* q, const void* K,
                                  const void* V, const int32_t* idx, float* part_o,
                                  float* part_lse, int32_t* status, cudaStream_t st);
 cudaError_t launch_select_topk_row(const Dims& D, bool bf16, int64_t n_stride,
                                    const float* sigma, const void* qc, const void* klm,
-                                   const float* blm, int32_t* idx, float* s_sel, cudaStream_t st);
+                                   const float* blm, int32_t* idx, float* s_sel, cudaStream_t st,
+                                   const float* gmax = nullptr, int64_t g_stride = 0);
 cudaError_t launch_select_merge(const Dims& D, bool bf16, int n_split, const float* part_v,
                                 const int32_t* part_c, const void* qc, const void* klm,
                                 const float* blm, int32_t* idx, float* s_sel, cudaStream_t st);

@@ -672,6 +672,11 @@ __global__ void __launch_bounds__(kStreamThreads) select_stream_kernel(
 //      register lists and a warp merge otherwise -- and writes idx and the per-head scores.  If
 //      more than kSurvivorCap candidates tie at or above theta, step 4 runs over all candidates
 //      (slower, same result).
+// With the streaming scorer's group maxima (gmax: the max of each 32 consecutive chunks), steps
+// 1 and 3 read far less: the lane maxima are taken over group maxima (each group max is a
+// chunk's score, so theta stays a lower bound of the row's K-th best, now as a value, every tie
+// passing), and step 3 reads only the groups whose maximum reaches theta, which hold every
+// candidate.
 constexpr int kTopkWarps = 4;
 constexpr int kTopkThreads = 32 * kTopkWarps;
 constexpr int kSurvivorCap = 1024;
@@ -702,7 +707,7 @@ template <typename T, int D_, int GM, int KM>
 __global__ void __launch_bounds__(kTopkThreads) select_topk_row_kernel(
     Dims D, int64_t n_stride, const float* __restrict__ sigma, const T* __restrict__ qc,
     const T* __restrict__ klm, const float* __restrict__ blm, int32_t* __restrict__ idx,
-    float* __restrict__ s_sel) {
+    float* __restrict__ s_sel, const float* __restrict__ gmax, int64_t g_stride) {
   __shared__ float sv[kSurvivorCap];
   __shared__ int scn[kSurvivorCap];
   __shared__ float th_v[kTopkWarps];
@@ -729,11 +734,25 @@ __global__ void __launch_bounds__(kTopkThreads) select_topk_row_kernel(
   const int64_t n4 = n >> 2;
   // this warp's quarter of the row's float4 vectors (the scalar tail goes to the last warp)
   const int64_t w0 = n4 * warp / kTopkWarps, w1 = n4 * (warp + 1) / kTopkWarps;
+  // with group maxima: this warp's quarter of the row's groups of 32 chunks
+  const float* gr = gmax ? gmax + row * g_stride : nullptr;
+  const int64_t n_g = (n + 31) >> 5;
+  const int64_t g0 = n_g * warp / kTopkWarps, g1 = n_g * (warp + 1) / kTopkWarps;
   // 1. lane maxima (a lane's chunks come in increasing order: a strict compare keeps the lower
-  //    index on ties)
+  //    index on ties; over group maxima the chunk stays unknown, INT_MAX)
   float mv = -INFINITY;
   int mc = INT_MAX;
-  for (int64_t q0 = w0; q0 < w1; q0 += 32 * kTopkBatch) {
+  for (int64_t q0 = g0; gr && q0 < g1; q0 += 32 * kTopkBatch) {
+    float t[kTopkBatch];
+#pragma unroll
+    for (int u = 0; u < kTopkBatch; ++u) {
+      const int64_t gi = q0 + u * 32 + lane;
+      t[u] = gi < g1 ? __ldg(gr + gi) : -INFINITY;
+    }
+#pragma unroll
+    for (int u = 0; u < kTopkBatch; ++u) mv = fmaxf(mv, t[u]);
+  }
+  for (int64_t q0 = w0; !gr && q0 < w1; q0 += 32 * kTopkBatch) {
     float4 t[kTopkBatch];
 #pragma unroll
     for (int u = 0; u < kTopkBatch; ++u) {
@@ -750,7 +769,7 @@ __global__ void __launch_bounds__(kTopkThreads) select_topk_row_kernel(
       if (t[u].w > mv) { mv = t[u].w; mc = c + 3; }
     }
   }
-  if (warp == kTopkWarps - 1) {
+  if (!gr && warp == kTopkWarps - 1) {
     for (int64_t c = n4 * 4 + lane; c < n; c += 32) {
       const float v = __ldg(sr + c);
       if (better(v, (int)c, mv, mc)) { mv = v; mc = (int)c; }
@@ -785,7 +804,36 @@ __global__ void __launch_bounds__(kTopkThreads) select_topk_row_kernel(
     if (keep && pos < kCapW) { svw[pos] = v; scw[pos] = c; }
     ns_w += __popc(m);
   };
-  for (int64_t q0 = w0; q0 < w1; q0 += 32 * kTopkBatch) {
+  // over group maxima: 32 groups per round; the chunks of up to 8 groups that reach theta are
+  // loaded together (one per lane each, in chunk order), then appended
+  for (int64_t gb = g0; gr && gb < g1; gb += 32) {
+    // (lanes past the warp's groups never flag: with theta = -inf they would pass the compare
+    // and pull in another warp's groups)
+    const bool in = gb + lane < g1;
+    const float gm = in ? __ldg(gr + gb + lane) : -INFINITY;
+    unsigned m = __ballot_sync(0xffffffffu, in && gm >= tv);
+    while (m) {
+      int gs[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        gs[k] = m ? __ffs(m) - 1 : -1;
+        m &= m - 1u;
+      }
+      float v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int64_t c = (gb + gs[k]) * 32 + lane;
+        v[k] = gs[k] >= 0 && c < n ? __ldg(sr + c) : -INFINITY;
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (gs[k] < 0) break;   // (warp-uniform)
+        const int64_t c = (gb + gs[k]) * 32 + lane;
+        append(c < n && !better(tv, tcc, v[k], (int)c), v[k], (int)c);
+      }
+    }
+  }
+  for (int64_t q0 = w0; !gr && q0 < w1; q0 += 32 * kTopkBatch) {
     float4 t[kTopkBatch];
 #pragma unroll
     for (int u = 0; u < kTopkBatch; ++u) {
@@ -810,7 +858,7 @@ __global__ void __launch_bounds__(kTopkThreads) select_topk_row_kernel(
       append(k3, t[u].w, c + 3);
     }
   }
-  if (warp == kTopkWarps - 1) {
+  if (!gr && warp == kTopkWarps - 1) {
     for (int64_t c0 = n4 * 4; c0 < n; c0 += 32) {
       const int64_t c = c0 + lane;
       const float v = c < n ? __ldg(sr + c) : -INFINITY;
@@ -893,10 +941,10 @@ template <typename T, int D_, int GM, int KM>
 struct TopkRowRun {
   static cudaError_t run(const Dims* D, int64_t n_stride, const float* sigma, const void* qc,
                          const void* klm, const float* blm, int32_t* idx, float* s_sel,
-                         cudaStream_t st) {
+                         const float* gmax, int64_t g_stride, cudaStream_t st) {
     const int64_t rows = D->B * D->Hkv * D->N_q;
     select_topk_row_kernel<T, D_, GM, KM><<<(unsigned)rows, kTopkThreads, 0, st>>>(
-        *D, n_stride, sigma, (const T*)qc, (const T*)klm, blm, idx, s_sel);
+        *D, n_stride, sigma, (const T*)qc, (const T*)klm, blm, idx, s_sel, gmax, g_stride);
     return cudaGetLastError();
   }
 };
@@ -1064,10 +1112,11 @@ cudaError_t launch_select_stream(const Dims& D, bool bf16, int cps, int n_split,
 
 cudaError_t launch_select_topk_row(const Dims& D, bool bf16, int64_t n_stride,
                                    const float* sigma, const void* qc, const void* klm,
-                                   const float* blm, int32_t* idx, float* s_sel, cudaStream_t st) {
+                                   const float* blm, int32_t* idx, float* s_sel, cudaStream_t st,
+                                   const float* gmax, int64_t g_stride) {
   if (D.B * D.Hkv * D.N_q == 0) return cudaSuccess;
   return dispatch_tdgk<TopkRowRun>(bf16, D.d, D.G, D.K, &D, n_stride, sigma, qc, klm, blm, idx,
-                                   s_sel, st);
+                                   s_sel, gmax, g_stride, st);
 }
 
 }  // namespace hils

@@ -15,7 +15,10 @@
 // block) are split into contiguous ranges, one per CTA, so a CTA's stream crosses few rows.
 // Warp 0: TMA producer (a ring of stages, each one landmark tile plus the row's query tile);
 // warp 1: TMEM owner and MMA issuer;
-// warps 2-5: epilogue (tcgen05.ld of 16 columns, group max, scale, bias, mask c < n).
+// warps 2-5: epilogue (tcgen05.ld of 16 columns, group max, scale, bias, mask c < n; with gmax,
+// each warp also writes the max of its 32 consecutive sigmas, -inf past n, for the top-K
+// kernel's two-level scan).
+// g_stride: group maxima per row (at least 4 per tile).
 // Every mbarrier wait gives up after a bounded number of polls and records HILS_ERR_TIMEOUT.
 #include <cudaTypedefs.h>
 
@@ -58,7 +61,8 @@ __global__ void __launch_bounds__(kStThreads, kStCtasPerSm)
                             const __grid_constant__ CUtensorMap tmB, Dims D, int64_t tiles_per_row,
                             int64_t n_tiles_total, int64_t n_stride,
                             const float* __restrict__ blm, float* __restrict__ sigma,
-                            int32_t* __restrict__ status) {
+                            int32_t* __restrict__ status, float* __restrict__ gmax,
+                            int64_t g_stride) {
   using SH = StShape<DD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -179,7 +183,12 @@ __global__ void __launch_bounds__(kStThreads, kStCtasPerSm)
 #pragma unroll
       for (int h = 1; h < kStCols; ++h)
         if (h < G) m = fmaxf(m, v[h]);
-      if (live) sigma[row * n_stride + c] = fmaf(m, D.scale, bias);
+      const float s = fmaf(m, D.scale, bias);
+      if (live) sigma[row * n_stride + c] = s;
+      if (gmax) {
+        const float gm = warp_max(live ? s : -INFINITY);   // chunks c - lane .. c - lane + 31
+        if (lane == 0) gmax[row * g_stride + (c >> 5)] = gm;
+      }
     }
     if (!ok) record_status(status, kStatusTimeout);
   }
@@ -207,7 +216,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_st() {
 
 template <int DD>
 cudaError_t launch_st_t(const Dims& D, const void* qc, const void* klm, const float* blm,
-                        float* sigma, int64_t n_stride, int32_t* status, cudaStream_t st) {
+                        float* sigma, int64_t n_stride, int32_t* status, cudaStream_t st,
+                        float* gmax, int64_t g_stride) {
   using SH = StShape<DD>;
   auto enc = get_encode_st();
   if (!enc) return cudaErrorInvalidValue;
@@ -253,7 +263,7 @@ cudaError_t launch_st_t(const Dims& D, const void* qc, const void* klm, const fl
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SH::SMEM);
   if (e != cudaSuccess) return e;
   kern<<<(unsigned)grid, kStThreads, SH::SMEM, st>>>(tmA, tmB, D, tiles_per_row, total, n_stride,
-                                                     blm, sigma, status);
+                                                     blm, sigma, status, gmax, g_stride);
   return cudaGetLastError();
 }
 
@@ -268,10 +278,12 @@ bool stream_tc_supported(const Dims& D, bool bf16) {
 
 cudaError_t launch_select_stream_tc(const Dims& D, const void* qc, const void* klm,
                                     const float* blm, float* sigma, int64_t n_stride,
-                                    int32_t* status, cudaStream_t st) {
+                                    int32_t* status, cudaStream_t st, float* gmax,
+                                    int64_t g_stride) {
   if (D.B * D.Hkv * D.N_q == 0 || D.C == 0) return cudaSuccess;
-  if (D.d == 128) return launch_st_t<128>(D, qc, klm, blm, sigma, n_stride, status, st);
-  return launch_st_t<64>(D, qc, klm, blm, sigma, n_stride, status, st);
+  if (D.d == 128)
+    return launch_st_t<128>(D, qc, klm, blm, sigma, n_stride, status, st, gmax, g_stride);
+  return launch_st_t<64>(D, qc, klm, blm, sigma, n_stride, status, st, gmax, g_stride);
 }
 
 }  // namespace hils

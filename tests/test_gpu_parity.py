@@ -119,6 +119,9 @@ EDGE_CASES = {
                               q_pos0=4991, N_q=5),
     "decode_s128_g16": dict(B=1, Hq=16, Hkv=1, N=12345, d=128, S=128, K=12, W_=2048,
                             q_pos0=12344, N_q=1),
+    # rows of at least 16384 eligible chunks: the two-level top-K (group maxima), two queries
+    "decode_long_rows": dict(B=1, Hq=4, Hkv=1, N=560000, d=64, S=32, K=16, W_=300,
+                             q_pos0=559998, N_q=2),
     # the tensor-core units kernel's head bounds (4, 8, 16) at S = 64, with G below its bound
     "decode_s64_g3": dict(B=2, Hq=6, Hkv=2, N=7000, d=128, S=64, K=16, W_=300,
                           q_pos0=6999, N_q=1),

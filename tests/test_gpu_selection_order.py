@@ -60,6 +60,10 @@ CASES = {
     # one row over 4,680 chunks (one top-K CTA for the whole row)
     "decode_one_row": (dict(B=1, Hq=8, Hkv=1, N=300000, d=128, S=64, K=16, W_=512,
                             q_pos0=299999, N_q=1), torch.bfloat16, "select_stream_tc, select_topk"),
+    # one row over 18,734 chunks: the two-level top-K over the streaming scorer's group maxima
+    "decode_long_row": (dict(B=1, Hq=8, Hkv=1, N=600000, d=64, S=32, K=16, W_=512,
+                             q_pos0=599999, N_q=1), torch.bfloat16,
+                        "select_stream_tc with group maxima, two-level select_topk"),
     "decode_multi_query": (dict(B=2, Hq=4, Hkv=2, N=9000, d=128, S=64, K=8, W_=256,
                                 q_pos0=8996, N_q=4), torch.bfloat16,
                            "select_stream_tc, select_topk"),
