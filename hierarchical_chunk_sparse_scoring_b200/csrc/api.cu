@@ -24,10 +24,8 @@ constexpr size_t kStatusBytes = 256;
 constexpr int kChunksPerSplit = 512;
 constexpr int64_t kDecodeMaxQueries = 16;
 constexpr int kStreamRows = 1024;  // landmark rows per streaming CTA (a ring of bulk copies)
-// decode rows from this many eligible chunks take the two-level top-K (group maxima): shorter
-// rows are read in one or two rounds per lane anyway, and there the group maxima's looser
-// threshold lets more candidates through than it saves (measured on 2K- and 8K-chunk rows)
-constexpr int64_t kTopkGroupMinChunks = 16384;
+// decode rows from this many eligible chunks take the two-level top-K (group maxima)
+constexpr int64_t kTopkGroupMinChunks = 1024;
 
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }

@@ -742,12 +742,17 @@ __global__ void __launch_bounds__(kTopkThreads) select_topk_row_kernel(
   //    index on ties; over group maxima the chunk stays unknown, INT_MAX)
   float mv = -INFINITY;
   int mc = INT_MAX;
-  for (int64_t q0 = g0; gr && q0 < g1; q0 += 32 * kTopkBatch) {
+  // (a row of at most 32 * kTopkBatch groups is read whole by every warp, one round per lane:
+  // each lane's maximum then covers four times as many chunks, and theta, the same in every
+  // warp, is that much tighter)
+  const bool whole = n_g <= 32 * kTopkBatch;
+  const int64_t p0 = whole ? 0 : g0, p1 = whole ? n_g : g1;
+  for (int64_t q0 = p0; gr && q0 < p1; q0 += 32 * kTopkBatch) {
     float t[kTopkBatch];
 #pragma unroll
     for (int u = 0; u < kTopkBatch; ++u) {
       const int64_t gi = q0 + u * 32 + lane;
-      t[u] = gi < g1 ? __ldg(gr + gi) : -INFINITY;
+      t[u] = gi < p1 ? __ldg(gr + gi) : -INFINITY;
     }
 #pragma unroll
     for (int u = 0; u < kTopkBatch; ++u) mv = fmaxf(mv, t[u]);
