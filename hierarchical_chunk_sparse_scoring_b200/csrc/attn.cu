@@ -181,12 +181,12 @@ __device__ __forceinline__ void fuse_row(const Dims& D, int n_pieces, int64_t ro
   const float* pr = part_o + row * NU * d;
   if (NU <= 64 && d == 128) {
     // lanes hold the weights of units lane and lane + 32 (scores read once); every lane reads its
-    // 4 output columns of all units, 16 loads in flight per batch, the first batch issued before
-    // the score loads so that both are in flight together
-    float v[16][4];
+    // 4 output columns of all units, 32 loads in flight per batch (two rounds for up to 64
+    // units), the first batch issued before the score loads so that both are in flight together
+    float v[32][4];
     auto load_batch = [&](int u0) {
 #pragma unroll
-      for (int e2 = 0; e2 < 16; ++e2) {
+      for (int e2 = 0; e2 < 32; ++e2) {
         if (u0 + e2 < NU) {
           load4cg(pr + (int64_t)(u0 + e2) * 128 + lane * 4, v[e2]);
         } else {
@@ -203,12 +203,12 @@ __device__ __forceinline__ void fuse_row(const Dims& D, int n_pieces, int64_t ro
     const float Z = warp_sum(e0 + e1);
     const float w0 = e0 / Z, w1 = e1 / Z;
     float o[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int u0 = 0; u0 < NU; u0 += 16) {
+    for (int u0 = 0; u0 < NU; u0 += 32) {
       if (u0 > 0) load_batch(u0);
-      const float wsrc = u0 < 32 ? w0 : w1;   // a batch lies on one side of unit 32
+      const float wsrc = u0 < 32 ? w0 : w1;   // batch 0: units 0-31, batch 1: units 32-63
 #pragma unroll
-      for (int e2 = 0; e2 < 16; ++e2) {
-        const float w = __shfl_sync(0xffffffffu, wsrc, (u0 + e2) & 31);
+      for (int e2 = 0; e2 < 32; ++e2) {
+        const float w = __shfl_sync(0xffffffffu, wsrc, e2);
 #pragma unroll
         for (int x = 0; x < 4; ++x) o[x] = fmaf(w, v[e2][x], o[x]);
       }
