@@ -382,6 +382,132 @@ __global__ void __launch_bounds__(kQhThreads, 3)
   }
 }
 
+// bf16, d = 128, r a multiple of 16: the correction of a block's 32 tokens, one head at a time,
+// as a product on the tensor cores, dq[128 dims x 32 tokens] = W_up[h] [128 x r] . u^T [r x 32],
+// with m16n8k16 tiles (bf16 operands, fp32 accumulators).  W_up[h] is bf16 already; u (fp32,
+// from the down-projection) enters as two bf16 parts, hi = bf16(u) and lo = bf16(u - hi), each
+// multiplied in turn, so the product keeps u to about 2^-17 of itself.  Warp w takes the dim
+// tiles mp = w % 4 and mp + 4 (so a lane holds dims m and m + 64, whole rotation pairs) and the
+// token tiles 2 (w / 4) and 2 (w / 4) + 1.  The head's q tile [32 tokens x 128] is staged in
+// shared memory by 16-byte loads, the turned q and q_cal tiles are written there in the
+// accumulator's order and stored by 16-byte writes (rows padded to 136 elements so the
+// fragment-order accesses spread over the banks).  Two barriers per head order the reuse.
+constexpr int kQmLd = 136;   // staged row stride (elements)
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void split_bf16x2(float x, float y, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x - __low2float(h), y - __high2float(h));
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+__global__ void __launch_bounds__(kQhThreads, 3)
+    qcal_hope_mma_kernel(int64_t N_q, int64_t Hq, int64_t q_pos0, int r, double base,
+                         double train_len, const __nv_bfloat16* __restrict__ q,
+                         const float* __restrict__ u, const __nv_bfloat16* __restrict__ W_up,
+                         __nv_bfloat16* __restrict__ q_out, __nv_bfloat16* __restrict__ qc_out) {
+  constexpr int DD = 128, HALF = 64;
+  static_assert(kQhTokens == 32 && kQhThreads == 256, "8 warps x (2 dim tiles, 2 token tiles)");
+  __shared__ float2 sCS[kQhTokens * HALF];
+  __shared__ __align__(16) __nv_bfloat16 sQ[kQhTokens * kQmLd];
+  __shared__ __align__(16) __nv_bfloat16 sX[kQhTokens * kQmLd];
+  __shared__ __align__(16) __nv_bfloat16 sC[kQhTokens * kQmLd];
+  const int64_t b = blockIdx.y;
+  const int64_t i0 = (int64_t)blockIdx.x * kQhTokens;
+  angle_table<DD>(sCS, q_pos0 + i0, base, train_len);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, tq = lane & 3;   // fragment row group and thread in group
+  const int mp = warp & 3;                  // dim tiles mp and mp + 4
+  const int nt0 = 2 * (warp >> 2);          // token tiles nt0 and nt0 + 1
+  // 16-byte pieces of the 32 x 128 tile: two per thread (piece p: token p / 16, dims 8 (p % 16))
+  constexpr int kPieces = kQhTokens * DD / 8;
+  for (int64_t h = 0; h < Hq; ++h) {
+    const int64_t row0 = ((b * Hq + h) * N_q + i0) * DD;   // the block's first token row
+#pragma unroll
+    for (int p = threadIdx.x; p < kPieces; p += kQhThreads) {
+      const int t = p >> 4, c8 = (p & 15) * 8;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (i0 + t < N_q) v = __ldg(reinterpret_cast<const uint4*>(q + row0 + t * DD + c8));
+      *reinterpret_cast<uint4*>(sQ + t * kQmLd + c8) = v;
+    }
+    float acc[2][2][4];
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[a][n][e] = 0.f;
+    for (int kc = 0; kc < r; kc += 16) {
+      uint32_t af[2][4];
+#pragma unroll
+      for (int a = 0; a < 2; ++a) {
+        const __nv_bfloat16* w0 = W_up + (h * DD + 16 * (mp + 4 * a) + g) * r + kc + 2 * tq;
+        const __nv_bfloat16* w1 = w0 + 8 * r;
+        af[a][0] = __ldg(reinterpret_cast<const uint32_t*>(w0));
+        af[a][1] = __ldg(reinterpret_cast<const uint32_t*>(w1));
+        af[a][2] = __ldg(reinterpret_cast<const uint32_t*>(w0 + 8));
+        af[a][3] = __ldg(reinterpret_cast<const uint32_t*>(w1 + 8));
+      }
+#pragma unroll
+      for (int n = 0; n < 2; ++n) {
+        const int64_t i = i0 + 8 * (nt0 + n) + g;   // this lane's token of the B fragment
+        float2 u0 = make_float2(0.f, 0.f), u1 = make_float2(0.f, 0.f);
+        if (i < N_q) {
+          const float* ur = u + (b * N_q + i) * (Hq * r) + h * r + kc + 2 * tq;
+          u0 = __ldg(reinterpret_cast<const float2*>(ur));
+          u1 = __ldg(reinterpret_cast<const float2*>(ur + 8));
+        }
+        uint32_t b0h, b0l, b1h, b1l;
+        split_bf16x2(u0.x, u0.y, b0h, b0l);
+        split_bf16x2(u1.x, u1.y, b1h, b1l);
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+          mma_bf16_16816(acc[a][n], af[a], b0h, b1h);
+          mma_bf16_16816(acc[a][n], af[a], b0l, b1l);
+        }
+      }
+    }
+    __syncthreads();   // the q tile (and, for h = 0, the angle table) is in place; the previous
+                       // head's output tiles have been stored
+    // accumulator element e of token tile n: dim 16 * tile + g + 8 * (e >> 1), token
+    // 8 * (nt0 + n) + 2 * tq + (e & 1); tiles mp and mp + 4 hold the two dims of a pair
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int t = 8 * (nt0 + n) + 2 * tq + (e & 1);   // token in the block
+        const int m = 16 * mp + g + 8 * (e >> 1);          // pair (m, m + 64)
+        const float xa = __bfloat162float(sQ[t * kQmLd + m]);
+        const float xb = __bfloat162float(sQ[t * kQmLd + HALF + m]);
+        const float ca = xa + acc[0][n][e], cb = xb + acc[1][n][e];
+        const float2 cs = sCS[t * HALF + m];
+        sX[t * kQmLd + m] = __float2bfloat16_rn(xa * cs.x - xb * cs.y);
+        sX[t * kQmLd + HALF + m] = __float2bfloat16_rn(xa * cs.y + xb * cs.x);
+        sC[t * kQmLd + m] = __float2bfloat16_rn(ca * cs.x - cb * cs.y);
+        sC[t * kQmLd + HALF + m] = __float2bfloat16_rn(ca * cs.y + cb * cs.x);
+      }
+    }
+    __syncthreads();   // both output tiles complete; sQ free for the next head
+#pragma unroll
+    for (int p = threadIdx.x; p < kPieces; p += kQhThreads) {
+      const int t = p >> 4, c8 = (p & 15) * 8;
+      if (i0 + t < N_q) {
+        *reinterpret_cast<uint4*>(q_out + row0 + t * DD + c8) =
+            *reinterpret_cast<const uint4*>(sX + t * kQmLd + c8);
+        *reinterpret_cast<uint4*>(qc_out + row0 + t * DD + c8) =
+            *reinterpret_cast<const uint4*>(sC + t * kQmLd + c8);
+      }
+    }
+  }
+}
+
 // x [B H, N, d] -> R(x), token n at position pos0 + n; grid (token blocks), every (b, h) in turn.
 template <typename T, int DD>
 __global__ void __launch_bounds__(kQhThreads)
@@ -443,7 +569,12 @@ cudaError_t launch_qcal_hope(int64_t B, int64_t Hq, int64_t N_q, int64_t d, int6
       N_q, Hq, q_pos0, r, base, train_len, static_cast<const TT*>(q), u,                       \
       static_cast<const TT*>(W_up), static_cast<TT*>(q_out), static_cast<TT*>(qc_out))
   if (bf16) {
-    if (d == 128) HILS_QH(__nv_bfloat16, 128);
+    if (d == 128 && r > 0 && r % 16 == 0)
+      qcal_hope_mma_kernel<<<grid, kQhThreads, 0, st>>>(
+          N_q, Hq, q_pos0, r, base, train_len, static_cast<const __nv_bfloat16*>(q), u,
+          static_cast<const __nv_bfloat16*>(W_up), static_cast<__nv_bfloat16*>(q_out),
+          static_cast<__nv_bfloat16*>(qc_out));
+    else if (d == 128) HILS_QH(__nv_bfloat16, 128);
     else HILS_QH(__nv_bfloat16, 64);
   } else {
     if (d == 128) HILS_QH(float, 128);
