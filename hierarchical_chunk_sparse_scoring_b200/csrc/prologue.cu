@@ -8,7 +8,7 @@
 // turn by pos * base^(-2m/d); the others are left as they are (NoPE).  q and q_cal are turned at
 // the query's position, keys at their own (hope_rotate).
 //
-// Two kernels:
+// Kernels:
 //   qdown_kernel   u = hidden W_down^T for all heads at once: [B N_q, d_model] x [Hq r, d_model]^T,
 //                  a dense contraction on the tcgen05 tensor cores (bf16 operands by TMA with the
 //                  128-byte swizzle, fp32 accumulator in TMEM, 128 x BN tiles, a 4-stage ring).
@@ -19,6 +19,8 @@
 //                  p theta_m reduced modulo 2 pi in fp64 once (p up to 2^22 makes an fp32
 //                  product lose whole radians), then sincosf, kept in shared memory for all
 //                  heads.  hope_rotate_kernel turns keys the same way.
+//   qcal_hope_mma_kernel  the same pass for bf16, d = 128 and r a multiple of 16, with W_up u on
+//                  m16n8k16 tensor-core tiles and the q / output tiles staged in shared memory.
 #include <cudaTypedefs.h>
 
 #include <type_traits>
