@@ -68,6 +68,21 @@ def test_workspace_size(lib):
     assert hb.workspace_size(_params(Hq=6, Hkv=4)) == 0   # Hq % Hkv != 0
 
 
+def test_decode_group_maxima_region(lib):
+    # rows of 1024 eligible chunks or more on the tensor-core streaming scorer (bf16) get the
+    # two-level top-K's group maxima (4 per 128-chunk tile, one aligned region); fp32 decode
+    # streams on the CUDA cores and has none.  n = 1023 and 1024 share every other region
+    # (same sigma row stride, same 1024-token window).
+    def dec(n, dtype=torch.bfloat16):
+        pos = n * 64 + 1024 - 1
+        return hb.workspace_size(_params(B=1, Hq=8, Hkv=2, N_q=1, N_kv=pos + 1, q_pos0=pos,
+                                         dtype=dtype))
+    rows, g_stride = 1 * 2 * 1, (1024 + 127) // 128 * 4
+    region = (rows * g_stride * 4 + 255) // 256 * 256
+    assert dec(1024) - dec(1023) == region
+    assert dec(1024, torch.float32) == dec(1023, torch.float32)
+
+
 def test_prefill_workspace_layout(lib):
     # status word, then idx [B, Hkv, N_q, K]; per-head scores [B, Hq, N_q, K] only where the
     # tensor-core attention does not score the selected chunks itself: one head per KV group
