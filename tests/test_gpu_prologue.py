@@ -49,6 +49,8 @@ CASES = {
     # name: (B, Hq, N_q, d, d_model, r, q_pos0, base, train_len, dtype)
     "bf16_d128_r16": (1, 8, 300, 128, 512, 16, 1000, 10000.0, 8192.0, torch.bfloat16),
     "bf16_n512_dm4096": (1, 32, 1000, 128, 4096, 16, 0, 10000.0, 32768.0, torch.bfloat16),
+    # tensor-core up-projection: two sequences, r = 32 (two k steps), a ragged token block
+    "bf16_b2_r32": (2, 4, 200, 128, 256, 32, 50, 10000.0, 8192.0, torch.bfloat16),
     "fp32_d64_r16": (2, 4, 77, 64, 128, 16, 5, 10000.0, 4096.0, torch.float32),
     "fp32_d128_r8_far": (1, 8, 200, 128, 256, 8, (1 << 22) - 200, 500000.0, 1e7,
                          torch.float32),
