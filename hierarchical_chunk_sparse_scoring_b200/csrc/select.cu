@@ -668,15 +668,15 @@ __global__ void __launch_bounds__(kStreamThreads) select_stream_kernel(
 //      the row's K-th best;
 //   3. every candidate >= theta is appended to a shared list (ballot compaction; typically a
 //      few dozen);
-//   4. warp 0 takes the exact top-K of that list -- one bitonic sort when it holds at most 32,
+//   4. warp 0 takes the exact top-K of that list -- one bitonic sort when it holds at most 64,
 //      register lists and a warp merge otherwise -- and writes idx and the per-head scores.  If
-//      more than kSurvivorCap candidates tie at or above theta, step 4 runs over all candidates
-//      (slower, same result).
+//      a warp has more candidates than its quarter of kSurvivorCap (many ties at theta), step 4
+//      runs over the whole row instead (slower, same result).
 // With the streaming scorer's group maxima (gmax: the max of each 32 consecutive chunks), steps
 // 1 and 3 read far less: the lane maxima are taken over group maxima (each group max is a
 // chunk's score, so theta stays a lower bound of the row's K-th best, now as a value, every tie
-// passing), and step 3 reads only the groups whose maximum reaches theta, which hold every
-// candidate.
+// passing; a row of at most 256 groups is read whole by every warp, for a tighter theta), and
+// step 3 reads only the groups whose maximum reaches theta, which hold every candidate.
 constexpr int kTopkWarps = 4;
 constexpr int kTopkThreads = 32 * kTopkWarps;
 constexpr int kSurvivorCap = 1024;
